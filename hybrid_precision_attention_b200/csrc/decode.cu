@@ -1,0 +1,555 @@
+// decode.cu — one decode step of attention over the hybrid K4V4 / FP16 cache.
+//
+// HyQuant digest (agihunt.info), prefill/decode paragraph, and the repository
+// README, Overview item 3: the decode cache stores most positions K4V4 and the
+// vertical-line and recent positions FP16, and dequantisation is fused into the
+// attention scan (online softmax over quantised blocks) so no FP16 cache is
+// materialised.  The pages' kernel is Triton for SM80+; this is a B200 design.
+//
+// Design (bandwidth-bound: ~160 B of K4V4 per token and kv head):
+//   * grid = (splits S, Hkv, B); every CTA owns one GQA group (all G <= 8 query
+//     heads of a kv head share one pass over the bytes) and a contiguous range
+//     of the head's tile list: packed tiles (64 positions: 4 KB K codes, 4 KB V
+//     codes, 1 KB + 1 KB scale/zero, 16 B of the VL bitmap), then VL tiles and
+//     recent tiles (16 FP16 rows each);
+//   * one producer lane streams tiles into an 8-stage shared-memory ring with
+//     1-D bulk async copies (cp.async.bulk, mbarrier completion, no multicast);
+//   * 4 consumer warps take whole tiles round-robin.  Nibbles become fp16 in
+//     registers (exponent-bias trick + one fma with the group's scale/zero), and
+//     both products run on tensor cores with mma.m16n8k16 (f32 accumulate):
+//       S^T[keys x 8 queries] = K^ (16 keys x 16 dims) . Q^T
+//       O^T[dims x 8 queries] += V^T (16 dims x 16 keys) . P^T
+//     P^T comes from the S^T accumulators by an 8x8 movmatrix transpose.  Dims
+//     and keys are permuted inside each MMA so that every thread dequantises one
+//     whole group from contiguous nibbles and the shared-memory reads are free
+//     of bank conflicts;
+//   * per-warp online softmax in the exp2 domain, a CTA merge in shared memory,
+//     then split partials (m, l, O) go to the workspace and the last CTA of each
+//     (b, kv head) merges them with a log-sum-exp (atomic ticket, no waiting);
+//   * the new token is attended from its input pointer and written into the
+//     ring; the last CTA of the grid advances T.
+#include "common.cuh"
+
+namespace hq {
+namespace {
+
+constexpr int NCONS = 4;                       // consumer warps
+constexpr int NTHREADS = (NCONS + 1) * 32;     // + producer warp
+constexpr int NSTAGES = 8;
+constexpr int PK = 64;                         // positions per packed tile
+constexpr int FT = 16;                         // rows per FP16 tile
+constexpr int FSTRIDE = 272;                   // bytes per FP16 row in shared memory (256 + 16)
+constexpr int OFF_VC = 4096, OFF_KS = 8192, OFF_VS = 9216, OFF_MASK = 10240;
+constexpr int OFF_FV = FT * FSTRIDE;           // V rows of an FP16 tile
+constexpr int STAGE_BYTES = 10368;             // max(10256, 2 * 16 * 272 = 8704), 128-aligned
+constexpr int PART_FLOATS = 16 + 8 * D;        // m[8], l[8], O[8][128]
+constexpr uint32_t PK_TX = 4096 * 2 + 1024 * 2 + 16;
+
+// key slot -> shared-memory row inside a 16-key block.  Packed tiles (64-byte
+// rows): {0,5,1,4,2,7,3,6, 8,13,9,12,10,15,11,14}; FP16 tiles (272-byte rows):
+// {0,2,1,3,4,6,5,7, 8,10,9,11,12,14,13,15}.  Both keep the QK rows of a
+// quarter-warp and the PV rows of a warp on distinct banks.
+__device__ __forceinline__ int pi_pk(int s) {
+  const int x = s & 7;
+  return (s & 8) + ((x & 1) ? 4 + ((x >> 1) ^ 1) : (x >> 1));
+}
+__device__ __forceinline__ int pi_fp(int s) {
+  const int x = s & 7;
+  return (s & 8) + (x & 4) + ((x & 1) << 1) + ((x >> 1) & 1);
+}
+
+struct Geo {
+  int n_packed, n_vl, T, NP, NV, NR, NT;
+};
+
+__device__ __forceinline__ Geo geo_of(int n_packed, int n_vl, int T) {
+  Geo g;
+  g.n_packed = n_packed;
+  g.n_vl = n_vl;
+  g.T = T;
+  g.NP = (n_packed + PK - 1) / PK;
+  g.NV = (n_vl + FT - 1) / FT;
+  g.NR = (T + 1 - n_packed + FT - 1) / FT;  // recent positions [n_packed, T) incl. the new token
+  g.NT = g.NP + g.NV + g.NR;
+  return g;
+}
+
+struct WarpState {
+  float m[2], l[2];
+  float o[8][4];
+};
+
+// Online-softmax update for NMT 16-key blocks whose S^T accumulators are in s.
+// Returns the P^T B-fragments (two per block) in pb.
+template <int NMT>
+__device__ __forceinline__ void softmax_update(WarpState& ws, float (&s)[NMT][4], uint32_t (&pb)[NMT][2]) {
+  float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < NMT; ++i) {
+    mx0 = fmaxf(mx0, fmaxf(s[i][0], s[i][2]));
+    mx1 = fmaxf(mx1, fmaxf(s[i][1], s[i][3]));
+  }
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+  }
+  const float mn0 = fmaxf(ws.m[0], mx0), mn1 = fmaxf(ws.m[1], mx1);
+  const float ref0 = mn0 == -INFINITY ? 0.f : mn0;
+  const float ref1 = mn1 == -INFINITY ? 0.f : mn1;
+  const float c0 = ex2(ws.m[0] - ref0), c1 = ex2(ws.m[1] - ref1);
+  ws.m[0] = mn0;
+  ws.m[1] = mn1;
+  ws.l[0] *= c0;
+  ws.l[1] *= c1;
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    ws.o[m][0] *= c0;
+    ws.o[m][2] *= c0;
+    ws.o[m][1] *= c1;
+    ws.o[m][3] *= c1;
+  }
+#pragma unroll
+  for (int i = 0; i < NMT; ++i) {
+    const float p0 = ex2(s[i][0] - ref0), p1 = ex2(s[i][1] - ref1);
+    const float p2 = ex2(s[i][2] - ref0), p3 = ex2(s[i][3] - ref1);
+    ws.l[0] += p0 + p2;
+    ws.l[1] += p1 + p3;
+    pb[i][0] = movmatrix_t(pack_f16x2(p0, p1));
+    pb[i][1] = movmatrix_t(pack_f16x2(p2, p3));
+  }
+}
+
+// one K4V4 packed tile (64 positions) by one warp
+__device__ __forceinline__ void packed_tile(WarpState& ws, const uint8_t* st, const uint32_t (&qf)[8][2], int tile, int n_packed,
+                                            float qscale, int g, int t) {
+  const uint8_t* kc = st;
+  const uint8_t* vc = st + OFF_VC;
+  const uint32_t* ks = reinterpret_cast<const uint32_t*>(st + OFF_KS);
+  const uint32_t* vs = reinterpret_cast<const uint32_t*>(st + OFF_VS);
+  const uint32_t* mk = reinterpret_cast<const uint32_t*>(st + OFF_MASK) + 2 * (tile & 1);
+  const int base = tile * PK;
+  const bool full = base + PK <= n_packed;
+
+  // ---- S^T = K^ . Q^T for 4 blocks of 16 keys
+  float s[4][4];
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+    const int ra = 16 * mt + pi_pk(g), rb = 16 * mt + pi_pk(g + 8);
+    const uint4 ka = *reinterpret_cast<const uint4*>(kc + ra * 64 + 16 * t);
+    const uint4 kb = *reinterpret_cast<const uint4*>(kc + rb * 64 + 16 * t);
+    const uint32_t za = ks[ra * 4 + t], zb = ks[rb * 4 + t];
+    const uint32_t sa2 = prmt(za, za, 0x1010), za2 = prmt(za, za, 0x3232);
+    const uint32_t sb2 = prmt(zb, zb, 0x1010), zb2 = prmt(zb, zb, 0x3232);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w};
+    const uint32_t wb[4] = {kb.x, kb.y, kb.z, kb.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t xa = wa[i] >> (8 * h), xb = wb[i] >> (8 * h);
+        const uint32_t a0 = hfma2_u(nib_lo(xa), sa2, za2);
+        const uint32_t a2 = hfma2_u(nib_hi(xa), sa2, za2);
+        const uint32_t a1 = hfma2_u(nib_lo(xb), sb2, zb2);
+        const uint32_t a3 = hfma2_u(nib_hi(xb), sb2, zb2);
+        mma16816(acc, a0, a1, a2, a3, qf[2 * i + h][0], qf[2 * i + h][1]);
+      }
+    }
+    // mask: beyond n_packed, or a vertical line (its FP16 row is read instead)
+    const int la = 16 * mt + pi_pk(g), lb = 16 * mt + pi_pk(g + 8);
+    const bool va = (base + la < n_packed) && !((mk[la >> 5] >> (la & 31)) & 1u);
+    const bool vb = (base + lb < n_packed) && !((mk[lb >> 5] >> (lb & 31)) & 1u);
+    s[mt][0] = va ? acc[0] * qscale : -INFINITY;
+    s[mt][1] = va ? acc[1] * qscale : -INFINITY;
+    s[mt][2] = vb ? acc[2] * qscale : -INFINITY;
+    s[mt][3] = vb ? acc[3] * qscale : -INFINITY;
+  }
+  uint32_t pb[4][2];
+  softmax_update<4>(ws, s, pb);
+
+  // ---- O^T += V^T . P^T, one k-step per 16-key block
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+    const int r0 = 16 * mt + pi_pk(2 * t), r1 = 16 * mt + pi_pk(2 * t + 1);
+    const int r2 = 16 * mt + pi_pk(2 * t + 8), r3 = 16 * mt + pi_pk(2 * t + 9);
+    // two 32-bit loads per row, issued in a per-thread order that keeps the
+    // warp's accesses on distinct banks
+    const int e = t >> 1;
+    const uint32_t* v0 = reinterpret_cast<const uint32_t*>(vc + r0 * 64) + 2 * g;
+    const uint32_t* v1 = reinterpret_cast<const uint32_t*>(vc + r1 * 64) + 2 * g;
+    const uint32_t* v2 = reinterpret_cast<const uint32_t*>(vc + r2 * 64) + 2 * g;
+    const uint32_t* v3 = reinterpret_cast<const uint32_t*>(vc + r3 * 64) + 2 * g;
+    uint32_t x0a = v0[e], x0b = v0[e ^ 1], x1a = v1[e], x1b = v1[e ^ 1];
+    uint32_t x2a = v2[e], x2b = v2[e ^ 1], x3a = v3[e], x3b = v3[e ^ 1];
+    // un-rotate: w?0 = word 2g, w?1 = word 2g+1
+    const uint32_t w00 = e ? x0b : x0a, w01 = e ? x0a : x0b;
+    const uint32_t w10 = e ? x1b : x1a, w11 = e ? x1a : x1b;
+    const uint32_t w20 = e ? x2b : x2a, w21 = e ? x2a : x2b;
+    const uint32_t w30 = e ? x3b : x3a, w31 = e ? x3a : x3b;
+    const int grp = g >> 1;
+    const uint32_t z0 = vs[r0 * 4 + grp], z1 = vs[r1 * 4 + grp], z2 = vs[r2 * 4 + grp], z3 = vs[r3 * 4 + grp];
+    const uint32_t s01 = prmt(z0, z1, 0x5410), o01 = prmt(z0, z1, 0x7632);
+    const uint32_t s23 = prmt(z2, z3, 0x5410), o23 = prmt(z2, z3, 0x7632);
+    // pair nibbles of the two keys: x?[k] holds dims 16g + 4k .. 16g + 4k + 3 of both keys
+    uint32_t xab[4], xcd[4];
+    xab[0] = prmt(w00, w10, 0x5410);
+    xab[1] = prmt(w00, w10, 0x7632);
+    xab[2] = prmt(w01, w11, 0x5410);
+    xab[3] = prmt(w01, w11, 0x7632);
+    xcd[0] = prmt(w20, w30, 0x5410);
+    xcd[1] = prmt(w20, w30, 0x7632);
+    xcd[2] = prmt(w21, w31, 0x5410);
+    xcd[3] = prmt(w21, w31, 0x7632);
+    bool zero_ab = false, zero_cd = false;
+    uint32_t keep_ab = 0xFFFFFFFFu, keep_cd = 0xFFFFFFFFu;
+    if (!full) {  // rows past n_packed may hold stale records: zero them out of P.V
+      const bool a = base + r0 < n_packed, b = base + r1 < n_packed;
+      const bool cc = base + r2 < n_packed, dd = base + r3 < n_packed;
+      keep_ab = (a ? 0x0000FFFFu : 0u) | (b ? 0xFFFF0000u : 0u);
+      keep_cd = (cc ? 0x0000FFFFu : 0u) | (dd ? 0xFFFF0000u : 0u);
+      zero_ab = !(a && b);
+      zero_cd = !(cc && dd);
+    }
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      const uint32_t yab = xab[m >> 1] >> (8 * (m & 1));
+      const uint32_t ycd = xcd[m >> 1] >> (8 * (m & 1));
+      uint32_t a0 = hfma2_u(nib_lo(yab), s01, o01);
+      uint32_t a1 = hfma2_u(nib_hi(yab), s01, o01);
+      uint32_t a2 = hfma2_u(nib_lo(ycd), s23, o23);
+      uint32_t a3 = hfma2_u(nib_hi(ycd), s23, o23);
+      if (zero_ab) { a0 &= keep_ab; a1 &= keep_ab; }
+      if (zero_cd) { a2 &= keep_cd; a3 &= keep_cd; }
+      mma16816(ws.o[m], a0, a1, a2, a3, pb[mt][0], pb[mt][1]);
+    }
+  }
+}
+
+// one FP16 tile (16 rows at FSTRIDE) by one warp; `nvalid` leading rows are real
+__device__ __forceinline__ void fp16_tile(WarpState& ws, const uint8_t* st, const uint32_t (&qf)[8][2], int nvalid,
+                                          float qscale, int g, int t) {
+  const uint8_t* kb = st;
+  const uint8_t* vb = st + OFF_FV;
+  const int ra = pi_fp(g), rb = pi_fp(g + 8);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 ua = *reinterpret_cast<const uint4*>(kb + ra * FSTRIDE + 64 * t + 16 * i);
+    const uint4 ub = *reinterpret_cast<const uint4*>(kb + rb * FSTRIDE + 64 * t + 16 * i);
+    // k-step 2i: (d0,d4) and (d1,d5); k-step 2i+1: (d2,d6) and (d3,d7)
+    mma16816(acc, prmt(ua.x, ua.z, 0x5410), prmt(ub.x, ub.z, 0x5410), prmt(ua.x, ua.z, 0x7632), prmt(ub.x, ub.z, 0x7632),
+             qf[2 * i][0], qf[2 * i][1]);
+    mma16816(acc, prmt(ua.y, ua.w, 0x5410), prmt(ub.y, ub.w, 0x5410), prmt(ua.y, ua.w, 0x7632), prmt(ub.y, ub.w, 0x7632),
+             qf[2 * i + 1][0], qf[2 * i + 1][1]);
+  }
+  float s[1][4];
+  const bool va = ra < nvalid, vbv = rb < nvalid;
+  s[0][0] = va ? acc[0] * qscale : -INFINITY;
+  s[0][1] = va ? acc[1] * qscale : -INFINITY;
+  s[0][2] = vbv ? acc[2] * qscale : -INFINITY;
+  s[0][3] = vbv ? acc[3] * qscale : -INFINITY;
+  uint32_t pb[1][2];
+  softmax_update<1>(ws, s, pb);
+
+  const int r0 = pi_fp(2 * t), r1 = pi_fp(2 * t + 1), r2 = pi_fp(2 * t + 8), r3 = pi_fp(2 * t + 9);
+  const uint4 a0l = *reinterpret_cast<const uint4*>(vb + r0 * FSTRIDE + 32 * g);
+  const uint4 a0h = *reinterpret_cast<const uint4*>(vb + r0 * FSTRIDE + 32 * g + 16);
+  const uint4 a1l = *reinterpret_cast<const uint4*>(vb + r1 * FSTRIDE + 32 * g);
+  const uint4 a1h = *reinterpret_cast<const uint4*>(vb + r1 * FSTRIDE + 32 * g + 16);
+  const uint4 a2l = *reinterpret_cast<const uint4*>(vb + r2 * FSTRIDE + 32 * g);
+  const uint4 a2h = *reinterpret_cast<const uint4*>(vb + r2 * FSTRIDE + 32 * g + 16);
+  const uint4 a3l = *reinterpret_cast<const uint4*>(vb + r3 * FSTRIDE + 32 * g);
+  const uint4 a3h = *reinterpret_cast<const uint4*>(vb + r3 * FSTRIDE + 32 * g + 16);
+  uint32_t w0[8] = {a0l.x, a0l.y, a0l.z, a0l.w, a0h.x, a0h.y, a0h.z, a0h.w};
+  uint32_t w1[8] = {a1l.x, a1l.y, a1l.z, a1l.w, a1h.x, a1h.y, a1h.z, a1h.w};
+  uint32_t w2[8] = {a2l.x, a2l.y, a2l.z, a2l.w, a2h.x, a2h.y, a2h.z, a2h.w};
+  uint32_t w3[8] = {a3l.x, a3l.y, a3l.z, a3l.w, a3h.x, a3h.y, a3h.z, a3h.w};
+  if (nvalid < FT) {  // rows not copied this time hold stale bytes: keep them out of P.V
+    const uint32_t k0 = r0 < nvalid ? 0xFFFFFFFFu : 0u, k1 = r1 < nvalid ? 0xFFFFFFFFu : 0u;
+    const uint32_t k2 = r2 < nvalid ? 0xFFFFFFFFu : 0u, k3 = r3 < nvalid ? 0xFFFFFFFFu : 0u;
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      w0[m] &= k0; w1[m] &= k1; w2[m] &= k2; w3[m] &= k3;
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    mma16816(ws.o[m], prmt(w0[m], w1[m], 0x5410), prmt(w0[m], w1[m], 0x7632), prmt(w2[m], w3[m], 0x5410),
+             prmt(w2[m], w3[m], 0x7632), pb[0][0], pb[0][1]);
+  }
+}
+
+__global__ void __launch_bounds__(NTHREADS, 2)
+decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* __restrict__ k_new,
+              const uint16_t* __restrict__ v_new, uint16_t* __restrict__ out, float qscale, int S,
+              float* __restrict__ parts, unsigned int* __restrict__ tickets) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ __align__(8) uint64_t full[NSTAGES], empty[NSTAGES];
+  __shared__ int s_last;
+
+  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int bh = b * c.Hkv + kvh;
+  const int G = c.Hq / c.Hkv;
+  const int R = c.W + HQ_STAGE;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+
+  const int T = c.state[HQ_STATE_T];
+  const int n_packed = c.state[HQ_STATE_NPACKED];
+  const int n_vl = c.state[HQ_STATE_NVL];
+  if (T - n_packed >= R || T >= c.cap) {  // staging full / no room: do nothing
+    if (split == 0 && kvh == 0 && b == 0 && threadIdx.x == 0)
+      set_err(c.state, T >= c.cap ? HQ_DEVERR_CAPACITY : HQ_DEVERR_STAGING_FULL);
+    return;
+  }
+  const Geo geo = geo_of(n_packed, n_vl, T);
+  const int t_lo = static_cast<int>((static_cast<long long>(split) * geo.NT) / S);
+  const int t_hi = static_cast<int>((static_cast<long long>(split + 1) * geo.NT) / S);
+  const int ntile = t_hi - t_lo;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NSTAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    fence_mbar_init();
+  }
+  // append the new token: ring slot T % R and query-buffer slot T % HQ_QBUF
+  if (split == 0) {
+    const int slot = T % R;
+    for (int i = threadIdx.x; i < 2 * D / 8; i += NTHREADS) {
+      const int which = i / (D / 8), ch = i % (D / 8);
+      const uint4* s = reinterpret_cast<const uint4*>((which ? v_new : k_new) + static_cast<size_t>(bh) * D) + ch;
+      uint4* d = reinterpret_cast<uint4*>((which ? c.vr : c.kr) + (static_cast<size_t>(bh) * R + slot) * D) + ch;
+      *d = *s;
+    }
+    for (int i = threadIdx.x; i < G * D / 8; i += NTHREADS) {
+      const int h = kvh * G + i / (D / 8), ch = i % (D / 8);
+      const uint4* s = reinterpret_cast<const uint4*>(q + (static_cast<size_t>(b) * c.Hq + h) * D) + ch;
+      uint4* d = reinterpret_cast<uint4*>(c.qbuf + ((static_cast<size_t>(b) * c.Hq + h) * HQ_QBUF + (T % HQ_QBUF)) * D) + ch;
+      *d = *s;
+    }
+  }
+  __syncthreads();
+
+  WarpState ws;
+  ws.m[0] = ws.m[1] = -INFINITY;
+  ws.l[0] = ws.l[1] = 0.f;
+#pragma unroll
+  for (int m = 0; m < 8; ++m) ws.o[m][0] = ws.o[m][1] = ws.o[m][2] = ws.o[m][3] = 0.f;
+
+  if (warp == NCONS) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      for (int i = 0; i < ntile; ++i) {
+        const int s = i % NSTAGES;
+        if (i >= NSTAGES && !mbar_wait(&empty[s], ((i / NSTAGES) & 1) ^ 1, c.state)) break;
+        uint8_t* st = smem + s * STAGE_BYTES;
+        const int tile = t_lo + i;
+        if (tile < geo.NP) {
+          const size_t row0 = static_cast<size_t>(bh) * c.cap + static_cast<size_t>(tile) * PK;
+          mbar_arrive_expect_tx(&full[s], PK_TX);
+          bulk_g2s(st, c.kq + row0 * (D / 2), 4096, &full[s]);
+          bulk_g2s(st + OFF_VC, c.vq + row0 * (D / 2), 4096, &full[s]);
+          bulk_g2s(st + OFF_KS, c.ksz + row0 * 4, 1024, &full[s]);
+          bulk_g2s(st + OFF_VS, c.vsz + row0 * 4, 1024, &full[s]);
+          bulk_g2s(st + OFF_MASK, c.vl_mask + static_cast<size_t>(bh) * (c.cap / 32) + 4 * (tile >> 1), 16, &full[s]);
+        } else if (tile < geo.NP + geo.NV) {
+          const int r0 = (tile - geo.NP) * FT;
+          const int nr = min(FT, n_vl - r0);
+          mbar_arrive_expect_tx(&full[s], nr * 2 * D * 2);
+          for (int r = 0; r < nr; ++r) {
+            const size_t row = static_cast<size_t>(bh) * c.vl_cap + r0 + r;
+            bulk_g2s(st + r * FSTRIDE, c.kf + row * D, 2 * D, &full[s]);
+            bulk_g2s(st + OFF_FV + r * FSTRIDE, c.vf + row * D, 2 * D, &full[s]);
+          }
+        } else {
+          const int p0 = n_packed + (tile - geo.NP - geo.NV) * FT;
+          const int nr = min(FT, T + 1 - p0);
+          mbar_arrive_expect_tx(&full[s], nr * 2 * D * 2);
+          for (int r = 0; r < nr; ++r) {
+            const int p = p0 + r;
+            const uint16_t* ks;
+            const uint16_t* vs;
+            if (p < T) {
+              ks = c.kr + (static_cast<size_t>(bh) * R + (p % R)) * D;
+              vs = c.vr + (static_cast<size_t>(bh) * R + (p % R)) * D;
+            } else {
+              ks = k_new + static_cast<size_t>(bh) * D;
+              vs = v_new + static_cast<size_t>(bh) * D;
+            }
+            bulk_g2s(st + r * FSTRIDE, ks, 2 * D, &full[s]);
+            bulk_g2s(st + OFF_FV + r * FSTRIDE, vs, 2 * D, &full[s]);
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- consumers
+    // Q^T fragments in the permuted dim order (thread t covers dims 32t .. 32t+31)
+    uint32_t qf[8][2];
+    if (g < G) {
+      const uint4* qp = reinterpret_cast<const uint4*>(q + (static_cast<size_t>(b) * c.Hq + kvh * G + g) * D + 32 * t);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 u = qp[i];
+        qf[2 * i][0] = prmt(u.x, u.z, 0x5410);
+        qf[2 * i][1] = prmt(u.x, u.z, 0x7632);
+        qf[2 * i + 1][0] = prmt(u.y, u.w, 0x5410);
+        qf[2 * i + 1][1] = prmt(u.y, u.w, 0x7632);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) qf[j][0] = qf[j][1] = 0u;
+    }
+    for (int i = warp; i < ntile; i += NCONS) {
+      const int s = i % NSTAGES;
+      // the timeout decision is made warp-uniform so the warp never splits
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (i / NSTAGES) & 1, c.state))) break;
+      const uint8_t* st = smem + s * STAGE_BYTES;
+      const int tile = t_lo + i;
+      if (tile < geo.NP) {
+        packed_tile(ws, st, qf, tile, n_packed, qscale, g, t);
+      } else if (tile < geo.NP + geo.NV) {
+        fp16_tile(ws, st, qf, min(FT, n_vl - (tile - geo.NP) * FT), qscale, g, t);
+      } else {
+        fp16_tile(ws, st, qf, min(FT, T + 1 - (n_packed + (tile - geo.NP - geo.NV) * FT)), qscale, g, t);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    // l: sum the per-thread partial sums over the 8 lanes of a query column
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      ws.l[0] += __shfl_xor_sync(0xffffffffu, ws.l[0], o);
+      ws.l[1] += __shfl_xor_sync(0xffffffffu, ws.l[1], o);
+    }
+  }
+  __syncthreads();  // (A) every tile consumed: stage memory is free for the merge
+  if (warp < NCONS) {
+    float* wsm = reinterpret_cast<float*>(smem) + warp * PART_FLOATS;
+    if (g == 0) {
+      wsm[2 * t] = ws.m[0];
+      wsm[2 * t + 1] = ws.m[1];
+      wsm[8 + 2 * t] = ws.l[0];
+      wsm[8 + 2 * t + 1] = ws.l[1];
+    }
+    float* wo = wsm + 16;
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      wo[(2 * t) * D + 16 * g + 2 * m] = ws.o[m][0];
+      wo[(2 * t + 1) * D + 16 * g + 2 * m] = ws.o[m][1];
+      wo[(2 * t) * D + 16 * g + 2 * m + 1] = ws.o[m][2];
+      wo[(2 * t + 1) * D + 16 * g + 2 * m + 1] = ws.o[m][3];
+    }
+  }
+  __syncthreads();  // (B) warp states visible
+
+  // ---------------------------------------------------------------- CTA merge -> split partial
+  float* part = parts + (static_cast<size_t>(bh) * S + split) * PART_FLOATS;
+  const float* wsm = reinterpret_cast<const float*>(smem);
+  for (int i = threadIdx.x; i < 8 * D + 16; i += NTHREADS) {
+    if (i < 8) {
+      float mm = -INFINITY;
+      for (int w = 0; w < NCONS; ++w) mm = fmaxf(mm, wsm[w * PART_FLOATS + i]);
+      float ll = 0.f;
+      for (int w = 0; w < NCONS; ++w) {
+        const float mw = wsm[w * PART_FLOATS + i];
+        ll += mw == -INFINITY ? 0.f : wsm[w * PART_FLOATS + 8 + i] * ex2(mw - mm);
+      }
+      part[i] = mm;
+      part[8 + i] = ll;
+    } else if (i >= 16) {
+      const int qc = (i - 16) / D;
+      float mm = -INFINITY;
+      for (int w = 0; w < NCONS; ++w) mm = fmaxf(mm, wsm[w * PART_FLOATS + qc]);
+      float acc = 0.f;
+      for (int w = 0; w < NCONS; ++w) {
+        const float mw = wsm[w * PART_FLOATS + qc];
+        acc += mw == -INFINITY ? 0.f : wsm[w * PART_FLOATS + i] * ex2(mw - mm);
+      }
+      part[i] = acc;
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (atomicAdd(&tickets[1 + bh], 1u) == static_cast<unsigned>(S - 1)) ? 1 : 0;
+  __syncthreads();
+  if (s_last) {
+    __threadfence();
+    // log-sum-exp merge of the S partials of this (b, kv head)
+    const float* pb = parts + static_cast<size_t>(bh) * S * PART_FLOATS;
+    for (int i = threadIdx.x; i < G * D; i += NTHREADS) {
+      const int qc = i / D, dd = i % D;
+      float mm = -INFINITY;
+      for (int sp = 0; sp < S; ++sp) mm = fmaxf(mm, __ldcg(pb + sp * PART_FLOATS + qc));
+      float ll = 0.f, acc = 0.f;
+      for (int sp = 0; sp < S; ++sp) {
+        const float ms = __ldcg(pb + sp * PART_FLOATS + qc);
+        if (ms == -INFINITY) continue;
+        const float w = ex2(ms - mm);
+        ll += __ldcg(pb + sp * PART_FLOATS + 8 + qc) * w;
+        acc += __ldcg(pb + sp * PART_FLOATS + 16 + qc * D + dd) * w;
+      }
+      out[(static_cast<size_t>(b) * c.Hq + kvh * G + qc) * D + dd] = __half_as_ushort(__float2half_rn(acc / ll));
+    }
+    if (threadIdx.x == 0) {
+      tickets[1 + bh] = 0u;
+      __threadfence();
+    }
+  }
+  // grid-wide: the last CTA advances T (every CTA has read the state by now)
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned total = gridDim.x * gridDim.y * gridDim.z;
+    if (atomicAdd(&tickets[0], 1u) == total - 1) {
+      c.state[HQ_STATE_T] = T + 1;
+      c.state[HQ_STATE_NQ] = min(c.state[HQ_STATE_NQ] + 1, HQ_QBUF);
+      tickets[0] = 0u;
+      __threadfence();
+    }
+  }
+}
+
+}  // namespace
+
+int decode_splits(const hq_cache& c, int sms) {
+  const int units = c.B * c.Hkv;
+  const int nt_max = c.cap / PK + c.vl_cap / FT + (c.W + HQ_STAGE + 1 + FT - 1) / FT;
+  int s = (2 * sms + units - 1) / units;
+  const int cap_s = (nt_max + 3) / 4;
+  if (s > cap_s) s = cap_s;
+  if (s < 1) s = 1;
+  return s;
+}
+
+// counters: [0] grid ticket, [1 + b*Hkv + h] split tickets; zero between calls
+size_t decode_counter_bytes(const hq_cache& c) { return ((4ull * (1 + c.B * c.Hkv) + 255) / 256) * 256; }
+
+size_t decode_workspace(const hq_cache& c, int sms) {
+  const int S = decode_splits(c, sms);
+  return decode_counter_bytes(c) + static_cast<size_t>(c.B) * c.Hkv * S * PART_FLOATS * sizeof(float);
+}
+
+hq_status launch_decode(const hq_cache& c, const uint16_t* q, const uint16_t* kn, const uint16_t* vn, uint16_t* out,
+                        float sm_scale, void* ws, int sms, cudaStream_t st) {
+  const int S = decode_splits(c, sms);
+  const int smem = NSTAGES * STAGE_BYTES;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static bool attr_done[64] = {};
+  if (dev >= 64 || !attr_done[dev]) {
+    if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return HQ_ERR_CUDA;
+    if (dev < 64) attr_done[dev] = true;
+  }
+  unsigned int* tickets = reinterpret_cast<unsigned int*>(ws);
+  float* parts = reinterpret_cast<float*>(static_cast<char*>(ws) + decode_counter_bytes(c));
+  dim3 grid(S, c.Hkv, c.B);
+  decode_kernel<<<grid, NTHREADS, smem, st>>>(c, q, kn, vn, out, sm_scale * LOG2E, S, parts, tickets);
+  return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+}
+
+}  // namespace hq

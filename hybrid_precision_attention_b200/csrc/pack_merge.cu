@@ -1,0 +1,270 @@
+// pack_merge.cu — K4V4 packing and the staging -> hybrid merge.
+//
+// HyQuant digest (agihunt.info), prefill/decode paragraph: new decode tokens
+// are staged first and merged into the hybrid layout later; the VL set chosen
+// by the selector keeps FP16 rows, everything that leaves the recent window
+// is stored 4-bit.  The K4V4 arithmetic follows the format definition in
+// hq.h exactly (float32 RN subtract/divide, rint to even, fp16 RN), so the
+// packed bytes are bit-identical to the definition.
+//
+// Kernels (all bandwidth-trivial next to decode; one warp per row):
+//   pack_rows      positions [lo, hi) of every (b, kv head) -> K4V4 records
+//   ring_fill      init only: last min(W, L) prefix rows -> FP16 ring
+//   vl_gather      merge only: new VL rows -> workspace (old VL row, ring row,
+//                  or the dequantised record rounded once to fp16); clears old bits
+//   vl_install     rows -> VL store, positions, bitmap bits, state update
+#include "common.cuh"
+
+namespace hq {
+namespace {
+
+struct Dims {
+  int B, Hkv, cap, vl_cap, R, W;
+};
+
+__device__ __forceinline__ Dims dims_of(const hq_cache& c) { return Dims{c.B, c.Hkv, c.cap, c.vl_cap, c.W + HQ_STAGE, c.W}; }
+
+// Pack one 128-value fp16 row into 64 code bytes + 4 (scale, zero) words.
+// Warp-cooperative: lane l owns values 4l .. 4l+3 (group l / 8).
+__device__ __forceinline__ void pack_row_warp(const uint16_t* __restrict__ src, uint8_t* __restrict__ codes,
+                                              uint32_t* __restrict__ sz, int lane) {
+  const uint2 raw = *reinterpret_cast<const uint2*>(src + 4 * lane);
+  float x[4];
+  x[0] = __half2float(__ushort_as_half(static_cast<unsigned short>(raw.x & 0xFFFFu)));
+  x[1] = __half2float(__ushort_as_half(static_cast<unsigned short>(raw.x >> 16)));
+  x[2] = __half2float(__ushort_as_half(static_cast<unsigned short>(raw.y & 0xFFFFu)));
+  x[3] = __half2float(__ushort_as_half(static_cast<unsigned short>(raw.y >> 16)));
+  float mn = fminf(fminf(x[0], x[1]), fminf(x[2], x[3]));
+  float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  // scale = fp16_RN(fp32(mx - mn) / 15), zero = mn (an fp16 value, exact in fp32)
+  const float span = __fsub_rn(mx, mn);
+  const __half scale_h = __float2half_rn(__fdiv_rn(span, 15.0f));
+  const float scale = __half2float(scale_h);
+  uint32_t q[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float r = scale == 0.0f ? 0.0f : rintf(__fdiv_rn(__fsub_rn(x[i], mn), scale));
+    r = fminf(fmaxf(r, 0.0f), 15.0f);
+    q[i] = static_cast<uint32_t>(r);
+  }
+  const uint32_t two = (q[0] | (q[1] << 4)) | ((q[2] | (q[3] << 4)) << 8);
+  reinterpret_cast<uint16_t*>(codes)[lane] = static_cast<uint16_t>(two);
+  if ((lane & 7) == 0) {
+    const uint32_t zbits = __half_as_ushort(__float2half_rn(mn));  // exact: mn is an fp16 value
+    sz[lane >> 3] = static_cast<uint32_t>(__half_as_ushort(scale_h)) | (zbits << 16);
+  }
+}
+
+// Rows [lo, hi) of every (b, kv head), K and V.  Init: src = dense [B,Hkv,L,D],
+// lo = 0, hi = max(L - W, 0).  Merge: src = ring, lo = n_packed, hi = T - W
+// (read from state).
+__global__ void pack_rows_kernel(hq_cache c, const uint16_t* __restrict__ kd, const uint16_t* __restrict__ vd, int L,
+                                 int init) {
+  const Dims d = dims_of(c);
+  int lo, hi;
+  if (init) {
+    lo = 0;
+    hi = max(L - d.W, 0);
+  } else {
+    lo = c.state[HQ_STATE_NPACKED];
+    hi = max(lo, c.state[HQ_STATE_T] - d.W);
+  }
+  const int n = hi - lo;
+  if (n <= 0) return;
+  const int lane = threadIdx.x & 31;
+  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  const long long total = 2ll * d.B * d.Hkv * n;  // (K or V) x (b, h) x rows
+  for (long long w = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); w < total; w += warps) {
+    const int which = static_cast<int>(w & 1);
+    const long long rest = w >> 1;
+    const int p = lo + static_cast<int>(rest % n);
+    const long long bh = rest / n;
+    const uint16_t* src;
+    if (init) {
+      src = (which ? vd : kd) + (bh * L + p) * D;
+    } else {
+      src = (which ? c.vr : c.kr) + (bh * d.R + (p % d.R)) * D;
+    }
+    uint8_t* codes = (which ? c.vq : c.kq) + (bh * d.cap + p) * (D / 2);
+    uint32_t* sz = (which ? c.vsz : c.ksz) + (bh * d.cap + p) * (D / HQ_GROUP);
+    pack_row_warp(src, codes, sz, lane);
+  }
+}
+
+// Init: prefix rows [max(L-W,0), L) -> ring slots p % R.
+__global__ void ring_fill_kernel(hq_cache c, const uint16_t* __restrict__ kd, const uint16_t* __restrict__ vd, int L) {
+  const Dims d = dims_of(c);
+  const int lo = max(L - d.W, 0);
+  const int n = L - lo;
+  if (n <= 0) return;
+  const long long total = 2ll * d.B * d.Hkv * n * (D / 8);  // 16-byte chunks
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int chunk = static_cast<int>(i % (D / 8));
+    long long r = i / (D / 8);
+    const int which = static_cast<int>(r & 1);
+    r >>= 1;
+    const int p = lo + static_cast<int>(r % n);
+    const long long bh = r / n;
+    const uint4* s = reinterpret_cast<const uint4*>((which ? vd : kd) + (bh * L + p) * D) + chunk;
+    uint4* t = reinterpret_cast<uint4*>((which ? c.vr : c.kr) + (bh * d.R + (p % d.R)) * D) + chunk;
+    *t = *s;
+  }
+}
+
+__device__ __forceinline__ int find_sorted(const int32_t* __restrict__ a, int n, int key) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (a[mid] < key) lo = mid + 1; else hi = mid;
+  }
+  return (lo < n && a[lo] == key) ? lo : -1;
+}
+
+// Merge: gather the FP16 rows of the new VL set into the workspace and clear the
+// bitmap bits of the old set.  One warp per (b, h, r, K|V).
+__global__ void vl_gather_kernel(hq_cache c, uint16_t* __restrict__ wsk, uint16_t* __restrict__ wsv) {
+  const Dims d = dims_of(c);
+  const int n_packed = c.state[HQ_STATE_NPACKED];
+  const int n_vl = c.state[HQ_STATE_NVL];
+  const int k = min(c.state[HQ_STATE_KSEL], d.vl_cap);
+  const int lane = threadIdx.x & 31;
+  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  const long long total = 2ll * d.B * d.Hkv * k;
+  for (long long w = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); w < total; w += warps) {
+    const int which = static_cast<int>(w & 1);
+    const long long rest = w >> 1;
+    const int r = static_cast<int>(rest % k);
+    const long long bh = rest / k;
+    const int p = c.vl_sel[bh * d.vl_cap + r];
+    uint16_t* dst = (which ? wsv : wsk) + (bh * d.vl_cap + r) * D;
+    if (p < 0 || p >= max(n_packed, c.state[HQ_STATE_T] - d.W)) {  // not a position the merge can hold
+      if (lane == 0) set_err(c.state, HQ_DEVERR_VL_CAPACITY);
+      continue;
+    }
+    const int old = find_sorted(c.vl_pos + bh * d.vl_cap, n_vl, p);
+    if (old >= 0) {
+      const uint16_t* s = (which ? c.vf : c.kf) + (bh * d.vl_cap + old) * D;
+      reinterpret_cast<uint2*>(dst)[lane] = reinterpret_cast<const uint2*>(s)[lane];
+    } else if (p >= n_packed) {
+      const uint16_t* s = (which ? c.vr : c.kr) + (bh * d.R + (p % d.R)) * D;
+      reinterpret_cast<uint2*>(dst)[lane] = reinterpret_cast<const uint2*>(s)[lane];
+    } else {
+      // promoted packed position: fp16(zero + q * scale); q * scale is exact in
+      // float64 and the sum is rounded once, then once more to fp16 (RN).
+      const uint8_t* codes = (which ? c.vq : c.kq) + (bh * d.cap + p) * (D / 2);
+      const uint32_t szw = (which ? c.vsz : c.ksz)[(bh * d.cap + p) * (D / HQ_GROUP) + (lane >> 3)];
+      const double sc = static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(szw & 0xFFFFu))));
+      const double ze = static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(szw >> 16))));
+      const uint32_t two = reinterpret_cast<const uint16_t*>(codes)[lane];
+      uint32_t out[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const uint32_t byte = (two >> (8 * i)) & 0xFFu;
+        const double v0 = __dadd_rn(ze, __dmul_rn(static_cast<double>(byte & 15u), sc));
+        const double v1 = __dadd_rn(ze, __dmul_rn(static_cast<double>(byte >> 4), sc));
+        out[i] = static_cast<uint32_t>(__half_as_ushort(__double2half(v0))) |
+                 (static_cast<uint32_t>(__half_as_ushort(__double2half(v1))) << 16);
+      }
+      reinterpret_cast<uint2*>(dst)[lane] = make_uint2(out[0], out[1]);
+    }
+  }
+  // clear the old set's bitmap bits (nothing in this kernel reads the bitmap)
+  const long long tot2 = static_cast<long long>(d.B) * d.Hkv * n_vl;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < tot2;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long bh = i / n_vl;
+    const int r = static_cast<int>(i % n_vl);
+    const int p = c.vl_pos[bh * d.vl_cap + r];
+    atomicAnd(c.vl_mask + bh * (d.cap / 32) + (p >> 5), ~(1u << (p & 31)));
+  }
+}
+
+// Install rows into the VL store.  Init: rows from the dense prefix; merge: rows
+// from the workspace.  Sets bitmap bits, writes vl_pos.  The last block to finish
+// (ticket) updates the state words.
+__global__ void vl_install_kernel(hq_cache c, const uint16_t* __restrict__ srck, const uint16_t* __restrict__ srcv, int L,
+                                  int init, unsigned int* __restrict__ ticket) {
+  const Dims d = dims_of(c);
+  const int k = min(c.state[HQ_STATE_KSEL], d.vl_cap);
+  const long long chunks = 2ll * d.B * d.Hkv * k * (D / 8);
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < chunks;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int ch = static_cast<int>(i % (D / 8));
+    long long r = i / (D / 8);
+    const int which = static_cast<int>(r & 1);
+    r >>= 1;
+    const int row = static_cast<int>(r % k);
+    const long long bh = r / k;
+    const int p = c.vl_sel[bh * d.vl_cap + row];
+    const int limit = init ? max(L - d.W, 0) : max(c.state[HQ_STATE_NPACKED], c.state[HQ_STATE_T] - d.W);
+    if (p < 0 || p >= limit) {
+      if (ch == 0 && which == 0) set_err(c.state, HQ_DEVERR_VL_CAPACITY);
+      continue;
+    }
+    const uint16_t* s = init ? ((which ? srcv : srck) + (bh * L + p) * D) : ((which ? srcv : srck) + (bh * d.vl_cap + row) * D);
+    uint16_t* t = (which ? c.vf : c.kf) + (bh * d.vl_cap + row) * D;
+    reinterpret_cast<uint4*>(t)[ch] = reinterpret_cast<const uint4*>(s)[ch];
+    if (ch == 0 && which == 0) {
+      c.vl_pos[bh * d.vl_cap + row] = p;
+      atomicOr(c.vl_mask + bh * (d.cap / 32) + (p >> 5), 1u << (p & 31));
+    }
+  }
+  // state update by the last block (every block has read state above)
+  __syncthreads();
+  __shared__ unsigned int last;
+  if (threadIdx.x == 0) {
+    __threadfence();
+    last = (atomicAdd(ticket, 1u) == gridDim.x - 1) ? 1u : 0u;
+  }
+  __syncthreads();
+  if (last && threadIdx.x == 0) {
+    if (init) {
+      c.state[HQ_STATE_T] = L;
+      c.state[HQ_STATE_NPACKED] = max(L - d.W, 0);
+      c.state[HQ_STATE_NQ] = 0;
+    } else {
+      const int t = c.state[HQ_STATE_T];
+      c.state[HQ_STATE_NPACKED] = max(c.state[HQ_STATE_NPACKED], t - d.W);
+    }
+    c.state[HQ_STATE_NVL] = k;
+    *ticket = 0u;
+  }
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ host launchers
+
+hq_status launch_pack_merge(const hq_cache& c, const uint16_t* kd, const uint16_t* vd, int L, void* ws, cudaStream_t st) {
+  const int init = kd != nullptr;
+  const int threads = 256;
+  int sms = 148;
+  {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  unsigned int* ticket = reinterpret_cast<unsigned int*>(ws);
+  uint16_t* wsk = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + 256);
+  uint16_t* wsv = wsk + static_cast<size_t>(c.B) * c.Hkv * c.vl_cap * D;
+  if (init) {
+    if (cudaMemsetAsync(c.vl_mask, 0, static_cast<size_t>(c.B) * c.Hkv * (c.cap / 32) * 4, st) != cudaSuccess) return HQ_ERR_CUDA;
+  }
+  pack_rows_kernel<<<sms * 4, threads, 0, st>>>(c, kd, vd, L, init);
+  if (init) {
+    ring_fill_kernel<<<sms, threads, 0, st>>>(c, kd, vd, L);
+    vl_install_kernel<<<sms, threads, 0, st>>>(c, kd, vd, L, 1, ticket);
+  } else {
+    vl_gather_kernel<<<sms * 2, threads, 0, st>>>(c, wsk, wsv);
+    vl_install_kernel<<<sms, threads, 0, st>>>(c, wsk, wsv, L, 0, ticket);
+  }
+  return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+}
+
+}  // namespace hq

@@ -1,0 +1,227 @@
+"""Thin Python binding over libhq.so (argument marshalling only).
+
+Every function here has the name of the C entry point it calls and does no
+arithmetic of its own: tensors are passed as device pointers, the status code
+is checked, and a non-zero status raises :class:`HqError`.  PyTorch is used for
+device memory and streams only.  If ``libhq.so`` is missing, importing this
+module raises: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhq.so")
+
+HQ_HEAD_DIM = 128
+HQ_STAGE = 64
+HQ_QBUF = 64
+STATE_T, STATE_NPACKED, STATE_NVL, STATE_NQ, STATE_KSEL, STATE_ERR = range(6)
+STATE_WORDS = 8
+OP_SELECT, OP_MERGE, OP_DECODE = 0, 1, 2
+DEVERR_STAGING_FULL, DEVERR_CAPACITY, DEVERR_VL_CAPACITY, DEVERR_TIMEOUT = 1, 2, 4, 8
+
+
+class HqError(RuntimeError):
+    pass
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is not built: run `python -m hybrid_precision_attention_b200.build`")
+_lib = ctypes.CDLL(LIB_PATH)
+
+
+class HqCacheStruct(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "Hq", "Hkv", "D", "W", "rho_bp", "cap", "vl_cap")] + [
+        (n, ctypes.c_void_p)
+        for n in ("kq", "vq", "ksz", "vsz", "kf", "vf", "vl_pos", "vl_mask", "kr", "vr", "qbuf", "vl_sel", "state")
+    ]
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+_S = ctypes.c_size_t
+_CP = ctypes.POINTER(HqCacheStruct)
+
+_lib.hq_abi_version.restype = _I
+_lib.hq_status_str.restype = ctypes.c_char_p
+_lib.hq_status_str.argtypes = [_I]
+_lib.hq_cache_validate.restype = _I
+_lib.hq_cache_validate.argtypes = [_CP]
+_lib.hq_workspace_bytes.restype = _S
+_lib.hq_workspace_bytes.argtypes = [_CP, _I, _I]
+_lib.hq_cache_reset.restype = _I
+_lib.hq_cache_reset.argtypes = [_CP, _P]
+_lib.hq_select_vlines.restype = _I
+_lib.hq_select_vlines.argtypes = [_CP, _P, _I, _P, _I, _P, _P, _S, _P]
+_lib.hq_pack_merge.restype = _I
+_lib.hq_pack_merge.argtypes = [_CP, _P, _P, _I, _P, _S, _P]
+_lib.hq_decode_attn.restype = _I
+_lib.hq_decode_attn.argtypes = [_CP, _P, _P, _P, _P, ctypes.c_float, _P, _S, _P]
+_lib.hq_prefill_workspace_bytes.restype = _S
+_lib.hq_prefill_workspace_bytes.argtypes = [_I, _I, _I, _I, _I]
+_lib.hq_prefill_attn.restype = _I
+_lib.hq_prefill_attn.argtypes = [_I, _I, _I, _I, _I, _P, _P, _P, _P, _I, _I, _I, ctypes.c_float, _P, _P, _S, _P]
+
+EXPORTED = ("hq_abi_version", "hq_status_str", "hq_cache_validate", "hq_workspace_bytes", "hq_cache_reset",
+            "hq_select_vlines", "hq_pack_merge", "hq_decode_attn", "hq_prefill_workspace_bytes", "hq_prefill_attn")
+
+
+def _check(st: int, what: str):
+    if st != 0:
+        raise HqError(f"{what}: {_lib.hq_status_str(st).decode()} (status {st})")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, dtype, shape, name):
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_cuda or not t.is_contiguous():
+        raise HqError(f"{name}: expected contiguous CUDA {dtype} {tuple(shape)}, got {t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def k_of(n: int, rho_bp: int) -> int:
+    """ceil(rho * n) in integer basis points (same rule as the kernels)."""
+    if n <= 0 or rho_bp <= 0:
+        return 0
+    return min(n, (n * rho_bp + 9999) // 10000)
+
+
+def abi_version() -> int:
+    return int(_lib.hq_abi_version())
+
+
+class HybridCache:
+    """Device buffers of one layer's hybrid cache (layout: include/hq.h, struct hq_cache)."""
+
+    def __init__(self, B: int, Hq: int, Hkv: int, cap: int, W: int = 128, rho_bp: int = 500, vl_cap: int = None,
+                 device="cuda", D: int = HQ_HEAD_DIM):
+        cap = ((cap + 127) // 128) * 128
+        if vl_cap is None:
+            vl_cap = max(16, ((k_of(max(cap - W, 0), rho_bp) + 15) // 16) * 16)
+        self.B, self.Hq, self.Hkv, self.D, self.W, self.rho_bp, self.cap, self.vl_cap = B, Hq, Hkv, D, W, rho_bp, cap, vl_cap
+        self.R = W + HQ_STAGE
+        dev = torch.device(device)
+        z = lambda shape, dt: torch.zeros(shape, dtype=dt, device=dev)
+        self.kq = z((B, Hkv, cap, D // 2), torch.uint8)
+        self.vq = z((B, Hkv, cap, D // 2), torch.uint8)
+        self.ksz = z((B, Hkv, cap, D // 32), torch.int32)
+        self.vsz = z((B, Hkv, cap, D // 32), torch.int32)
+        self.kf = z((B, Hkv, vl_cap, D), torch.float16)
+        self.vf = z((B, Hkv, vl_cap, D), torch.float16)
+        self.vl_pos = z((B, Hkv, vl_cap), torch.int32)
+        self.vl_mask = z((B, Hkv, cap // 32), torch.int32)
+        self.kr = z((B, Hkv, self.R, D), torch.float16)
+        self.vr = z((B, Hkv, self.R, D), torch.float16)
+        self.qbuf = z((B, Hq, HQ_QBUF, D), torch.float16)
+        self.vl_sel = z((B, Hkv, vl_cap), torch.int32)
+        self.state_t = z((STATE_WORDS,), torch.int32)
+        self.c = HqCacheStruct(B, Hq, Hkv, D, W, rho_bp, cap, vl_cap, *[t.data_ptr() for t in (
+            self.kq, self.vq, self.ksz, self.vsz, self.kf, self.vf, self.vl_pos, self.vl_mask, self.kr, self.vr,
+            self.qbuf, self.vl_sel, self.state_t)])
+        _check(_lib.hq_cache_validate(ctypes.byref(self.c)), "hq_cache_validate")
+        self._ws = {}
+
+    def workspace(self, op: int, L: int = 0) -> torch.Tensor:
+        n = int(_lib.hq_workspace_bytes(ctypes.byref(self.c), op, L))
+        if n == 0:
+            raise HqError("hq_workspace_bytes returned 0")
+        w = self._ws.get(op)
+        if w is None or w.numel() < n:
+            w = torch.zeros(n, dtype=torch.uint8, device=self.kq.device)
+            self._ws[op] = w
+        return w
+
+    def state(self) -> dict:
+        s = self.state_t.tolist()
+        return {"T": s[STATE_T], "n_packed": s[STATE_NPACKED], "n_vl": s[STATE_NVL], "n_q": s[STATE_NQ],
+                "k_sel": s[STATE_KSEL], "err": s[STATE_ERR]}
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in (self.kq, self.vq, self.ksz, self.vsz, self.kf, self.vf,
+                                                          self.vl_pos, self.vl_mask, self.kr, self.vr, self.qbuf,
+                                                          self.vl_sel, self.state_t))
+
+
+# ----------------------------------------------------------------------------- entry points
+
+def hq_cache_reset(cache: HybridCache, stream=None):
+    _check(_lib.hq_cache_reset(ctypes.byref(cache.c), _stream(stream)), "hq_cache_reset")
+
+
+def hq_select_vlines(cache: HybridCache, k_dense=None, q_ext=None, scores_out=None, stream=None):
+    """Init mode when k_dense [B,Hkv,L,D] and q_ext [B,Hq,nq,D] are given, else decode mode."""
+    L = nq = 0
+    if k_dense is not None:
+        L = k_dense.shape[2]
+        nq = q_ext.shape[2]
+        _need(k_dense, torch.float16, (cache.B, cache.Hkv, L, cache.D), "k_dense")
+        _need(q_ext, torch.float16, (cache.B, cache.Hq, nq, cache.D), "q_ext")
+    if scores_out is not None:
+        _need(scores_out, torch.float32, (cache.B, cache.Hkv, cache.cap), "scores_out")
+    ws = cache.workspace(OP_SELECT, L)
+    _check(_lib.hq_select_vlines(ctypes.byref(cache.c), _ptr(k_dense), L, _ptr(q_ext), nq, _ptr(scores_out),
+                                 _ptr(ws), ws.numel(), _stream(stream)), "hq_select_vlines")
+
+
+def hq_pack_merge(cache: HybridCache, k_dense=None, v_dense=None, stream=None):
+    """Init mode with dense K/V [B,Hkv,L,D]; merge mode with neither."""
+    L = 0
+    if k_dense is not None:
+        L = k_dense.shape[2]
+        _need(k_dense, torch.float16, (cache.B, cache.Hkv, L, cache.D), "k_dense")
+        _need(v_dense, torch.float16, (cache.B, cache.Hkv, L, cache.D), "v_dense")
+    ws = cache.workspace(OP_MERGE)
+    _check(_lib.hq_pack_merge(ctypes.byref(cache.c), _ptr(k_dense), _ptr(v_dense), L, _ptr(ws), ws.numel(),
+                              _stream(stream)), "hq_pack_merge")
+
+
+def hq_decode_attn(cache: HybridCache, q, k_new, v_new, out=None, sm_scale: float = None, stream=None):
+    _need(q, torch.float16, (cache.B, cache.Hq, cache.D), "q")
+    _need(k_new, torch.float16, (cache.B, cache.Hkv, cache.D), "k_new")
+    _need(v_new, torch.float16, (cache.B, cache.Hkv, cache.D), "v_new")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, torch.float16, (cache.B, cache.Hq, cache.D), "out")
+    if sm_scale is None:
+        sm_scale = cache.D ** -0.5
+    ws = cache.workspace(OP_DECODE)
+    _check(_lib.hq_decode_attn(ctypes.byref(cache.c), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out),
+                               ctypes.c_float(sm_scale), _ptr(ws), ws.numel(), _stream(stream)), "hq_decode_attn")
+    return out
+
+
+def hq_prefill_workspace_bytes(B, Hq, Hkv, L, D=HQ_HEAD_DIM) -> int:
+    return int(_lib.hq_prefill_workspace_bytes(B, Hq, Hkv, L, D))
+
+
+def hq_prefill_attn(q, k, v, vl_pos, n_vl: int, W: int, sm_scale: float = None, out=None, ws=None, stream=None):
+    """q [B,Hq,L,D], k/v [B,Hkv,L,D] fp16; vl_pos int32 [B,Hkv,stride] (first n_vl ascending)."""
+    B, Hq, L, D = q.shape
+    Hkv = k.shape[1]
+    _need(q, torch.float16, (B, Hq, L, D), "q")
+    _need(k, torch.float16, (B, Hkv, L, D), "k")
+    _need(v, torch.float16, (B, Hkv, L, D), "v")
+    _need(vl_pos, torch.int32, (B, Hkv, vl_pos.shape[2]), "vl_pos")
+    if out is None:
+        out = torch.empty_like(q)
+    n = hq_prefill_workspace_bytes(B, Hq, Hkv, L, D)
+    if ws is None:
+        ws = torch.empty(max(n, 1), dtype=torch.uint8, device=q.device)
+    if sm_scale is None:
+        sm_scale = D ** -0.5
+    _check(_lib.hq_prefill_attn(B, Hq, Hkv, L, D, _ptr(q), _ptr(k), _ptr(v), _ptr(vl_pos), n_vl, vl_pos.shape[2], W,
+                                ctypes.c_float(sm_scale), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
+           "hq_prefill_attn")
+    return out

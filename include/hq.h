@@ -1,0 +1,238 @@
+/*
+ * hq.h — C ABI of libhq.so: hybrid-precision attention on NVIDIA B200 (sm_100a).
+ *
+ * What the library computes is the hot path of HyQuant ("HyQuant:
+ * Hybrid-Precision Quantization for LLM Attention"):
+ *
+ *   - keys are split three ways: vertical-line (VL) positions and a recent
+ *     window stay FP16, every other position is stored 4-bit (K4V4)
+ *     (agihunt.info digest of the paper, method paragraph; repository README,
+ *     Overview);
+ *   - decode attention runs over that hybrid cache with dequantisation fused
+ *     into the online-softmax KV scan, so no FP16 copy of the cache is ever
+ *     materialised (digest, prefill/decode paragraph; README Overview item 3);
+ *   - the VL set is the top-rho (default 5 %) of the non-window prefix by
+ *     accumulated column attention mass, re-identified every 64 tokens from at
+ *     most 64 buffered FP16 queries (digest, method paragraph; README Overview
+ *     item 1 and "Overhead");
+ *   - new tokens are staged and merged into the hybrid layout later (digest,
+ *     prefill/decode paragraph);
+ *   - prefill is one FlashAttention-style causal pass whose quantised tiles run
+ *     on low-precision tensor cores while VL and window tiles stay FP16, under a
+ *     single online softmax (digest, prefill/decode paragraph; README Overview
+ *     item 2).
+ *
+ * K4V4 layout (the pages name the format but print no layout; this library
+ * fixes it): per token and head, D = 128 values in 4 groups of 32;
+ * scale = fp16(fp32(max - min) / 15), zero = min (fp16);
+ * q = clamp(rint_even((x - zero) / scale), 0, 15) with float32 RN arithmetic
+ * (q = 0 when scale == 0); two nibbles per byte, low nibble first; the
+ * dequantised value is zero + q * scale.
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers, 16-byte aligned, owned by the
+ *     caller; the library allocates nothing and keeps no global state.
+ *   - fp16 tensors are passed as uint16_t* (IEEE binary16 bit patterns).
+ *   - Calls are asynchronous on `stream`.  Arguments are validated on the host
+ *     before anything is launched; on a non-HQ_OK status nothing was launched.
+ *   - Conditions that depend on device-resident lengths (a full staging area,
+ *     an exhausted capacity) cannot be seen by the host: the kernels skip their
+ *     work and OR a HQ_DEVERR_* bit into state[HQ_STATE_ERR]; read it after
+ *     synchronising.  No kernel traps or spins without a bound.
+ *   - Batches are uniform-length: every (batch, head) has the same length T.
+ */
+#ifndef HQ_H
+#define HQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define HQ_ABI_VERSION 1
+#define HQ_HEAD_DIM 128       /* D: the only head size built */
+#define HQ_GROUP 32           /* K4V4 group length along D */
+#define HQ_STAGE 64           /* staged tokens before a merge = reselection period */
+#define HQ_QBUF 64            /* buffered queries kept for the column-mass estimate */
+#define HQ_MAX_GQA 8          /* query heads per kv head supported by the decode kernel */
+
+typedef struct CUstream_st* hq_stream_t;  /* same type as cudaStream_t */
+
+#if defined(__GNUC__)
+#define HQ_API __attribute__((visibility("default")))
+#else
+#define HQ_API
+#endif
+
+typedef enum hq_status {
+  HQ_OK = 0,
+  HQ_ERR_INVALID = 1,      /* null/misaligned pointer, bad shape or argument */
+  HQ_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement (e.g. D != 128) */
+  HQ_ERR_WORKSPACE = 3,    /* workspace missing or smaller than hq_*_workspace_bytes() */
+  HQ_ERR_CAPACITY = 4,     /* a host-visible size exceeds the cache's capacity */
+  HQ_ERR_CUDA = 5          /* a CUDA runtime call or launch failed */
+} hq_status;
+
+/* device-side error bits, OR-ed into state[HQ_STATE_ERR] */
+#define HQ_DEVERR_STAGING_FULL 0x1u  /* decode with HQ_STAGE tokens staged: select + merge first */
+#define HQ_DEVERR_CAPACITY 0x2u      /* T would exceed cap */
+#define HQ_DEVERR_VL_CAPACITY 0x4u   /* k = ceil(rho * n) exceeds vl_cap (clamped) */
+#define HQ_DEVERR_TIMEOUT 0x8u       /* a bounded wait gave up (never expected) */
+
+/* words of the device-resident state vector (int32[HQ_STATE_WORDS]) */
+enum {
+  HQ_STATE_T = 0,         /* current length: positions 0 .. T-1 are cached */
+  HQ_STATE_NPACKED = 1,   /* positions 0 .. n_packed-1 have a K4V4 record */
+  HQ_STATE_NVL = 2,       /* rows in the VL store */
+  HQ_STATE_NQ = 3,        /* valid buffered queries (<= HQ_QBUF) */
+  HQ_STATE_KSEL = 4,      /* entries written to vl_sel by the last hq_select_vlines */
+  HQ_STATE_ERR = 5,       /* HQ_DEVERR_* bits */
+  HQ_STATE_WORDS = 8
+};
+
+/*
+ * The hybrid KV cache of one attention layer.  Every array is caller-owned
+ * device memory laid out as stated ([..] = row-major shape, innermost last).
+ * R = W + HQ_STAGE is the FP16 ring length.
+ *
+ *   kq, vq    uint8  [B, Hkv, cap, D/2]   K4V4 codes, dense by position
+ *   ksz, vsz  uint32 [B, Hkv, cap, D/32]  per group: scale fp16 bits | zero fp16 bits << 16
+ *   kf, vf    fp16   [B, Hkv, vl_cap, D]  VL store rows, in vl_pos order
+ *   vl_pos    int32  [B, Hkv, vl_cap]     VL positions, ascending (first n_vl valid)
+ *   vl_mask   uint32 [B, Hkv, cap/32]     bit p set <=> position p is in the VL store
+ *   kr, vr    fp16   [B, Hkv, R, D]       recent window + staging; position p at slot p % R
+ *   qbuf      fp16   [B, Hq, HQ_QBUF, D]  buffered decode queries; position p at slot p % HQ_QBUF
+ *   vl_sel    int32  [B, Hkv, vl_cap]     output of hq_select_vlines, input of hq_pack_merge
+ *   state     int32  [HQ_STATE_WORDS]     device-resident lengths (see HQ_STATE_*)
+ *
+ * Limits checked by hq_cache_validate(): D == 128; Hq % Hkv == 0 and
+ * Hq / Hkv <= HQ_MAX_GQA; W >= 0; 0 <= rho_bp <= 10000; cap a positive
+ * multiple of 128; vl_cap a positive multiple of 16.
+ * Fields W and rho_bp fix the method's window and VL ratio (basis points:
+ * 500 = 5 %).  The fp16 positions in [n_packed, T) live in the ring, VL rows
+ * in kf/vf, every other position < n_packed is read from its K4V4 record.
+ */
+typedef struct hq_cache {
+  int32_t B, Hq, Hkv, D;
+  int32_t W, rho_bp, cap, vl_cap;
+  uint8_t* kq;
+  uint8_t* vq;
+  uint32_t* ksz;
+  uint32_t* vsz;
+  uint16_t* kf;
+  uint16_t* vf;
+  int32_t* vl_pos;
+  uint32_t* vl_mask;
+  uint16_t* kr;
+  uint16_t* vr;
+  uint16_t* qbuf;
+  int32_t* vl_sel;
+  int32_t* state;
+} hq_cache;
+
+/* Operation codes for hq_workspace_bytes. */
+enum { HQ_OP_SELECT = 0, HQ_OP_MERGE = 1, HQ_OP_DECODE = 2 };
+
+HQ_API int32_t hq_abi_version(void);
+HQ_API const char* hq_status_str(hq_status s);
+
+/* Host-side check of a cache descriptor (shapes, limits, 16-byte alignment of
+ * every pointer).  Returns HQ_OK or HQ_ERR_INVALID / HQ_ERR_UNSUPPORTED. */
+HQ_API hq_status hq_cache_validate(const hq_cache* c);
+
+/* Bytes of device workspace an operation needs for this cache; `L` is the
+ * prefix length for an init-mode select/merge (ignored otherwise).
+ * HQ_OP_DECODE and HQ_OP_MERGE workspaces start with completion counters:
+ * zero-fill the workspace once before its first use; the kernels return the
+ * counters to zero at the end of every call.  A workspace must not be shared
+ * by calls that can run at the same time. */
+HQ_API size_t hq_workspace_bytes(const hq_cache* c, int32_t op, int32_t L);
+
+/*
+ * Reset the cache to empty: state words to 0 and the VL bitmap cleared.
+ */
+HQ_API hq_status hq_cache_reset(const hq_cache* c, hq_stream_t stream);
+
+/*
+ * Vertical-line selection (digest, method paragraph; README Overview item 1).
+ * For every (b, kv head): column mass
+ *     score_j = sum over the group's query heads h and buffered queries i of
+ *               softmax_{j' <= p_i}(q_{h,i} . k_{j'} * sm_scale)[j],
+ * for j in the non-window prefix [0, n), n = T - W, sm_scale = 1/sqrt(D);
+ * then the k = ceil(n * rho_bp / 10000) largest scores (ties -> lower
+ * position) are written to c->vl_sel in ascending position order and k to
+ * state[HQ_STATE_KSEL].
+ *
+ * Init mode (k_dense != NULL): keys are the dense FP16 prefix
+ *   k_dense [B, Hkv, L, D], T = L; queries q_ext [B, Hq, nq, D] sit at
+ *   positions L-nq .. L-1 (1 <= nq <= HQ_QBUF, nq <= L).  The cache's state
+ *   is not read.
+ * Decode mode (k_dense == NULL, q_ext == NULL): keys are the cache in its
+ *   current representation (VL rows FP16, other packed positions
+ *   dequantised, ring FP16), T and the buffered queries come from state/qbuf.
+ * scores_out (optional, may be NULL): float [B, Hkv, cap] receives the scores
+ *   (entries >= n are unspecified).
+ * Errors: HQ_ERR_INVALID for bad pointers/shapes; k > vl_cap is clamped and
+ *   flagged with HQ_DEVERR_VL_CAPACITY.
+ */
+HQ_API hq_status hq_select_vlines(const hq_cache* c, const uint16_t* k_dense, int32_t L,
+                           const uint16_t* q_ext, int32_t nq, float* scores_out,
+                           void* ws, size_t ws_bytes, hq_stream_t stream);
+
+/*
+ * Staging -> hybrid merge (digest, prefill/decode paragraph).
+ * Init mode (k_dense, v_dense != NULL, both [B, Hkv, L, D] FP16): install a
+ *   prefix of L tokens: positions [0, L-W) get their K4V4 records, the last
+ *   min(W, L) positions go to the ring, the VL store is filled from c->vl_sel
+ *   (state[HQ_STATE_KSEL] entries, FP16 rows taken from the dense prefix);
+ *   state becomes T = L, n_packed = max(L-W, 0), n_q = 0.  Requires L <= cap.
+ * Merge mode (both NULL): positions [n_packed, T-W) leave the window and get
+ *   their K4V4 records; the VL store is rebuilt from c->vl_sel: a row keeps the
+ *   position's current FP16 value when it has one (old VL row or ring),
+ *   otherwise it is the dequantised record rounded once to FP16; n_packed
+ *   becomes max(n_packed, T-W).  Records are never rewritten.
+ */
+HQ_API hq_status hq_pack_merge(const hq_cache* c, const uint16_t* k_dense, const uint16_t* v_dense,
+                        int32_t L, void* ws, size_t ws_bytes, hq_stream_t stream);
+
+/*
+ * One decode step (digest, prefill/decode paragraph; README Overview item 3):
+ * append k_new, v_new [B, Hkv, D] at position T (ring) and q [B, Hq, D] to
+ * the query buffer, then
+ *     out[b, h] = softmax(q[b,h] . K^T * sm_scale) V
+ * over all T+1 positions, each key/value in its stored representation
+ * (dequantisation fused into the scan; split-K over the sequence with a
+ * log-sum-exp merge).  out: fp16 [B, Hq, D].  Increments T.
+ * If HQ_STAGE tokens are already staged (T - n_packed == W + HQ_STAGE) or
+ * T == cap, nothing is written and HQ_DEVERR_STAGING_FULL / _CAPACITY is set.
+ */
+HQ_API hq_status hq_decode_attn(const hq_cache* c, const uint16_t* q, const uint16_t* k_new,
+                         const uint16_t* v_new, uint16_t* out, float sm_scale,
+                         void* ws, size_t ws_bytes, hq_stream_t stream);
+
+/*
+ * Hybrid causal prefill (digest, prefill/decode paragraph; README Overview
+ * item 2, modes "vquant_vert" / "hybrid_full"): for query i and key j <= i,
+ *   j is a window key if i - W < j <= i, else a VL key if j is in vl_pos[b, kvh],
+ *   else a quantised key;
+ * window and VL keys use FP16 Q, K, V; quantised keys use FP8 e4m3 Q, K, V with
+ * one float32 scale per (b, head, 128 positions) (scale = amax / 448, values
+ * stored as e4m3_RN_sat(x / scale)); one softmax covers all three classes.
+ *   q [B, Hq, L, D], k, v [B, Hkv, L, D], out [B, Hq, L, D]: fp16
+ *   vl_pos int32 [B, Hkv, vl_stride], first n_vl entries ascending, < L
+ * Workspace: hq_prefill_workspace_bytes().
+ */
+HQ_API size_t hq_prefill_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t L, int32_t D);
+HQ_API hq_status hq_prefill_attn(int32_t B, int32_t Hq, int32_t Hkv, int32_t L, int32_t D,
+                          const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                          const int32_t* vl_pos, int32_t n_vl, int32_t vl_stride, int32_t W,
+                          float sm_scale, uint16_t* out, void* ws, size_t ws_bytes,
+                          hq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HQ_H */

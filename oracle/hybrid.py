@@ -92,11 +92,6 @@ class HybridCacheRef:
         """Install a prefix of L tokens.  Selects VL lines on the tail queries
         (keys all FP16), packs [0, L - W) and keeps [L - W, L) in FP16."""
         B, Hkv, L, D = K16.shape
-        assert L <= self.cap
-        self.k16[:, :, :L] = K16
-        self.v16[:, :, :L] = V16
-        self.T = L
-        self.n_packed = 0
         n = max(L - self.W, 0)
         nq = q_tail.shape[2]
         qpos = np.tile(np.arange(L - nq, L), self.G)
@@ -106,32 +101,47 @@ class HybridCacheRef:
             for h in range(Hkv):
                 qs = q_tail[b, h * self.G:(h + 1) * self.G].reshape(-1, D).astype(np.float64)
                 new_vl[b][h], scores[b][h] = select.select_vlines(K16[b, h].astype(np.float64), qs, qpos, n, self.rho_bp, self.sm_scale)
-        self.merge(new_vl)
-        self.qbuf = []
+        self.install_prefix(K16, V16, new_vl)
         return new_vl, scores
+
+    def install_prefix(self, K16, V16, vl_sets):
+        """Install a prefix with given VL sets (the selection step done elsewhere)."""
+        B, Hkv, L, D = K16.shape
+        assert L <= self.cap
+        self.k16[:, :, :L] = K16
+        self.v16[:, :, :L] = V16
+        self.T = L
+        self.n_packed = 0
+        self.vl = [[np.zeros(0, np.int64) for _ in range(Hkv)] for _ in range(B)]
+        self.merge(vl_sets)
+        self.qbuf = []
 
     # ------------------------------------------------------------------ decode
     def staged(self) -> int:
         return self.T - self.n_packed - self.W if self.T > 0 else 0
 
-    def decode(self, q, k_new, v_new):
-        """One decode step: append (k_new, v_new) at position T and attend.
-
-        q [B, Hq, D], k_new/v_new [B, Hkv, D] float16.  Returns float64 [B, Hq, D].
-        """
+    def append(self, q, k_new, v_new):
+        """The state change of a decode step (new token staged, query buffered)."""
         if self.T - self.n_packed >= self.W + STAGE:
             raise RuntimeError("staging full: reselect and merge first")
         t = self.T
         self.k16[:, :, t] = k_new
         self.v16[:, :, t] = v_new
         self.T = t + 1
+        self.qbuf.append((t, np.array(q, np.float16)))
+        self.qbuf = self.qbuf[-QBUF:]
+
+    def decode(self, q, k_new, v_new):
+        """One decode step: append (k_new, v_new) at position T and attend.
+
+        q [B, Hq, D], k_new/v_new [B, Hkv, D] float16.  Returns float64 [B, Hq, D].
+        """
+        self.append(q, k_new, v_new)
         out = np.empty((self.B, self.Hq, self.D))
         for b in range(self.B):
             for h in range(self.Hkv):
                 K, V = self.rep(b, h)
                 out[b, h * self.G:(h + 1) * self.G] = attend(q[b, h * self.G:(h + 1) * self.G], K, V, self.sm_scale)
-        self.qbuf.append((t, np.array(q, np.float16)))
-        self.qbuf = self.qbuf[-QBUF:]
         return out
 
     # ------------------------------------------------------------------ reselect + merge

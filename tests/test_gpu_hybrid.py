@@ -1,0 +1,103 @@
+"""GPU parity: K4V4 pack, VL selection, staging merge and decode attention
+against the CPU oracle, through the C ABI (libhq.so)."""
+import numpy as np
+import pytest
+import torch
+
+from hybrid_precision_attention_b200 import synth
+from tests._gpu import Pair, check_decode, dev, hq
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,L,W,rho", [
+    (1, 32, 8, 1024, 128, 500),     # the 1K decode layer (Llama-3.1-8B attention shape)
+    (2, 8, 2, 1000, 100, 500),      # ragged: L, L - W not multiples of any tile
+    (1, 8, 8, 333, 64, 700),        # GQA 1
+    (1, 16, 2, 700, 128, 500),      # GQA 8
+    (1, 4, 2, 200, 0, 0),           # strict 4-bit: no window, no lines
+    (1, 4, 1, 150, 200, 500),       # window longer than the prefix: nothing packed
+    (1, 4, 1, 70, 16, 10000),       # every non-window position a line
+])
+def test_prefix_init_and_decode(B, Hq, Hkv, L, W, rho):
+    p = Pair(B, Hq, Hkv, L, W, rho, cap=L + 200, seed=L)
+    p.init()
+    q, k, v = synth.decode_tokens(L, B, Hq, Hkv, 5)
+    for t in range(5):
+        out, ref = p.decode(q[t], k[t], v[t])
+        check_decode(out, ref, f"step {t}")
+    assert p.g.state()["T"] == L + 5 and p.g.state()["n_q"] == 5
+
+
+def test_decode_loop_with_reselection():
+    """64 decode steps, staging full, reselect + merge, 64 more, reselect + merge."""
+    B, Hq, Hkv, L, W = 1, 32, 8, 1024, 128
+    p = Pair(B, Hq, Hkv, L, W, 500, cap=L + 256, seed=5)
+    p.init()
+    q, k, v = synth.decode_tokens(5, B, Hq, Hkv, 140)
+    t = 0
+    for rnd in range(2):
+        for _ in range(64):
+            out, ref = p.decode(q[t], k[t], v[t])
+            check_decode(out, ref, f"step {t}")
+            t += 1
+        # staging full: the kernel refuses the step and flags it
+        H = hq()
+        sentinel = torch.full((B, Hq, 128), 7.0, dtype=torch.float16, device="cuda")
+        H.hq_decode_attn(p.g, dev(q[t]), dev(k[t]), dev(v[t]), out=sentinel)
+        torch.cuda.synchronize()
+        st = p.g.state()
+        assert st["err"] & H.DEVERR_STAGING_FULL and st["T"] == L + t
+        assert torch.all(sentinel == 7.0)
+        p.g.state_t[H.STATE_ERR] = 0
+        p.reselect_merge()
+        assert p.g.state()["n_packed"] == L + t - W
+    for _ in range(3):
+        out, ref = p.decode(q[t], k[t], v[t])
+        check_decode(out, ref, f"step {t}")
+        t += 1
+
+
+def test_reselect_before_staging_is_full():
+    """A merge with fewer than 64 staged tokens packs only what left the window."""
+    p = Pair(1, 8, 2, 500, 64, 500, cap=800, seed=9)
+    p.init()
+    q, k, v = synth.decode_tokens(9, 1, 8, 2, 20)
+    for t in range(10):
+        out, ref = p.decode(q[t], k[t], v[t])
+        check_decode(out, ref)
+    p.reselect_merge()
+    assert p.g.state()["n_packed"] == 510 - 64
+    for t in range(10, 20):
+        out, ref = p.decode(q[t], k[t], v[t])
+        check_decode(out, ref)
+
+
+def test_capacity_flag():
+    H = hq()
+    p = Pair(1, 4, 1, 120, 8, 500, cap=128, seed=3)
+    p.init()
+    q, k, v = synth.decode_tokens(3, 1, 4, 1, 10)
+    for t in range(8):
+        out, ref = p.decode(q[t], k[t], v[t])
+        check_decode(out, ref)
+    H.hq_decode_attn(p.g, dev(q[8]), dev(k[8]), dev(v[8]))
+    torch.cuda.synchronize()
+    assert p.g.state()["err"] & H.DEVERR_CAPACITY and p.g.state()["T"] == 128
+
+
+@pytest.mark.slow
+def test_full_size_32k_layer():
+    """The 32K decode layer (B=1, Hq=32, Hkv=8): init, one step, 64-step period, reselect + merge, one step."""
+    B, Hq, Hkv, L, W = 1, 32, 8, 32768, 128
+    p = Pair(B, Hq, Hkv, L, W, 500, cap=L + 128, seed=0)
+    p.init()
+    q, k, v = synth.decode_tokens(0, B, Hq, Hkv, 65)
+    out, ref = p.decode(q[0], k[0], v[0])
+    check_decode(out, ref, "first step")
+    for t in range(1, 64):
+        hq().hq_decode_attn(p.g, dev(q[t]), dev(k[t]), dev(v[t]))
+        p.r.append(q[t], k[t], v[t])
+    p.reselect_merge()
+    out, ref = p.decode(q[64], k[64], v[64])
+    check_decode(out, ref, "after merge")
