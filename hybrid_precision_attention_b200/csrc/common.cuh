@@ -16,6 +16,12 @@ namespace hq {
 constexpr int D = HQ_HEAD_DIM;
 constexpr float LOG2E = 1.4426950408889634f;
 
+__host__ __device__ __forceinline__ int ring_len(int W) { return HQ_RING_LEN(W); }
+
+// release / acquire fences at GPU scope (cheaper than the sequentially
+// consistent fence behind __threadfence)
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -7,13 +7,17 @@
 // materialised.  The pages' kernel is Triton for SM80+; this is a B200 design.
 //
 // Design (bandwidth-bound: ~160 B of K4V4 per token and kv head):
-//   * grid = (splits S, Hkv, B); every CTA owns one GQA group (all G <= 8 query
-//     heads of a kv head share one pass over the bytes) and a contiguous range
-//     of the head's tile list: packed tiles (64 positions: 4 KB K codes, 4 KB V
-//     codes, 1 KB + 1 KB scale/zero, 16 B of the VL bitmap), then VL tiles and
-//     recent tiles (16 FP16 rows each);
-//   * one producer lane streams tiles into an 8-stage shared-memory ring with
-//     1-D bulk async copies (cp.async.bulk, mbarrier completion, no multicast);
+//   * grid = (splits S, Hkv, B), one wave (S * Hkv * B <= 3 CTAs per SM); every
+//     CTA owns one GQA group (all G <= 8 query heads of a kv head share one
+//     pass over the bytes) and a contiguous range of the head's tile list:
+//     packed tiles (64 positions: 4 KB K codes, 4 KB V codes, 1 KB + 1 KB
+//     scale/zero, 16 B of the VL bitmap), VL tiles (16 FP16 rows of the VL
+//     store), ring tiles (16 slots of the FP16 ring, which is a multiple of 16
+//     long, so a tile is one contiguous copy) and a last tile holding the new
+//     token read straight from its input pointer;
+//   * a producer warp streams tiles into a 6-stage shared-memory ring with
+//     large 1-D bulk async copies (cp.async.bulk, mbarrier completion, no
+//     multicast): 5 copies per packed tile, 2 per FP16 tile;
 //   * 4 consumer warps take whole tiles round-robin.  Nibbles become fp16 in
 //     registers (exponent-bias trick + one fma with the group's scale/zero), and
 //     both products run on tensor cores with mma.m16n8k16 (f32 accumulate):
@@ -21,13 +25,14 @@
 //       O^T[dims x 8 queries] += V^T (16 dims x 16 keys) . P^T
 //     P^T comes from the S^T accumulators by an 8x8 movmatrix transpose.  Dims
 //     and keys are permuted inside each MMA so that every thread dequantises one
-//     whole group from contiguous nibbles and the shared-memory reads are free
-//     of bank conflicts;
+//     whole group from contiguous nibbles and the packed-tile shared-memory
+//     reads are free of bank conflicts;
 //   * per-warp online softmax in the exp2 domain, a CTA merge in shared memory,
 //     then split partials (m, l, O) go to the workspace and the last CTA of each
 //     (b, kv head) merges them with a log-sum-exp (atomic ticket, no waiting);
-//   * the new token is attended from its input pointer and written into the
-//     ring; the last CTA of the grid advances T.
+//   * the last CTA of each (b, kv head) also appends that head's new token to
+//     the ring and its queries to the query buffer (every split of the head is
+//     done reading by then); the last CTA of the grid advances T.
 #include "common.cuh"
 
 namespace hq {
@@ -35,20 +40,20 @@ namespace {
 
 constexpr int NCONS = 4;                       // consumer warps
 constexpr int NTHREADS = (NCONS + 1) * 32;     // + producer warp
-constexpr int NSTAGES = 8;
+constexpr int NSTAGES = 6;
 constexpr int PK = 64;                         // positions per packed tile
 constexpr int FT = 16;                         // rows per FP16 tile
-constexpr int FSTRIDE = 272;                   // bytes per FP16 row in shared memory (256 + 16)
+constexpr int FSTRIDE = 256;                   // bytes per FP16 row in shared memory (one contiguous copy)
 constexpr int OFF_VC = 4096, OFF_KS = 8192, OFF_VS = 9216, OFF_MASK = 10240;
 constexpr int OFF_FV = FT * FSTRIDE;           // V rows of an FP16 tile
-constexpr int STAGE_BYTES = 10368;             // max(10256, 2 * 16 * 272 = 8704), 128-aligned
+constexpr int STAGE_BYTES = 10368;             // max(10256, 2 * 16 * 256 = 8192), 128-aligned
 constexpr int PART_FLOATS = 16 + 8 * D;        // m[8], l[8], O[8][128]
 constexpr uint32_t PK_TX = 4096 * 2 + 1024 * 2 + 16;
 
 // key slot -> shared-memory row inside a 16-key block.  Packed tiles (64-byte
-// rows): {0,5,1,4,2,7,3,6, 8,13,9,12,10,15,11,14}; FP16 tiles (272-byte rows):
-// {0,2,1,3,4,6,5,7, 8,10,9,11,12,14,13,15}.  Both keep the QK rows of a
-// quarter-warp and the PV rows of a warp on distinct banks.
+// rows): {0,5,1,4,2,7,3,6, 8,13,9,12,10,15,11,14}; FP16 tiles (256-byte rows):
+// {0,2,1,3,4,6,5,7, 8,10,9,11,12,14,13,15}.  The packed map keeps the QK rows
+// of a quarter-warp and the PV rows of a warp on distinct banks.
 __device__ __forceinline__ int pi_pk(int s) {
   const int x = s & 7;
   return (s & 8) + ((x & 1) ? 4 + ((x >> 1) ^ 1) : (x >> 1));
@@ -59,19 +64,43 @@ __device__ __forceinline__ int pi_fp(int s) {
 }
 
 struct Geo {
-  int n_packed, n_vl, T, NP, NV, NR, NT;
+  int n_packed, n_vl, T, R, NP, NV, NR, NT;
 };
 
-__device__ __forceinline__ Geo geo_of(int n_packed, int n_vl, int T) {
+// tiles of one (b, kv head): [0, NP) packed, [NP, NP+NV) VL, [NP+NV, NT-1) ring
+// (R/16 slot tiles), NT-1 the new token
+__device__ __forceinline__ Geo geo_of(int n_packed, int n_vl, int T, int R) {
   Geo g;
   g.n_packed = n_packed;
   g.n_vl = n_vl;
   g.T = T;
+  g.R = R;
   g.NP = (n_packed + PK - 1) / PK;
   g.NV = (n_vl + FT - 1) / FT;
-  g.NR = (T + 1 - n_packed + FT - 1) / FT;  // recent positions [n_packed, T) incl. the new token
+  g.NR = R / FT + 1;
   g.NT = g.NP + g.NV + g.NR;
   return g;
+}
+
+// 16-bit mask of the valid rows of FP16 tile `tile`
+__device__ __forceinline__ uint32_t fp16_valid(const Geo& g, int tile) {
+  if (tile < g.NP + g.NV) {
+    const int first = (tile - g.NP) * FT;
+    const int n = min(FT, g.n_vl - first);
+    return n >= FT ? 0xFFFFu : ((1u << n) - 1u);
+  }
+  const int j = tile - g.NP - g.NV;
+  if (j == g.NR - 1) return 1u;  // the new token
+  // ring slot s holds position p = n_packed + ((s - n_packed) mod R); valid iff p < T
+  const int base = g.n_packed % g.R;
+  uint32_t m = 0;
+#pragma unroll 4
+  for (int r = 0; r < FT; ++r) {
+    int off = FT * j + r - base;
+    off += off < 0 ? g.R : 0;
+    m |= (g.n_packed + off < g.T ? 1u : 0u) << r;
+  }
+  return m;
 }
 
 struct WarpState {
@@ -131,103 +160,104 @@ __device__ __forceinline__ void packed_tile(WarpState& ws, const uint8_t* st, co
   const int base = tile * PK;
   const bool full = base + PK <= n_packed;
 
-  // ---- S^T = K^ . Q^T for 4 blocks of 16 keys
-  float s[4][4];
+  // two halves of 32 keys, each: S^T = K^ . Q^T (2 blocks of 16 keys),
+  // online-softmax step, O^T += V^T . P^T
+#pragma unroll 1
+  for (int hf = 0; hf < 2; ++hf) {
+    float s[2][4];
 #pragma unroll
-  for (int mt = 0; mt < 4; ++mt) {
-    const int ra = 16 * mt + pi_pk(g), rb = 16 * mt + pi_pk(g + 8);
-    const uint4 ka = *reinterpret_cast<const uint4*>(kc + ra * 64 + 16 * t);
-    const uint4 kb = *reinterpret_cast<const uint4*>(kc + rb * 64 + 16 * t);
-    const uint32_t za = ks[ra * 4 + t], zb = ks[rb * 4 + t];
-    const uint32_t sa2 = prmt(za, za, 0x1010), za2 = prmt(za, za, 0x3232);
-    const uint32_t sb2 = prmt(zb, zb, 0x1010), zb2 = prmt(zb, zb, 0x3232);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w};
-    const uint32_t wb[4] = {kb.x, kb.y, kb.z, kb.w};
+    for (int j = 0; j < 2; ++j) {
+      const int mt = 2 * hf + j;
+      const int ra = 16 * mt + pi_pk(g), rb = 16 * mt + pi_pk(g + 8);
+      const uint4 ka = *reinterpret_cast<const uint4*>(kc + ra * 64 + 16 * t);
+      const uint4 kb = *reinterpret_cast<const uint4*>(kc + rb * 64 + 16 * t);
+      const uint32_t za = ks[ra * 4 + t], zb = ks[rb * 4 + t];
+      const uint32_t sa2 = prmt(za, za, 0x1010), za2 = prmt(za, za, 0x3232);
+      const uint32_t sb2 = prmt(zb, zb, 0x1010), zb2 = prmt(zb, zb, 0x3232);
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w};
+      const uint32_t wb[4] = {kb.x, kb.y, kb.z, kb.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < 4; ++i) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t xa = wa[i] >> (8 * h), xb = wb[i] >> (8 * h);
-        const uint32_t a0 = hfma2_u(nib_lo(xa), sa2, za2);
-        const uint32_t a2 = hfma2_u(nib_hi(xa), sa2, za2);
-        const uint32_t a1 = hfma2_u(nib_lo(xb), sb2, zb2);
-        const uint32_t a3 = hfma2_u(nib_hi(xb), sb2, zb2);
-        mma16816(acc, a0, a1, a2, a3, qf[2 * i + h][0], qf[2 * i + h][1]);
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t xa = wa[i] >> (8 * h), xb = wb[i] >> (8 * h);
+          const uint32_t a0 = hfma2_u(nib_lo(xa), sa2, za2);
+          const uint32_t a2 = hfma2_u(nib_hi(xa), sa2, za2);
+          const uint32_t a1 = hfma2_u(nib_lo(xb), sb2, zb2);
+          const uint32_t a3 = hfma2_u(nib_hi(xb), sb2, zb2);
+          mma16816(acc, a0, a1, a2, a3, qf[2 * i + h][0], qf[2 * i + h][1]);
+        }
       }
+      // mask: beyond n_packed, or a vertical line (its FP16 row is read instead)
+      const bool va = (base + ra < n_packed) && !((mk[ra >> 5] >> (ra & 31)) & 1u);
+      const bool vb = (base + rb < n_packed) && !((mk[rb >> 5] >> (rb & 31)) & 1u);
+      s[j][0] = va ? acc[0] * qscale : -INFINITY;
+      s[j][1] = va ? acc[1] * qscale : -INFINITY;
+      s[j][2] = vb ? acc[2] * qscale : -INFINITY;
+      s[j][3] = vb ? acc[3] * qscale : -INFINITY;
     }
-    // mask: beyond n_packed, or a vertical line (its FP16 row is read instead)
-    const int la = 16 * mt + pi_pk(g), lb = 16 * mt + pi_pk(g + 8);
-    const bool va = (base + la < n_packed) && !((mk[la >> 5] >> (la & 31)) & 1u);
-    const bool vb = (base + lb < n_packed) && !((mk[lb >> 5] >> (lb & 31)) & 1u);
-    s[mt][0] = va ? acc[0] * qscale : -INFINITY;
-    s[mt][1] = va ? acc[1] * qscale : -INFINITY;
-    s[mt][2] = vb ? acc[2] * qscale : -INFINITY;
-    s[mt][3] = vb ? acc[3] * qscale : -INFINITY;
-  }
-  uint32_t pb[4][2];
-  softmax_update<4>(ws, s, pb);
+    uint32_t pb[2][2];
+    softmax_update<2>(ws, s, pb);
 
-  // ---- O^T += V^T . P^T, one k-step per 16-key block
 #pragma unroll
-  for (int mt = 0; mt < 4; ++mt) {
-    const int r0 = 16 * mt + pi_pk(2 * t), r1 = 16 * mt + pi_pk(2 * t + 1);
-    const int r2 = 16 * mt + pi_pk(2 * t + 8), r3 = 16 * mt + pi_pk(2 * t + 9);
-    // two 32-bit loads per row, issued in a per-thread order that keeps the
-    // warp's accesses on distinct banks
-    const int e = t >> 1;
-    const uint32_t* v0 = reinterpret_cast<const uint32_t*>(vc + r0 * 64) + 2 * g;
-    const uint32_t* v1 = reinterpret_cast<const uint32_t*>(vc + r1 * 64) + 2 * g;
-    const uint32_t* v2 = reinterpret_cast<const uint32_t*>(vc + r2 * 64) + 2 * g;
-    const uint32_t* v3 = reinterpret_cast<const uint32_t*>(vc + r3 * 64) + 2 * g;
-    uint32_t x0a = v0[e], x0b = v0[e ^ 1], x1a = v1[e], x1b = v1[e ^ 1];
-    uint32_t x2a = v2[e], x2b = v2[e ^ 1], x3a = v3[e], x3b = v3[e ^ 1];
-    // un-rotate: w?0 = word 2g, w?1 = word 2g+1
-    const uint32_t w00 = e ? x0b : x0a, w01 = e ? x0a : x0b;
-    const uint32_t w10 = e ? x1b : x1a, w11 = e ? x1a : x1b;
-    const uint32_t w20 = e ? x2b : x2a, w21 = e ? x2a : x2b;
-    const uint32_t w30 = e ? x3b : x3a, w31 = e ? x3a : x3b;
-    const int grp = g >> 1;
-    const uint32_t z0 = vs[r0 * 4 + grp], z1 = vs[r1 * 4 + grp], z2 = vs[r2 * 4 + grp], z3 = vs[r3 * 4 + grp];
-    const uint32_t s01 = prmt(z0, z1, 0x5410), o01 = prmt(z0, z1, 0x7632);
-    const uint32_t s23 = prmt(z2, z3, 0x5410), o23 = prmt(z2, z3, 0x7632);
-    // pair nibbles of the two keys: x?[k] holds dims 16g + 4k .. 16g + 4k + 3 of both keys
-    uint32_t xab[4], xcd[4];
-    xab[0] = prmt(w00, w10, 0x5410);
-    xab[1] = prmt(w00, w10, 0x7632);
-    xab[2] = prmt(w01, w11, 0x5410);
-    xab[3] = prmt(w01, w11, 0x7632);
-    xcd[0] = prmt(w20, w30, 0x5410);
-    xcd[1] = prmt(w20, w30, 0x7632);
-    xcd[2] = prmt(w21, w31, 0x5410);
-    xcd[3] = prmt(w21, w31, 0x7632);
-    bool zero_ab = false, zero_cd = false;
-    uint32_t keep_ab = 0xFFFFFFFFu, keep_cd = 0xFFFFFFFFu;
-    if (!full) {  // rows past n_packed may hold stale records: zero them out of P.V
-      const bool a = base + r0 < n_packed, b = base + r1 < n_packed;
-      const bool cc = base + r2 < n_packed, dd = base + r3 < n_packed;
-      keep_ab = (a ? 0x0000FFFFu : 0u) | (b ? 0xFFFF0000u : 0u);
-      keep_cd = (cc ? 0x0000FFFFu : 0u) | (dd ? 0xFFFF0000u : 0u);
-      zero_ab = !(a && b);
-      zero_cd = !(cc && dd);
-    }
+    for (int j = 0; j < 2; ++j) {
+      const int mt = 2 * hf + j;
+      const int r0 = 16 * mt + pi_pk(2 * t), r1 = 16 * mt + pi_pk(2 * t + 1);
+      const int r2 = 16 * mt + pi_pk(2 * t + 8), r3 = 16 * mt + pi_pk(2 * t + 9);
+      // two 32-bit loads per row, issued in a per-thread order that keeps the
+      // warp's accesses on distinct banks
+      const int e = t >> 1;
+      const uint32_t* v0 = reinterpret_cast<const uint32_t*>(vc + r0 * 64) + 2 * g;
+      const uint32_t* v1 = reinterpret_cast<const uint32_t*>(vc + r1 * 64) + 2 * g;
+      const uint32_t* v2 = reinterpret_cast<const uint32_t*>(vc + r2 * 64) + 2 * g;
+      const uint32_t* v3 = reinterpret_cast<const uint32_t*>(vc + r3 * 64) + 2 * g;
+      const uint32_t x0a = v0[e], x0b = v0[e ^ 1], x1a = v1[e], x1b = v1[e ^ 1];
+      const uint32_t x2a = v2[e], x2b = v2[e ^ 1], x3a = v3[e], x3b = v3[e ^ 1];
+      // un-rotate: w?0 = word 2g, w?1 = word 2g+1
+      const uint32_t w00 = e ? x0b : x0a, w01 = e ? x0a : x0b;
+      const uint32_t w10 = e ? x1b : x1a, w11 = e ? x1a : x1b;
+      const uint32_t w20 = e ? x2b : x2a, w21 = e ? x2a : x2b;
+      const uint32_t w30 = e ? x3b : x3a, w31 = e ? x3a : x3b;
+      const int grp = g >> 1;
+      const uint32_t z0 = vs[r0 * 4 + grp], z1 = vs[r1 * 4 + grp], z2 = vs[r2 * 4 + grp], z3 = vs[r3 * 4 + grp];
+      const uint32_t s01 = prmt(z0, z1, 0x5410), o01 = prmt(z0, z1, 0x7632);
+      const uint32_t s23 = prmt(z2, z3, 0x5410), o23 = prmt(z2, z3, 0x7632);
+      // pair nibbles of the two keys: x?[k] holds dims 16g + 4k .. 16g + 4k + 3 of both keys
+      uint32_t xab[4], xcd[4];
+      xab[0] = prmt(w00, w10, 0x5410);
+      xab[1] = prmt(w00, w10, 0x7632);
+      xab[2] = prmt(w01, w11, 0x5410);
+      xab[3] = prmt(w01, w11, 0x7632);
+      xcd[0] = prmt(w20, w30, 0x5410);
+      xcd[1] = prmt(w20, w30, 0x7632);
+      xcd[2] = prmt(w21, w31, 0x5410);
+      xcd[3] = prmt(w21, w31, 0x7632);
+      uint32_t keep_ab = 0xFFFFFFFFu, keep_cd = 0xFFFFFFFFu;
+      if (!full) {  // rows past n_packed may hold stale records: zero them out of P.V
+        keep_ab = (base + r0 < n_packed ? 0x0000FFFFu : 0u) | (base + r1 < n_packed ? 0xFFFF0000u : 0u);
+        keep_cd = (base + r2 < n_packed ? 0x0000FFFFu : 0u) | (base + r3 < n_packed ? 0xFFFF0000u : 0u);
+      }
 #pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      const uint32_t yab = xab[m >> 1] >> (8 * (m & 1));
-      const uint32_t ycd = xcd[m >> 1] >> (8 * (m & 1));
-      uint32_t a0 = hfma2_u(nib_lo(yab), s01, o01);
-      uint32_t a1 = hfma2_u(nib_hi(yab), s01, o01);
-      uint32_t a2 = hfma2_u(nib_lo(ycd), s23, o23);
-      uint32_t a3 = hfma2_u(nib_hi(ycd), s23, o23);
-      if (zero_ab) { a0 &= keep_ab; a1 &= keep_ab; }
-      if (zero_cd) { a2 &= keep_cd; a3 &= keep_cd; }
-      mma16816(ws.o[m], a0, a1, a2, a3, pb[mt][0], pb[mt][1]);
+      for (int m = 0; m < 8; ++m) {
+        const uint32_t yab = xab[m >> 1] >> (8 * (m & 1));
+        const uint32_t ycd = xcd[m >> 1] >> (8 * (m & 1));
+        uint32_t a0 = hfma2_u(nib_lo(yab), s01, o01);
+        uint32_t a1 = hfma2_u(nib_hi(yab), s01, o01);
+        uint32_t a2 = hfma2_u(nib_lo(ycd), s23, o23);
+        uint32_t a3 = hfma2_u(nib_hi(ycd), s23, o23);
+        if (!full) {
+          a0 &= keep_ab; a1 &= keep_ab;
+          a2 &= keep_cd; a3 &= keep_cd;
+        }
+        mma16816(ws.o[m], a0, a1, a2, a3, pb[j][0], pb[j][1]);
+      }
     }
   }
 }
 
-// one FP16 tile (16 rows at FSTRIDE) by one warp; `nvalid` leading rows are real
-__device__ __forceinline__ void fp16_tile(WarpState& ws, const uint8_t* st, const uint32_t (&qf)[8][2], int nvalid,
+// one FP16 tile (16 rows at FSTRIDE) by one warp; bit r of `valid` marks row r as real
+__device__ __forceinline__ void fp16_tile(WarpState& ws, const uint8_t* st, const uint32_t (&qf)[8][2], uint32_t valid,
                                           float qscale, int g, int t) {
   const uint8_t* kb = st;
   const uint8_t* vb = st + OFF_FV;
@@ -244,7 +274,7 @@ __device__ __forceinline__ void fp16_tile(WarpState& ws, const uint8_t* st, cons
              qf[2 * i + 1][0], qf[2 * i + 1][1]);
   }
   float s[1][4];
-  const bool va = ra < nvalid, vbv = rb < nvalid;
+  const bool va = (valid >> ra) & 1u, vbv = (valid >> rb) & 1u;
   s[0][0] = va ? acc[0] * qscale : -INFINITY;
   s[0][1] = va ? acc[1] * qscale : -INFINITY;
   s[0][2] = vbv ? acc[2] * qscale : -INFINITY;
@@ -265,9 +295,9 @@ __device__ __forceinline__ void fp16_tile(WarpState& ws, const uint8_t* st, cons
   uint32_t w1[8] = {a1l.x, a1l.y, a1l.z, a1l.w, a1h.x, a1h.y, a1h.z, a1h.w};
   uint32_t w2[8] = {a2l.x, a2l.y, a2l.z, a2l.w, a2h.x, a2h.y, a2h.z, a2h.w};
   uint32_t w3[8] = {a3l.x, a3l.y, a3l.z, a3l.w, a3h.x, a3h.y, a3h.z, a3h.w};
-  if (nvalid < FT) {  // rows not copied this time hold stale bytes: keep them out of P.V
-    const uint32_t k0 = r0 < nvalid ? 0xFFFFFFFFu : 0u, k1 = r1 < nvalid ? 0xFFFFFFFFu : 0u;
-    const uint32_t k2 = r2 < nvalid ? 0xFFFFFFFFu : 0u, k3 = r3 < nvalid ? 0xFFFFFFFFu : 0u;
+  if (valid != 0xFFFFu) {  // invalid rows may hold stale bytes: keep them out of P.V
+    const uint32_t k0 = ((valid >> r0) & 1u) ? 0xFFFFFFFFu : 0u, k1 = ((valid >> r1) & 1u) ? 0xFFFFFFFFu : 0u;
+    const uint32_t k2 = ((valid >> r2) & 1u) ? 0xFFFFFFFFu : 0u, k3 = ((valid >> r3) & 1u) ? 0xFFFFFFFFu : 0u;
 #pragma unroll
     for (int m = 0; m < 8; ++m) {
       w0[m] &= k0; w1[m] &= k1; w2[m] &= k2; w3[m] &= k3;
@@ -280,7 +310,7 @@ __device__ __forceinline__ void fp16_tile(WarpState& ws, const uint8_t* st, cons
   }
 }
 
-__global__ void __launch_bounds__(NTHREADS, 2)
+__global__ void __launch_bounds__(NTHREADS, 3)
 decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* __restrict__ k_new,
               const uint16_t* __restrict__ v_new, uint16_t* __restrict__ out, float qscale, int S,
               float* __restrict__ parts, unsigned int* __restrict__ tickets) {
@@ -291,19 +321,19 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int bh = b * c.Hkv + kvh;
   const int G = c.Hq / c.Hkv;
-  const int R = c.W + HQ_STAGE;
+  const int R = ring_len(c.W);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
 
   const int T = c.state[HQ_STATE_T];
   const int n_packed = c.state[HQ_STATE_NPACKED];
   const int n_vl = c.state[HQ_STATE_NVL];
-  if (T - n_packed >= R || T >= c.cap) {  // staging full / no room: do nothing
+  if (T - n_packed >= c.W + HQ_STAGE || T >= c.cap) {  // staging full / no room: do nothing
     if (split == 0 && kvh == 0 && b == 0 && threadIdx.x == 0)
       set_err(c.state, T >= c.cap ? HQ_DEVERR_CAPACITY : HQ_DEVERR_STAGING_FULL);
     return;
   }
-  const Geo geo = geo_of(n_packed, n_vl, T);
+  const Geo geo = geo_of(n_packed, n_vl, T, R);
   const int t_lo = static_cast<int>((static_cast<long long>(split) * geo.NT) / S);
   const int t_hi = static_cast<int>((static_cast<long long>(split + 1) * geo.NT) / S);
   const int ntile = t_hi - t_lo;
@@ -315,22 +345,6 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
     }
     fence_mbar_init();
   }
-  // append the new token: ring slot T % R and query-buffer slot T % HQ_QBUF
-  if (split == 0) {
-    const int slot = T % R;
-    for (int i = threadIdx.x; i < 2 * D / 8; i += NTHREADS) {
-      const int which = i / (D / 8), ch = i % (D / 8);
-      const uint4* s = reinterpret_cast<const uint4*>((which ? v_new : k_new) + static_cast<size_t>(bh) * D) + ch;
-      uint4* d = reinterpret_cast<uint4*>((which ? c.vr : c.kr) + (static_cast<size_t>(bh) * R + slot) * D) + ch;
-      *d = *s;
-    }
-    for (int i = threadIdx.x; i < G * D / 8; i += NTHREADS) {
-      const int h = kvh * G + i / (D / 8), ch = i % (D / 8);
-      const uint4* s = reinterpret_cast<const uint4*>(q + (static_cast<size_t>(b) * c.Hq + h) * D) + ch;
-      uint4* d = reinterpret_cast<uint4*>(c.qbuf + ((static_cast<size_t>(b) * c.Hq + h) * HQ_QBUF + (T % HQ_QBUF)) * D) + ch;
-      *d = *s;
-    }
-  }
   __syncthreads();
 
   WarpState ws;
@@ -341,47 +355,47 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
 
   if (warp == NCONS) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      for (int i = 0; i < ntile; ++i) {
-        const int s = i % NSTAGES;
-        if (i >= NSTAGES && !mbar_wait(&empty[s], ((i / NSTAGES) & 1) ^ 1, c.state)) break;
-        uint8_t* st = smem + s * STAGE_BYTES;
-        const int tile = t_lo + i;
-        if (tile < geo.NP) {
-          const size_t row0 = static_cast<size_t>(bh) * c.cap + static_cast<size_t>(tile) * PK;
-          mbar_arrive_expect_tx(&full[s], PK_TX);
-          bulk_g2s(st, c.kq + row0 * (D / 2), 4096, &full[s]);
-          bulk_g2s(st + OFF_VC, c.vq + row0 * (D / 2), 4096, &full[s]);
-          bulk_g2s(st + OFF_KS, c.ksz + row0 * 4, 1024, &full[s]);
-          bulk_g2s(st + OFF_VS, c.vsz + row0 * 4, 1024, &full[s]);
+    // every lane of the producer warp issues copies (a packed tile: 5 bulk
+    // copies; an FP16 tile: one per row and K/V, up to 32)
+    for (int i = 0; i < ntile; ++i) {
+      const int s = i % NSTAGES;
+      const bool ok = i < NSTAGES || mbar_wait(&empty[s], ((i / NSTAGES) & 1) ^ 1, c.state);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      uint8_t* st = smem + s * STAGE_BYTES;
+      const int tile = t_lo + i;
+      if (tile < geo.NP) {
+        if (lane == 0) mbar_arrive_expect_tx(&full[s], PK_TX);
+        __syncwarp();
+        const size_t row0 = static_cast<size_t>(bh) * c.cap + static_cast<size_t>(tile) * PK;
+        if (lane == 0) bulk_g2s(st, c.kq + row0 * (D / 2), 4096, &full[s]);
+        else if (lane == 1) bulk_g2s(st + OFF_VC, c.vq + row0 * (D / 2), 4096, &full[s]);
+        else if (lane == 2) bulk_g2s(st + OFF_KS, c.ksz + row0 * 4, 1024, &full[s]);
+        else if (lane == 3) bulk_g2s(st + OFF_VS, c.vsz + row0 * 4, 1024, &full[s]);
+        else if (lane == 4)
           bulk_g2s(st + OFF_MASK, c.vl_mask + static_cast<size_t>(bh) * (c.cap / 32) + 4 * (tile >> 1), 16, &full[s]);
-        } else if (tile < geo.NP + geo.NV) {
-          const int r0 = (tile - geo.NP) * FT;
-          const int nr = min(FT, n_vl - r0);
-          mbar_arrive_expect_tx(&full[s], nr * 2 * D * 2);
-          for (int r = 0; r < nr; ++r) {
-            const size_t row = static_cast<size_t>(bh) * c.vl_cap + r0 + r;
-            bulk_g2s(st + r * FSTRIDE, c.kf + row * D, 2 * D, &full[s]);
-            bulk_g2s(st + OFF_FV + r * FSTRIDE, c.vf + row * D, 2 * D, &full[s]);
-          }
+      } else {
+        // FP16 tile: one contiguous copy for K and one for V
+        const int j = tile - geo.NP - geo.NV;
+        const uint16_t* ksrc;
+        const uint16_t* vsrc;
+        uint32_t bytes = FT * 2 * D;
+        if (j < 0) {
+          const size_t row = static_cast<size_t>(bh) * c.vl_cap + static_cast<size_t>(tile - geo.NP) * FT;
+          ksrc = c.kf + row * D;
+          vsrc = c.vf + row * D;
+        } else if (j < geo.NR - 1) {
+          const size_t row = static_cast<size_t>(bh) * R + static_cast<size_t>(j) * FT;
+          ksrc = c.kr + row * D;
+          vsrc = c.vr + row * D;
         } else {
-          const int p0 = n_packed + (tile - geo.NP - geo.NV) * FT;
-          const int nr = min(FT, T + 1 - p0);
-          mbar_arrive_expect_tx(&full[s], nr * 2 * D * 2);
-          for (int r = 0; r < nr; ++r) {
-            const int p = p0 + r;
-            const uint16_t* ks;
-            const uint16_t* vs;
-            if (p < T) {
-              ks = c.kr + (static_cast<size_t>(bh) * R + (p % R)) * D;
-              vs = c.vr + (static_cast<size_t>(bh) * R + (p % R)) * D;
-            } else {
-              ks = k_new + static_cast<size_t>(bh) * D;
-              vs = v_new + static_cast<size_t>(bh) * D;
-            }
-            bulk_g2s(st + r * FSTRIDE, ks, 2 * D, &full[s]);
-            bulk_g2s(st + OFF_FV + r * FSTRIDE, vs, 2 * D, &full[s]);
-          }
+          ksrc = k_new + static_cast<size_t>(bh) * D;
+          vsrc = v_new + static_cast<size_t>(bh) * D;
+          bytes = 2 * D;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[s], 2 * bytes);
+          bulk_g2s(st, ksrc, bytes, &full[s]);
+          bulk_g2s(st + OFF_FV, vsrc, bytes, &full[s]);
         }
       }
     }
@@ -412,10 +426,8 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
       const int tile = t_lo + i;
       if (tile < geo.NP) {
         packed_tile(ws, st, qf, tile, n_packed, qscale, g, t);
-      } else if (tile < geo.NP + geo.NV) {
-        fp16_tile(ws, st, qf, min(FT, n_vl - (tile - geo.NP) * FT), qscale, g, t);
       } else {
-        fp16_tile(ws, st, qf, min(FT, T + 1 - (n_packed + (tile - geo.NP - geo.NV) * FT)), qscale, g, t);
+        fp16_tile(ws, st, qf, fp16_valid(geo, tile), qscale, g, t);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
@@ -448,68 +460,125 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
   __syncthreads();  // (B) warp states visible
 
   // ---------------------------------------------------------------- CTA merge -> split partial
-  float* part = parts + (static_cast<size_t>(bh) * S + split) * PART_FLOATS;
+  __shared__ float s_cw[NCONS][8];
+  __shared__ float s_cm[8], s_cl[8];
+  __shared__ int s_glast;
   const float* wsm = reinterpret_cast<const float*>(smem);
-  for (int i = threadIdx.x; i < 8 * D + 16; i += NTHREADS) {
-    if (i < 8) {
-      float mm = -INFINITY;
-      for (int w = 0; w < NCONS; ++w) mm = fmaxf(mm, wsm[w * PART_FLOATS + i]);
-      float ll = 0.f;
-      for (int w = 0; w < NCONS; ++w) {
-        const float mw = wsm[w * PART_FLOATS + i];
-        ll += mw == -INFINITY ? 0.f : wsm[w * PART_FLOATS + 8 + i] * ex2(mw - mm);
-      }
-      part[i] = mm;
-      part[8 + i] = ll;
-    } else if (i >= 16) {
-      const int qc = (i - 16) / D;
-      float mm = -INFINITY;
-      for (int w = 0; w < NCONS; ++w) mm = fmaxf(mm, wsm[w * PART_FLOATS + qc]);
-      float acc = 0.f;
-      for (int w = 0; w < NCONS; ++w) {
-        const float mw = wsm[w * PART_FLOATS + qc];
-        acc += mw == -INFINITY ? 0.f : wsm[w * PART_FLOATS + i] * ex2(mw - mm);
-      }
-      part[i] = acc;
+  if (threadIdx.x < 8) {
+    const int qc = threadIdx.x;
+    float mm = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NCONS; ++w) mm = fmaxf(mm, wsm[w * PART_FLOATS + qc]);
+    float ll = 0.f;
+#pragma unroll
+    for (int w = 0; w < NCONS; ++w) {
+      const float mw = wsm[w * PART_FLOATS + qc];
+      const float wt = mw == -INFINITY ? 0.f : ex2(mw - mm);
+      s_cw[w][qc] = wt;
+      ll += wt * wsm[w * PART_FLOATS + 8 + qc];
     }
+    s_cm[qc] = mm;
+    s_cl[qc] = ll;
   }
-  __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) s_last = (atomicAdd(&tickets[1 + bh], 1u) == static_cast<unsigned>(S - 1)) ? 1 : 0;
-  __syncthreads();
-  if (s_last) {
-    __threadfence();
-    // log-sum-exp merge of the S partials of this (b, kv head)
-    const float* pb = parts + static_cast<size_t>(bh) * S * PART_FLOATS;
-    for (int i = threadIdx.x; i < G * D; i += NTHREADS) {
-      const int qc = i / D, dd = i % D;
-      float mm = -INFINITY;
-      for (int sp = 0; sp < S; ++sp) mm = fmaxf(mm, __ldcg(pb + sp * PART_FLOATS + qc));
-      float ll = 0.f, acc = 0.f;
-      for (int sp = 0; sp < S; ++sp) {
-        const float ms = __ldcg(pb + sp * PART_FLOATS + qc);
-        if (ms == -INFINITY) continue;
-        const float w = ex2(ms - mm);
-        ll += __ldcg(pb + sp * PART_FLOATS + 8 + qc) * w;
-        acc += __ldcg(pb + sp * PART_FLOATS + 16 + qc * D + dd) * w;
-      }
-      out[(static_cast<size_t>(b) * c.Hq + kvh * G + qc) * D + dd] = __half_as_ushort(__float2half_rn(acc / ll));
-    }
-    if (threadIdx.x == 0) {
-      tickets[1 + bh] = 0u;
-      __threadfence();
-    }
+  float* part = parts + (static_cast<size_t>(bh) * S + split) * PART_FLOATS;
+  if (threadIdx.x < 8) {
+    part[threadIdx.x] = s_cm[threadIdx.x];
+    part[8 + threadIdx.x] = s_cl[threadIdx.x];
   }
-  // grid-wide: the last CTA advances T (every CTA has read the state by now)
+  for (int i = threadIdx.x; i < 8 * D / 4; i += NTHREADS) {
+    const int qc = (4 * i) / D;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < NCONS; ++w) {
+      const float4 o = reinterpret_cast<const float4*>(wsm + w * PART_FLOATS + 16)[i];
+      const float wt = s_cw[w][qc];
+      acc.x = fmaf(wt, o.x, acc.x);
+      acc.y = fmaf(wt, o.y, acc.y);
+      acc.z = fmaf(wt, o.z, acc.z);
+      acc.w = fmaf(wt, o.w, acc.w);
+    }
+    reinterpret_cast<float4*>(part + 16)[i] = acc;
+  }
+  // completion tickets: every thread releases its part of the partial, then one
+  // thread learns whether this is the last split of its (b, kv head) and/or the
+  // last CTA of the grid; the last CTA acquires before reading the partials
+  fence_acq_rel_gpu();
+  __syncthreads();
   if (threadIdx.x == 0) {
-    __threadfence();
-    const unsigned total = gridDim.x * gridDim.y * gridDim.z;
-    if (atomicAdd(&tickets[0], 1u) == total - 1) {
-      c.state[HQ_STATE_T] = T + 1;
-      c.state[HQ_STATE_NQ] = min(c.state[HQ_STATE_NQ] + 1, HQ_QBUF);
-      tickets[0] = 0u;
-      __threadfence();
+    s_last = atomicAdd(&tickets[1 + bh], 1u) == static_cast<unsigned>(S - 1);
+    s_glast = atomicAdd(&tickets[0], 1u) == gridDim.x * gridDim.y * gridDim.z - 1;
+  }
+  __syncthreads();
+  if (s_last || s_glast) fence_acq_rel_gpu();
+  if (s_last) {
+    // log-sum-exp merge of the S partials of this (b, kv head): m and l of every
+    // split are fetched in parallel, the weights computed once, then each thread
+    // sums its outputs over the splits with independent loads in flight.
+    const float* pb = parts + static_cast<size_t>(bh) * S * PART_FLOATS;
+    float* sm_m = reinterpret_cast<float*>(smem);      // [S][8]
+    float* sm_l = sm_m + S * 8;                        // [S][8]
+    float* sm_w = sm_l + S * 8;                        // [S][8] normalised weights
+    for (int i = threadIdx.x; i < S * 8; i += NTHREADS) {
+      sm_m[i] = __ldcg(pb + (i >> 3) * PART_FLOATS + (i & 7));
+      sm_l[i] = __ldcg(pb + (i >> 3) * PART_FLOATS + 8 + (i & 7));
     }
+    __syncthreads();
+    if (threadIdx.x < 8) {
+      const int qc = threadIdx.x;
+      float mm = -INFINITY;
+      for (int sp = 0; sp < S; ++sp) mm = fmaxf(mm, sm_m[sp * 8 + qc]);
+      float ll = 0.f;
+      for (int sp = 0; sp < S; ++sp) {
+        const float ms = sm_m[sp * 8 + qc];
+        if (ms != -INFINITY) ll += sm_l[sp * 8 + qc] * ex2(ms - mm);
+      }
+      s_cm[qc] = mm;
+      s_cl[qc] = ll > 0.f ? 1.0f / ll : 0.f;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < S * 8; i += NTHREADS) {
+      const float ms = sm_m[i];
+      sm_w[i] = ms == -INFINITY ? 0.f : ex2(ms - s_cm[i & 7]) * s_cl[i & 7];
+    }
+    __syncthreads();
+    for (int it = threadIdx.x; it < G * (D / 2); it += NTHREADS) {
+      const int qc = it / (D / 2), d2 = it % (D / 2);
+      const float2* src = reinterpret_cast<const float2*>(pb + 16 + qc * D) + d2;
+      float ax = 0.f, ay = 0.f;
+#pragma unroll 8
+      for (int sp = 0; sp < S; ++sp) {
+        const float2 o = __ldcg(src + sp * (PART_FLOATS / 2));
+        const float w = sm_w[sp * 8 + qc];
+        ax = fmaf(w, o.x, ax);
+        ay = fmaf(w, o.y, ay);
+      }
+      reinterpret_cast<__half2*>(out + (static_cast<size_t>(b) * c.Hq + kvh * G + qc) * D)[d2] = __floats2half2_rn(ax, ay);
+    }
+    // every split of this head has consumed its tiles: append the new token to
+    // the ring (slot T % R) and this group's queries to the query buffer
+    const int slot = T % R;
+    for (int i = threadIdx.x; i < (2 + G) * (D / 8); i += NTHREADS) {
+      const int row = i / (D / 8), ch = i % (D / 8);
+      const uint4* src;
+      uint4* dst;
+      if (row < 2) {
+        src = reinterpret_cast<const uint4*>((row ? v_new : k_new) + static_cast<size_t>(bh) * D) + ch;
+        dst = reinterpret_cast<uint4*>((row ? c.vr : c.kr) + (static_cast<size_t>(bh) * R + slot) * D) + ch;
+      } else {
+        const size_t h = static_cast<size_t>(b) * c.Hq + kvh * G + (row - 2);
+        src = reinterpret_cast<const uint4*>(q + h * D) + ch;
+        dst = reinterpret_cast<uint4*>(c.qbuf + (h * HQ_QBUF + (T % HQ_QBUF)) * D) + ch;
+      }
+      *dst = *src;
+    }
+    if (threadIdx.x == 0) tickets[1 + bh] = 0u;
+  }
+  // the last CTA of the grid advances T (every CTA read the state at its start)
+  if (s_glast && threadIdx.x == 0) {
+    c.state[HQ_STATE_T] = T + 1;
+    c.state[HQ_STATE_NQ] = min(c.state[HQ_STATE_NQ] + 1, HQ_QBUF);
+    tickets[0] = 0u;
   }
 }
 
@@ -517,10 +586,11 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
 
 int decode_splits(const hq_cache& c, int sms) {
   const int units = c.B * c.Hkv;
-  const int nt_max = c.cap / PK + c.vl_cap / FT + (c.W + HQ_STAGE + 1 + FT - 1) / FT;
-  int s = (2 * sms + units - 1) / units;
+  const int nt_max = c.cap / PK + c.vl_cap / FT + ring_len(c.W) / FT + 1;
+  int s = (3 * sms) / units;  // one wave: 3 CTAs per SM
   const int cap_s = (nt_max + 3) / 4;
   if (s > cap_s) s = cap_s;
+  if (s > 64) s = 64;
   if (s < 1) s = 1;
   return s;
 }

@@ -22,7 +22,7 @@ struct Dims {
   int B, Hkv, cap, vl_cap, R, W;
 };
 
-__device__ __forceinline__ Dims dims_of(const hq_cache& c) { return Dims{c.B, c.Hkv, c.cap, c.vl_cap, c.W + HQ_STAGE, c.W}; }
+__device__ __forceinline__ Dims dims_of(const hq_cache& c) { return Dims{c.B, c.Hkv, c.cap, c.vl_cap, ring_len(c.W), c.W}; }
 
 // Pack one 128-value fp16 row into 64 code bytes + 4 (scale, zero) words.
 // Warp-cooperative: lane l owns values 4l .. 4l+3 (group l / 8).

@@ -87,7 +87,7 @@ __device__ __forceinline__ int find_sorted(const int32_t* __restrict__ a, int n,
 __device__ void load_keys(const SelArgs& a, const SelGeo& g, int bh, int j0, uint8_t* ks) {
   const hq_cache& c = a.c;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int R = c.W + HQ_STAGE;
+  const int R = ring_len(c.W);
   for (int r = warp; r < CH; r += NW_SEL) {
     const int p = j0 + r;
     uint2 v = make_uint2(0u, 0u);
@@ -408,12 +408,16 @@ hq_status launch_select(const hq_cache& c, const uint16_t* kd, int L, const uint
   a.scores = scores_out ? scores_out : reinterpret_cast<float*>(w);
   a.qscale = (1.0f / sqrtf(static_cast<float>(D))) * LOG2E;
   const size_t smem = select_smem_bytes(c);
+  // the attribute is raised once per device to the size of the largest group (HQ_MAX_GQA)
+  hq_cache cmax = c;
+  cmax.Hq = cmax.Hkv * HQ_MAX_GQA;
+  const int smem_max = static_cast<int>(select_smem_bytes(cmax));
   int dev = 0;
   cudaGetDevice(&dev);
   static bool attr_done[64] = {};
   if (dev >= 64 || !attr_done[dev]) {
-    if (cudaFuncSetAttribute(select_pass<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess ||
-        cudaFuncSetAttribute(select_pass<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+    if (cudaFuncSetAttribute(select_pass<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max) != cudaSuccess ||
+        cudaFuncSetAttribute(select_pass<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max) != cudaSuccess)
       return HQ_ERR_CUDA;
     if (dev < 64) attr_done[dev] = true;
   }

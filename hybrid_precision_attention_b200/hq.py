@@ -111,7 +111,7 @@ class HybridCache:
         if vl_cap is None:
             vl_cap = max(16, ((k_of(max(cap - W, 0), rho_bp) + 15) // 16) * 16)
         self.B, self.Hq, self.Hkv, self.D, self.W, self.rho_bp, self.cap, self.vl_cap = B, Hq, Hkv, D, W, rho_bp, cap, vl_cap
-        self.R = W + HQ_STAGE
+        self.R = ((W + HQ_STAGE + 15) // 16) * 16   # HQ_RING_LEN(W)
         dev = torch.device(device)
         z = lambda shape, dt: torch.zeros(shape, dtype=dt, device=dev)
         self.kq = z((B, Hkv, cap, D // 2), torch.uint8)

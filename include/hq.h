@@ -57,6 +57,8 @@ extern "C" {
 #define HQ_STAGE 64           /* staged tokens before a merge = reselection period */
 #define HQ_QBUF 64            /* buffered queries kept for the column-mass estimate */
 #define HQ_MAX_GQA 8          /* query heads per kv head supported by the decode kernel */
+/* FP16 ring length for a window W: W + HQ_STAGE rounded up to a multiple of 16 */
+#define HQ_RING_LEN(W) ((((W) + HQ_STAGE) + 15) / 16 * 16)
 
 typedef struct CUstream_st* hq_stream_t;  /* same type as cudaStream_t */
 
@@ -95,7 +97,7 @@ enum {
 /*
  * The hybrid KV cache of one attention layer.  Every array is caller-owned
  * device memory laid out as stated ([..] = row-major shape, innermost last).
- * R = W + HQ_STAGE is the FP16 ring length.
+ * R = HQ_RING_LEN(W) is the FP16 ring length (W + HQ_STAGE rounded up to 16).
  *
  *   kq, vq    uint8  [B, Hkv, cap, D/2]   K4V4 codes, dense by position
  *   ksz, vsz  uint32 [B, Hkv, cap, D/32]  per group: scale fp16 bits | zero fp16 bits << 16

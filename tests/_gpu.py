@@ -3,8 +3,11 @@ on the same seeded inputs and compare them.
 
 Tolerances (the reasoning is in the design notes):
   decode output        max-abs <= 2e-3 and rel-L2 <= 1e-3 against the float64 oracle
-  column-mass scores   relative error <= SCORE_RTOL per score (float32 sums of
-                       exp2 on tensor-core logits; packed keys rebuilt in fp16)
+  column-mass scores   relative error <= SCORE_RTOL per score.  The kernel
+                       rebuilds each packed key as fp16 (one rounding, <= 2^-11
+                       relative per element, ~2e-4 nat on a logit) and sums
+                       float32 exp2 weights; the measured worst case is ~2e-4,
+                       so the bound is 5e-4 and the tie band twice that
   selected positions   exact when the GPU's own float32 scores are fed to the
                        oracle's stable top-k; against the oracle's float64
                        scores, a position may differ only inside the band
@@ -18,8 +21,8 @@ import torch
 
 from oracle import formats, hybrid, select as osel
 
-SCORE_RTOL = 2e-4
-BAND_RTOL = 5e-4
+SCORE_RTOL = 5e-4
+BAND_RTOL = 1e-3
 DEC_MAXABS = 2e-3
 DEC_RELL2 = 1e-3
 
@@ -51,6 +54,9 @@ def check_decode(out_gpu: torch.Tensor, ref: np.ndarray, what=""):
 def check_selection(gpu_scores: np.ndarray, gpu_sel: np.ndarray, ref_scores: np.ndarray, k: int, what=""):
     """gpu_scores/ref_scores over the n candidates of one (b, kv head); gpu_sel = the GPU's k positions."""
     n = ref_scores.shape[0]
+    if n == 0:
+        assert k == 0 and len(gpu_sel) == 0, what
+        return 0.0
     g = gpu_scores[:n].astype(np.float64)
     rel = np.abs(g - ref_scores) / np.maximum(np.abs(ref_scores), 1e-30)
     assert rel.max() <= SCORE_RTOL, f"{what} score rel err {rel.max():.3e}"
