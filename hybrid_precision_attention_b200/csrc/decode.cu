@@ -18,7 +18,9 @@
 //   * a producer warp streams tiles into a 6-stage shared-memory ring with
 //     large 1-D bulk async copies (cp.async.bulk, mbarrier completion, no
 //     multicast): 5 copies per packed tile, 2 per FP16 tile;
-//   * 4 consumer warps take whole tiles round-robin.  Nibbles become fp16 in
+//   * 3 consumer warps take whole tiles round-robin, each owning 2 of the 6
+//     stages (tile i -> stage i % 6 -> warp i % 3), so every stage has a single
+//     consumer and a waiter is never a full barrier phase behind.  Nibbles become fp16 in
 //     registers (exponent-bias trick + one fma with the group's scale/zero), and
 //     both products run on tensor cores with mma.m16n8k16 (f32 accumulate):
 //       S^T[keys x 8 queries] = K^ (16 keys x 16 dims) . Q^T
@@ -38,9 +40,14 @@
 namespace hq {
 namespace {
 
-constexpr int NCONS = 4;                       // consumer warps
+constexpr int NCONS = 3;                       // consumer warps
 constexpr int NTHREADS = (NCONS + 1) * 32;     // + producer warp
 constexpr int NSTAGES = 6;
+// Each stage must have exactly one consumer warp: a parity wait on an mbarrier
+// only tells the current phase from the one before it, so a warp that reached a
+// stage while another warp's earlier tile there had not landed yet would see the
+// older completed phase and consume the wrong data.
+static_assert(NSTAGES % NCONS == 0, "every stage needs a single owner warp");
 constexpr int PK = 64;                         // positions per packed tile
 constexpr int FT = 16;                         // rows per FP16 tile
 constexpr int FSTRIDE = 256;                   // bytes per FP16 row in shared memory (one contiguous copy)
@@ -317,6 +324,8 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t full[NSTAGES], empty[NSTAGES];
   __shared__ int s_last;
+  __shared__ int s_timeout;      // a bounded wait gave up somewhere in this CTA
+  __shared__ int s_issued[NSTAGES];  // tiles issued into each stage
 
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int bh = b * c.Hkv + kvh;
@@ -342,7 +351,9 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
     for (int i = 0; i < NSTAGES; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
+      s_issued[i] = 0;
     }
+    s_timeout = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -360,7 +371,11 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
     for (int i = 0; i < ntile; ++i) {
       const int s = i % NSTAGES;
       const bool ok = i < NSTAGES || mbar_wait(&empty[s], ((i / NSTAGES) & 1) ^ 1, c.state);
-      if (!__all_sync(0xffffffffu, ok)) break;
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) s_timeout = 1;
+        break;
+      }
+      if (lane == 0) s_issued[s] = i / NSTAGES + 1;
       uint8_t* st = smem + s * STAGE_BYTES;
       const int tile = t_lo + i;
       if (tile < geo.NP) {
@@ -421,7 +436,10 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
     for (int i = warp; i < ntile; i += NCONS) {
       const int s = i % NSTAGES;
       // the timeout decision is made warp-uniform so the warp never splits
-      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (i / NSTAGES) & 1, c.state))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (i / NSTAGES) & 1, c.state))) {
+        if (lane == 0) s_timeout = 1;
+        break;
+      }
       const uint8_t* st = smem + s * STAGE_BYTES;
       const int tile = t_lo + i;
       if (tile < geo.NP) {
@@ -440,6 +458,14 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
     }
   }
   __syncthreads();  // (A) every tile consumed: stage memory is free for the merge
+  if (s_timeout) {
+    // never expected: before the stage memory is reused or the CTA exits, wait
+    // (bounded) for every bulk copy this CTA issued to land
+    if (threadIdx.x == 0)
+      for (int st = 0; st < NSTAGES; ++st)
+        if (s_issued[st] > 0) mbar_wait(&full[st], (s_issued[st] - 1) & 1, c.state);
+    __syncthreads();
+  }
   if (warp < NCONS) {
     float* wsm = reinterpret_cast<float*>(smem) + warp * PART_FLOATS;
     if (g == 0) {

@@ -142,6 +142,8 @@ class Pair:
         H = hq()
         out = H.hq_decode_attn(self.g, dev(q), dev(k), dev(v))
         ref = self.r.decode(q, k, v)
+        st = self.g.state()
+        assert st["err"] == 0 and st["T"] == self.r.T, st
         return out, ref
 
     def reselect_merge(self, check=True):
@@ -164,6 +166,7 @@ class Pair:
         H.hq_pack_merge(self.g)
         self.r.merge(vl)
         torch.cuda.synchronize()
+        assert self.g.state()["err"] == 0, self.g.state()
         if check:
             self.check_state()
         return vl
