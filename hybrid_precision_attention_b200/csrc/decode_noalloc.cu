@@ -1,0 +1,82 @@
+// decode_noalloc.cu — hq_decode_attn_noalloc: the decode step for callers that
+// must not allocate device memory.
+//
+// hq_decode_attn needs a caller-provided workspace (split-K partials and
+// completion counters).  Some callers cannot obtain one: a plugin running inside
+// a serving engine that owns every byte of device memory and forbids allocation
+// once it is up, or a latency-critical loop where cudaMalloc / cudaFree would
+// synchronise the device.  This entry point takes its workspace from a fixed
+// scratch array compiled into the library instead.
+//
+//   * The scratch is a file-scope __device__ array of HQ_NOALLOC_SCRATCH_BYTES
+//     (4 MiB).  Every GPU on which the library is loaded holds one copy until the
+//     process exits.
+//   * Host code cannot use the array's name as a device address, so the first
+//     call on each device (with that device current) looks the address up with
+//     cudaGetSymbolAddress and remembers it.  Make that first call before any
+//     stream capture.
+//   * All calls on a device share the one array and it keeps whatever the last
+//     call left in it: each call clears the completion counters (an async
+//     memset on the caller's stream) before the kernel.  Two calls whose
+//     executions overlap on the GPU (different streams, no ordering) race on
+//     the array and must not be issued.
+//   * No allocation happens here: no cudaMalloc, cudaFree or allocating library
+//     routine.  A cache whose decode workspace would exceed the array is
+//     rejected with HQ_ERR_WORKSPACE before anything is launched.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "common.cuh"
+
+namespace hq {
+hq_status launch_decode(const hq_cache& c, const uint16_t* q, const uint16_t* kn, const uint16_t* vn, uint16_t* out,
+                        float sm_scale, void* ws, int sms, cudaStream_t st);
+size_t decode_workspace(const hq_cache& c, int sms);
+size_t decode_counter_bytes(const hq_cache& c);
+}  // namespace hq
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[HQ_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of this device's scratch array (looked up once per device).
+hq_status scratch_address(int dev, void** out) {
+  if (dev < 0 || dev >= kMaxDevices) return HQ_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return HQ_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return HQ_OK;
+}
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" HQ_API hq_status hq_decode_attn_noalloc(const hq_cache* c, const uint16_t* q, const uint16_t* k_new,
+                                                   const uint16_t* v_new, uint16_t* out, float sm_scale,
+                                                   hq_stream_t stream) {
+  hq_status s = hq_cache_validate(c);
+  if (s != HQ_OK) return s;
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(out)) return HQ_ERR_INVALID;
+  if (!(sm_scale > 0.0f)) return HQ_ERR_INVALID;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HQ_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return HQ_ERR_CUDA;
+  if (hq::decode_workspace(*c, sms) > HQ_NOALLOC_SCRATCH_BYTES) return HQ_ERR_WORKSPACE;
+  void* ws = nullptr;
+  s = scratch_address(dev, &ws);
+  if (s != HQ_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // the counters must start at zero; the rest of the scratch is written before it is read
+  if (cudaMemsetAsync(ws, 0, hq::decode_counter_bytes(*c), st) != cudaSuccess) return HQ_ERR_CUDA;
+  return hq::launch_decode(*c, q, k_new, v_new, out, sm_scale, ws, sms, st);
+}

@@ -61,13 +61,16 @@ _lib.hq_pack_merge.restype = _I
 _lib.hq_pack_merge.argtypes = [_CP, _P, _P, _I, _P, _S, _P]
 _lib.hq_decode_attn.restype = _I
 _lib.hq_decode_attn.argtypes = [_CP, _P, _P, _P, _P, ctypes.c_float, _P, _S, _P]
+_lib.hq_decode_attn_noalloc.restype = _I
+_lib.hq_decode_attn_noalloc.argtypes = [_CP, _P, _P, _P, _P, ctypes.c_float, _P]
 _lib.hq_prefill_workspace_bytes.restype = _S
 _lib.hq_prefill_workspace_bytes.argtypes = [_I, _I, _I, _I, _I]
 _lib.hq_prefill_attn.restype = _I
 _lib.hq_prefill_attn.argtypes = [_I, _I, _I, _I, _I, _P, _P, _P, _P, _I, _I, _I, ctypes.c_float, _P, _P, _S, _P]
 
 EXPORTED = ("hq_abi_version", "hq_status_str", "hq_cache_validate", "hq_workspace_bytes", "hq_cache_reset",
-            "hq_select_vlines", "hq_pack_merge", "hq_decode_attn", "hq_prefill_workspace_bytes", "hq_prefill_attn")
+            "hq_select_vlines", "hq_pack_merge", "hq_decode_attn", "hq_decode_attn_noalloc",
+            "hq_prefill_workspace_bytes", "hq_prefill_attn")
 
 
 def _check(st: int, what: str):
@@ -199,6 +202,23 @@ def hq_decode_attn(cache: HybridCache, q, k_new, v_new, out=None, sm_scale: floa
     ws = cache.workspace(OP_DECODE)
     _check(_lib.hq_decode_attn(ctypes.byref(cache.c), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out),
                                ctypes.c_float(sm_scale), _ptr(ws), ws.numel(), _stream(stream)), "hq_decode_attn")
+    return out
+
+
+def hq_decode_attn_noalloc(cache: HybridCache, q, k_new, v_new, out=None, sm_scale: float = None, stream=None):
+    """hq_decode_attn for callers that may not allocate device memory: no
+    workspace argument, the library's fixed scratch array is used instead (see
+    include/hq.h for its size and sharing rules)."""
+    _need(q, torch.float16, (cache.B, cache.Hq, cache.D), "q")
+    _need(k_new, torch.float16, (cache.B, cache.Hkv, cache.D), "k_new")
+    _need(v_new, torch.float16, (cache.B, cache.Hkv, cache.D), "v_new")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, torch.float16, (cache.B, cache.Hq, cache.D), "out")
+    if sm_scale is None:
+        sm_scale = cache.D ** -0.5
+    _check(_lib.hq_decode_attn_noalloc(ctypes.byref(cache.c), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out),
+                                       ctypes.c_float(sm_scale), _stream(stream)), "hq_decode_attn_noalloc")
     return out
 
 

@@ -233,6 +233,29 @@ HQ_API hq_status hq_prefill_attn(int32_t B, int32_t Hq, int32_t Hkv, int32_t L, 
                           float sm_scale, uint16_t* out, void* ws, size_t ws_bytes,
                           hq_stream_t stream);
 
+/*
+ * Allocation-free decode step.  The paper has no counterpart: this is a
+ * deployment variant of hq_decode_attn for callers that may not allocate
+ * device memory at all, such as a plugin inside a serving engine that owns all
+ * device memory, or a latency-critical loop where cudaMalloc / cudaFree would
+ * synchronise the device.  Arguments and result are those of hq_decode_attn,
+ * minus the workspace: the library uses a fixed scratch array of
+ * HQ_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until the
+ * process exits.
+ *   - The first call on a device (with that device current) looks up the
+ *     array's device address; make that first call before any stream capture.
+ *   - All calls on a device share the array and it keeps the last call's
+ *     contents; each call clears what must start at zero itself.  Calls whose
+ *     executions can overlap on the GPU (unordered streams) race on the array:
+ *     order them on one stream.
+ *   - Returns HQ_ERR_WORKSPACE when this cache's decode workspace
+ *     (hq_workspace_bytes(c, HQ_OP_DECODE, 0)) exceeds HQ_NOALLOC_SCRATCH_BYTES;
+ *     nothing is launched then.  It never calls cudaMalloc or cudaFree.
+ */
+#define HQ_NOALLOC_SCRATCH_BYTES (4u << 20)
+HQ_API hq_status hq_decode_attn_noalloc(const hq_cache* c, const uint16_t* q, const uint16_t* k_new,
+                                        const uint16_t* v_new, uint16_t* out, float sm_scale, hq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
