@@ -18,6 +18,20 @@ constexpr float LOG2E = 1.4426950408889634f;
 
 __host__ __device__ __forceinline__ int ring_len(int W) { return HQ_RING_LEN(W); }
 
+// K4V4 page of position p of (b, kv head) bh
+__host__ __device__ __forceinline__ uint8_t* page_of(const hq_cache& c, size_t bh, int p) {
+  return c.pages + (bh * static_cast<size_t>(c.cap / HQ_PAGE_POSITIONS) + (p >> 6)) * HQ_PAGE_BYTES;
+}
+__host__ __device__ __forceinline__ uint8_t* row_codes(uint8_t* page, int which, int p) {
+  return page + (which ? HQ_PAGE_VCODES : HQ_PAGE_KCODES) + (p & 63) * (HQ_HEAD_DIM / 2);
+}
+__host__ __device__ __forceinline__ uint32_t* row_sz(uint8_t* page, int which, int p) {
+  return reinterpret_cast<uint32_t*>(page + (which ? HQ_PAGE_VSZ : HQ_PAGE_KSZ) + (p & 63) * 16);
+}
+__host__ __device__ __forceinline__ uint32_t* page_mask(uint8_t* page) {
+  return reinterpret_cast<uint32_t*>(page + HQ_PAGE_VLMASK);
+}
+
 // release / acquire fences at GPU scope (cheaper than the sequentially
 // consistent fence behind __threadfence)
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }

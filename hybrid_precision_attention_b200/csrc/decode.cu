@@ -7,20 +7,22 @@
 // materialised.  The pages' kernel is Triton for SM80+; this is a B200 design.
 //
 // Design (bandwidth-bound: ~160 B of K4V4 per token and kv head):
-//   * grid = (splits S, Hkv, B), one wave (S * Hkv * B <= 3 CTAs per SM); every
+//   * grid = (splits S, Hkv, B), one wave (a wide CTA per SM, or 3 narrow CTAs
+//     per SM for large batches); every
 //     CTA owns one GQA group (all G <= 8 query heads of a kv head share one
 //     pass over the bytes) and a contiguous range of the head's tile list:
-//     packed tiles (64 positions: 4 KB K codes, 4 KB V codes, 1 KB + 1 KB
-//     scale/zero, 16 B of the VL bitmap), VL tiles (16 FP16 rows of the VL
+//     packed tiles (one page of 64 positions: 4 KB K codes, 4 KB V codes,
+//     1 KB + 1 KB scale/zero, the VL bitmap), VL tiles (16 FP16 rows of the VL
 //     store), ring tiles (16 slots of the FP16 ring, which is a multiple of 16
 //     long, so a tile is one contiguous copy) and a last tile holding the new
 //     token read straight from its input pointer;
-//   * a producer warp streams tiles into a 6-stage shared-memory ring with
+//   * a producer warp streams tiles into a 2 NC-stage shared-memory ring with
 //     large 1-D bulk async copies (cp.async.bulk, mbarrier completion, no
-//     multicast): 5 copies per packed tile, 2 per FP16 tile;
-//   * 3 consumer warps take whole tiles round-robin, each owning 2 of the 6
-//     stages (tile i -> stage i % 6 -> warp i % 3), so every stage has a single
-//     consumer and a waiter is never a full barrier phase behind.  Nibbles become fp16 in
+//     multicast): 1 copy per packed tile, 2 per FP16 tile;
+//   * NC consumer warps take whole tiles round-robin, each owning 2 of the 2 NC
+//     stages (tile i -> stage i % 2NC -> warp i % NC), so every stage has a
+//     single consumer and a waiter is never a full barrier phase behind; splits
+//     get equal shares of the bytes.  Nibbles become fp16 in
 //     registers (exponent-bias trick + one fma with the group's scale/zero), and
 //     both products run on tensor cores with mma.m16n8k16 (f32 accumulate):
 //       S^T[keys x 8 queries] = K^ (16 keys x 16 dims) . Q^T
@@ -40,14 +42,16 @@
 namespace hq {
 namespace {
 
-constexpr int NCONS = 3;                       // consumer warps
-constexpr int NTHREADS = (NCONS + 1) * 32;     // + producer warp
-constexpr int NSTAGES = 6;
+// Two CTA shapes, one kernel template (NC consumer warps, 2 stages each, one
+// producer warp):
+//   wide  : NC = 9, 18 stages, 1 CTA per SM   (few kv heads: fewer, longer splits)
+//   narrow: NC = 3,  6 stages, 3 CTAs per SM  (large batches)
 // Each stage must have exactly one consumer warp: a parity wait on an mbarrier
 // only tells the current phase from the one before it, so a warp that reached a
 // stage while another warp's earlier tile there had not landed yet would see the
-// older completed phase and consume the wrong data.
-static_assert(NSTAGES % NCONS == 0, "every stage needs a single owner warp");
+// older completed phase and consume the wrong data.  With NSTAGES = 2 NC,
+// stage s belongs to warp s % NC.
+constexpr int NC_WIDE = 9, NC_NARROW = 3;
 constexpr int PK = 64;                         // positions per packed tile
 constexpr int FT = 16;                         // rows per FP16 tile
 constexpr int FSTRIDE = 256;                   // bytes per FP16 row in shared memory (one contiguous copy)
@@ -55,7 +59,9 @@ constexpr int OFF_VC = 4096, OFF_KS = 8192, OFF_VS = 9216, OFF_MASK = 10240;
 constexpr int OFF_FV = FT * FSTRIDE;           // V rows of an FP16 tile
 constexpr int STAGE_BYTES = 10368;             // max(10256, 2 * 16 * 256 = 8192), 128-aligned
 constexpr int PART_FLOATS = 16 + 8 * D;        // m[8], l[8], O[8][128]
-constexpr uint32_t PK_TX = 4096 * 2 + 1024 * 2 + 16;
+constexpr uint32_t PK_TX = HQ_PAGE_VLMASK + 16;   // codes, scale/zero words and the bitmap: one copy
+static_assert(OFF_VC == HQ_PAGE_VCODES && OFF_KS == HQ_PAGE_KSZ && OFF_VS == HQ_PAGE_VSZ && OFF_MASK == HQ_PAGE_VLMASK,
+              "a packed stage is a verbatim copy of the page prefix");
 
 // key slot -> shared-memory row inside a 16-key block.  Packed tiles (64-byte
 // rows): {0,5,1,4,2,7,3,6, 8,13,9,12,10,15,11,14}; FP16 tiles (256-byte rows):
@@ -163,7 +169,7 @@ __device__ __forceinline__ void packed_tile(WarpState& ws, const uint8_t* st, co
   const uint8_t* vc = st + OFF_VC;
   const uint32_t* ks = reinterpret_cast<const uint32_t*>(st + OFF_KS);
   const uint32_t* vs = reinterpret_cast<const uint32_t*>(st + OFF_VS);
-  const uint32_t* mk = reinterpret_cast<const uint32_t*>(st + OFF_MASK) + 2 * (tile & 1);
+  const uint32_t* mk = reinterpret_cast<const uint32_t*>(st + OFF_MASK);
   const int base = tile * PK;
   const bool full = base + PK <= n_packed;
 
@@ -317,10 +323,14 @@ __device__ __forceinline__ void fp16_tile(WarpState& ws, const uint8_t* st, cons
   }
 }
 
-__global__ void __launch_bounds__(NTHREADS, 3)
+template <int NCONS, int MINB>
+__global__ void __launch_bounds__((NCONS + 1) * 32, MINB)
 decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* __restrict__ k_new,
               const uint16_t* __restrict__ v_new, uint16_t* __restrict__ out, float qscale, int S,
               float* __restrict__ parts, unsigned int* __restrict__ tickets) {
+  constexpr int NSTAGES = 2 * NCONS;
+  constexpr int NTHREADS = (NCONS + 1) * 32;
+  static_assert(NSTAGES % NCONS == 0, "every stage needs a single owner warp");
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t full[NSTAGES], empty[NSTAGES];
   __shared__ int s_last;
@@ -343,8 +353,14 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
     return;
   }
   const Geo geo = geo_of(n_packed, n_vl, T, R);
-  const int t_lo = static_cast<int>((static_cast<long long>(split) * geo.NT) / S);
-  const int t_hi = static_cast<int>((static_cast<long long>(split + 1) * geo.NT) / S);
+  // splits get equal shares of the bytes: a packed tile (10 KB) counts 5, an
+  // FP16 tile (8 KB) counts 4
+  const long long wp = 5ll * geo.NP;
+  const long long wt = wp + 4ll * (geo.NV + geo.NR);
+  const long long w_lo = (static_cast<long long>(split) * wt) / S;
+  const long long w_hi = (static_cast<long long>(split + 1) * wt) / S;
+  const int t_lo = static_cast<int>(w_lo <= wp ? (w_lo + 4) / 5 : geo.NP + (w_lo - wp + 3) / 4);
+  const int t_hi = static_cast<int>(w_hi <= wp ? (w_hi + 4) / 5 : geo.NP + (w_hi - wp + 3) / 4);
   const int ntile = t_hi - t_lo;
 
   if (threadIdx.x == 0) {
@@ -366,51 +382,42 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
 
   if (warp == NCONS) {
     // ---------------------------------------------------------------- producer
-    // every lane of the producer warp issues copies (a packed tile: 5 bulk
-    // copies; an FP16 tile: one per row and K/V, up to 32)
-    for (int i = 0; i < ntile; ++i) {
-      const int s = i % NSTAGES;
-      const bool ok = i < NSTAGES || mbar_wait(&empty[s], ((i / NSTAGES) & 1) ^ 1, c.state);
-      if (!__all_sync(0xffffffffu, ok)) {
-        if (lane == 0) s_timeout = 1;
-        break;
-      }
-      if (lane == 0) s_issued[s] = i / NSTAGES + 1;
-      uint8_t* st = smem + s * STAGE_BYTES;
-      const int tile = t_lo + i;
-      if (tile < geo.NP) {
-        if (lane == 0) mbar_arrive_expect_tx(&full[s], PK_TX);
-        __syncwarp();
-        const size_t row0 = static_cast<size_t>(bh) * c.cap + static_cast<size_t>(tile) * PK;
-        if (lane == 0) bulk_g2s(st, c.kq + row0 * (D / 2), 4096, &full[s]);
-        else if (lane == 1) bulk_g2s(st + OFF_VC, c.vq + row0 * (D / 2), 4096, &full[s]);
-        else if (lane == 2) bulk_g2s(st + OFF_KS, c.ksz + row0 * 4, 1024, &full[s]);
-        else if (lane == 3) bulk_g2s(st + OFF_VS, c.vsz + row0 * 4, 1024, &full[s]);
-        else if (lane == 4)
-          bulk_g2s(st + OFF_MASK, c.vl_mask + static_cast<size_t>(bh) * (c.cap / 32) + 4 * (tile >> 1), 16, &full[s]);
-      } else {
-        // FP16 tile: one contiguous copy for K and one for V
-        const int j = tile - geo.NP - geo.NV;
-        const uint16_t* ksrc;
-        const uint16_t* vsrc;
-        uint32_t bytes = FT * 2 * D;
-        if (j < 0) {
-          const size_t row = static_cast<size_t>(bh) * c.vl_cap + static_cast<size_t>(tile - geo.NP) * FT;
-          ksrc = c.kf + row * D;
-          vsrc = c.vf + row * D;
-        } else if (j < geo.NR - 1) {
-          const size_t row = static_cast<size_t>(bh) * R + static_cast<size_t>(j) * FT;
-          ksrc = c.kr + row * D;
-          vsrc = c.vr + row * D;
-        } else {
-          ksrc = k_new + static_cast<size_t>(bh) * D;
-          vsrc = v_new + static_cast<size_t>(bh) * D;
-          bytes = 2 * D;
+    // one lane issues everything (1 bulk copy per packed page, 2 per FP16
+    // tile); its loop is kept short because it shares issue slots with the
+    // consumer warps
+    if (lane == 0) {
+      const size_t npg = static_cast<size_t>(c.cap / PK);
+      const uint8_t* page = c.pages + (static_cast<size_t>(bh) * npg + t_lo) * HQ_PAGE_BYTES;
+      const uint16_t* kf = c.kf + static_cast<size_t>(bh) * c.vl_cap * D;
+      const uint16_t* vf = c.vf + static_cast<size_t>(bh) * c.vl_cap * D;
+      const uint16_t* kr = c.kr + static_cast<size_t>(bh) * R * D;
+      const uint16_t* vr = c.vr + static_cast<size_t>(bh) * R * D;
+      int s = 0;
+      uint32_t ph = 1;  // flips to 0 when the ring first wraps: the wait at i = NSTAGES is for phase 0
+      for (int i = 0; i < ntile; ++i) {
+        if (i >= NSTAGES && !mbar_wait(&empty[s], ph, c.state)) {
+          s_timeout = 1;
+          break;
         }
-        if (lane == 0) {
+        s_issued[s] = i / NSTAGES + 1;
+        uint8_t* st = smem + s * STAGE_BYTES;
+        const int tile = t_lo + i;
+        if (tile < geo.NP) {
+          mbar_arrive_expect_tx(&full[s], PK_TX);
+          bulk_g2s(st, page, PK_TX, &full[s]);
+          page += HQ_PAGE_BYTES;
+        } else {
+          const int v = tile - geo.NP, j = v - geo.NV;
+          const uint16_t* ksrc = j < 0 ? kf + v * (FT * D) : (j < geo.NR - 1 ? kr + j * (FT * D) : k_new + bh * D);
+          const uint16_t* vsrc = j < 0 ? vf + v * (FT * D) : (j < geo.NR - 1 ? vr + j * (FT * D) : v_new + bh * D);
+          const uint32_t bytes = j == geo.NR - 1 ? 2 * D : FT * 2 * D;
           mbar_arrive_expect_tx(&full[s], 2 * bytes);
           bulk_g2s(st, ksrc, bytes, &full[s]);
           bulk_g2s(st + OFF_FV, vsrc, bytes, &full[s]);
+        }
+        if (++s == NSTAGES) {
+          s = 0;
+          ph ^= 1;
         }
       }
     }
@@ -538,48 +545,34 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
   __syncthreads();
   if (s_last || s_glast) fence_acq_rel_gpu();
   if (s_last) {
-    // log-sum-exp merge of the S partials of this (b, kv head): m and l of every
-    // split are fetched in parallel, the weights computed once, then each thread
-    // sums its outputs over the splits with independent loads in flight.
+    // log-sum-exp merge of the S partials of this (b, kv head), in one pass: each
+    // thread owns 4 output dims of one query and streams (m, l, O) of every
+    // split, 8 splits' loads in flight at a time, merging online
     const float* pb = parts + static_cast<size_t>(bh) * S * PART_FLOATS;
-    float* sm_m = reinterpret_cast<float*>(smem);      // [S][8]
-    float* sm_l = sm_m + S * 8;                        // [S][8]
-    float* sm_w = sm_l + S * 8;                        // [S][8] normalised weights
-    for (int i = threadIdx.x; i < S * 8; i += NTHREADS) {
-      sm_m[i] = __ldcg(pb + (i >> 3) * PART_FLOATS + (i & 7));
-      sm_l[i] = __ldcg(pb + (i >> 3) * PART_FLOATS + 8 + (i & 7));
-    }
-    __syncthreads();
-    if (threadIdx.x < 8) {
-      const int qc = threadIdx.x;
-      float mm = -INFINITY;
-      for (int sp = 0; sp < S; ++sp) mm = fmaxf(mm, sm_m[sp * 8 + qc]);
-      float ll = 0.f;
-      for (int sp = 0; sp < S; ++sp) {
-        const float ms = sm_m[sp * 8 + qc];
-        if (ms != -INFINITY) ll += sm_l[sp * 8 + qc] * ex2(ms - mm);
-      }
-      s_cm[qc] = mm;
-      s_cl[qc] = ll > 0.f ? 1.0f / ll : 0.f;
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < S * 8; i += NTHREADS) {
-      const float ms = sm_m[i];
-      sm_w[i] = ms == -INFINITY ? 0.f : ex2(ms - s_cm[i & 7]) * s_cl[i & 7];
-    }
-    __syncthreads();
-    for (int it = threadIdx.x; it < G * (D / 2); it += NTHREADS) {
-      const int qc = it / (D / 2), d2 = it % (D / 2);
-      const float2* src = reinterpret_cast<const float2*>(pb + 16 + qc * D) + d2;
-      float ax = 0.f, ay = 0.f;
+    for (int it = threadIdx.x; it < G * (D / 4); it += NTHREADS) {
+      const int qc = it / (D / 4), d4 = it % (D / 4);
+      const float4* src = reinterpret_cast<const float4*>(pb + 16 + qc * D) + d4;
+      float mrun = -INFINITY, lrun = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 8
       for (int sp = 0; sp < S; ++sp) {
-        const float2 o = __ldcg(src + sp * (PART_FLOATS / 2));
-        const float w = sm_w[sp * 8 + qc];
-        ax = fmaf(w, o.x, ax);
-        ay = fmaf(w, o.y, ay);
+        const float ms = __ldcg(pb + sp * PART_FLOATS + qc);
+        const float ls = __ldcg(pb + sp * PART_FLOATS + 8 + qc);
+        const float4 o = __ldcg(src + sp * (PART_FLOATS / 4));
+        const float mn = fmaxf(mrun, ms);
+        const float a = mrun == -INFINITY ? 0.f : ex2(mrun - mn);
+        const float w = ms == -INFINITY ? 0.f : ex2(ms - mn);
+        lrun = lrun * a + ls * w;
+        acc.x = acc.x * a + o.x * w;
+        acc.y = acc.y * a + o.y * w;
+        acc.z = acc.z * a + o.z * w;
+        acc.w = acc.w * a + o.w * w;
+        mrun = mn;
       }
-      reinterpret_cast<__half2*>(out + (static_cast<size_t>(b) * c.Hq + kvh * G + qc) * D)[d2] = __floats2half2_rn(ax, ay);
+      const float inv = lrun > 0.f ? 1.0f / lrun : 0.f;
+      __half2* dst = reinterpret_cast<__half2*>(out + (static_cast<size_t>(b) * c.Hq + kvh * G + qc) * D) + 2 * d4;
+      dst[0] = __floats2half2_rn(acc.x * inv, acc.y * inv);
+      dst[1] = __floats2half2_rn(acc.z * inv, acc.w * inv);
     }
     // every split of this head has consumed its tiles: append the new token to
     // the ring (slot T % R) and this group's queries to the query buffer
@@ -610,16 +603,28 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
 
 }  // namespace
 
-int decode_splits(const hq_cache& c, int sms) {
+// Launch shape: the wide CTA (one per SM) when every (b, kv head) can get at
+// least 4 of them, else 3 narrow CTAs per SM; never more than one wave.
+struct DecodeShape {
+  int S;      // splits per (b, kv head)
+  bool wide;
+};
+
+DecodeShape decode_shape(const hq_cache& c, int sms) {
   const int units = c.B * c.Hkv;
   const int nt_max = c.cap / PK + c.vl_cap / FT + ring_len(c.W) / FT + 1;
-  int s = (3 * sms) / units;  // one wave: 3 CTAs per SM
-  const int cap_s = (nt_max + 3) / 4;
+  DecodeShape d;
+  d.wide = sms / units >= 4;
+  int s = d.wide ? sms / units : (3 * sms) / units;
+  const int cap_s = d.wide ? (nt_max + 8) / 9 : (nt_max + 2) / 3;  // at least ~one tile per consumer warp
   if (s > cap_s) s = cap_s;
   if (s > 64) s = 64;
   if (s < 1) s = 1;
-  return s;
+  d.S = s;
+  return d;
 }
+
+int decode_splits(const hq_cache& c, int sms) { return decode_shape(c, sms).S; }
 
 // counters: [0] grid ticket, [1 + b*Hkv + h] split tickets; zero between calls
 size_t decode_counter_bytes(const hq_cache& c) { return ((4ull * (1 + c.B * c.Hkv) + 255) / 256) * 256; }
@@ -631,20 +636,28 @@ size_t decode_workspace(const hq_cache& c, int sms) {
 
 hq_status launch_decode(const hq_cache& c, const uint16_t* q, const uint16_t* kn, const uint16_t* vn, uint16_t* out,
                         float sm_scale, void* ws, int sms, cudaStream_t st) {
-  const int S = decode_splits(c, sms);
-  const int smem = NSTAGES * STAGE_BYTES;
+  const DecodeShape shp = decode_shape(c, sms);
+  const int nc = shp.wide ? NC_WIDE : NC_NARROW;
+  const int smem = 2 * nc * STAGE_BYTES;
   int dev = 0;
   cudaGetDevice(&dev);
   static bool attr_done[64] = {};
   if (dev >= 64 || !attr_done[dev]) {
-    if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(decode_kernel<NC_WIDE, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             2 * NC_WIDE * STAGE_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(decode_kernel<NC_NARROW, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             2 * NC_NARROW * STAGE_BYTES) != cudaSuccess)
       return HQ_ERR_CUDA;
     if (dev < 64) attr_done[dev] = true;
   }
   unsigned int* tickets = reinterpret_cast<unsigned int*>(ws);
   float* parts = reinterpret_cast<float*>(static_cast<char*>(ws) + decode_counter_bytes(c));
-  dim3 grid(S, c.Hkv, c.B);
-  decode_kernel<<<grid, NTHREADS, smem, st>>>(c, q, kn, vn, out, sm_scale * LOG2E, S, parts, tickets);
+  dim3 grid(shp.S, c.Hkv, c.B);
+  if (shp.wide)
+    decode_kernel<NC_WIDE, 1><<<grid, (NC_WIDE + 1) * 32, smem, st>>>(c, q, kn, vn, out, sm_scale * LOG2E, shp.S, parts, tickets);
+  else
+    decode_kernel<NC_NARROW, 3><<<grid, (NC_NARROW + 1) * 32, smem, st>>>(c, q, kn, vn, out, sm_scale * LOG2E, shp.S, parts,
+                                                                          tickets);
   return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 

@@ -57,8 +57,7 @@ hq_status hq_cache_validate(const hq_cache* c) {
   if (c->W < 0 || c->rho_bp < 0 || c->rho_bp > 10000) return HQ_ERR_INVALID;
   if (c->cap <= 0 || c->cap % 128 != 0 || c->vl_cap <= 0 || c->vl_cap % 16 != 0) return HQ_ERR_INVALID;
   if (c->B > 65535 || c->Hkv > 65535) return HQ_ERR_UNSUPPORTED;
-  const void* ptrs[] = {c->kq, c->vq, c->ksz, c->vsz, c->kf, c->vf, c->vl_pos, c->vl_mask,
-                        c->kr, c->vr, c->qbuf, c->vl_sel, c->state};
+  const void* ptrs[] = {c->pages, c->kf, c->vf, c->vl_pos, c->kr, c->vr, c->qbuf, c->vl_sel, c->state};
   for (const void* p : ptrs)
     if (!aligned16(p)) return HQ_ERR_INVALID;
   return HQ_OK;
@@ -83,7 +82,8 @@ hq_status hq_cache_reset(const hq_cache* c, hq_stream_t stream) {
   if (s != HQ_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(c->state, 0, HQ_STATE_WORDS * sizeof(int32_t), st) != cudaSuccess) return HQ_ERR_CUDA;
-  if (cudaMemsetAsync(c->vl_mask, 0, static_cast<size_t>(c->B) * c->Hkv * (c->cap / 32) * 4, st) != cudaSuccess)
+  if (cudaMemset2DAsync(c->pages + HQ_PAGE_VLMASK, HQ_PAGE_BYTES, 0, 8,
+                        static_cast<size_t>(c->B) * c->Hkv * (c->cap / HQ_PAGE_POSITIONS), st) != cudaSuccess)
     return HQ_ERR_CUDA;
   return HQ_OK;
 }

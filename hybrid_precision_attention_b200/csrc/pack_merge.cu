@@ -90,9 +90,8 @@ __global__ void pack_rows_kernel(hq_cache c, const uint16_t* __restrict__ kd, co
     } else {
       src = (which ? c.vr : c.kr) + (bh * d.R + (p % d.R)) * D;
     }
-    uint8_t* codes = (which ? c.vq : c.kq) + (bh * d.cap + p) * (D / 2);
-    uint32_t* sz = (which ? c.vsz : c.ksz) + (bh * d.cap + p) * (D / HQ_GROUP);
-    pack_row_warp(src, codes, sz, lane);
+    uint8_t* page = page_of(c, bh, p);
+    pack_row_warp(src, row_codes(page, which, p), row_sz(page, which, p), lane);
   }
 }
 
@@ -157,8 +156,9 @@ __global__ void vl_gather_kernel(hq_cache c, uint16_t* __restrict__ wsk, uint16_
     } else {
       // promoted packed position: fp16(zero + q * scale); q * scale is exact in
       // float64 and the sum is rounded once, then once more to fp16 (RN).
-      const uint8_t* codes = (which ? c.vq : c.kq) + (bh * d.cap + p) * (D / 2);
-      const uint32_t szw = (which ? c.vsz : c.ksz)[(bh * d.cap + p) * (D / HQ_GROUP) + (lane >> 3)];
+      uint8_t* page = page_of(c, bh, p);
+      const uint8_t* codes = row_codes(page, which, p);
+      const uint32_t szw = row_sz(page, which, p)[lane >> 3];
       const double sc = static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(szw & 0xFFFFu))));
       const double ze = static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(szw >> 16))));
       const uint32_t two = reinterpret_cast<const uint16_t*>(codes)[lane];
@@ -181,7 +181,7 @@ __global__ void vl_gather_kernel(hq_cache c, uint16_t* __restrict__ wsk, uint16_
     const long long bh = i / n_vl;
     const int r = static_cast<int>(i % n_vl);
     const int p = c.vl_pos[bh * d.vl_cap + r];
-    atomicAnd(c.vl_mask + bh * (d.cap / 32) + (p >> 5), ~(1u << (p & 31)));
+    atomicAnd(page_mask(page_of(c, bh, p)) + ((p & 63) >> 5), ~(1u << (p & 31)));
   }
 }
 
@@ -212,7 +212,7 @@ __global__ void vl_install_kernel(hq_cache c, const uint16_t* __restrict__ srck,
     reinterpret_cast<uint4*>(t)[ch] = reinterpret_cast<const uint4*>(s)[ch];
     if (ch == 0 && which == 0) {
       c.vl_pos[bh * d.vl_cap + row] = p;
-      atomicOr(c.vl_mask + bh * (d.cap / 32) + (p >> 5), 1u << (p & 31));
+      atomicOr(page_mask(page_of(c, bh, p)) + ((p & 63) >> 5), 1u << (p & 31));
     }
   }
   // state update by the last block (every block has read state above)
@@ -254,7 +254,9 @@ hq_status launch_pack_merge(const hq_cache& c, const uint16_t* kd, const uint16_
   uint16_t* wsk = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + 256);
   uint16_t* wsv = wsk + static_cast<size_t>(c.B) * c.Hkv * c.vl_cap * D;
   if (init) {
-    if (cudaMemsetAsync(c.vl_mask, 0, static_cast<size_t>(c.B) * c.Hkv * (c.cap / 32) * 4, st) != cudaSuccess) return HQ_ERR_CUDA;
+    if (cudaMemset2DAsync(c.pages + HQ_PAGE_VLMASK, HQ_PAGE_BYTES, 0, 8,
+                          static_cast<size_t>(c.B) * c.Hkv * (c.cap / HQ_PAGE_POSITIONS), st) != cudaSuccess)
+      return HQ_ERR_CUDA;
   }
   pack_rows_kernel<<<sms * 4, threads, 0, st>>>(c, kd, vd, L, init);
   if (init) {

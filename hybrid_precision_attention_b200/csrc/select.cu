@@ -96,13 +96,13 @@ __device__ void load_keys(const SelArgs& a, const SelGeo& g, int bh, int j0, uin
         v = reinterpret_cast<const uint2*>(a.k_dense + (static_cast<size_t>(bh) * a.L + p) * D)[lane];
       } else if (p >= g.n_packed) {
         v = reinterpret_cast<const uint2*>(c.kr + (static_cast<size_t>(bh) * R + (p % R)) * D)[lane];
-      } else if ((c.vl_mask[static_cast<size_t>(bh) * (c.cap / 32) + (p >> 5)] >> (p & 31)) & 1u) {
+      } else if ((page_mask(page_of(c, bh, p))[(p & 63) >> 5] >> (p & 31)) & 1u) {
         const int idx = find_sorted(c.vl_pos + static_cast<size_t>(bh) * c.vl_cap, g.n_vl, p);
         if (idx >= 0) v = reinterpret_cast<const uint2*>(c.kf + (static_cast<size_t>(bh) * c.vl_cap + idx) * D)[lane];
       } else {
-        const size_t row = static_cast<size_t>(bh) * c.cap + p;
-        const uint32_t two = reinterpret_cast<const uint16_t*>(c.kq + row * (D / 2))[lane];
-        const uint32_t szw = c.ksz[row * 4 + (lane >> 3)];
+        uint8_t* page = page_of(c, bh, p);
+        const uint32_t two = reinterpret_cast<const uint16_t*>(row_codes(page, 0, p))[lane];
+        const uint32_t szw = row_sz(page, 0, p)[lane >> 3];
         const uint32_t s2 = prmt(szw, szw, 0x1010), z2 = prmt(szw, szw, 0x3232);
         // nibbles of byte 0 -> dims 4l, 4l+1 ; byte 1 -> dims 4l+2, 4l+3
         const uint32_t x0 = prmt(two, 0u, 0x4040);   // byte0 at bits 0..7 and 16..23

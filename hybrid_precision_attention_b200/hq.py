@@ -11,6 +11,7 @@ from __future__ import annotations
 import ctypes
 import os
 
+import numpy as np
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -19,6 +20,9 @@ LIB_PATH = os.path.join(_PKG, "libhq.so")
 HQ_HEAD_DIM = 128
 HQ_STAGE = 64
 HQ_QBUF = 64
+PAGE_POSITIONS = 64
+PAGE_BYTES = 10304
+PAGE_KCODES, PAGE_VCODES, PAGE_KSZ, PAGE_VSZ, PAGE_VLMASK = 0, 4096, 8192, 9216, 10240
 STATE_T, STATE_NPACKED, STATE_NVL, STATE_NQ, STATE_KSEL, STATE_ERR = range(6)
 STATE_WORDS = 8
 OP_SELECT, OP_MERGE, OP_DECODE = 0, 1, 2
@@ -37,7 +41,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 class HqCacheStruct(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("B", "Hq", "Hkv", "D", "W", "rho_bp", "cap", "vl_cap")] + [
         (n, ctypes.c_void_p)
-        for n in ("kq", "vq", "ksz", "vsz", "kf", "vf", "vl_pos", "vl_mask", "kr", "vr", "qbuf", "vl_sel", "state")
+        for n in ("pages", "kf", "vf", "vl_pos", "kr", "vr", "qbuf", "vl_sel", "state")
     ]
 
 
@@ -117,22 +121,17 @@ class HybridCache:
         self.R = ((W + HQ_STAGE + 15) // 16) * 16   # HQ_RING_LEN(W)
         dev = torch.device(device)
         z = lambda shape, dt: torch.zeros(shape, dtype=dt, device=dev)
-        self.kq = z((B, Hkv, cap, D // 2), torch.uint8)
-        self.vq = z((B, Hkv, cap, D // 2), torch.uint8)
-        self.ksz = z((B, Hkv, cap, D // 32), torch.int32)
-        self.vsz = z((B, Hkv, cap, D // 32), torch.int32)
+        self.pages = z((B, Hkv, cap // PAGE_POSITIONS, PAGE_BYTES), torch.uint8)
         self.kf = z((B, Hkv, vl_cap, D), torch.float16)
         self.vf = z((B, Hkv, vl_cap, D), torch.float16)
         self.vl_pos = z((B, Hkv, vl_cap), torch.int32)
-        self.vl_mask = z((B, Hkv, cap // 32), torch.int32)
         self.kr = z((B, Hkv, self.R, D), torch.float16)
         self.vr = z((B, Hkv, self.R, D), torch.float16)
         self.qbuf = z((B, Hq, HQ_QBUF, D), torch.float16)
         self.vl_sel = z((B, Hkv, vl_cap), torch.int32)
         self.state_t = z((STATE_WORDS,), torch.int32)
         self.c = HqCacheStruct(B, Hq, Hkv, D, W, rho_bp, cap, vl_cap, *[t.data_ptr() for t in (
-            self.kq, self.vq, self.ksz, self.vsz, self.kf, self.vf, self.vl_pos, self.vl_mask, self.kr, self.vr,
-            self.qbuf, self.vl_sel, self.state_t)])
+            self.pages, self.kf, self.vf, self.vl_pos, self.kr, self.vr, self.qbuf, self.vl_sel, self.state_t)])
         _check(_lib.hq_cache_validate(ctypes.byref(self.c)), "hq_cache_validate")
         self._ws = {}
 
@@ -142,7 +141,7 @@ class HybridCache:
             raise HqError("hq_workspace_bytes returned 0")
         w = self._ws.get(op)
         if w is None or w.numel() < n:
-            w = torch.zeros(n, dtype=torch.uint8, device=self.kq.device)
+            w = torch.zeros(n, dtype=torch.uint8, device=self.pages.device)
             self._ws[op] = w
         return w
 
@@ -152,9 +151,21 @@ class HybridCache:
                 "k_sel": s[STATE_KSEL], "err": s[STATE_ERR]}
 
     def nbytes(self) -> int:
-        return sum(t.numel() * t.element_size() for t in (self.kq, self.vq, self.ksz, self.vsz, self.kf, self.vf,
-                                                          self.vl_pos, self.vl_mask, self.kr, self.vr, self.qbuf,
-                                                          self.vl_sel, self.state_t))
+        return sum(t.numel() * t.element_size() for t in (self.pages, self.kf, self.vf, self.vl_pos, self.kr, self.vr,
+                                                          self.qbuf, self.vl_sel, self.state_t))
+
+    def packed(self) -> dict:
+        """The K4V4 store by position (host copies): codes kq/vq uint8 [B,Hkv,cap,D/2],
+        scale/zero words ksz/vsz uint32 [B,Hkv,cap,D/32], VL bitmap vl_bits bool [B,Hkv,cap]."""
+        pg = self.pages.cpu().numpy()
+        B, H, npg, _ = pg.shape
+        D = self.D
+        take = lambda off, width: pg[..., off:off + 64 * width].reshape(B, H, npg * 64, width)
+        m = pg[..., PAGE_VLMASK:PAGE_VLMASK + 8].copy()
+        bits = np.unpackbits(m, axis=-1, bitorder="little").reshape(B, H, npg * 64).astype(bool)
+        return {"kq": take(PAGE_KCODES, D // 2), "vq": take(PAGE_VCODES, D // 2),
+                "ksz": take(PAGE_KSZ, 16).copy().view(np.uint32), "vsz": take(PAGE_VSZ, 16).copy().view(np.uint32),
+                "vl_bits": bits}
 
 
 # ----------------------------------------------------------------------------- entry points

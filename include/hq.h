@@ -51,12 +51,20 @@
 extern "C" {
 #endif
 
-#define HQ_ABI_VERSION 1
+#define HQ_ABI_VERSION 2
 #define HQ_HEAD_DIM 128       /* D: the only head size built */
 #define HQ_GROUP 32           /* K4V4 group length along D */
 #define HQ_STAGE 64           /* staged tokens before a merge = reselection period */
 #define HQ_QBUF 64            /* buffered queries kept for the column-mass estimate */
 #define HQ_MAX_GQA 8          /* query heads per kv head supported by the decode kernel */
+/* K4V4 store page: 64 positions of one (batch, kv head), one contiguous block */
+#define HQ_PAGE_POSITIONS 64
+#define HQ_PAGE_BYTES 10304
+#define HQ_PAGE_KCODES 0        /* [64][D/2] K codes, row r = position 64 j + r */
+#define HQ_PAGE_VCODES 4096     /* [64][D/2] V codes */
+#define HQ_PAGE_KSZ 8192        /* [64][D/32] uint32 K (scale bits | zero bits << 16) */
+#define HQ_PAGE_VSZ 9216        /* [64][D/32] uint32 V (scale | zero << 16) */
+#define HQ_PAGE_VLMASK 10240    /* 2 uint32: bit r of word r/32 <=> position 64 j + r is a vertical line */
 /* FP16 ring length for a window W: W + HQ_STAGE rounded up to a multiple of 16 */
 #define HQ_RING_LEN(W) ((((W) + HQ_STAGE) + 15) / 16 * 16)
 
@@ -99,11 +107,13 @@ enum {
  * device memory laid out as stated ([..] = row-major shape, innermost last).
  * R = HQ_RING_LEN(W) is the FP16 ring length (W + HQ_STAGE rounded up to 16).
  *
- *   kq, vq    uint8  [B, Hkv, cap, D/2]   K4V4 codes, dense by position
- *   ksz, vsz  uint32 [B, Hkv, cap, D/32]  per group: scale fp16 bits | zero fp16 bits << 16
+ *   pages     uint8  [B, Hkv, cap/64, HQ_PAGE_BYTES]  the K4V4 store, one page per 64
+ *             positions (layout HQ_PAGE_*): codes of both K and V, their per-group
+ *             (scale, zero) words and the VL bitmap of the page's positions, so
+ *             that one contiguous copy brings a whole page on chip; bytes
+ *             10248 .. HQ_PAGE_BYTES-1 are padding
  *   kf, vf    fp16   [B, Hkv, vl_cap, D]  VL store rows, in vl_pos order
  *   vl_pos    int32  [B, Hkv, vl_cap]     VL positions, ascending (first n_vl valid)
- *   vl_mask   uint32 [B, Hkv, cap/32]     bit p set <=> position p is in the VL store
  *   kr, vr    fp16   [B, Hkv, R, D]       recent window + staging; position p at slot p % R
  *   qbuf      fp16   [B, Hq, HQ_QBUF, D]  buffered decode queries; position p at slot p % HQ_QBUF
  *   vl_sel    int32  [B, Hkv, vl_cap]     output of hq_select_vlines, input of hq_pack_merge
@@ -119,14 +129,10 @@ enum {
 typedef struct hq_cache {
   int32_t B, Hq, Hkv, D;
   int32_t W, rho_bp, cap, vl_cap;
-  uint8_t* kq;
-  uint8_t* vq;
-  uint32_t* ksz;
-  uint32_t* vsz;
+  uint8_t* pages;
   uint16_t* kf;
   uint16_t* vf;
   int32_t* vl_pos;
-  uint32_t* vl_mask;
   uint16_t* kr;
   uint16_t* vr;
   uint16_t* qbuf;
@@ -153,7 +159,7 @@ HQ_API hq_status hq_cache_validate(const hq_cache* c);
 HQ_API size_t hq_workspace_bytes(const hq_cache* c, int32_t op, int32_t L);
 
 /*
- * Reset the cache to empty: state words to 0 and the VL bitmap cleared.
+ * Reset the cache to empty: state words to 0 and the VL bitmap of every page cleared.
  */
 HQ_API hq_status hq_cache_reset(const hq_cache* c, hq_stream_t stream);
 

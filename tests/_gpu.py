@@ -116,27 +116,27 @@ class Pair:
         np_ = self.r.n_packed
         g = self.g
         assert g.state()["n_packed"] == np_
-        kq = g.kq.cpu().numpy()[:, :, :np_]
-        vq = g.vq.cpu().numpy()[:, :, :np_]
+        pk = g.packed()
+        kq = pk["kq"][:, :, :np_]
+        vq = pk["vq"][:, :, :np_]
         assert np.array_equal(kq, self.r.kq[:, :, :np_]), "K codes differ"
         assert np.array_equal(vq, self.r.vq[:, :, :np_]), "V codes differ"
-        ksz = g.ksz.cpu().numpy().view(np.uint32)[:, :, :np_]
-        vsz = g.vsz.cpu().numpy().view(np.uint32)[:, :, :np_]
+        ksz = pk["ksz"][:, :, :np_]
+        vsz = pk["vsz"][:, :, :np_]
         assert np.array_equal(ksz, sz_words(self.r.ks[:, :, :np_], self.r.kz[:, :, :np_])), "K scale/zero differ"
         assert np.array_equal(vsz, sz_words(self.r.vs[:, :, :np_], self.r.vz[:, :, :np_])), "V scale/zero differ"
         nvl = g.state()["n_vl"]
         kf = g.kf.cpu().numpy()
         vf = g.vf.cpu().numpy()
         pos = g.vl_pos.cpu().numpy()
-        mask = g.vl_mask.cpu().numpy().view(np.uint32)
+        bits_all = pk["vl_bits"]
         for b in range(self.B):
             for h in range(self.Hkv):
                 assert nvl == len(self.r.vl[b][h])
                 assert np.array_equal(pos[b, h, :nvl], self.r.vl[b][h])
                 assert np.array_equal(kf[b, h, :nvl].view(np.uint16), self.r.kf[b][h].view(np.uint16)), "VL K rows differ"
                 assert np.array_equal(vf[b, h, :nvl].view(np.uint16), self.r.vf[b][h].view(np.uint16)), "VL V rows differ"
-                bits = np.unpackbits(mask[b, h].view(np.uint8), bitorder="little")
-                assert np.array_equal(np.nonzero(bits)[0], self.r.vl[b][h]), "VL bitmap differs"
+                assert np.array_equal(np.nonzero(bits_all[b, h])[0], self.r.vl[b][h]), "VL bitmap differs"
 
     def decode(self, q, k, v):
         H = hq()

@@ -27,7 +27,7 @@ def test_library_exports_every_declared_symbol():
     missing = [n for n in _declared() if not hasattr(lib, n)]
     assert not missing, missing
     lib.hq_abi_version.restype = ctypes.c_int32
-    assert lib.hq_abi_version() == 1
+    assert lib.hq_abi_version() == 2
     lib.hq_status_str.restype = ctypes.c_char_p
     assert lib.hq_status_str(0) == b"ok"
 
@@ -41,11 +41,11 @@ def test_host_validation_without_gpu():
     from hybrid_precision_attention_b200.hq import HqCacheStruct
     buf = ctypes.create_string_buffer(4096 + 16)
     base = (ctypes.addressof(buf) + 15) & ~15
-    good = HqCacheStruct(1, 32, 8, 128, 128, 500, 1024, 64, *([base] * 13))
+    good = HqCacheStruct(1, 32, 8, 128, 128, 500, 1024, 64, *([base] * 9))
     lib.hq_cache_validate.restype = ctypes.c_int32
     assert lib.hq_cache_validate(ctypes.byref(good)) == 0
     for field, val, want in (("D", 64, 2), ("Hq", 30, 1), ("cap", 1000, 1), ("vl_cap", 20, 1), ("rho_bp", 10001, 1),
-                             ("kq", base + 4, 1), ("state", 0, 1), ("Hq", 80, 2)):
+                             ("pages", base + 4, 1), ("state", 0, 1), ("Hq", 80, 2)):
         bad = HqCacheStruct.from_buffer_copy(good)
         setattr(bad, field, val)
         assert lib.hq_cache_validate(ctypes.byref(bad)) == want, field

@@ -18,6 +18,7 @@ pytestmark = pytest.mark.gpu
     (1, 4, 2, 200, 0, 0),           # strict 4-bit: no window, no lines
     (1, 4, 1, 150, 200, 500),       # window longer than the prefix: nothing packed
     (1, 4, 1, 70, 16, 10000),       # every non-window position a line
+    (8, 32, 8, 300, 64, 500),       # 64 (b, kv head) units: the narrow CTA shape (3 per SM)
 ])
 def test_prefix_init_and_decode(B, Hq, Hkv, L, W, rho):
     p = Pair(B, Hq, Hkv, L, W, rho, cap=L + 200, seed=L)
