@@ -1,0 +1,114 @@
+"""GPU parity of the hybrid-precision causal prefill (tcgen05 kernel) against
+the float64 oracle, through the C ABI.
+
+Tolerance: rel-L2 <= 2e-2 of the whole output (or of the sampled rows).  Both
+sides use the same e4m3 codes (checked bit-exactly below); the kernel rounds P
+to fp16 and stores V's e4m3 value times its block scale as fp16, each a
+relative error near 2^-11, far inside the bound.
+"""
+import numpy as np
+import pytest
+import torch
+
+from hybrid_precision_attention_b200 import synth
+from oracle import attention as oatt, formats, select as osel
+from tests._gpu import dev, hq
+
+pytestmark = pytest.mark.gpu
+PF_RELL2 = 2e-2
+SM = 1 / np.sqrt(128)
+
+
+def _vl_sets(lay_k, Q, W, rho_bp, G):
+    """Vertical lines from the column mass of the last 64 queries (oracle selection)."""
+    B, Hkv, L, D = lay_k.shape
+    n = max(L - W, 0)
+    nq = min(64, L)
+    qpos = np.tile(np.arange(L - nq, L), G)
+    out = []
+    for b in range(B):
+        row = []
+        for h in range(Hkv):
+            qs = Q[b, h * G:(h + 1) * G, L - nq:].reshape(-1, D).astype(np.float64)
+            idx, _ = osel.select_vlines(lay_k[b, h].astype(np.float64), qs, qpos, n, rho_bp, SM)
+            row.append(idx)
+        out.append(row)
+    return out
+
+
+def _vl_tensor(vl, B, Hkv):
+    stride = max(16, max((len(v) for r in vl for v in r), default=0))
+    t = np.zeros((B, Hkv, stride), np.int32)
+    n = len(vl[0][0])
+    for b in range(B):
+        for h in range(Hkv):
+            assert len(vl[b][h]) == n
+            t[b, h, :n] = vl[b][h]
+    return t, n
+
+
+def _run(B, Hq, Hkv, L, W, rho_bp, seed, rows=None, heads=None):
+    H = hq()
+    lay = synth.planted_layer(seed, B, Hq, Hkv, L)
+    Q = synth.full_queries(seed, B, Hq, Hkv, L)
+    G = Hq // Hkv
+    vl = _vl_sets(lay.k, Q, W, rho_bp, G)
+    vlt, n_vl = _vl_tensor(vl, B, Hkv)
+    out = H.hq_prefill_attn(dev(Q), dev(lay.k), dev(lay.v), dev(vlt), n_vl, W)
+    torch.cuda.synchronize()
+    got = out.float().cpu().numpy().astype(np.float64)
+    ref = oatt.prefill_ref(Q, lay.k, lay.v, vl, W, SM, rows=rows, heads=heads)
+    return got, ref
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,L,W,rho", [
+    (1, 4, 1, 128, 128, 500),     # one tile: window only
+    (1, 4, 1, 300, 64, 500),      # ragged tiles, FP8 + VL + window
+    (1, 8, 2, 1000, 128, 500),    # GQA 4, several FP8 tiles
+    (2, 2, 2, 520, 100, 700),     # GQA 1, batch 2, window not a tile multiple
+    (1, 8, 1, 400, 0, 500),       # no window: FP8 and VL only
+    (1, 4, 1, 200, 500, 500),     # window longer than the prompt: plain FP16 causal
+    (1, 4, 1, 384, 32, 0),        # no vertical lines
+])
+def test_prefill_matches_oracle(B, Hq, Hkv, L, W, rho):
+    got, ref = _run(B, Hq, Hkv, L, W, rho, seed=L + W)
+    assert np.all(np.isfinite(got))
+    for (b, h), r in ref.items():
+        g = got[b, h]
+        rel = np.linalg.norm(g - r) / np.linalg.norm(r)
+        assert rel <= PF_RELL2, (b, h, rel)
+
+
+def test_prefill_fp8_codes_match_oracle():
+    """The pre-pass e4m3 codes of Q (first region of the workspace after the error word) are bit-exact."""
+    H = hq()
+    B, Hq, Hkv, L = 1, 4, 1, 300
+    lay = synth.planted_layer(3, B, Hq, Hkv, L)
+    Q = synth.full_queries(3, B, Hq, Hkv, L)
+    vlt = np.zeros((B, Hkv, 16), np.int32)
+    ws = torch.zeros(H.hq_prefill_workspace_bytes(B, Hq, Hkv, L), dtype=torch.uint8, device="cuda")
+    H.hq_prefill_attn(dev(Q), dev(lay.k), dev(lay.v), dev(vlt), 0, 64, ws=ws)
+    torch.cuda.synchronize()
+    Lp = 384
+    q8 = ws[1024:1024 + B * Hq * Lp * 128].cpu().numpy().reshape(B, Hq, Lp, 128)[:, :, :L]
+    # decode the e4m3 bytes with the OCP bit layout and compare to the oracle's rounding
+    codes = q8.astype(np.int64)
+    sign = np.where(codes & 0x80, -1.0, 1.0)
+    e = (codes >> 3) & 0xF
+    m = codes & 0x7
+    val = sign * np.where(e == 0, m / 8.0 * 2.0 ** -6, (1 + m / 8.0) * 2.0 ** (e - 7))
+    want = formats.fp8_quantize(Q, formats.fp8_block_scales(Q))
+    assert np.array_equal(val, want)
+    assert ws[:4].cpu().numpy().view(np.uint32)[0] == 0
+
+
+@pytest.mark.slow
+def test_prefill_full_size_32k():
+    """The 32K prefill layer (B=1, Hq=32, Hkv=8): sampled rows of a few heads against the oracle."""
+    L = 32768
+    rows = np.unique(np.concatenate([np.arange(0, 64, 7), np.linspace(64, L - 1, 40).astype(np.int64), [L - 1]]))
+    got, ref = _run(1, 32, 8, L, 128, 500, seed=0, rows=rows, heads=[(0, 0), (0, 13), (0, 31)])
+    for (b, h), r in ref.items():
+        g = got[b, h, rows]
+        rel = np.linalg.norm(g - r) / np.linalg.norm(r)
+        assert rel <= PF_RELL2, (b, h, rel)
