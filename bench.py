@@ -82,6 +82,66 @@ def load_peaks():
     return 6650.0, "fallback"
 
 
+def load_bf16_peak():
+    """Dense bf16 tensor peak (TFLOP/s): the burst figure, for a kernel timed on its own."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        return float(json.load(open(p))["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
+PF_L, PF_HQ, PF_HKV = 32768, 32, 8
+
+
+def prefill_flops(L, Hq, D=128):
+    """Algorithmic FLOPs of causal attention: 2 GEMMs x 2 flops x D x Hq x L(L+1)/2."""
+    return 4.0 * D * Hq * L * (L + 1) / 2
+
+
+def run_prefill(dev, reps=5, warmup=2):
+    """Time hq_prefill_attn on the 32K layer (B=1, Hq=32, Hkv=8, W=128, 5 % vertical lines chosen
+    from the column mass of the last 64 queries); returns the JSON object of the prefill leg."""
+    import torch
+    from hybrid_precision_attention_b200 import hq, synth
+    lay = synth.planted_layer(0, 1, PF_HQ, PF_HKV, PF_L)
+    Q = synth.full_queries(0, 1, PF_HQ, PF_HKV, PF_L)
+    q_d = torch.from_numpy(Q).to(dev)
+    k_d, v_d = torch.from_numpy(lay.k).to(dev), torch.from_numpy(lay.v).to(dev)
+    # vertical lines from the prompt's own last 64 queries
+    c = hq.HybridCache(1, PF_HQ, PF_HKV, PF_L, W, RHO_BP, device=dev)
+    hq.hq_select_vlines(c, k_d, q_d[:, :, PF_L - 64:].contiguous())
+    torch.cuda.synchronize()
+    n_vl = c.state()["k_sel"]
+    vl = c.vl_sel
+    out = torch.empty_like(q_d)
+    ws = torch.empty(hq.hq_prefill_workspace_bytes(1, PF_HQ, PF_HKV, PF_L), dtype=torch.uint8, device=dev)
+    for _ in range(warmup):
+        hq.hq_prefill_attn(q_d, k_d, v_d, vl, n_vl, W, out=out, ws=ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        hq.hq_prefill_attn(q_d, k_d, v_d, vl, n_vl, W, out=out, ws=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    err = int(ws[:4].cpu().numpy().view(np.uint32)[0])
+    assert err == 0, err
+    ms = e0.elapsed_time(e1) / reps
+    flops = prefill_flops(PF_L, PF_HQ)
+    tflops = flops / (ms * 1e-3) / 1e12
+    bf16, kind = load_bf16_peak()
+    fp8 = 2.0 * bf16
+    mixed = 1.0 / (0.5 / fp8 + 0.5 / bf16)
+    return {"workload": f"causal hybrid prefill, B=1, L=32768, Hq=32, Hkv=8, D=128, W=128, rho=5% ({n_vl} lines per kv head)",
+            "ms": ms, "tflops": tflops, "calls": reps,
+            "roofline": {"kernel": "prefill (pre-pass + prefill_kernel)", "bound": "tensor", "achieved": tflops,
+                         "peak": fp8, "unit": "TFLOP/s", "frac": tflops / fp8, "traffic": None,
+                         "peak_kind": f"{kind} bf16 x 2 (nominal fp8/bf16 ratio)",
+                         "mixed_ceiling": mixed,
+                         "note": "QK of quantised tiles on e4m3 (fp8 rate), P.V on f16 (bf16 rate): half the flops at "
+                                 "each rate, so the ceiling of this mix is the mixed_ceiling figure"}}
+
+
 def decode_traffic_record():
     """DRAM bytes per decode launch from the committed ncu summary, if it matches the current kernel source."""
     src = open(os.path.join(ROOT, "hybrid_precision_attention_b200", "csrc", "decode.cu"), "rb").read()
@@ -352,6 +412,10 @@ def run_ours(args, rank, world, local_rank):
                "d2h_bytes_per_step": PERIOD * COPIES * out.numel() * 2,
                "steps": n_e2e, "api": "hq_decode_attn / hq_select_vlines / hq_pack_merge via the Python binding, eager"}
 
+    prefill = None
+    if not args.no_prefill:
+        prefill = run_prefill(dev)
+
     if rank != 0:
         return
     cpu = None
@@ -369,7 +433,8 @@ def run_ours(args, rank, world, local_rank):
                        "rho": RHO_BP / 10000, "layer_copies": COPIES, "decode_tokens_per_step": PERIOD,
                        "l2": f"{COPIES} rotating layer copies, {COPIES * caches[0].nbytes() / 1e6:.0f} MB working set > 126 MB L2",
                        "parallelism": f"replicas x{world}"},
-            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "prefill": prefill,
+            "gpu_launches": launches_per_step * args.steps,
             "clocks": sampler.summary()}
     print(json.dumps(line), flush=True)
 
@@ -394,6 +459,25 @@ def profile_decode():
     print("profile-decode ok", st)
 
 
+def profile_prefill():
+    """Small case for ncu captures: the hybrid prefill at L=8192 (B=1, Hq=32, Hkv=8), three calls."""
+    import torch
+    from hybrid_precision_attention_b200 import hq, synth
+    Lp = 8192
+    lay = synth.planted_layer(2, 1, PF_HQ, PF_HKV, Lp)
+    Q = torch.from_numpy(synth.full_queries(2, 1, PF_HQ, PF_HKV, Lp)).cuda()
+    k, v = torch.from_numpy(lay.k).cuda(), torch.from_numpy(lay.v).cuda()
+    c = hq.HybridCache(1, PF_HQ, PF_HKV, Lp, W, RHO_BP)
+    hq.hq_select_vlines(c, k, Q[:, :, Lp - 64:].contiguous())
+    torch.cuda.synchronize()
+    ws = torch.empty(hq.hq_prefill_workspace_bytes(1, PF_HQ, PF_HKV, Lp), dtype=torch.uint8, device="cuda")
+    for _ in range(3):
+        hq.hq_prefill_attn(Q, k, v, c.vl_sel, c.state()["k_sel"], W, ws=ws)
+    torch.cuda.synchronize()
+    assert int(ws[:4].cpu().numpy().view(np.uint32)[0]) == 0
+    print("profile-prefill ok")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -403,10 +487,15 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--profile-decode", action="store_true", help="small case for ncu: 4 decode steps of one 32K layer")
+    ap.add_argument("--profile-prefill", action="store_true", help="small case for ncu: 3 prefill calls at L=8192")
     args = ap.parse_args()
     if args.profile_decode:
         profile_decode()
+        return
+    if args.profile_prefill:
+        profile_prefill()
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
