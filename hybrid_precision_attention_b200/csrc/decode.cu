@@ -51,7 +51,10 @@ namespace {
 // stage while another warp's earlier tile there had not landed yet would see the
 // older completed phase and consume the wrong data.  With NSTAGES = 2 NC,
 // stage s belongs to warp s % NC.
-constexpr int NC_WIDE = 9, NC_NARROW = 3;
+#ifndef HQ_DECODE_NC_WIDE
+#define HQ_DECODE_NC_WIDE 9
+#endif
+constexpr int NC_WIDE = HQ_DECODE_NC_WIDE, NC_NARROW = 3;
 constexpr int PK = 64;                         // positions per packed tile
 constexpr int FT = 16;                         // rows per FP16 tile
 constexpr int FSTRIDE = 256;                   // bytes per FP16 row in shared memory (one contiguous copy)
@@ -114,6 +117,17 @@ __device__ __forceinline__ uint32_t fp16_valid(const Geo& g, int tile) {
     m |= (g.n_packed + off < g.T ? 1u : 0u) << r;
   }
   return m;
+}
+
+// This split's tile range [t_lo, t_hi): splits get equal shares of the bytes
+// (a packed tile, 10 KB, counts 5; an FP16 tile, 8 KB, counts 4).
+__device__ __forceinline__ void split_range(const Geo& geo, int split, int S, int& t_lo, int& t_hi) {
+  const long long wp = 5ll * geo.NP;
+  const long long wt = wp + 4ll * (geo.NV + geo.NR);
+  const long long w_lo = (static_cast<long long>(split) * wt) / S;
+  const long long w_hi = (static_cast<long long>(split + 1) * wt) / S;
+  t_lo = static_cast<int>(w_lo <= wp ? (w_lo + 4) / 5 : geo.NP + (w_lo - wp + 3) / 4);
+  t_hi = static_cast<int>(w_hi <= wp ? (w_hi + 4) / 5 : geo.NP + (w_hi - wp + 3) / 4);
 }
 
 struct WarpState {
@@ -344,25 +358,6 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
 
-  const int T = c.state[HQ_STATE_T];
-  const int n_packed = c.state[HQ_STATE_NPACKED];
-  const int n_vl = c.state[HQ_STATE_NVL];
-  if (T - n_packed >= c.W + HQ_STAGE || T >= c.cap) {  // staging full / no room: do nothing
-    if (split == 0 && kvh == 0 && b == 0 && threadIdx.x == 0)
-      set_err(c.state, T >= c.cap ? HQ_DEVERR_CAPACITY : HQ_DEVERR_STAGING_FULL);
-    return;
-  }
-  const Geo geo = geo_of(n_packed, n_vl, T, R);
-  // splits get equal shares of the bytes: a packed tile (10 KB) counts 5, an
-  // FP16 tile (8 KB) counts 4
-  const long long wp = 5ll * geo.NP;
-  const long long wt = wp + 4ll * (geo.NV + geo.NR);
-  const long long w_lo = (static_cast<long long>(split) * wt) / S;
-  const long long w_hi = (static_cast<long long>(split + 1) * wt) / S;
-  const int t_lo = static_cast<int>(w_lo <= wp ? (w_lo + 4) / 5 : geo.NP + (w_lo - wp + 3) / 4);
-  const int t_hi = static_cast<int>(w_hi <= wp ? (w_hi + 4) / 5 : geo.NP + (w_hi - wp + 3) / 4);
-  const int ntile = t_hi - t_lo;
-
   if (threadIdx.x == 0) {
     for (int i = 0; i < NSTAGES; ++i) {
       mbar_init(&full[i], 1);
@@ -372,6 +367,48 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
     s_timeout = 0;
     fence_mbar_init();
   }
+  if (threadIdx.x == NCONS * 32) {
+    // Before the dependency wait, warm L2 with this split's packed pages and VL
+    // rows.  The lengths read here may be stale (the previous grid can still be
+    // writing them): they only steer a prefetch hint, and the ranges are clamped
+    // to the buffers, so a stale value costs bandwidth, never correctness.
+    const int pT = *reinterpret_cast<volatile const int*>(c.state + HQ_STATE_T);
+    const int pnp = *reinterpret_cast<volatile const int*>(c.state + HQ_STATE_NPACKED);
+    const int pnv = *reinterpret_cast<volatile const int*>(c.state + HQ_STATE_NVL);
+    const Geo pg = geo_of(min(max(pnp, 0), c.cap), min(max(pnv, 0), c.vl_cap), pT, R);
+    int p_lo, p_hi;
+    split_range(pg, split, S, p_lo, p_hi);
+    const int npg = c.cap / PK;
+    const int a0 = min(max(p_lo, 0), npg), a1 = min(max(min(p_hi, pg.NP), a0), npg);
+    const uint8_t* pages = c.pages + static_cast<size_t>(bh) * npg * HQ_PAGE_BYTES;
+    for (int pgi = a0; pgi < a1; pgi += 16)  // 16 pages (165 KB) per prefetch
+      prefetch_l2(pages + static_cast<size_t>(pgi) * HQ_PAGE_BYTES, min(16, a1 - pgi) * HQ_PAGE_BYTES);
+    const int v0 = min(max(p_lo - pg.NP, 0), c.vl_cap / FT), v1 = min(max(p_hi - pg.NP, v0), min(pg.NV, c.vl_cap / FT));
+    if (v1 > v0) {
+      const size_t off = (static_cast<size_t>(bh) * c.vl_cap + v0 * FT) * D;
+      prefetch_l2(c.kf + off, (v1 - v0) * FT * D * 2);
+      prefetch_l2(c.vf + off, (v1 - v0) * FT * D * 2);
+    }
+  }
+  // programmatic dependent launch: everything this kernel reads (the state, the
+  // cache, the previous step's appended token) was written by earlier kernels,
+  // so wait for them first; then let the next step's grid start launching onto
+  // the SMs that free up (it waits here in turn)
+  griddep_wait();
+  griddep_launch_dependents();
+  const int T = c.state[HQ_STATE_T];
+  const int n_packed = c.state[HQ_STATE_NPACKED];
+  const int n_vl = c.state[HQ_STATE_NVL];
+  if (T - n_packed >= c.W + HQ_STAGE || T >= c.cap) {  // staging full / no room: do nothing
+    if (split == 0 && kvh == 0 && b == 0 && threadIdx.x == 0)
+      set_err(c.state, T >= c.cap ? HQ_DEVERR_CAPACITY : HQ_DEVERR_STAGING_FULL);
+    return;
+  }
+  const Geo geo = geo_of(n_packed, n_vl, T, R);
+  int t_lo, t_hi;
+  split_range(geo, split, S, t_lo, t_hi);
+  const int ntile = t_hi - t_lo;
+
   __syncthreads();
 
   WarpState ws;
@@ -382,30 +419,31 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
 
   if (warp == NCONS) {
     // ---------------------------------------------------------------- producer
-    // one lane issues everything (1 bulk copy per packed page, 2 per FP16
-    // tile); its loop is kept short because it shares issue slots with the
-    // consumer warps
-    if (lane == 0) {
+    // lane s owns stage s and issues tiles s, s + NSTAGES, s + 2 NSTAGES, ...
+    // (1 bulk copy per packed page, 2 per FP16 tile): the initial fill of every
+    // stage leaves in one instruction, and a refill waits only for its own stage
+    static_assert(NSTAGES <= 32, "one producer lane per stage");
+    if (lane < NSTAGES) {
+      const int s = lane;
       const size_t npg = static_cast<size_t>(c.cap / PK);
-      const uint8_t* page = c.pages + (static_cast<size_t>(bh) * npg + t_lo) * HQ_PAGE_BYTES;
+      const uint8_t* pages = c.pages + static_cast<size_t>(bh) * npg * HQ_PAGE_BYTES;
       const uint16_t* kf = c.kf + static_cast<size_t>(bh) * c.vl_cap * D;
       const uint16_t* vf = c.vf + static_cast<size_t>(bh) * c.vl_cap * D;
       const uint16_t* kr = c.kr + static_cast<size_t>(bh) * R * D;
       const uint16_t* vr = c.vr + static_cast<size_t>(bh) * R * D;
-      int s = 0;
-      uint32_t ph = 1;  // flips to 0 when the ring first wraps: the wait at i = NSTAGES is for phase 0
-      for (int i = 0; i < ntile; ++i) {
-        if (i >= NSTAGES && !mbar_wait(&empty[s], ph, c.state)) {
+      uint8_t* st = smem + s * STAGE_BYTES;
+      int k = 0;  // uses of this stage so far
+      for (int i = s; i < ntile; i += NSTAGES, ++k) {
+        // the k-th refill waits for the consumer's k-th release (phase k - 1)
+        if (k > 0 && !mbar_wait(&empty[s], (k - 1) & 1, c.state)) {
           s_timeout = 1;
           break;
         }
-        s_issued[s] = i / NSTAGES + 1;
-        uint8_t* st = smem + s * STAGE_BYTES;
+        s_issued[s] = k + 1;
         const int tile = t_lo + i;
         if (tile < geo.NP) {
           mbar_arrive_expect_tx(&full[s], PK_TX);
-          bulk_g2s(st, page, PK_TX, &full[s]);
-          page += HQ_PAGE_BYTES;
+          bulk_g2s(st, pages + static_cast<size_t>(tile) * HQ_PAGE_BYTES, PK_TX, &full[s]);
         } else {
           const int v = tile - geo.NP, j = v - geo.NV;
           const uint16_t* ksrc = j < 0 ? kf + v * (FT * D) : (j < geo.NR - 1 ? kr + j * (FT * D) : k_new + bh * D);
@@ -414,10 +452,6 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
           mbar_arrive_expect_tx(&full[s], 2 * bytes);
           bulk_g2s(st, ksrc, bytes, &full[s]);
           bulk_g2s(st + OFF_FV, vsrc, bytes, &full[s]);
-        }
-        if (++s == NSTAGES) {
-          s = 0;
-          ph ^= 1;
         }
       }
     }
@@ -493,104 +527,120 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
   __syncthreads();  // (B) warp states visible
 
   // ---------------------------------------------------------------- CTA merge -> split partial
-  __shared__ float s_cw[NCONS][8];
-  __shared__ float s_cm[8], s_cl[8];
+  // each thread owns 4 dims of one query and weighs the NC warp states itself
+  // (NC exp2 per thread instead of a third barrier)
   __shared__ int s_glast;
   const float* wsm = reinterpret_cast<const float*>(smem);
-  if (threadIdx.x < 8) {
-    const int qc = threadIdx.x;
+  float* part = parts + (static_cast<size_t>(bh) * S + split) * PART_FLOATS;
+  for (int i = threadIdx.x; i < 8 * D / 4; i += NTHREADS) {
+    const int qc = (4 * i) / D;
     float mm = -INFINITY;
 #pragma unroll
     for (int w = 0; w < NCONS; ++w) mm = fmaxf(mm, wsm[w * PART_FLOATS + qc]);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float ll = 0.f;
 #pragma unroll
     for (int w = 0; w < NCONS; ++w) {
       const float mw = wsm[w * PART_FLOATS + qc];
       const float wt = mw == -INFINITY ? 0.f : ex2(mw - mm);
-      s_cw[w][qc] = wt;
-      ll += wt * wsm[w * PART_FLOATS + 8 + qc];
-    }
-    s_cm[qc] = mm;
-    s_cl[qc] = ll;
-  }
-  __syncthreads();
-  float* part = parts + (static_cast<size_t>(bh) * S + split) * PART_FLOATS;
-  if (threadIdx.x < 8) {
-    part[threadIdx.x] = s_cm[threadIdx.x];
-    part[8 + threadIdx.x] = s_cl[threadIdx.x];
-  }
-  for (int i = threadIdx.x; i < 8 * D / 4; i += NTHREADS) {
-    const int qc = (4 * i) / D;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int w = 0; w < NCONS; ++w) {
       const float4 o = reinterpret_cast<const float4*>(wsm + w * PART_FLOATS + 16)[i];
-      const float wt = s_cw[w][qc];
       acc.x = fmaf(wt, o.x, acc.x);
       acc.y = fmaf(wt, o.y, acc.y);
       acc.z = fmaf(wt, o.z, acc.z);
       acc.w = fmaf(wt, o.w, acc.w);
+      ll = fmaf(wt, wsm[w * PART_FLOATS + 8 + qc], ll);
     }
     reinterpret_cast<float4*>(part + 16)[i] = acc;
+    if ((4 * i) % D == 0) {
+      part[qc] = mm;
+      part[8 + qc] = ll;
+    }
   }
-  // completion tickets: every thread releases its part of the partial, then one
-  // thread learns whether this is the last split of its (b, kv head) and/or the
-  // last CTA of the grid; the last CTA acquires before reading the partials
-  fence_acq_rel_gpu();
+  // the new token's K / V rows and this group's queries, loaded now so that the
+  // append after the ticket is stores only (inputs: no ordering concerns)
+  const int slot = T % R;
+  constexpr int APPEND_MAX = (2 + HQ_MAX_GQA) * (D / 8);
+  static_assert(APPEND_MAX <= 2 * NTHREADS, "at most two 16-byte chunks of the append per thread");
+  uint4 app[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+  uint4* app_dst[2] = {nullptr, nullptr};
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int e = threadIdx.x + k * NTHREADS;
+    if (e < (2 + G) * (D / 8)) {
+      const int row = e / (D / 8), ch = e % (D / 8);
+      if (row < 2) {
+        app[k] = reinterpret_cast<const uint4*>((row ? v_new : k_new) + static_cast<size_t>(bh) * D)[ch];
+        app_dst[k] = reinterpret_cast<uint4*>((row ? c.vr : c.kr) + (static_cast<size_t>(bh) * R + slot) * D) + ch;
+      } else {
+        const size_t h = static_cast<size_t>(b) * c.Hq + kvh * G + (row - 2);
+        app[k] = reinterpret_cast<const uint4*>(q + h * D)[ch];
+        app_dst[k] = reinterpret_cast<uint4*>(c.qbuf + (h * HQ_QBUF + (T % HQ_QBUF)) * D) + ch;
+      }
+    }
+  }
+  // completion tickets: the barrier orders every thread's partial writes before
+  // thread 0's gpu-scope release; the two counters are bumped together; the
+  // last CTA of the head (and/or of the grid) acquires before the barrier that
+  // releases its other threads to read the partials
   __syncthreads();
   if (threadIdx.x == 0) {
-    s_last = atomicAdd(&tickets[1 + bh], 1u) == static_cast<unsigned>(S - 1);
-    s_glast = atomicAdd(&tickets[0], 1u) == gridDim.x * gridDim.y * gridDim.z - 1;
+    fence_acq_rel_gpu();
+    const unsigned int th = atomicAdd(&tickets[1 + bh], 1u);
+    const unsigned int tg = atomicAdd(&tickets[0], 1u);
+    s_last = th == static_cast<unsigned>(S - 1);
+    s_glast = tg == gridDim.x * gridDim.y * gridDim.z - 1;
+    if (s_last || s_glast) fence_acq_rel_gpu();
   }
   __syncthreads();
-  if (s_last || s_glast) fence_acq_rel_gpu();
   if (s_last) {
-    // log-sum-exp merge of the S partials of this (b, kv head), in one pass: each
-    // thread owns 4 output dims of one query and streams (m, l, O) of every
-    // split, 8 splits' loads in flight at a time, merging online
+    // log-sum-exp merge of the S partials of this (b, kv head): the (m, l) of
+    // every split go to shared memory first, so that the weights are known and
+    // each thread (one query, 4 dims) then has all its O loads in flight at once
     const float* pb = parts + static_cast<size_t>(bh) * S * PART_FLOATS;
+    float* sm_m = reinterpret_cast<float*>(smem);      // [S][8]: m, then the split weight
+    float* sm_l = sm_m + 64 * 8;                        // [S][8]
+    float* sm_inv = sm_l + 64 * 8;                      // [8]
+    for (int i = threadIdx.x; i < S * 8; i += NTHREADS) {
+      sm_m[i] = __ldcg(pb + (i >> 3) * PART_FLOATS + (i & 7));
+      sm_l[i] = __ldcg(pb + (i >> 3) * PART_FLOATS + 8 + (i & 7));
+    }
+    __syncthreads();
+    if (threadIdx.x < G) {
+      const int qc = threadIdx.x;
+      float mm = -INFINITY;
+      for (int sp = 0; sp < S; ++sp) mm = fmaxf(mm, sm_m[sp * 8 + qc]);
+      float ll = 0.f;
+      for (int sp = 0; sp < S; ++sp) {
+        const float ms = sm_m[sp * 8 + qc];
+        const float w = ms == -INFINITY ? 0.f : ex2(ms - mm);
+        sm_m[sp * 8 + qc] = w;
+        ll += w * sm_l[sp * 8 + qc];
+      }
+      sm_inv[qc] = ll > 0.f ? 1.0f / ll : 0.f;
+    }
+    __syncthreads();
     for (int it = threadIdx.x; it < G * (D / 4); it += NTHREADS) {
       const int qc = it / (D / 4), d4 = it % (D / 4);
       const float4* src = reinterpret_cast<const float4*>(pb + 16 + qc * D) + d4;
-      float mrun = -INFINITY, lrun = 0.f;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
+#pragma unroll 16
       for (int sp = 0; sp < S; ++sp) {
-        const float ms = __ldcg(pb + sp * PART_FLOATS + qc);
-        const float ls = __ldcg(pb + sp * PART_FLOATS + 8 + qc);
         const float4 o = __ldcg(src + sp * (PART_FLOATS / 4));
-        const float mn = fmaxf(mrun, ms);
-        const float a = mrun == -INFINITY ? 0.f : ex2(mrun - mn);
-        const float w = ms == -INFINITY ? 0.f : ex2(ms - mn);
-        lrun = lrun * a + ls * w;
-        acc.x = acc.x * a + o.x * w;
-        acc.y = acc.y * a + o.y * w;
-        acc.z = acc.z * a + o.z * w;
-        acc.w = acc.w * a + o.w * w;
-        mrun = mn;
+        const float w = sm_m[sp * 8 + qc];
+        acc.x = fmaf(w, o.x, acc.x);
+        acc.y = fmaf(w, o.y, acc.y);
+        acc.z = fmaf(w, o.z, acc.z);
+        acc.w = fmaf(w, o.w, acc.w);
       }
-      const float inv = lrun > 0.f ? 1.0f / lrun : 0.f;
+      const float inv = sm_inv[qc];
       __half2* dst = reinterpret_cast<__half2*>(out + (static_cast<size_t>(b) * c.Hq + kvh * G + qc) * D) + 2 * d4;
       dst[0] = __floats2half2_rn(acc.x * inv, acc.y * inv);
       dst[1] = __floats2half2_rn(acc.z * inv, acc.w * inv);
     }
     // every split of this head has consumed its tiles: append the new token to
     // the ring (slot T % R) and this group's queries to the query buffer
-    const int slot = T % R;
-    for (int i = threadIdx.x; i < (2 + G) * (D / 8); i += NTHREADS) {
-      const int row = i / (D / 8), ch = i % (D / 8);
-      const uint4* src;
-      uint4* dst;
-      if (row < 2) {
-        src = reinterpret_cast<const uint4*>((row ? v_new : k_new) + static_cast<size_t>(bh) * D) + ch;
-        dst = reinterpret_cast<uint4*>((row ? c.vr : c.kr) + (static_cast<size_t>(bh) * R + slot) * D) + ch;
-      } else {
-        const size_t h = static_cast<size_t>(b) * c.Hq + kvh * G + (row - 2);
-        src = reinterpret_cast<const uint4*>(q + h * D) + ch;
-        dst = reinterpret_cast<uint4*>(c.qbuf + (h * HQ_QBUF + (T % HQ_QBUF)) * D) + ch;
-      }
-      *dst = *src;
-    }
+    if (app_dst[0]) *app_dst[0] = app[0];
+    if (app_dst[1]) *app_dst[1] = app[1];
     if (threadIdx.x == 0) tickets[1 + bh] = 0u;
   }
   // the last CTA of the grid advances T (every CTA read the state at its start)
@@ -616,7 +666,7 @@ DecodeShape decode_shape(const hq_cache& c, int sms) {
   DecodeShape d;
   d.wide = sms / units >= 4;
   int s = d.wide ? sms / units : (3 * sms) / units;
-  const int cap_s = d.wide ? (nt_max + 8) / 9 : (nt_max + 2) / 3;  // at least ~one tile per consumer warp
+  const int cap_s = d.wide ? (nt_max + NC_WIDE - 1) / NC_WIDE : (nt_max + NC_NARROW - 1) / NC_NARROW;  // ~one tile per consumer warp
   if (s > cap_s) s = cap_s;
   if (s > 64) s = 64;
   if (s < 1) s = 1;
@@ -652,13 +702,21 @@ hq_status launch_decode(const hq_cache& c, const uint16_t* q, const uint16_t* kn
   }
   unsigned int* tickets = reinterpret_cast<unsigned int*>(ws);
   float* parts = reinterpret_cast<float*>(static_cast<char*>(ws) + decode_counter_bytes(c));
-  dim3 grid(shp.S, c.Hkv, c.B);
-  if (shp.wide)
-    decode_kernel<NC_WIDE, 1><<<grid, (NC_WIDE + 1) * 32, smem, st>>>(c, q, kn, vn, out, sm_scale * LOG2E, shp.S, parts, tickets);
-  else
-    decode_kernel<NC_NARROW, 3><<<grid, (NC_NARROW + 1) * 32, smem, st>>>(c, q, kn, vn, out, sm_scale * LOG2E, shp.S, parts,
-                                                                          tickets);
-  return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(shp.S, c.Hkv, c.B);
+  cfg.blockDim = dim3((nc + 1) * 32, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const float qs = sm_scale * LOG2E;
+  const cudaError_t e = shp.wide
+      ? cudaLaunchKernelEx(&cfg, decode_kernel<NC_WIDE, 1>, c, q, kn, vn, out, qs, shp.S, parts, tickets)
+      : cudaLaunchKernelEx(&cfg, decode_kernel<NC_NARROW, 3>, c, q, kn, vn, out, qs, shp.S, parts, tickets);
+  return e == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 
 }  // namespace hq
