@@ -137,6 +137,13 @@ struct WarpState {
 
 // Online-softmax update for NMT 16-key blocks whose S^T accumulators are in s.
 // Returns the P^T B-fragments (two per block) in pb.
+// Online-softmax update for NMT 16-key blocks whose S^T accumulators are in s.
+// Returns the P^T B-fragments (two per block) in pb.  The running max moves
+// lazily: only when a query's tile max exceeds it by more than LAZY_MAX (log2
+// units), so most tiles skip the rescale of O and l; p then stays below
+// 2^LAZY_MAX, well inside fp16, and l accumulates in fp32.
+constexpr float LAZY_MAX = 8.0f;
+
 template <int NMT>
 __device__ __forceinline__ void softmax_update(WarpState& ws, float (&s)[NMT][4], uint32_t (&pb)[NMT][2]) {
   float mx0 = -INFINITY, mx1 = -INFINITY;
@@ -150,21 +157,24 @@ __device__ __forceinline__ void softmax_update(WarpState& ws, float (&s)[NMT][4]
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
   }
-  const float mn0 = fmaxf(ws.m[0], mx0), mn1 = fmaxf(ws.m[1], mx1);
-  const float ref0 = mn0 == -INFINITY ? 0.f : mn0;
-  const float ref1 = mn1 == -INFINITY ? 0.f : mn1;
-  const float c0 = ex2(ws.m[0] - ref0), c1 = ex2(ws.m[1] - ref1);
-  ws.m[0] = mn0;
-  ws.m[1] = mn1;
-  ws.l[0] *= c0;
-  ws.l[1] *= c1;
+  const bool up0 = mx0 > ws.m[0] + LAZY_MAX, up1 = mx1 > ws.m[1] + LAZY_MAX;
+  if (__any_sync(0xffffffffu, up0 || up1)) {
+    // exp2(-inf) = 0 when the old max is -inf (O and l are still zero then)
+    const float c0 = up0 ? ex2(ws.m[0] - mx0) : 1.f, c1 = up1 ? ex2(ws.m[1] - mx1) : 1.f;
+    ws.m[0] = up0 ? mx0 : ws.m[0];
+    ws.m[1] = up1 ? mx1 : ws.m[1];
+    ws.l[0] *= c0;
+    ws.l[1] *= c1;
 #pragma unroll
-  for (int m = 0; m < 8; ++m) {
-    ws.o[m][0] *= c0;
-    ws.o[m][2] *= c0;
-    ws.o[m][1] *= c1;
-    ws.o[m][3] *= c1;
+    for (int m = 0; m < 8; ++m) {
+      ws.o[m][0] *= c0;
+      ws.o[m][2] *= c0;
+      ws.o[m][1] *= c1;
+      ws.o[m][3] *= c1;
+    }
   }
+  const float ref0 = ws.m[0] == -INFINITY ? 0.f : ws.m[0];
+  const float ref1 = ws.m[1] == -INFINITY ? 0.f : ws.m[1];
 #pragma unroll
   for (int i = 0; i < NMT; ++i) {
     const float p0 = ex2(s[i][0] - ref0), p1 = ex2(s[i][1] - ref1);
@@ -176,7 +186,8 @@ __device__ __forceinline__ void softmax_update(WarpState& ws, float (&s)[NMT][4]
   }
 }
 
-// one K4V4 packed tile (64 positions) by one warp
+// one K4V4 packed tile (64 positions) by one warp: S^T = K^ . Q^T for the four
+// 16-key blocks, one online-softmax step for all 64 keys, O^T += V^T . P^T
 __device__ __forceinline__ void packed_tile(WarpState& ws, const uint8_t* st, const uint32_t (&qf)[8][2], int tile, int n_packed,
                                             float qscale, int g, int t) {
   const uint8_t* kc = st;
@@ -186,99 +197,103 @@ __device__ __forceinline__ void packed_tile(WarpState& ws, const uint8_t* st, co
   const uint32_t* mk = reinterpret_cast<const uint32_t*>(st + OFF_MASK);
   const int base = tile * PK;
   const bool full = base + PK <= n_packed;
+  const int pa = pi_pk(g), pbk = pi_pk(g + 8);
+  // additive score bias of this thread's 8 key rows: -inf beyond n_packed or on
+  // a vertical line (its FP16 row is read instead), else 0
+  const uint32_t m0 = mk[0], m1 = mk[1];
+  float bias[4][2];
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+    const uint32_t w = (mt >> 1) ? m1 : m0;
+    const int ra = 16 * mt + pa, rb = 16 * mt + pbk;
+    const bool va = (full || base + ra < n_packed) && !((w >> (ra & 31)) & 1u);
+    const bool vb = (full || base + rb < n_packed) && !((w >> (rb & 31)) & 1u);
+    bias[mt][0] = va ? 0.f : -INFINITY;
+    bias[mt][1] = vb ? 0.f : -INFINITY;
+  }
 
-  // two halves of 32 keys, each: S^T = K^ . Q^T (2 blocks of 16 keys),
-  // online-softmax step, O^T += V^T . P^T
-#pragma unroll 1
-  for (int hf = 0; hf < 2; ++hf) {
-    float s[2][4];
+  float s[4][4];
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int mt = 2 * hf + j;
-      const int ra = 16 * mt + pi_pk(g), rb = 16 * mt + pi_pk(g + 8);
-      const uint4 ka = *reinterpret_cast<const uint4*>(kc + ra * 64 + 16 * t);
-      const uint4 kb = *reinterpret_cast<const uint4*>(kc + rb * 64 + 16 * t);
-      const uint32_t za = ks[ra * 4 + t], zb = ks[rb * 4 + t];
-      const uint32_t sa2 = prmt(za, za, 0x1010), za2 = prmt(za, za, 0x3232);
-      const uint32_t sb2 = prmt(zb, zb, 0x1010), zb2 = prmt(zb, zb, 0x3232);
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w};
-      const uint32_t wb[4] = {kb.x, kb.y, kb.z, kb.w};
+  for (int mt = 0; mt < 4; ++mt) {
+    const int ra = 16 * mt + pa, rb = 16 * mt + pbk;
+    const uint4 ka = *reinterpret_cast<const uint4*>(kc + ra * 64 + 16 * t);
+    const uint4 kb = *reinterpret_cast<const uint4*>(kc + rb * 64 + 16 * t);
+    const uint32_t za = ks[ra * 4 + t], zb = ks[rb * 4 + t];
+    const uint32_t sa2 = prmt(za, za, 0x1010), za2 = prmt(za, za, 0x3232);
+    const uint32_t sb2 = prmt(zb, zb, 0x1010), zb2 = prmt(zb, zb, 0x3232);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w};
+    const uint32_t wb[4] = {kb.x, kb.y, kb.z, kb.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 4; ++i) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t xa = wa[i] >> (8 * h), xb = wb[i] >> (8 * h);
-          const uint32_t a0 = hfma2_u(nib_lo(xa), sa2, za2);
-          const uint32_t a2 = hfma2_u(nib_hi(xa), sa2, za2);
-          const uint32_t a1 = hfma2_u(nib_lo(xb), sb2, zb2);
-          const uint32_t a3 = hfma2_u(nib_hi(xb), sb2, zb2);
-          mma16816(acc, a0, a1, a2, a3, qf[2 * i + h][0], qf[2 * i + h][1]);
-        }
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t xa = wa[i] >> (8 * h), xb = wb[i] >> (8 * h);
+        const uint32_t a0 = hfma2_u(nib_lo(xa), sa2, za2);
+        const uint32_t a2 = hfma2_u(nib_hi(xa), sa2, za2);
+        const uint32_t a1 = hfma2_u(nib_lo(xb), sb2, zb2);
+        const uint32_t a3 = hfma2_u(nib_hi(xb), sb2, zb2);
+        mma16816(acc, a0, a1, a2, a3, qf[2 * i + h][0], qf[2 * i + h][1]);
       }
-      // mask: beyond n_packed, or a vertical line (its FP16 row is read instead)
-      const bool va = (base + ra < n_packed) && !((mk[ra >> 5] >> (ra & 31)) & 1u);
-      const bool vb = (base + rb < n_packed) && !((mk[rb >> 5] >> (rb & 31)) & 1u);
-      s[j][0] = va ? acc[0] * qscale : -INFINITY;
-      s[j][1] = va ? acc[1] * qscale : -INFINITY;
-      s[j][2] = vb ? acc[2] * qscale : -INFINITY;
-      s[j][3] = vb ? acc[3] * qscale : -INFINITY;
     }
-    uint32_t pb[2][2];
-    softmax_update<2>(ws, s, pb);
+    s[mt][0] = fmaf(acc[0], qscale, bias[mt][0]);
+    s[mt][1] = fmaf(acc[1], qscale, bias[mt][0]);
+    s[mt][2] = fmaf(acc[2], qscale, bias[mt][1]);
+    s[mt][3] = fmaf(acc[3], qscale, bias[mt][1]);
+  }
+  uint32_t pb[4][2];
+  softmax_update<4>(ws, s, pb);
 
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int mt = 2 * hf + j;
-      const int r0 = 16 * mt + pi_pk(2 * t), r1 = 16 * mt + pi_pk(2 * t + 1);
-      const int r2 = 16 * mt + pi_pk(2 * t + 8), r3 = 16 * mt + pi_pk(2 * t + 9);
-      // two 32-bit loads per row, issued in a per-thread order that keeps the
-      // warp's accesses on distinct banks
-      const int e = t >> 1;
-      const uint32_t* v0 = reinterpret_cast<const uint32_t*>(vc + r0 * 64) + 2 * g;
-      const uint32_t* v1 = reinterpret_cast<const uint32_t*>(vc + r1 * 64) + 2 * g;
-      const uint32_t* v2 = reinterpret_cast<const uint32_t*>(vc + r2 * 64) + 2 * g;
-      const uint32_t* v3 = reinterpret_cast<const uint32_t*>(vc + r3 * 64) + 2 * g;
-      const uint32_t x0a = v0[e], x0b = v0[e ^ 1], x1a = v1[e], x1b = v1[e ^ 1];
-      const uint32_t x2a = v2[e], x2b = v2[e ^ 1], x3a = v3[e], x3b = v3[e ^ 1];
-      // un-rotate: w?0 = word 2g, w?1 = word 2g+1
-      const uint32_t w00 = e ? x0b : x0a, w01 = e ? x0a : x0b;
-      const uint32_t w10 = e ? x1b : x1a, w11 = e ? x1a : x1b;
-      const uint32_t w20 = e ? x2b : x2a, w21 = e ? x2a : x2b;
-      const uint32_t w30 = e ? x3b : x3a, w31 = e ? x3a : x3b;
-      const int grp = g >> 1;
-      const uint32_t z0 = vs[r0 * 4 + grp], z1 = vs[r1 * 4 + grp], z2 = vs[r2 * 4 + grp], z3 = vs[r3 * 4 + grp];
-      const uint32_t s01 = prmt(z0, z1, 0x5410), o01 = prmt(z0, z1, 0x7632);
-      const uint32_t s23 = prmt(z2, z3, 0x5410), o23 = prmt(z2, z3, 0x7632);
-      // pair nibbles of the two keys: x?[k] holds dims 16g + 4k .. 16g + 4k + 3 of both keys
-      uint32_t xab[4], xcd[4];
-      xab[0] = prmt(w00, w10, 0x5410);
-      xab[1] = prmt(w00, w10, 0x7632);
-      xab[2] = prmt(w01, w11, 0x5410);
-      xab[3] = prmt(w01, w11, 0x7632);
-      xcd[0] = prmt(w20, w30, 0x5410);
-      xcd[1] = prmt(w20, w30, 0x7632);
-      xcd[2] = prmt(w21, w31, 0x5410);
-      xcd[3] = prmt(w21, w31, 0x7632);
-      uint32_t keep_ab = 0xFFFFFFFFu, keep_cd = 0xFFFFFFFFu;
-      if (!full) {  // rows past n_packed may hold stale records: zero them out of P.V
-        keep_ab = (base + r0 < n_packed ? 0x0000FFFFu : 0u) | (base + r1 < n_packed ? 0xFFFF0000u : 0u);
-        keep_cd = (base + r2 < n_packed ? 0x0000FFFFu : 0u) | (base + r3 < n_packed ? 0xFFFF0000u : 0u);
-      }
+  for (int mt = 0; mt < 4; ++mt) {
+    const int r0 = 16 * mt + pi_pk(2 * t), r1 = 16 * mt + pi_pk(2 * t + 1);
+    const int r2 = 16 * mt + pi_pk(2 * t + 8), r3 = 16 * mt + pi_pk(2 * t + 9);
+    // two 32-bit loads per row, issued in a per-thread order that keeps the
+    // warp's accesses on distinct banks
+    const int e = t >> 1;
+    const uint32_t* v0 = reinterpret_cast<const uint32_t*>(vc + r0 * 64) + 2 * g;
+    const uint32_t* v1 = reinterpret_cast<const uint32_t*>(vc + r1 * 64) + 2 * g;
+    const uint32_t* v2 = reinterpret_cast<const uint32_t*>(vc + r2 * 64) + 2 * g;
+    const uint32_t* v3 = reinterpret_cast<const uint32_t*>(vc + r3 * 64) + 2 * g;
+    const uint32_t x0a = v0[e], x0b = v0[e ^ 1], x1a = v1[e], x1b = v1[e ^ 1];
+    const uint32_t x2a = v2[e], x2b = v2[e ^ 1], x3a = v3[e], x3b = v3[e ^ 1];
+    // un-rotate: w?0 = word 2g, w?1 = word 2g+1
+    const uint32_t w00 = e ? x0b : x0a, w01 = e ? x0a : x0b;
+    const uint32_t w10 = e ? x1b : x1a, w11 = e ? x1a : x1b;
+    const uint32_t w20 = e ? x2b : x2a, w21 = e ? x2a : x2b;
+    const uint32_t w30 = e ? x3b : x3a, w31 = e ? x3a : x3b;
+    const int grp = g >> 1;
+    const uint32_t z0 = vs[r0 * 4 + grp], z1 = vs[r1 * 4 + grp], z2 = vs[r2 * 4 + grp], z3 = vs[r3 * 4 + grp];
+    const uint32_t s01 = prmt(z0, z1, 0x5410), o01 = prmt(z0, z1, 0x7632);
+    const uint32_t s23 = prmt(z2, z3, 0x5410), o23 = prmt(z2, z3, 0x7632);
+    // pair nibbles of the two keys: x?[k] holds dims 16g + 4k .. 16g + 4k + 3 of both keys
+    uint32_t xab[4], xcd[4];
+    xab[0] = prmt(w00, w10, 0x5410);
+    xab[1] = prmt(w00, w10, 0x7632);
+    xab[2] = prmt(w01, w11, 0x5410);
+    xab[3] = prmt(w01, w11, 0x7632);
+    xcd[0] = prmt(w20, w30, 0x5410);
+    xcd[1] = prmt(w20, w30, 0x7632);
+    xcd[2] = prmt(w21, w31, 0x5410);
+    xcd[3] = prmt(w21, w31, 0x7632);
+    uint32_t keep_ab = 0xFFFFFFFFu, keep_cd = 0xFFFFFFFFu;
+    if (!full) {  // rows past n_packed may hold stale records: zero them out of P.V
+      keep_ab = (base + r0 < n_packed ? 0x0000FFFFu : 0u) | (base + r1 < n_packed ? 0xFFFF0000u : 0u);
+      keep_cd = (base + r2 < n_packed ? 0x0000FFFFu : 0u) | (base + r3 < n_packed ? 0xFFFF0000u : 0u);
+    }
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const uint32_t yab = xab[m >> 1] >> (8 * (m & 1));
-        const uint32_t ycd = xcd[m >> 1] >> (8 * (m & 1));
-        uint32_t a0 = hfma2_u(nib_lo(yab), s01, o01);
-        uint32_t a1 = hfma2_u(nib_hi(yab), s01, o01);
-        uint32_t a2 = hfma2_u(nib_lo(ycd), s23, o23);
-        uint32_t a3 = hfma2_u(nib_hi(ycd), s23, o23);
-        if (!full) {
-          a0 &= keep_ab; a1 &= keep_ab;
-          a2 &= keep_cd; a3 &= keep_cd;
-        }
-        mma16816(ws.o[m], a0, a1, a2, a3, pb[j][0], pb[j][1]);
+    for (int m = 0; m < 8; ++m) {
+      const uint32_t yab = xab[m >> 1] >> (8 * (m & 1));
+      const uint32_t ycd = xcd[m >> 1] >> (8 * (m & 1));
+      uint32_t a0 = hfma2_u(nib_lo(yab), s01, o01);
+      uint32_t a1 = hfma2_u(nib_hi(yab), s01, o01);
+      uint32_t a2 = hfma2_u(nib_lo(ycd), s23, o23);
+      uint32_t a3 = hfma2_u(nib_hi(ycd), s23, o23);
+      if (!full) {
+        a0 &= keep_ab; a1 &= keep_ab;
+        a2 &= keep_cd; a3 &= keep_cd;
       }
+      mma16816(ws.o[m], a0, a1, a2, a3, pb[mt][0], pb[mt][1]);
     }
   }
 }

@@ -12,7 +12,8 @@
 //   ring_fill      init only: last min(W, L) prefix rows -> FP16 ring
 //   vl_gather      merge only: new VL rows -> workspace (old VL row, ring row,
 //                  or the dequantised record rounded once to fp16); clears old bits
-//   vl_install     rows -> VL store, positions, bitmap bits, state update
+//   vl_install     rows -> VL store, positions, bitmap bits, per-page first VL row,
+//                  state update
 #include "common.cuh"
 
 namespace hq {
@@ -212,7 +213,12 @@ __global__ void vl_install_kernel(hq_cache c, const uint16_t* __restrict__ srck,
     reinterpret_cast<uint4*>(t)[ch] = reinterpret_cast<const uint4*>(s)[ch];
     if (ch == 0 && which == 0) {
       c.vl_pos[bh * d.vl_cap + row] = p;
-      atomicOr(page_mask(page_of(c, bh, p)) + ((p & 63) >> 5), 1u << (p & 31));
+      uint8_t* page = page_of(c, bh, p);
+      atomicOr(page_mask(page) + ((p & 63) >> 5), 1u << (p & 31));
+      // the first vertical line of a page records its VL-store row (rows are in
+      // ascending position order), so readers find a line's row by a popcount
+      if (row == 0 || (c.vl_sel[bh * d.vl_cap + row - 1] >> 6) != (p >> 6))
+        *reinterpret_cast<int32_t*>(page + HQ_PAGE_VLBASE) = row;
     }
   }
   // state update by the last block (every block has read state above)

@@ -8,29 +8,42 @@
 // score_j = sum over the group's query heads h and buffered queries i of
 //           softmax_{j' <= p_i}(q_{h,i} . k_j' * sm_scale)[j],   j < n = T - W.
 //
-// Kernels
-//   select_pass<LSE>   per key chunk of 128: S = Q . K^T on tensor cores
-//                      (mma.m16n8k16, keys rebuilt in shared memory in their
-//                      current representation) -> per-(query, chunk) running
-//                      max / sum in the exp2 domain
-//   lse_merge          per-query log-sum-exp over the chunks
-//   select_pass<COL>   recompute S, p = exp2(S - lse), column sums over all
-//                      queries of the group -> score_j (no atomics in global
-//                      memory: one CTA owns each key)
-//   topk               one CTA per (b, kv head): 4 rounds of 8-bit radix
-//                      select on the float bit patterns (scores are >= 0, so
-//                      the bit order is the value order) -> exact k-th value,
-//                      then a block scan writes the chosen positions in
-//                      ascending order, ties to the lowest positions
-#include "common.cuh"
+// Both passes run on the tcgen05 tensor cores, one CTA per (key range, b, kv
+// head), all M = G x nq queries of the group in shared memory:
+//   sel_pass<false>  S = Q . K^T (M rows of 128 queries, N = 128 keys) into
+//                    TMEM; per query row a running max / sum in the exp2
+//                    domain over the CTA's keys -> (m, l) partial per row
+//   sel_pass<true>   per-row log-sum-exp from the partials, then
+//                    S^T = K . Q^T (M = 128 keys, N = the queries) into TMEM;
+//                    per key (one TMEM lane per thread) the sum over queries of
+//                    exp2(s - lse) -> score_j.  No atomics: each key's score is
+//                    finished inside one CTA.
+//   topk             one CTA per (b, kv head): 8-bit radix select on the float
+//                    bit patterns (scores are >= 0, so the bit order is the value
+//                    order) over the scores held in shared memory -> exact k-th
+//                    value, then an ordered compaction writes the chosen
+//                    positions ascending, ties to the lowest positions
+// Keys are rebuilt as fp16 in their current representation (dense prefix in
+// init mode; ring, VL row or dequantised K4V4 record in decode mode) by four
+// builder warps straight into the 128-byte-swizzled K-major operand layout.
+// Warp roles (416 threads): warps 0-7 epilogue (column half = warp / 4, TMEM
+// lane quarter = warp % 4), warps 8-11 key builders (one key row per thread),
+// warp 12 TMEM allocation and the MMA issue.  Every mbarrier wait is bounded
+// (about 1 s); a timeout sets HQ_DEVERR_TIMEOUT and the CTA drains its MMAs
+// before releasing TMEM.
+#include "tc.cuh"
 
 namespace hq {
 namespace {
 
-constexpr int CH = 128;          // keys per chunk
-constexpr int SROW = 272;        // bytes per fp16 row in shared memory
-constexpr int NT_SEL = 256;      // threads
-constexpr int NW_SEL = NT_SEL / 32;
+constexpr int KT = 128;                  // keys per tile
+constexpr int EPI_WARPS = 8;
+constexpr int BLD_WARPS = 4;
+constexpr int MMA_WARP = EPI_WARPS + BLD_WARPS;
+constexpr int SEL_THREADS = (MMA_WARP + 1) * 32;
+constexpr int MAX_SPLITS = 32;           // CTAs per (b, kv head)
+constexpr int KSTAGE = KT * 256;         // one rebuilt key tile: 2 halves x [128 rows][128 B]
+constexpr uint32_t TMEM_COLS = 512;
 
 struct SelArgs {
   hq_cache c;
@@ -38,10 +51,10 @@ struct SelArgs {
   const uint16_t* q_ext;    // init mode: [B, Hq, nq, D]
   int L;                    // init mode length
   int nq_init;
-  float* lse_part;          // [B*Hkv, C, M] x (m, l)
-  float* lse;               // [B*Hkv, M]
-  float* scores;            // [B*Hkv, cap]
-  int C;                    // chunks in the grid (cap / CH)
+  float* lse_part;          // [B*Hkv][MAX_SPLITS][Mp] x (m, l)
+  float* scores;            // [B*Hkv][cap]
+  int S;                    // CTAs per (b, kv head)
+  int Mp;                   // query rows in shared memory: G * HQ_QBUF rounded up to 128
   float qscale;             // sm_scale * log2(e)
 };
 
@@ -67,214 +80,370 @@ __device__ __forceinline__ SelGeo sel_geo(const SelArgs& a) {
   return g;
 }
 
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
-__device__ __forceinline__ int find_sorted(const int32_t* __restrict__ a, int n, int key) {
-  int lo = 0, hi = n;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (a[mid] < key) lo = mid + 1; else hi = mid;
+__device__ __forceinline__ bool sel_wait(uint64_t* bar, uint32_t parity, int32_t* state, int* abort_flag) {
+  if (*reinterpret_cast<volatile int*>(abort_flag)) return false;
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*reinterpret_cast<volatile int*>(abort_flag)) return false;
+    if (global_ns() - t0 > 1000000000ull) {
+      set_err(state, HQ_DEVERR_TIMEOUT);
+      *reinterpret_cast<volatile int*>(abort_flag) = 1;
+      return false;
+    }
   }
-  return (lo < n && a[lo] == key) ? lo : -1;
 }
 
-// Fill shared memory with keys [j0, j0 + CH) of (b, kv head) in their current
-// representation (fp16).  One warp per key row; lane l owns dims 4l .. 4l+3.
-__device__ void load_keys(const SelArgs& a, const SelGeo& g, int bh, int j0, uint8_t* ks) {
+// 16-byte chunk `ch` (dims 8 ch .. 8 ch + 7) of row `r` in the 128-byte-swizzled
+// K-major layout of a tile whose halves (dims 0-63, 64-127) are `half_bytes` apart
+__device__ __forceinline__ uint32_t sw128_off(int r, int ch, int half_bytes) {
+  return (ch >> 3) * half_bytes + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
+}
+
+// Build key row j of (b, kv head) bh as fp16 into row r of a key stage.
+__device__ __forceinline__ void build_key_row(const SelArgs& a, const SelGeo& g, int bh, int j, uint8_t* stage, int r) {
   const hq_cache& c = a.c;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int R = ring_len(c.W);
-  for (int r = warp; r < CH; r += NW_SEL) {
-    const int p = j0 + r;
-    uint2 v = make_uint2(0u, 0u);
-    if (p < g.T) {
-      if (a.k_dense) {
-        v = reinterpret_cast<const uint2*>(a.k_dense + (static_cast<size_t>(bh) * a.L + p) * D)[lane];
-      } else if (p >= g.n_packed) {
-        v = reinterpret_cast<const uint2*>(c.kr + (static_cast<size_t>(bh) * R + (p % R)) * D)[lane];
-      } else if ((page_mask(page_of(c, bh, p))[(p & 63) >> 5] >> (p & 31)) & 1u) {
-        const int idx = find_sorted(c.vl_pos + static_cast<size_t>(bh) * c.vl_cap, g.n_vl, p);
-        if (idx >= 0) v = reinterpret_cast<const uint2*>(c.kf + (static_cast<size_t>(bh) * c.vl_cap + idx) * D)[lane];
+  const uint4* src = nullptr;
+  if (j < g.T) {
+    if (a.k_dense) {
+      src = reinterpret_cast<const uint4*>(a.k_dense + (static_cast<size_t>(bh) * a.L + j) * D);
+    } else if (j >= g.n_packed) {
+      src = reinterpret_cast<const uint4*>(c.kr + (static_cast<size_t>(bh) * ring_len(c.W) + (j % ring_len(c.W))) * D);
+    } else {
+      uint8_t* page = page_of(c, bh, j);
+      const uint32_t* mk = page_mask(page);
+      const uint32_t w = mk[(j & 63) >> 5];
+      if ((w >> (j & 31)) & 1u) {
+        // VL row: the page records the VL-store row of its first vertical line
+        const int base = *reinterpret_cast<const int32_t*>(page + HQ_PAGE_VLBASE);
+        const int below = ((j & 63) >= 32 ? __popc(mk[0]) : 0) + __popc(w & ((1u << (j & 31)) - 1u));
+        src = reinterpret_cast<const uint4*>(c.kf + (static_cast<size_t>(bh) * c.vl_cap + base + below) * D);
       } else {
-        uint8_t* page = page_of(c, bh, p);
-        const uint32_t two = reinterpret_cast<const uint16_t*>(row_codes(page, 0, p))[lane];
-        const uint32_t szw = row_sz(page, 0, p)[lane >> 3];
-        const uint32_t s2 = prmt(szw, szw, 0x1010), z2 = prmt(szw, szw, 0x3232);
-        // nibbles of byte 0 -> dims 4l, 4l+1 ; byte 1 -> dims 4l+2, 4l+3
-        const uint32_t x0 = prmt(two, 0u, 0x4040);   // byte0 at bits 0..7 and 16..23
-        const uint32_t x1 = prmt(two, 0u, 0x4141);   // byte1 at bits 0..7 and 16..23
-        // low nibble -> .x, high nibble (bits 20..23) -> .y
-        const uint32_t n0 = hfma2_u(and_or(x0, 0x00F0000Fu, MAGIC), 0x2C003C00u, 0xD400E400u);
-        const uint32_t n1 = hfma2_u(and_or(x1, 0x00F0000Fu, MAGIC), 0x2C003C00u, 0xD400E400u);
-        v.x = hfma2_u(n0, s2, z2);
-        v.y = hfma2_u(n1, s2, z2);
+        const uint4* codes = reinterpret_cast<const uint4*>(row_codes(page, 0, j));
+        const uint4 sz = *reinterpret_cast<const uint4*>(row_sz(page, 0, j));
+        const uint4 cw4[4] = {codes[0], codes[1], codes[2], codes[3]};
+        const uint32_t szw[4] = {sz.x, sz.y, sz.z, sz.w};
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {  // 16 code bytes = dims 32 q4 .. 32 q4 + 31 (group q4)
+          const uint32_t s2 = prmt(szw[q4], szw[q4], 0x1010), z2 = prmt(szw[q4], szw[q4], 0x3232);
+          const uint32_t wv[4] = {cw4[q4].x, cw4[q4].y, cw4[q4].z, cw4[q4].w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {  // word k: dims 32 q4 + 8 k .. + 7
+            uint32_t h[4];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              // bytes 2e, 2e+1 at bits 0..7 and 16..23: low nibbles -> dims (4e, 4e+2),
+              // high nibbles -> dims (4e+1, 4e+3)
+              const uint32_t x = prmt(wv[k], 0u, e ? 0x4342 : 0x4140);
+              const uint32_t lo = hfma2_u(nib_lo(x), s2, z2);
+              const uint32_t hi = hfma2_u(nib_hi(x), s2, z2);
+              h[2 * e] = prmt(lo, hi, 0x5410);      // dims 4e, 4e+1
+              h[2 * e + 1] = prmt(lo, hi, 0x7632);  // dims 4e+2, 4e+3
+            }
+            *reinterpret_cast<uint4*>(stage + sw128_off(r, 4 * q4 + k, KT * 128)) = make_uint4(h[0], h[1], h[2], h[3]);
+          }
+        }
+        return;
       }
     }
-    *reinterpret_cast<uint2*>(ks + r * SROW + 8 * lane) = v;
   }
+#pragma unroll
+  for (int ch = 0; ch < 16; ++ch)
+    *reinterpret_cast<uint4*>(stage + sw128_off(r, ch, KT * 128)) = src ? src[ch] : make_uint4(0u, 0u, 0u, 0u);
 }
 
 template <bool COL>
-__global__ void __launch_bounds__(NT_SEL) select_pass(SelArgs a) {
-  extern __shared__ __align__(128) uint8_t smem[];
+__global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  __shared__ __align__(8) uint64_t kfull[2], kfree[2], tfull[4], tfree[4], drain;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+
   const hq_cache& c = a.c;
-  const int chunk = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int bh = b * c.Hkv + kvh;
   const int G = c.Hq / c.Hkv;
+  const int Mp = a.Mp;
+  const int NACC = Mp / 128;
   const SelGeo g = sel_geo(a);
   const int M = G * g.nq;
-  const int j0 = chunk * CH;
-  const int lim = COL ? g.n : g.T;  // keys scored in this pass
-  if (j0 >= lim || M == 0) return;
-
-  uint8_t* qs = smem;
-  uint8_t* ks = smem + static_cast<size_t>(M) * SROW;
-  float* colsum = reinterpret_cast<float*>(ks + CH * SROW);   // [NW_SEL][CH], one row per warp
-  float* lse_s = colsum + NW_SEL * CH;                          // [M]
-
-  // queries: row r = h * nq + i  (head kvh*G + h, position qpos0 + i)
-  for (int e = threadIdx.x; e < M * (D / 8); e += NT_SEL) {
-    const int r = e / (D / 8), ch = e % (D / 8);
-    const int h = r / g.nq, i = r % g.nq;
-    const uint4* src;
-    if (a.k_dense) {
-      src = reinterpret_cast<const uint4*>(a.q_ext + ((static_cast<size_t>(b) * c.Hq + kvh * G + h) * g.nq + i) * D) + ch;
-    } else {
-      const int p = g.qpos0 + i;
-      src = reinterpret_cast<const uint4*>(c.qbuf + ((static_cast<size_t>(b) * c.Hq + kvh * G + h) * HQ_QBUF + (p % HQ_QBUF)) * D) + ch;
-    }
-    *reinterpret_cast<uint4*>(qs + r * SROW + 16 * ch) = *src;
-  }
-  load_keys(a, g, bh, j0, ks);
-  if (COL) {
-    for (int i = threadIdx.x; i < NW_SEL * CH; i += NT_SEL) colsum[i] = 0.f;
-    for (int i = threadIdx.x; i < M; i += NT_SEL) lse_s[i] = a.lse[static_cast<size_t>(bh) * (G * HQ_QBUF) + i];
-  }
-  __syncthreads();
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gq = lane >> 2, tq = lane & 3;
-  const int nmt = (M + 15) / 16;
-  for (int mt = warp; mt < nmt; mt += NW_SEL) {
-    float acc[16][4];
-#pragma unroll
-    for (int n = 0; n < 16; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      uint32_t a0, a1, a2, a3;
-      {
-        const int row = 16 * mt + (lane & 15);
-        const int col = 16 * kk + 8 * (lane >> 4);
-        ldsm_x4(smem_u32(qs + min(row, M - 1) * SROW + 2 * col), a0, a1, a2, a3);
-      }
-#pragma unroll
-      for (int np = 0; np < 8; ++np) {
-        // keys 16np .. 16np+15: x4 = (keys 0-7, dims 0-7), (keys 0-7, dims 8-15), (keys 8-15, dims 0-7), (keys 8-15, dims 8-15)
-        uint32_t b0, b1, b2, b3;
-        const int key = 16 * np + (lane & 7) + 8 * (lane >> 4);
-        const int col = 16 * kk + 8 * ((lane >> 3) & 1);
-        ldsm_x4(smem_u32(ks + key * SROW + 2 * col), b0, b1, b2, b3);
-        mma16816(acc[2 * np], a0, a1, a2, a3, b0, b1);
-        mma16816(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
-      }
+
+  // this CTA's key tiles: pass 0 covers every visible key [0, T), pass 1 the
+  // candidates [0, n)
+  const int lim = COL ? g.n : g.T;
+  const int ntl = (lim + KT - 1) / KT;
+  const int k_lo = (split * ntl) / a.S, k_hi = ((split + 1) * ntl) / a.S;
+  const int nt = M > 0 ? k_hi - k_lo : 0;
+  // TMEM buffers: pass 0 holds NACC accumulators of 128 columns per tile,
+  // pass 1 one accumulator of Mp columns
+  const int NBUF = max(1, 4 / NACC);
+
+  uint8_t* qs = sm;                          // 2 halves x [Mp][128 B]
+  uint8_t* ks = sm + Mp * 256;               // 2 stages x KSTAGE
+  float* aux = reinterpret_cast<float*>(ks + 2 * KSTAGE);
+  int* qpos = reinterpret_cast<int*>(aux);   // [Mp] query positions
+  float* lse = aux + Mp;                     // [Mp] pass 1: log-sum-exp (exp2 domain), +inf on padding rows
+  float* xch = aux + 2 * Mp;                 // [2][Mp] pass 0 (m, l) of column half 1; pass 1 [KT] partial sums
+
+  if (threadIdx.x == 0) {
+    mbar_init(&kfull[0], BLD_WARPS * 32);
+    mbar_init(&kfull[1], BLD_WARPS * 32);
+    mbar_init(&kfree[0], 1);
+    mbar_init(&kfree[1], 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tfree[i], EPI_WARPS * 32);
     }
-    // rows of this thread: r0 = 16mt + gq, r1 = r0 + 8 ; keys 8n + 2tq + {0,1}
-    const int r0 = 16 * mt + gq, r1 = r0 + 8;
-    const int p0 = g.qpos0 + (r0 % max(g.nq, 1)), p1 = g.qpos0 + (r1 % max(g.nq, 1));
-    const bool ok0 = r0 < M, ok1 = r1 < M;
+    mbar_init(&drain, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == MMA_WARP) {
+    tmem_alloc(&tmem_base_sh, TMEM_COLS);
+    tmem_relinquish();
+  }
+  // queries: row r = h * nq + i (head kvh*G + h, position qpos0 + i); rows >= M are zero
+  for (int e = threadIdx.x; e < Mp * (D / 8); e += SEL_THREADS) {
+    const int r = e / (D / 8), ch = e % (D / 8);
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (r < M) {
+      const int h = r / g.nq, i = r % g.nq;
+      const uint4* src;
+      if (a.k_dense) {
+        src = reinterpret_cast<const uint4*>(a.q_ext + ((static_cast<size_t>(b) * c.Hq + kvh * G + h) * g.nq + i) * D) + ch;
+      } else {
+        const int p = g.qpos0 + i;
+        src = reinterpret_cast<const uint4*>(c.qbuf + ((static_cast<size_t>(b) * c.Hq + kvh * G + h) * HQ_QBUF + (p % HQ_QBUF)) * D) + ch;
+      }
+      v = *src;
+    }
+    *reinterpret_cast<uint4*>(qs + sw128_off(r, ch, Mp * 128)) = v;
+  }
+  for (int r = threadIdx.x; r < Mp; r += SEL_THREADS) qpos[r] = r < M ? g.qpos0 + r % max(g.nq, 1) : -1;
+  if (COL) {
+    // per-row log-sum-exp over the pass-0 partials of every split
+    for (int r = threadIdx.x; r < Mp; r += SEL_THREADS) {
+      float z = INFINITY;
+      if (r < M) {
+        const float* lp = a.lse_part + (static_cast<size_t>(bh) * MAX_SPLITS) * Mp * 2 + 2 * r;
+        float mm = -INFINITY;
+        for (int sp = 0; sp < a.S; ++sp) mm = fmaxf(mm, __ldcg(lp + static_cast<size_t>(sp) * Mp * 2));
+        float ll = 0.f;
+        for (int sp = 0; sp < a.S; ++sp) {
+          const float ms = __ldcg(lp + static_cast<size_t>(sp) * Mp * 2);
+          if (ms != -INFINITY) ll += __ldcg(lp + static_cast<size_t>(sp) * Mp * 2 + 1) * ex2(ms - mm);
+        }
+        z = mm + log2f(ll);
+      }
+      lse[r] = z;
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const uint32_t sbase = smem_u32(sm);
+
+  if (warp == MMA_WARP) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      const uint32_t q_s = sbase, k_s = sbase + Mp * 256;
+      bool ok = true;
+      for (int t = 0; t < nt && ok; ++t) {
+        const int s = t & 1, buf = t % NBUF;
+        ok = sel_wait(&kfull[s], (t >> 1) & 1, c.state, &abort_flag);
+        if (ok && t >= NBUF) ok = sel_wait(&tfree[buf], ((t / NBUF) - 1) & 1, c.state, &abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t kst = k_s + s * KSTAGE;
+        if (!COL) {
+          constexpr uint32_t IDESC = idesc_make(0, 0, 0, 128, KT);
+          for (int acc = 0; acc < NACC; ++acc) {
+            const uint32_t d = tmem + (buf * NACC + acc) * 128;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t ao = (kk >> 2) * (Mp * 128) + acc * 16384 + 32 * (kk & 3);
+              const uint32_t bo = (kk >> 2) * (KT * 128) + 32 * (kk & 3);
+              umma_f16(d, sdesc_sw128(q_s + ao, 16, 1024), sdesc_sw128(kst + bo, 16, 1024), IDESC, kk > 0);
+            }
+          }
+        } else {
+          for (int nh = 0; nh * 256 < Mp; ++nh) {
+            const int N = min(256, Mp - 256 * nh);
+            const uint32_t idesc = idesc_make(0, 0, 0, 128, N);
+            const uint32_t d = tmem + buf * Mp + 256 * nh;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t ao = (kk >> 2) * (KT * 128) + 32 * (kk & 3);
+              const uint32_t bo = (kk >> 2) * (Mp * 128) + nh * 256 * 128 + 32 * (kk & 3);
+              umma_f16(d, sdesc_sw128(kst + ao, 16, 1024), sdesc_sw128(q_s + bo, 16, 1024), idesc, kk > 0);
+            }
+          }
+        }
+        umma_commit(&tfull[buf]);
+        umma_commit(&kfree[s]);
+      }
+      // every MMA issued completes before TMEM is released
+      umma_commit(&drain);
+      int dummy = 0;
+      sel_wait(&drain, 0, c.state, &dummy);
+    }
+    __syncwarp();
+  } else if (warp >= EPI_WARPS) {
+    // ------------------------------------------------------------ key builders
+    const int r = threadIdx.x - EPI_WARPS * 32;
+    for (int t = 0; t < nt; ++t) {
+      const int s = t & 1;
+      if (t >= 2 && !__all_sync(0xffffffffu, sel_wait(&kfree[s], ((t >> 1) - 1) & 1, c.state, &abort_flag))) break;
+      build_key_row(a, g, bh, (k_lo + t) * KT + r, ks + s * KSTAGE, r);
+      fence_proxy_async_smem();
+      mbar_arrive(&kfull[s]);
+    }
+  } else if (COL && M == 0) {
+    // no buffered queries: every candidate's column mass is zero
+    for (int j = k_lo * KT + threadIdx.x; j < min(k_hi * KT, g.n); j += EPI_WARPS * 32)
+      a.scores[static_cast<size_t>(bh) * c.cap + j] = 0.f;
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int qd = warp & 3, hc = warp >> 2;
+    const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
     if (!COL) {
-      float m0 = -INFINITY, m1 = -INFINITY;
+      // thread: query row acc * 128 + 32 qd + lane of every accumulator, key
+      // columns [64 hc, 64 hc + 64) of each tile
+      float m_run[4], l_run[4];
 #pragma unroll
-      for (int n = 0; n < 16; ++n) {
+      for (int i = 0; i < 4; ++i) { m_run[i] = -INFINITY; l_run[i] = 0.f; }
+      for (int t = 0; t < nt; ++t) {
+        const int buf = t % NBUF;
+        if (!__all_sync(0xffffffffu, sel_wait(&tfull[buf], (t / NBUF) & 1, c.state, &abort_flag))) break;
+        tc_fence_after();
+        const int j0 = (k_lo + t) * KT + 64 * hc;
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int j = j0 + 8 * n + 2 * tq + e;
-          if (j < lim && j <= p0) m0 = fmaxf(m0, acc[n][e] * a.qscale);
-          if (j < lim && j <= p1) m1 = fmaxf(m1, acc[n][2 + e] * a.qscale);
+        for (int acc = 0; acc < 4; ++acc) {
+          if (acc >= NACC) break;
+          const int row = acc * 128 + qd * 32 + lane;
+          const int p = qpos[row];
+          // keys j0 + c visible to this row: c <= min(p, T - 1) - j0
+          const int cmax = min(p, g.T - 1) - j0;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t u[32];
+            tmem_ld32(tmem + lane_base + (buf * NACC + acc) * 128 + 64 * hc + 32 * h, u);
+            tmem_wait_ld();
+            float mx = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float x = (32 * h + e <= cmax) ? __uint_as_float(u[e]) * a.qscale : -INFINITY;
+              u[e] = __float_as_uint(x);
+              mx = fmaxf(mx, x);
+            }
+            // lazy running max: move it only when the chunk max exceeds it by > 2^8
+            if (mx > m_run[acc] + 8.0f) {
+              l_run[acc] *= ex2(m_run[acc] - mx);
+              m_run[acc] = mx;
+            }
+            const float ref = m_run[acc] == -INFINITY ? 0.f : m_run[acc];
+            float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              l0 += ex2(__uint_as_float(u[e]) - ref);
+              l1 += ex2(__uint_as_float(u[e + 1]) - ref);
+            }
+            l_run[acc] += l0 + l1;
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&tfree[buf]);
+      }
+      // merge the two column halves, then the partial (m, l) of each row
+      if (hc == 1) {
+#pragma unroll
+        for (int acc = 0; acc < 4; ++acc) {
+          if (acc >= NACC) break;
+          const int row = acc * 128 + qd * 32 + lane;
+          xch[2 * row] = m_run[acc];
+          xch[2 * row + 1] = l_run[acc];
         }
       }
-      m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
-      m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 2));
-      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 1));
-      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 2));
-      float l0 = 0.f, l1 = 0.f;
+      asm volatile("bar.sync 1, %0;" ::"r"(EPI_WARPS * 32) : "memory");
+      if (hc == 0) {
+        float* lp = a.lse_part + ((static_cast<size_t>(bh) * MAX_SPLITS + split) * Mp) * 2;
 #pragma unroll
-      for (int n = 0; n < 16; ++n) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int j = j0 + 8 * n + 2 * tq + e;
-          if (j < lim && j <= p0) l0 += ex2(acc[n][e] * a.qscale - m0);
-          if (j < lim && j <= p1) l1 += ex2(acc[n][2 + e] * a.qscale - m1);
+        for (int acc = 0; acc < 4; ++acc) {
+          if (acc >= NACC) break;
+          const int row = acc * 128 + qd * 32 + lane;
+          const float m1 = xch[2 * row], l1 = xch[2 * row + 1];
+          const float mm = fmaxf(m_run[acc], m1);
+          float ll = 0.f;
+          if (mm != -INFINITY) ll = l_run[acc] * ex2(m_run[acc] - mm) + l1 * ex2(m1 - mm);
+          lp[2 * row] = mm;
+          lp[2 * row + 1] = ll;
         }
-      }
-      l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-      l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-      if (tq == 0) {
-        float* lp = a.lse_part + (static_cast<size_t>(bh) * a.C + chunk) * (G * HQ_QBUF) * 2;
-        if (ok0) { lp[2 * r0] = m0; lp[2 * r0 + 1] = l0; }
-        if (ok1) { lp[2 * r1] = m1; lp[2 * r1 + 1] = l1; }
       }
     } else {
-      const float z0 = ok0 ? lse_s[r0] : INFINITY, z1 = ok1 ? lse_s[r1] : INFINITY;
+      // thread: key qd * 32 + lane of each tile, query columns [hc Mp/2, (hc+1) Mp/2)
+      const int half = Mp / 2;
+      for (int t = 0; t < nt; ++t) {
+        const int buf = t % NBUF;
+        if (!__all_sync(0xffffffffu, sel_wait(&tfull[buf], (t / NBUF) & 1, c.state, &abort_flag))) break;
+        tc_fence_after();
+        const int j = (k_lo + t) * KT + qd * 32 + lane;
+        // queries that may not see key j: positions < j (only near the end)
+        const bool all_see = j <= g.qpos0;
+        float sum = 0.f;
+        for (int c0 = hc * half; c0 < (hc + 1) * half; c0 += 32) {
+          uint32_t u[32];
+          tmem_ld32(tmem + lane_base + buf * Mp + c0, u);
+          tmem_wait_ld();
+          float s0 = 0.f, s1 = 0.f;
+          const float4* lz = reinterpret_cast<const float4*>(lse + c0);
+          if (all_see) {
 #pragma unroll
-      for (int n = 0; n < 16; ++n) {
+            for (int e4 = 0; e4 < 8; ++e4) {
+              const float4 z = lz[e4];
+              s0 += ex2(fmaf(__uint_as_float(u[4 * e4]), a.qscale, -z.x));
+              s1 += ex2(fmaf(__uint_as_float(u[4 * e4 + 1]), a.qscale, -z.y));
+              s0 += ex2(fmaf(__uint_as_float(u[4 * e4 + 2]), a.qscale, -z.z));
+              s1 += ex2(fmaf(__uint_as_float(u[4 * e4 + 3]), a.qscale, -z.w));
+            }
+          } else {
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int j = j0 + 8 * n + 2 * tq + e;
-          float v = 0.f;
-          if (ok0 && j < lim && j <= p0) v += ex2(acc[n][e] * a.qscale - z0);
-          if (ok1 && j < lim && j <= p1) v += ex2(acc[n][2 + e] * a.qscale - z1);
-          // sum over the 8 row-groups of the warp (lanes with equal tq)
-          v += __shfl_xor_sync(0xffffffffu, v, 4);
-          v += __shfl_xor_sync(0xffffffffu, v, 8);
-          v += __shfl_xor_sync(0xffffffffu, v, 16);
-          if (gq == 0) colsum[warp * CH + 8 * n + 2 * tq + e] += v;
+            for (int e = 0; e < 32; ++e) {
+              const float v = ex2(fmaf(__uint_as_float(u[e]), a.qscale, -lse[c0 + e]));
+              s0 += qpos[c0 + e] >= j ? v : 0.f;
+            }
+          }
+          sum += s0 + s1;
         }
+        tc_fence_before();
+        mbar_arrive(&tfree[buf]);
+        // the two column halves of key j: half 1 hands its sum over, half 0 writes
+        if (hc == 1) xch[qd * 32 + lane] = sum;
+        asm volatile("bar.sync 1, %0;" ::"r"(EPI_WARPS * 32) : "memory");
+        if (hc == 0 && j < g.n) a.scores[static_cast<size_t>(bh) * c.cap + j] = sum + xch[qd * 32 + lane];
+        asm volatile("bar.sync 1, %0;" ::"r"(EPI_WARPS * 32) : "memory");
       }
     }
   }
-  if (COL) {
-    __syncthreads();
-    for (int i = threadIdx.x; i < CH; i += NT_SEL) {
-      const int j = j0 + i;
-      if (j < lim) {
-        float tot = 0.f;
-        for (int w = 0; w < NW_SEL; ++w) tot += colsum[w * CH + i];  // fixed order: deterministic
-        a.scores[static_cast<size_t>(bh) * c.cap + j] = tot;
-      }
-    }
-  }
-}
-
-// lse (exp2 domain) per query row over the chunks that hold keys
-__global__ void lse_merge(SelArgs a) {
-  const hq_cache& c = a.c;
-  const int bh = blockIdx.x;
-  const int G = c.Hq / c.Hkv;
-  const SelGeo g = sel_geo(a);
-  const int M = G * g.nq;
-  const int nch = (g.T + CH - 1) / CH;
-  for (int r = threadIdx.x; r < M; r += blockDim.x) {
-    float mm = -INFINITY;
-    for (int ch = 0; ch < nch; ++ch) mm = fmaxf(mm, a.lse_part[((static_cast<size_t>(bh) * a.C + ch) * (G * HQ_QBUF)) * 2 + 2 * r]);
-    float ll = 0.f;
-    for (int ch = 0; ch < nch; ++ch) {
-      const float* lp = a.lse_part + ((static_cast<size_t>(bh) * a.C + ch) * (G * HQ_QBUF)) * 2 + 2 * r;
-      if (lp[0] != -INFINITY) ll += lp[1] * ex2(lp[0] - mm);
-    }
-    a.lse[static_cast<size_t>(bh) * (G * HQ_QBUF) + r] = mm + log2f(ll);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 
 constexpr int TK_THREADS = 1024;
+constexpr int TK_SMEM_MAX = 49152;  // scores held in shared memory up to this many candidates
 
 // Exact top-k by radix select over the fp32 bit patterns (scores >= 0).
+// Histograms are per warp (no cross-warp atomics), lanes of a warp that hit
+// the same bin are combined with a match before one shared atomic.
+template <bool SMEM>
 __global__ void __launch_bounds__(TK_THREADS) topk_kernel(SelArgs a) {
   const hq_cache& c = a.c;
   const int bh = blockIdx.x;
@@ -291,12 +460,18 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(SelArgs a) {
   }
   if (bh == 0 && threadIdx.x == 0) c.state[HQ_STATE_KSEL] = k;
   if (k == 0) return;
-  const uint32_t* sc = reinterpret_cast<const uint32_t*>(a.scores + static_cast<size_t>(bh) * c.cap);
+  extern __shared__ uint32_t tk_smem[];
+  const uint32_t* gsc = reinterpret_cast<const uint32_t*>(a.scores + static_cast<size_t>(bh) * c.cap);
+  const uint32_t* sc = SMEM ? tk_smem : gsc;
   int32_t* out = c.vl_sel + static_cast<size_t>(bh) * c.vl_cap;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
-  __shared__ unsigned int hist[256];
+  __shared__ unsigned int hist[TK_THREADS / 32][256];
   __shared__ unsigned int s_prefix, s_need;
   __shared__ unsigned int warp_sums[TK_THREADS / 32][2];
+  if (SMEM) {
+    for (int j = threadIdx.x; j < n; j += TK_THREADS) tk_smem[j] = __ldcg(gsc + j);
+  }
   if (threadIdx.x == 0) {
     s_prefix = 0u;
     s_need = static_cast<unsigned>(k);
@@ -304,27 +479,38 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(SelArgs a) {
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
     const uint32_t hi_mask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
-    for (int i = threadIdx.x; i < 256; i += TK_THREADS) hist[i] = 0u;
+    for (int i = lane; i < 256; i += 32) hist[warp][i] = 0u;
     __syncthreads();
     const uint32_t prefix = s_prefix;
-    for (int j = threadIdx.x; j < n; j += TK_THREADS) {
-      const uint32_t v = sc[j];
-      if ((v & hi_mask) == (prefix & hi_mask)) atomicAdd(&hist[(v >> shift) & 0xFFu], 1u);
+    for (int j0 = warp * 32; j0 < n; j0 += TK_THREADS) {
+      const int j = j0 + lane;
+      const uint32_t v = j < n ? sc[j] : 0u;
+      const bool in = j < n && (v & hi_mask) == (prefix & hi_mask);
+      const uint32_t bin = in ? ((v >> shift) & 0xFFu) : 256u;
+      const unsigned int peers = __match_any_sync(0xffffffffu, bin);
+      if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[warp][bin], static_cast<unsigned>(__popc(peers)));
+    }
+    __syncthreads();
+    // total per bin over the warps, then the bin holding the k-th largest
+    if (threadIdx.x < 256) {
+      unsigned int s = 0u;
+      for (int w = 0; w < TK_THREADS / 32; ++w) s += hist[w][threadIdx.x];
+      hist[0][threadIdx.x] = s;
     }
     __syncthreads();
     if (threadIdx.x == 0) {
       unsigned int need = s_need, acc = 0u;
       int d = 255;
       for (; d > 0; --d) {
-        if (acc + hist[d] >= need) break;
-        acc += hist[d];
+        if (acc + hist[0][d] >= need) break;
+        acc += hist[0][d];
       }
       s_prefix = prefix | (static_cast<uint32_t>(d) << shift);
       s_need = need - acc;
     }
     __syncthreads();
   }
-  const uint32_t thr = s_prefix;      // exact k-th largest value
+  const uint32_t thr = s_prefix;        // exact k-th largest value
   const unsigned int take_eq = s_need;  // how many values equal to thr to take (lowest positions first)
 
   // ordered compaction: each thread owns a contiguous segment
@@ -336,8 +522,6 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(SelArgs a) {
     cnt_gt += v > thr;
     cnt_eq += v == thr;
   }
-  // block exclusive scan of (cnt_gt, cnt_eq)
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   unsigned int x = cnt_gt, y = cnt_eq;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -372,18 +556,15 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(SelArgs a) {
   }
 }
 
+int sel_mp(const hq_cache& c) { return (((c.Hq / c.Hkv) * HQ_QBUF + 127) / 128) * 128; }
+
+size_t sel_smem_bytes(int Mp) { return 1024 + static_cast<size_t>(Mp) * 256 + 2 * KSTAGE + 4 * static_cast<size_t>(Mp) * 4; }
+
 }  // namespace
 
-size_t select_smem_bytes(const hq_cache& c) {
-  const int M = (c.Hq / c.Hkv) * HQ_QBUF;
-  return static_cast<size_t>(M) * SROW + CH * SROW + NW_SEL * CH * 4 + M * 4;
-}
-
 size_t select_workspace(const hq_cache& c, bool need_scores) {
-  const int M = (c.Hq / c.Hkv) * HQ_QBUF;
-  const int C = c.cap / CH;
-  size_t bytes = static_cast<size_t>(c.B) * c.Hkv * C * M * 2 * 4;  // lse partials
-  bytes += static_cast<size_t>(c.B) * c.Hkv * M * 4;                  // lse
+  const int Mp = sel_mp(c);
+  size_t bytes = static_cast<size_t>(c.B) * c.Hkv * MAX_SPLITS * Mp * 2 * 4;  // (m, l) partials
   if (need_scores) bytes += static_cast<size_t>(c.B) * c.Hkv * c.cap * 4;
   return (bytes + 255) & ~static_cast<size_t>(255);
 }
@@ -396,36 +577,41 @@ hq_status launch_select(const hq_cache& c, const uint16_t* kd, int L, const uint
   a.q_ext = qe;
   a.L = L;
   a.nq_init = nq;
-  const int M = (c.Hq / c.Hkv) * HQ_QBUF;
-  // init mode: keys come from the dense prefix, which may be longer than cap
-  const int keys_cap = kd ? ((L + CH - 1) / CH) * CH : c.cap;
-  a.C = keys_cap / CH;
+  a.Mp = sel_mp(c);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int units = c.B * c.Hkv;
+  int S = sms / units;
+  const int keys_cap = kd ? L : c.cap;
+  S = min(S, (keys_cap + KT - 1) / KT);
+  S = max(1, min(S, MAX_SPLITS));
+  a.S = S;
   char* w = static_cast<char*>(ws);
   a.lse_part = reinterpret_cast<float*>(w);
-  w += static_cast<size_t>(c.B) * c.Hkv * a.C * M * 2 * 4;
-  a.lse = reinterpret_cast<float*>(w);
-  w += static_cast<size_t>(c.B) * c.Hkv * M * 4;
+  w += static_cast<size_t>(c.B) * c.Hkv * MAX_SPLITS * a.Mp * 2 * 4;
   a.scores = scores_out ? scores_out : reinterpret_cast<float*>(w);
   a.qscale = (1.0f / sqrtf(static_cast<float>(D))) * LOG2E;
-  const size_t smem = select_smem_bytes(c);
-  // the attribute is raised once per device to the size of the largest group (HQ_MAX_GQA)
-  hq_cache cmax = c;
-  cmax.Hq = cmax.Hkv * HQ_MAX_GQA;
-  const int smem_max = static_cast<int>(select_smem_bytes(cmax));
-  int dev = 0;
-  cudaGetDevice(&dev);
+  const size_t smem = sel_smem_bytes(a.Mp);
   static bool attr_done[64] = {};
   if (dev >= 64 || !attr_done[dev]) {
-    if (cudaFuncSetAttribute(select_pass<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max) != cudaSuccess ||
-        cudaFuncSetAttribute(select_pass<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max) != cudaSuccess)
+    const int smem_max = static_cast<int>(sel_smem_bytes(((HQ_MAX_GQA * HQ_QBUF + 127) / 128) * 128));
+    if (cudaFuncSetAttribute(sel_pass<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max) != cudaSuccess ||
+        cudaFuncSetAttribute(sel_pass<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max) != cudaSuccess ||
+        cudaFuncSetAttribute(topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, TK_SMEM_MAX * 4) !=
+            cudaSuccess)
       return HQ_ERR_CUDA;
     if (dev < 64) attr_done[dev] = true;
   }
-  dim3 grid(a.C, c.Hkv, c.B);
-  select_pass<false><<<grid, NT_SEL, smem, st>>>(a);
-  lse_merge<<<c.B * c.Hkv, 256, 0, st>>>(a);
-  select_pass<true><<<grid, NT_SEL, smem, st>>>(a);
-  topk_kernel<<<c.B * c.Hkv, TK_THREADS, 0, st>>>(a);
+  dim3 grid(S, c.Hkv, c.B);
+  sel_pass<false><<<grid, SEL_THREADS, smem, st>>>(a);
+  sel_pass<true><<<grid, SEL_THREADS, smem, st>>>(a);
+  // candidates n <= max(keys_cap - W, 0): shared-memory top-k when they fit
+  const int n_max = max(keys_cap - c.W, 0);
+  if (n_max <= TK_SMEM_MAX)
+    topk_kernel<true><<<c.B * c.Hkv, TK_THREADS, static_cast<size_t>(max(n_max, 1)) * 4, st>>>(a);
+  else
+    topk_kernel<false><<<c.B * c.Hkv, TK_THREADS, 0, st>>>(a);
   return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 

@@ -51,7 +51,7 @@
 extern "C" {
 #endif
 
-#define HQ_ABI_VERSION 2
+#define HQ_ABI_VERSION 3
 #define HQ_HEAD_DIM 128       /* D: the only head size built */
 #define HQ_GROUP 32           /* K4V4 group length along D */
 #define HQ_STAGE 64           /* staged tokens before a merge = reselection period */
@@ -65,6 +65,7 @@ extern "C" {
 #define HQ_PAGE_KSZ 8192        /* [64][D/32] uint32 K (scale bits | zero bits << 16) */
 #define HQ_PAGE_VSZ 9216        /* [64][D/32] uint32 V (scale | zero << 16) */
 #define HQ_PAGE_VLMASK 10240    /* 2 uint32: bit r of word r/32 <=> position 64 j + r is a vertical line */
+#define HQ_PAGE_VLBASE 10248    /* int32: VL-store row of the page's first vertical line (valid when the bitmap is non-zero) */
 /* FP16 ring length for a window W: W + HQ_STAGE rounded up to a multiple of 16 */
 #define HQ_RING_LEN(W) ((((W) + HQ_STAGE) + 15) / 16 * 16)
 
@@ -110,8 +111,9 @@ enum {
  *   pages     uint8  [B, Hkv, cap/64, HQ_PAGE_BYTES]  the K4V4 store, one page per 64
  *             positions (layout HQ_PAGE_*): codes of both K and V, their per-group
  *             (scale, zero) words and the VL bitmap of the page's positions, so
- *             that one contiguous copy brings a whole page on chip; bytes
- *             10248 .. HQ_PAGE_BYTES-1 are padding
+ *             that one contiguous copy brings a whole page on chip, and the VL-store
+ *             row of the page's first vertical line; bytes 10252 .. HQ_PAGE_BYTES-1
+ *             are padding
  *   kf, vf    fp16   [B, Hkv, vl_cap, D]  VL store rows, in vl_pos order
  *   vl_pos    int32  [B, Hkv, vl_cap]     VL positions, ascending (first n_vl valid)
  *   kr, vr    fp16   [B, Hkv, R, D]       recent window + staging; position p at slot p % R
