@@ -101,56 +101,96 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int ch, int half_bytes) {
   return (ch >> 3) * half_bytes + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
 }
 
-// Build key row j of (b, kv head) bh as fp16 into row r of a key stage.
-__device__ __forceinline__ void build_key_row(const SelArgs& a, const SelGeo& g, int bh, int j, uint8_t* stage, int r) {
+// A key row fetched ahead of its conversion: packed rows bring their 64 code
+// bytes and (scale, zero) words into registers; FP16 rows (dense prefix, ring,
+// VL store) only record where to copy from.
+struct KeyRow {
+  const uint4* src;  // FP16 source row, or null
+  uint4 code[4];
+  uint4 sz;
+  bool packed;
+};
+
+__device__ __forceinline__ KeyRow fetch_key_row(const SelArgs& a, const SelGeo& g, int bh, int j) {
   const hq_cache& c = a.c;
-  const uint4* src = nullptr;
-  if (j < g.T) {
-    if (a.k_dense) {
-      src = reinterpret_cast<const uint4*>(a.k_dense + (static_cast<size_t>(bh) * a.L + j) * D);
-    } else if (j >= g.n_packed) {
-      src = reinterpret_cast<const uint4*>(c.kr + (static_cast<size_t>(bh) * ring_len(c.W) + (j % ring_len(c.W))) * D);
+  KeyRow k;
+  k.src = nullptr;
+  k.packed = false;
+  if (j >= g.T) return k;
+  if (a.k_dense) {
+    k.src = reinterpret_cast<const uint4*>(a.k_dense + (static_cast<size_t>(bh) * a.L + j) * D);
+  } else if (j >= g.n_packed) {
+    k.src = reinterpret_cast<const uint4*>(c.kr + (static_cast<size_t>(bh) * ring_len(c.W) + (j % ring_len(c.W))) * D);
+  } else {
+    uint8_t* page = page_of(c, bh, j);
+    const uint32_t* mk = page_mask(page);
+    const uint32_t w = mk[(j & 63) >> 5];
+    if ((w >> (j & 31)) & 1u) {
+      // VL row: the page records the VL-store row of its first vertical line
+      const int base = *reinterpret_cast<const int32_t*>(page + HQ_PAGE_VLBASE);
+      const int below = ((j & 63) >= 32 ? __popc(mk[0]) : 0) + __popc(w & ((1u << (j & 31)) - 1u));
+      k.src = reinterpret_cast<const uint4*>(c.kf + (static_cast<size_t>(bh) * c.vl_cap + base + below) * D);
     } else {
-      uint8_t* page = page_of(c, bh, j);
-      const uint32_t* mk = page_mask(page);
-      const uint32_t w = mk[(j & 63) >> 5];
-      if ((w >> (j & 31)) & 1u) {
-        // VL row: the page records the VL-store row of its first vertical line
-        const int base = *reinterpret_cast<const int32_t*>(page + HQ_PAGE_VLBASE);
-        const int below = ((j & 63) >= 32 ? __popc(mk[0]) : 0) + __popc(w & ((1u << (j & 31)) - 1u));
-        src = reinterpret_cast<const uint4*>(c.kf + (static_cast<size_t>(bh) * c.vl_cap + base + below) * D);
-      } else {
-        const uint4* codes = reinterpret_cast<const uint4*>(row_codes(page, 0, j));
-        const uint4 sz = *reinterpret_cast<const uint4*>(row_sz(page, 0, j));
-        const uint4 cw4[4] = {codes[0], codes[1], codes[2], codes[3]};
-        const uint32_t szw[4] = {sz.x, sz.y, sz.z, sz.w};
+      const uint4* codes = reinterpret_cast<const uint4*>(row_codes(page, 0, j));
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {  // 16 code bytes = dims 32 q4 .. 32 q4 + 31 (group q4)
-          const uint32_t s2 = prmt(szw[q4], szw[q4], 0x1010), z2 = prmt(szw[q4], szw[q4], 0x3232);
-          const uint32_t wv[4] = {cw4[q4].x, cw4[q4].y, cw4[q4].z, cw4[q4].w};
+      for (int i = 0; i < 4; ++i) k.code[i] = codes[i];
+      k.sz = *reinterpret_cast<const uint4*>(row_sz(page, 0, j));
+      k.packed = true;
+    }
+  }
+  return k;
+}
+
+// Write a fetched key row as fp16 into row r of a key stage.
+__device__ __forceinline__ void store_key_row(const KeyRow& k, uint8_t* stage, int r) {
+  if (k.packed) {
+    const uint32_t szw[4] = {k.sz.x, k.sz.y, k.sz.z, k.sz.w};
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {  // word k: dims 32 q4 + 8 k .. + 7
-            uint32_t h[4];
+    for (int q4 = 0; q4 < 4; ++q4) {  // 16 code bytes = dims 32 q4 .. 32 q4 + 31 (group q4)
+      const uint32_t s2 = prmt(szw[q4], szw[q4], 0x1010), z2 = prmt(szw[q4], szw[q4], 0x3232);
+      const uint32_t wv[4] = {k.code[q4].x, k.code[q4].y, k.code[q4].z, k.code[q4].w};
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              // bytes 2e, 2e+1 at bits 0..7 and 16..23: low nibbles -> dims (4e, 4e+2),
-              // high nibbles -> dims (4e+1, 4e+3)
-              const uint32_t x = prmt(wv[k], 0u, e ? 0x4342 : 0x4140);
-              const uint32_t lo = hfma2_u(nib_lo(x), s2, z2);
-              const uint32_t hi = hfma2_u(nib_hi(x), s2, z2);
-              h[2 * e] = prmt(lo, hi, 0x5410);      // dims 4e, 4e+1
-              h[2 * e + 1] = prmt(lo, hi, 0x7632);  // dims 4e+2, 4e+3
-            }
-            *reinterpret_cast<uint4*>(stage + sw128_off(r, 4 * q4 + k, KT * 128)) = make_uint4(h[0], h[1], h[2], h[3]);
-          }
+      for (int kk = 0; kk < 4; ++kk) {  // word kk: dims 32 q4 + 8 kk .. + 7
+        uint32_t h[4];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          // bytes 2e, 2e+1 at bits 0..7 and 16..23: low nibbles -> dims (4e, 4e+2),
+          // high nibbles -> dims (4e+1, 4e+3)
+          const uint32_t x = prmt(wv[kk], 0u, e ? 0x4342 : 0x4140);
+          const uint32_t lo = hfma2_u(nib_lo(x), s2, z2);
+          const uint32_t hi = hfma2_u(nib_hi(x), s2, z2);
+          h[2 * e] = prmt(lo, hi, 0x5410);      // dims 4e, 4e+1
+          h[2 * e + 1] = prmt(lo, hi, 0x7632);  // dims 4e+2, 4e+3
         }
-        return;
+        *reinterpret_cast<uint4*>(stage + sw128_off(r, 4 * q4 + kk, KT * 128)) = make_uint4(h[0], h[1], h[2], h[3]);
       }
     }
+    return;
   }
 #pragma unroll
   for (int ch = 0; ch < 16; ++ch)
-    *reinterpret_cast<uint4*>(stage + sw128_off(r, ch, KT * 128)) = src ? src[ch] : make_uint4(0u, 0u, 0u, 0u);
+    *reinterpret_cast<uint4*>(stage + sw128_off(r, ch, KT * 128)) = k.src ? k.src[ch] : make_uint4(0u, 0u, 0u, 0u);
+}
+
+// L2 prefetch of the key bytes of tiles [k_lo, k_hi) (a hint, clamped to the buffers)
+__device__ __forceinline__ void prefetch_keys(const SelArgs& a, const SelGeo& g, int bh, int k_lo, int k_hi) {
+  const hq_cache& c = a.c;
+  const int j0 = k_lo * KT, j1 = min(k_hi * KT, g.T);
+  if (j1 <= j0) return;
+  if (a.k_dense) {
+    const uint8_t* p = reinterpret_cast<const uint8_t*>(a.k_dense + (static_cast<size_t>(bh) * a.L + j0) * D);
+    for (int off = 0; off < (j1 - j0) * D * 2; off += 65536) prefetch_l2(p + off, min(65536, (j1 - j0) * D * 2 - off));
+    return;
+  }
+  const int p0 = j0 / HQ_PAGE_POSITIONS, p1 = min((j1 + HQ_PAGE_POSITIONS - 1) / HQ_PAGE_POSITIONS,
+                                                  (g.n_packed + HQ_PAGE_POSITIONS - 1) / HQ_PAGE_POSITIONS);
+  for (int pg = p0; pg < p1; pg += 8)  // K codes, K (scale, zero) words and the bitmap of 8 pages at a time
+    for (int q = pg; q < min(pg + 8, p1); ++q) {
+      const uint8_t* page = c.pages + (static_cast<size_t>(bh) * (c.cap / HQ_PAGE_POSITIONS) + q) * HQ_PAGE_BYTES;
+      prefetch_l2(page + HQ_PAGE_KCODES, 4096);
+      prefetch_l2(page + HQ_PAGE_KSZ, 1024);
+      prefetch_l2(page + HQ_PAGE_VLMASK, 16);
+    }
 }
 
 template <bool COL>
@@ -201,6 +241,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
     abort_flag = 0;
     fence_mbar_init();
   }
+  if (threadIdx.x == EPI_WARPS * 32 && M > 0) prefetch_keys(a, g, bh, k_lo, k_hi);
   if (warp == MMA_WARP) {
     tmem_alloc(&tmem_base_sh, TMEM_COLS);
     tmem_relinquish();
@@ -229,12 +270,15 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
       float z = INFINITY;
       if (r < M) {
         const float* lp = a.lse_part + (static_cast<size_t>(bh) * MAX_SPLITS) * Mp * 2 + 2 * r;
-        float mm = -INFINITY;
-        for (int sp = 0; sp < a.S; ++sp) mm = fmaxf(mm, __ldcg(lp + static_cast<size_t>(sp) * Mp * 2));
-        float ll = 0.f;
+        float mm = -INFINITY, ll = 0.f;
+#pragma unroll 8
         for (int sp = 0; sp < a.S; ++sp) {
-          const float ms = __ldcg(lp + static_cast<size_t>(sp) * Mp * 2);
-          if (ms != -INFINITY) ll += __ldcg(lp + static_cast<size_t>(sp) * Mp * 2 + 1) * ex2(ms - mm);
+          const float2 ml = __ldcg(reinterpret_cast<const float2*>(lp + static_cast<size_t>(sp) * Mp * 2));
+          const float mn = fmaxf(mm, ml.x);
+          if (mn != -INFINITY) {
+            ll = ll * ex2(mm - mn) + ml.y * ex2(ml.x - mn);
+            mm = mn;
+          }
         }
         z = mm + log2f(ll);
       }
@@ -295,13 +339,18 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
     __syncwarp();
   } else if (warp >= EPI_WARPS) {
     // ------------------------------------------------------------ key builders
+    // one key row per thread; the next tile's row is fetched before this one
+    // is converted, so its load latency hides behind the conversion
     const int r = threadIdx.x - EPI_WARPS * 32;
+    KeyRow cur = fetch_key_row(a, g, bh, k_lo * KT + r);
     for (int t = 0; t < nt; ++t) {
       const int s = t & 1;
+      const KeyRow nxt = t + 1 < nt ? fetch_key_row(a, g, bh, (k_lo + t + 1) * KT + r) : cur;
       if (t >= 2 && !__all_sync(0xffffffffu, sel_wait(&kfree[s], ((t >> 1) - 1) & 1, c.state, &abort_flag))) break;
-      build_key_row(a, g, bh, (k_lo + t) * KT + r, ks + s * KSTAGE, r);
+      store_key_row(cur, ks + s * KSTAGE, r);
       fence_proxy_async_smem();
       mbar_arrive(&kfull[s]);
+      cur = nxt;
     }
   } else if (COL && M == 0) {
     // no buffered queries: every candidate's column mass is zero
@@ -482,6 +531,7 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(SelArgs a) {
     for (int i = lane; i < 256; i += 32) hist[warp][i] = 0u;
     __syncthreads();
     const uint32_t prefix = s_prefix;
+    const unsigned int need = s_need;  // read before the barrier after which one thread rewrites it
     for (int j0 = warp * 32; j0 < n; j0 += TK_THREADS) {
       const int j = j0 + lane;
       const uint32_t v = j < n ? sc[j] : 0u;
@@ -491,22 +541,31 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(SelArgs a) {
       if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[warp][bin], static_cast<unsigned>(__popc(peers)));
     }
     __syncthreads();
-    // total per bin over the warps, then the bin holding the k-th largest
+    // total per bin over the warps, then the bin holding the k-th largest: with
+    // suffix sums S_d = sum of bins >= d (non-increasing in d), it is the largest
+    // d with S_d >= need (bin 0 when no bin above reaches it)
+    __shared__ unsigned int s_wtot[8];
+    unsigned int cnt = 0u, suf = 0u;
     if (threadIdx.x < 256) {
-      unsigned int s = 0u;
-      for (int w = 0; w < TK_THREADS / 32; ++w) s += hist[w][threadIdx.x];
-      hist[0][threadIdx.x] = s;
+      const int d = 255 - threadIdx.x;  // thread i owns bin 255 - i: prefix sums over threads = suffix sums over bins
+      for (int w = 0; w < TK_THREADS / 32; ++w) cnt += hist[w][d];
+      suf = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned int v = __shfl_up_sync(0xffffffffu, suf, o);
+        if (lane >= o) suf += v;
+      }
+      if (lane == 31) s_wtot[warp] = suf;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      unsigned int need = s_need, acc = 0u;
-      int d = 255;
-      for (; d > 0; --d) {
-        if (acc + hist[0][d] >= need) break;
-        acc += hist[0][d];
+    if (threadIdx.x < 256) {
+      for (int w = 0; w < warp; ++w) suf += s_wtot[w];
+      const int d = 255 - threadIdx.x;
+      const unsigned int above = suf - cnt;  // S_{d+1}
+      if ((suf >= need && above < need) || (d == 0 && suf < need)) {
+        s_prefix = prefix | (static_cast<uint32_t>(d) << shift);
+        s_need = need - above;
       }
-      s_prefix = prefix | (static_cast<uint32_t>(d) << shift);
-      s_need = need - acc;
     }
     __syncthreads();
   }
