@@ -21,19 +21,25 @@
 //                    e4m3 codes (Q, K) or the e4m3 value times the scale stored as
 //                    fp16 (V, so that P.V runs on the f16 tensor path with no
 //                    per-key scale); rows past L are zero
-//   vl_prep          VL bitmap per (b, kv head) and the VL rows of K and V gathered
-//                    into contiguous 128-row tiles (positions padded with INT_MAX)
+//   kbias_init       score bias of the e4m3 key blocks: 0, or -inf past L
+//   vl_prep          -inf bias on the vertical lines and the VL rows of K and V
+//                    gathered into contiguous 128-row tiles (positions padded with
+//                    INT_MAX)
 //   prefill_kernel   one CTA per (128-query tile, query head, batch):
 //                      warps 0-3  softmax, one query row per thread = one TMEM lane
-//                      warp 4     TMA producer (Q once; K/V tiles, 2 stages)
+//                      warp 4     TMA producers: lane 0 Q once and the K tiles (with
+//                                 their score bias or VL positions and K scales),
+//                                 lane 1 the V tiles; 2 stages each
 //                      warp 5     TMEM allocation and the tcgen05.mma issue
 //                    key tiles in order: FP8 tiles (QK on kind::f8f6f4), VL tiles
-//                    and window tiles (QK on kind::f16); S = Q K^T lands in TMEM,
-//                    the softmax reads it, writes P (fp16) to shared memory in the
-//                    128-byte-swizzled K-major layout, and O += P V (kind::f16,
-//                    V MN-major) accumulates in TMEM.  QK of tile t+1 overlaps the
-//                    softmax of tile t.  The running max is refreshed lazily (O in
-//                    TMEM is rescaled only when the max grows by more than 2^8).
+//                    and window tiles (QK on kind::f16); S = Q K^T lands in one of
+//                    two TMEM buffers, the softmax reads it, writes P (fp16) to
+//                    shared memory in the 128-byte-swizzled K-major layout, and
+//                    O += P V (kind::f16, V MN-major) accumulates in TMEM.  QK runs
+//                    two tiles ahead of the softmax; a K stage is free once its QK
+//                    is done, a V stage once its PV is.  The running max is
+//                    refreshed lazily (O in TMEM is rescaled only when the max
+//                    grows by more than 2^8).
 // All mbarrier waits are bounded (about 1 s); a timeout sets the error word and
 // the CTA drains its copies and MMAs before releasing TMEM.
 #include <climits>
@@ -50,13 +56,15 @@ constexpr float E4M3_MAX = 448.0f;
 // shared memory map (byte offsets from a 1024-byte aligned base)
 constexpr int SM_Q8 = 0;                        // Q e4m3   [128][128 B]            16 KB
 constexpr int SM_Q16 = 16384;                   // Q fp16   2 x [128][128 B]        32 KB
-constexpr int SM_KV = 49152;                    // 2 stages x (K 32 KB + V 32 KB)
-constexpr int KV_STAGE = 65536;
-constexpr int SM_P = SM_KV + 2 * KV_STAGE;      // P fp16   2 x [128][128 B]        32 KB
-constexpr int SM_AUX = SM_P + 32768;            // 2 stages x 512 B (VL bitmap or VL positions)
-constexpr int SM_USED = SM_AUX + 1024;
+constexpr int SM_K = 49152;                     // 2 K stages x 32 KB (e4m3 tiles use the first 16 KB)
+constexpr int SM_V = SM_K + 2 * 32768;          // 2 V stages x 32 KB (fp16, 2 x [128 keys][128 B])
+constexpr int SM_P = SM_V + 2 * 32768;          // P fp16   2 x [128][128 B]        32 KB
+constexpr int SM_AUX = SM_P + 32768;            // 2 K stages x 1 KB: [0,512) mask bias or VL positions, [512,528) K scales
+constexpr int AUX_STAGE = 1024;
+constexpr int SM_USED = SM_AUX + 2 * AUX_STAGE;
 constexpr int PF_SMEM = SM_USED + 1024;         // + slack for the 1024-byte alignment
-constexpr uint32_t TMEM_COLS = 256;             // S: columns 0..127, O: columns 128..255
+constexpr uint32_t TMEM_COLS = 512;             // S double buffer: columns 0..255, O: 256..383
+constexpr uint32_t TM_O = 256;
 constexpr uint32_t IDESC_QK = idesc_make(0, 0, 0, TQ, TKEY);   // K-major A and B
 constexpr uint32_t IDESC_PV = idesc_make(0, 0, 1, TQ, 128);    // A = P K-major, B = V MN-major
 
@@ -68,9 +76,9 @@ struct PfArgs {
   int B, Hq, Hkv, L, Lp, nblk, W, n_vl, nvlp;
   float qk_scale;        // sm_scale * log2(e)
   const float* sq;       // [B*Hq][nblk]
-  const float* sk;       // [B*Hkv][nblk]
-  const uint32_t* vlbits;  // [B*Hkv][Lp/32]
-  const int32_t* vlpos;    // [B*Hkv][nvlp], INT_MAX padded
+  const float* sk;       // [B*Hkv][nblk] (16-byte readable past the end)
+  const float* kbias;    // [B*Hkv][Lp]: -inf on vertical lines and past L, else 0
+  const int32_t* vlpos;  // [B*Hkv][nvlp], INT_MAX padded
   uint16_t* out;         // [B, Hq, L, D]
   uint32_t* err;         // device error word
 };
@@ -81,6 +89,7 @@ __device__ __forceinline__ bool waitb(uint64_t* bar, uint32_t parity, uint32_t* 
   const uint64_t t0 = global_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
+    if (*reinterpret_cast<volatile int*>(abort_flag)) return false;
     if (global_ns() - t0 > 1000000000ull) {
       atomicOr(err, 1u);
       *reinterpret_cast<volatile int*>(abort_flag) = 1;
@@ -124,10 +133,17 @@ __device__ __forceinline__ Sched schedule(const PfArgs& a, int bk) {
   return s;
 }
 
+// Tiles t of a CTA in order: [0, nA) e4m3 key blocks 0 .. nA-1, [nA, nA+nB) VL
+// tiles, then the window's fp16 key blocks from ktw0.  Pipeline (all waits bounded):
+//   K lane   K(t) -> K stage t%2 (+ mask bias / VL positions and the K scales)
+//   V lane   V(t) -> V stage t%2
+//   MMA      QK(t) -> S buffer t%2 (two tiles ahead of the softmax), PV(t) -> O
+//   softmax  S(t) -> P (fp16, shared memory) -> PV(t)
 __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_constant__ Tmaps tm, const PfArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  __shared__ __align__(8) uint64_t q_full, s_full, s_free, p_full, o_done, drain, kv_full[2], kv_empty[2];
+  __shared__ __align__(8) uint64_t q_full, p_full, o_done, drain, k_full[2], k_empty[2], v_full[2], v_empty[2],
+      s_full[2], s_free[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -140,14 +156,16 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
 
   if (threadIdx.x == 0) {
     mbar_init(&q_full, 1);
-    mbar_init(&s_full, 1);
-    mbar_init(&s_free, 128);
     mbar_init(&p_full, 128);
     mbar_init(&o_done, 1);
     mbar_init(&drain, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 128);
     }
     abort_flag = 0;
     fence_mbar_init();
@@ -163,7 +181,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
   const uint32_t sm_base = smem_u32(sm);
 
   if (warp == 4) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ TMA producers
+    // lane 0: Q once, then the K tiles with their auxiliary data; lane 1: the V
+    // tiles.  The two lanes wait on different barriers independently.
     if (lane == 0) {
       mbar_arrive_expect_tx(&q_full, 16384 + 32768);
       tma_load_3d(sm + SM_Q8, &tm.q8, 0, sc.q0, bq, &q_full);
@@ -172,32 +192,30 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
       int issued[2] = {0, 0};
       for (int t = 0; t < sc.nT; ++t) {
         const int s = t & 1;
-        if (t >= 2 && !waitb(&kv_empty[s], ((t >> 1) - 1) & 1, a.err, &abort_flag)) break;
-        uint8_t* K = sm + SM_KV + s * KV_STAGE;
-        uint8_t* V = K + 32768;
-        uint8_t* aux = sm + SM_AUX + s * 512;
+        // the stage is free once QK(t-2) is done and the softmax has read the
+        // stage's mask bias / VL positions / K scales of tile t-2
+        if (t >= 2 && !(waitb(&k_empty[s], ((t >> 1) - 1) & 1, a.err, &abort_flag) &&
+                        waitb(&s_free[s], ((t >> 1) - 1) & 1, a.err, &abort_flag)))
+          break;
+        uint8_t* K = sm + SM_K + s * 32768;
+        uint8_t* aux = sm + SM_AUX + s * AUX_STAGE;
         if (t < sc.nA) {
           const int kt = t;
-          mbar_arrive_expect_tx(&kv_full[s], 16384 + 32768 + 16);
-          tma_load_3d(K, &tm.k8, 0, kt * TKEY, bk, &kv_full[s]);
-          tma_load_3d(V, &tm.v8, 0, kt * TKEY, bk, &kv_full[s]);
-          tma_load_3d(V + 16384, &tm.v8, 64, kt * TKEY, bk, &kv_full[s]);
-          bulk_g2s(aux, a.vlbits + static_cast<size_t>(bk) * (a.Lp / 32) + 4 * kt, 16, &kv_full[s]);
+          mbar_arrive_expect_tx(&k_full[s], 16384 + 512 + 16);
+          tma_load_3d(K, &tm.k8, 0, kt * TKEY, bk, &k_full[s]);
+          bulk_g2s(aux, a.kbias + static_cast<size_t>(bk) * a.Lp + kt * TKEY, 512, &k_full[s]);
+          bulk_g2s(aux + 512, a.sk + ((static_cast<size_t>(bk) * a.nblk + kt) & ~static_cast<size_t>(3)), 16, &k_full[s]);
         } else if (t < sc.nA + sc.nB) {
           const int v = t - sc.nA;
-          mbar_arrive_expect_tx(&kv_full[s], 65536 + 512);
-          tma_load_3d(K, &tm.kvl, 0, v * TKEY, bk, &kv_full[s]);
-          tma_load_3d(K + 16384, &tm.kvl, 64, v * TKEY, bk, &kv_full[s]);
-          tma_load_3d(V, &tm.vvl, 0, v * TKEY, bk, &kv_full[s]);
-          tma_load_3d(V + 16384, &tm.vvl, 64, v * TKEY, bk, &kv_full[s]);
-          bulk_g2s(aux, a.vlpos + static_cast<size_t>(bk) * a.nvlp + v * TKEY, 512, &kv_full[s]);
+          mbar_arrive_expect_tx(&k_full[s], 32768 + 512);
+          tma_load_3d(K, &tm.kvl, 0, v * TKEY, bk, &k_full[s]);
+          tma_load_3d(K + 16384, &tm.kvl, 64, v * TKEY, bk, &k_full[s]);
+          bulk_g2s(aux, a.vlpos + static_cast<size_t>(bk) * a.nvlp + v * TKEY, 512, &k_full[s]);
         } else {
           const int kt = sc.ktw0 + (t - sc.nA - sc.nB);
-          mbar_arrive_expect_tx(&kv_full[s], 65536);
-          tma_load_3d(K, &tm.k16, 0, kt * TKEY, bk, &kv_full[s]);
-          tma_load_3d(K + 16384, &tm.k16, 64, kt * TKEY, bk, &kv_full[s]);
-          tma_load_3d(V, &tm.v16, 0, kt * TKEY, bk, &kv_full[s]);
-          tma_load_3d(V + 16384, &tm.v16, 64, kt * TKEY, bk, &kv_full[s]);
+          mbar_arrive_expect_tx(&k_full[s], 32768);
+          tma_load_3d(K, &tm.k16, 0, kt * TKEY, bk, &k_full[s]);
+          tma_load_3d(K + 16384, &tm.k16, 64, kt * TKEY, bk, &k_full[s]);
         }
         issued[s] = (t >> 1) + 1;
       }
@@ -205,19 +223,51 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
         // never expected: let every issued copy land before the CTA can exit
         int dummy = 0;
         for (int s = 0; s < 2; ++s)
-          if (issued[s] > 0) waitb(&kv_full[s], (issued[s] - 1) & 1, a.err, &dummy);
+          if (issued[s] > 0) waitb(&k_full[s], (issued[s] - 1) & 1, a.err, &dummy);
         waitb(&q_full, 0, a.err, &dummy);
+      }
+    } else if (lane == 1) {
+      int issued[2] = {0, 0};
+      for (int t = 0; t < sc.nT; ++t) {
+        const int s = t & 1;
+        if (t >= 2 && !waitb(&v_empty[s], ((t >> 1) - 1) & 1, a.err, &abort_flag)) break;
+        uint8_t* V = sm + SM_V + s * 32768;
+        const CUtensorMap* map;
+        int row;
+        if (t < sc.nA) {
+          map = &tm.v8;
+          row = t * TKEY;
+        } else if (t < sc.nA + sc.nB) {
+          map = &tm.vvl;
+          row = (t - sc.nA) * TKEY;
+        } else {
+          map = &tm.v16;
+          row = (sc.ktw0 + (t - sc.nA - sc.nB)) * TKEY;
+        }
+        mbar_arrive_expect_tx(&v_full[s], 32768);
+        tma_load_3d(V, map, 0, row, bk, &v_full[s]);
+        tma_load_3d(V + 16384, map, 64, row, bk, &v_full[s]);
+        issued[s] = (t >> 1) + 1;
+      }
+      if (abort_flag) {
+        int dummy = 0;
+        for (int s = 0; s < 2; ++s)
+          if (issued[s] > 0) waitb(&v_full[s], (issued[s] - 1) & 1, a.err, &dummy);
       }
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
-      const uint32_t S = tmem, O = tmem + 128;
       const uint32_t q8 = sm_base + SM_Q8, q16 = sm_base + SM_Q16, p = sm_base + SM_P;
       bool ok = waitb(&q_full, 0, a.err, &abort_flag);
-      auto issue_qk = [&](int t) {
+      // QK(t) into S buffer t%2, once K(t) landed and the softmax has read S(t-2)
+      auto issue_qk = [&](int t) -> bool {
         const int s = t & 1;
-        const uint32_t K = sm_base + SM_KV + s * KV_STAGE;
+        if (!waitb(&k_full[s], (t >> 1) & 1, a.err, &abort_flag)) return false;
+        if (t >= 2 && !waitb(&s_free[s], ((t >> 1) - 1) & 1, a.err, &abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t S = tmem + 128 * s;
+        const uint32_t K = sm_base + SM_K + s * 32768;
         if (t < sc.nA) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
@@ -229,37 +279,27 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
             umma_f16(S, sdesc_sw128(q16 + off, 16, 1024), sdesc_sw128(K + off, 16, 1024), IDESC_QK, kk > 0);
           }
         }
-        umma_commit(&s_full);
+        umma_commit(&s_full[s]);
+        umma_commit(&k_empty[s]);
+        return true;
       };
-      if (ok && sc.nT > 0) {
-        ok = waitb(&kv_full[0], 0, a.err, &abort_flag);
-        if (ok) {
-          tc_fence_after();
-          issue_qk(0);
-        }
-      }
+      if (ok && sc.nT > 0) ok = issue_qk(0);
+      if (ok && sc.nT > 1) ok = issue_qk(1);
       for (int t = 0; ok && t < sc.nT; ++t) {
         const int s = t & 1;
-        if (t + 1 < sc.nT) {
-          // QK of the next tile as soon as its K/V landed and the softmax has read S
-          ok = waitb(&kv_full[(t + 1) & 1], ((t + 1) >> 1) & 1, a.err, &abort_flag) &&
-               waitb(&s_free, t & 1, a.err, &abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          issue_qk(t + 1);
-        }
-        ok = waitb(&p_full, t & 1, a.err, &abort_flag);
+        ok = waitb(&p_full, t & 1, a.err, &abort_flag) && waitb(&v_full[s], (t >> 1) & 1, a.err, &abort_flag);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t V = sm_base + SM_KV + s * KV_STAGE + 32768;
+        const uint32_t V = sm_base + SM_V + s * 32768;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t aoff = (kk >> 2) * 16384 + 32 * (kk & 3);
-          umma_f16(O, sdesc_sw128(p + aoff, 16, 1024), sdesc_sw128(V + 2048 * kk, 16384, 1024), IDESC_PV,
+          umma_f16(tmem + TM_O, sdesc_sw128(p + aoff, 16, 1024), sdesc_sw128(V + 2048 * kk, 16384, 1024), IDESC_PV,
                    (t > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&o_done);
-        umma_commit(&kv_empty[s]);
+        umma_commit(&v_empty[s]);
+        if (t + 2 < sc.nT) ok = issue_qk(t + 2);
       }
       // every MMA this thread issued completes before TMEM is released
       umma_commit(&drain);
@@ -277,35 +317,46 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
     bool ok = true;
     for (int t = 0; t < sc.nT; ++t) {
       const int s = t & 1;
-      ok = ok && waitb(&s_full, t & 1, a.err, &abort_flag);
+      ok = ok && waitb(&s_full[s], (t >> 1) & 1, a.err, &abort_flag);
       if (!__all_sync(0xffffffffu, ok)) ok = false;
       if (!ok) break;
       tc_fence_after();
       float x[TKEY];
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        uint32_t u[32];
-        tmem_ld32(trow + 32 * c4, u);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) x[32 * c4 + e] = __uint_as_float(u[e]);
-      }
-      tc_fence_before();
-      mbar_arrive(&s_free);
+      for (int c4 = 0; c4 < 4; ++c4) tmem_ld32f(trow + 128 * s + 32 * c4, x + 32 * c4);
+      tmem_wait_ld();
 
       // scale and mask this tile's scores
-      const uint8_t* aux = sm + SM_AUX + s * 512;
+      const uint8_t* aux = sm + SM_AUX + s * AUX_STAGE;
       float mt = -INFINITY;
       if (t < sc.nA) {
         const int kt = t;
-        const float scl = sqv * a.sk[static_cast<size_t>(bk) * a.nblk + kt] * a.qk_scale;
-        const uint32_t* bits = reinterpret_cast<const uint32_t*>(aux);
-        const int jlim = min(i - a.W, a.L - 1) - kt * TKEY;  // valid columns c <= jlim (and not a vertical line)
+        const float skv = reinterpret_cast<const float*>(aux + 512)[(static_cast<size_t>(bk) * a.nblk + kt) & 3];
+        const float scl = sqv * skv * a.qk_scale;
+        const float4* bias = reinterpret_cast<const float4*>(aux);
+        const int jlim = i - a.W - kt * TKEY;  // causal limit of this row: columns c <= jlim
+        if (jlim >= TKEY - 1) {
 #pragma unroll
-        for (int c = 0; c < TKEY; ++c) {
-          const bool v = c <= jlim && !((bits[c >> 5] >> (c & 31)) & 1u);
-          x[c] = v ? x[c] * scl : -INFINITY;
-          mt = fmaxf(mt, x[c]);
+          for (int c4 = 0; c4 < TKEY / 4; ++c4) {
+            const float4 bb = bias[c4];
+            x[4 * c4] = fmaf(x[4 * c4], scl, bb.x);
+            x[4 * c4 + 1] = fmaf(x[4 * c4 + 1], scl, bb.y);
+            x[4 * c4 + 2] = fmaf(x[4 * c4 + 2], scl, bb.z);
+            x[4 * c4 + 3] = fmaf(x[4 * c4 + 3], scl, bb.w);
+            mt = fmaxf(mt, fmaxf(fmaxf(x[4 * c4], x[4 * c4 + 1]), fmaxf(x[4 * c4 + 2], x[4 * c4 + 3])));
+          }
+        } else {
+#pragma unroll
+          for (int c4 = 0; c4 < TKEY / 4; ++c4) {
+            const float4 bb = bias[c4];
+            const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = 4 * c4 + e;
+              x[c] = c <= jlim ? fmaf(x[c], scl, bv[e]) : -INFINITY;
+              mt = fmaxf(mt, x[c]);
+            }
+          }
         }
       } else if (t < sc.nA + sc.nB) {
         const int32_t* vp = reinterpret_cast<const int32_t*>(aux);
@@ -326,47 +377,50 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
           mt = fmaxf(mt, x[c]);
         }
       }
+      // S(t) is in registers and the stage's auxiliary data has been read: the S
+      // buffer and the K stage's aux area may be refilled
+      tc_fence_before();
+      mbar_arrive(&s_free[s]);
       // lazy running max: only move it (and rescale O) when it grows by > 2^8
       const bool grow = mt > m_run + 8.0f;
-      bool waited_o = false;
-      if (__any_sync(0xffffffffu, grow)) {
-        const float m_new = grow ? mt : m_run;
-        const float alpha = (grow && m_run != -INFINITY) ? ex2(m_run - m_new) : (grow ? 0.f : 1.f);
+      const bool any_grow = __any_sync(0xffffffffu, grow);
+      float alpha = 1.f;
+      if (grow) {
+        alpha = m_run != -INFINITY ? ex2(m_run - mt) : 0.f;
+        m_run = mt;
         l_run *= alpha;
-        if (t > 0) {
-          // O holds P.V of earlier tiles: rescale it once PV of tile t-1 is done
-          ok = waitb(&o_done, (t - 1) & 1, a.err, &abort_flag);
-          if (!__all_sync(0xffffffffu, ok)) ok = false;
-          if (!ok) break;
-          waited_o = true;
-          tc_fence_after();
-#pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
-            uint32_t u[32];
-            tmem_ld32(trow + 128 + 32 * c4, u);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
-            tmem_st32(trow + 128 + 32 * c4, u);
-          }
-          tmem_wait_st();
-        }
-        m_run = m_new;
       }
       // P = exp2(s - m_run) in fp16, row sum in fp32
       const float mref = m_run == -INFINITY ? 0.f : m_run;
       uint32_t pk[TKEY / 2];
+      float l0 = 0.f, l1 = 0.f;
 #pragma unroll
       for (int c = 0; c < TKEY; c += 2) {
         const float p0 = ex2(x[c] - mref), p1 = ex2(x[c + 1] - mref);
-        l_run += p0 + p1;
+        l0 += p0;
+        l1 += p1;
         pk[c / 2] = pack_f16x2(p0, p1);
       }
-      if (t > 0 && !waited_o) {
-        // the P buffer is free once PV of tile t-1 has read it
+      l_run += l0 + l1;
+      // O holds P.V of earlier tiles and the P buffer is read by PV of tile t-1:
+      // wait for it, then (if the max moved) rescale O in TMEM
+      if (t > 0) {
         ok = waitb(&o_done, (t - 1) & 1, a.err, &abort_flag);
         if (!__all_sync(0xffffffffu, ok)) ok = false;
         if (!ok) break;
+        if (any_grow) {
+          tc_fence_after();
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            uint32_t u[32];
+            tmem_ld32(trow + TM_O + 32 * c4, u);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
+            tmem_st32(trow + TM_O + 32 * c4, u);
+          }
+          tmem_wait_st();
+        }
       }
       // store P row r (K-major, 128-byte swizzle: 16-byte chunk k of the row goes
       // to chunk k ^ (r % 8) of the 128-byte line; keys 64..127 in region 1)
@@ -390,7 +444,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
         uint32_t u[32];
-        tmem_ld32(trow + 128 + 32 * c4, u);
+        tmem_ld32(trow + TM_O + 32 * c4, u);
         tmem_wait_ld();
         if (i < a.L) {
 #pragma unroll
@@ -406,7 +460,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
       }
     }
   }
-  __syncwarp();  // producer / MMA warps: lanes 1..31 wait for lane 0 before the CTA barrier
+  __syncwarp();  // producer / MMA warps: lanes wait for their issuing lanes before the CTA barrier
   tc_fence_before();
   __syncthreads();
   if (warp == 5) {
@@ -484,10 +538,19 @@ __global__ void __launch_bounds__(256) fp8_block_quant(const uint16_t* __restric
   }
 }
 
-// VL bitmap and gathered VL rows of K and V; grid (nvlp / 128, B*Hkv).  Row r of
-// (b, kv head) holds position vl_pos[r] (r < n_vl) or zeros with position INT_MAX.
+// Score bias of the e4m3 key blocks, [B*Hkv][Lp]: 0 for positions < L, -inf past L
+// (vl_prep then marks the vertical lines -inf too: they are read as fp16 tiles).
+__global__ void kbias_init(float* __restrict__ kbias, int L, int Lp, size_t n) {
+  for (size_t e = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n;
+       e += static_cast<size_t>(gridDim.x) * blockDim.x)
+    kbias[e] = static_cast<int>(e % Lp) < L ? 0.f : -INFINITY;
+}
+
+// Gathered VL rows of K and V and the -inf bias of their positions; grid
+// (nvlp / 128, B*Hkv).  Row r of (b, kv head) holds position vl_pos[r] (r < n_vl)
+// or zeros with position INT_MAX.
 __global__ void vl_prep(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v, const int32_t* __restrict__ vl_pos,
-                        int n_vl, int vl_stride, int L, int Lp, int nvlp, uint32_t* __restrict__ vlbits,
+                        int n_vl, int vl_stride, int L, int Lp, int nvlp, float* __restrict__ kbias,
                         uint16_t* __restrict__ kvl, uint16_t* __restrict__ vvl, int32_t* __restrict__ vlpos_pad) {
   const int bh = blockIdx.y;
   const int r0 = blockIdx.x * TKEY;
@@ -501,7 +564,7 @@ __global__ void vl_prep(const uint16_t* __restrict__ k, const uint16_t* __restri
         pos = p;
         kk = reinterpret_cast<const uint4*>(k + (static_cast<size_t>(bh) * L + p) * D)[ch];
         vv = reinterpret_cast<const uint4*>(v + (static_cast<size_t>(bh) * L + p) * D)[ch];
-        if (ch == 0) atomicOr(vlbits + static_cast<size_t>(bh) * (Lp / 32) + (p >> 5), 1u << (p & 31));
+        if (ch == 0) kbias[static_cast<size_t>(bh) * Lp + p] = -INFINITY;
       }
     }
     reinterpret_cast<uint4*>(kvl + (static_cast<size_t>(bh) * nvlp + r) * D)[ch] = kk;
@@ -543,7 +606,7 @@ bool make_map(CUtensorMap* m, const void* base, bool fp16, int rows, int heads, 
 }
 
 struct PfLayout {
-  size_t err, q8, k8, v8, sq, sk, sv, vlbits, kvl, vvl, vlpos, total;
+  size_t err, q8, k8, v8, sq, sk, sv, kbias, kvl, vvl, vlpos, total;
   int Lp, nblk, nvlp;
 };
 
@@ -561,7 +624,7 @@ PfLayout pf_layout(int B, int Hq, int Hkv, int L, int n_vl) {
   l.sq = o; o = al(o + static_cast<size_t>(B) * Hq * l.nblk * 4);
   l.sk = o; o = al(o + static_cast<size_t>(B) * Hkv * l.nblk * 4);
   l.sv = o; o = al(o + static_cast<size_t>(B) * Hkv * l.nblk * 4);
-  l.vlbits = o; o = al(o + static_cast<size_t>(B) * Hkv * (l.Lp / 32) * 4);
+  l.kbias = o; o = al(o + static_cast<size_t>(B) * Hkv * l.Lp * 4);
   l.kvl = o; o = al(o + static_cast<size_t>(B) * Hkv * l.nvlp * D * 2);
   l.vvl = o; o = al(o + static_cast<size_t>(B) * Hkv * l.nvlp * D * 2);
   l.vlpos = o; o = al(o + static_cast<size_t>(B) * Hkv * l.nvlp * 4);
@@ -588,7 +651,7 @@ hq_status launch_prefill(int B, int Hq, int Hkv, int L, const uint16_t* q, const
   float* sq = reinterpret_cast<float*>(w + ly.sq);
   float* sk = reinterpret_cast<float*>(w + ly.sk);
   float* sv = reinterpret_cast<float*>(w + ly.sv);
-  uint32_t* vlbits = reinterpret_cast<uint32_t*>(w + ly.vlbits);
+  float* kbias = reinterpret_cast<float*>(w + ly.kbias);
   uint16_t* kvl = reinterpret_cast<uint16_t*>(w + ly.kvl);
   uint16_t* vvl = reinterpret_cast<uint16_t*>(w + ly.vvl);
   int32_t* vlpos = reinterpret_cast<int32_t*>(w + ly.vlpos);
@@ -601,16 +664,16 @@ hq_status launch_prefill(int B, int Hq, int Hkv, int L, const uint16_t* q, const
     return HQ_ERR_CUDA;
 
   if (cudaMemsetAsync(err, 0, 16, st) != cudaSuccess) return HQ_ERR_CUDA;
-  if (cudaMemsetAsync(vlbits, 0, static_cast<size_t>(B) * Hkv * (ly.Lp / 32) * 4, st) != cudaSuccess) return HQ_ERR_CUDA;
+  kbias_init<<<256, 256, 0, st>>>(kbias, L, ly.Lp, static_cast<size_t>(B) * Hkv * ly.Lp);
   fp8_block_quant<<<dim3(ly.nblk, Hq, B), 256, 0, st>>>(q, Hq, L, ly.Lp, ly.nblk, q8, nullptr, sq);
   fp8_block_quant<<<dim3(ly.nblk, Hkv, B), 256, 0, st>>>(k, Hkv, L, ly.Lp, ly.nblk, k8, nullptr, sk);
   fp8_block_quant<<<dim3(ly.nblk, Hkv, B), 256, 0, st>>>(v, Hkv, L, ly.Lp, ly.nblk, nullptr, v8, sv);
-  vl_prep<<<dim3(ly.nvlp / TKEY, B * Hkv), 256, 0, st>>>(k, v, vl_pos, n_vl, vl_stride, L, ly.Lp, ly.nvlp, vlbits, kvl, vvl,
+  vl_prep<<<dim3(ly.nvlp / TKEY, B * Hkv), 256, 0, st>>>(k, v, vl_pos, n_vl, vl_stride, L, ly.Lp, ly.nvlp, kbias, kvl, vvl,
                                                          vlpos);
   PfArgs a;
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.L = L; a.Lp = ly.Lp; a.nblk = ly.nblk; a.W = W; a.n_vl = n_vl; a.nvlp = ly.nvlp;
   a.qk_scale = sm_scale * LOG2E;
-  a.sq = sq; a.sk = sk; a.vlbits = vlbits; a.vlpos = vlpos; a.out = out; a.err = err;
+  a.sq = sq; a.sk = sk; a.kbias = kbias; a.vlpos = vlpos; a.out = out; a.err = err;
   int dev = 0;
   cudaGetDevice(&dev);
   static bool attr_done[64] = {};
