@@ -18,6 +18,12 @@ constexpr float LOG2E = 1.4426950408889634f;
 
 __host__ __device__ __forceinline__ int ring_len(int W) { return HQ_RING_LEN(W); }
 
+// Host side: HQ_OK when e is cudaSuccess, else HQ_ERR_CUDA after recording the
+// CUDA error name and `where` for hq_last_error() (per host thread).
+hq_status cuda_status(cudaError_t e, const char* where);
+// Host side: a failure path; always HQ_ERR_CUDA, recording `where` and e.
+hq_status cuda_fail(cudaError_t e, const char* where);
+
 // K4V4 page of position p of (b, kv head) bh
 __host__ __device__ __forceinline__ uint8_t* page_of(const hq_cache& c, size_t bh, int p) {
   return c.pages + (bh * static_cast<size_t>(c.cap / HQ_PAGE_POSITIONS) + (p >> 6)) * HQ_PAGE_BYTES;

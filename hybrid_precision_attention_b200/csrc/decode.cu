@@ -712,7 +712,7 @@ hq_status launch_decode(const hq_cache& c, const uint16_t* q, const uint16_t* kn
                              2 * NC_WIDE * STAGE_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(decode_kernel<NC_NARROW, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              2 * NC_NARROW * STAGE_BYTES) != cudaSuccess)
-      return HQ_ERR_CUDA;
+      return cuda_fail(cudaGetLastError(), "decode attributes");
     if (dev < 64) attr_done[dev] = true;
   }
   unsigned int* tickets = reinterpret_cast<unsigned int*>(ws);
@@ -731,7 +731,7 @@ hq_status launch_decode(const hq_cache& c, const uint16_t* q, const uint16_t* kn
   const cudaError_t e = shp.wide
       ? cudaLaunchKernelEx(&cfg, decode_kernel<NC_WIDE, 1>, c, q, kn, vn, out, qs, shp.S, parts, tickets)
       : cudaLaunchKernelEx(&cfg, decode_kernel<NC_NARROW, 3>, c, q, kn, vn, out, qs, shp.S, parts, tickets);
-  return e == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+  return cuda_status(e, "decode launch");
 }
 
 }  // namespace hq

@@ -50,7 +50,8 @@ hq_status scratch_address(int dev, void** out) {
   std::lock_guard<std::mutex> lock(g_mu);
   if (g_scratch_addr[dev] == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return HQ_ERR_CUDA;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) return hq::cuda_fail(e, "scratch address");
     g_scratch_addr[dev] = p;
   }
   *out = g_scratch_addr[dev];
@@ -69,14 +70,16 @@ extern "C" HQ_API hq_status hq_decode_attn_noalloc(const hq_cache* c, const uint
   if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(out)) return HQ_ERR_INVALID;
   if (!(sm_scale > 0.0f)) return HQ_ERR_INVALID;
   int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) != cudaSuccess) return HQ_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return HQ_ERR_CUDA;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return hq::cuda_fail(e, "device query");
   if (hq::decode_workspace(*c, sms) > HQ_NOALLOC_SCRATCH_BYTES) return HQ_ERR_WORKSPACE;
   void* ws = nullptr;
   s = scratch_address(dev, &ws);
   if (s != HQ_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // the counters must start at zero; the rest of the scratch is written before it is read
-  if (cudaMemsetAsync(ws, 0, hq::decode_counter_bytes(*c), st) != cudaSuccess) return HQ_ERR_CUDA;
+  e = cudaMemsetAsync(ws, 0, hq::decode_counter_bytes(*c), st);
+  if (e != cudaSuccess) return hq::cuda_fail(e, "counter reset");
   return hq::launch_decode(*c, q, k_new, v_new, out, sm_scale, ws, sms, st);
 }

@@ -4,6 +4,8 @@
 // the kernels live in decode.cu, select.cu, pack_merge.cu and prefill.cu.
 #include <cuda_runtime.h>
 
+#include <cstdio>
+
 #include "common.cuh"
 
 namespace hq {
@@ -33,7 +35,23 @@ int sm_count() {
 
 }  // namespace
 
+namespace hq {
+thread_local char g_last_error[256] = "";
+hq_status cuda_status(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return HQ_OK;
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s", where, cudaGetErrorName(e));
+  return HQ_ERR_CUDA;
+}
+hq_status cuda_fail(cudaError_t e, const char* where) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s", where, e == cudaSuccess ? "driver call failed" : cudaGetErrorName(e));
+  return HQ_ERR_CUDA;
+}
+}  // namespace hq
+
 extern "C" {
+
+const char* hq_last_error(void) { return hq::g_last_error; }
+
 
 int32_t hq_abi_version(void) { return HQ_ABI_VERSION; }
 
@@ -81,11 +99,11 @@ hq_status hq_cache_reset(const hq_cache* c, hq_stream_t stream) {
   hq_status s = hq_cache_validate(c);
   if (s != HQ_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(c->state, 0, HQ_STATE_WORDS * sizeof(int32_t), st) != cudaSuccess) return HQ_ERR_CUDA;
-  if (cudaMemset2DAsync(c->pages + HQ_PAGE_VLMASK, HQ_PAGE_BYTES, 0, 8,
-                        static_cast<size_t>(c->B) * c->Hkv * (c->cap / HQ_PAGE_POSITIONS), st) != cudaSuccess)
-    return HQ_ERR_CUDA;
-  return HQ_OK;
+  cudaError_t e = cudaMemsetAsync(c->state, 0, HQ_STATE_WORDS * sizeof(int32_t), st);
+  if (e != cudaSuccess) return hq::cuda_status(e, "reset state");
+  e = cudaMemset2DAsync(c->pages + HQ_PAGE_VLMASK, HQ_PAGE_BYTES, 0, 8,
+                        static_cast<size_t>(c->B) * c->Hkv * (c->cap / HQ_PAGE_POSITIONS), st);
+  return hq::cuda_status(e, "reset bitmaps");
 }
 
 hq_status hq_select_vlines(const hq_cache* c, const uint16_t* k_dense, int32_t L, const uint16_t* q_ext, int32_t nq,

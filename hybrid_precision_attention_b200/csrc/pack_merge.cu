@@ -262,7 +262,7 @@ hq_status launch_pack_merge(const hq_cache& c, const uint16_t* kd, const uint16_
   if (init) {
     if (cudaMemset2DAsync(c.pages + HQ_PAGE_VLMASK, HQ_PAGE_BYTES, 0, 8,
                           static_cast<size_t>(c.B) * c.Hkv * (c.cap / HQ_PAGE_POSITIONS), st) != cudaSuccess)
-      return HQ_ERR_CUDA;
+      return cuda_fail(cudaGetLastError(), "merge setup");
   }
   pack_rows_kernel<<<sms * 4, threads, 0, st>>>(c, kd, vd, L, init);
   if (init) {
@@ -272,7 +272,7 @@ hq_status launch_pack_merge(const hq_cache& c, const uint16_t* kd, const uint16_
     vl_gather_kernel<<<sms * 2, threads, 0, st>>>(c, wsk, wsv);
     vl_install_kernel<<<sms, threads, 0, st>>>(c, wsk, wsv, L, 0, ticket);
   }
-  return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+  return cuda_status(cudaGetLastError(), "merge launch");
 }
 
 }  // namespace hq

@@ -43,6 +43,7 @@
 // All mbarrier waits are bounded (about 1 s); a timeout sets the error word and
 // the CTA drains its copies and MMAs before releasing TMEM.
 #include <climits>
+#include <cstdio>
 #include <cuda_fp8.h>
 
 #include "tc.cuh"
@@ -661,9 +662,9 @@ hq_status launch_prefill(int B, int Hq, int Hkv, int L, const uint16_t* q, const
       !make_map(&tm.k8, k8, false, ly.Lp, B * Hkv, 128) || !make_map(&tm.v8, v8, true, ly.Lp, B * Hkv, 64) ||
       !make_map(&tm.k16, k, true, L, B * Hkv, 64) || !make_map(&tm.v16, v, true, L, B * Hkv, 64) ||
       !make_map(&tm.kvl, kvl, true, ly.nvlp, B * Hkv, 64) || !make_map(&tm.vvl, vvl, true, ly.nvlp, B * Hkv, 64))
-    return HQ_ERR_CUDA;
+    return cuda_fail(cudaSuccess, "prefill tensor maps");
 
-  if (cudaMemsetAsync(err, 0, 16, st) != cudaSuccess) return HQ_ERR_CUDA;
+  if (cudaMemsetAsync(err, 0, 16, st) != cudaSuccess) return cuda_fail(cudaGetLastError(), "prefill setup");
   kbias_init<<<256, 256, 0, st>>>(kbias, L, ly.Lp, static_cast<size_t>(B) * Hkv * ly.Lp);
   fp8_block_quant<<<dim3(ly.nblk, Hq, B), 256, 0, st>>>(q, Hq, L, ly.Lp, ly.nblk, q8, nullptr, sq);
   fp8_block_quant<<<dim3(ly.nblk, Hkv, B), 256, 0, st>>>(k, Hkv, L, ly.Lp, ly.nblk, k8, nullptr, sk);
@@ -679,11 +680,21 @@ hq_status launch_prefill(int B, int Hq, int Hkv, int L, const uint16_t* q, const
   static bool attr_done[64] = {};
   if (dev >= 64 || !attr_done[dev]) {
     if (cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PF_SMEM) != cudaSuccess)
-      return HQ_ERR_CUDA;
+      return cuda_fail(cudaGetLastError(), "prefill setup");
     if (dev < 64) attr_done[dev] = true;
   }
   prefill_kernel<<<dim3(ly.nblk, Hq, B), PF_THREADS, PF_SMEM, st>>>(tm, a);
-  return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    // name the kernel's resources in the message (launch-resource failures)
+    cudaFuncAttributes fa;
+    char where[120] = "prefill launch";
+    if (cudaFuncGetAttributes(&fa, prefill_kernel) == cudaSuccess)
+      snprintf(where, sizeof(where), "prefill launch (regs %d, local %zu B, static smem %zu B, max threads %d)", fa.numRegs,
+               fa.localSizeBytes, fa.sharedSizeBytes, fa.maxThreadsPerBlock);
+    return cuda_fail(e, where);
+  }
+  return HQ_OK;
 }
 
 }  // namespace hq

@@ -101,13 +101,19 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int ch, int half_bytes) {
   return (ch >> 3) * half_bytes + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
 }
 
-// A key row fetched ahead of its conversion: packed rows bring their 64 code
-// bytes and (scale, zero) words into registers; FP16 rows (dense prefix, ring,
-// VL store) only record where to copy from.
+// A key row fetched ahead of its conversion.  Rows below n_packed bring their
+// 64 code bytes, (scale, zero) words, the page's bitmap word and first-VL row
+// into registers with independent loads (no branch on the bitmap before they
+// are issued); FP16 rows (dense prefix, ring) record their source, which is
+// warmed in L2 and copied to shared memory with cp.async when stored.  A
+// vertical line's FP16 row is found from the bitmap once the loads are back.
 struct KeyRow {
   const uint4* src;  // FP16 source row, or null
   uint4 code[4];
   uint4 sz;
+  uint2 mask;       // the page's bitmap words
+  int vlbase;        // VL-store row of the page's first vertical line
+  int j;             // position
   bool packed;
 };
 
@@ -116,6 +122,9 @@ __device__ __forceinline__ KeyRow fetch_key_row(const SelArgs& a, const SelGeo& 
   KeyRow k;
   k.src = nullptr;
   k.packed = false;
+  k.mask = make_uint2(0u, 0u);
+  k.vlbase = 0;
+  k.j = j;
   if (j >= g.T) return k;
   if (a.k_dense) {
     k.src = reinterpret_cast<const uint4*>(a.k_dense + (static_cast<size_t>(bh) * a.L + j) * D);
@@ -123,26 +132,43 @@ __device__ __forceinline__ KeyRow fetch_key_row(const SelArgs& a, const SelGeo& 
     k.src = reinterpret_cast<const uint4*>(c.kr + (static_cast<size_t>(bh) * ring_len(c.W) + (j % ring_len(c.W))) * D);
   } else {
     uint8_t* page = page_of(c, bh, j);
-    const uint32_t* mk = page_mask(page);
-    const uint32_t w = mk[(j & 63) >> 5];
-    if ((w >> (j & 31)) & 1u) {
-      // VL row: the page records the VL-store row of its first vertical line
-      const int base = *reinterpret_cast<const int32_t*>(page + HQ_PAGE_VLBASE);
-      const int below = ((j & 63) >= 32 ? __popc(mk[0]) : 0) + __popc(w & ((1u << (j & 31)) - 1u));
-      k.src = reinterpret_cast<const uint4*>(c.kf + (static_cast<size_t>(bh) * c.vl_cap + base + below) * D);
-    } else {
-      const uint4* codes = reinterpret_cast<const uint4*>(row_codes(page, 0, j));
+    const uint4* codes = reinterpret_cast<const uint4*>(row_codes(page, 0, j));
 #pragma unroll
-      for (int i = 0; i < 4; ++i) k.code[i] = codes[i];
-      k.sz = *reinterpret_cast<const uint4*>(row_sz(page, 0, j));
-      k.packed = true;
-    }
+    for (int i = 0; i < 4; ++i) k.code[i] = codes[i];
+    k.sz = *reinterpret_cast<const uint4*>(row_sz(page, 0, j));
+    k.mask = *reinterpret_cast<const uint2*>(page_mask(page));
+    k.vlbase = *reinterpret_cast<const int32_t*>(page + HQ_PAGE_VLBASE);
+    k.packed = true;
   }
+  if (k.src) prefetch_l2(k.src, D * 2);
   return k;
 }
 
-// Write a fetched key row as fp16 into row r of a key stage.
-__device__ __forceinline__ void store_key_row(const KeyRow& k, uint8_t* stage, int r) {
+// Source of a fetched row that must be copied as FP16 (a vertical line of a
+// packed page, or a dense / ring row); null for a row to dequantise or zero.
+__device__ __forceinline__ const uint4* key_row_src(const SelArgs& a, int bh, const KeyRow& k) {
+  if (!k.packed) return k.src;
+  const bool hi = (k.j & 63) >= 32;
+  const uint32_t w = hi ? k.mask.y : k.mask.x;
+  if (!((w >> (k.j & 31)) & 1u)) return nullptr;
+  const int below = __popc(w & ((1u << (k.j & 31)) - 1u)) + (hi ? __popc(k.mask.x) : 0);
+  return reinterpret_cast<const uint4*>(a.c.kf + (static_cast<size_t>(bh) * a.c.vl_cap + k.vlbase + below) * D);
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Write a fetched key row as fp16 into row r of a key stage (FP16 sources by
+// cp.async: the caller waits for them before publishing the stage).
+__device__ __forceinline__ void store_key_row(const SelArgs& a, int bh, const KeyRow& k, uint8_t* stage, int r) {
+  const uint4* src = key_row_src(a, bh, k);
+  if (src) {
+#pragma unroll
+    for (int ch = 0; ch < 16; ++ch) cp_async16(stage + sw128_off(r, ch, KT * 128), src + ch);
+    return;
+  }
   if (k.packed) {
     const uint32_t szw[4] = {k.sz.x, k.sz.y, k.sz.z, k.sz.w};
 #pragma unroll
@@ -168,8 +194,7 @@ __device__ __forceinline__ void store_key_row(const KeyRow& k, uint8_t* stage, i
     return;
   }
 #pragma unroll
-  for (int ch = 0; ch < 16; ++ch)
-    *reinterpret_cast<uint4*>(stage + sw128_off(r, ch, KT * 128)) = k.src ? k.src[ch] : make_uint4(0u, 0u, 0u, 0u);
+  for (int ch = 0; ch < 16; ++ch) *reinterpret_cast<uint4*>(stage + sw128_off(r, ch, KT * 128)) = make_uint4(0u, 0u, 0u, 0u);
 }
 
 // L2 prefetch of the key bytes of tiles [k_lo, k_hi) (a hint, clamped to the buffers)
@@ -347,10 +372,16 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
       const int s = t & 1;
       const KeyRow nxt = t + 1 < nt ? fetch_key_row(a, g, bh, (k_lo + t + 1) * KT + r) : cur;
       if (t >= 2 && !__all_sync(0xffffffffu, sel_wait(&kfree[s], ((t >> 1) - 1) & 1, c.state, &abort_flag))) break;
-      store_key_row(cur, ks + s * KSTAGE, r);
+      store_key_row(a, bh, cur, ks + s * KSTAGE, r);
+      cp_async_wait_all();
       fence_proxy_async_smem();
       mbar_arrive(&kfull[s]);
       cur = nxt;
+      // the next tile's loads are back by now: warm L2 with its vertical lines' rows
+      if (t + 1 < nt && cur.packed) {
+        const uint4* vsrc = key_row_src(a, bh, cur);
+        if (vsrc) prefetch_l2(vsrc, D * 2);
+      }
     }
   } else if (COL && M == 0) {
     // no buffered queries: every candidate's column mass is zero
@@ -487,12 +518,33 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
 }
 
 constexpr int TK_THREADS = 1024;
-constexpr int TK_SMEM_MAX = 49152;  // scores held in shared memory up to this many candidates
+constexpr int TK_VPT = 48;                          // candidates per thread held in registers
+constexpr int TK_SMEM_MAX = TK_THREADS * TK_VPT;    // 49152 candidates
 
-// Exact top-k by radix select over the fp32 bit patterns (scores >= 0).
-// Histograms are per warp (no cross-warp atomics), lanes of a warp that hit
-// the same bin are combined with a match before one shared atomic.
-template <bool SMEM>
+// shared-memory slot of candidate j: one pad word per 32, so that threads owning
+// consecutive 48-candidate segments read distinct banks
+__device__ __forceinline__ int tk_slot(int j) { return j + (j >> 5); }
+
+// block-wide sum of one value per thread (1024 threads); every thread gets it
+__device__ __forceinline__ unsigned int tk_block_sum(unsigned int v, unsigned int* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = __reduce_add_sync(0xffffffffu, v);
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  const unsigned int tot = __reduce_add_sync(0xffffffffu, red[lane]);
+  __syncthreads();
+  return tot;
+}
+
+// Exact top-k of the column-mass scores of one (b, kv head).  Scores are >= 0,
+// so their fp32 bit patterns order like the values.  The k-th largest pattern
+// is found bit by bit from the top (keep a bit when at least k candidates are
+// >= the pattern with it set); each thread holds a contiguous segment of the
+// candidates in registers, so every step is register compares and one block
+// sum.  An ordered compaction then writes the chosen positions ascending, ties
+// at the threshold to the lowest positions.  Beyond TK_SMEM_MAX candidates
+// (REG = false) the same steps re-read the scores from global memory.
+template <bool REG>
 __global__ void __launch_bounds__(TK_THREADS) topk_kernel(SelArgs a) {
   const hq_cache& c = a.c;
   const int bh = blockIdx.x;
@@ -510,77 +562,52 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(SelArgs a) {
   if (bh == 0 && threadIdx.x == 0) c.state[HQ_STATE_KSEL] = k;
   if (k == 0) return;
   extern __shared__ uint32_t tk_smem[];
+  __shared__ unsigned int red[32];
   const uint32_t* gsc = reinterpret_cast<const uint32_t*>(a.scores + static_cast<size_t>(bh) * c.cap);
-  const uint32_t* sc = SMEM ? tk_smem : gsc;
   int32_t* out = c.vl_sel + static_cast<size_t>(bh) * c.vl_cap;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
-  __shared__ unsigned int hist[TK_THREADS / 32][256];
-  __shared__ unsigned int s_prefix, s_need;
-  __shared__ unsigned int warp_sums[TK_THREADS / 32][2];
-  if (SMEM) {
-    for (int j = threadIdx.x; j < n; j += TK_THREADS) tk_smem[j] = __ldcg(gsc + j);
-  }
-  if (threadIdx.x == 0) {
-    s_prefix = 0u;
-    s_need = static_cast<unsigned>(k);
-  }
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    const uint32_t hi_mask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
-    for (int i = lane; i < 256; i += 32) hist[warp][i] = 0u;
+  const int per = (n + TK_THREADS - 1) / TK_THREADS;  // <= TK_VPT when REG
+  const int lo = threadIdx.x * per, cnt = max(0, min(per, n - lo));
+  uint32_t v[REG ? TK_VPT : 1];
+  if (REG) {
+    for (int j = threadIdx.x; j < n; j += TK_THREADS) tk_smem[tk_slot(j)] = __ldcg(gsc + j);
     __syncthreads();
-    const uint32_t prefix = s_prefix;
-    const unsigned int need = s_need;  // read before the barrier after which one thread rewrites it
-    for (int j0 = warp * 32; j0 < n; j0 += TK_THREADS) {
-      const int j = j0 + lane;
-      const uint32_t v = j < n ? sc[j] : 0u;
-      const bool in = j < n && (v & hi_mask) == (prefix & hi_mask);
-      const uint32_t bin = in ? ((v >> shift) & 0xFFu) : 256u;
-      const unsigned int peers = __match_any_sync(0xffffffffu, bin);
-      if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[warp][bin], static_cast<unsigned>(__popc(peers)));
-    }
-    __syncthreads();
-    // total per bin over the warps, then the bin holding the k-th largest: with
-    // suffix sums S_d = sum of bins >= d (non-increasing in d), it is the largest
-    // d with S_d >= need (bin 0 when no bin above reaches it)
-    __shared__ unsigned int s_wtot[8];
-    unsigned int cnt = 0u, suf = 0u;
-    if (threadIdx.x < 256) {
-      const int d = 255 - threadIdx.x;  // thread i owns bin 255 - i: prefix sums over threads = suffix sums over bins
-      for (int w = 0; w < TK_THREADS / 32; ++w) cnt += hist[w][d];
-      suf = cnt;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const unsigned int v = __shfl_up_sync(0xffffffffu, suf, o);
-        if (lane >= o) suf += v;
-      }
-      if (lane == 31) s_wtot[warp] = suf;
-    }
-    __syncthreads();
-    if (threadIdx.x < 256) {
-      for (int w = 0; w < warp; ++w) suf += s_wtot[w];
-      const int d = 255 - threadIdx.x;
-      const unsigned int above = suf - cnt;  // S_{d+1}
-      if ((suf >= need && above < need) || (d == 0 && suf < need)) {
-        s_prefix = prefix | (static_cast<uint32_t>(d) << shift);
-        s_need = need - above;
-      }
-    }
-    __syncthreads();
+    for (int e = 0; e < (REG ? TK_VPT : 1); ++e) v[e] = e < cnt ? tk_smem[tk_slot(lo + e)] : 0u;
   }
-  const uint32_t thr = s_prefix;        // exact k-th largest value
-  const unsigned int take_eq = s_need;  // how many values equal to thr to take (lowest positions first)
 
-  // ordered compaction: each thread owns a contiguous segment
-  const int per = (n + TK_THREADS - 1) / TK_THREADS;
-  const int lo = threadIdx.x * per, hi = min(n, lo + per);
-  unsigned int cnt_gt = 0, cnt_eq = 0;
-  for (int j = lo; j < hi; ++j) {
-    const uint32_t v = sc[j];
-    cnt_gt += v > thr;
-    cnt_eq += v == thr;
+  uint32_t thr = 0u;
+  for (int bit = 30; bit >= 0; --bit) {  // bit 31 (sign) is 0 for every score
+    const uint32_t cand = thr | (1u << bit);
+    unsigned int ge = 0u;
+    if (REG) {
+#pragma unroll
+      for (int e = 0; e < (REG ? TK_VPT : 1); ++e) ge += (e < cnt && v[e] >= cand) ? 1u : 0u;
+    } else {
+      for (int j = threadIdx.x; j < n; j += TK_THREADS) ge += __ldcg(gsc + j) >= cand ? 1u : 0u;
+    }
+    if (tk_block_sum(ge, red) >= static_cast<unsigned>(k)) thr = cand;
   }
+  // thr is the exact k-th largest value: take every value above it and the
+  // lowest-positioned (k - #above) of those equal to it
+  unsigned int cnt_gt = 0u, cnt_eq = 0u;
+  if (REG) {
+#pragma unroll
+    for (int e = 0; e < (REG ? TK_VPT : 1); ++e) {
+      cnt_gt += (e < cnt && v[e] > thr) ? 1u : 0u;
+      cnt_eq += (e < cnt && v[e] == thr) ? 1u : 0u;
+    }
+  } else {
+    for (int e = 0; e < cnt; ++e) {
+      const uint32_t x = __ldcg(gsc + lo + e);
+      cnt_gt += x > thr ? 1u : 0u;
+      cnt_eq += x == thr ? 1u : 0u;
+    }
+  }
+  const unsigned int take_eq = static_cast<unsigned>(k) - tk_block_sum(cnt_gt, red);
+  // block exclusive scan of (cnt_gt, cnt_eq) in thread (= position) order
+  __shared__ unsigned int warp_sums[TK_THREADS / 32][2];
   unsigned int x = cnt_gt, y = cnt_eq;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -590,30 +617,35 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(SelArgs a) {
   if (lane == 31) { warp_sums[warp][0] = x; warp_sums[warp][1] = y; }
   __syncthreads();
   if (warp == 0) {
-    unsigned int wx = lane < TK_THREADS / 32 ? warp_sums[lane][0] : 0u;
-    unsigned int wy = lane < TK_THREADS / 32 ? warp_sums[lane][1] : 0u;
+    unsigned int wx = warp_sums[lane][0], wy = warp_sums[lane][1];
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const unsigned int xo = __shfl_up_sync(0xffffffffu, wx, o), yo = __shfl_up_sync(0xffffffffu, wy, o);
       if (lane >= o) { wx += xo; wy += yo; }
     }
-    if (lane < TK_THREADS / 32) { warp_sums[lane][0] = wx; warp_sums[lane][1] = wy; }
+    warp_sums[lane][0] = wx;
+    warp_sums[lane][1] = wy;
   }
   __syncthreads();
   unsigned int ex_gt = x - cnt_gt + (warp > 0 ? warp_sums[warp - 1][0] : 0u);
   unsigned int ex_eq = y - cnt_eq + (warp > 0 ? warp_sums[warp - 1][1] : 0u);
   // output slot of position j = (#gt before j) + min(#eq before j, take_eq)
-  for (int j = lo; j < hi; ++j) {
-    const uint32_t v = sc[j];
-    if (v > thr) {
+#pragma unroll
+  for (int e = 0; e < (REG ? TK_VPT : 1 << 30); ++e) {
+    if (e >= cnt) break;
+    const int j = lo + e;
+    const uint32_t x = REG ? v[REG ? e : 0] : __ldcg(gsc + j);
+    if (x > thr) {
       out[ex_gt + min(ex_eq, take_eq)] = j;
       ++ex_gt;
-    } else if (v == thr) {
+    } else if (x == thr) {
       if (ex_eq < take_eq) out[ex_gt + ex_eq] = j;
       ++ex_eq;
     }
   }
 }
+
+int tk_slot_host(int n) { return n + (n >> 5) + 1; }
 
 int sel_mp(const hq_cache& c) { return (((c.Hq / c.Hkv) * HQ_QBUF + 127) / 128) * 128; }
 
@@ -657,21 +689,21 @@ hq_status launch_select(const hq_cache& c, const uint16_t* kd, int L, const uint
     const int smem_max = static_cast<int>(sel_smem_bytes(((HQ_MAX_GQA * HQ_QBUF + 127) / 128) * 128));
     if (cudaFuncSetAttribute(sel_pass<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max) != cudaSuccess ||
         cudaFuncSetAttribute(sel_pass<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max) != cudaSuccess ||
-        cudaFuncSetAttribute(topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, TK_SMEM_MAX * 4) !=
-            cudaSuccess)
-      return HQ_ERR_CUDA;
+        cudaFuncSetAttribute(topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(tk_slot_host(TK_SMEM_MAX)) * 4) != cudaSuccess)
+      return cuda_fail(cudaGetLastError(), "select setup");
     if (dev < 64) attr_done[dev] = true;
   }
   dim3 grid(S, c.Hkv, c.B);
   sel_pass<false><<<grid, SEL_THREADS, smem, st>>>(a);
   sel_pass<true><<<grid, SEL_THREADS, smem, st>>>(a);
-  // candidates n <= max(keys_cap - W, 0): shared-memory top-k when they fit
+  // candidates n <= max(keys_cap - W, 0): held in registers when they fit
   const int n_max = max(keys_cap - c.W, 0);
   if (n_max <= TK_SMEM_MAX)
-    topk_kernel<true><<<c.B * c.Hkv, TK_THREADS, static_cast<size_t>(max(n_max, 1)) * 4, st>>>(a);
+    topk_kernel<true><<<c.B * c.Hkv, TK_THREADS, static_cast<size_t>(tk_slot_host(max(n_max, 1))) * 4, st>>>(a);
   else
     topk_kernel<false><<<c.B * c.Hkv, TK_THREADS, 0, st>>>(a);
-  return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+  return cuda_status(cudaGetLastError(), "select launch");
 }
 
 }  // namespace hq

@@ -53,6 +53,8 @@ _CP = ctypes.POINTER(HqCacheStruct)
 _lib.hq_abi_version.restype = _I
 _lib.hq_status_str.restype = ctypes.c_char_p
 _lib.hq_status_str.argtypes = [_I]
+_lib.hq_last_error.restype = ctypes.c_char_p
+_lib.hq_last_error.argtypes = []
 _lib.hq_cache_validate.restype = _I
 _lib.hq_cache_validate.argtypes = [_CP]
 _lib.hq_workspace_bytes.restype = _S
@@ -72,14 +74,15 @@ _lib.hq_prefill_workspace_bytes.argtypes = [_I, _I, _I, _I, _I]
 _lib.hq_prefill_attn.restype = _I
 _lib.hq_prefill_attn.argtypes = [_I, _I, _I, _I, _I, _P, _P, _P, _P, _I, _I, _I, ctypes.c_float, _P, _P, _S, _P]
 
-EXPORTED = ("hq_abi_version", "hq_status_str", "hq_cache_validate", "hq_workspace_bytes", "hq_cache_reset",
+EXPORTED = ("hq_abi_version", "hq_status_str", "hq_last_error", "hq_cache_validate", "hq_workspace_bytes", "hq_cache_reset",
             "hq_select_vlines", "hq_pack_merge", "hq_decode_attn", "hq_decode_attn_noalloc",
             "hq_prefill_workspace_bytes", "hq_prefill_attn")
 
 
 def _check(st: int, what: str):
     if st != 0:
-        raise HqError(f"{what}: {_lib.hq_status_str(st).decode()} (status {st})")
+        detail = f" [{_lib.hq_last_error().decode()}]" if st == 5 else ""
+        raise HqError(f"{what}: {_lib.hq_status_str(st).decode()} (status {st}){detail}")
 
 
 def _ptr(t):

@@ -148,6 +148,11 @@ enum { HQ_OP_SELECT = 0, HQ_OP_MERGE = 1, HQ_OP_DECODE = 2 };
 HQ_API int32_t hq_abi_version(void);
 HQ_API const char* hq_status_str(hq_status s);
 
+/* After a call returned HQ_ERR_CUDA: which step failed and the CUDA error name
+ * (e.g. "prefill launch: cudaErrorLaunchOutOfResources").  Per host thread;
+ * the string stays valid until the next failing call on that thread. */
+HQ_API const char* hq_last_error(void);
+
 /* Host-side check of a cache descriptor (shapes, limits, 16-byte alignment of
  * every pointer).  Returns HQ_OK or HQ_ERR_INVALID / HQ_ERR_UNSUPPORTED. */
 HQ_API hq_status hq_cache_validate(const hq_cache* c);

@@ -16,7 +16,8 @@ def _declared():
 def test_header_declares_the_entry_points():
     names = _declared()
     for n in ("hq_select_vlines", "hq_pack_merge", "hq_decode_attn", "hq_prefill_attn", "hq_workspace_bytes",
-              "hq_prefill_workspace_bytes", "hq_status_str", "hq_cache_validate", "hq_cache_reset", "hq_abi_version"):
+              "hq_prefill_workspace_bytes", "hq_status_str", "hq_last_error", "hq_cache_validate", "hq_cache_reset",
+              "hq_abi_version"):
         assert n in names
 
 
