@@ -52,20 +52,24 @@ namespace hq {
 namespace {
 
 constexpr int TQ = 128, TKEY = 128;
-constexpr int PF_THREADS = 192;
+constexpr int PF_THREADS = 320;                 // 2 softmax warpgroups, a TMA warp, an MMA warp
+constexpr int W_TMA = 8, W_MMA = 9;
 constexpr float E4M3_MAX = 448.0f;
-// shared memory map (byte offsets from a 1024-byte aligned base)
-constexpr int SM_Q8 = 0;                        // Q e4m3   [128][128 B]            16 KB
-constexpr int SM_Q16 = 16384;                   // Q fp16   2 x [128][128 B]        32 KB
-constexpr int SM_K = 49152;                     // 2 K stages x 32 KB (e4m3 tiles use the first 16 KB)
-constexpr int SM_V = SM_K + 2 * 32768;          // 2 V stages x 32 KB (fp16, 2 x [128 keys][128 B])
-constexpr int SM_P = SM_V + 2 * 32768;          // P fp16   2 x [128][128 B]        32 KB
-constexpr int SM_AUX = SM_P + 32768;            // 2 K stages x 1 KB: [0,512) mask bias or VL positions, [512,528) K scales
-constexpr int AUX_STAGE = 1024;
-constexpr int SM_USED = SM_AUX + 2 * AUX_STAGE;
+// shared memory map (byte offsets from a 1024-byte aligned base); the CTA holds
+// two query tiles (A: rows q0 .. q0+127, B: q0+128 .. q0+255) that share every
+// K / V tile.  The fp16 query tiles are needed only by the fp16 key tiles, which
+// come first; afterwards their 64 KB hold a second K / V stage.
+constexpr int SM_Q8 = 0;                        // Q e4m3  2 tiles x [128][128 B]             32 KB
+constexpr int SM_Q16 = 32768;                   // Q fp16  2 tiles x 2 x [128][128 B]         64 KB  (later K / V stage 1)
+constexpr int SM_K = SM_Q16 + 65536;            // K stage 0 (e4m3 tiles use the first 16 KB)  32 KB
+constexpr int SM_V = SM_K + 32768;              // V stage 0 fp16 2 x [128 keys][128 B]        32 KB
+constexpr int SM_P = SM_V + 32768;              // P fp16  2 tiles x 2 x [128][128 B]          64 KB
+constexpr int SM_AUX = SM_P + 65536;            // 2 stages x 512 B: mask bias (e4m3 tiles) or VL positions
+constexpr int SM_KS = SM_AUX + 1024;            // 2 stages x 16 B: the 16-byte chunk holding the e4m3 tile's K scale
+constexpr int SM_USED = SM_KS + 32;
 constexpr int PF_SMEM = SM_USED + 1024;         // + slack for the 1024-byte alignment
-constexpr uint32_t TMEM_COLS = 512;             // S double buffer: columns 0..255, O: 256..383
-constexpr uint32_t TM_O = 256;
+constexpr uint32_t TMEM_COLS = 512;             // S_A 0..127, S_B 128..255, O_A 256..383, O_B 384..511
+constexpr uint32_t TM_S = 0, TM_O = 256;
 constexpr uint32_t IDESC_QK = idesc_make(0, 0, 0, TQ, TKEY);   // K-major A and B
 constexpr uint32_t IDESC_PV = idesc_make(0, 0, 1, TQ, 128);    // A = P K-major, B = V MN-major
 
@@ -99,9 +103,9 @@ __device__ __forceinline__ bool waitb(uint64_t* bar, uint32_t parity, uint32_t* 
   }
 }
 
-// per-CTA tile schedule
+// per-CTA tile schedule (the union of what the two query tiles need)
 struct Sched {
-  int qt, q0, imax, nA, nB, nC, ktw0, nvv, nT;
+  int pr, q0, imax, nA, nB, nC, ktw0, nvv, nT;
 };
 
 __device__ __forceinline__ int count_le(const int32_t* a, int n, int key) {
@@ -115,10 +119,10 @@ __device__ __forceinline__ int count_le(const int32_t* a, int n, int key) {
 
 __device__ __forceinline__ Sched schedule(const PfArgs& a, int bk) {
   Sched s;
-  s.qt = gridDim.x - 1 - blockIdx.x;  // longest rows first
-  s.q0 = s.qt * TQ;
-  s.imax = min(s.q0 + TQ - 1, a.L - 1);
-  const int jmax = s.imax - a.W;  // largest key any row of the tile sees outside its window
+  s.pr = gridDim.x - 1 - blockIdx.x;  // longest rows first
+  s.q0 = s.pr * 2 * TQ;
+  s.imax = min(s.q0 + 2 * TQ - 1, a.L - 1);
+  const int jmax = s.imax - a.W;  // largest key any row of the pair sees outside its window
   s.nA = jmax >= 0 ? jmax / TKEY + 1 : 0;
   s.nvv = jmax >= 0 ? count_le(a.vlpos + static_cast<size_t>(bk) * a.nvlp, a.n_vl, jmax) : 0;
   s.nB = (s.nvv + TKEY - 1) / TKEY;
@@ -134,17 +138,97 @@ __device__ __forceinline__ Sched schedule(const PfArgs& a, int bk) {
   return s;
 }
 
-// Tiles t of a CTA in order: [0, nA) e4m3 key blocks 0 .. nA-1, [nA, nA+nB) VL
-// tiles, then the window's fp16 key blocks from ktw0.  Pipeline (all waits bounded):
-//   K lane   K(t) -> K stage t%2 (+ mask bias / VL positions and the K scales)
-//   V lane   V(t) -> V stage t%2
-//   MMA      QK(t) -> S buffer t%2 (two tiles ahead of the softmax), PV(t) -> O
-//   softmax  S(t) -> P (fp16, shared memory) -> PV(t)
+// Tile order of a CTA: [0, nB) VL tiles, [nB, nF) the window's fp16 key blocks
+// from ktw0 (nF = nB + nC), then [nF, nT) the e4m3 key blocks 0 .. nA-1.
+// Stages: the fp16 tiles all use stage 0; e4m3 tile nF + j uses stage j % 2
+// (stage 1 lives where the fp16 query tiles were).  use = how many tiles used
+// the stage before this one (its barrier phase).
+struct TileSlot {
+  int stage, use, prev;  // prev: the tile that used the stage before (-1: none)
+};
+__device__ __forceinline__ TileSlot slot_of(int t, int nF) {
+  TileSlot z;
+  if (t < nF) {
+    z.stage = 0;
+    z.use = t;
+    z.prev = t - 1;
+  } else {
+    const int j = t - nF;
+    z.stage = j & 1;
+    z.use = z.stage == 0 ? nF + j / 2 : j / 2;
+    z.prev = j >= 2 ? t - 2 : (z.stage == 0 ? nF - 1 : -1);
+  }
+  return z;
+}
+
+// Scale and mask 32 scores of row i (columns c0 .. c0+31 of tile t) in place;
+// returns their max.  Columns a row must not see become -inf.
+__device__ __forceinline__ float scale_mask32(float (&x)[32], int c0, int t, const Sched& sc, const PfArgs& a,
+                                              const uint8_t* aux, float scl, int i) {
+  float mt = -INFINITY;
+  const int nF = sc.nB + sc.nC;
+  if (t >= nF) {
+    float bv[32];
+#pragma unroll
+    for (int c4 = 0; c4 < 8; ++c4) {
+      const float4 bb = reinterpret_cast<const float4*>(aux)[c0 / 4 + c4];
+      bv[4 * c4] = bb.x;
+      bv[4 * c4 + 1] = bb.y;
+      bv[4 * c4 + 2] = bb.z;
+      bv[4 * c4 + 3] = bb.w;
+    }
+    const int jlim = i - a.W - (t - nF) * TKEY - c0;  // causal limit: local columns c <= jlim
+    float m2[2] = {-INFINITY, -INFINITY};
+    if (jlim >= 31) {
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        x[c] = fmaf(x[c], scl, bv[c]);
+        m2[c & 1] = fmaxf(m2[c & 1], x[c]);
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        x[c] = c <= jlim ? fmaf(x[c], scl, bv[c]) : -INFINITY;
+        m2[c & 1] = fmaxf(m2[c & 1], x[c]);
+      }
+    }
+    mt = fmaxf(m2[0], m2[1]);
+  } else if (t < sc.nB) {
+    const int32_t* vp = reinterpret_cast<const int32_t*>(aux) + c0;
+    const int lim = i - a.W;
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      x[c] = vp[c] <= lim ? x[c] * a.qk_scale : -INFINITY;
+      mt = fmaxf(mt, x[c]);
+    }
+  } else {
+    const int kt = sc.ktw0 + (t - sc.nB);
+    const int lo = i - a.W + 1 - kt * TKEY - c0, hi = i - kt * TKEY - c0;  // window: lo <= c <= hi
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      x[c] = (c >= lo && c <= hi) ? x[c] * a.qk_scale : -INFINITY;
+      mt = fmaxf(mt, x[c]);
+    }
+  }
+  return mt;
+}
+
+// Per tile (all waits bounded):
+//   K lane   K(t) + aux into its stage once QK_A, QK_B of the stage's previous
+//            tile are done and both softmax groups have read that tile's aux
+//   V lane   V(t) into its stage once PV_A, PV_B of the stage's previous tile are done
+//   MMA      event-driven: QK_g(t) when K(t) landed and group g has read S_g(t-1);
+//            PV_g(t) when P_g(t) and V(t) landed
+//   softmax  group g, one pass over S_g(t): scale, mask, exp2 against the
+//            running max, P_g(t) to shared memory; only when a row's tile max
+//            exceeds its running max by more than 2^8 (every row's first
+//            tile, rarely later) is the pass redone with the new max and O_g
+//            rescaled
 __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_constant__ Tmaps tm, const PfArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  __shared__ __align__(8) uint64_t q_full, p_full, o_done, drain, k_full[2], k_empty[2], v_full[2], v_empty[2],
-      s_full[2], s_free[2];
+  __shared__ __align__(8) uint64_t q_full, q16_free, drain, k_full[2], k_empty[2], aux_free[2], v_full[2], v_empty[2],
+      s_full[2], s_free[2], p_full[2], o_done[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -154,24 +238,27 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
   const int bq = b * a.Hq + hq, bk = b * a.Hkv + kvh;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Sched sc = schedule(a, bk);
+  const int nF = sc.nB + sc.nC;
 
   if (threadIdx.x == 0) {
     mbar_init(&q_full, 1);
-    mbar_init(&p_full, 128);
-    mbar_init(&o_done, 1);
+    mbar_init(&q16_free, 1);
     mbar_init(&drain, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&k_full[i], 1);
-      mbar_init(&k_empty[i], 1);
-      mbar_init(&v_full[i], 1);
-      mbar_init(&v_empty[i], 1);
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&k_full[g], 1);
+      mbar_init(&k_empty[g], 1);
+      mbar_init(&aux_free[g], 256);
+      mbar_init(&v_full[g], 1);
+      mbar_init(&v_empty[g], 1);
+      mbar_init(&s_full[g], 1);
+      mbar_init(&s_free[g], 128);
+      mbar_init(&p_full[g], 128);
+      mbar_init(&o_done[g], 1);
     }
     abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == W_MMA) {
     tmem_alloc(&tmem_base_sh, TMEM_COLS);
     tmem_relinquish();
   }
@@ -180,127 +267,175 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
   const uint32_t sm_base = smem_u32(sm);
+  auto k_stage = [&](int st) -> uint32_t { return st == 0 ? SM_K : SM_Q16; };
+  auto v_stage = [&](int st) -> uint32_t { return st == 0 ? SM_V : SM_Q16 + 32768; };
 
-  if (warp == 4) {
+  if (warp == W_TMA) {
     // ------------------------------------------------------------ TMA producers
-    // lane 0: Q once, then the K tiles with their auxiliary data; lane 1: the V
-    // tiles.  The two lanes wait on different barriers independently.
+    // lane 0: both query tiles once, then the K tiles with their auxiliary data;
+    // lane 1: the V tiles.  The two lanes wait on different barriers.
     if (lane == 0) {
-      mbar_arrive_expect_tx(&q_full, 16384 + 32768);
-      tma_load_3d(sm + SM_Q8, &tm.q8, 0, sc.q0, bq, &q_full);
-      tma_load_3d(sm + SM_Q16, &tm.q16, 0, sc.q0, bq, &q_full);
-      tma_load_3d(sm + SM_Q16 + 16384, &tm.q16, 64, sc.q0, bq, &q_full);
+      mbar_arrive_expect_tx(&q_full, 2 * (16384 + 32768));
+      for (int g = 0; g < 2; ++g) {
+        const int qr = sc.q0 + g * TQ;
+        tma_load_3d(sm + SM_Q8 + g * 16384, &tm.q8, 0, qr, bq, &q_full);
+        tma_load_3d(sm + SM_Q16 + g * 32768, &tm.q16, 0, qr, bq, &q_full);
+        tma_load_3d(sm + SM_Q16 + g * 32768 + 16384, &tm.q16, 64, qr, bq, &q_full);
+      }
       int issued[2] = {0, 0};
-      for (int t = 0; t < sc.nT; ++t) {
-        const int s = t & 1;
-        // the stage is free once QK(t-2) is done and the softmax has read the
-        // stage's mask bias / VL positions / K scales of tile t-2
-        if (t >= 2 && !(waitb(&k_empty[s], ((t >> 1) - 1) & 1, a.err, &abort_flag) &&
-                        waitb(&s_free[s], ((t >> 1) - 1) & 1, a.err, &abort_flag)))
-          break;
-        uint8_t* K = sm + SM_K + s * 32768;
-        uint8_t* aux = sm + SM_AUX + s * AUX_STAGE;
-        if (t < sc.nA) {
-          const int kt = t;
-          mbar_arrive_expect_tx(&k_full[s], 16384 + 512 + 16);
-          tma_load_3d(K, &tm.k8, 0, kt * TKEY, bk, &k_full[s]);
-          bulk_g2s(aux, a.kbias + static_cast<size_t>(bk) * a.Lp + kt * TKEY, 512, &k_full[s]);
-          bulk_g2s(aux + 512, a.sk + ((static_cast<size_t>(bk) * a.nblk + kt) & ~static_cast<size_t>(3)), 16, &k_full[s]);
-        } else if (t < sc.nA + sc.nB) {
-          const int v = t - sc.nA;
-          mbar_arrive_expect_tx(&k_full[s], 32768 + 512);
-          tma_load_3d(K, &tm.kvl, 0, v * TKEY, bk, &k_full[s]);
-          tma_load_3d(K + 16384, &tm.kvl, 64, v * TKEY, bk, &k_full[s]);
-          bulk_g2s(aux, a.vlpos + static_cast<size_t>(bk) * a.nvlp + v * TKEY, 512, &k_full[s]);
-        } else {
-          const int kt = sc.ktw0 + (t - sc.nA - sc.nB);
-          mbar_arrive_expect_tx(&k_full[s], 32768);
-          tma_load_3d(K, &tm.k16, 0, kt * TKEY, bk, &k_full[s]);
-          tma_load_3d(K + 16384, &tm.k16, 64, kt * TKEY, bk, &k_full[s]);
+      bool ok = true;
+      for (int t = 0; ok && t < sc.nT; ++t) {
+        const TileSlot z = slot_of(t, nF);
+        // the stage is free once both QKs of its previous tile are done and both
+        // softmax groups have read that tile's aux (barriers counted per use of
+        // the stage, so a wait is never more than one phase behind)
+        if (z.prev >= 0) {
+          const int pu = slot_of(z.prev, nF).use;
+          ok = waitb(&k_empty[z.stage], pu & 1, a.err, &abort_flag) && waitb(&aux_free[z.stage], pu & 1, a.err, &abort_flag);
         }
-        issued[s] = (t >> 1) + 1;
+        if (ok && t == nF) {
+          // every fp16 QK is done (the stage-0 wait above) and the fp16 query
+          // tiles have landed: their region may now serve as stage 1
+          ok = waitb(&q_full, 0, a.err, &abort_flag);
+          if (ok) mbar_arrive(&q16_free);
+        }
+        if (!ok) break;
+        uint8_t* K = sm + k_stage(z.stage);
+        uint8_t* aux = sm + SM_AUX + z.stage * 512;
+        if (t >= nF) {
+          const int kt = t - nF;
+          mbar_arrive_expect_tx(&k_full[z.stage], 16384 + 512 + 16);
+          tma_load_3d(K, &tm.k8, 0, kt * TKEY, bk, &k_full[z.stage]);
+          bulk_g2s(aux, a.kbias + static_cast<size_t>(bk) * a.Lp + kt * TKEY, 512, &k_full[z.stage]);
+          bulk_g2s(sm + SM_KS + z.stage * 16, a.sk + ((static_cast<size_t>(bk) * a.nblk + kt) & ~static_cast<size_t>(3)), 16,
+                   &k_full[z.stage]);
+        } else if (t < sc.nB) {
+          mbar_arrive_expect_tx(&k_full[0], 32768 + 512);
+          tma_load_3d(K, &tm.kvl, 0, t * TKEY, bk, &k_full[0]);
+          tma_load_3d(K + 16384, &tm.kvl, 64, t * TKEY, bk, &k_full[0]);
+          bulk_g2s(aux, a.vlpos + static_cast<size_t>(bk) * a.nvlp + t * TKEY, 512, &k_full[0]);
+        } else {
+          const int kt = sc.ktw0 + (t - sc.nB);
+          mbar_arrive_expect_tx(&k_full[0], 32768);
+          tma_load_3d(K, &tm.k16, 0, kt * TKEY, bk, &k_full[0]);
+          tma_load_3d(K + 16384, &tm.k16, 64, kt * TKEY, bk, &k_full[0]);
+        }
+        issued[z.stage] = z.use + 1;
       }
       if (abort_flag) {
         // never expected: let every issued copy land before the CTA can exit
         int dummy = 0;
-        for (int s = 0; s < 2; ++s)
-          if (issued[s] > 0) waitb(&k_full[s], (issued[s] - 1) & 1, a.err, &dummy);
+        for (int st = 0; st < 2; ++st)
+          if (issued[st] > 0) waitb(&k_full[st], (issued[st] - 1) & 1, a.err, &dummy);
         waitb(&q_full, 0, a.err, &dummy);
       }
     } else if (lane == 1) {
       int issued[2] = {0, 0};
-      for (int t = 0; t < sc.nT; ++t) {
-        const int s = t & 1;
-        if (t >= 2 && !waitb(&v_empty[s], ((t >> 1) - 1) & 1, a.err, &abort_flag)) break;
-        uint8_t* V = sm + SM_V + s * 32768;
+      bool ok = true;
+      for (int t = 0; ok && t < sc.nT; ++t) {
+        const TileSlot z = slot_of(t, nF);
+        if (z.prev >= 0) ok = waitb(&v_empty[z.stage], slot_of(z.prev, nF).use & 1, a.err, &abort_flag);
+        // V stage 1 is the second fp16 query tile: free once the K lane says so
+        if (ok && z.stage == 1 && z.use == 0) ok = waitb(&q16_free, 0, a.err, &abort_flag);
+        if (!ok) break;
+        uint8_t* V = sm + v_stage(z.stage);
         const CUtensorMap* map;
         int row;
-        if (t < sc.nA) {
+        if (t >= nF) {
           map = &tm.v8;
-          row = t * TKEY;
-        } else if (t < sc.nA + sc.nB) {
+          row = (t - nF) * TKEY;
+        } else if (t < sc.nB) {
           map = &tm.vvl;
-          row = (t - sc.nA) * TKEY;
+          row = t * TKEY;
         } else {
           map = &tm.v16;
-          row = (sc.ktw0 + (t - sc.nA - sc.nB)) * TKEY;
+          row = (sc.ktw0 + (t - sc.nB)) * TKEY;
         }
-        mbar_arrive_expect_tx(&v_full[s], 32768);
-        tma_load_3d(V, map, 0, row, bk, &v_full[s]);
-        tma_load_3d(V + 16384, map, 64, row, bk, &v_full[s]);
-        issued[s] = (t >> 1) + 1;
+        mbar_arrive_expect_tx(&v_full[z.stage], 32768);
+        tma_load_3d(V, map, 0, row, bk, &v_full[z.stage]);
+        tma_load_3d(V + 16384, map, 64, row, bk, &v_full[z.stage]);
+        issued[z.stage] = z.use + 1;
       }
       if (abort_flag) {
         int dummy = 0;
-        for (int s = 0; s < 2; ++s)
-          if (issued[s] > 0) waitb(&v_full[s], (issued[s] - 1) & 1, a.err, &dummy);
+        for (int st = 0; st < 2; ++st)
+          if (issued[st] > 0) waitb(&v_full[st], (issued[st] - 1) & 1, a.err, &dummy);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == W_MMA) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
-      const uint32_t q8 = sm_base + SM_Q8, q16 = sm_base + SM_Q16, p = sm_base + SM_P;
       bool ok = waitb(&q_full, 0, a.err, &abort_flag);
-      // QK(t) into S buffer t%2, once K(t) landed and the softmax has read S(t-2)
-      auto issue_qk = [&](int t) -> bool {
-        const int s = t & 1;
-        if (!waitb(&k_full[s], (t >> 1) & 1, a.err, &abort_flag)) return false;
-        if (t >= 2 && !waitb(&s_free[s], ((t >> 1) - 1) & 1, a.err, &abort_flag)) return false;
+      auto issue_qk = [&](int g, int t, int st) {
         tc_fence_after();
-        const uint32_t S = tmem + 128 * s;
-        const uint32_t K = sm_base + SM_K + s * 32768;
-        if (t < sc.nA) {
+        const uint32_t S = tmem + TM_S + 128 * g;
+        const uint32_t K = sm_base + k_stage(st);
+        if (t >= nF) {
+          const uint32_t q8 = sm_base + SM_Q8 + g * 16384;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             umma_f8(S, sdesc_sw128(q8 + 32 * kk, 16, 1024), sdesc_sw128(K + 32 * kk, 16, 1024), IDESC_QK, kk > 0);
         } else {
+          const uint32_t q16 = sm_base + SM_Q16 + g * 32768;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = (kk >> 2) * 16384 + 32 * (kk & 3);
             umma_f16(S, sdesc_sw128(q16 + off, 16, 1024), sdesc_sw128(K + off, 16, 1024), IDESC_QK, kk > 0);
           }
         }
-        umma_commit(&s_full[s]);
-        umma_commit(&k_empty[s]);
-        return true;
+        umma_commit(&s_full[g]);
       };
-      if (ok && sc.nT > 0) ok = issue_qk(0);
-      if (ok && sc.nT > 1) ok = issue_qk(1);
-      for (int t = 0; ok && t < sc.nT; ++t) {
-        const int s = t & 1;
-        ok = waitb(&p_full, t & 1, a.err, &abort_flag) && waitb(&v_full[s], (t >> 1) & 1, a.err, &abort_flag);
-        if (!ok) break;
+      auto issue_pv = [&](int g, int t, int st) {
         tc_fence_after();
-        const uint32_t V = sm_base + SM_V + s * 32768;
+        const uint32_t p = sm_base + SM_P + g * 32768;
+        const uint32_t V = sm_base + v_stage(st);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t aoff = (kk >> 2) * 16384 + 32 * (kk & 3);
-          umma_f16(tmem + TM_O, sdesc_sw128(p + aoff, 16, 1024), sdesc_sw128(V + 2048 * kk, 16384, 1024), IDESC_PV,
-                   (t > 0 || kk > 0) ? 1u : 0u);
+          umma_f16(tmem + TM_O + 128 * g, sdesc_sw128(p + aoff, 16, 1024), sdesc_sw128(V + 2048 * kk, 16384, 1024),
+                   IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&o_done);
-        umma_commit(&v_empty[s]);
-        if (t + 2 < sc.nT) ok = issue_qk(t + 2);
+        umma_commit(&o_done[g]);
+      };
+      // Event-driven issue: whichever of QK_A, QK_B, PV_A, PV_B is ready goes
+      // next.  The groups stay within a stage's reuse distance of each other,
+      // which keeps every probed barrier within one phase.
+      int tq[2] = {0, 0}, tp[2] = {0, 0};
+      uint64_t t_last = global_ns();
+      while (ok && (tp[0] < sc.nT || tp[1] < sc.nT)) {
+        bool progress = false;
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          const int t = tq[g];
+          if (t < sc.nT) {
+            const TileSlot z = slot_of(t, nF);
+            if (mbar_test_wait(&k_full[z.stage], z.use & 1) && (t == 0 || mbar_test_wait(&s_free[g], (t - 1) & 1))) {
+              issue_qk(g, t, z.stage);
+              if (tq[g ^ 1] > t) umma_commit(&k_empty[z.stage]);  // both QKs of tile t issued
+              tq[g] = t + 1;
+              progress = true;
+            }
+          }
+          const int u = tp[g];
+          if (u < tq[g]) {
+            const TileSlot z = slot_of(u, nF);
+            if (mbar_test_wait(&p_full[g], u & 1) && mbar_test_wait(&v_full[z.stage], z.use & 1)) {
+              issue_pv(g, u, z.stage);
+              if (tp[g ^ 1] > u) umma_commit(&v_empty[z.stage]);  // both PVs of tile u issued
+              tp[g] = u + 1;
+              progress = true;
+            }
+          }
+        }
+        if (progress) {
+          t_last = global_ns();
+        } else if (*reinterpret_cast<volatile int*>(&abort_flag)) {
+          ok = false;
+        } else if (global_ns() - t_last > 1000000000ull) {
+          atomicOr(a.err, 1u);
+          abort_flag = 1;
+          ok = false;
+        }
       }
       // every MMA this thread issued completes before TMEM is released
       umma_commit(&drain);
@@ -308,144 +443,111 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
       waitb(&drain, 0, a.err, &dummy);
     }
   } else {
-    // ------------------------------------------------------------ softmax (warps 0..3)
-    const int r = threadIdx.x;  // row within the tile = TMEM lane
-    const int i = sc.q0 + r;
-    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const uint32_t prow = sm_base + SM_P + r * 128;
+    // ------------------------------------------------------------ softmax (warps 0..7)
+    const int g = warp >> 2;          // query tile of this warpgroup
+    const int r = threadIdx.x & 127;  // row within the tile = TMEM lane
+    const int i = sc.q0 + g * TQ + r;
+    const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t srow = trow + TM_S + 128 * g, orow = trow + TM_O + 128 * g;
+    const uint32_t prow = sm_base + SM_P + g * 32768 + r * 128;
     float m_run = -INFINITY, l_run = 0.f;
-    const float sqv = a.sq[static_cast<size_t>(bq) * a.nblk + sc.qt];
+    // tile B of the last pair may lie wholly past L (its rows are never stored)
+    const float sqv = a.sq[static_cast<size_t>(bq) * a.nblk + min(sc.pr * 2 + g, a.nblk - 1)];
     bool ok = true;
     for (int t = 0; t < sc.nT; ++t) {
-      const int s = t & 1;
-      ok = ok && waitb(&s_full[s], (t >> 1) & 1, a.err, &abort_flag);
+      const TileSlot z = slot_of(t, nF);
+      const uint8_t* aux = sm + SM_AUX + z.stage * 512;
+      ok = ok && waitb(&s_full[g], t & 1, a.err, &abort_flag);
+      // P_g is read by PV_g(t-1): wait for it before storing this tile's P
+      if (t > 0) ok = ok && waitb(&o_done[g], (t - 1) & 1, a.err, &abort_flag);
       if (!__all_sync(0xffffffffu, ok)) ok = false;
       if (!ok) break;
       tc_fence_after();
-      float x[TKEY];
+      const float scl = t >= nF ? sqv * reinterpret_cast<const float*>(sm + SM_KS + z.stage * 16)
+                                           [(static_cast<size_t>(bk) * a.nblk + (t - nF)) & 3] * a.qk_scale
+                                : a.qk_scale;
+      float mt = -INFINITY, lt = 0.f;
+      bool redo = false;
+      for (int pass = 0; pass < 2; ++pass) {
+        // P = exp2(s - m_run) in fp16 into shared memory (K-major, 128-byte
+        // swizzle: 16-byte chunk k of the row goes to chunk k ^ (r % 8) of its
+        // 128-byte line; keys 64..127 in region 1), row sum in fp32
+        const float mref = m_run == -INFINITY ? 0.f : m_run;
+        float l0 = 0.f, l1 = 0.f, mx = -INFINITY;
+        float x[32];
+        tmem_ld32f(srow, x);
+        tmem_wait_ld();
+#pragma unroll 1
+        for (int c4 = 0; c4 < 4; ++c4) {
+          mx = fmaxf(mx, scale_mask32(x, 32 * c4, t, sc, a, aux, scl, i));
+          uint32_t pk[16];
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) tmem_ld32f(trow + 128 * s + 32 * c4, x + 32 * c4);
-      tmem_wait_ld();
-
-      // scale and mask this tile's scores
-      const uint8_t* aux = sm + SM_AUX + s * AUX_STAGE;
-      float mt = -INFINITY;
-      if (t < sc.nA) {
-        const int kt = t;
-        const float skv = reinterpret_cast<const float*>(aux + 512)[(static_cast<size_t>(bk) * a.nblk + kt) & 3];
-        const float scl = sqv * skv * a.qk_scale;
-        const float4* bias = reinterpret_cast<const float4*>(aux);
-        const int jlim = i - a.W - kt * TKEY;  // causal limit of this row: columns c <= jlim
-        if (jlim >= TKEY - 1) {
-#pragma unroll
-          for (int c4 = 0; c4 < TKEY / 4; ++c4) {
-            const float4 bb = bias[c4];
-            x[4 * c4] = fmaf(x[4 * c4], scl, bb.x);
-            x[4 * c4 + 1] = fmaf(x[4 * c4 + 1], scl, bb.y);
-            x[4 * c4 + 2] = fmaf(x[4 * c4 + 2], scl, bb.z);
-            x[4 * c4 + 3] = fmaf(x[4 * c4 + 3], scl, bb.w);
-            mt = fmaxf(mt, fmaxf(fmaxf(x[4 * c4], x[4 * c4 + 1]), fmaxf(x[4 * c4 + 2], x[4 * c4 + 3])));
+          for (int c = 0; c < 32; c += 2) {
+            const float p0 = ex2(x[c] - mref), p1 = ex2(x[c + 1] - mref);
+            l0 += p0;
+            l1 += p1;
+            pk[c / 2] = pack_f16x2(p0, p1);
           }
-        } else {
+          if (c4 < 3) tmem_ld32f(srow + 32 * (c4 + 1), x);  // next chunk in flight during the stores
 #pragma unroll
-          for (int c4 = 0; c4 < TKEY / 4; ++c4) {
-            const float4 bb = bias[c4];
-            const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = 4 * c4 + e;
-              x[c] = c <= jlim ? fmaf(x[c], scl, bv[e]) : -INFINITY;
-              mt = fmaxf(mt, x[c]);
-            }
+          for (int k = 0; k < 4; ++k) {
+            const int kc = 4 * c4 + k;  // 16-byte chunk of the row (8 keys)
+            const uint32_t addr = prow + (kc >> 3) * 16384 + ((((kc & 7) ^ (r & 7))) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * k]), "r"(pk[4 * k + 1]),
+                         "r"(pk[4 * k + 2]), "r"(pk[4 * k + 3])
+                         : "memory");
           }
+          if (c4 < 3) tmem_wait_ld();
         }
-      } else if (t < sc.nA + sc.nB) {
-        const int32_t* vp = reinterpret_cast<const int32_t*>(aux);
-        const int lim = i - a.W;
-#pragma unroll
-        for (int c = 0; c < TKEY; ++c) {
-          const bool v = vp[c] <= lim;
-          x[c] = v ? x[c] * a.qk_scale : -INFINITY;
-          mt = fmaxf(mt, x[c]);
+        mt = mx;
+        lt = l0 + l1;
+        // lazy running max: move it only when a row's tile max exceeds it by
+        // more than 2^8 (then p could leave the fp16 range); that row's P is
+        // recomputed against the new max and O rescaled
+        const bool grow = mt > m_run + 8.0f;
+        if (pass == 1 || !__any_sync(0xffffffffu, grow)) break;
+        redo = true;
+        // per row: alpha = 1 unless this row's max moved
+        float alpha = 1.f;
+        if (grow) {
+          alpha = m_run != -INFINITY ? ex2(m_run - mt) : 0.f;
+          m_run = mt;
+          l_run *= alpha;
         }
-      } else {
-        const int kt = sc.ktw0 + (t - sc.nA - sc.nB);
-        const int lo = i - a.W + 1 - kt * TKEY, hi = i - kt * TKEY;  // window: lo <= c <= hi
-#pragma unroll
-        for (int c = 0; c < TKEY; ++c) {
-          const bool v = c >= lo && c <= hi;
-          x[c] = v ? x[c] * a.qk_scale : -INFINITY;
-          mt = fmaxf(mt, x[c]);
-        }
-      }
-      // S(t) is in registers and the stage's auxiliary data has been read: the S
-      // buffer and the K stage's aux area may be refilled
-      tc_fence_before();
-      mbar_arrive(&s_free[s]);
-      // lazy running max: only move it (and rescale O) when it grows by > 2^8
-      const bool grow = mt > m_run + 8.0f;
-      const bool any_grow = __any_sync(0xffffffffu, grow);
-      float alpha = 1.f;
-      if (grow) {
-        alpha = m_run != -INFINITY ? ex2(m_run - mt) : 0.f;
-        m_run = mt;
-        l_run *= alpha;
-      }
-      // P = exp2(s - m_run) in fp16, row sum in fp32
-      const float mref = m_run == -INFINITY ? 0.f : m_run;
-      uint32_t pk[TKEY / 2];
-      float l0 = 0.f, l1 = 0.f;
-#pragma unroll
-      for (int c = 0; c < TKEY; c += 2) {
-        const float p0 = ex2(x[c] - mref), p1 = ex2(x[c + 1] - mref);
-        l0 += p0;
-        l1 += p1;
-        pk[c / 2] = pack_f16x2(p0, p1);
-      }
-      l_run += l0 + l1;
-      // O holds P.V of earlier tiles and the P buffer is read by PV of tile t-1:
-      // wait for it, then (if the max moved) rescale O in TMEM
-      if (t > 0) {
-        ok = waitb(&o_done, (t - 1) & 1, a.err, &abort_flag);
-        if (!__all_sync(0xffffffffu, ok)) ok = false;
-        if (!ok) break;
-        if (any_grow) {
-          tc_fence_after();
-#pragma unroll
+        // the TMEM accesses are warp-collective (.sync.aligned): the whole warp
+        // rescales its O rows, rows whose max did not move by 1
+        if (t > 0) {
+#pragma unroll 1
           for (int c4 = 0; c4 < 4; ++c4) {
             uint32_t u[32];
-            tmem_ld32(trow + TM_O + 32 * c4, u);
+            tmem_ld32(orow + 32 * c4, u);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
-            tmem_st32(trow + TM_O + 32 * c4, u);
+            tmem_st32(orow + 32 * c4, u);
           }
           tmem_wait_st();
         }
       }
-      // store P row r (K-major, 128-byte swizzle: 16-byte chunk k of the row goes
-      // to chunk k ^ (r % 8) of the 128-byte line; keys 64..127 in region 1)
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const uint32_t addr = prow + (k >> 3) * 16384 + ((((k & 7) ^ (r & 7))) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * k]), "r"(pk[4 * k + 1]),
-                     "r"(pk[4 * k + 2]), "r"(pk[4 * k + 3])
-                     : "memory");
-      }
-      fence_proxy_async_smem();
+      (void)redo;
+      l_run += lt;
+      // S_g(t) and the stage's auxiliary data have been read for the last time
       tc_fence_before();
-      mbar_arrive(&p_full);
+      mbar_arrive(&s_free[g]);
+      mbar_arrive(&aux_free[z.stage]);
+      fence_proxy_async_smem();
+      mbar_arrive(&p_full[g]);
     }
     // epilogue: O / l -> fp16 row
-    if (ok && sc.nT > 0) ok = waitb(&o_done, (sc.nT - 1) & 1, a.err, &abort_flag);
+    if (ok && sc.nT > 0) ok = waitb(&o_done[g], (sc.nT - 1) & 1, a.err, &abort_flag);
     if (__all_sync(0xffffffffu, ok) && sc.nT > 0) {
       tc_fence_after();
       const float inv = l_run > 0.f ? 1.0f / l_run : 0.f;
       uint16_t* dst = a.out + (static_cast<size_t>(bq) * a.L + i) * D;
-#pragma unroll
+#pragma unroll 1
       for (int c4 = 0; c4 < 4; ++c4) {
         uint32_t u[32];
-        tmem_ld32(trow + TM_O + 32 * c4, u);
+        tmem_ld32(orow + 32 * c4, u);
         tmem_wait_ld();
         if (i < a.L) {
 #pragma unroll
@@ -464,7 +566,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
   __syncwarp();  // producer / MMA warps: lanes wait for their issuing lanes before the CTA barrier
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == W_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
@@ -683,7 +785,7 @@ hq_status launch_prefill(int B, int Hq, int Hkv, int L, const uint16_t* q, const
       return cuda_fail(cudaGetLastError(), "prefill setup");
     if (dev < 64) attr_done[dev] = true;
   }
-  prefill_kernel<<<dim3(ly.nblk, Hq, B), PF_THREADS, PF_SMEM, st>>>(tm, a);
+  prefill_kernel<<<dim3((ly.nblk + 1) / 2, Hq, B), PF_THREADS, PF_SMEM, st>>>(tm, a);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     // name the kernel's resources in the message (launch-resource failures)
