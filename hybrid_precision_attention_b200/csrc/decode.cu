@@ -44,7 +44,7 @@ namespace {
 
 // Two CTA shapes, one kernel template (NC consumer warps, 2 stages each, one
 // producer warp):
-//   wide  : NC = 9, 18 stages, 1 CTA per SM   (few kv heads: fewer, longer splits)
+//   wide  : NC = 11, 22 stages, 1 CTA per SM  (few kv heads: fewer, longer splits)
 //   narrow: NC = 3,  6 stages, 3 CTAs per SM  (large batches)
 // Each stage must have exactly one consumer warp: a parity wait on an mbarrier
 // only tells the current phase from the one before it, so a warp that reached a
@@ -52,7 +52,7 @@ namespace {
 // older completed phase and consume the wrong data.  With NSTAGES = 2 NC,
 // stage s belongs to warp s % NC.
 #ifndef HQ_DECODE_NC_WIDE
-#define HQ_DECODE_NC_WIDE 9
+#define HQ_DECODE_NC_WIDE 11
 #endif
 constexpr int NC_WIDE = HQ_DECODE_NC_WIDE, NC_NARROW = 3;
 constexpr int PK = 64;                         // positions per packed tile
