@@ -459,6 +459,28 @@ def profile_decode():
     print("profile-decode ok", st)
 
 
+def profile_select():
+    """Small case for ncu captures: a decode-mode reselection of one 32K layer (prefix install, 64 decode
+    steps filling the query buffer, L2 flushed, then hq_select_vlines: two passes and the top-k)."""
+    import torch
+    from hybrid_precision_attention_b200 import hq, synth
+    lay = synth.planted_layer(0, B, HQ, HKV, L)
+    k_d, v_d, qt_d = [torch.from_numpy(a).cuda() for a in (lay.k, lay.v, lay.q_tail)]
+    c = hq.HybridCache(B, HQ, HKV, L + 256, W, RHO_BP)
+    hq.hq_select_vlines(c, k_d, qt_d)
+    hq.hq_pack_merge(c, k_d, v_d)
+    q, k, v = [torch.from_numpy(a).cuda() for a in synth.decode_tokens(1, B, HQ, HKV, PERIOD)]
+    for i in range(PERIOD):
+        hq.hq_decode_attn(c, q[i], k[i], v[i])
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    flush.zero_()
+    hq.hq_select_vlines(c)
+    torch.cuda.synchronize()
+    st = c.state()
+    assert st["err"] == 0 and st["n_q"] == PERIOD and st["k_sel"] > 0, st
+    print("profile-select ok", st)
+
+
 def profile_prefill():
     """Small case for ncu captures: the hybrid prefill at L=8192 (B=1, Hq=32, Hkv=8), three calls."""
     import torch
@@ -490,12 +512,16 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--profile-decode", action="store_true", help="small case for ncu: 4 decode steps of one 32K layer")
     ap.add_argument("--profile-prefill", action="store_true", help="small case for ncu: 3 prefill calls at L=8192")
+    ap.add_argument("--profile-select", action="store_true", help="small case for ncu: one decode-mode reselection at 32K")
     args = ap.parse_args()
     if args.profile_decode:
         profile_decode()
         return
     if args.profile_prefill:
         profile_prefill()
+        return
+    if args.profile_select:
+        profile_select()
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
