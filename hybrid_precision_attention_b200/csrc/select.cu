@@ -44,6 +44,7 @@ constexpr int SEL_THREADS = (MMA_WARP + 1) * 32;
 constexpr int MAX_SPLITS = 32;           // CTAs per (b, kv head)
 constexpr int KSTAGE = KT * 256;         // one rebuilt key tile: 2 halves x [128 rows][128 B]
 constexpr uint32_t TMEM_COLS = 512;
+constexpr int HBINS = 2048;              // score histogram: bits 30..20 of the (non-negative) fp32 pattern
 
 struct SelArgs {
   hq_cache c;
@@ -53,6 +54,7 @@ struct SelArgs {
   int nq_init;
   float* lse_part;          // [B*Hkv][MAX_SPLITS][Mp] x (m, l)
   float* scores;            // [B*Hkv][cap]
+  uint32_t* hist;           // [B*Hkv][HBINS] histogram of the scores' bits 30..20
   int S;                    // CTAs per (b, kv head)
   int Mp;                   // query rows in shared memory: G * HQ_QBUF rounded up to 128
   float qscale;             // sm_scale * log2(e)
@@ -252,6 +254,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
   int* qpos = reinterpret_cast<int*>(aux);   // [Mp] query positions
   float* lse = aux + Mp;                     // [Mp] pass 1: log-sum-exp (exp2 domain), +inf on padding rows
   float* xch = aux + 2 * Mp;                 // [2][Mp] pass 0 (m, l) of column half 1; pass 1 [KT] partial sums
+  uint32_t* shist = reinterpret_cast<uint32_t*>(aux + 4 * Mp);  // [HBINS] pass 1: this CTA's score histogram
 
   if (threadIdx.x == 0) {
     mbar_init(&kfull[0], BLD_WARPS * 32);
@@ -289,6 +292,13 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
     *reinterpret_cast<uint4*>(qs + sw128_off(r, ch, Mp * 128)) = v;
   }
   for (int r = threadIdx.x; r < Mp; r += SEL_THREADS) qpos[r] = r < M ? g.qpos0 + r % max(g.nq, 1) : -1;
+  if (!COL) {
+    // the head's score histogram is rebuilt by pass 1: each split clears a slice
+    uint32_t* gh = a.hist + static_cast<size_t>(bh) * HBINS;
+    for (int e = (split * HBINS) / a.S + threadIdx.x; e < ((split + 1) * HBINS) / a.S; e += SEL_THREADS) gh[e] = 0u;
+  } else {
+    for (int e = threadIdx.x; e < HBINS; e += SEL_THREADS) shist[e] = 0u;
+  }
   if (COL) {
     // per-row log-sum-exp over the pass-0 partials of every split
     for (int r = threadIdx.x; r < Mp; r += SEL_THREADS) {
@@ -387,6 +397,8 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
     // no buffered queries: every candidate's column mass is zero
     for (int j = k_lo * KT + threadIdx.x; j < min(k_hi * KT, g.n); j += EPI_WARPS * 32)
       a.scores[static_cast<size_t>(bh) * c.cap + j] = 0.f;
+    if (threadIdx.x == 0 && min(k_hi * KT, g.n) > k_lo * KT)
+      atomicAdd(a.hist + static_cast<size_t>(bh) * HBINS, static_cast<unsigned>(min(k_hi * KT, g.n) - k_lo * KT));
   } else {
     // ------------------------------------------------------------ epilogue
     const int qd = warp & 3, hc = warp >> 2;
@@ -504,9 +516,17 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
         // the two column halves of key j: half 1 hands its sum over, half 0 writes
         if (hc == 1) xch[qd * 32 + lane] = sum;
         asm volatile("bar.sync 1, %0;" ::"r"(EPI_WARPS * 32) : "memory");
-        if (hc == 0 && j < g.n) a.scores[static_cast<size_t>(bh) * c.cap + j] = sum + xch[qd * 32 + lane];
+        if (hc == 0 && j < g.n) {
+          const float sc_j = sum + xch[qd * 32 + lane];
+          a.scores[static_cast<size_t>(bh) * c.cap + j] = sc_j;
+          atomicAdd(shist + (__float_as_uint(sc_j) >> 20), 1u);
+        }
         asm volatile("bar.sync 1, %0;" ::"r"(EPI_WARPS * 32) : "memory");
       }
+      // this CTA's histogram into the head's
+      uint32_t* gh = a.hist + static_cast<size_t>(bh) * HBINS;
+      for (int e = threadIdx.x; e < HBINS; e += EPI_WARPS * 32)
+        if (shist[e]) atomicAdd(gh + e, shist[e]);
     }
   }
   tc_fence_before();
@@ -518,12 +538,8 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
 }
 
 constexpr int TK_THREADS = 1024;
-constexpr int TK_VPT = 48;                          // candidates per thread held in registers
-constexpr int TK_SMEM_MAX = TK_THREADS * TK_VPT;    // 49152 candidates
-
-// shared-memory slot of candidate j: one pad word per 32, so that threads owning
-// consecutive 48-candidate segments read distinct banks
-__device__ __forceinline__ int tk_slot(int j) { return j + (j >> 5); }
+constexpr int TK_SMEM_MAX = 49152;  // scores held in shared memory up to this many candidates
+constexpr int TK_CAND_MAX = 8192;   // values of the threshold's histogram bin held in shared memory
 
 // block-wide sum of one value per thread (1024 threads); every thread gets it
 __device__ __forceinline__ unsigned int tk_block_sum(unsigned int v, unsigned int* red) {
@@ -537,15 +553,15 @@ __device__ __forceinline__ unsigned int tk_block_sum(unsigned int v, unsigned in
 }
 
 // Exact top-k of the column-mass scores of one (b, kv head).  Scores are >= 0,
-// so their fp32 bit patterns order like the values.  The k-th largest pattern
-// is found bit by bit from the top (keep a bit when at least k candidates are
-// >= the pattern with it set); each thread holds a contiguous segment of the
-// candidates in registers, so every step is register compares and one block
-// sum.  An ordered compaction then writes the chosen positions ascending, ties
-// at the threshold to the lowest positions.  Beyond TK_SMEM_MAX candidates
-// (REG = false) the same steps re-read the scores from global memory.
-template <bool REG>
-__global__ void __launch_bounds__(TK_THREADS) topk_kernel(SelArgs a) {
+// so their fp32 bit patterns order like the values.  (1) The histogram of bits
+// 30..20 that the column-mass pass built gives the bin holding the k-th
+// largest value and how many values lie above it.  (2) The values of that bin
+// are gathered into shared memory.  (3) Its low 20 bits are found bit by bit
+// (keep a bit when at least the needed number of candidates are >= the pattern
+// with it set).  (4) An ordered compaction over contiguous per-thread segments
+// writes the chosen positions ascending, ties at the threshold to the lowest
+// positions.  A bin too large for shared memory is searched in global memory.
+__global__ void __launch_bounds__(TK_THREADS) topk_kernel(SelArgs a, int smem_scores) {
   const hq_cache& c = a.c;
   const int bh = blockIdx.x;
   const SelGeo g = sel_geo(a);
@@ -561,101 +577,144 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(SelArgs a) {
   }
   if (bh == 0 && threadIdx.x == 0) c.state[HQ_STATE_KSEL] = k;
   if (k == 0) return;
-  extern __shared__ uint32_t tk_smem[];
+  extern __shared__ uint32_t tk_smem[];  // [TK_CAND_MAX] bin values, then [smem_scores] scores
   __shared__ unsigned int red[32];
+  __shared__ unsigned int s_bin, s_above, s_cnt;
+  __shared__ unsigned int wsum[TK_THREADS / 32];
   const uint32_t* gsc = reinterpret_cast<const uint32_t*>(a.scores + static_cast<size_t>(bh) * c.cap);
+  uint32_t* cand = tk_smem;
+  // the scores are staged in shared memory (all loads in flight at once) when they fit
+  const bool staged = n <= smem_scores;
+  uint32_t* ssc = tk_smem + TK_CAND_MAX;
+  if (staged) {
+#pragma unroll 8
+    for (int j = threadIdx.x; j < n; j += TK_THREADS) ssc[j] = __ldcg(gsc + j);
+  }
+  const uint32_t* sc = staged ? ssc : gsc;
+  const uint32_t* hh = a.hist + static_cast<size_t>(bh) * HBINS;
   int32_t* out = c.vl_sel + static_cast<size_t>(bh) * c.vl_cap;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
-  const int per = (n + TK_THREADS - 1) / TK_THREADS;  // <= TK_VPT when REG
-  const int lo = threadIdx.x * per, cnt = max(0, min(per, n - lo));
-  uint32_t v[REG ? TK_VPT : 1];
-  if (REG) {
-    for (int j = threadIdx.x; j < n; j += TK_THREADS) tk_smem[tk_slot(j)] = __ldcg(gsc + j);
-    __syncthreads();
-#pragma unroll
-    for (int e = 0; e < (REG ? TK_VPT : 1); ++e) v[e] = e < cnt ? tk_smem[tk_slot(lo + e)] : 0u;
-  }
-
-  uint32_t thr = 0u;
-  for (int bit = 30; bit >= 0; --bit) {  // bit 31 (sign) is 0 for every score
-    const uint32_t cand = thr | (1u << bit);
-    unsigned int ge = 0u;
-    if (REG) {
-#pragma unroll
-      for (int e = 0; e < (REG ? TK_VPT : 1); ++e) ge += (e < cnt && v[e] >= cand) ? 1u : 0u;
-    } else {
-      for (int j = threadIdx.x; j < n; j += TK_THREADS) ge += __ldcg(gsc + j) >= cand ? 1u : 0u;
-    }
-    if (tk_block_sum(ge, red) >= static_cast<unsigned>(k)) thr = cand;
-  }
-  // thr is the exact k-th largest value: take every value above it and the
-  // lowest-positioned (k - #above) of those equal to it
-  unsigned int cnt_gt = 0u, cnt_eq = 0u;
-  if (REG) {
-#pragma unroll
-    for (int e = 0; e < (REG ? TK_VPT : 1); ++e) {
-      cnt_gt += (e < cnt && v[e] > thr) ? 1u : 0u;
-      cnt_eq += (e < cnt && v[e] == thr) ? 1u : 0u;
-    }
-  } else {
-    for (int e = 0; e < cnt; ++e) {
-      const uint32_t x = __ldcg(gsc + lo + e);
-      cnt_gt += x > thr ? 1u : 0u;
-      cnt_eq += x == thr ? 1u : 0u;
-    }
-  }
-  const unsigned int take_eq = static_cast<unsigned>(k) - tk_block_sum(cnt_gt, red);
-  // block exclusive scan of (cnt_gt, cnt_eq) in thread (= position) order
-  __shared__ unsigned int warp_sums[TK_THREADS / 32][2];
-  unsigned int x = cnt_gt, y = cnt_eq;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const unsigned int xo = __shfl_up_sync(0xffffffffu, x, o), yo = __shfl_up_sync(0xffffffffu, y, o);
-    if (lane >= o) { x += xo; y += yo; }
-  }
-  if (lane == 31) { warp_sums[warp][0] = x; warp_sums[warp][1] = y; }
-  __syncthreads();
-  if (warp == 0) {
-    unsigned int wx = warp_sums[lane][0], wy = warp_sums[lane][1];
+  // (1) thread i owns bins 2047 - 2i (higher) and 2046 - 2i; an inclusive scan
+  // over threads gives the suffix sums S_d = #values in bins >= d
+  {
+    const int d1 = HBINS - 1 - 2 * threadIdx.x, d0 = d1 - 1;
+    const unsigned int h1 = __ldcg(hh + d1), h0 = __ldcg(hh + d0);
+    unsigned int x = h1 + h0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const unsigned int xo = __shfl_up_sync(0xffffffffu, wx, o), yo = __shfl_up_sync(0xffffffffu, wy, o);
-      if (lane >= o) { wx += xo; wy += yo; }
+      const unsigned int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
     }
-    warp_sums[lane][0] = wx;
-    warp_sums[lane][1] = wy;
+    if (lane == 31) wsum[warp] = x;
+    if (threadIdx.x == 0) {
+      s_cnt = 0u;
+      s_bin = 0u;  // only if the histogram disagreed with the scores (never expected)
+      s_above = 0u;
+    }
+    __syncthreads();
+    for (int w = 0; w < warp; ++w) x += wsum[w];
+    const unsigned int S0 = x, S1 = x - h0, Sabove = x - h0 - h1;  // S_{d0}, S_{d1}, S_{d1+1}
+    const unsigned int kk = static_cast<unsigned int>(k);
+    if (S1 >= kk && Sabove < kk) {
+      s_bin = d1;
+      s_above = Sabove;
+    } else if (S0 >= kk && S1 < kk) {
+      s_bin = d0;
+      s_above = S1;
+    }
+    __syncthreads();
   }
-  __syncthreads();
-  unsigned int ex_gt = x - cnt_gt + (warp > 0 ? warp_sums[warp - 1][0] : 0u);
-  unsigned int ex_eq = y - cnt_eq + (warp > 0 ? warp_sums[warp - 1][1] : 0u);
-  // output slot of position j = (#gt before j) + min(#eq before j, take_eq)
-#pragma unroll
-  for (int e = 0; e < (REG ? TK_VPT : 1 << 30); ++e) {
-    if (e >= cnt) break;
-    const int j = lo + e;
-    const uint32_t x = REG ? v[REG ? e : 0] : __ldcg(gsc + j);
-    if (x > thr) {
-      out[ex_gt + min(ex_eq, take_eq)] = j;
-      ++ex_gt;
-    } else if (x == thr) {
-      if (ex_eq < take_eq) out[ex_gt + ex_eq] = j;
-      ++ex_eq;
+  const uint32_t bin = s_bin;
+  const unsigned int need = static_cast<unsigned int>(k) - min(s_above, static_cast<unsigned int>(k) - 1u);  // >= 1
+  const unsigned int nbin = __ldcg(hh + bin);
+  const bool in_smem = nbin <= static_cast<unsigned int>(TK_CAND_MAX);
+  // (2) the bin's values
+  if (in_smem) {
+    for (int j0 = 0; j0 < n; j0 += TK_THREADS) {
+      const int j = j0 + threadIdx.x;
+      const uint32_t v = j < n ? sc[j] : 0u;
+      const bool hit = j < n && (v >> 20) == bin;
+      const unsigned int m = __ballot_sync(0xffffffffu, hit);
+      unsigned int base = 0u;
+      if (lane == 0 && m) base = atomicAdd(&s_cnt, static_cast<unsigned>(__popc(m)));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      const unsigned int slot = base + __popc(m & ((1u << lane) - 1u));
+      if (hit && slot < nbin) cand[slot] = v;  // nbin <= TK_CAND_MAX: the list never overflows
     }
+    __syncthreads();
+  }
+  const int ncand = in_smem ? static_cast<int>(min(s_cnt, nbin)) : n;
+  // (3) low 20 bits of the k-th largest
+  uint32_t thr = bin << 20;
+  for (int bit = 19; bit >= 0; --bit) {
+    const uint32_t cnd = thr | (1u << bit);
+    unsigned int ge = 0u;
+    for (int e = threadIdx.x; e < ncand; e += TK_THREADS) {
+      const uint32_t v = in_smem ? cand[e] : sc[e];
+      ge += ((v >> 20) == bin && v >= cnd) ? 1u : 0u;
+    }
+    if (tk_block_sum(ge, red) >= need) thr = cnd;
+  }
+  // (4) everything above thr, and the lowest-positioned of those equal to it
+  unsigned int gtb = 0u;
+  for (int e = threadIdx.x; e < ncand; e += TK_THREADS) {
+    const uint32_t v = in_smem ? cand[e] : sc[e];
+    gtb += ((v >> 20) == bin && v > thr) ? 1u : 0u;
+  }
+  const unsigned int take_eq = static_cast<unsigned int>(k) - s_above - tk_block_sum(gtb, red);
+  // ordered compaction in rounds of 1024 consecutive positions (coalesced
+  // reads): a position's slot = (#gt before it) + min(#eq before it, take_eq)
+  __shared__ unsigned int rg[TK_THREADS / 32 + 1], re[TK_THREADS / 32 + 1];
+  unsigned int base_gt = 0u, base_eq = 0u;
+  const unsigned int lt_mask = (1u << lane) - 1u;
+  for (int j0 = 0; j0 < n; j0 += TK_THREADS) {
+    const int j = j0 + threadIdx.x;
+    const uint32_t v = j < n ? sc[j] : 0u;
+    const bool gt = j < n && v > thr, eq = j < n && v == thr;
+    const unsigned int bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
+    if (lane == 0) {
+      rg[warp] = __popc(bg);
+      re[warp] = __popc(be);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // exclusive prefix over the 32 warps' counts, totals in slot 32
+      unsigned int xg2 = rg[lane], xe2 = re[lane];
+      const unsigned int og = xg2, oe = xe2;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned int yg = __shfl_up_sync(0xffffffffu, xg2, o), ye = __shfl_up_sync(0xffffffffu, xe2, o);
+        if (lane >= o) { xg2 += yg; xe2 += ye; }
+      }
+      rg[lane] = xg2 - og;
+      re[lane] = xe2 - oe;
+      if (lane == 31) { rg[32] = xg2; re[32] = xe2; }
+    }
+    __syncthreads();
+    const unsigned int pg = rg[warp], pe = re[warp], tg = rg[32], te = re[32];
+    const unsigned int xg = base_gt + pg + __popc(bg & lt_mask), xe = base_eq + pe + __popc(be & lt_mask);
+    if (gt) out[xg + min(xe, take_eq)] = j;
+    else if (eq && xe < take_eq) out[xg + xe] = j;
+    base_gt += tg;
+    base_eq += te;
+    __syncthreads();
   }
 }
 
-int tk_slot_host(int n) { return n + (n >> 5) + 1; }
 
 int sel_mp(const hq_cache& c) { return (((c.Hq / c.Hkv) * HQ_QBUF + 127) / 128) * 128; }
 
-size_t sel_smem_bytes(int Mp) { return 1024 + static_cast<size_t>(Mp) * 256 + 2 * KSTAGE + 4 * static_cast<size_t>(Mp) * 4; }
+size_t sel_smem_bytes(int Mp) {
+  return 1024 + static_cast<size_t>(Mp) * 256 + 2 * KSTAGE + 4 * static_cast<size_t>(Mp) * 4 + HBINS * 4;
+}
 
 }  // namespace
 
 size_t select_workspace(const hq_cache& c, bool need_scores) {
   const int Mp = sel_mp(c);
   size_t bytes = static_cast<size_t>(c.B) * c.Hkv * MAX_SPLITS * Mp * 2 * 4;  // (m, l) partials
+  bytes += static_cast<size_t>(c.B) * c.Hkv * HBINS * 4;                       // score histograms
   if (need_scores) bytes += static_cast<size_t>(c.B) * c.Hkv * c.cap * 4;
   return (bytes + 255) & ~static_cast<size_t>(255);
 }
@@ -681,6 +740,8 @@ hq_status launch_select(const hq_cache& c, const uint16_t* kd, int L, const uint
   char* w = static_cast<char*>(ws);
   a.lse_part = reinterpret_cast<float*>(w);
   w += static_cast<size_t>(c.B) * c.Hkv * MAX_SPLITS * a.Mp * 2 * 4;
+  a.hist = reinterpret_cast<uint32_t*>(w);
+  w += static_cast<size_t>(c.B) * c.Hkv * HBINS * 4;
   a.scores = scores_out ? scores_out : reinterpret_cast<float*>(w);
   a.qscale = (1.0f / sqrtf(static_cast<float>(D))) * LOG2E;
   const size_t smem = sel_smem_bytes(a.Mp);
@@ -689,20 +750,17 @@ hq_status launch_select(const hq_cache& c, const uint16_t* kd, int L, const uint
     const int smem_max = static_cast<int>(sel_smem_bytes(((HQ_MAX_GQA * HQ_QBUF + 127) / 128) * 128));
     if (cudaFuncSetAttribute(sel_pass<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max) != cudaSuccess ||
         cudaFuncSetAttribute(sel_pass<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max) != cudaSuccess ||
-        cudaFuncSetAttribute(topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(tk_slot_host(TK_SMEM_MAX)) * 4) != cudaSuccess)
+        cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (TK_CAND_MAX + TK_SMEM_MAX) * 4) !=
+            cudaSuccess)
       return cuda_fail(cudaGetLastError(), "select setup");
     if (dev < 64) attr_done[dev] = true;
   }
   dim3 grid(S, c.Hkv, c.B);
   sel_pass<false><<<grid, SEL_THREADS, smem, st>>>(a);
   sel_pass<true><<<grid, SEL_THREADS, smem, st>>>(a);
-  // candidates n <= max(keys_cap - W, 0): held in registers when they fit
-  const int n_max = max(keys_cap - c.W, 0);
-  if (n_max <= TK_SMEM_MAX)
-    topk_kernel<true><<<c.B * c.Hkv, TK_THREADS, static_cast<size_t>(tk_slot_host(max(n_max, 1))) * 4, st>>>(a);
-  else
-    topk_kernel<false><<<c.B * c.Hkv, TK_THREADS, 0, st>>>(a);
+  // shared memory: the bin's values and, when they fit, the scores themselves
+  const int smem_scores = min(max(keys_cap - c.W, 0), TK_SMEM_MAX);
+  topk_kernel<<<c.B * c.Hkv, TK_THREADS, static_cast<size_t>(TK_CAND_MAX + smem_scores) * 4, st>>>(a, smem_scores);
   return cuda_status(cudaGetLastError(), "select launch");
 }
 
