@@ -163,6 +163,7 @@ __device__ __forceinline__ TileSlot slot_of(int t, int nF) {
 
 // Scale and mask 32 scores of row i (columns c0 .. c0+31 of tile t) in place;
 // returns their max.  Columns a row must not see become -inf.
+template <bool MAX>
 __device__ __forceinline__ float scale_mask32(float (&x)[32], int c0, int t, const Sched& sc, const PfArgs& a,
                                               const uint8_t* aux, float scl, int i) {
   float mt = -INFINITY;
@@ -183,23 +184,23 @@ __device__ __forceinline__ float scale_mask32(float (&x)[32], int c0, int t, con
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
         x[c] = fmaf(x[c], scl, bv[c]);
-        m2[c & 1] = fmaxf(m2[c & 1], x[c]);
+        if (MAX) m2[c & 1] = fmaxf(m2[c & 1], x[c]);
       }
     } else {
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
         x[c] = c <= jlim ? fmaf(x[c], scl, bv[c]) : -INFINITY;
-        m2[c & 1] = fmaxf(m2[c & 1], x[c]);
+        if (MAX) m2[c & 1] = fmaxf(m2[c & 1], x[c]);
       }
     }
-    mt = fmaxf(m2[0], m2[1]);
+    if (MAX) mt = fmaxf(m2[0], m2[1]);
   } else if (t < sc.nB) {
     const int32_t* vp = reinterpret_cast<const int32_t*>(aux) + c0;
     const int lim = i - a.W;
 #pragma unroll
     for (int c = 0; c < 32; ++c) {
       x[c] = vp[c] <= lim ? x[c] * a.qk_scale : -INFINITY;
-      mt = fmaxf(mt, x[c]);
+      if (MAX) mt = fmaxf(mt, x[c]);
     }
   } else {
     const int kt = sc.ktw0 + (t - sc.nB);
@@ -207,7 +208,7 @@ __device__ __forceinline__ float scale_mask32(float (&x)[32], int c0, int t, con
 #pragma unroll
     for (int c = 0; c < 32; ++c) {
       x[c] = (c >= lo && c <= hi) ? x[c] * a.qk_scale : -INFINITY;
-      mt = fmaxf(mt, x[c]);
+      if (MAX) mt = fmaxf(mt, x[c]);
     }
   }
   return mt;
@@ -466,20 +467,61 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
       const float scl = t >= nF ? sqv * reinterpret_cast<const float*>(sm + SM_KS + z.stage * 16)
                                            [(static_cast<size_t>(bk) * a.nblk + (t - nF)) & 3] * a.qk_scale
                                 : a.qk_scale;
-      float mt = -INFINITY, lt = 0.f;
-      bool redo = false;
-      for (int pass = 0; pass < 2; ++pass) {
+      // One pass per tile: P = exp2(s - m_run) against the running max, the
+      // row sum in fp32.  A row sum above 2^8 (or not finite) means some p may
+      // have left the safe fp16 range because the row's max moved up: only then
+      // is the tile's exact max taken (another pass over S), the running max
+      // moved, O rescaled and P recomputed (p <= 2^8 otherwise, and the sum and
+      // O accumulate in fp32).
+      float lt = 0.f;
+      // a row without a running max yet (its first tile, or all keys so far
+      // masked) takes the exact-max path directly
+      const int pass_first = __any_sync(0xffffffffu, m_run == -INFINITY) ? 1 : 0;
+      for (int pass = pass_first; pass < 3; ++pass) {
+        if (pass == 1) {
+          // the exact row max of this tile
+          float mt = -INFINITY;
+#pragma unroll 1
+          for (int c4 = 0; c4 < 4; ++c4) {
+            float x[32];
+            tmem_ld32f(srow + 32 * c4, x);
+            tmem_wait_ld();
+            mt = fmaxf(mt, scale_mask32<true>(x, 32 * c4, t, sc, a, aux, scl, i));
+          }
+          const bool grow = mt > m_run;
+          float alpha = 1.f;
+          if (grow) {
+            alpha = m_run != -INFINITY ? ex2(m_run - mt) : 0.f;
+            m_run = mt;
+            l_run *= alpha;
+          }
+          // the TMEM accesses are warp-collective (.sync.aligned): the whole warp
+          // rescales its O rows, rows whose max did not move by 1
+          if (t > 0) {
+#pragma unroll 1
+            for (int c4 = 0; c4 < 4; ++c4) {
+              uint32_t u[32];
+              tmem_ld32(orow + 32 * c4, u);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
+              tmem_st32(orow + 32 * c4, u);
+            }
+            tmem_wait_st();
+          }
+          continue;
+        }
         // P = exp2(s - m_run) in fp16 into shared memory (K-major, 128-byte
         // swizzle: 16-byte chunk k of the row goes to chunk k ^ (r % 8) of its
         // 128-byte line; keys 64..127 in region 1), row sum in fp32
         const float mref = m_run == -INFINITY ? 0.f : m_run;
-        float l0 = 0.f, l1 = 0.f, mx = -INFINITY;
+        float l0 = 0.f, l1 = 0.f;
         float x[32];
         tmem_ld32f(srow, x);
         tmem_wait_ld();
 #pragma unroll 1
         for (int c4 = 0; c4 < 4; ++c4) {
-          mx = fmaxf(mx, scale_mask32(x, 32 * c4, t, sc, a, aux, scl, i));
+          scale_mask32<false>(x, 32 * c4, t, sc, a, aux, scl, i);
           uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
@@ -499,37 +541,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
           }
           if (c4 < 3) tmem_wait_ld();
         }
-        mt = mx;
         lt = l0 + l1;
-        // lazy running max: move it only when a row's tile max exceeds it by
-        // more than 2^8 (then p could leave the fp16 range); that row's P is
-        // recomputed against the new max and O rescaled
-        const bool grow = mt > m_run + 8.0f;
-        if (pass == 1 || !__any_sync(0xffffffffu, grow)) break;
-        redo = true;
-        // per row: alpha = 1 unless this row's max moved
-        float alpha = 1.f;
-        if (grow) {
-          alpha = m_run != -INFINITY ? ex2(m_run - mt) : 0.f;
-          m_run = mt;
-          l_run *= alpha;
-        }
-        // the TMEM accesses are warp-collective (.sync.aligned): the whole warp
-        // rescales its O rows, rows whose max did not move by 1
-        if (t > 0) {
-#pragma unroll 1
-          for (int c4 = 0; c4 < 4; ++c4) {
-            uint32_t u[32];
-            tmem_ld32(orow + 32 * c4, u);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
-            tmem_st32(orow + 32 * c4, u);
-          }
-          tmem_wait_st();
-        }
+        if (pass == 2) break;
+        const bool grow = !(lt <= 256.0f);  // also true for inf / NaN
+        if (!__any_sync(0xffffffffu, grow)) break;
       }
-      (void)redo;
       l_run += lt;
       // S_g(t) and the stage's auxiliary data have been read for the last time
       tc_fence_before();
