@@ -21,9 +21,11 @@
 //     multicast): 1 copy per packed tile, 2 per FP16 tile;
 //   * NC consumer warps take whole tiles round-robin, each owning 2 of the 2 NC
 //     stages (tile i -> stage i % 2NC -> warp i % NC), so every stage has a
-//     single consumer and a waiter is never a full barrier phase behind; splits
-//     get equal shares of the bytes.  Nibbles become fp16 in
-//     registers (exponent-bias trick + one fma with the group's scale/zero), and
+//     single consumer and a waiter is never a full barrier phase behind; every
+//     split gets an even share of the packed tiles and an even share of the
+//     FP16 tiles, so both its bytes and its arithmetic are balanced.  Nibbles
+//     become fp16 in registers (exponent-bias trick + one fma with the group's
+//     scale/zero), and
 //     both products run on tensor cores with mma.m16n8k16 (f32 accumulate):
 //       S^T[keys x 8 queries] = K^ (16 keys x 16 dims) . Q^T
 //       O^T[dims x 8 queries] += V^T (16 dims x 16 keys) . P^T
@@ -119,15 +121,26 @@ __device__ __forceinline__ uint32_t fp16_valid(const Geo& g, int tile) {
   return m;
 }
 
-// This split's tile range [t_lo, t_hi): splits get equal shares of the bytes
-// (a packed tile, 10 KB, counts 5; an FP16 tile, 8 KB, counts 4).
-__device__ __forceinline__ void split_range(const Geo& geo, int split, int S, int& t_lo, int& t_hi) {
-  const long long wp = 5ll * geo.NP;
-  const long long wt = wp + 4ll * (geo.NV + geo.NR);
-  const long long w_lo = (static_cast<long long>(split) * wt) / S;
-  const long long w_hi = (static_cast<long long>(split + 1) * wt) / S;
-  t_lo = static_cast<int>(w_lo <= wp ? (w_lo + 4) / 5 : geo.NP + (w_lo - wp + 3) / 4);
-  t_hi = static_cast<int>(w_hi <= wp ? (w_hi + 4) / 5 : geo.NP + (w_hi - wp + 3) / 4);
+// This split's tiles: an even share of the packed tiles [p_lo, p_lo + n_p)
+// and an even share of the FP16 tiles [f_lo, f_lo + n_f) (VL, ring, new
+// token), numbered 0 .. n_p + n_f - 1 packed first.  Consumer warps take them
+// round-robin, so the FP16 tiles (8 KB each, like a packed tile's 10 KB, but
+// about a tenth of its arithmetic) land on the warps that got one packed tile
+// fewer: the slowest warp of a split does ceil(n_p / NC) packed tiles plus at
+// most one FP16 tile, and every split streams about the same bytes.
+struct SplitTiles {
+  int p_lo, n_p, f_lo, n_f;
+  __device__ __forceinline__ int tile(int i) const { return i < n_p ? p_lo + i : f_lo + (i - n_p); }
+};
+__device__ __forceinline__ SplitTiles split_tiles(const Geo& geo, int split, int S) {
+  SplitTiles r;
+  const int NF = geo.NT - geo.NP;
+  r.p_lo = static_cast<int>((static_cast<long long>(split) * geo.NP) / S);
+  r.n_p = static_cast<int>((static_cast<long long>(split + 1) * geo.NP) / S) - r.p_lo;
+  const int f0 = static_cast<int>((static_cast<long long>(split) * NF) / S);
+  r.f_lo = geo.NP + f0;
+  r.n_f = static_cast<int>((static_cast<long long>(split + 1) * NF) / S) - f0;
+  return r;
 }
 
 struct WarpState {
@@ -391,14 +404,14 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
     const int pnp = *reinterpret_cast<volatile const int*>(c.state + HQ_STATE_NPACKED);
     const int pnv = *reinterpret_cast<volatile const int*>(c.state + HQ_STATE_NVL);
     const Geo pg = geo_of(min(max(pnp, 0), c.cap), min(max(pnv, 0), c.vl_cap), pT, R);
-    int p_lo, p_hi;
-    split_range(pg, split, S, p_lo, p_hi);
+    const SplitTiles pr = split_tiles(pg, split, S);
     const int npg = c.cap / PK;
-    const int a0 = min(max(p_lo, 0), npg), a1 = min(max(min(p_hi, pg.NP), a0), npg);
+    const int a0 = min(max(pr.p_lo, 0), npg), a1 = min(max(pr.p_lo + pr.n_p, a0), npg);
     const uint8_t* pages = c.pages + static_cast<size_t>(bh) * npg * HQ_PAGE_BYTES;
     for (int pgi = a0; pgi < a1; pgi += 16)  // 16 pages (165 KB) per prefetch
       prefetch_l2(pages + static_cast<size_t>(pgi) * HQ_PAGE_BYTES, min(16, a1 - pgi) * HQ_PAGE_BYTES);
-    const int v0 = min(max(p_lo - pg.NP, 0), c.vl_cap / FT), v1 = min(max(p_hi - pg.NP, v0), min(pg.NV, c.vl_cap / FT));
+    const int v0 = min(max(pr.f_lo - pg.NP, 0), c.vl_cap / FT);
+    const int v1 = min(max(pr.f_lo + pr.n_f - pg.NP, v0), min(pg.NV, c.vl_cap / FT));
     if (v1 > v0) {
       const size_t off = (static_cast<size_t>(bh) * c.vl_cap + v0 * FT) * D;
       prefetch_l2(c.kf + off, (v1 - v0) * FT * D * 2);
@@ -420,9 +433,8 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
     return;
   }
   const Geo geo = geo_of(n_packed, n_vl, T, R);
-  int t_lo, t_hi;
-  split_range(geo, split, S, t_lo, t_hi);
-  const int ntile = t_hi - t_lo;
+  const SplitTiles sp = split_tiles(geo, split, S);
+  const int ntile = sp.n_p + sp.n_f;
 
   __syncthreads();
 
@@ -455,7 +467,7 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
           break;
         }
         s_issued[s] = k + 1;
-        const int tile = t_lo + i;
+        const int tile = sp.tile(i);
         if (tile < geo.NP) {
           mbar_arrive_expect_tx(&full[s], PK_TX);
           bulk_g2s(st, pages + static_cast<size_t>(tile) * HQ_PAGE_BYTES, PK_TX, &full[s]);
@@ -497,7 +509,7 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
         break;
       }
       const uint8_t* st = smem + s * STAGE_BYTES;
-      const int tile = t_lo + i;
+      const int tile = sp.tile(i);
       if (tile < geo.NP) {
         packed_tile(ws, st, qf, tile, n_packed, qscale, g, t);
       } else {
