@@ -59,6 +59,30 @@ def test_decode_loop_with_reselection():
         t += 1
 
 
+def test_decode_from_an_empty_cache():
+    """No prefix at all: the first step attends to its own token alone; the cache
+    then grows by decode steps only, and the first reselection + merge (over
+    decoded positions, with the query buffer just filled) packs what left the
+    window; decoding continues over packed, VL and ring positions."""
+    B, Hq, Hkv, W = 2, 8, 2, 32
+    p = Pair(B, Hq, Hkv, 64, W, 500, cap=256, seed=21)  # the drawn prefix is never installed
+    assert p.g.state()["T"] == 0
+    q, k, v = synth.decode_tokens(21, B, Hq, Hkv, W + 64 + 5)
+    out, ref = p.decode(q[0], k[0], v[0])
+    check_decode(out, ref, "first step")
+    G = Hq // Hkv
+    want = np.repeat(v[0].astype(np.float32), G, axis=1)  # softmax over one key: the new V row
+    assert np.allclose(out.float().cpu().numpy(), want, atol=2e-3)
+    for t in range(1, W + 64):
+        out, ref = p.decode(q[t], k[t], v[t])
+        check_decode(out, ref, f"step {t}")
+    p.reselect_merge()
+    assert p.g.state()["n_packed"] == 64
+    for t in range(W + 64, W + 69):
+        out, ref = p.decode(q[t], k[t], v[t])
+        check_decode(out, ref, f"step {t}")
+
+
 def test_reselect_before_staging_is_full():
     """A merge with fewer than 64 staged tokens packs only what left the window."""
     p = Pair(1, 8, 2, 500, 64, 500, cap=800, seed=9)
