@@ -620,13 +620,30 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
   }
   __syncthreads();
   if (s_last) {
-    // log-sum-exp merge of the S partials of this (b, kv head): the (m, l) of
-    // every split go to shared memory first, so that the weights are known and
-    // each thread (one query, 4 dims) then has all its O loads in flight at once
+    // log-sum-exp merge of the S partials of this (b, kv head).  The threads
+    // split into ngrp groups, each summing the O partials of every ngrp-th split
+    // for one (query, 4 dims) item; a thread's first PER O loads are issued
+    // before the (m, l) of the splits are gathered and weighed, so both round
+    // trips to L2 overlap, and the groups' sums meet in shared memory.
     const float* pb = parts + static_cast<size_t>(bh) * S * PART_FLOATS;
     float* sm_m = reinterpret_cast<float*>(smem);      // [S][8]: m, then the split weight
     float* sm_l = sm_m + 64 * 8;                        // [S][8]
     float* sm_inv = sm_l + 64 * 8;                      // [8]
+    float4* red = reinterpret_cast<float4*>(sm_inv + 8);  // [ngrp][items]
+    constexpr int PER = 8;
+    const int items = G * (D / 4);
+    const bool grouped = items <= NTHREADS;             // else one pass over items per thread stride
+    const int ngrp = grouped ? max(1, min(NTHREADS / items, S)) : 1;
+    const int grp = grouped ? threadIdx.x / items : 0;
+    const int it0 = threadIdx.x - grp * items;
+    const bool mine = grouped && grp < ngrp;
+    const float4* osrc = reinterpret_cast<const float4*>(pb + 16 + (it0 / (D / 4)) * D) + it0 % (D / 4);
+    float4 ov[PER];
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      const int sp = grp + j * ngrp;
+      ov[j] = (mine && sp < S) ? __ldcg(osrc + sp * (PART_FLOATS / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     for (int i = threadIdx.x; i < S * 8; i += NTHREADS) {
       sm_m[i] = __ldcg(pb + (i >> 3) * PART_FLOATS + (i & 7));
       sm_l[i] = __ldcg(pb + (i >> 3) * PART_FLOATS + 8 + (i & 7));
@@ -646,23 +663,64 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
       sm_inv[qc] = ll > 0.f ? 1.0f / ll : 0.f;
     }
     __syncthreads();
-    for (int it = threadIdx.x; it < G * (D / 4); it += NTHREADS) {
+    auto store_out = [&](int it, const float4& acc) {
       const int qc = it / (D / 4), d4 = it % (D / 4);
-      const float4* src = reinterpret_cast<const float4*>(pb + 16 + qc * D) + d4;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 16
-      for (int sp = 0; sp < S; ++sp) {
-        const float4 o = __ldcg(src + sp * (PART_FLOATS / 4));
-        const float w = sm_m[sp * 8 + qc];
-        acc.x = fmaf(w, o.x, acc.x);
-        acc.y = fmaf(w, o.y, acc.y);
-        acc.z = fmaf(w, o.z, acc.z);
-        acc.w = fmaf(w, o.w, acc.w);
-      }
       const float inv = sm_inv[qc];
       __half2* dst = reinterpret_cast<__half2*>(out + (static_cast<size_t>(b) * c.Hq + kvh * G + qc) * D) + 2 * d4;
       dst[0] = __floats2half2_rn(acc.x * inv, acc.y * inv);
       dst[1] = __floats2half2_rn(acc.z * inv, acc.w * inv);
+    };
+    if (grouped) {
+      if (mine) {
+        const int qc = it0 / (D / 4);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+          const int sp = grp + j * ngrp;
+          const float w = sp < S ? sm_m[sp * 8 + qc] : 0.f;
+          acc.x = fmaf(w, ov[j].x, acc.x);
+          acc.y = fmaf(w, ov[j].y, acc.y);
+          acc.z = fmaf(w, ov[j].z, acc.z);
+          acc.w = fmaf(w, ov[j].w, acc.w);
+        }
+        for (int sp = grp + PER * ngrp; sp < S; sp += ngrp) {  // more than PER splits per group
+          const float4 o = __ldcg(osrc + sp * (PART_FLOATS / 4));
+          const float w = sm_m[sp * 8 + qc];
+          acc.x = fmaf(w, o.x, acc.x);
+          acc.y = fmaf(w, o.y, acc.y);
+          acc.z = fmaf(w, o.z, acc.z);
+          acc.w = fmaf(w, o.w, acc.w);
+        }
+        red[grp * items + it0] = acc;
+      }
+      __syncthreads();
+      if (threadIdx.x < items) {
+        float4 acc = red[threadIdx.x];
+        for (int g2 = 1; g2 < ngrp; ++g2) {
+          const float4 o = red[g2 * items + threadIdx.x];
+          acc.x += o.x;
+          acc.y += o.y;
+          acc.z += o.z;
+          acc.w += o.w;
+        }
+        store_out(threadIdx.x, acc);
+      }
+    } else {
+      for (int it = threadIdx.x; it < items; it += NTHREADS) {
+        const int qc = it / (D / 4), d4 = it % (D / 4);
+        const float4* src = reinterpret_cast<const float4*>(pb + 16 + qc * D) + d4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int sp = 0; sp < S; ++sp) {
+          const float4 o = __ldcg(src + sp * (PART_FLOATS / 4));
+          const float w = sm_m[sp * 8 + qc];
+          acc.x = fmaf(w, o.x, acc.x);
+          acc.y = fmaf(w, o.y, acc.y);
+          acc.z = fmaf(w, o.z, acc.z);
+          acc.w = fmaf(w, o.w, acc.w);
+        }
+        store_out(it, acc);
+      }
     }
     // every split of this head has consumed its tiles: append the new token to
     // the ring (slot T % R) and this group's queries to the query buffer
