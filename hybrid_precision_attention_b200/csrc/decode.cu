@@ -64,6 +64,7 @@ constexpr int OFF_VC = 4096, OFF_KS = 8192, OFF_VS = 9216, OFF_MASK = 10240;
 constexpr int OFF_FV = FT * FSTRIDE;           // V rows of an FP16 tile
 constexpr int STAGE_BYTES = 10368;             // max(10256, 2 * 16 * 256 = 8192), 128-aligned
 constexpr int PART_FLOATS = 16 + 8 * D;        // m[8], l[8], O[8][128]
+constexpr int MAX_SPLITS = 64;                 // splits per (b, kv head)
 constexpr uint32_t PK_TX = HQ_PAGE_VLMASK + 16;   // codes, scale/zero words and the bitmap: one copy
 static_assert(OFF_VC == HQ_PAGE_VCODES && OFF_KS == HQ_PAGE_KSZ && OFF_VS == HQ_PAGE_VSZ && OFF_MASK == HQ_PAGE_VLMASK,
               "a packed stage is a verbatim copy of the page prefix");
@@ -626,9 +627,8 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
     // before the (m, l) of the splits are gathered and weighed, so both round
     // trips to L2 overlap, and the groups' sums meet in shared memory.
     const float* pb = parts + static_cast<size_t>(bh) * S * PART_FLOATS;
-    float* sm_m = reinterpret_cast<float*>(smem);      // [S][8]: m, then the split weight
-    float* sm_l = sm_m + 64 * 8;                        // [S][8]
-    float* sm_inv = sm_l + 64 * 8;                      // [8]
+    float* sm_m = reinterpret_cast<float*>(smem);      // [S][8]: the split weights
+    float* sm_inv = sm_m + 2 * 64 * 8;                  // [8]
     float4* red = reinterpret_cast<float4*>(sm_inv + 8);  // [ngrp][items]
     constexpr int PER = 8;
     const int items = G * (D / 4);
@@ -644,23 +644,30 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
       const int sp = grp + j * ngrp;
       ov[j] = (mine && sp < S) ? __ldcg(osrc + sp * (PART_FLOATS / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    for (int i = threadIdx.x; i < S * 8; i += NTHREADS) {
-      sm_m[i] = __ldcg(pb + (i >> 3) * PART_FLOATS + (i & 7));
-      sm_l[i] = __ldcg(pb + (i >> 3) * PART_FLOATS + 8 + (i & 7));
-    }
-    __syncthreads();
-    if (threadIdx.x < G) {
-      const int qc = threadIdx.x;
-      float mm = -INFINITY;
-      for (int sp = 0; sp < S; ++sp) mm = fmaxf(mm, sm_m[sp * 8 + qc]);
-      float ll = 0.f;
-      for (int sp = 0; sp < S; ++sp) {
-        const float ms = sm_m[sp * 8 + qc];
-        const float w = ms == -INFINITY ? 0.f : ex2(ms - mm);
-        sm_m[sp * 8 + qc] = w;
-        ll += w * sm_l[sp * 8 + qc];
+    // split weights: warp qc weighs query qc's splits, lane s holding splits s
+    // and s + 32 (S <= 64), with warp-wide max and sum
+    static_assert(MAX_SPLITS <= 64, "two splits per lane");
+    for (int qc = warp; qc < G; qc += NTHREADS / 32) {
+      float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+      if (lane < S) {
+        m0 = __ldcg(pb + lane * PART_FLOATS + qc);
+        l0 = __ldcg(pb + lane * PART_FLOATS + 8 + qc);
       }
-      sm_inv[qc] = ll > 0.f ? 1.0f / ll : 0.f;
+      if (lane + 32 < S) {
+        m1 = __ldcg(pb + (lane + 32) * PART_FLOATS + qc);
+        l1 = __ldcg(pb + (lane + 32) * PART_FLOATS + 8 + qc);
+      }
+      float mm = fmaxf(m0, m1);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, o));
+      const float w0 = m0 == -INFINITY ? 0.f : ex2(m0 - mm);
+      const float w1 = m1 == -INFINITY ? 0.f : ex2(m1 - mm);
+      float ll = w0 * l0 + w1 * l1;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ll += __shfl_xor_sync(0xffffffffu, ll, o);
+      if (lane < S) sm_m[lane * 8 + qc] = w0;
+      if (lane + 32 < S) sm_m[(lane + 32) * 8 + qc] = w1;
+      if (lane == 0) sm_inv[qc] = ll > 0.f ? 1.0f / ll : 0.f;
     }
     __syncthreads();
     auto store_out = [&](int it, const float4& acc) {
@@ -753,7 +760,7 @@ DecodeShape decode_shape(const hq_cache& c, int sms) {
   int s = d.wide ? sms / units : (3 * sms) / units;
   const int cap_s = d.wide ? (nt_max + NC_WIDE - 1) / NC_WIDE : (nt_max + NC_NARROW - 1) / NC_NARROW;  // ~one tile per consumer warp
   if (s > cap_s) s = cap_s;
-  if (s > 64) s = 64;
+  if (s > MAX_SPLITS) s = MAX_SPLITS;
   if (s < 1) s = 1;
   d.S = s;
   return d;
