@@ -241,6 +241,21 @@ def oracle_sample(min_seconds=10.0, max_steps=64, steps=None):
     return gbs, float(np.mean(times)), i, threads, times, nbytes
 
 
+def aggregate_ranks(ms_local, units_local, world, device):
+    """The job's timed duration and work over all ranks: the max of the ranks'
+    device-timed durations (the job ends with its slowest rank) and the sum of
+    the units (bytes) they processed.  Every rank makes the same two collectives."""
+    if world == 1:
+        return float(ms_local), float(units_local)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms_local)], dtype=torch.float64, device=device)
+    u = torch.tensor([float(units_local)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -353,12 +368,9 @@ def run_ours(args, rank, world, local_rank):
     dec_ms = [evs[i][0].elapsed_time(evs[i][1]) for i in range(args.steps)]
     mnt_ms = [evs[i][1].elapsed_time(evs[i][2]) for i in range(args.steps)]
     total_ms = evs[0][0].elapsed_time(evs[-1][2])
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms_max = float(t.item())
     bytes_local = sum(period_bytes(T_first + PERIOD * i) for i in range(args.steps)) * COPIES
-    value = bytes_local * world / (total_ms_max * 1e-3) / 1e9
+    total_ms_max, bytes_all = aggregate_ranks(total_ms, bytes_local, world, dev)
+    value = bytes_all / (total_ms_max * 1e-3) / 1e9
     n_decodes = PERIOD * COPIES * args.steps
     us_per_decode = total_ms_max * 1e3 / n_decodes
     peak, peak_kind = load_peaks()
@@ -403,11 +415,9 @@ def run_ours(args, rank, world, local_rank):
             e1.record(stream)
         torch.cuda.synchronize()
         e_ms = e0.elapsed_time(e1)
-        te = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e_bytes = sum(period_bytes(T_e + PERIOD * i) for i in range(n_e2e)) * COPIES * world
-        e2e = {"value": e_bytes / (float(te.item()) * 1e-3) / 1e9, "unit": UNIT,
+        e_ms_max, e_bytes = aggregate_ranks(e_ms, sum(period_bytes(T_e + PERIOD * i) for i in range(n_e2e)) * COPIES,
+                                            world, dev)
+        e2e = {"value": e_bytes / (e_ms_max * 1e-3) / 1e9, "unit": UNIT,
                "h2d_bytes_per_step": PERIOD * COPIES * (qd.numel() + kd.numel() + vd.numel()) * 2,
                "d2h_bytes_per_step": PERIOD * COPIES * out.numel() * 2,
                "steps": n_e2e, "api": "hq_decode_attn / hq_select_vlines / hq_pack_merge via the Python binding, eager"}
