@@ -81,3 +81,27 @@ def test_decode_uses_current_representation():
         K, V = c.rep(0, 0)
         assert K.shape[0] == 400 + t + 1
         assert np.allclose(o[0], attend(qd[t, 0], K, V, 1 / np.sqrt(128)), rtol=0, atol=0)
+
+
+def test_decode_from_an_empty_cache_closed_forms():
+    """No prefix: the first step is a softmax over one key, so every query head
+    returns its kv head's new V row exactly; the second step is a two-key
+    softmax in closed form over the two FP16 rows (both still in the window)."""
+    B, Hq, Hkv, W = 1, 4, 2, 8
+    G = Hq // Hkv
+    r = hybrid.HybridCacheRef(B, Hq, Hkv, W, 500, 64)
+    q, k, v = synth.decode_tokens(4, B, Hq, Hkv, 2)
+    o0 = r.decode(q[0], k[0], v[0])
+    for h in range(Hq):
+        assert np.array_equal(o0[0, h], v[0][0, h // G].astype(np.float64))
+    o1 = r.decode(q[1], k[1], v[1])
+    sm = 1.0 / np.sqrt(128)
+    for h in range(Hq):
+        kv = h // G
+        K = np.stack([k[0][0, kv], k[1][0, kv]]).astype(np.float64)
+        V = np.stack([v[0][0, kv], v[1][0, kv]]).astype(np.float64)
+        s = K @ q[1][0, h].astype(np.float64) * sm
+        p = np.exp(s - s.max())
+        want = (p / p.sum()) @ V
+        assert np.allclose(o1[0, h], want, rtol=1e-12, atol=1e-12)
+    assert r.T == 2 and r.n_packed == 0
