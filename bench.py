@@ -32,6 +32,7 @@ bounded sample of the same workload (single decode steps of the 32K layer).
 from __future__ import annotations
 
 import argparse
+import datetime
 import hashlib
 import json
 import os
@@ -158,9 +159,13 @@ def decode_traffic_record():
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+    """nvidia-smi clocks and throttle reasons, sampled every INTERVAL_MS from
+    start() on (nvidia-smi needs a moment before its first sample, so start it
+    before the warm-up); summary() keeps the samples whose own timestamps fall
+    between begin() and end(), i.e. inside the timed region."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+    INTERVAL_MS = 25
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
 
@@ -168,11 +173,12 @@ class ClockSampler:
         self.index = index
         self.proc = None
         self.lines = []
+        self.t_begin = self.t_end = None
 
-    def __enter__(self):
+    def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", str(self.INTERVAL_MS)],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -180,31 +186,55 @@ class ClockSampler:
             self.proc = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def begin(self):
+        self.t_begin = datetime.datetime.now()
 
-    def __exit__(self, *a):
+    def end(self):
+        self.t_end = datetime.datetime.now()
+
+    def stop(self):
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+            self.t.join(timeout=5)
+
+    def __enter__(self):
+        self.start()
+        self.begin()
+        return self
+
+    def __exit__(self, *a):
+        self.end()
+        self.stop()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
 
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        slack = datetime.timedelta(milliseconds=self.INTERVAL_MS)
         for ln in self.lines:
             parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 8:
+            if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[0]))
-                mx = float(parts[1])
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
+            except ValueError:
+                ts = None
+            if ts is not None and self.t_begin is not None and self.t_end is not None:
+                if ts < self.t_begin - slack or ts > self.t_end + slack:
+                    continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
             except ValueError:
                 continue
-            for nm, val in zip(names, parts[4:8]):
+            for nm, val in zip(names, parts[5:9]):
                 if val.lower().startswith("active"):
                     reasons.add(nm)
         if not sm:
@@ -344,22 +374,26 @@ def run_ours(args, rank, world, local_rank):
         if ev is not None:
             ev[2].record(stream)
 
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            step()
-    stream.synchronize()
-    T_first = caches[0].state()["T"]
-    # timed region
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    sampler = ClockSampler(local_rank)
-    with sampler:
+    sampler = ClockSampler(local_rank).start()  # sampling from the warm-up on; summarised over the timed region
+    try:
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                step()
+        stream.synchronize()
+        T_first = caches[0].state()["T"]
+        # timed region
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        sampler.begin()
         with torch.cuda.stream(stream):
             for i in range(args.steps):
                 step(evs[i])
         torch.cuda.synchronize()
+        sampler.end()
+    finally:
+        sampler.stop()
     if world > 1:
         dist.barrier()
     for c in caches:
@@ -540,7 +574,6 @@ def main():
         run_reference(args, rank, world)
         return
     if world > 1:
-        import datetime
         import torch
         import torch.distributed as dist
         torch.cuda.set_device(local_rank)
