@@ -20,8 +20,9 @@ definition written out:
   ``q[2b] | q[2b+1] << 4``.
 * the dequantised value is ``zero + q * scale``.
 
-FP8 e4m3 (prefill's quantised tiles; HyQuant README, Overview item 2: "the
-bulk of the attention GEMMs run in low precision (INT8/FP8 ...)").  The
+FP8 e4m3 (prefill's quantised tiles; HyQuant README, Overview item 2: most of
+prefill's attention matrix products use a low-precision format such as INT8
+or FP8).  The
 rounding below is written from the OCP 8-bit floating point specification
 (E4M3: bias 7, 3 mantissa bits, no infinities, largest finite 448, smallest
 subnormal 2^-9), round-to-nearest-even with saturation to +-448.  Per-block
