@@ -31,7 +31,9 @@
  *
  * Conventions for every entry point
  *   - All tensor pointers are DEVICE pointers, 16-byte aligned, owned by the
- *     caller; the library allocates nothing and keeps no global state.
+ *     caller; the library allocates nothing.  Its only state is the last error
+ *     message of each host thread (hq_last_error) and, for
+ *     hq_decode_attn_noalloc alone, a fixed device scratch array of its own.
  *   - fp16 tensors are passed as uint16_t* (IEEE binary16 bit patterns).
  *   - Calls are asynchronous on `stream`.  Arguments are validated on the host
  *     before anything is launched; on a non-HQ_OK status nothing was launched.
