@@ -16,13 +16,14 @@
 //   sel_pass<true>   per-row log-sum-exp from the partials, then
 //                    S^T = K . Q^T (M = 128 keys, N = the queries) into TMEM;
 //                    per key (one TMEM lane per thread) the sum over queries of
-//                    exp2(s - lse) -> score_j.  No atomics: each key's score is
-//                    finished inside one CTA.
-//   topk             one CTA per (b, kv head): 8-bit radix select on the float
-//                    bit patterns (scores are >= 0, so the bit order is the value
-//                    order) over the scores held in shared memory -> exact k-th
-//                    value, then an ordered compaction writes the chosen
-//                    positions ascending, ties to the lowest positions
+//                    exp2(s - lse) -> score_j, and a histogram of the scores'
+//                    bits 30..20 (scores are >= 0, so the bit order is the value
+//                    order).  Each key's score is finished inside one CTA.
+//   topk             one CTA per (b, kv head): the bin holding the k-th largest
+//                    score from the histogram, the bin's scores gathered into
+//                    shared memory, a bit-by-bit search of their low 20 bits ->
+//                    the exact k-th value, then an ordered compaction writes the
+//                    chosen positions ascending, ties to the lowest positions
 // Keys are rebuilt as fp16 in their current representation (dense prefix in
 // init mode; ring, VL row or dequantised K4V4 record in decode mode) by four
 // builder warps straight into the 128-byte-swizzled K-major operand layout.
