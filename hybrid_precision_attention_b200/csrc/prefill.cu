@@ -25,21 +25,26 @@
 //   vl_prep          -inf bias on the vertical lines and the VL rows of K and V
 //                    gathered into contiguous 128-row tiles (positions padded with
 //                    INT_MAX)
-//   prefill_kernel   one CTA per (128-query tile, query head, batch):
-//                      warps 0-3  softmax, one query row per thread = one TMEM lane
-//                      warp 4     TMA producers: lane 0 Q once and the K tiles (with
-//                                 their score bias or VL positions and K scales),
-//                                 lane 1 the V tiles; 2 stages each
-//                      warp 5     TMEM allocation and the tcgen05.mma issue
-//                    key tiles in order: FP8 tiles (QK on kind::f8f6f4), VL tiles
-//                    and window tiles (QK on kind::f16); S = Q K^T lands in one of
-//                    two TMEM buffers, the softmax reads it, writes P (fp16) to
-//                    shared memory in the 128-byte-swizzled K-major layout, and
-//                    O += P V (kind::f16, V MN-major) accumulates in TMEM.  QK runs
-//                    two tiles ahead of the softmax; a K stage is free once its QK
-//                    is done, a V stage once its PV is.  The running max is
-//                    refreshed lazily (O in TMEM is rescaled only when the max
-//                    grows by more than 2^8).
+//   prefill_kernel   one CTA per (pair of 128-query tiles, query head, batch),
+//                    longest rows first; both query tiles share every K / V tile:
+//                      warps 0-7  two softmax warpgroups, one per query tile, one
+//                                 query row per thread = one TMEM lane
+//                      warp 8     TMA producers: lane 0 both query tiles once and
+//                                 the K tiles (with their score bias or VL
+//                                 positions and K scales), lane 1 the V tiles
+//                      warp 9     TMEM allocation and the tcgen05.mma issue,
+//                                 event-driven over the four MMAs of a tile
+//                    key tiles in order: VL tiles and the window's tiles first
+//                    (QK on kind::f16 with the fp16 queries), then the e4m3 tiles
+//                    (QK on kind::f8f6f4); once the fp16 tiles are done, the
+//                    64 KB of fp16 queries serve as a second K / V stage.  S = Q K^T
+//                    of each query tile lands in its own TMEM columns; its softmax
+//                    group reads S, writes P (fp16) to shared memory in the
+//                    128-byte-swizzled K-major layout, and O += P V (kind::f16,
+//                    V MN-major) accumulates in TMEM.  One pass per tile against
+//                    the running max; only when a row sum leaves 2^8 (every row's
+//                    first tile, rarely later) is the exact tile max taken, O
+//                    rescaled and P recomputed.
 // All mbarrier waits are bounded (about 1 s); a timeout sets the error word and
 // the CTA drains its copies and MMAs before releasing TMEM.
 #include <climits>
