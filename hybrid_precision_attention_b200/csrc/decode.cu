@@ -38,7 +38,10 @@
 //     (b, kv head) merges them with a log-sum-exp (atomic ticket, no waiting);
 //   * the last CTA of each (b, kv head) also appends that head's new token to
 //     the ring and its queries to the query buffer (every split of the head is
-//     done reading by then); the last CTA of the grid advances T.
+//     done reading by then); the last CTA of the grid advances T;
+//   * launched with programmatic dependent launch: a CTA prefetches its split's
+//     pages and VL rows into L2 before it waits for the previous grid, and lets
+//     the next grid launch as soon as its own wait is over.
 #include "common.cuh"
 
 namespace hq {
