@@ -18,9 +18,11 @@ whole step (decode + selection + merge), in GB/s, with microseconds per
 decode token-layer alongside.
 
 Algorithmic bytes of one decode step of one (b, kv head): 160 B per K4V4
-position (64 + 16 bytes of K codes/scales and the same for V), 512 B per FP16
-position (vertical lines, recent window and staged tokens, the new token
-included), plus the query and output rows.
+position outside the vertical-line set (64 + 16 bytes of K codes/scales and the
+same for V), 512 B per FP16 position (vertical lines, recent window and staged
+tokens, the new token included), plus the query and output rows.  A vertical
+line's key and value are read from the VL store; the K4V4 record that its page
+still carries is layout overhead, seen in the ncu traffic, not counted here.
 
 Multi-GPU: the path has no exchange step; ``--gpus N`` (under torchrun) runs N
 independent replicas, one per GPU, the timing is the max over ranks and the
@@ -62,9 +64,10 @@ def k_of(n, rho_bp):
 
 
 def decode_bytes(n_packed, n_vl, T):
-    """Algorithmic bytes of one decode step (all kv heads) at the given state (before the step)."""
+    """Algorithmic bytes of one decode step (all kv heads) at the given state (before the step):
+    packed positions outside the VL set at 160 B, FP16 rows (VL, ring, new token) at 512 B."""
     fp16_rows = n_vl + (T + 1 - n_packed)
-    per_head = n_packed * 160 + fp16_rows * 512
+    per_head = (n_packed - n_vl) * 160 + fp16_rows * 512
     return B * HKV * per_head + 2 * B * HQ * D * 2
 
 
