@@ -173,7 +173,11 @@ class ClockSampler:
               "clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index):
-        self.index = index
+        # nvidia-smi numbers GPUs physically; under CUDA_VISIBLE_DEVICES the
+        # process's device `index` is the index-th entry of that list (an index
+        # or a UUID, both of which nvidia-smi -i accepts)
+        visible = [x.strip() for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
+        self.index = visible[index] if index < len(visible) else str(index)
         self.proc = None
         self.lines = []
         self.t_begin = self.t_end = None

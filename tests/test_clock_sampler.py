@@ -60,3 +60,10 @@ def test_missing_nvidia_smi_reads_as_unavailable(tmp_path, monkeypatch):
     monkeypatch.setenv("PATH", str(tmp_path))
     out = _run(bench.ClockSampler(0), warm=0.0, timed=0.05, after=0.0)
     assert out == {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+
+
+def test_sampler_queries_the_visible_gpu(monkeypatch):
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "5,GPU-1234")
+    assert bench.ClockSampler(0).index == "5" and bench.ClockSampler(1).index == "GPU-1234"
+    monkeypatch.delenv("CUDA_VISIBLE_DEVICES")
+    assert bench.ClockSampler(0).index == "0"
