@@ -148,3 +148,29 @@ def test_prefill_hybrid_error_below_uniform_fp8():
     wide = attention.prefill_head(Q[0, 0], lay.k[0, 0], lay.v[0, 0], is_vl, 256, SM)
     assert _mse(hyb, ref) < _mse(uni, ref)
     assert _mse(wide, ref) < _mse(hyb, ref)
+
+
+def test_prefill_ref_maps_query_heads_to_their_kv_head():
+    """The multi-head driver: query head hq of batch b reads kv head hq // G of
+    the same batch (GQA groups of consecutive query heads) with that kv head's
+    own vertical lines.  Checked head by head against the per-(i, j) loops on
+    inputs where every kv head and batch differs."""
+    rng = np.random.default_rng(6)
+    B, Hq, Hkv, L, W = 2, 4, 2, 20, 3
+    G = Hq // Hkv
+    Q = (rng.standard_normal((B, Hq, L, 128)) * 2).astype(np.float16)
+    K = (rng.standard_normal((B, Hkv, L, 128)) * 2).astype(np.float16)
+    V = rng.standard_normal((B, Hkv, L, 128)).astype(np.float16)
+    vl = [[np.array([0, 4, 11]), np.array([2, 7])], [np.array([1, 5, 6, 13]), np.array([3])]]
+    got = attention.prefill_ref(Q, K, V, vl, W, SM)
+    assert sorted(got) == [(b, h) for b in range(B) for h in range(Hq)]
+    for b in range(B):
+        for hq in range(Hq):
+            kv = hq // G
+            is_vl = np.zeros(L, bool)
+            is_vl[vl[b][kv]] = True
+            want = _prefill_loops(Q[b, hq], K[b, kv], V[b, kv], is_vl, W, SM)
+            assert np.allclose(got[(b, hq)], want, rtol=1e-11, atol=1e-13), (b, hq)
+    # a subset of heads and rows gives the same rows
+    sub = attention.prefill_ref(Q, K, V, vl, W, SM, rows=np.arange(8, 20), heads=[(1, 3), (0, 1)])
+    assert np.array_equal(sub[(1, 3)], got[(1, 3)][8:]) and np.array_equal(sub[(0, 1)], got[(0, 1)][8:])

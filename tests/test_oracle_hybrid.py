@@ -72,15 +72,130 @@ def test_promotion_and_demotion_rules():
     assert np.array_equal(K[drop], formats.dequant_k4v4(cc, s, z))
 
 
-def test_decode_uses_current_representation():
-    lay, c, _, _ = _cache(B=1, Hkv=1, Hq=4)
-    qd, kd, vd = synth.decode_tokens(1, 1, 4, 1, 3)
-    from oracle.attention import attend
+def _rep_by_hand(K16, packed_upto, vl_rows, upto):
+    """Keys [0, upto) of one (b, kv head) built row by row from the raw FP16
+    history: a vertical line gives its VL row, a packed position the
+    dequantisation of the record its own FP16 value packs to, anything later
+    its FP16 value (no call into the cache object)."""
+    D = K16.shape[-1]
+    out = np.empty((upto, D))
+    for j in range(upto):
+        if j in vl_rows:
+            out[j] = vl_rows[j].astype(np.float64)
+        elif j < packed_upto:
+            c, s, z = formats.pack_k4v4(K16[j][None])
+            out[j] = formats.dequant_k4v4(c, s, z)[0]
+        else:
+            out[j] = K16[j].astype(np.float64)
+    return out
+
+
+def _column_mass_by_hand(K, queries, n, sm):
+    """queries: list of (position, q row); explicit loops over heads, queries and keys."""
+    mass = np.zeros(n)
+    for p, q in queries:
+        logits = [sum(float(q[d]) * K[j, d] for d in range(K.shape[1])) * sm for j in range(p + 1)]
+        mx = max(logits)
+        w = [np.exp(x - mx) for x in logits]
+        z = sum(w)
+        for j in range(min(n, p + 1)):
+            mass[j] += w[j] / z
+    return mass
+
+
+def test_reselect_brute_force_pre_merge():
+    """Decode-mode reselection (HyQuant digest, method paragraph: the column mass
+    of the buffered queries, recomputed every 64 tokens) against explicit loops.
+    Every buffered query of every head of the group is paired with its own
+    position (a query sees keys j <= its position only), the keys are taken in
+    the representation they have before the merge (the positions about to leave
+    the window are still FP16), and the k largest scores are kept."""
+    B, Hq, Hkv, L, W, steps = 2, 4, 2, 24, 4, 6
+    G = Hq // Hkv
+    lay = synth.planted_layer(31, B, Hq, Hkv, L)
+    c = hybrid.HybridCacheRef(B, Hq, Hkv, W, 2500, cap=64)
+    vl0, _ = c.init_from_prefix(lay.k, lay.v, lay.q_tail)
+    qd, kd, vd = synth.decode_tokens(31, B, Hq, Hkv, steps)
+    for t in range(steps):
+        c.decode(qd[t], kd[t], vd[t])
+    T = L + steps
+    assert c.T == T and c.n_packed == L - W and c.staged() == steps
+    K16 = np.concatenate([lay.k, np.moveaxis(kd, 0, 2)], axis=2)      # [B, Hkv, T, D] raw history
+    n = T - W
+    kk = select.k_of(n, 2500)
+    vl, scores = c.reselect()
+    for b in range(B):
+        for h in range(Hkv):
+            rows = {int(p): lay.k[b, h, p] for p in vl0[b][h]}         # prefix VL rows are the dense rows
+            K = _rep_by_hand(K16[b, h], L - W, rows, T)
+            queries = [(L + t, qd[t, b, hh]) for hh in range(h * G, (h + 1) * G) for t in range(steps)]
+            want = _column_mass_by_hand(K, queries, n, 1 / np.sqrt(128))
+            assert np.allclose(scores[b][h], want, rtol=1e-11, atol=1e-14), (b, h)
+            order = sorted(range(n), key=lambda j: (-want[j], j))[:kk]
+            assert list(vl[b][h]) == sorted(order), (b, h)
+    # the state is untouched by the reselection itself
+    assert c.T == T and c.n_packed == L - W
+
+
+def test_reselect_with_an_empty_query_buffer():
+    """Right after a prefix install nothing is buffered: every score is zero and
+    the stable top-k keeps the lowest k positions."""
+    lay, c, _, _ = _cache(L=200, W=32, B=1, Hq=4, Hkv=2)
+    assert c.qbuf == []
+    vl, sc = c.reselect()
+    n = 200 - 32
+    for h in range(2):
+        assert np.array_equal(sc[0][h], np.zeros(n))
+        assert np.array_equal(vl[0][h], np.arange(select.k_of(n, 500)))
+
+
+def test_merge_keeps_fp16_of_a_line_that_just_left_the_window():
+    """A position that leaves the window at this merge and is selected as a
+    vertical line keeps its FP16 value (it still has one), not its new record;
+    this holds for a prefix position and for a decoded one alike."""
+    lay, c, vl0, _ = _cache(L=300, W=40, B=1, Hq=2, Hkv=1)
+    qd, kd, vd = synth.decode_tokens(2, 1, 2, 1, 64)
+    for t in range(64):
+        c.decode(qd[t], kd[t], vd[t])
+    old_np = c.n_packed
+    assert old_np == 260 and c.T == 364
+    K16 = np.concatenate([lay.k[0, 0], kd[:, 0, 0]])
+    V16 = np.concatenate([lay.v[0, 0], vd[:, 0, 0]])
+    exited = [262, 290, 311]            # in [old_np, T - W) = [260, 324); 311 is a decoded token
+    new = np.array(sorted(list(vl0[0][0][:3]) + exited), np.int64)
+    c.merge([[new]])
+    assert c.n_packed == 324
+    K, V = c.rep(0, 0)
+    for p in exited:
+        assert np.array_equal(K[p], K16[p].astype(np.float64))
+        assert np.array_equal(V[p], V16[p].astype(np.float64))
+        # and that differs from the record the position now has
+        deq = formats.dequant_k4v4(c.kq[0, 0, p], c.ks[0, 0, p], c.kz[0, 0, p])
+        assert not np.array_equal(K[p], deq)
+        cc, s, z = formats.pack_k4v4(K16[p])
+        assert np.array_equal(c.kq[0, 0, p], cc)
+
+
+def test_decode_against_loops_over_a_hand_built_cache():
+    """Decode steps over a prefix with lines, window and staged tokens equal
+    softmax loops over keys/values built row by row from the raw history."""
+    B, Hq, Hkv, L, W = 1, 4, 2, 40, 8
+    G = Hq // Hkv
+    lay = synth.planted_layer(17, B, Hq, Hkv, L)
+    c = hybrid.HybridCacheRef(B, Hq, Hkv, W, 1000, cap=64)
+    vl0, _ = c.init_from_prefix(lay.k, lay.v, lay.q_tail)
+    qd, kd, vd = synth.decode_tokens(17, B, Hq, Hkv, 3)
+    from oracle.attention import attend_loops
     for t in range(3):
         o = c.decode(qd[t], kd[t], vd[t])
-        K, V = c.rep(0, 0)
-        assert K.shape[0] == 400 + t + 1
-        assert np.allclose(o[0], attend(qd[t, 0], K, V, 1 / np.sqrt(128)), rtol=0, atol=0)
+        T = L + t + 1
+        for h in range(Hkv):
+            K16 = np.concatenate([lay.k[0, h], kd[:t + 1, 0, h]])
+            V16 = np.concatenate([lay.v[0, h], vd[:t + 1, 0, h]])
+            K = _rep_by_hand(K16, L - W, {int(p): lay.k[0, h, p] for p in vl0[0][h]}, T)
+            V = _rep_by_hand(V16, L - W, {int(p): lay.v[0, h, p] for p in vl0[0][h]}, T)
+            want = attend_loops(qd[t, 0, h * G:(h + 1) * G], K, V, 1 / np.sqrt(128))
+            assert np.allclose(o[0, h * G:(h + 1) * G], want, rtol=1e-11, atol=1e-13), (t, h)
 
 
 def test_decode_from_an_empty_cache_closed_forms():
