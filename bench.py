@@ -63,19 +63,19 @@ def k_of(n, rho_bp):
     return 0 if n <= 0 or rho_bp <= 0 else min(n, (n * rho_bp + 9999) // 10000)
 
 
-def decode_bytes(n_packed, n_vl, T):
+def decode_bytes(n_packed, n_vl, T, b=B, hkv=HKV, hq=HQ):
     """Algorithmic bytes of one decode step (all kv heads) at the given state (before the step):
     packed positions outside the VL set at 160 B, FP16 rows (VL, ring, new token) at 512 B."""
     fp16_rows = n_vl + (T + 1 - n_packed)
     per_head = (n_packed - n_vl) * 160 + fp16_rows * 512
-    return B * HKV * per_head + 2 * B * HQ * D * 2
+    return b * hkv * per_head + 2 * b * hq * D * 2
 
 
-def period_bytes(T0):
-    """Algorithmic decode bytes of one 64-token period starting right after a merge at length T0."""
+def period_bytes(T0, b=B, hkv=HKV, hq=HQ, tokens=PERIOD):
+    """Algorithmic decode bytes of `tokens` decode steps starting right after a merge at length T0."""
     n_packed = T0 - W
     n_vl = k_of(n_packed, RHO_BP)
-    return sum(decode_bytes(n_packed, n_vl, T0 + t) for t in range(PERIOD))
+    return sum(decode_bytes(n_packed, n_vl, T0 + t, b, hkv, hq) for t in range(tokens))
 
 
 def load_peaks():
@@ -84,6 +84,16 @@ def load_peaks():
         d = json.load(open(p))
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def load_extra_peaks():
+    """Peaks this repository measured on the same GPUs (the committed record
+    profiles/peaks_b200.json, written by `bench.py --measure-peaks`): the dense
+    e4m3 tensor peak and the read-only HBM streaming ceiling."""
+    p = os.path.join(ROOT, "profiles", "peaks_b200.json")
+    if os.path.exists(p):
+        return json.load(open(p))
+    return {}
 
 
 def load_bf16_peak():
@@ -118,7 +128,7 @@ def run_prefill(dev, reps=5, warmup=2):
     n_vl = c.state()["k_sel"]
     vl = c.vl_sel
     out = torch.empty_like(q_d)
-    ws = torch.empty(hq.hq_prefill_workspace_bytes(1, PF_HQ, PF_HKV, PF_L), dtype=torch.uint8, device=dev)
+    ws = torch.empty(hq.hq_prefill_workspace_bytes(1, PF_HQ, PF_HKV, PF_L, vl.shape[2]), dtype=torch.uint8, device=dev)
     for _ in range(warmup):
         hq.hq_prefill_attn(q_d, k_d, v_d, vl, n_vl, W, out=out, ws=ws)
     torch.cuda.synchronize()
@@ -134,31 +144,44 @@ def run_prefill(dev, reps=5, warmup=2):
     flops = prefill_flops(PF_L, PF_HQ)
     tflops = flops / (ms * 1e-3) / 1e12
     bf16, kind = load_bf16_peak()
-    fp8 = 2.0 * bf16
+    extra = load_extra_peaks()
+    if "fp8_e4m3_tflops" in extra:
+        fp8, fp8_kind = float(extra["fp8_e4m3_tflops"]), "measured e4m3 GEMM (profiles/peaks_b200.json)"
+    else:
+        fp8, fp8_kind = 2.0 * bf16, f"{kind} bf16 x 2 (nominal fp8/bf16 ratio)"
     mixed = 1.0 / (0.5 / fp8 + 0.5 / bf16)
     return {"workload": f"causal hybrid prefill, B=1, L=32768, Hq=32, Hkv=8, D=128, W=128, rho=5% ({n_vl} lines per kv head)",
             "ms": ms, "tflops": tflops, "calls": reps,
             "roofline": {"kernel": "prefill (pre-pass + prefill_kernel)", "bound": "tensor", "achieved": tflops,
                          "peak": fp8, "unit": "TFLOP/s", "frac": tflops / fp8, "traffic": None,
-                         "peak_kind": f"{kind} bf16 x 2 (nominal fp8/bf16 ratio)",
+                         "peak_kind": fp8_kind,
                          "mixed_ceiling": mixed,
                          "note": "QK of quantised tiles on e4m3 (fp8 rate), P.V on f16 (bf16 rate): half the flops at "
                                  "each rate, so the ceiling of this mix is the mixed_ceiling figure"}}
 
 
-def decode_traffic_record():
-    """DRAM bytes per decode launch from the committed ncu summary, if it matches the current kernel source."""
-    src = open(os.path.join(ROOT, "hybrid_precision_attention_b200", "csrc", "decode.cu"), "rb").read()
-    sha = hashlib.sha256(src).hexdigest()
-    p = os.path.join(ROOT, "profiles", "decode_kernel_32k.md")
+def decode_traffic_record(bytes_per_launch):
+    """DRAM traffic of a decode launch from the committed ncu record
+    (profiles/decode_kernel_32k.traffic.json: the captured launch's T, its
+    algorithmic bytes and its DRAM read + write bytes), scaled to this run's
+    average launch by algorithmic bytes (the traffic grows with the positions
+    scanned).  None unless the record was taken on the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", "decode_kernel_32k.traffic.json")
     if not os.path.exists(p):
-        return None
-    txt = open(p).read()
-    m_sha = re.search(r"decode\.cu sha256:\s*([0-9a-f]{64})", txt)
-    m_b = re.search(r"dram bytes per launch \(read \+ write\):\s*([0-9]+)", txt)
-    if not m_sha or not m_b or m_sha.group(1) != sha:
-        return None
-    return int(m_b.group(1))
+        return None, None
+    rec = json.load(open(p))
+    if rec.get("sources_sha256") != kernel_sources_sha("decode.cu"):
+        return None, rec
+    scaled = rec["dram_bytes"] * bytes_per_launch / rec["algorithmic_bytes"]
+    return scaled, rec
+
+
+def kernel_sources_sha(*names):
+    """sha256 over the named kernel sources plus the shared device header."""
+    h = hashlib.sha256()
+    for n in list(names) + ["common.cuh"]:
+        h.update(open(os.path.join(ROOT, "hybrid_precision_attention_b200", "csrc", n), "rb").read())
+    return h.hexdigest()
 
 
 class ClockSampler:
@@ -423,10 +446,15 @@ def run_ours(args, rank, world, local_rank):
     dec_avg_us = sum(dec_ms) * 1e3 / n_decodes
     bytes_per_launch = bytes_local / n_decodes
     achieved = bytes_per_launch / (dec_avg_us * 1e-6) / 1e9
-    traffic = decode_traffic_record()
+    traffic, trec = decode_traffic_record(bytes_per_launch)
+    extra = load_extra_peaks()
     roof = {"kernel": "decode_kernel", "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-            "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
-            "avg_launch_us": dec_avg_us, "algorithmic_bytes_per_launch": bytes_per_launch}
+            "frac": achieved / peak, "traffic": traffic, "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json)",
+            "avg_launch_us": dec_avg_us, "algorithmic_bytes_per_launch": bytes_per_launch,
+            "traffic_record": trec}
+    if "hbm_read_gbs" in extra:
+        roof["read_ceiling_gbs"] = float(extra["hbm_read_gbs"])
+        roof["frac_of_read_ceiling"] = achieved / float(extra["hbm_read_gbs"])
 
     # end-to-end leg: the public API with host buffers, copies inside the timed region
     e2e = None
@@ -470,6 +498,22 @@ def run_ours(args, rank, world, local_rank):
     if not args.no_prefill:
         prefill = run_prefill(dev)
 
+    working_set_mb = COPIES * caches[0].nbytes() / 1e6
+    legs = {}
+    if not args.no_legs and world == 1:
+        for c in caches:
+            c._ws.clear()
+        del caches
+        torch.cuda.empty_cache()
+        legs["decode_1k"] = run_small_layer_leg(dev)
+        torch.cuda.empty_cache()
+        legs["qwen3_8b_36_layers_b16"] = run_multilayer_leg(dev, 36, 16, 32)
+        legs["qwen3_32b_64_layers_b32"] = run_multilayer_leg(dev, 64, 32, 64, seed0=900)
+        for lg in ("qwen3_8b_36_layers_b16", "qwen3_32b_64_layers_b32"):
+            legs[lg]["frac_of_copy_peak"] = legs[lg]["gbs"] / peak
+            if "hbm_read_gbs" in extra:
+                legs[lg]["frac_of_read_ceiling"] = legs[lg]["gbs"] / float(extra["hbm_read_gbs"])
+
     if rank != 0:
         return
     cpu = None
@@ -478,6 +522,20 @@ def run_ours(args, rank, world, local_rank):
         cpu = {"value": gbs, "unit": UNIT, "cores": threads, "kind": "oracle",
                "sample": f"{n} single decode steps of the 32K layer by the float64 oracle ({sec:.2f} s each); "
                          f"prefix install not timed"}
+        if legs:
+            g1, s1 = oracle_unit_rate(HQ, 1024, steps=8)
+            legs["decode_1k"]["cpu_baseline"] = {"value": s1 * 1e6, "unit": "us per decode step", "cores": threads,
+                                                 "kind": "oracle", "sample": "8 single decode steps of the 1K layer"}
+            legs["qwen3_8b_36_layers_b16"]["cpu_baseline"] = {
+                "value": gbs, "unit": UNIT, "cores": threads, "kind": "oracle",
+                "sample": "extrapolated: the 32K layer's single-step oracle rate (one (layer, b) unit of this shape), "
+                          "the same bytes per second for all 576 units"}
+            g4, s4 = oracle_unit_rate(64, 32768, steps=2)
+            legs["qwen3_32b_64_layers_b32"]["cpu_baseline"] = {
+                "value": g4, "unit": UNIT, "cores": threads, "kind": "oracle",
+                "steps_per_s": 1.0 / (s4 * 64 * 32),
+                "sample": f"extrapolated: 2 single decode steps of one (layer, b) unit (Hq=64, Hkv=8, 32K) at "
+                          f"{s4:.2f} s each, multiplied by 64 layers x 32 sequences for steps/s"}
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
@@ -485,12 +543,256 @@ def run_ours(args, rank, world, local_rank):
             "select_merge_share": sum(mnt_ms) / max(sum(dec_ms) + sum(mnt_ms), 1e-9),
             "config": {"workload": WORKLOAD, "B": B, "Hq": HQ, "Hkv": HKV, "D": D, "prefix": L, "W": W,
                        "rho": RHO_BP / 10000, "layer_copies": COPIES, "decode_tokens_per_step": PERIOD,
-                       "l2": f"{COPIES} rotating layer copies, {COPIES * caches[0].nbytes() / 1e6:.0f} MB working set > 126 MB L2",
+                       "l2": f"{COPIES} rotating layer copies, {working_set_mb:.0f} MB working set > 126 MB L2",
                        "parallelism": f"replicas x{world}"},
-            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "prefill": prefill,
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "prefill": prefill, "legs": legs,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": sampler.summary()}
     print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- further workloads
+
+def _events(n):
+    import torch
+    return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+
+def run_small_layer_leg(dev, steps=4, copies=72):
+    """Decode at a 1K prefix (B=1, Hq=32, Hkv=8): `copies` rotating copies of the
+    layer (about 180 MB, larger than L2), one CUDA graph per 64-token period of
+    decode launches (one per token and copy) and one for the copies'
+    reselection + merge.  Reports microseconds per decode step, with and
+    without the amortised reselection + merge."""
+    import torch
+    from hybrid_precision_attention_b200 import hq, synth
+    Ls = 1024
+    cap = Ls + PERIOD * (steps + 4) + 256
+    lay = synth.planted_layer(7, B, HQ, HKV, Ls)
+    k_d, v_d, qt_d = [torch.from_numpy(a).to(dev) for a in (lay.k, lay.v, lay.q_tail)]
+    caches = []
+    for _ in range(copies):
+        c = hq.HybridCache(B, HQ, HKV, cap, W, RHO_BP, device=dev)
+        hq.hq_select_vlines(c, k_d, qt_d)
+        hq.hq_pack_merge(c, k_d, v_d)
+        for op in (hq.OP_SELECT, hq.OP_MERGE, hq.OP_DECODE):
+            c.workspace(op)
+        caches.append(c)
+    qn, kn, vn = synth.decode_tokens(8, B, HQ, HKV, PERIOD)
+    q_t, k_t, v_t = [torch.from_numpy(a).to(dev) for a in (qn, kn, vn)]
+    out = torch.empty((B, HQ, D), dtype=torch.float16, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def dec():
+        for t in range(PERIOD):
+            for c in caches:
+                hq.hq_decode_attn(c, q_t[t], k_t[t], v_t[t], out=out, stream=stream)
+
+    def mnt():
+        for c in caches:
+            hq.hq_select_vlines(c, stream=stream)
+            hq.hq_pack_merge(c, stream=stream)
+
+    with torch.cuda.stream(stream):
+        dec()
+        mnt()
+    stream.synchronize()
+    g_dec, g_mnt = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_dec, stream=stream):
+        dec()
+    with torch.cuda.graph(g_mnt, stream=stream):
+        mnt()
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            g_dec.replay()
+            g_mnt.replay()
+    stream.synchronize()
+    T0 = caches[0].state()["T"]
+    evs = [_events(3) for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for i in range(steps):
+            evs[i][0].record(stream)
+            g_dec.replay()
+            evs[i][1].record(stream)
+            g_mnt.replay()
+            evs[i][2].record(stream)
+    torch.cuda.synchronize()
+    for c in caches:
+        assert c.state()["err"] == 0, c.state()
+    dec_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    tot_ms = sum(e[0].elapsed_time(e[2]) for e in evs)
+    n = PERIOD * copies * steps
+    nbytes = sum(period_bytes(T0 + PERIOD * i) for i in range(steps)) * copies
+    return {"workload": f"decode, one layer, B=1, Hq=32, Hkv=8, D=128, prefix {Ls}, rho=5%, W=128; {copies} rotating "
+                        f"layer copies ({copies * caches[0].nbytes() / 1e6:.0f} MB > L2); CUDA graphs of 64-token periods",
+            "us_per_decode_step": dec_ms * 1e3 / n, "us_per_decode_step_with_select_merge": tot_ms * 1e3 / n,
+            "gbs": nbytes / (dec_ms * 1e-3) / 1e9, "periods": steps, "decode_launches": n,
+            "select_merge_share": (tot_ms - dec_ms) / tot_ms}
+
+
+def run_multilayer_leg(dev, layers, b, hq_heads, tokens=8, warm=2, seed0=800):
+    """One decode step over every layer of a model-shaped cache held resident
+    (prefix 32768, Hkv=8, D=128, rho=5%, W=128, planted generator drawn on the
+    device), timed with CUDA events over `tokens` steps replayed from a CUDA
+    graph of one step (a decode launch per layer); then one reselection +
+    merge of every layer, timed on its own, to give the 64-token period cost."""
+    import torch
+    from hybrid_precision_attention_b200 import hq, synth
+    Ll = 32768
+    caches = []
+    for layer in range(layers):
+        k, v, q_tail, _ = synth.planted_layer_device(seed0 + layer, b, hq_heads, HKV, Ll, dev)
+        c = hq.HybridCache(b, hq_heads, HKV, Ll + 128, W, RHO_BP, device=dev)
+        hq.hq_select_vlines(c, k, q_tail)
+        hq.hq_pack_merge(c, k, v)
+        del k, v, q_tail
+        c.workspace(hq.OP_DECODE)
+        caches.append(c)
+    torch.cuda.synchronize()
+    for c in caches:
+        c._ws.pop(hq.OP_SELECT, None)   # the init-mode selection workspace is sized for a dense prefix
+    torch.cuda.empty_cache()
+    cache_gb = sum(c.nbytes() for c in caches) / 1e9
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed0 + 99)
+    qs = torch.randn((tokens + warm, b, hq_heads, D), generator=gen, device=dev).to(torch.float16)
+    ks = torch.randn((tokens + warm, b, HKV, D), generator=gen, device=dev).to(torch.float16)
+    vs = torch.randn((tokens + warm, b, HKV, D), generator=gen, device=dev).to(torch.float16)
+    q_in = torch.empty((b, hq_heads, D), dtype=torch.float16, device=dev)
+    k_in = torch.empty((b, HKV, D), dtype=torch.float16, device=dev)
+    v_in = torch.empty((b, HKV, D), dtype=torch.float16, device=dev)
+    out = torch.empty((b, hq_heads, D), dtype=torch.float16, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def one_step():
+        for c in caches:
+            hq.hq_decode_attn(c, q_in, k_in, v_in, out=out, stream=stream)
+
+    def feed(i):
+        q_in.copy_(qs[i], non_blocking=True)
+        k_in.copy_(ks[i], non_blocking=True)
+        v_in.copy_(vs[i], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        feed(0)
+        one_step()           # eager: sets function attributes
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        one_step()
+    with torch.cuda.stream(stream):
+        for i in range(1, warm):
+            feed(i)
+            g.replay()
+    stream.synchronize()
+    T0 = caches[0].state()["T"]
+    evs = _events(2 * tokens)
+    with torch.cuda.stream(stream):
+        for i in range(tokens):
+            feed(warm + i)
+            evs[2 * i].record(stream)
+            g.replay()
+            evs[2 * i + 1].record(stream)
+    torch.cuda.synchronize()
+    for c in caches:
+        st = c.state()
+        assert st["err"] == 0 and st["T"] == T0 + tokens, st
+    step_ms = [evs[2 * i].elapsed_time(evs[2 * i + 1]) for i in range(tokens)]
+    n_packed = Ll - W
+    n_vl = k_of(n_packed, RHO_BP)
+    nbytes = sum(decode_bytes(n_packed, n_vl, T0 + i, b, HKV, hq_heads) for i in range(tokens)) * layers
+    ms = float(np.mean(step_ms))
+    # one reselection + merge of every layer (the tokens decoded so far are the buffered queries)
+    e0, e1 = _events(2)
+    with torch.cuda.stream(stream):
+        for c in caches:
+            c.workspace(hq.OP_SELECT)
+            c.workspace(hq.OP_MERGE)
+        e0.record(stream)
+        for c in caches:
+            hq.hq_select_vlines(c, stream=stream)
+            hq.hq_pack_merge(c, stream=stream)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    for c in caches:
+        assert c.state()["err"] == 0, c.state()
+    mnt_ms = e0.elapsed_time(e1)
+    gbs = nbytes / (sum(step_ms) * 1e-3) / 1e9
+    res = {"workload": f"{layers} layers resident, B={b}, Hq={hq_heads}, Hkv=8, D=128, prefix 32768, rho=5%, W=128 "
+                       f"({cache_gb:.1f} GB of hybrid cache); one decode step over every layer from a CUDA graph",
+           "ms_per_step": ms, "steps_per_s": 1e3 / ms, "tokens_per_s": b * 1e3 / ms,
+           "gb_per_step": nbytes / tokens / 1e9, "gbs": gbs, "steps": tokens,
+           "select_merge_ms_all_layers": mnt_ms,
+           "ms_per_step_with_select_merge_amortised": ms + mnt_ms / PERIOD,
+           "select_merge_share_of_period": mnt_ms / (PERIOD * ms + mnt_ms)}
+    del caches
+    torch.cuda.empty_cache()
+    return res
+
+
+def oracle_unit_rate(Hq_, Ls, steps=2):
+    """Oracle GB/s on single decode steps of one (layer, b) unit: B=1, Hq_, Hkv=8, prefix Ls."""
+    from hybrid_precision_attention_b200 import synth
+    from oracle import hybrid
+    lay = synth.planted_layer(5, 1, Hq_, HKV, Ls)
+    c = hybrid.HybridCacheRef(1, Hq_, HKV, W, RHO_BP, Ls + 64)
+    c.init_from_prefix(lay.k, lay.v, lay.q_tail)
+    q, k, v = synth.decode_tokens(5, 1, Hq_, HKV, steps)
+    tt, bb = 0.0, 0
+    for i in range(steps):
+        st = (c.n_packed, len(c.vl[0][0]), c.T)
+        t0 = time.perf_counter()
+        c.decode(q[i], k[i], v[i])
+        tt += time.perf_counter() - t0
+        bb += decode_bytes(*st, 1, HKV, Hq_)
+    return bb / tt / 1e9, tt / steps
+
+
+def measure_peaks(dev):
+    """The dense e4m3 GEMM peak (torch._scaled_mm, 8192^3, per-tensor scales,
+    bf16 out; best of 20 by CUDA events) and the read-only HBM ceiling (the
+    library's streaming-read helper over 8 GiB, best of 10 at 1..4 CTAs per
+    SM).  Prints one JSON line: the record committed as profiles/peaks_b200.json."""
+    import torch
+    from hybrid_precision_attention_b200 import hq
+    n = 8192
+    a = torch.randn((n, n), device=dev).to(torch.float8_e4m3fn)
+    bt = torch.randn((n, n), device=dev).to(torch.float8_e4m3fn).t()
+    one = torch.ones((), device=dev)
+    for _ in range(5):
+        torch._scaled_mm(a, bt, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+    best = 1e9
+    for _ in range(20):
+        e0, e1 = _events(2)
+        e0.record()
+        torch._scaled_mm(a, bt, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    fp8 = 2.0 * n ** 3 / (best * 1e-3) / 1e12
+    del a, bt
+    buf = torch.ones(8 << 30, dtype=torch.uint8, device=dev)
+    sink = torch.zeros(4, dtype=torch.int32, device=dev)
+    rd = {}
+    for cps in (1, 2, 3, 4):
+        for _ in range(2):
+            hq.hq_diag_stream_read(buf, sink, cps)
+        tb = 1e9
+        for _ in range(10):
+            e0, e1 = _events(2)
+            e0.record()
+            hq.hq_diag_stream_read(buf, sink, cps)
+            e1.record()
+            torch.cuda.synchronize()
+            tb = min(tb, e0.elapsed_time(e1))
+        rd[cps] = buf.numel() / (tb * 1e-3) / 1e9
+    best_cps = max(rd, key=rd.get)
+    rec = {"fp8_e4m3_tflops": fp8, "fp8_how": f"torch._scaled_mm e4m3 x e4m3 -> bf16, {n}^3 (2 n^3 flops), best of 20, CUDA events",
+           "hbm_read_gbs": rd[best_cps], "hbm_read_how": f"hq_diag_stream_read over 8 GiB (16-byte streaming loads, "
+                                                         f"{best_cps} CTAs of 512 threads per SM), best of 10, CUDA events",
+           "hbm_read_by_ctas_per_sm": rd, "gpu": torch.cuda.get_device_name(dev),
+           "when": datetime.datetime.utcnow().strftime("%Y-%m-%dT%H:%M:%SZ")}
+    print(json.dumps(rec), flush=True)
 
 
 def profile_decode():
@@ -546,7 +848,7 @@ def profile_prefill():
     c = hq.HybridCache(1, PF_HQ, PF_HKV, Lp, W, RHO_BP)
     hq.hq_select_vlines(c, k, Q[:, :, Lp - 64:].contiguous())
     torch.cuda.synchronize()
-    ws = torch.empty(hq.hq_prefill_workspace_bytes(1, PF_HQ, PF_HKV, Lp), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(hq.hq_prefill_workspace_bytes(1, PF_HQ, PF_HKV, Lp, c.vl_sel.shape[2]), dtype=torch.uint8, device="cuda")
     for _ in range(3):
         hq.hq_prefill_attn(Q, k, v, c.vl_sel, c.state()["k_sel"], W, ws=ws)
     torch.cuda.synchronize()
@@ -564,6 +866,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-legs", action="store_true", help="skip the 1K, 36-layer and 64-layer decode workloads")
+    ap.add_argument("--measure-peaks", action="store_true", help="measure the e4m3 GEMM peak and the read-only HBM ceiling")
     ap.add_argument("--profile-decode", action="store_true", help="small case for ncu: 4 decode steps of one 32K layer")
     ap.add_argument("--profile-prefill", action="store_true", help="small case for ncu: 3 prefill calls at L=8192")
     ap.add_argument("--profile-select", action="store_true", help="small case for ncu: one decode-mode reselection at 32K")
@@ -576,6 +880,10 @@ def main():
         return
     if args.profile_select:
         profile_select()
+        return
+    if args.measure_peaks:
+        import torch
+        measure_peaks(torch.device("cuda", 0))
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

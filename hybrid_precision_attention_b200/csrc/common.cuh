@@ -9,6 +9,9 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "../../include/hq.h"
 
 namespace hq {
@@ -23,6 +26,24 @@ __host__ __device__ __forceinline__ int ring_len(int W) { return HQ_RING_LEN(W);
 hq_status cuda_status(cudaError_t e, const char* where);
 // Host side: a failure path; always HQ_ERR_CUDA, recording `where` and e.
 hq_status cuda_fail(cudaError_t e, const char* where);
+
+// Host side: runs `set` (a kernel-attribute set-up) once per device for one
+// call site.  Thread-safe: concurrent first calls on a device wait for the one
+// that runs `set`; a failed set-up is not recorded, so the next call retries.
+struct DeviceOnce {
+  static constexpr int kMaxDevices = 64;
+  std::atomic<bool> done[kMaxDevices] = {};
+  std::mutex mu;
+  template <class F>
+  cudaError_t run(int dev, F&& set) {
+    if (dev >= 0 && dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev >= 0 && dev < kMaxDevices && done[dev].load(std::memory_order_relaxed)) return cudaSuccess;
+    const cudaError_t e = set();
+    if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) done[dev].store(true, std::memory_order_release);
+    return e;
+  }
+};
 
 // K4V4 page of position p of (b, kv head) bh
 __host__ __device__ __forceinline__ uint8_t* page_of(const hq_cache& c, size_t bh, int p) {

@@ -786,15 +786,16 @@ hq_status launch_decode(const hq_cache& c, const uint16_t* q, const uint16_t* kn
   const int smem = 2 * nc * STAGE_BYTES;
   int dev = 0;
   cudaGetDevice(&dev);
-  static bool attr_done[64] = {};
-  if (dev >= 64 || !attr_done[dev]) {
-    if (cudaFuncSetAttribute(decode_kernel<NC_WIDE, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             2 * NC_WIDE * STAGE_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(decode_kernel<NC_NARROW, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             2 * NC_NARROW * STAGE_BYTES) != cudaSuccess)
-      return cuda_fail(cudaGetLastError(), "decode attributes");
-    if (dev < 64) attr_done[dev] = true;
-  }
+  static DeviceOnce attrs;
+  const cudaError_t ea = attrs.run(dev, [] {
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<NC_WIDE, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         2 * NC_WIDE * STAGE_BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(decode_kernel<NC_NARROW, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               2 * NC_NARROW * STAGE_BYTES);
+    return e;
+  });
+  if (ea != cudaSuccess) return cuda_fail(ea, "decode attributes");
   unsigned int* tickets = reinterpret_cast<unsigned int*>(ws);
   float* parts = reinterpret_cast<float*>(static_cast<char*>(ws) + decode_counter_bytes(c));
   cudaLaunchConfig_t cfg = {};

@@ -13,8 +13,12 @@
 //     process exits.
 //   * Host code cannot use the array's name as a device address, so the first
 //     call on each device (with that device current) looks the address up with
-//     cudaGetSymbolAddress and remembers it.  Make that first call before any
-//     stream capture.
+//     cudaGetSymbolAddress and remembers it, together with the id of the
+//     device's current context.  A later call that finds a different context
+//     (the device was reset, or its primary context released and created
+//     again, which reloads the library's device code) looks it up again.  Make
+//     the first call on a device, and the first call after such a reset,
+//     before any stream capture.
 //   * All calls on a device share the one array and it keeps whatever the last
 //     call left in it: each call clears the completion counters (an async
 //     memset on the caller's stream) before the kernel.  Two calls whose
@@ -23,6 +27,7 @@
 //   * No allocation happens here: no cudaMalloc, cudaFree or allocating library
 //     routine.  A cache whose decode workspace would exceed the array is
 //     rejected with HQ_ERR_WORKSPACE before anything is launched.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -43,16 +48,48 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[HQ_NOALLOC_SCRA
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_scratch_addr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};
 
-// Device address of this device's scratch array (looked up once per device).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Id of the calling thread's current context (0 when it cannot be read, in
+// which case the address found first is kept).
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current && get_id && get_current(&ctx) == CUDA_SUCCESS && ctx != nullptr && get_id(ctx, &id) == CUDA_SUCCESS)
+    return id;
+  return 0;
+}
+
+// Device address of this device's scratch array (looked up once per device
+// and context).
 hq_status scratch_address(int dev, void** out) {
   if (dev < 0 || dev >= kMaxDevices) return HQ_ERR_UNSUPPORTED;
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  if (g_scratch_addr[dev] == nullptr || (ctx != 0 && ctx != g_scratch_ctx[dev])) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || p == nullptr) return hq::cuda_fail(e, "scratch address");
     g_scratch_addr[dev] = p;
+    // the lookup made the device's context current if no call had yet: record its id
+    g_scratch_ctx[dev] = ctx != 0 ? ctx : current_context_id();
   }
   *out = g_scratch_addr[dev];
   return HQ_OK;

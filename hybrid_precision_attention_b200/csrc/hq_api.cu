@@ -16,7 +16,7 @@ size_t decode_workspace(const hq_cache& c, int sms);
 size_t select_workspace(const hq_cache& c, bool need_scores);
 hq_status launch_select(const hq_cache& c, const uint16_t* kd, int L, const uint16_t* qe, int nq, float* scores_out,
                         void* ws, cudaStream_t st);
-size_t prefill_workspace(int B, int Hq, int Hkv, int L);
+size_t prefill_workspace(int B, int Hq, int Hkv, int L, int vl_stride);
 hq_status launch_prefill(int B, int Hq, int Hkv, int L, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                          const int32_t* vl_pos, int n_vl, int vl_stride, int W, float sm_scale, uint16_t* out, void* ws,
                          cudaStream_t st);
@@ -149,9 +149,9 @@ hq_status hq_decode_attn(const hq_cache* c, const uint16_t* q, const uint16_t* k
   return hq::launch_decode(*c, q, k_new, v_new, out, sm_scale, ws, sms, reinterpret_cast<cudaStream_t>(stream));
 }
 
-size_t hq_prefill_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t L, int32_t D) {
-  if (D != HQ_HEAD_DIM || B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || Hq % Hkv) return 0;
-  return hq::prefill_workspace(B, Hq, Hkv, L);
+size_t hq_prefill_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t L, int32_t D, int32_t vl_stride) {
+  if (D != HQ_HEAD_DIM || B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || Hq % Hkv || vl_stride < 0) return 0;
+  return hq::prefill_workspace(B, Hq, Hkv, L, vl_stride);
 }
 
 hq_status hq_prefill_attn(int32_t B, int32_t Hq, int32_t Hkv, int32_t L, int32_t D, const uint16_t* q,
@@ -161,7 +161,7 @@ hq_status hq_prefill_attn(int32_t B, int32_t Hq, int32_t Hkv, int32_t L, int32_t
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || L <= 0 || W < 0 || !(sm_scale > 0.0f)) return HQ_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return HQ_ERR_INVALID;
   if (n_vl < 0 || n_vl > vl_stride || (n_vl > 0 && !aligned16(vl_pos))) return HQ_ERR_INVALID;
-  if (!aligned16(ws) || ws_bytes < hq::prefill_workspace(B, Hq, Hkv, L)) return HQ_ERR_WORKSPACE;
+  if (!aligned16(ws) || ws_bytes < hq::prefill_workspace(B, Hq, Hkv, L, vl_stride)) return HQ_ERR_WORKSPACE;
   return hq::launch_prefill(B, Hq, Hkv, L, q, k, v, vl_pos, n_vl, vl_stride, W, sm_scale, out, ws,
                             reinterpret_cast<cudaStream_t>(stream));
 }

@@ -758,14 +758,16 @@ PfLayout pf_layout(int B, int Hq, int Hkv, int L, int n_vl) {
 
 }  // namespace
 
-// Workspace for any VL set of up to L positions.  Bytes [0, 4) of the workspace
-// receive the kernel's error word (non-zero if a bounded wait gave up).
-size_t prefill_workspace(int B, int Hq, int Hkv, int L) { return pf_layout(B, Hq, Hkv, L, L).total; }
+// Workspace for any VL set of up to vl_stride positions.  Bytes [0, 4) of the
+// workspace receive the kernel's error word (non-zero if a bounded wait gave up).
+size_t prefill_workspace(int B, int Hq, int Hkv, int L, int vl_stride) {
+  return pf_layout(B, Hq, Hkv, L, min(max(vl_stride, 0), L)).total;
+}
 
 hq_status launch_prefill(int B, int Hq, int Hkv, int L, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                          const int32_t* vl_pos, int n_vl, int vl_stride, int W, float sm_scale, uint16_t* out, void* ws,
                          cudaStream_t st) {
-  if (n_vl > L) return HQ_ERR_INVALID;
+  if (n_vl > L || n_vl > vl_stride) return HQ_ERR_INVALID;
   const PfLayout ly = pf_layout(B, Hq, Hkv, L, n_vl);
   char* w = static_cast<char*>(ws);
   uint32_t* err = reinterpret_cast<uint32_t*>(w + ly.err);
@@ -800,12 +802,10 @@ hq_status launch_prefill(int B, int Hq, int Hkv, int L, const uint16_t* q, const
   a.sq = sq; a.sk = sk; a.kbias = kbias; a.vlpos = vlpos; a.out = out; a.err = err;
   int dev = 0;
   cudaGetDevice(&dev);
-  static bool attr_done[64] = {};
-  if (dev >= 64 || !attr_done[dev]) {
-    if (cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PF_SMEM) != cudaSuccess)
-      return cuda_fail(cudaGetLastError(), "prefill setup");
-    if (dev < 64) attr_done[dev] = true;
-  }
+  static DeviceOnce attrs;
+  const cudaError_t ea = attrs.run(
+      dev, [] { return cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PF_SMEM); });
+  if (ea != cudaSuccess) return cuda_fail(ea, "prefill setup");
   prefill_kernel<<<dim3((ly.nblk + 1) / 2, Hq, B), PF_THREADS, PF_SMEM, st>>>(tm, a);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {

@@ -746,16 +746,16 @@ hq_status launch_select(const hq_cache& c, const uint16_t* kd, int L, const uint
   a.scores = scores_out ? scores_out : reinterpret_cast<float*>(w);
   a.qscale = (1.0f / sqrtf(static_cast<float>(D))) * LOG2E;
   const size_t smem = sel_smem_bytes(a.Mp);
-  static bool attr_done[64] = {};
-  if (dev >= 64 || !attr_done[dev]) {
+  static DeviceOnce attrs;
+  const cudaError_t ea = attrs.run(dev, [] {
     const int smem_max = static_cast<int>(sel_smem_bytes(((HQ_MAX_GQA * HQ_QBUF + 127) / 128) * 128));
-    if (cudaFuncSetAttribute(sel_pass<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max) != cudaSuccess ||
-        cudaFuncSetAttribute(sel_pass<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max) != cudaSuccess ||
-        cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (TK_CAND_MAX + TK_SMEM_MAX) * 4) !=
-            cudaSuccess)
-      return cuda_fail(cudaGetLastError(), "select setup");
-    if (dev < 64) attr_done[dev] = true;
-  }
+    cudaError_t e = cudaFuncSetAttribute(sel_pass<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(sel_pass<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (TK_CAND_MAX + TK_SMEM_MAX) * 4);
+    return e;
+  });
+  if (ea != cudaSuccess) return cuda_fail(ea, "select setup");
   dim3 grid(S, c.Hkv, c.B);
   sel_pass<false><<<grid, SEL_THREADS, smem, st>>>(a);
   sel_pass<true><<<grid, SEL_THREADS, smem, st>>>(a);

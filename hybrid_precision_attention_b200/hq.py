@@ -70,13 +70,16 @@ _lib.hq_decode_attn.argtypes = [_CP, _P, _P, _P, _P, ctypes.c_float, _P, _S, _P]
 _lib.hq_decode_attn_noalloc.restype = _I
 _lib.hq_decode_attn_noalloc.argtypes = [_CP, _P, _P, _P, _P, ctypes.c_float, _P]
 _lib.hq_prefill_workspace_bytes.restype = _S
-_lib.hq_prefill_workspace_bytes.argtypes = [_I, _I, _I, _I, _I]
+_lib.hq_prefill_workspace_bytes.argtypes = [_I, _I, _I, _I, _I, _I]
 _lib.hq_prefill_attn.restype = _I
 _lib.hq_prefill_attn.argtypes = [_I, _I, _I, _I, _I, _P, _P, _P, _P, _I, _I, _I, ctypes.c_float, _P, _P, _S, _P]
 
+_lib.hq_diag_stream_read.restype = _I
+_lib.hq_diag_stream_read.argtypes = [_P, _S, _P, _I, _P]
+
 EXPORTED = ("hq_abi_version", "hq_status_str", "hq_last_error", "hq_cache_validate", "hq_workspace_bytes", "hq_cache_reset",
             "hq_select_vlines", "hq_pack_merge", "hq_decode_attn", "hq_decode_attn_noalloc",
-            "hq_prefill_workspace_bytes", "hq_prefill_attn")
+            "hq_prefill_workspace_bytes", "hq_prefill_attn", "hq_diag_stream_read")
 
 
 def _check(st: int, what: str):
@@ -236,8 +239,19 @@ def hq_decode_attn_noalloc(cache: HybridCache, q, k_new, v_new, out=None, sm_sca
     return out
 
 
-def hq_prefill_workspace_bytes(B, Hq, Hkv, L, D=HQ_HEAD_DIM) -> int:
-    return int(_lib.hq_prefill_workspace_bytes(B, Hq, Hkv, L, D))
+def hq_prefill_workspace_bytes(B, Hq, Hkv, L, vl_stride, D=HQ_HEAD_DIM) -> int:
+    return int(_lib.hq_prefill_workspace_bytes(B, Hq, Hkv, L, D, vl_stride))
+
+
+def prefill_ws_regions(B, Hq, Hkv, L, D=HQ_HEAD_DIM) -> dict:
+    """Byte offsets of the documented prefill workspace regions (include/hq.h):
+    the error word, the e4m3 codes of Q and K, the fp16 values of V."""
+    Lp = (L + 127) // 128 * 128
+    al = lambda x: (x + 1023) // 1024 * 1024
+    q8 = al(16)
+    k8 = al(q8 + B * Hq * Lp * D)
+    v8 = al(k8 + B * Hkv * Lp * D)
+    return {"err": 0, "q8": q8, "k8": k8, "v16": v8, "Lp": Lp}
 
 
 def hq_prefill_attn(q, k, v, vl_pos, n_vl: int, W: int, sm_scale: float = None, out=None, ws=None, stream=None):
@@ -250,7 +264,7 @@ def hq_prefill_attn(q, k, v, vl_pos, n_vl: int, W: int, sm_scale: float = None, 
     _need(vl_pos, torch.int32, (B, Hkv, vl_pos.shape[2]), "vl_pos")
     if out is None:
         out = torch.empty_like(q)
-    n = hq_prefill_workspace_bytes(B, Hq, Hkv, L, D)
+    n = hq_prefill_workspace_bytes(B, Hq, Hkv, L, vl_pos.shape[2], D)
     if ws is None:
         ws = torch.empty(max(n, 1), dtype=torch.uint8, device=q.device)
     if sm_scale is None:
@@ -259,3 +273,9 @@ def hq_prefill_attn(q, k, v, vl_pos, n_vl: int, W: int, sm_scale: float = None, 
                                 ctypes.c_float(sm_scale), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
            "hq_prefill_attn")
     return out
+
+
+def hq_diag_stream_read(buf, sink, ctas_per_sm: int = 2, stream=None):
+    """Read-only HBM streaming pass over a device tensor (measurement helper)."""
+    _check(_lib.hq_diag_stream_read(_ptr(buf), buf.numel() * buf.element_size(), _ptr(sink), ctas_per_sm,
+                                    _stream(stream)), "hq_diag_stream_read")

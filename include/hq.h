@@ -53,7 +53,7 @@
 extern "C" {
 #endif
 
-#define HQ_ABI_VERSION 3
+#define HQ_ABI_VERSION 4
 #define HQ_HEAD_DIM 128       /* D: the only head size built */
 #define HQ_GROUP 32           /* K4V4 group length along D */
 #define HQ_STAGE 64           /* staged tokens before a merge = reselection period */
@@ -239,9 +239,20 @@ HQ_API hq_status hq_decode_attn(const hq_cache* c, const uint16_t* q, const uint
  * stored as e4m3_RN_sat(x / scale)); one softmax covers all three classes.
  *   q [B, Hq, L, D], k, v [B, Hkv, L, D], out [B, Hq, L, D]: fp16
  *   vl_pos int32 [B, Hkv, vl_stride], first n_vl entries ascending, < L
- * Workspace: hq_prefill_workspace_bytes().
+ *     (0 <= n_vl <= min(vl_stride, L))
+ * Workspace: at least hq_prefill_workspace_bytes(B, Hq, Hkv, L, D, vl_stride)
+ * bytes, 16-byte aligned; one call's workspace must not be shared with a call
+ * that can run at the same time.  It holds, in this order (each region starting
+ * on a 1024-byte boundary, Lp = L rounded up to a multiple of 128):
+ *   bytes [0, 4)  uint32 error word, cleared by the call: non-zero when a
+ *                 bounded wait of the kernel gave up (never expected; the
+ *                 output is then incomplete); read it after synchronising;
+ *   e4m3 codes of Q [B, Hq, Lp, D], e4m3 codes of K [B, Hkv, Lp, D],
+ *   fp16 values fp16(fp32(e4m3(V / scale)) * scale) of V [B, Hkv, Lp, D],
+ *   then the per-block scales and gathered VL rows (internal).
+ * Rows past L of the three coded tensors are zero.
  */
-HQ_API size_t hq_prefill_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t L, int32_t D);
+HQ_API size_t hq_prefill_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t L, int32_t D, int32_t vl_stride);
 HQ_API hq_status hq_prefill_attn(int32_t B, int32_t Hq, int32_t Hkv, int32_t L, int32_t D,
                           const uint16_t* q, const uint16_t* k, const uint16_t* v,
                           const int32_t* vl_pos, int32_t n_vl, int32_t vl_stride, int32_t W,
@@ -259,6 +270,9 @@ HQ_API hq_status hq_prefill_attn(int32_t B, int32_t Hq, int32_t Hkv, int32_t L, 
  * process exits.
  *   - The first call on a device (with that device current) looks up the
  *     array's device address; make that first call before any stream capture.
+ *     After the device is reset (cudaDeviceReset, or its primary context
+ *     released and created again) the next call sees a new context and looks
+ *     the address up again: make that call before any capture as well.
  *   - All calls on a device share the array and it keeps the last call's
  *     contents; each call clears what must start at zero itself.  Calls whose
  *     executions can overlap on the GPU (unordered streams) race on the array:
@@ -270,6 +284,17 @@ HQ_API hq_status hq_prefill_attn(int32_t B, int32_t Hq, int32_t Hkv, int32_t L, 
 #define HQ_NOALLOC_SCRATCH_BYTES (4u << 20)
 HQ_API hq_status hq_decode_attn_noalloc(const hq_cache* c, const uint16_t* q, const uint16_t* k_new,
                                         const uint16_t* v_new, uint16_t* out, float sm_scale, hq_stream_t stream);
+
+/*
+ * Measurement helper (no counterpart in the method): reads `bytes` (a multiple
+ * of 16) of device memory at `src` (16-byte aligned) with 16-byte streaming
+ * loads from sms * ctas_per_sm CTAs of 512 threads (1 <= ctas_per_sm <= 4),
+ * and XORs what it read into *sink (device, 4-byte aligned) so the loads are
+ * kept.  Timing it over a buffer far larger than L2 gives the read-only HBM
+ * bandwidth ceiling that a scan such as the decode step can approach.
+ */
+HQ_API hq_status hq_diag_stream_read(const void* src, size_t bytes, uint32_t* sink, int32_t ctas_per_sm,
+                                     hq_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -28,7 +28,7 @@ def test_library_exports_every_declared_symbol():
     missing = [n for n in _declared() if not hasattr(lib, n)]
     assert not missing, missing
     lib.hq_abi_version.restype = ctypes.c_int32
-    assert lib.hq_abi_version() == 3
+    assert lib.hq_abi_version() == 4
     lib.hq_status_str.restype = ctypes.c_char_p
     assert lib.hq_status_str(0) == b"ok"
 

@@ -25,7 +25,7 @@ def lib():
                        ("hq_pack_merge", [CP, P, P, I, P, S, P]),
                        ("hq_decode_attn", [CP, P, P, P, P, F, P, S, P]),
                        ("hq_prefill_attn", [I, I, I, I, I, P, P, P, P, I, I, I, F, P, P, S, P]),
-                       ("hq_prefill_workspace_bytes", [I, I, I, I, I]),
+                       ("hq_prefill_workspace_bytes", [I, I, I, I, I, I]),
                        ("hq_workspace_bytes", [CP, I, I]),
                        ("hq_status_str", [I]),
                        ("hq_last_error", [])):
@@ -100,10 +100,13 @@ def test_decode_rejections(lib, mem):
 
 def test_prefill_rejections(lib, mem):
     _, a = mem
-    need = lib.hq_prefill_workspace_bytes(1, 32, 8, 1000, 128)
+    need = lib.hq_prefill_workspace_bytes(1, 32, 8, 1000, 128, 64)
     assert need > 0
-    assert lib.hq_prefill_workspace_bytes(1, 32, 8, 1000, 64) == 0
-    assert lib.hq_prefill_workspace_bytes(1, 30, 8, 1000, 128) == 0
+    # the gathered vertical-line rows are sized by the row stride, not by L
+    assert lib.hq_prefill_workspace_bytes(1, 32, 8, 1000, 128, 1000) > need
+    assert lib.hq_prefill_workspace_bytes(1, 32, 8, 1000, 128, -1) == 0
+    assert lib.hq_prefill_workspace_bytes(1, 32, 8, 1000, 64, 64) == 0
+    assert lib.hq_prefill_workspace_bytes(1, 30, 8, 1000, 128, 64) == 0
     s = 1 / math.sqrt(128)
     pf = lambda B, Hq, Hkv, L, D, n_vl, stride, W, sc, ws, wsb, vl=a, q=a: lib.hq_prefill_attn(
         B, Hq, Hkv, L, D, q, a, a, vl, n_vl, stride, W, sc, a, ws, wsb, None)

@@ -113,7 +113,9 @@ def test_capacity_flag():
 
 @pytest.mark.slow
 def test_full_size_32k_layer():
-    """The 32K decode layer (B=1, Hq=32, Hkv=8): init, one step, 64-step period, reselect + merge, one step."""
+    """The 32K decode layer (B=1, Hq=32, Hkv=8): init, one step, a 64-step period
+    (every 8th step checked, so the ring's wrap at this geometry is covered),
+    reselect + merge, one step."""
     B, Hq, Hkv, L, W = 1, 32, 8, 32768, 128
     p = Pair(B, Hq, Hkv, L, W, 500, cap=L + 128, seed=0)
     p.init()
@@ -121,8 +123,12 @@ def test_full_size_32k_layer():
     out, ref = p.decode(q[0], k[0], v[0])
     check_decode(out, ref, "first step")
     for t in range(1, 64):
-        hq().hq_decode_attn(p.g, dev(q[t]), dev(k[t]), dev(v[t]))
-        p.r.append(q[t], k[t], v[t])
+        if t % 8 == 0 or t == 63:   # every 8th step (and the last, with the ring full) against the oracle
+            out, ref = p.decode(q[t], k[t], v[t])
+            check_decode(out, ref, f"step {t}")
+        else:
+            hq().hq_decode_attn(p.g, dev(q[t]), dev(k[t]), dev(v[t]))
+            p.r.append(q[t], k[t], v[t])
     p.reselect_merge()
     out, ref = p.decode(q[64], k[64], v[64])
     check_decode(out, ref, "after merge")

@@ -7,17 +7,20 @@ Two workloads of the method's evaluation shapes, every layer resident at once:
 Each layer is drawn on the device with the planted-vertical-line recipe, its
 vertical lines are selected from its own last 64 queries and the prefix is
 packed; then one decode step runs over every layer.  Sampled (layer, b, kv head)
-units are checked against the oracle, which rebuilds that unit's cache from the
-dense prefix and the GPU's vertical-line set: the K4V4 records bit-exactly, the
-VL rows bit-exactly, and the decode output within the decode tolerances.
+units are checked against the oracle: the unit's column-mass scores against the
+oracle's float64 column mass of the same keys and queries (and the selected set
+against its stable top-k, outside the tie band); then, on a cache the oracle
+rebuilds from the dense prefix and the GPU's vertical-line set, the K4V4
+records bit-exactly, the VL rows bit-exactly, and the decode output within the
+decode tolerances.
 """
 import numpy as np
 import pytest
 import torch
 
 from hybrid_precision_attention_b200 import synth
-from oracle import formats, hybrid
-from tests._gpu import check_decode, hq, sz_words
+from oracle import formats, hybrid, select as osel
+from tests._gpu import check_decode, check_selection, hq, sz_words
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -30,11 +33,14 @@ def _run_layers(n_layers, B, Hq, Hkv, L, W, samples, seed0):
     for layer in range(n_layers):
         k, v, q_tail, _ = synth.planted_layer_device(seed0 + layer, B, Hq, Hkv, L, "cuda")
         c = H.HybridCache(B, Hq, Hkv, cap, W, 500)
-        H.hq_select_vlines(c, k, q_tail)
+        mine = [(ly, b, h) for (ly, b, h) in samples if ly == layer]
+        scores = torch.zeros((B, Hkv, c.cap), dtype=torch.float32, device="cuda") if mine else None
+        H.hq_select_vlines(c, k, q_tail, scores_out=scores)
         H.hq_pack_merge(c, k, v)
-        for (ly, b, h) in samples:
-            if ly == layer:
-                kept[(ly, b, h)] = (k[b, h].cpu().numpy(), v[b, h].cpu().numpy())
+        for (ly, b, h) in mine:
+            kept[(ly, b, h)] = (k[b, h].cpu().numpy(), v[b, h].cpu().numpy(),
+                                q_tail[b, h * G:(h + 1) * G].cpu().numpy(), scores[b, h].cpu().numpy())
+        del scores
         del k, v, q_tail
         caches.append(c)
     torch.cuda.synchronize()
@@ -58,10 +64,17 @@ def _run_layers(n_layers, B, Hq, Hkv, L, W, samples, seed0):
 
 
 def _check_unit(c, kept, step, ly, b, h, L, W, G):
-    k16, v16 = kept[(ly, b, h)]
+    k16, v16, qg, gsc = kept[(ly, b, h)]
     n_vl = c.state()["n_vl"]
     vl = c.vl_pos[b, h, :n_vl].cpu().numpy().astype(np.int64)
     assert np.all(np.diff(vl) > 0) and vl.max() < L - W
+    # the unit's column mass (the last 64 prefix queries of its G heads, keys in FP16) and its selection
+    n = L - W
+    nq = qg.shape[1]
+    ref = osel.column_mass(k16.astype(np.float64), qg.reshape(-1, 128).astype(np.float64),
+                           np.tile(np.arange(L - nq, L), G), n, 1 / np.sqrt(128))
+    assert n_vl == osel.k_of(n, 500)
+    check_selection(gsc, vl, ref, n_vl, f"layer {ly} unit ({b},{h}) selection")
     # K4V4 records of the packed prefix, bit-exact (this unit's pages only)
     H = hq()
     pg = c.pages[b, h].cpu().numpy()

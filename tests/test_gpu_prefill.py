@@ -79,27 +79,49 @@ def test_prefill_matches_oracle(B, Hq, Hkv, L, W, rho):
         assert rel <= PF_RELL2, (b, h, rel)
 
 
-def test_prefill_fp8_codes_match_oracle():
-    """The pre-pass e4m3 codes of Q (first region of the workspace after the error word) are bit-exact."""
-    H = hq()
-    B, Hq, Hkv, L = 1, 4, 1, 300
-    lay = synth.planted_layer(3, B, Hq, Hkv, L)
-    Q = synth.full_queries(3, B, Hq, Hkv, L)
-    vlt = np.zeros((B, Hkv, 16), np.int32)
-    ws = torch.zeros(H.hq_prefill_workspace_bytes(B, Hq, Hkv, L), dtype=torch.uint8, device="cuda")
-    H.hq_prefill_attn(dev(Q), dev(lay.k), dev(lay.v), dev(vlt), 0, 64, ws=ws)
-    torch.cuda.synchronize()
-    Lp = 384
-    q8 = ws[1024:1024 + B * Hq * Lp * 128].cpu().numpy().reshape(B, Hq, Lp, 128)[:, :, :L]
-    # decode the e4m3 bytes with the OCP bit layout and compare to the oracle's rounding
-    codes = q8.astype(np.int64)
+def _e4m3_decode(codes):
+    """Real values of e4m3 bytes from the OCP bit layout (bias 7, 3 mantissa bits)."""
+    codes = codes.astype(np.int64)
     sign = np.where(codes & 0x80, -1.0, 1.0)
     e = (codes >> 3) & 0xF
     m = codes & 0x7
-    val = sign * np.where(e == 0, m / 8.0 * 2.0 ** -6, (1 + m / 8.0) * 2.0 ** (e - 7))
-    want = formats.fp8_quantize(Q, formats.fp8_block_scales(Q))
-    assert np.array_equal(val, want)
-    assert ws[:4].cpu().numpy().view(np.uint32)[0] == 0
+    return sign * np.where(e == 0, m / 8.0 * 2.0 ** -6, (1 + m / 8.0) * 2.0 ** (e - 7))
+
+
+def test_prefill_fp8_pre_pass_matches_oracle():
+    """The pre-pass outputs the workspace exposes (include/hq.h, prefill
+    workspace regions): the e4m3 codes of Q and K, bit-exact against the
+    oracle's per-block rounding, and V's fp16 values fp16(fp32(e4m3) * scale),
+    bit-exact against the same rounding of the oracle's codes and scales."""
+    H = hq()
+    B, Hq, Hkv, L = 2, 4, 2, 300
+    lay = synth.planted_layer(3, B, Hq, Hkv, L)
+    Q = synth.full_queries(3, B, Hq, Hkv, L)
+    vlt = np.zeros((B, Hkv, 16), np.int32)
+    ws = torch.zeros(H.hq_prefill_workspace_bytes(B, Hq, Hkv, L, 16), dtype=torch.uint8, device="cuda")
+    H.hq_prefill_attn(dev(Q), dev(lay.k), dev(lay.v), dev(vlt), 0, 64, ws=ws)
+    torch.cuda.synchronize()
+    r = H.prefill_ws_regions(B, Hq, Hkv, L)
+    Lp = r["Lp"]
+    w = ws.cpu().numpy()
+    assert w[:4].view(np.uint32)[0] == 0
+    q8 = w[r["q8"]:r["q8"] + B * Hq * Lp * 128].reshape(B, Hq, Lp, 128)
+    k8 = w[r["k8"]:r["k8"] + B * Hkv * Lp * 128].reshape(B, Hkv, Lp, 128)
+    v16 = w[r["v16"]:r["v16"] + B * Hkv * Lp * 128 * 2].view(np.float16).reshape(B, Hkv, Lp, 128)
+    for name, x, got in (("Q", Q, q8), ("K", lay.k, k8)):
+        for b in range(B):
+            for h in range(x.shape[1]):
+                want = formats.fp8_quantize(x[b, h], formats.fp8_block_scales(x[b, h]))
+                assert np.array_equal(_e4m3_decode(got[b, h, :L]), want), (name, b, h)
+                assert not got[b, h, L:].any(), (name, b, h)
+    for b in range(B):
+        for h in range(Hkv):
+            sv = formats.fp8_block_scales(lay.v[b, h])
+            code = formats.fp8_quantize(lay.v[b, h], sv)
+            blk = np.repeat(sv.astype(np.float32), 128)[:L]
+            want = (code.astype(np.float32) * blk[:, None]).astype(np.float16)
+            assert np.array_equal(v16[b, h, :L].view(np.uint16), want.view(np.uint16)), (b, h)
+            assert not v16[b, h, L:].view(np.uint16).any(), (b, h)
 
 
 @pytest.mark.slow
