@@ -27,7 +27,12 @@ Readings taken where the pages are silent (each listed in the design notes):
 * reselection uses the keys' pre-merge representation, then the merge packs the
   positions that left the window and installs the new VL set;
 * VL sets are per (batch, kv head) (the KV layout is per kv head under GQA) and
-  the column mass sums over the group's query heads.
+  the column mass sums over the group's query heads;
+* scores are recomputed at each reselection from the buffered queries; with
+  ``accumulate=True`` (the other reading of the README's "running column-mass
+  score") each reselection instead adds its column mass to a running score
+  per position, started from the prefix selection's column mass, and the
+  top-k runs on the running scores.
 """
 from __future__ import annotations
 
@@ -41,7 +46,8 @@ QBUF = 64       # buffered queries used by the column-mass estimate
 
 
 class HybridCacheRef:
-    def __init__(self, B: int, Hq: int, Hkv: int, W: int, rho_bp: int, cap: int, D: int = 128):
+    def __init__(self, B: int, Hq: int, Hkv: int, W: int, rho_bp: int, cap: int, D: int = 128,
+                 accumulate: bool = False):
         assert Hq % Hkv == 0 and D % formats.GROUP == 0
         self.B, self.Hq, self.Hkv, self.D, self.W, self.rho_bp, self.cap = B, Hq, Hkv, D, W, rho_bp, cap
         self.G = Hq // Hkv
@@ -60,6 +66,8 @@ class HybridCacheRef:
         self.T = 0
         self.n_packed = 0
         self.qbuf = []          # list of (position, q [B, Hq, D] float16), newest last
+        self.accumulate = accumulate
+        self.acc = np.zeros((B, Hkv, cap))   # running column mass per position (accumulate=True)
 
     # ------------------------------------------------------------------ helpers
     def _pack_range(self, lo: int, hi: int):
@@ -102,7 +110,28 @@ class HybridCacheRef:
                 qs = q_tail[b, h * self.G:(h + 1) * self.G].reshape(-1, D).astype(np.float64)
                 new_vl[b][h], scores[b][h] = select.select_vlines(K16[b, h].astype(np.float64), qs, qpos, n, self.rho_bp, self.sm_scale)
         self.install_prefix(K16, V16, new_vl)
+        self._start_running(scores, n)
         return new_vl, scores
+
+    def _start_running(self, scores, n):
+        self.acc[:] = 0.0
+        for b in range(self.B):
+            for h in range(self.Hkv):
+                self.acc[b, h, :n] = scores[b][h]
+
+    def start_running_scores(self, K16, q_tail):
+        """The prefix selection's column mass (keys all FP16, the tail queries)
+        as the starting running score, for a prefix installed with
+        :meth:`install_prefix` (whose VL sets were chosen elsewhere)."""
+        B, Hkv, L, D = K16.shape
+        n = max(L - self.W, 0)
+        nq = q_tail.shape[2]
+        qpos = np.tile(np.arange(L - nq, L), self.G)
+        sc = [[select.column_mass(K16[b, h].astype(np.float64),
+                                  q_tail[b, h * self.G:(h + 1) * self.G].reshape(-1, D).astype(np.float64),
+                                  qpos, n, self.sm_scale) for h in range(Hkv)] for b in range(B)]
+        self._start_running(sc, n)
+        return sc
 
     def install_prefix(self, K16, V16, vl_sets):
         """Install a prefix with given VL sets (the selection step done elsewhere)."""
@@ -158,10 +187,14 @@ class HybridCacheRef:
                 K, _ = self.rep(b, h)
                 qs = qs_all[b, h * self.G:(h + 1) * self.G].reshape(-1, self.D).astype(np.float64)
                 if qs.shape[0] == 0:
-                    scores[b][h] = np.zeros(n)
-                    new_vl[b][h] = select.topk_stable(scores[b][h], select.k_of(n, self.rho_bp))
+                    mass = np.zeros(n)
                 else:
-                    new_vl[b][h], scores[b][h] = select.select_vlines(K, qs, qpos, n, self.rho_bp, self.sm_scale)
+                    mass = select.column_mass(K, qs, qpos, n, self.sm_scale)
+                if self.accumulate:
+                    self.acc[b, h, :n] += mass
+                    mass = self.acc[b, h, :n].copy()
+                scores[b][h] = mass
+                new_vl[b][h] = select.topk_stable(mass, select.k_of(n, self.rho_bp))
         return new_vl, scores
 
     def merge(self, new_vl):

@@ -220,3 +220,62 @@ def test_decode_from_an_empty_cache_closed_forms():
         want = (p / p.sum()) @ V
         assert np.allclose(o1[0, h], want, rtol=1e-12, atol=1e-12)
     assert r.T == 2 and r.n_packed == 0
+
+
+def test_running_scores_accumulate_over_reselections():
+    """accumulate=True (the running column-mass reading of README Overview
+    item 1): the score of a position is the prefix selection's column mass
+    plus the column mass of every later reselection, each taken from explicit
+    loops over the keys as they were at that reselection; the set is the
+    stable top-k of the running score.  Positions that entered the scored
+    prefix later start from zero."""
+    B, Hq, Hkv, L, W, steps = 1, 4, 2, 24, 4, 5
+    G = Hq // Hkv
+    sm = 1 / np.sqrt(128)
+    lay = synth.planted_layer(37, B, Hq, Hkv, L)
+    c = hybrid.HybridCacheRef(B, Hq, Hkv, W, 2500, cap=64, accumulate=True)
+    vl0, sc0 = c.init_from_prefix(lay.k, lay.v, lay.q_tail)
+    n0 = L - W
+    nq = lay.q_tail.shape[2]
+    running = np.zeros((Hkv, 64))
+    for h in range(Hkv):
+        K = lay.k[0, h].astype(np.float64)
+        queries = [(L - nq + i, lay.q_tail[0, hh, i]) for hh in range(h * G, (h + 1) * G) for i in range(nq)]
+        running[h, :n0] = _column_mass_by_hand(K, queries, n0, sm)
+        assert np.allclose(c.acc[0, h, :n0], running[h, :n0], rtol=1e-11, atol=1e-14)
+    qd, kd, vd = synth.decode_tokens(37, B, Hq, Hkv, 2 * steps)
+    K16 = np.concatenate([lay.k, np.moveaxis(kd, 0, 2)], axis=2)
+    vl_prev = {h: {int(p): lay.k[0, h, p] for p in vl0[0][h]} for h in range(Hkv)}
+    for period in range(2):
+        for t in range(period * steps, (period + 1) * steps):
+            c.decode(qd[t], kd[t], vd[t])
+        T = L + (period + 1) * steps
+        n = T - W
+        # keys as they are before this merge: the previous merge packed [0, n_packed)
+        packed_upto = c.n_packed
+        vl, scores = c.reselect()
+        kk = select.k_of(n, 2500)
+        for h in range(Hkv):
+            K = _rep_by_hand(K16[0, h], packed_upto, vl_prev[h], T)
+            buffered = list(range(0, (period + 1) * steps))
+            queries = [(L + t, qd[t, 0, hh]) for hh in range(h * G, (h + 1) * G) for t in buffered]
+            running[h, :n] += _column_mass_by_hand(K, queries, n, sm)
+            assert np.allclose(scores[0][h], running[h, :n], rtol=1e-11, atol=1e-14), (period, h)
+            order = sorted(range(n), key=lambda j: (-running[h, j], j))[:kk]
+            assert list(vl[0][h]) == sorted(order)
+        c.merge(vl)
+        # rows of the new set: FP16 values for lines that had one, else dequantised records rounded once
+        for h in range(Hkv):
+            vl_prev[h] = {int(p): c.kf[0][h][r] for r, p in enumerate(vl[0][h])}
+
+
+def test_running_scores_start_from_the_prefix_selection():
+    """start_running_scores (a prefix installed with sets chosen elsewhere)
+    gives the same running scores as init_from_prefix."""
+    lay = synth.planted_layer(38, 1, 4, 2, 100)
+    a = hybrid.HybridCacheRef(1, 4, 2, 16, 500, cap=128, accumulate=True)
+    vl, _ = a.init_from_prefix(lay.k, lay.v, lay.q_tail)
+    b = hybrid.HybridCacheRef(1, 4, 2, 16, 500, cap=128, accumulate=True)
+    b.install_prefix(lay.k, lay.v, vl)
+    b.start_running_scores(lay.k, lay.q_tail)
+    assert np.array_equal(a.acc, b.acc)
