@@ -795,6 +795,49 @@ def measure_peaks(dev):
     print(json.dumps(rec), flush=True)
 
 
+def ablation_sweep(dev, Ls=8192, Ws=(0, 64, 128, 256, 512), rhos=(0, 100, 250, 500, 1000), steps=4):
+    """Accuracy ablation over the window W and the vertical-line ratio rho on
+    the planted generator (HyQuant digest, results paragraph: a wider window or
+    a higher ratio lowers the prefill error).  For every (W, rho): the hybrid
+    prefill's relative L2 error and the hybrid decode's (over `steps` tokens)
+    against the same kernels with every key FP16 (W >= L).  One JSON line per
+    point."""
+    import torch
+    from hybrid_precision_attention_b200 import hq, synth
+    B_, Hq_, Hkv_ = 1, 32, 8
+    lay = synth.planted_layer(3, B_, Hq_, Hkv_, Ls)
+    Q = torch.from_numpy(synth.full_queries(3, B_, Hq_, Hkv_, Ls)).to(dev)
+    k, v = torch.from_numpy(lay.k).to(dev), torch.from_numpy(lay.v).to(dev)
+    qt = Q[:, :, Ls - 64:].contiguous()
+    qd, kd, vd = [torch.from_numpy(a).to(dev) for a in synth.decode_tokens(3, B_, Hq_, Hkv_, steps)]
+    rel = lambda a, b: float(torch.linalg.vector_norm((a.float() - b.float())) / torch.linalg.vector_norm(b.float()))
+    no_vl = torch.zeros((B_, Hkv_, 16), dtype=torch.int32, device=dev)
+    exact_pf = hq.hq_prefill_attn(Q, k, v, no_vl, 0, Ls)
+
+    def decode_run(W_, rho_):
+        c = hq.HybridCache(B_, Hq_, Hkv_, Ls + steps + 64, W_, rho_, device=dev)
+        hq.hq_select_vlines(c, k, qt)
+        hq.hq_pack_merge(c, k, v)
+        outs = [hq.hq_decode_attn(c, qd[t], kd[t], vd[t]).clone() for t in range(steps)]
+        torch.cuda.synchronize()
+        assert c.state()["err"] == 0, c.state()
+        return c, torch.stack(outs)
+
+    _, exact_dec = decode_run(Ls + 64, 0)
+    rows = []
+    for W_ in Ws:
+        for rho_ in rhos:
+            c, dec = decode_run(W_, rho_)
+            n_vl = c.state()["n_vl"]
+            pf = hq.hq_prefill_attn(Q, k, v, c.vl_pos, n_vl, W_)
+            torch.cuda.synchronize()
+            row = {"L": Ls, "W": W_, "rho": rho_ / 10000, "lines_per_kv_head": n_vl,
+                   "prefill_rel_l2": rel(pf, exact_pf), "decode_rel_l2": rel(dec, exact_dec)}
+            rows.append(row)
+            print(json.dumps(row), flush=True)
+    return rows
+
+
 def profile_decode():
     """Small case for ncu captures: one 32K layer cache, 4 decode steps with an L2 flush before each."""
     import torch
@@ -868,6 +911,7 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-legs", action="store_true", help="skip the 1K, 36-layer and 64-layer decode workloads")
     ap.add_argument("--measure-peaks", action="store_true", help="measure the e4m3 GEMM peak and the read-only HBM ceiling")
+    ap.add_argument("--sweep", action="store_true", help="accuracy ablation over W and rho on the planted generator")
     ap.add_argument("--profile-decode", action="store_true", help="small case for ncu: 4 decode steps of one 32K layer")
     ap.add_argument("--profile-prefill", action="store_true", help="small case for ncu: 3 prefill calls at L=8192")
     ap.add_argument("--profile-select", action="store_true", help="small case for ncu: one decode-mode reselection at 32K")
@@ -884,6 +928,10 @@ def main():
     if args.measure_peaks:
         import torch
         measure_peaks(torch.device("cuda", 0))
+        return
+    if args.sweep:
+        import torch
+        ablation_sweep(torch.device("cuda", 0))
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -45,9 +45,38 @@ struct DeviceOnce {
   }
 };
 
-// K4V4 page of position p of (b, kv head) bh
-__host__ __device__ __forceinline__ uint8_t* page_of(const hq_cache& c, size_t bh, int p) {
-  return c.pages + (bh * static_cast<size_t>(c.cap / HQ_PAGE_POSITIONS) + (p >> 6)) * HQ_PAGE_BYTES;
+// State row of sequence b.
+__host__ __device__ __forceinline__ int32_t* state_row(const hq_cache& c, int b) { return c.state + b * HQ_STATE_WORDS; }
+
+// Pool index of page j (positions 64 j .. 64 j + 63) of (b, kv head) bh: the
+// dense layout when there is no page table, else the table entry; -1 when the
+// entry lies outside the pool.
+__device__ __forceinline__ long long page_index(const hq_cache& c, size_t bh, int j) {
+  const size_t npg = static_cast<size_t>(c.cap / HQ_PAGE_POSITIONS);
+  if (c.page_table == nullptr) return static_cast<long long>(bh * npg + j);
+  const int idx = c.page_table[bh * npg + j];
+  return (idx >= 0 && idx < c.n_pages) ? idx : -1;
+}
+
+// K4V4 page of position p of (b, kv head) bh, for readers: an entry outside the
+// pool reads pool page 0 instead (memory-safe) and flags HQ_DEVERR_PAGE.
+__device__ __forceinline__ uint8_t* page_of(const hq_cache& c, size_t bh, int p) {
+  const long long idx = page_index(c, bh, p >> 6);
+  if (idx < 0) {
+    atomicOr(reinterpret_cast<unsigned int*>(state_row(c, static_cast<int>(bh / c.Hkv)) + HQ_STATE_ERR), HQ_DEVERR_PAGE);
+    return c.pages;
+  }
+  return c.pages + static_cast<size_t>(idx) * HQ_PAGE_BYTES;
+}
+
+// The same for writers: null for an entry outside the pool (flagged; the caller skips the write).
+__device__ __forceinline__ uint8_t* page_for_write(const hq_cache& c, size_t bh, int p) {
+  const long long idx = page_index(c, bh, p >> 6);
+  if (idx < 0) {
+    atomicOr(reinterpret_cast<unsigned int*>(state_row(c, static_cast<int>(bh / c.Hkv)) + HQ_STATE_ERR), HQ_DEVERR_PAGE);
+    return nullptr;
+  }
+  return c.pages + static_cast<size_t>(idx) * HQ_PAGE_BYTES;
 }
 __host__ __device__ __forceinline__ uint8_t* row_codes(uint8_t* page, int which, int p) {
   return page + (which ? HQ_PAGE_VCODES : HQ_PAGE_KCODES) + (p & 63) * (HQ_HEAD_DIM / 2);

@@ -7,39 +7,44 @@
 // materialised.  The pages' kernel is Triton for SM80+; this is a B200 design.
 //
 // Design (bandwidth-bound: ~160 B of K4V4 per token and kv head):
-//   * grid = (splits S, Hkv, B), one wave (a wide CTA per SM, or 3 narrow CTAs
-//     per SM for large batches); every
-//     CTA owns one GQA group (all G <= 8 query heads of a kv head share one
-//     pass over the bytes) and a contiguous range of the head's tile list:
-//     packed tiles (one page of 64 positions: 4 KB K codes, 4 KB V codes,
-//     1 KB + 1 KB scale/zero, the VL bitmap), VL tiles (16 FP16 rows of the VL
-//     store), ring tiles (16 slots of the FP16 ring, which is a multiple of 16
-//     long, so a tile is one contiguous copy) and a last tile holding the new
-//     token read straight from its input pointer;
+//   * work: every (b, kv head) is a unit whose tile list holds its packed
+//     tiles (one page of 64 positions: 4 KB K codes, 4 KB V codes, 1 KB + 1 KB
+//     scale/zero, the VL bitmap), its FP16 tiles (16 rows of the VL store, 16
+//     slots of the FP16 ring, which is a multiple of 16 long, so a tile is one
+//     contiguous copy) and a last tile with the new token read straight from
+//     its input pointer; the FP16 tiles are interleaved evenly among the
+//     packed ones;
+//   * grid: persistent, one CTA per SM (stream-K).  The units' tile lists are
+//     concatenated and cut into equal contiguous ranges, one per CTA, so every
+//     SM streams the same number of tiles whatever the batch size or the
+//     sequences' lengths (each sequence has its own state row); a range may
+//     cover parts of several units, one segment per unit.  Every unit also
+//     carries a small phantom weight in the cut, which bounds how many
+//     segments a range can hold;
 //   * a producer warp streams tiles into a 2 NC-stage shared-memory ring with
 //     large 1-D bulk async copies (cp.async.bulk, mbarrier completion, no
 //     multicast): 1 copy per packed tile, 2 per FP16 tile;
-//   * NC consumer warps take whole tiles round-robin, each owning 2 of the 2 NC
+//   * NC consumer warps take tiles round-robin, each owning 2 of the 2 NC
 //     stages (tile i -> stage i % 2NC -> warp i % NC), so every stage has a
-//     single consumer and a waiter is never a full barrier phase behind; every
-//     split gets an even share of the packed tiles and an even share of the
-//     FP16 tiles, so both its bytes and its arithmetic are balanced.  Nibbles
-//     become fp16 in registers (exponent-bias trick + one fma with the group's
-//     scale/zero), and
-//     both products run on tensor cores with mma.m16n8k16 (f32 accumulate):
+//     single consumer and a waiter is never a full barrier phase behind.
+//     Nibbles become fp16 in registers (exponent-bias trick + one fma with the
+//     group's scale/zero), and both products run on tensor cores with
+//     mma.m16n8k16 (f32 accumulate):
 //       S^T[keys x 8 queries] = K^ (16 keys x 16 dims) . Q^T
 //       O^T[dims x 8 queries] += V^T (16 dims x 16 keys) . P^T
 //     P^T comes from the S^T accumulators by an 8x8 movmatrix transpose.  Dims
 //     and keys are permuted inside each MMA so that every thread dequantises one
 //     whole group from contiguous nibbles and the packed-tile shared-memory
 //     reads are free of bank conflicts;
-//   * per-warp online softmax in the exp2 domain, a CTA merge in shared memory,
-//     then split partials (m, l, O) go to the workspace and the last CTA of each
-//     (b, kv head) merges them with a log-sum-exp (atomic ticket, no waiting);
-//   * the last CTA of each (b, kv head) also appends that head's new token to
-//     the ring and its queries to the query buffer (every split of the head is
-//     done reading by then); the last CTA of the grid advances T;
-//   * launched with programmatic dependent launch: a CTA prefetches its split's
+//   * per-warp online softmax in the exp2 domain.  At the end of a segment
+//     every consumer warp leaves its state in the stage of its last tile (held
+//     back from the producer until the merge is done), the consumers merge the
+//     warp states into the segment's partial (m, l, O) in the workspace, and
+//     the last CTA to finish a unit merges that unit's partials with a
+//     log-sum-exp (atomic ticket, no waiting), appends the unit's new token to
+//     the ring and its queries to the query buffer (every CTA of the unit is
+//     done reading by then); the last CTA of the grid advances the lengths;
+//   * launched with programmatic dependent launch: a CTA prefetches its range's
 //     pages and VL rows into L2 before it waits for the previous grid, and lets
 //     the next grid launch as soon as its own wait is over.
 #include "common.cuh"
@@ -47,19 +52,18 @@
 namespace hq {
 namespace {
 
-// Two CTA shapes, one kernel template (NC consumer warps, 2 stages each, one
-// producer warp):
-//   wide  : NC = 11, 22 stages, 1 CTA per SM  (few kv heads: fewer, longer splits)
-//   narrow: NC = 3,  6 stages, 3 CTAs per SM  (large batches)
+// NC consumer warps with 2 stages each, one producer warp, one CTA per SM.
 // Each stage must have exactly one consumer warp: a parity wait on an mbarrier
 // only tells the current phase from the one before it, so a warp that reached a
 // stage while another warp's earlier tile there had not landed yet would see the
 // older completed phase and consume the wrong data.  With NSTAGES = 2 NC,
 // stage s belongs to warp s % NC.
-#ifndef HQ_DECODE_NC_WIDE
-#define HQ_DECODE_NC_WIDE 11
+#ifndef HQ_DECODE_NC
+#define HQ_DECODE_NC 11
 #endif
-constexpr int NC_WIDE = HQ_DECODE_NC_WIDE, NC_NARROW = 3;
+constexpr int NC = HQ_DECODE_NC;
+constexpr int NSTAGES = 2 * NC;
+constexpr int NTHREADS = (NC + 1) * 32;
 constexpr int PK = 64;                         // positions per packed tile
 constexpr int FT = 16;                         // rows per FP16 tile
 constexpr int FSTRIDE = 256;                   // bytes per FP16 row in shared memory (one contiguous copy)
@@ -67,10 +71,15 @@ constexpr int OFF_VC = 4096, OFF_KS = 8192, OFF_VS = 9216, OFF_MASK = 10240;
 constexpr int OFF_FV = FT * FSTRIDE;           // V rows of an FP16 tile
 constexpr int STAGE_BYTES = 10368;             // max(10256, 2 * 16 * 256 = 8192), 128-aligned
 constexpr int PART_FLOATS = 16 + 8 * D;        // m[8], l[8], O[8][128]
-constexpr int MAX_SPLITS = 64;                 // splits per (b, kv head)
+constexpr int MAX_UNITS = 2048;                // (b, kv head) units per call
+constexpr int MAXSEG = 96;                     // segments (units) one CTA's range can touch
+constexpr int PHANTOM_DIV = 32;                // phantom weight per unit = ceil(tiles / (CTAs x 32))
+constexpr int MIN_TILES = 4;                   // at least this many tiles per CTA
+constexpr int SCAN_PER = (MAX_UNITS + NTHREADS - 1) / NTHREADS;  // units per thread in the scan
 constexpr uint32_t PK_TX = HQ_PAGE_VLMASK + 16;   // codes, scale/zero words and the bitmap: one copy
 static_assert(OFF_VC == HQ_PAGE_VCODES && OFF_KS == HQ_PAGE_KSZ && OFF_VS == HQ_PAGE_VSZ && OFF_MASK == HQ_PAGE_VLMASK,
               "a packed stage is a verbatim copy of the page prefix");
+static_assert(PART_FLOATS * 4 <= STAGE_BYTES, "a warp state fits in one stage");
 
 // key slot -> shared-memory row inside a 16-key block.  Packed tiles (64-byte
 // rows): {0,5,1,4,2,7,3,6, 8,13,9,12,10,15,11,14}; FP16 tiles (256-byte rows):
@@ -85,66 +94,219 @@ __device__ __forceinline__ int pi_fp(int s) {
   return (s & 8) + (x & 4) + ((x & 1) << 1) + ((x >> 1) & 1);
 }
 
-struct Geo {
-  int n_packed, n_vl, T, R, NP, NV, NR, NT;
+// ------------------------------------------------------------------ work decomposition
+
+// One unit's lengths and tile counts (from its sequence's state row).
+struct UnitGeo {
+  int n_packed, n_vl, T;
+  int NP, NV, NF, NT;   // packed tiles, VL tiles, FP16 tiles (VL + ring + new token), all
 };
 
-// tiles of one (b, kv head): [0, NP) packed, [NP, NP+NV) VL, [NP+NV, NT-1) ring
-// (R/16 slot tiles), NT-1 the new token
-__device__ __forceinline__ Geo geo_of(int n_packed, int n_vl, int T, int R) {
-  Geo g;
+__device__ __forceinline__ UnitGeo unit_geo(int n_packed, int n_vl, int T, int R) {
+  UnitGeo g;
   g.n_packed = n_packed;
   g.n_vl = n_vl;
   g.T = T;
-  g.R = R;
   g.NP = (n_packed + PK - 1) / PK;
   g.NV = (n_vl + FT - 1) / FT;
-  g.NR = R / FT + 1;
-  g.NT = g.NP + g.NV + g.NR;
+  g.NF = g.NV + R / FT + 1;
+  g.NT = g.NP + g.NF;
   return g;
 }
 
-// 16-bit mask of the valid rows of FP16 tile `tile`
-__device__ __forceinline__ uint32_t fp16_valid(const Geo& g, int tile) {
-  if (tile < g.NP + g.NV) {
-    const int first = (tile - g.NP) * FT;
-    const int n = min(FT, g.n_vl - first);
+// A sequence takes no step when its staging area is full or T reached cap.
+__device__ __forceinline__ bool refused(const hq_cache& c, int T, int n_packed) {
+  return T - n_packed >= c.W + HQ_STAGE || T >= c.cap;
+}
+
+// Number of FP16 tiles among the unit's first k tiles (FP16 tiles spread evenly).
+__device__ __forceinline__ int fp16_before(const UnitGeo& g, int k) {
+  return static_cast<int>((static_cast<long long>(k) * g.NF) / g.NT);
+}
+
+// Walks a unit's tiles k, k + stride, k + 2 stride, ... keeping f = fp16_before(k)
+// and the remainder of k NF / NT, so each step needs no division: tile k is an
+// FP16 tile iff the remainder plus NF reaches NT.
+struct TileWalk {
+  int k, f, rem, qd, rd, NF, NT;
+  __device__ __forceinline__ void start(const UnitGeo& g, int k0, int stride) {
+    NF = g.NF;
+    NT = g.NT;
+    k = k0;
+    const long long x = static_cast<long long>(k0) * NF;
+    f = static_cast<int>(x / NT);
+    rem = static_cast<int>(x - static_cast<long long>(f) * NT);
+    const long long y = static_cast<long long>(stride) * NF;
+    qd = static_cast<int>(y / NT);
+    rd = static_cast<int>(y - static_cast<long long>(qd) * NT);
+  }
+  // the packed tile index (>= 0), or -(FP16 tile index) - 1
+  __device__ __forceinline__ int tile() const { return rem + NF >= NT ? -f - 1 : k - f; }
+  __device__ __forceinline__ void step(int stride) {
+    k += stride;
+    f += qd;
+    rem += rd;
+    if (rem >= NT) {
+      rem -= NT;
+      ++f;
+    }
+  }
+};
+
+// 16-bit mask of the valid rows of FP16 tile j (VL tiles, then ring tiles, then the new token)
+__device__ __forceinline__ uint32_t fp16_valid(const UnitGeo& g, int j, int R) {
+  if (j < g.NV) {
+    const int n = min(FT, g.n_vl - j * FT);
     return n >= FT ? 0xFFFFu : ((1u << n) - 1u);
   }
-  const int j = tile - g.NP - g.NV;
-  if (j == g.NR - 1) return 1u;  // the new token
+  const int r = j - g.NV;
+  if (r == R / FT) return 1u;  // the new token
   // ring slot s holds position p = n_packed + ((s - n_packed) mod R); valid iff p < T
-  const int base = g.n_packed % g.R;
+  const int base = g.n_packed % R;
   uint32_t m = 0;
 #pragma unroll 4
-  for (int r = 0; r < FT; ++r) {
-    int off = FT * j + r - base;
-    off += off < 0 ? g.R : 0;
-    m |= (g.n_packed + off < g.T ? 1u : 0u) << r;
+  for (int i = 0; i < FT; ++i) {
+    int off = FT * r + i - base;
+    off += off < 0 ? R : 0;
+    m |= (g.n_packed + off < g.T ? 1u : 0u) << i;
   }
   return m;
 }
 
-// This split's tiles: an even share of the packed tiles [p_lo, p_lo + n_p)
-// and an even share of the FP16 tiles [f_lo, f_lo + n_f) (VL, ring, new
-// token), numbered 0 .. n_p + n_f - 1 packed first.  Consumer warps take them
-// round-robin, so the FP16 tiles (8 KB each, like a packed tile's 10 KB, but
-// about a tenth of its arithmetic) land on the warps that got one packed tile
-// fewer: the slowest warp of a split does ceil(n_p / NC) packed tiles plus at
-// most one FP16 tile, and every split streams about the same bytes.
-struct SplitTiles {
-  int p_lo, n_p, f_lo, n_f;
-  __device__ __forceinline__ int tile(int i) const { return i < n_p ? p_lo + i : f_lo + (i - n_p); }
+// A CTA's share of one unit: CTA-local tiles [a, b) are the unit's tiles k0 .. k0 + b - a - 1.
+struct Seg {
+  int u, a, b, k0, first_cta, ncta;
 };
-__device__ __forceinline__ SplitTiles split_tiles(const Geo& geo, int split, int S) {
-  SplitTiles r;
-  const int NF = geo.NT - geo.NP;
-  r.p_lo = static_cast<int>((static_cast<long long>(split) * geo.NP) / S);
-  r.n_p = static_cast<int>((static_cast<long long>(split + 1) * geo.NP) / S) - r.p_lo;
-  const int f0 = static_cast<int>((static_cast<long long>(split) * NF) / S);
-  r.f_lo = geo.NP + f0;
-  r.n_f = static_cast<int>((static_cast<long long>(split + 1) * NF) / S) - f0;
-  return r;
+
+// The CTA's range and segments (shared memory), built by all NTHREADS threads.
+struct Plan {
+  int nseg, ntile, ceff;
+  Seg seg[MAXSEG];
+};
+
+// Cut the batch's tile lists into ranges and record this CTA's segments.
+// `stale`: state read with volatile loads before the dependency wait (it may
+// be one step old; the plan then only steers prefetches).  `red` is scratch
+// for NTHREADS / 32 + 2 ints.
+__device__ void make_plan(const hq_cache& c, int R, Plan& p, int* red, bool stale) {
+  const int U = c.B * c.Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid < MAXSEG) p.seg[tid].u = -1;
+  // tile counts of this thread's units (refused sequences: none)
+  int nt[SCAN_PER];
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < SCAN_PER; ++i) {
+    const int u = tid * SCAN_PER + i;
+    nt[i] = 0;
+    if (u < U) {
+      const int32_t* st = state_row(c, u / c.Hkv);
+      int T, np, nv;
+      if (stale) {
+        T = *reinterpret_cast<volatile const int*>(st + HQ_STATE_T);
+        np = *reinterpret_cast<volatile const int*>(st + HQ_STATE_NPACKED);
+        nv = *reinterpret_cast<volatile const int*>(st + HQ_STATE_NVL);
+        np = min(max(np, 0), c.cap);
+        nv = min(max(nv, 0), c.vl_cap);
+      } else {
+        T = st[HQ_STATE_T];
+        np = st[HQ_STATE_NPACKED];
+        nv = st[HQ_STATE_NVL];
+      }
+      if (!refused(c, T, np)) nt[i] = unit_geo(np, nv, T, R).NT;
+    }
+    sum += nt[i];
+  }
+  // block-wide exclusive scan of the per-thread sums
+  int x = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) red[warp] = x;
+  if (tid == 0) {
+    p.nseg = 0;
+    red[NTHREADS / 32] = -1;  // u0
+  }
+  __syncthreads();
+  int before = 0, total = 0;
+  for (int w = 0; w < NTHREADS / 32; ++w) {
+    const int v = red[w];
+    before += w < warp ? v : 0;
+    total += v;
+  }
+  const int excl = before + x - sum;  // tiles of all units before this thread's first unit
+  // phantom weight X per unit bounds the units a range can touch (at most
+  // N / (ceff X) + U / ceff + 2 <= 32 + 48 + 2 < MAXSEG); ceff CTAs share the work
+  const long long N = total;
+  // (at least U / 48 CTAs, so that with the phantom weight no range touches more than MAXSEG units)
+  const int ceff = static_cast<int>(min(static_cast<long long>(gridDim.x),
+                                        max(max(1ll, (N + MIN_TILES - 1) / MIN_TILES), static_cast<long long>((U + 47) / 48))));
+  const long long X = max(1ll, (N + static_cast<long long>(ceff) * PHANTOM_DIV - 1) / (static_cast<long long>(ceff) * PHANTOM_DIV));
+  const long long Wt = N + static_cast<long long>(U) * X;
+  const long long w0 = (static_cast<long long>(blockIdx.x) * Wt) / ceff;
+  const long long w1 = (static_cast<long long>(blockIdx.x + 1) * Wt) / ceff;
+  // CTA whose range holds weight position w
+  auto cta_of = [&](long long w) { return static_cast<int>(((w + 1) * ceff - 1) / Wt); };
+  // the unit holding w0: unit u spans weights [S_u, S_u + X + NT_u), S_u = tiles before + u X
+  int tb = excl;
+#pragma unroll
+  for (int i = 0; i < SCAN_PER; ++i) {
+    const int u = tid * SCAN_PER + i;
+    if (u < U) {
+      const long long S = tb + static_cast<long long>(u) * X;
+      if (S <= w0 && w0 < S + X + nt[i]) red[NTHREADS / 32] = u;
+    }
+    tb += nt[i];
+  }
+  __syncthreads();
+  const int u0 = red[NTHREADS / 32];
+  // every unit of [u0, u0 + MAXSEG) that holds tiles of this CTA's range becomes a segment
+  tb = excl;
+#pragma unroll
+  for (int i = 0; i < SCAN_PER; ++i) {
+    const int u = tid * SCAN_PER + i;
+    if (u < U && u >= u0 && u0 >= 0 && nt[i] > 0) {
+      const long long S = tb + static_cast<long long>(u) * X + X;  // first tile's weight
+      const long long lo = max(S, w0), hi = min(S + nt[i], w1);
+      if (lo < hi) {
+        if (u - u0 < MAXSEG) {
+          Seg& s = p.seg[u - u0];
+          s.u = u;
+          s.k0 = static_cast<int>(lo - S);
+          s.a = static_cast<int>(lo - w0);  // weights of earlier units' phantoms are not tiles: fixed below
+          s.b = static_cast<int>(hi - lo);  // count for now
+          s.first_cta = cta_of(S);
+          s.ncta = cta_of(S + nt[i] - 1) - s.first_cta + 1;
+          atomicMax(&p.nseg, u - u0 + 1);
+        } else {
+          set_err(state_row(c, 0), HQ_DEVERR_TIMEOUT);  // never expected: the phantom weight bounds the count
+        }
+      }
+    }
+    tb += nt[i];
+  }
+  __syncthreads();
+  if (tid == 0) {
+    // CTA-local tile numbering: segments back to back, empty slots skipped
+    int at = 0, k = 0;
+    for (int i = 0; i < p.nseg; ++i) {
+      Seg& s = p.seg[i];
+      const bool used = s.u == u0 + i && s.b > 0;
+      if (!used) continue;
+      const int n = s.b;
+      Seg t = s;
+      t.a = at;
+      t.b = at + n;
+      at += n;
+      p.seg[k++] = t;
+    }
+    p.nseg = blockIdx.x < ceff ? k : 0;
+    p.ntile = blockIdx.x < ceff ? at : 0;
+    p.ceff = ceff;
+  }
+  __syncthreads();
 }
 
 struct WarpState {
@@ -369,22 +531,68 @@ __device__ __forceinline__ void fp16_tile(WarpState& ws, const uint8_t* st, cons
   }
 }
 
-template <int NCONS, int MINB>
-__global__ void __launch_bounds__((NCONS + 1) * 32, MINB)
+
+// Load this unit's Q^T fragments (the G query heads of kv head kvh of sequence b,
+// in the permuted dim order: thread t covers dims 32t .. 32t+31); columns >= G are zero.
+__device__ __forceinline__ void load_q(const hq_cache& c, const uint16_t* __restrict__ q, int b, int kvh, int G, int g,
+                                       int t, uint32_t (&qf)[8][2]) {
+  if (g < G) {
+    const uint4* qp = reinterpret_cast<const uint4*>(q + (static_cast<size_t>(b) * c.Hq + kvh * G + g) * D + 32 * t);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 u = qp[i];
+      qf[2 * i][0] = prmt(u.x, u.z, 0x5410);
+      qf[2 * i][1] = prmt(u.x, u.z, 0x7632);
+      qf[2 * i + 1][0] = prmt(u.y, u.w, 0x5410);
+      qf[2 * i + 1][1] = prmt(u.y, u.w, 0x7632);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) qf[j][0] = qf[j][1] = 0u;
+  }
+}
+
+__device__ __forceinline__ void consumer_bar() { asm volatile("bar.sync 1, %0;" ::"r"(NC * 32) : "memory"); }
+
+__device__ __forceinline__ UnitGeo geo_of_unit(const hq_cache& c, int u, int R) {
+  const int32_t* st = state_row(c, u / c.Hkv);
+  return unit_geo(st[HQ_STATE_NPACKED], st[HQ_STATE_NVL], st[HQ_STATE_T], R);
+}
+
+// Source of FP16 tile j of unit bh (K rows, V rows, bytes per half)
+__device__ __forceinline__ void fp16_src(const hq_cache& c, const UnitGeo& g, int bh, int j, int R,
+                                         const uint16_t* k_new, const uint16_t* v_new, const uint16_t*& ks,
+                                         const uint16_t*& vs, uint32_t& bytes) {
+  if (j < g.NV) {
+    const size_t off = (static_cast<size_t>(bh) * c.vl_cap + j * FT) * D;
+    ks = c.kf + off;
+    vs = c.vf + off;
+    bytes = FT * 2 * D;
+  } else if (j - g.NV < R / FT) {
+    const size_t off = (static_cast<size_t>(bh) * R + (j - g.NV) * FT) * D;
+    ks = c.kr + off;
+    vs = c.vr + off;
+    bytes = FT * 2 * D;
+  } else {
+    ks = k_new + static_cast<size_t>(bh) * D;
+    vs = v_new + static_cast<size_t>(bh) * D;
+    bytes = 2 * D;
+  }
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1)
 decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* __restrict__ k_new,
-              const uint16_t* __restrict__ v_new, uint16_t* __restrict__ out, float qscale, int S,
+              const uint16_t* __restrict__ v_new, uint16_t* __restrict__ out, float qscale,
               float* __restrict__ parts, unsigned int* __restrict__ tickets) {
-  constexpr int NSTAGES = 2 * NCONS;
-  constexpr int NTHREADS = (NCONS + 1) * 32;
-  static_assert(NSTAGES % NCONS == 0, "every stage needs a single owner warp");
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t full[NSTAGES], empty[NSTAGES];
-  __shared__ int s_last;
-  __shared__ int s_timeout;      // a bounded wait gave up somewhere in this CTA
+  __shared__ Plan plan;
+  __shared__ int red[NTHREADS / 32 + 2];
+  __shared__ int s_timeout;          // a bounded wait gave up somewhere in this CTA
   __shared__ int s_issued[NSTAGES];  // tiles issued into each stage
+  __shared__ int s_held[NC];         // stage holding each consumer warp's state at a segment end (-1: none)
+  __shared__ int s_last;
 
-  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  const int bh = b * c.Hkv + kvh;
   const int G = c.Hq / c.Hkv;
   const int R = ring_len(c.W);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -399,27 +607,30 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
     s_timeout = 0;
     fence_mbar_init();
   }
-  if (threadIdx.x == NCONS * 32) {
-    // Before the dependency wait, warm L2 with this split's packed pages and VL
-    // rows.  The lengths read here may be stale (the previous grid can still be
-    // writing them): they only steer a prefetch hint, and the ranges are clamped
-    // to the buffers, so a stale value costs bandwidth, never correctness.
-    const int pT = *reinterpret_cast<volatile const int*>(c.state + HQ_STATE_T);
-    const int pnp = *reinterpret_cast<volatile const int*>(c.state + HQ_STATE_NPACKED);
-    const int pnv = *reinterpret_cast<volatile const int*>(c.state + HQ_STATE_NVL);
-    const Geo pg = geo_of(min(max(pnp, 0), c.cap), min(max(pnv, 0), c.vl_cap), pT, R);
-    const SplitTiles pr = split_tiles(pg, split, S);
-    const int npg = c.cap / PK;
-    const int a0 = min(max(pr.p_lo, 0), npg), a1 = min(max(pr.p_lo + pr.n_p, a0), npg);
-    const uint8_t* pages = c.pages + static_cast<size_t>(bh) * npg * HQ_PAGE_BYTES;
-    for (int pgi = a0; pgi < a1; pgi += 16)  // 16 pages (165 KB) per prefetch
-      prefetch_l2(pages + static_cast<size_t>(pgi) * HQ_PAGE_BYTES, min(16, a1 - pgi) * HQ_PAGE_BYTES);
-    const int v0 = min(max(pr.f_lo - pg.NP, 0), c.vl_cap / FT);
-    const int v1 = min(max(pr.f_lo + pr.n_f - pg.NP, v0), min(pg.NV, c.vl_cap / FT));
-    if (v1 > v0) {
-      const size_t off = (static_cast<size_t>(bh) * c.vl_cap + v0 * FT) * D;
-      prefetch_l2(c.kf + off, (v1 - v0) * FT * D * 2);
-      prefetch_l2(c.vf + off, (v1 - v0) * FT * D * 2);
+  // Before the dependency wait, plan on the (possibly stale) lengths and warm
+  // L2 with this range's pages and VL rows: a prefetch is a hint, the ranges
+  // are clamped to the buffers, so a stale plan costs bandwidth, never
+  // correctness.
+  make_plan(c, R, plan, red, true);
+  if (warp == NC) {
+    for (int si = 0; si < plan.nseg; ++si) {
+      const Seg s = plan.seg[si];
+      const int32_t* st = state_row(c, s.u / c.Hkv);
+      const int np = min(max(*reinterpret_cast<volatile const int*>(st + HQ_STATE_NPACKED), 0), c.cap);
+      const int nv = min(max(*reinterpret_cast<volatile const int*>(st + HQ_STATE_NVL), 0), c.vl_cap);
+      const UnitGeo ug = unit_geo(np, nv, *reinterpret_cast<volatile const int*>(st + HQ_STATE_T), R);
+      const int k1 = s.k0 + (s.b - s.a);
+      const int p0 = s.k0 - fp16_before(ug, s.k0), p1 = min(k1 - fp16_before(ug, k1), c.cap / PK);
+      for (int pg = p0 + lane; pg < p1; pg += 32) {  // one page per lane
+        const long long idx = page_index(c, s.u, pg);
+        if (idx >= 0) prefetch_l2(c.pages + static_cast<size_t>(idx) * HQ_PAGE_BYTES, PK_TX);
+      }
+      const int v0 = min(fp16_before(ug, s.k0), ug.NV), v1 = min(fp16_before(ug, k1), min(ug.NV, c.vl_cap / FT));
+      if (lane == 0 && v1 > v0) {
+        const size_t off = (static_cast<size_t>(s.u) * c.vl_cap + v0 * FT) * D;
+        prefetch_l2(c.kf + off, (v1 - v0) * FT * D * 2);
+        prefetch_l2(c.vf + off, (v1 - v0) * FT * D * 2);
+      }
     }
   }
   // programmatic dependent launch: everything this kernel reads (the state, the
@@ -428,27 +639,20 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
   // the SMs that free up (it waits here in turn)
   griddep_wait();
   griddep_launch_dependents();
-  const int T = c.state[HQ_STATE_T];
-  const int n_packed = c.state[HQ_STATE_NPACKED];
-  const int n_vl = c.state[HQ_STATE_NVL];
-  if (T - n_packed >= c.W + HQ_STAGE || T >= c.cap) {  // staging full / no room: do nothing
-    if (split == 0 && kvh == 0 && b == 0 && threadIdx.x == 0)
-      set_err(c.state, T >= c.cap ? HQ_DEVERR_CAPACITY : HQ_DEVERR_STAGING_FULL);
-    return;
+  __syncthreads();  // the stale plan is no longer read
+  make_plan(c, R, plan, red, false);
+  if (blockIdx.x == 0) {  // sequences that take no step are flagged (once)
+    for (int b = threadIdx.x; b < c.B; b += NTHREADS) {
+      int32_t* st = state_row(c, b);
+      const int T = st[HQ_STATE_T], np = st[HQ_STATE_NPACKED];
+      if (refused(c, T, np)) set_err(st, T >= c.cap ? HQ_DEVERR_CAPACITY : HQ_DEVERR_STAGING_FULL);
+    }
   }
-  const Geo geo = geo_of(n_packed, n_vl, T, R);
-  const SplitTiles sp = split_tiles(geo, split, S);
-  const int ntile = sp.n_p + sp.n_f;
+  const int ntile = plan.ntile, nseg = plan.nseg;
 
-  __syncthreads();
-
-  WarpState ws;
-  ws.m[0] = ws.m[1] = -INFINITY;
-  ws.l[0] = ws.l[1] = 0.f;
-#pragma unroll
-  for (int m = 0; m < 8; ++m) ws.o[m][0] = ws.o[m][1] = ws.o[m][2] = ws.o[m][3] = 0.f;
-
-  if (warp == NCONS) {
+  if (ntile == 0) {
+    // no tiles for this CTA: it only takes its grid ticket below
+  } else if (warp == NC) {
     // ---------------------------------------------------------------- producer
     // lane s owns stage s and issues tiles s, s + NSTAGES, s + 2 NSTAGES, ...
     // (1 bulk copy per packed page, 2 per FP16 tile): the initial fill of every
@@ -456,351 +660,342 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
     static_assert(NSTAGES <= 32, "one producer lane per stage");
     if (lane < NSTAGES) {
       const int s = lane;
-      const size_t npg = static_cast<size_t>(c.cap / PK);
-      const uint8_t* pages = c.pages + static_cast<size_t>(bh) * npg * HQ_PAGE_BYTES;
-      const uint16_t* kf = c.kf + static_cast<size_t>(bh) * c.vl_cap * D;
-      const uint16_t* vf = c.vf + static_cast<size_t>(bh) * c.vl_cap * D;
-      const uint16_t* kr = c.kr + static_cast<size_t>(bh) * R * D;
-      const uint16_t* vr = c.vr + static_cast<size_t>(bh) * R * D;
       uint8_t* st = smem + s * STAGE_BYTES;
-      int k = 0;  // uses of this stage so far
+      int32_t* srow0 = state_row(c, 0);
+      int k = 0;   // uses of this stage so far
+      int si = 0;  // segment cursor
+      UnitGeo ug = geo_of_unit(c, plan.seg[0].u, R);
+      TileWalk tw;
+      bool fresh = true;
       for (int i = s; i < ntile; i += NSTAGES, ++k) {
+        while (i >= plan.seg[si].b) {
+          ++si;
+          ug = geo_of_unit(c, plan.seg[si].u, R);
+          fresh = true;
+        }
+        const Seg sg = plan.seg[si];
+        if (fresh) {
+          tw.start(ug, sg.k0 + (i - sg.a), NSTAGES);
+          fresh = false;
+        } else {
+          tw.step(NSTAGES);
+        }
+        int32_t* srow = state_row(c, sg.u / c.Hkv);
         // the k-th refill waits for the consumer's k-th release (phase k - 1)
-        if (k > 0 && !mbar_wait(&empty[s], (k - 1) & 1, c.state)) {
+        if (k > 0 && !mbar_wait(&empty[s], (k - 1) & 1, srow)) {
           s_timeout = 1;
           break;
         }
         s_issued[s] = k + 1;
-        const int tile = sp.tile(i);
-        if (tile < geo.NP) {
+        const int tl = tw.tile();
+        if (tl >= 0) {
           mbar_arrive_expect_tx(&full[s], PK_TX);
-          bulk_g2s(st, pages + static_cast<size_t>(tile) * HQ_PAGE_BYTES, PK_TX, &full[s]);
+          bulk_g2s(st, page_of(c, sg.u, tl * PK), PK_TX, &full[s]);
         } else {
-          const int v = tile - geo.NP, j = v - geo.NV;
-          const uint16_t* ksrc = j < 0 ? kf + v * (FT * D) : (j < geo.NR - 1 ? kr + j * (FT * D) : k_new + bh * D);
-          const uint16_t* vsrc = j < 0 ? vf + v * (FT * D) : (j < geo.NR - 1 ? vr + j * (FT * D) : v_new + bh * D);
-          const uint32_t bytes = j == geo.NR - 1 ? 2 * D : FT * 2 * D;
+          const uint16_t *ks, *vs;
+          uint32_t bytes;
+          fp16_src(c, ug, sg.u, -tl - 1, R, k_new, v_new, ks, vs, bytes);
           mbar_arrive_expect_tx(&full[s], 2 * bytes);
-          bulk_g2s(st, ksrc, bytes, &full[s]);
-          bulk_g2s(st + OFF_FV, vsrc, bytes, &full[s]);
+          bulk_g2s(st, ks, bytes, &full[s]);
+          bulk_g2s(st + OFF_FV, vs, bytes, &full[s]);
         }
       }
+      (void)srow0;
     }
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- consumers
-    // Q^T fragments in the permuted dim order (thread t covers dims 32t .. 32t+31)
-    uint32_t qf[8][2];
-    if (g < G) {
-      const uint4* qp = reinterpret_cast<const uint4*>(q + (static_cast<size_t>(b) * c.Hq + kvh * G + g) * D + 32 * t);
+    const int NTHR = NC * 32;
+    for (int si = 0; si < nseg; ++si) {
+      const Seg sg = plan.seg[si];
+      const int u = sg.u, b = u / c.Hkv, kvh = u % c.Hkv;
+      int32_t* srow = state_row(c, b);
+      const UnitGeo ug = geo_of_unit(c, u, R);
+      uint32_t qf[8][2];
+      load_q(c, q, b, kvh, G, g, t, qf);
+      WarpState ws;
+      ws.m[0] = ws.m[1] = -INFINITY;
+      ws.l[0] = ws.l[1] = 0.f;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 u = qp[i];
-        qf[2 * i][0] = prmt(u.x, u.z, 0x5410);
-        qf[2 * i][1] = prmt(u.x, u.z, 0x7632);
-        qf[2 * i + 1][0] = prmt(u.y, u.w, 0x5410);
-        qf[2 * i + 1][1] = prmt(u.y, u.w, 0x7632);
+      for (int m = 0; m < 8; ++m) ws.o[m][0] = ws.o[m][1] = ws.o[m][2] = ws.o[m][3] = 0.f;
+      // this warp's tiles of the segment: i = sg.a + ((warp - sg.a) mod NC), step NC
+      int i = sg.a + ((warp - sg.a) % NC + NC) % NC;
+      int held = -1;
+      TileWalk tw;
+      tw.start(ug, sg.k0 + (i - sg.a), NC);
+      for (; i < sg.b; i += NC, tw.step(NC)) {
+        const int s = i % NSTAGES;
+        // the timeout decision is made warp-uniform so the warp never splits
+        if (!__all_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&s_timeout) == 0 &&
+                                         mbar_wait(&full[s], (i / NSTAGES) & 1, srow))) {
+          if (lane == 0) s_timeout = 1;
+          break;
+        }
+        const uint8_t* st = smem + s * STAGE_BYTES;
+        const int tl = tw.tile();
+        if (tl >= 0) {
+          packed_tile(ws, st, qf, tl, ug.n_packed, qscale, g, t);
+        } else {
+          fp16_tile(ws, st, qf, fp16_valid(ug, -tl - 1, R), qscale, g, t);
+        }
+        __syncwarp();
+        if (i + NC < sg.b) {
+          if (lane == 0) mbar_arrive(&empty[s]);
+        } else {
+          held = s;  // the last tile of the segment: keep the stage for the warp state
+        }
       }
-    } else {
+      // l: sum the per-thread partial sums over the 8 lanes of a query column
 #pragma unroll
-      for (int j = 0; j < 8; ++j) qf[j][0] = qf[j][1] = 0u;
-    }
-    for (int i = warp; i < ntile; i += NCONS) {
-      const int s = i % NSTAGES;
-      // the timeout decision is made warp-uniform so the warp never splits
-      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (i / NSTAGES) & 1, c.state))) {
-        if (lane == 0) s_timeout = 1;
-        break;
+      for (int o = 4; o < 32; o <<= 1) {
+        ws.l[0] += __shfl_xor_sync(0xffffffffu, ws.l[0], o);
+        ws.l[1] += __shfl_xor_sync(0xffffffffu, ws.l[1], o);
       }
-      const uint8_t* st = smem + s * STAGE_BYTES;
-      const int tile = sp.tile(i);
-      if (tile < geo.NP) {
-        packed_tile(ws, st, qf, tile, n_packed, qscale, g, t);
-      } else {
-        fp16_tile(ws, st, qf, fp16_valid(geo, tile), qscale, g, t);
+      if (held >= 0) {
+        float* wsm = reinterpret_cast<float*>(smem + held * STAGE_BYTES);
+        if (g == 0) {
+          wsm[2 * t] = ws.m[0];
+          wsm[2 * t + 1] = ws.m[1];
+          wsm[8 + 2 * t] = ws.l[0];
+          wsm[8 + 2 * t + 1] = ws.l[1];
+        }
+        float* wo = wsm + 16;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          wo[(2 * t) * D + 16 * g + 2 * m] = ws.o[m][0];
+          wo[(2 * t + 1) * D + 16 * g + 2 * m] = ws.o[m][1];
+          wo[(2 * t) * D + 16 * g + 2 * m + 1] = ws.o[m][2];
+          wo[(2 * t + 1) * D + 16 * g + 2 * m + 1] = ws.o[m][3];
+        }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-    }
-    // l: sum the per-thread partial sums over the 8 lanes of a query column
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      ws.l[0] += __shfl_xor_sync(0xffffffffu, ws.l[0], o);
-      ws.l[1] += __shfl_xor_sync(0xffffffffu, ws.l[1], o);
-    }
-  }
-  __syncthreads();  // (A) every tile consumed: stage memory is free for the merge
-  if (s_timeout) {
-    // never expected: before the stage memory is reused or the CTA exits, wait
-    // (bounded) for every bulk copy this CTA issued to land
-    if (threadIdx.x == 0)
-      for (int st = 0; st < NSTAGES; ++st)
-        if (s_issued[st] > 0) mbar_wait(&full[st], (s_issued[st] - 1) & 1, c.state);
-    __syncthreads();
-  }
-  if (warp < NCONS) {
-    float* wsm = reinterpret_cast<float*>(smem) + warp * PART_FLOATS;
-    if (g == 0) {
-      wsm[2 * t] = ws.m[0];
-      wsm[2 * t + 1] = ws.m[1];
-      wsm[8 + 2 * t] = ws.l[0];
-      wsm[8 + 2 * t + 1] = ws.l[1];
-    }
-    float* wo = wsm + 16;
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      wo[(2 * t) * D + 16 * g + 2 * m] = ws.o[m][0];
-      wo[(2 * t + 1) * D + 16 * g + 2 * m] = ws.o[m][1];
-      wo[(2 * t) * D + 16 * g + 2 * m + 1] = ws.o[m][2];
-      wo[(2 * t + 1) * D + 16 * g + 2 * m + 1] = ws.o[m][3];
-    }
-  }
-  __syncthreads();  // (B) warp states visible
-
-  // ---------------------------------------------------------------- CTA merge -> split partial
-  // each thread owns 4 dims of one query and weighs the NC warp states itself
-  // (NC exp2 per thread instead of a third barrier)
-  __shared__ int s_glast;
-  const float* wsm = reinterpret_cast<const float*>(smem);
-  float* part = parts + (static_cast<size_t>(bh) * S + split) * PART_FLOATS;
-  for (int i = threadIdx.x; i < 8 * D / 4; i += NTHREADS) {
-    const int qc = (4 * i) / D;
-    float mm = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < NCONS; ++w) mm = fmaxf(mm, wsm[w * PART_FLOATS + qc]);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float ll = 0.f;
-#pragma unroll
-    for (int w = 0; w < NCONS; ++w) {
-      const float mw = wsm[w * PART_FLOATS + qc];
-      const float wt = mw == -INFINITY ? 0.f : ex2(mw - mm);
-      const float4 o = reinterpret_cast<const float4*>(wsm + w * PART_FLOATS + 16)[i];
-      acc.x = fmaf(wt, o.x, acc.x);
-      acc.y = fmaf(wt, o.y, acc.y);
-      acc.z = fmaf(wt, o.z, acc.z);
-      acc.w = fmaf(wt, o.w, acc.w);
-      ll = fmaf(wt, wsm[w * PART_FLOATS + 8 + qc], ll);
-    }
-    reinterpret_cast<float4*>(part + 16)[i] = acc;
-    if ((4 * i) % D == 0) {
-      part[qc] = mm;
-      part[8 + qc] = ll;
-    }
-  }
-  // the new token's K / V rows and this group's queries, loaded now so that the
-  // append after the ticket is stores only (inputs: no ordering concerns)
-  const int slot = T % R;
-  constexpr int APPEND_MAX = (2 + HQ_MAX_GQA) * (D / 8);
-  static_assert(APPEND_MAX <= 2 * NTHREADS, "at most two 16-byte chunks of the append per thread");
-  uint4 app[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
-  uint4* app_dst[2] = {nullptr, nullptr};
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int e = threadIdx.x + k * NTHREADS;
-    if (e < (2 + G) * (D / 8)) {
-      const int row = e / (D / 8), ch = e % (D / 8);
-      if (row < 2) {
-        app[k] = reinterpret_cast<const uint4*>((row ? v_new : k_new) + static_cast<size_t>(bh) * D)[ch];
-        app_dst[k] = reinterpret_cast<uint4*>((row ? c.vr : c.kr) + (static_cast<size_t>(bh) * R + slot) * D) + ch;
-      } else {
-        const size_t h = static_cast<size_t>(b) * c.Hq + kvh * G + (row - 2);
-        app[k] = reinterpret_cast<const uint4*>(q + h * D)[ch];
-        app_dst[k] = reinterpret_cast<uint4*>(c.qbuf + (h * HQ_QBUF + (T % HQ_QBUF)) * D) + ch;
-      }
-    }
-  }
-  // completion tickets: the barrier orders every thread's partial writes before
-  // thread 0's gpu-scope release; the two counters are bumped together; the
-  // last CTA of the head (and/or of the grid) acquires before the barrier that
-  // releases its other threads to read the partials
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    fence_acq_rel_gpu();
-    const unsigned int th = atomicAdd(&tickets[1 + bh], 1u);
-    const unsigned int tg = atomicAdd(&tickets[0], 1u);
-    s_last = th == static_cast<unsigned>(S - 1);
-    s_glast = tg == gridDim.x * gridDim.y * gridDim.z - 1;
-    if (s_last || s_glast) fence_acq_rel_gpu();
-  }
-  __syncthreads();
-  if (s_last) {
-    // log-sum-exp merge of the S partials of this (b, kv head).  The threads
-    // split into ngrp groups, each summing the O partials of every ngrp-th split
-    // for one (query, 4 dims) item; a thread's first PER O loads are issued
-    // before the (m, l) of the splits are gathered and weighed, so both round
-    // trips to L2 overlap, and the groups' sums meet in shared memory.
-    const float* pb = parts + static_cast<size_t>(bh) * S * PART_FLOATS;
-    float* sm_m = reinterpret_cast<float*>(smem);      // [S][8]: the split weights
-    float* sm_inv = sm_m + 2 * 64 * 8;                  // [8]
-    float4* red = reinterpret_cast<float4*>(sm_inv + 8);  // [ngrp][items]
-    constexpr int PER = 8;
-    const int items = G * (D / 4);
-    const bool grouped = items <= NTHREADS;             // else one pass over items per thread stride
-    const int ngrp = grouped ? max(1, min(NTHREADS / items, S)) : 1;
-    const int grp = grouped ? threadIdx.x / items : 0;
-    const int it0 = threadIdx.x - grp * items;
-    const bool mine = grouped && grp < ngrp;
-    const float4* osrc = reinterpret_cast<const float4*>(pb + 16 + (it0 / (D / 4)) * D) + it0 % (D / 4);
-    float4 ov[PER];
-#pragma unroll
-    for (int j = 0; j < PER; ++j) {
-      const int sp = grp + j * ngrp;
-      ov[j] = (mine && sp < S) ? __ldcg(osrc + sp * (PART_FLOATS / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    // split weights: warp qc weighs query qc's splits, lane s holding splits s
-    // and s + 32 (S <= 64), with warp-wide max and sum
-    static_assert(MAX_SPLITS <= 64, "two splits per lane");
-    for (int qc = warp; qc < G; qc += NTHREADS / 32) {
-      float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-      if (lane < S) {
-        m0 = __ldcg(pb + lane * PART_FLOATS + qc);
-        l0 = __ldcg(pb + lane * PART_FLOATS + 8 + qc);
-      }
-      if (lane + 32 < S) {
-        m1 = __ldcg(pb + (lane + 32) * PART_FLOATS + qc);
-        l1 = __ldcg(pb + (lane + 32) * PART_FLOATS + 8 + qc);
-      }
-      float mm = fmaxf(m0, m1);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, o));
-      const float w0 = m0 == -INFINITY ? 0.f : ex2(m0 - mm);
-      const float w1 = m1 == -INFINITY ? 0.f : ex2(m1 - mm);
-      float ll = w0 * l0 + w1 * l1;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ll += __shfl_xor_sync(0xffffffffu, ll, o);
-      if (lane < S) sm_m[lane * 8 + qc] = w0;
-      if (lane + 32 < S) sm_m[(lane + 32) * 8 + qc] = w1;
-      if (lane == 0) sm_inv[qc] = ll > 0.f ? 1.0f / ll : 0.f;
-    }
-    __syncthreads();
-    auto store_out = [&](int it, const float4& acc) {
-      const int qc = it / (D / 4), d4 = it % (D / 4);
-      const float inv = sm_inv[qc];
-      __half2* dst = reinterpret_cast<__half2*>(out + (static_cast<size_t>(b) * c.Hq + kvh * G + qc) * D) + 2 * d4;
-      dst[0] = __floats2half2_rn(acc.x * inv, acc.y * inv);
-      dst[1] = __floats2half2_rn(acc.z * inv, acc.w * inv);
-    };
-    if (grouped) {
-      if (mine) {
-        const int qc = it0 / (D / 4);
+      if (lane == 0) s_held[warp] = held;
+      consumer_bar();  // (A) warp states visible
+      // ------------------------------------------------------------ CTA merge -> segment partial
+      // each thread owns 4 dims of one query and weighs the warp states itself
+      const int c_slot = blockIdx.x + u;  // partial slot of (this CTA, unit u)
+      float* part = parts + static_cast<size_t>(c_slot) * PART_FLOATS;
+      // scratch for the unit merge: a held stage (every segment has a tile, so some
+      // warp holds one unless a wait timed out; then stage 0, which stays in bounds)
+      int scratch = 0;
+      for (int w = NC - 1; w >= 0; --w)
+        if (s_held[w] >= 0) scratch = s_held[w];
+      for (int it = threadIdx.x; it < 8 * D / 4; it += NTHR) {
+        const int qc = (4 * it) / D;
+        float mm = -INFINITY;
+        for (int w = 0; w < NC; ++w)
+          if (s_held[w] >= 0) mm = fmaxf(mm, reinterpret_cast<const float*>(smem + s_held[w] * STAGE_BYTES)[qc]);
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float ll = 0.f;
+        for (int w = 0; w < NC; ++w) {
+          if (s_held[w] < 0) continue;
+          const float* wsm = reinterpret_cast<const float*>(smem + s_held[w] * STAGE_BYTES);
+          const float mw = wsm[qc];
+          const float wt = mw == -INFINITY ? 0.f : ex2(mw - mm);
+          const float4 o = reinterpret_cast<const float4*>(wsm + 16)[it];
+          acc.x = fmaf(wt, o.x, acc.x);
+          acc.y = fmaf(wt, o.y, acc.y);
+          acc.z = fmaf(wt, o.z, acc.z);
+          acc.w = fmaf(wt, o.w, acc.w);
+          ll = fmaf(wt, wsm[8 + qc], ll);
+        }
+        reinterpret_cast<float4*>(part + 16)[it] = acc;
+        if ((4 * it) % D == 0) {
+          part[qc] = mm;
+          part[8 + qc] = ll;
+        }
+      }
+      // the new token's K / V rows and this group's queries, loaded now so that the
+      // append after the ticket is stores only (inputs: no ordering concerns)
+      const int T = ug.T;
+      const int slot = T % R;
+      const int bh = u;
+      constexpr int APPEND_MAX = (2 + HQ_MAX_GQA) * (D / 8);
+      static_assert(APPEND_MAX <= 2 * NC * 32, "at most two 16-byte chunks of the append per consumer thread");
+      uint4 app[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+      uint4* app_dst[2] = {nullptr, nullptr};
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int e = threadIdx.x + k * NTHR;
+        if (e < (2 + G) * (D / 8)) {
+          const int row = e / (D / 8), ch = e % (D / 8);
+          if (row < 2) {
+            app[k] = reinterpret_cast<const uint4*>((row ? v_new : k_new) + static_cast<size_t>(bh) * D)[ch];
+            app_dst[k] = reinterpret_cast<uint4*>((row ? c.vr : c.kr) + (static_cast<size_t>(bh) * R + slot) * D) + ch;
+          } else {
+            const size_t h = static_cast<size_t>(b) * c.Hq + kvh * G + (row - 2);
+            app[k] = reinterpret_cast<const uint4*>(q + h * D)[ch];
+            app_dst[k] = reinterpret_cast<uint4*>(c.qbuf + (h * HQ_QBUF + (T % HQ_QBUF)) * D) + ch;
+          }
+        }
+      }
+      // completion ticket of the unit: the barrier orders every thread's partial
+      // writes before thread 0's gpu-scope release; the last CTA acquires before
+      // the barrier that releases its other threads to read the partials
+      consumer_bar();  // (B) partial written, warp states read
+      if (threadIdx.x == 0) {
+        fence_acq_rel_gpu();
+        const unsigned int th = atomicAdd(&tickets[1 + u], 1u);
+        s_last = th == static_cast<unsigned>(sg.ncta - 1);
+        if (s_last) fence_acq_rel_gpu();
+      }
+      consumer_bar();  // (C)
+      if (s_last) {
+        // log-sum-exp merge of the unit's partials (slots first_cta + u ..), in the
+        // scratch stage.  The threads split into ngrp groups, each summing the O
+        // partials of every ngrp-th CTA for one (query, 4 dims) item; a thread's
+        // first PER O loads are issued before the (m, l) of the partials are
+        // gathered and weighed, so both round trips to L2 overlap.
+        const int S = sg.ncta;
+        const float* pb = parts + static_cast<size_t>(sg.first_cta + u) * PART_FLOATS;
+        float* sm_m = reinterpret_cast<float*>(smem + scratch * STAGE_BYTES);  // [S][8] weights
+        float* sm_inv = sm_m + 8 * S;                                          // [8]
+        float4* red4 = reinterpret_cast<float4*>(sm_inv + 8);                  // [ngrp][items]
+        constexpr int PER = 8;
+        const int items = G * (D / 4);
+        const int room = (STAGE_BYTES - 4 * (8 * S + 8)) / (16 * items);      // groups the scratch stage holds
+        const int ngrp = max(1, min(min(NTHR / items, S), room));
+        const int grp = threadIdx.x / items;
+        const int it0 = threadIdx.x - grp * items;
+        const bool mine = grp < ngrp;
+        const float4* osrc = reinterpret_cast<const float4*>(pb + 16 + (it0 / (D / 4)) * D) + it0 % (D / 4);
+        float4 ov[PER];
 #pragma unroll
         for (int j = 0; j < PER; ++j) {
           const int sp = grp + j * ngrp;
-          const float w = sp < S ? sm_m[sp * 8 + qc] : 0.f;
-          acc.x = fmaf(w, ov[j].x, acc.x);
-          acc.y = fmaf(w, ov[j].y, acc.y);
-          acc.z = fmaf(w, ov[j].z, acc.z);
-          acc.w = fmaf(w, ov[j].w, acc.w);
+          ov[j] = (mine && sp < S) ? __ldcg(osrc + sp * (PART_FLOATS / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        for (int sp = grp + PER * ngrp; sp < S; sp += ngrp) {  // more than PER splits per group
-          const float4 o = __ldcg(osrc + sp * (PART_FLOATS / 4));
-          const float w = sm_m[sp * 8 + qc];
-          acc.x = fmaf(w, o.x, acc.x);
-          acc.y = fmaf(w, o.y, acc.y);
-          acc.z = fmaf(w, o.z, acc.z);
-          acc.w = fmaf(w, o.w, acc.w);
+        // partial weights: warp qc weighs query qc's partials, lane s holding s, s + 32, ...
+        for (int qc = warp; qc < G; qc += NC) {
+          float mm = -INFINITY;
+          for (int sp = lane; sp < S; sp += 32) mm = fmaxf(mm, __ldcg(pb + sp * PART_FLOATS + qc));
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, o));
+          float ll = 0.f;
+          for (int sp = lane; sp < S; sp += 32) {
+            const float m0 = __ldcg(pb + sp * PART_FLOATS + qc);
+            const float w0 = m0 == -INFINITY ? 0.f : ex2(m0 - mm);
+            ll = fmaf(w0, __ldcg(pb + sp * PART_FLOATS + 8 + qc), ll);
+            sm_m[sp * 8 + qc] = w0;
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) ll += __shfl_xor_sync(0xffffffffu, ll, o);
+          if (lane == 0) sm_inv[qc] = ll > 0.f ? 1.0f / ll : 0.f;
         }
-        red[grp * items + it0] = acc;
+        consumer_bar();
+        if (mine) {
+          const int qc = it0 / (D / 4);
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int j = 0; j < PER; ++j) {
+            const int sp = grp + j * ngrp;
+            const float w = sp < S ? sm_m[sp * 8 + qc] : 0.f;
+            acc.x = fmaf(w, ov[j].x, acc.x);
+            acc.y = fmaf(w, ov[j].y, acc.y);
+            acc.z = fmaf(w, ov[j].z, acc.z);
+            acc.w = fmaf(w, ov[j].w, acc.w);
+          }
+          for (int sp = grp + PER * ngrp; sp < S; sp += ngrp) {  // more than PER partials per group
+            const float4 o = __ldcg(osrc + sp * (PART_FLOATS / 4));
+            const float w = sm_m[sp * 8 + qc];
+            acc.x = fmaf(w, o.x, acc.x);
+            acc.y = fmaf(w, o.y, acc.y);
+            acc.z = fmaf(w, o.z, acc.z);
+            acc.w = fmaf(w, o.w, acc.w);
+          }
+          red4[grp * items + it0] = acc;
+        }
+        consumer_bar();
+        for (int it = threadIdx.x; it < items; it += NTHR) {
+          float4 acc = red4[it];
+          for (int g2 = 1; g2 < ngrp; ++g2) {
+            const float4 o = red4[g2 * items + it];
+            acc.x += o.x;
+            acc.y += o.y;
+            acc.z += o.z;
+            acc.w += o.w;
+          }
+          const int qc = it / (D / 4), d4 = it % (D / 4);
+          const float inv = sm_inv[qc];
+          __half2* dst = reinterpret_cast<__half2*>(out + (static_cast<size_t>(b) * c.Hq + kvh * G + qc) * D) + 2 * d4;
+          dst[0] = __floats2half2_rn(acc.x * inv, acc.y * inv);
+          dst[1] = __floats2half2_rn(acc.z * inv, acc.w * inv);
+        }
+        // every CTA of this unit has consumed its tiles: append the new token to
+        // the ring (slot T % R) and this group's queries to the query buffer
+        if (app_dst[0]) *app_dst[0] = app[0];
+        if (app_dst[1]) *app_dst[1] = app[1];
+        if (threadIdx.x == 0) tickets[1 + u] = 0u;
       }
-      __syncthreads();
-      if (threadIdx.x < items) {
-        float4 acc = red[threadIdx.x];
-        for (int g2 = 1; g2 < ngrp; ++g2) {
-          const float4 o = red[g2 * items + threadIdx.x];
-          acc.x += o.x;
-          acc.y += o.y;
-          acc.z += o.z;
-          acc.w += o.w;
-        }
-        store_out(threadIdx.x, acc);
-      }
-    } else {
-      for (int it = threadIdx.x; it < items; it += NTHREADS) {
-        const int qc = it / (D / 4), d4 = it % (D / 4);
-        const float4* src = reinterpret_cast<const float4*>(pb + 16 + qc * D) + d4;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-        for (int sp = 0; sp < S; ++sp) {
-          const float4 o = __ldcg(src + sp * (PART_FLOATS / 4));
-          const float w = sm_m[sp * 8 + qc];
-          acc.x = fmaf(w, o.x, acc.x);
-          acc.y = fmaf(w, o.y, acc.y);
-          acc.z = fmaf(w, o.z, acc.z);
-          acc.w = fmaf(w, o.w, acc.w);
-        }
-        store_out(it, acc);
+      // (D) scratch and warp states no longer read: give the held stages back (the
+      // generic-proxy writes to them are ordered before the producer's next bulk copy)
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      consumer_bar();
+      if (held >= 0 && lane == 0) mbar_arrive(&empty[held]);
+    }
+  }
+  __syncthreads();  // every tile consumed
+  if (s_timeout) {
+    // never expected: before the CTA exits, wait (bounded) for every bulk copy
+    // this CTA issued to land
+    if (threadIdx.x == 0)
+      for (int st = 0; st < NSTAGES; ++st)
+        if (s_issued[st] > 0) mbar_wait(&full[st], (s_issued[st] - 1) & 1, state_row(c, 0));
+    __syncthreads();
+  }
+  // The last CTA of the grid advances the lengths.  Every CTA planned from the
+  // state rows, so no T may change before all of them have (a sequence's T
+  // decides whether it takes a step): the grid ticket orders the update after
+  // every CTA's plan and every unit's append.
+  if (threadIdx.x == 0) {
+    fence_acq_rel_gpu();
+    s_last = atomicAdd(&tickets[0], 1u) == gridDim.x - 1;
+    if (s_last) fence_acq_rel_gpu();
+  }
+  __syncthreads();
+  if (s_last) {
+    for (int b = threadIdx.x; b < c.B; b += NTHREADS) {
+      int32_t* st = state_row(c, b);
+      const int T = st[HQ_STATE_T];
+      if (!refused(c, T, st[HQ_STATE_NPACKED])) {
+        st[HQ_STATE_T] = T + 1;
+        st[HQ_STATE_NQ] = min(st[HQ_STATE_NQ] + 1, HQ_QBUF);
       }
     }
-    // every split of this head has consumed its tiles: append the new token to
-    // the ring (slot T % R) and this group's queries to the query buffer
-    if (app_dst[0]) *app_dst[0] = app[0];
-    if (app_dst[1]) *app_dst[1] = app[1];
-    if (threadIdx.x == 0) tickets[1 + bh] = 0u;
-  }
-  // the last CTA of the grid advances T (every CTA read the state at its start)
-  if (s_glast && threadIdx.x == 0) {
-    c.state[HQ_STATE_T] = T + 1;
-    c.state[HQ_STATE_NQ] = min(c.state[HQ_STATE_NQ] + 1, HQ_QBUF);
-    tickets[0] = 0u;
+    if (threadIdx.x == 0) tickets[0] = 0u;
   }
 }
 
 }  // namespace
 
-// Launch shape: the wide CTA (one per SM) when every (b, kv head) can get at
-// least 4 of them, else 3 narrow CTAs per SM; never more than one wave.
-struct DecodeShape {
-  int S;      // splits per (b, kv head)
-  bool wide;
-};
-
-DecodeShape decode_shape(const hq_cache& c, int sms) {
-  const int units = c.B * c.Hkv;
-  const int nt_max = c.cap / PK + c.vl_cap / FT + ring_len(c.W) / FT + 1;
-  DecodeShape d;
-  d.wide = sms / units >= 4;
-  int s = d.wide ? sms / units : (3 * sms) / units;
-  const int cap_s = d.wide ? (nt_max + NC_WIDE - 1) / NC_WIDE : (nt_max + NC_NARROW - 1) / NC_NARROW;  // ~one tile per consumer warp
-  if (s > cap_s) s = cap_s;
-  if (s > MAX_SPLITS) s = MAX_SPLITS;
-  if (s < 1) s = 1;
-  d.S = s;
-  return d;
-}
-
-int decode_splits(const hq_cache& c, int sms) { return decode_shape(c, sms).S; }
-
-// counters: [0] grid ticket, [1 + b*Hkv + h] split tickets; zero between calls
+// counters: [0] grid ticket, [1 + u] unit tickets; zero between calls
 size_t decode_counter_bytes(const hq_cache& c) { return ((4ull * (1 + c.B * c.Hkv) + 255) / 256) * 256; }
 
+// partial slots: (CTA c, unit u) -> c + u, at most sms + units - 1 of them
 size_t decode_workspace(const hq_cache& c, int sms) {
-  const int S = decode_splits(c, sms);
-  return decode_counter_bytes(c) + static_cast<size_t>(c.B) * c.Hkv * S * PART_FLOATS * sizeof(float);
+  return decode_counter_bytes(c) + (static_cast<size_t>(sms) + static_cast<size_t>(c.B) * c.Hkv) * PART_FLOATS * sizeof(float);
 }
+
+bool decode_supported(const hq_cache& c) { return c.B * c.Hkv <= MAX_UNITS; }
+
+// one CTA per SM, at most MAX_CTAS (the unit merge keeps one weight per CTA in a stage)
+constexpr int MAX_CTAS = 160;
 
 hq_status launch_decode(const hq_cache& c, const uint16_t* q, const uint16_t* kn, const uint16_t* vn, uint16_t* out,
                         float sm_scale, void* ws, int sms, cudaStream_t st) {
-  const DecodeShape shp = decode_shape(c, sms);
-  const int nc = shp.wide ? NC_WIDE : NC_NARROW;
-  const int smem = 2 * nc * STAGE_BYTES;
+  if (!decode_supported(c)) return HQ_ERR_UNSUPPORTED;
+  const int smem = NSTAGES * STAGE_BYTES;
   int dev = 0;
   cudaGetDevice(&dev);
   static DeviceOnce attrs;
   const cudaError_t ea = attrs.run(dev, [] {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<NC_WIDE, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         2 * NC_WIDE * STAGE_BYTES);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(decode_kernel<NC_NARROW, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               2 * NC_NARROW * STAGE_BYTES);
-    return e;
+    return cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, NSTAGES * STAGE_BYTES);
   });
   if (ea != cudaSuccess) return cuda_fail(ea, "decode attributes");
   unsigned int* tickets = reinterpret_cast<unsigned int*>(ws);
   float* parts = reinterpret_cast<float*>(static_cast<char*>(ws) + decode_counter_bytes(c));
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(shp.S, c.Hkv, c.B);
-  cfg.blockDim = dim3((nc + 1) * 32, 1, 1);
+  cfg.gridDim = dim3(min(sms, MAX_CTAS), 1, 1);
+  cfg.blockDim = dim3(NTHREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -809,10 +1004,7 @@ hq_status launch_decode(const hq_cache& c, const uint16_t* q, const uint16_t* kn
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const float qs = sm_scale * LOG2E;
-  const cudaError_t e = shp.wide
-      ? cudaLaunchKernelEx(&cfg, decode_kernel<NC_WIDE, 1>, c, q, kn, vn, out, qs, shp.S, parts, tickets)
-      : cudaLaunchKernelEx(&cfg, decode_kernel<NC_NARROW, 3>, c, q, kn, vn, out, qs, shp.S, parts, tickets);
-  return cuda_status(e, "decode launch");
+  return cuda_status(cudaLaunchKernelEx(&cfg, decode_kernel, c, q, kn, vn, out, qs, parts, tickets), "decode launch");
 }
 
 }  // namespace hq

@@ -39,6 +39,7 @@ hq_status launch_decode(const hq_cache& c, const uint16_t* q, const uint16_t* kn
                         float sm_scale, void* ws, int sms, cudaStream_t st);
 size_t decode_workspace(const hq_cache& c, int sms);
 size_t decode_counter_bytes(const hq_cache& c);
+bool decode_supported(const hq_cache& c);
 }  // namespace hq
 
 namespace {
@@ -106,6 +107,7 @@ extern "C" HQ_API hq_status hq_decode_attn_noalloc(const hq_cache* c, const uint
   if (s != HQ_OK) return s;
   if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(out)) return HQ_ERR_INVALID;
   if (!(sm_scale > 0.0f)) return HQ_ERR_INVALID;
+  if (!hq::decode_supported(*c)) return HQ_ERR_UNSUPPORTED;
   int dev = 0, sms = 148;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

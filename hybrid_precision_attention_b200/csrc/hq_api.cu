@@ -9,10 +9,12 @@
 #include "common.cuh"
 
 namespace hq {
+hq_status launch_clear_bitmaps(const hq_cache& c, int sms, cudaStream_t st);
 hq_status launch_pack_merge(const hq_cache& c, const uint16_t* kd, const uint16_t* vd, int L, void* ws, cudaStream_t st);
 hq_status launch_decode(const hq_cache& c, const uint16_t* q, const uint16_t* kn, const uint16_t* vn, uint16_t* out,
                         float sm_scale, void* ws, int sms, cudaStream_t st);
 size_t decode_workspace(const hq_cache& c, int sms);
+bool decode_supported(const hq_cache& c);
 size_t select_workspace(const hq_cache& c, bool need_scores);
 hq_status launch_select(const hq_cache& c, const uint16_t* kd, int L, const uint16_t* qe, int nq, float* scores_out,
                         void* ws, cudaStream_t st);
@@ -78,6 +80,9 @@ hq_status hq_cache_validate(const hq_cache* c) {
   const void* ptrs[] = {c->pages, c->kf, c->vf, c->vl_pos, c->kr, c->vr, c->qbuf, c->vl_sel, c->state};
   for (const void* p : ptrs)
     if (!aligned16(p)) return HQ_ERR_INVALID;
+  if (c->page_table != nullptr && ((reinterpret_cast<uintptr_t>(c->page_table) & 3u) != 0 || c->n_pages < 1))
+    return HQ_ERR_INVALID;
+  if (c->score_acc != nullptr && (reinterpret_cast<uintptr_t>(c->score_acc) & 15u) != 0) return HQ_ERR_INVALID;
   return HQ_OK;
 }
 
@@ -99,11 +104,13 @@ hq_status hq_cache_reset(const hq_cache* c, hq_stream_t stream) {
   hq_status s = hq_cache_validate(c);
   if (s != HQ_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemsetAsync(c->state, 0, HQ_STATE_WORDS * sizeof(int32_t), st);
+  cudaError_t e = cudaMemsetAsync(c->state, 0, static_cast<size_t>(c->B) * HQ_STATE_WORDS * sizeof(int32_t), st);
   if (e != cudaSuccess) return hq::cuda_status(e, "reset state");
-  e = cudaMemset2DAsync(c->pages + HQ_PAGE_VLMASK, HQ_PAGE_BYTES, 0, 8,
-                        static_cast<size_t>(c->B) * c->Hkv * (c->cap / HQ_PAGE_POSITIONS), st);
-  return hq::cuda_status(e, "reset bitmaps");
+  if (c->score_acc != nullptr) {
+    e = cudaMemsetAsync(c->score_acc, 0, static_cast<size_t>(c->B) * c->Hkv * c->cap * sizeof(float), st);
+    if (e != cudaSuccess) return hq::cuda_status(e, "reset running scores");
+  }
+  return hq::launch_clear_bitmaps(*c, sm_count(), st);
 }
 
 hq_status hq_select_vlines(const hq_cache* c, const uint16_t* k_dense, int32_t L, const uint16_t* q_ext, int32_t nq,
@@ -144,6 +151,7 @@ hq_status hq_decode_attn(const hq_cache* c, const uint16_t* q, const uint16_t* k
   if (s != HQ_OK) return s;
   if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(out)) return HQ_ERR_INVALID;
   if (!(sm_scale > 0.0f)) return HQ_ERR_INVALID;
+  if (!hq::decode_supported(*c)) return HQ_ERR_UNSUPPORTED;
   const int sms = sm_count();
   if (!aligned16(ws) || ws_bytes < hq::decode_workspace(*c, sms)) return HQ_ERR_WORKSPACE;
   return hq::launch_decode(*c, q, k_new, v_new, out, sm_scale, ws, sms, reinterpret_cast<cudaStream_t>(stream));

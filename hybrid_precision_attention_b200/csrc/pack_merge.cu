@@ -62,36 +62,37 @@ __device__ __forceinline__ void pack_row_warp(const uint16_t* __restrict__ src, 
 }
 
 // Rows [lo, hi) of every (b, kv head), K and V.  Init: src = dense [B,Hkv,L,D],
-// lo = 0, hi = max(L - W, 0).  Merge: src = ring, lo = n_packed, hi = T - W
-// (read from state).
+// lo = 0, hi = max(L - W, 0) for every sequence.  Merge: src = ring, and per
+// sequence lo = n_packed, hi = T - W (from its state row; at most R rows, the
+// ring's length, since the ring holds every position in [n_packed, T)).
 __global__ void pack_rows_kernel(hq_cache c, const uint16_t* __restrict__ kd, const uint16_t* __restrict__ vd, int L,
                                  int init) {
   const Dims d = dims_of(c);
-  int lo, hi;
-  if (init) {
-    lo = 0;
-    hi = max(L - d.W, 0);
-  } else {
-    lo = c.state[HQ_STATE_NPACKED];
-    hi = max(lo, c.state[HQ_STATE_T] - d.W);
-  }
-  const int n = hi - lo;
-  if (n <= 0) return;
+  const int nmax = init ? max(L - d.W, 0) : d.R;
+  if (nmax <= 0) return;
   const int lane = threadIdx.x & 31;
   const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
-  const long long total = 2ll * d.B * d.Hkv * n;  // (K or V) x (b, h) x rows
+  const long long total = 2ll * d.B * d.Hkv * nmax;  // (K or V) x (b, h) x rows
   for (long long w = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); w < total; w += warps) {
     const int which = static_cast<int>(w & 1);
     const long long rest = w >> 1;
-    const int p = lo + static_cast<int>(rest % n);
-    const long long bh = rest / n;
+    const int r = static_cast<int>(rest % nmax);
+    const long long bh = rest / nmax;
+    int p;
     const uint16_t* src;
     if (init) {
+      p = r;
       src = (which ? vd : kd) + (bh * L + p) * D;
     } else {
+      const int32_t* st = state_row(c, static_cast<int>(bh / d.Hkv));
+      const int lo = st[HQ_STATE_NPACKED];
+      const int hi = max(lo, st[HQ_STATE_T] - d.W);
+      p = lo + r;
+      if (p >= hi) continue;
       src = (which ? c.vr : c.kr) + (bh * d.R + (p % d.R)) * D;
     }
-    uint8_t* page = page_of(c, bh, p);
+    uint8_t* page = page_for_write(c, bh, p);
+    if (page == nullptr) continue;
     pack_row_warp(src, row_codes(page, which, p), row_sz(page, which, p), lane);
   }
 }
@@ -127,24 +128,27 @@ __device__ __forceinline__ int find_sorted(const int32_t* __restrict__ a, int n,
 }
 
 // Merge: gather the FP16 rows of the new VL set into the workspace and clear the
-// bitmap bits of the old set.  One warp per (b, h, r, K|V).
+// bitmap bits of the old set.  One warp per (b, h, r, K|V); every sequence
+// uses its own state row.
 __global__ void vl_gather_kernel(hq_cache c, uint16_t* __restrict__ wsk, uint16_t* __restrict__ wsv) {
   const Dims d = dims_of(c);
-  const int n_packed = c.state[HQ_STATE_NPACKED];
-  const int n_vl = c.state[HQ_STATE_NVL];
-  const int k = min(c.state[HQ_STATE_KSEL], d.vl_cap);
   const int lane = threadIdx.x & 31;
   const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
-  const long long total = 2ll * d.B * d.Hkv * k;
+  const long long total = 2ll * d.B * d.Hkv * d.vl_cap;
   for (long long w = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); w < total; w += warps) {
     const int which = static_cast<int>(w & 1);
     const long long rest = w >> 1;
-    const int r = static_cast<int>(rest % k);
-    const long long bh = rest / k;
+    const int r = static_cast<int>(rest % d.vl_cap);
+    const long long bh = rest / d.vl_cap;
+    int32_t* st = state_row(c, static_cast<int>(bh / d.Hkv));
+    const int k = min(st[HQ_STATE_KSEL], d.vl_cap);
+    if (r >= k) continue;
+    const int n_packed = st[HQ_STATE_NPACKED];
+    const int n_vl = st[HQ_STATE_NVL];
     const int p = c.vl_sel[bh * d.vl_cap + r];
     uint16_t* dst = (which ? wsv : wsk) + (bh * d.vl_cap + r) * D;
-    if (p < 0 || p >= max(n_packed, c.state[HQ_STATE_T] - d.W)) {  // not a position the merge can hold
-      if (lane == 0) set_err(c.state, HQ_DEVERR_VL_CAPACITY);
+    if (p < 0 || p >= max(n_packed, st[HQ_STATE_T] - d.W)) {  // not a position the merge can hold
+      if (lane == 0) set_err(st, HQ_DEVERR_VL_CAPACITY);
       continue;
     }
     const int old = find_sorted(c.vl_pos + bh * d.vl_cap, n_vl, p);
@@ -176,36 +180,40 @@ __global__ void vl_gather_kernel(hq_cache c, uint16_t* __restrict__ wsk, uint16_
     }
   }
   // clear the old set's bitmap bits (nothing in this kernel reads the bitmap)
-  const long long tot2 = static_cast<long long>(d.B) * d.Hkv * n_vl;
+  const long long tot2 = static_cast<long long>(d.B) * d.Hkv * d.vl_cap;
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < tot2;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long bh = i / n_vl;
-    const int r = static_cast<int>(i % n_vl);
+    const long long bh = i / d.vl_cap;
+    const int r = static_cast<int>(i % d.vl_cap);
+    if (r >= state_row(c, static_cast<int>(bh / d.Hkv))[HQ_STATE_NVL]) continue;
     const int p = c.vl_pos[bh * d.vl_cap + r];
-    atomicAnd(page_mask(page_of(c, bh, p)) + ((p & 63) >> 5), ~(1u << (p & 31)));
+    uint8_t* page = page_for_write(c, bh, p);
+    if (page) atomicAnd(page_mask(page) + ((p & 63) >> 5), ~(1u << (p & 31)));
   }
 }
 
 // Install rows into the VL store.  Init: rows from the dense prefix; merge: rows
 // from the workspace.  Sets bitmap bits, writes vl_pos.  The last block to finish
-// (ticket) updates the state words.
+// (ticket) updates the state rows.
 __global__ void vl_install_kernel(hq_cache c, const uint16_t* __restrict__ srck, const uint16_t* __restrict__ srcv, int L,
                                   int init, unsigned int* __restrict__ ticket) {
   const Dims d = dims_of(c);
-  const int k = min(c.state[HQ_STATE_KSEL], d.vl_cap);
-  const long long chunks = 2ll * d.B * d.Hkv * k * (D / 8);
+  const long long chunks = 2ll * d.B * d.Hkv * d.vl_cap * (D / 8);
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < chunks;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
     const int ch = static_cast<int>(i % (D / 8));
     long long r = i / (D / 8);
     const int which = static_cast<int>(r & 1);
     r >>= 1;
-    const int row = static_cast<int>(r % k);
-    const long long bh = r / k;
+    const int row = static_cast<int>(r % d.vl_cap);
+    const long long bh = r / d.vl_cap;
+    int32_t* st = state_row(c, static_cast<int>(bh / d.Hkv));
+    const int k = min(st[HQ_STATE_KSEL], d.vl_cap);
+    if (row >= k) continue;
     const int p = c.vl_sel[bh * d.vl_cap + row];
-    const int limit = init ? max(L - d.W, 0) : max(c.state[HQ_STATE_NPACKED], c.state[HQ_STATE_T] - d.W);
+    const int limit = init ? max(L - d.W, 0) : max(st[HQ_STATE_NPACKED], st[HQ_STATE_T] - d.W);
     if (p < 0 || p >= limit) {
-      if (ch == 0 && which == 0) set_err(c.state, HQ_DEVERR_VL_CAPACITY);
+      if (ch == 0 && which == 0) set_err(st, HQ_DEVERR_VL_CAPACITY);
       continue;
     }
     const uint16_t* s = init ? ((which ? srcv : srck) + (bh * L + p) * D) : ((which ? srcv : srck) + (bh * d.vl_cap + row) * D);
@@ -213,15 +221,17 @@ __global__ void vl_install_kernel(hq_cache c, const uint16_t* __restrict__ srck,
     reinterpret_cast<uint4*>(t)[ch] = reinterpret_cast<const uint4*>(s)[ch];
     if (ch == 0 && which == 0) {
       c.vl_pos[bh * d.vl_cap + row] = p;
-      uint8_t* page = page_of(c, bh, p);
-      atomicOr(page_mask(page) + ((p & 63) >> 5), 1u << (p & 31));
-      // the first vertical line of a page records its VL-store row (rows are in
-      // ascending position order), so readers find a line's row by a popcount
-      if (row == 0 || (c.vl_sel[bh * d.vl_cap + row - 1] >> 6) != (p >> 6))
-        *reinterpret_cast<int32_t*>(page + HQ_PAGE_VLBASE) = row;
+      uint8_t* page = page_for_write(c, bh, p);
+      if (page) {
+        atomicOr(page_mask(page) + ((p & 63) >> 5), 1u << (p & 31));
+        // the first vertical line of a page records its VL-store row (rows are in
+        // ascending position order), so readers find a line's row by a popcount
+        if (row == 0 || (c.vl_sel[bh * d.vl_cap + row - 1] >> 6) != (p >> 6))
+          *reinterpret_cast<int32_t*>(page + HQ_PAGE_VLBASE) = row;
+      }
     }
   }
-  // state update by the last block (every block has read state above)
+  // state update by the last block (every block has read the state rows above)
   __syncthreads();
   __shared__ unsigned int last;
   if (threadIdx.x == 0) {
@@ -229,17 +239,32 @@ __global__ void vl_install_kernel(hq_cache c, const uint16_t* __restrict__ srck,
     last = (atomicAdd(ticket, 1u) == gridDim.x - 1) ? 1u : 0u;
   }
   __syncthreads();
-  if (last && threadIdx.x == 0) {
-    if (init) {
-      c.state[HQ_STATE_T] = L;
-      c.state[HQ_STATE_NPACKED] = max(L - d.W, 0);
-      c.state[HQ_STATE_NQ] = 0;
-    } else {
-      const int t = c.state[HQ_STATE_T];
-      c.state[HQ_STATE_NPACKED] = max(c.state[HQ_STATE_NPACKED], t - d.W);
+  if (last) {
+    for (int b = threadIdx.x; b < d.B; b += blockDim.x) {
+      int32_t* st = state_row(c, b);
+      if (init) {
+        st[HQ_STATE_T] = L;
+        st[HQ_STATE_NPACKED] = max(L - d.W, 0);
+        st[HQ_STATE_NQ] = 0;
+      } else {
+        st[HQ_STATE_NPACKED] = max(st[HQ_STATE_NPACKED], st[HQ_STATE_T] - d.W);
+      }
+      st[HQ_STATE_NVL] = min(st[HQ_STATE_KSEL], d.vl_cap);
     }
-    c.state[HQ_STATE_NVL] = k;
-    *ticket = 0u;
+    if (threadIdx.x == 0) *ticket = 0u;
+  }
+}
+
+// Clear the VL bitmap of every page the descriptor's sequences own (through
+// the page table when there is one); entries outside the pool are skipped.
+__global__ void clear_bitmaps_kernel(hq_cache c) {
+  const int npg = c.cap / HQ_PAGE_POSITIONS;
+  const long long total = static_cast<long long>(c.B) * c.Hkv * npg;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long idx = page_index(c, static_cast<size_t>(i / npg), static_cast<int>(i % npg));
+    if (idx < 0) continue;
+    *reinterpret_cast<uint2*>(c.pages + static_cast<size_t>(idx) * HQ_PAGE_BYTES + HQ_PAGE_VLMASK) = make_uint2(0u, 0u);
   }
 }
 
@@ -259,11 +284,7 @@ hq_status launch_pack_merge(const hq_cache& c, const uint16_t* kd, const uint16_
   unsigned int* ticket = reinterpret_cast<unsigned int*>(ws);
   uint16_t* wsk = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + 256);
   uint16_t* wsv = wsk + static_cast<size_t>(c.B) * c.Hkv * c.vl_cap * D;
-  if (init) {
-    if (cudaMemset2DAsync(c.pages + HQ_PAGE_VLMASK, HQ_PAGE_BYTES, 0, 8,
-                          static_cast<size_t>(c.B) * c.Hkv * (c.cap / HQ_PAGE_POSITIONS), st) != cudaSuccess)
-      return cuda_fail(cudaGetLastError(), "merge setup");
-  }
+  if (init) clear_bitmaps_kernel<<<sms, threads, 0, st>>>(c);
   pack_rows_kernel<<<sms * 4, threads, 0, st>>>(c, kd, vd, L, init);
   if (init) {
     ring_fill_kernel<<<sms, threads, 0, st>>>(c, kd, vd, L);
@@ -273,6 +294,11 @@ hq_status launch_pack_merge(const hq_cache& c, const uint16_t* kd, const uint16_
     vl_install_kernel<<<sms, threads, 0, st>>>(c, wsk, wsv, L, 0, ticket);
   }
   return cuda_status(cudaGetLastError(), "merge launch");
+}
+
+hq_status launch_clear_bitmaps(const hq_cache& c, int sms, cudaStream_t st) {
+  clear_bitmaps_kernel<<<sms, 256, 0, st>>>(c);
+  return cuda_status(cudaGetLastError(), "reset bitmaps");
 }
 
 }  // namespace hq

@@ -24,6 +24,8 @@
 //                    shared memory, a bit-by-bit search of their low 20 bits ->
 //                    the exact k-th value, then an ordered compaction writes the
 //                    chosen positions ascending, ties to the lowest positions
+// With running scores (c.score_acc), pass 1 adds each key's column mass to its
+// stored sum (decode mode) or starts it (init mode) and ranks the sums.
 // Keys are rebuilt as fp16 in their current representation (dense prefix in
 // init mode; ring, VL row or dequantised K4V4 record in decode mode) by four
 // builder warps straight into the 128-byte-swizzled K-major operand layout.
@@ -65,7 +67,7 @@ struct SelGeo {
   int T, n, nq, qpos0, n_packed, n_vl;
 };
 
-__device__ __forceinline__ SelGeo sel_geo(const SelArgs& a) {
+__device__ __forceinline__ SelGeo sel_geo(const SelArgs& a, int b) {
   SelGeo g;
   if (a.k_dense) {
     g.T = a.L;
@@ -73,10 +75,11 @@ __device__ __forceinline__ SelGeo sel_geo(const SelArgs& a) {
     g.n_packed = 0;
     g.n_vl = 0;
   } else {
-    g.T = a.c.state[HQ_STATE_T];
-    g.nq = min(a.c.state[HQ_STATE_NQ], HQ_QBUF);
-    g.n_packed = a.c.state[HQ_STATE_NPACKED];
-    g.n_vl = a.c.state[HQ_STATE_NVL];
+    const int32_t* st = state_row(a.c, b);
+    g.T = st[HQ_STATE_T];
+    g.nq = min(st[HQ_STATE_NQ], HQ_QBUF);
+    g.n_packed = st[HQ_STATE_NPACKED];
+    g.n_vl = st[HQ_STATE_NVL];
   }
   g.n = max(g.T - a.c.W, 0);
   g.qpos0 = g.T - g.nq;
@@ -214,7 +217,9 @@ __device__ __forceinline__ void prefetch_keys(const SelArgs& a, const SelGeo& g,
                                                   (g.n_packed + HQ_PAGE_POSITIONS - 1) / HQ_PAGE_POSITIONS);
   for (int pg = p0; pg < p1; pg += 8)  // K codes, K (scale, zero) words and the bitmap of 8 pages at a time
     for (int q = pg; q < min(pg + 8, p1); ++q) {
-      const uint8_t* page = c.pages + (static_cast<size_t>(bh) * (c.cap / HQ_PAGE_POSITIONS) + q) * HQ_PAGE_BYTES;
+      const long long idx = page_index(c, bh, q);   // a hint: entries outside the pool are skipped
+      if (idx < 0) continue;
+      const uint8_t* page = c.pages + static_cast<size_t>(idx) * HQ_PAGE_BYTES;
       prefetch_l2(page + HQ_PAGE_KCODES, 4096);
       prefetch_l2(page + HQ_PAGE_KSZ, 1024);
       prefetch_l2(page + HQ_PAGE_VLMASK, 16);
@@ -235,7 +240,8 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
   const int G = c.Hq / c.Hkv;
   const int Mp = a.Mp;
   const int NACC = Mp / 128;
-  const SelGeo g = sel_geo(a);
+  const SelGeo g = sel_geo(a, b);
+  int32_t* const srow = state_row(c, b);
   const int M = G * g.nq;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -335,8 +341,8 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
       bool ok = true;
       for (int t = 0; t < nt && ok; ++t) {
         const int s = t & 1, buf = t % NBUF;
-        ok = sel_wait(&kfull[s], (t >> 1) & 1, c.state, &abort_flag);
-        if (ok && t >= NBUF) ok = sel_wait(&tfree[buf], ((t / NBUF) - 1) & 1, c.state, &abort_flag);
+        ok = sel_wait(&kfull[s], (t >> 1) & 1, srow, &abort_flag);
+        if (ok && t >= NBUF) ok = sel_wait(&tfree[buf], ((t / NBUF) - 1) & 1, srow, &abort_flag);
         if (!ok) break;
         tc_fence_after();
         const uint32_t kst = k_s + s * KSTAGE;
@@ -370,7 +376,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
       // every MMA issued completes before TMEM is released
       umma_commit(&drain);
       int dummy = 0;
-      sel_wait(&drain, 0, c.state, &dummy);
+      sel_wait(&drain, 0, srow, &dummy);
     }
     __syncwarp();
   } else if (warp >= EPI_WARPS) {
@@ -382,7 +388,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
     for (int t = 0; t < nt; ++t) {
       const int s = t & 1;
       const KeyRow nxt = t + 1 < nt ? fetch_key_row(a, g, bh, (k_lo + t + 1) * KT + r) : cur;
-      if (t >= 2 && !__all_sync(0xffffffffu, sel_wait(&kfree[s], ((t >> 1) - 1) & 1, c.state, &abort_flag))) break;
+      if (t >= 2 && !__all_sync(0xffffffffu, sel_wait(&kfree[s], ((t >> 1) - 1) & 1, srow, &abort_flag))) break;
       store_key_row(a, bh, cur, ks + s * KSTAGE, r);
       cp_async_wait_all();
       fence_proxy_async_smem();
@@ -412,7 +418,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
       for (int i = 0; i < 4; ++i) { m_run[i] = -INFINITY; l_run[i] = 0.f; }
       for (int t = 0; t < nt; ++t) {
         const int buf = t % NBUF;
-        if (!__all_sync(0xffffffffu, sel_wait(&tfull[buf], (t / NBUF) & 1, c.state, &abort_flag))) break;
+        if (!__all_sync(0xffffffffu, sel_wait(&tfull[buf], (t / NBUF) & 1, srow, &abort_flag))) break;
         tc_fence_after();
         const int j0 = (k_lo + t) * KT + 64 * hc;
 #pragma unroll
@@ -482,7 +488,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
       const int half = Mp / 2;
       for (int t = 0; t < nt; ++t) {
         const int buf = t % NBUF;
-        if (!__all_sync(0xffffffffu, sel_wait(&tfull[buf], (t / NBUF) & 1, c.state, &abort_flag))) break;
+        if (!__all_sync(0xffffffffu, sel_wait(&tfull[buf], (t / NBUF) & 1, srow, &abort_flag))) break;
         tc_fence_after();
         const int j = (k_lo + t) * KT + qd * 32 + lane;
         // queries that may not see key j: positions < j (only near the end)
@@ -518,7 +524,12 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
         if (hc == 1) xch[qd * 32 + lane] = sum;
         asm volatile("bar.sync 1, %0;" ::"r"(EPI_WARPS * 32) : "memory");
         if (hc == 0 && j < g.n) {
-          const float sc_j = sum + xch[qd * 32 + lane];
+          float sc_j = sum + xch[qd * 32 + lane];
+          if (c.score_acc) {  // running scores: decode mode adds to the stored sum, init mode starts it
+            float* acc = c.score_acc + static_cast<size_t>(bh) * c.cap + j;
+            if (!a.k_dense) sc_j += *acc;
+            *acc = sc_j;
+          }
           a.scores[static_cast<size_t>(bh) * c.cap + j] = sc_j;
           atomicAdd(shist + (__float_as_uint(sc_j) >> 20), 1u);
         }
@@ -565,7 +576,9 @@ __device__ __forceinline__ unsigned int tk_block_sum(unsigned int v, unsigned in
 __global__ void __launch_bounds__(TK_THREADS) topk_kernel(SelArgs a, int smem_scores) {
   const hq_cache& c = a.c;
   const int bh = blockIdx.x;
-  const SelGeo g = sel_geo(a);
+  const int b = bh / c.Hkv;
+  int32_t* const srow = state_row(c, b);
+  const SelGeo g = sel_geo(a, b);
   const int n = g.n;
   int k = 0;
   if (n > 0 && c.rho_bp > 0) {
@@ -573,10 +586,10 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(SelArgs a, int smem_sc
     k = static_cast<int>(min(static_cast<long long>(n), kk));
   }
   if (k > c.vl_cap) {
-    if (bh == 0 && threadIdx.x == 0) set_err(c.state, HQ_DEVERR_VL_CAPACITY);
+    if (bh % c.Hkv == 0 && threadIdx.x == 0) set_err(srow, HQ_DEVERR_VL_CAPACITY);
     k = c.vl_cap;
   }
-  if (bh == 0 && threadIdx.x == 0) c.state[HQ_STATE_KSEL] = k;
+  if (bh % c.Hkv == 0 && threadIdx.x == 0) srow[HQ_STATE_KSEL] = k;
   if (k == 0) return;
   extern __shared__ uint32_t tk_smem[];  // [TK_CAND_MAX] bin values, then [smem_scores] scores
   __shared__ unsigned int red[32];
@@ -756,6 +769,9 @@ hq_status launch_select(const hq_cache& c, const uint16_t* kd, int L, const uint
     return e;
   });
   if (ea != cudaSuccess) return cuda_fail(ea, "select setup");
+  if (kd != nullptr && c.score_acc != nullptr &&
+      cudaMemsetAsync(c.score_acc, 0, static_cast<size_t>(c.B) * c.Hkv * c.cap * sizeof(float), st) != cudaSuccess)
+    return cuda_fail(cudaGetLastError(), "select setup");
   dim3 grid(S, c.Hkv, c.B);
   sel_pass<false><<<grid, SEL_THREADS, smem, st>>>(a);
   sel_pass<true><<<grid, SEL_THREADS, smem, st>>>(a);

@@ -26,7 +26,7 @@ PAGE_KCODES, PAGE_VCODES, PAGE_KSZ, PAGE_VSZ, PAGE_VLMASK = 0, 4096, 8192, 9216,
 STATE_T, STATE_NPACKED, STATE_NVL, STATE_NQ, STATE_KSEL, STATE_ERR = range(6)
 STATE_WORDS = 8
 OP_SELECT, OP_MERGE, OP_DECODE = 0, 1, 2
-DEVERR_STAGING_FULL, DEVERR_CAPACITY, DEVERR_VL_CAPACITY, DEVERR_TIMEOUT = 1, 2, 4, 8
+DEVERR_STAGING_FULL, DEVERR_CAPACITY, DEVERR_VL_CAPACITY, DEVERR_TIMEOUT, DEVERR_PAGE = 1, 2, 4, 8, 16
 
 
 class HqError(RuntimeError):
@@ -41,8 +41,8 @@ _lib = ctypes.CDLL(LIB_PATH)
 class HqCacheStruct(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("B", "Hq", "Hkv", "D", "W", "rho_bp", "cap", "vl_cap")] + [
         (n, ctypes.c_void_p)
-        for n in ("pages", "kf", "vf", "vl_pos", "kr", "vr", "qbuf", "vl_sel", "state")
-    ]
+        for n in ("pages", "kf", "vf", "vl_pos", "kr", "vr", "qbuf", "vl_sel", "state", "page_table", "score_acc")
+    ] + [("n_pages", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 _P = ctypes.c_void_p
@@ -116,18 +116,35 @@ def abi_version() -> int:
 
 
 class HybridCache:
-    """Device buffers of one layer's hybrid cache (layout: include/hq.h, struct hq_cache)."""
+    """Device buffers of one layer's hybrid cache (layout: include/hq.h, struct hq_cache).
+
+    ``paged=True`` keeps the K4V4 store as a pool of ``n_pages`` pages (default:
+    exactly the pages the batch can use) with a page table ``[B, Hkv, cap/64]``;
+    ``page_order`` (optional, a permutation of the pool indices) fills the table,
+    else page j of (b, h) is pool page (b*Hkv + h)*(cap/64) + j."""
 
     def __init__(self, B: int, Hq: int, Hkv: int, cap: int, W: int = 128, rho_bp: int = 500, vl_cap: int = None,
-                 device="cuda", D: int = HQ_HEAD_DIM):
+                 device="cuda", D: int = HQ_HEAD_DIM, paged: bool = False, n_pages: int = None, page_order=None,
+                 running_scores: bool = False):
         cap = ((cap + 127) // 128) * 128
         if vl_cap is None:
             vl_cap = max(16, ((k_of(max(cap - W, 0), rho_bp) + 15) // 16) * 16)
         self.B, self.Hq, self.Hkv, self.D, self.W, self.rho_bp, self.cap, self.vl_cap = B, Hq, Hkv, D, W, rho_bp, cap, vl_cap
         self.R = ((W + HQ_STAGE + 15) // 16) * 16   # HQ_RING_LEN(W)
+        self.npg = cap // PAGE_POSITIONS
         dev = torch.device(device)
         z = lambda shape, dt: torch.zeros(shape, dtype=dt, device=dev)
-        self.pages = z((B, Hkv, cap // PAGE_POSITIONS, PAGE_BYTES), torch.uint8)
+        self.paged = paged
+        if paged:
+            self.n_pages = n_pages if n_pages is not None else B * Hkv * self.npg
+            self.pages = z((self.n_pages, PAGE_BYTES), torch.uint8)
+            order = torch.arange(B * Hkv * self.npg, dtype=torch.int32) if page_order is None else \
+                torch.as_tensor(page_order, dtype=torch.int32)
+            self.page_table = order.reshape(B, Hkv, self.npg).to(dev).contiguous()
+        else:
+            self.n_pages = 0
+            self.pages = z((B, Hkv, self.npg, PAGE_BYTES), torch.uint8)
+            self.page_table = None
         self.kf = z((B, Hkv, vl_cap, D), torch.float16)
         self.vf = z((B, Hkv, vl_cap, D), torch.float16)
         self.vl_pos = z((B, Hkv, vl_cap), torch.int32)
@@ -135,11 +152,18 @@ class HybridCache:
         self.vr = z((B, Hkv, self.R, D), torch.float16)
         self.qbuf = z((B, Hq, HQ_QBUF, D), torch.float16)
         self.vl_sel = z((B, Hkv, vl_cap), torch.int32)
-        self.state_t = z((STATE_WORDS,), torch.int32)
+        self.state_t = z((B, STATE_WORDS), torch.int32)
+        self.score_acc = z((B, Hkv, cap), torch.float32) if running_scores else None
         self.c = HqCacheStruct(B, Hq, Hkv, D, W, rho_bp, cap, vl_cap, *[t.data_ptr() for t in (
-            self.pages, self.kf, self.vf, self.vl_pos, self.kr, self.vr, self.qbuf, self.vl_sel, self.state_t)])
+            self.pages, self.kf, self.vf, self.vl_pos, self.kr, self.vr, self.qbuf, self.vl_sel, self.state_t)],
+            self.page_table.data_ptr() if paged else None,
+            self.score_acc.data_ptr() if running_scores else None, self.n_pages, 0)
         _check(_lib.hq_cache_validate(ctypes.byref(self.c)), "hq_cache_validate")
         self._ws = {}
+
+    def slot(self, b: int) -> "CacheSlot":
+        """Single-sequence view of batch row b (a B = 1 descriptor into the same buffers)."""
+        return CacheSlot(self, b)
 
     def workspace(self, op: int, L: int = 0) -> torch.Tensor:
         n = int(_lib.hq_workspace_bytes(ctypes.byref(self.c), op, L))
@@ -151,19 +175,47 @@ class HybridCache:
             self._ws[op] = w
         return w
 
-    def state(self) -> dict:
-        s = self.state_t.tolist()
-        return {"T": s[STATE_T], "n_packed": s[STATE_NPACKED], "n_vl": s[STATE_NVL], "n_q": s[STATE_NQ],
-                "k_sel": s[STATE_KSEL], "err": s[STATE_ERR]}
+    def states(self) -> list:
+        """Every sequence's state row as a dict."""
+        rows = self.state_t.cpu().tolist()
+        return [{"T": s[STATE_T], "n_packed": s[STATE_NPACKED], "n_vl": s[STATE_NVL], "n_q": s[STATE_NQ],
+                 "k_sel": s[STATE_KSEL], "err": s[STATE_ERR]} for s in rows]
+
+    def state(self, b: int = None) -> dict:
+        """State row b; with b omitted, the rows must agree (a uniform batch) and
+        the common row is returned, with the error bits of all rows OR-ed."""
+        rows = self.states()
+        if b is not None:
+            return rows[b]
+        out = dict(rows[0])
+        err = 0
+        for r in rows:
+            err |= r["err"]
+            for k in ("T", "n_packed", "n_vl", "n_q", "k_sel"):
+                if r[k] != out[k]:
+                    raise HqError(f"state rows differ ({k}): use state(b) or states() for a ragged batch")
+        out["err"] = err
+        return out
 
     def nbytes(self) -> int:
-        return sum(t.numel() * t.element_size() for t in (self.pages, self.kf, self.vf, self.vl_pos, self.kr, self.vr,
-                                                          self.qbuf, self.vl_sel, self.state_t))
+        ts = [self.pages, self.kf, self.vf, self.vl_pos, self.kr, self.vr, self.qbuf, self.vl_sel, self.state_t]
+        for t in (self.page_table, self.score_acc):
+            if t is not None:
+                ts.append(t)
+        return sum(t.numel() * t.element_size() for t in ts)
+
+    def page_bytes(self) -> np.ndarray:
+        """The K4V4 pages of every (b, h) in position order: uint8 [B, Hkv, cap/64, PAGE_BYTES] (host copy)."""
+        pg = self.pages.cpu().numpy()
+        if not self.paged:
+            return pg
+        tab = self.page_table.cpu().numpy().astype(np.int64)
+        return pg[np.clip(tab, 0, self.n_pages - 1)]
 
     def packed(self) -> dict:
         """The K4V4 store by position (host copies): codes kq/vq uint8 [B,Hkv,cap,D/2],
         scale/zero words ksz/vsz uint32 [B,Hkv,cap,D/32], VL bitmap vl_bits bool [B,Hkv,cap]."""
-        pg = self.pages.cpu().numpy()
+        pg = self.page_bytes()
         B, H, npg, _ = pg.shape
         D = self.D
         take = lambda off, width: pg[..., off:off + 64 * width].reshape(B, H, npg * 64, width)
@@ -172,6 +224,37 @@ class HybridCache:
         return {"kq": take(PAGE_KCODES, D // 2), "vq": take(PAGE_VCODES, D // 2),
                 "ksz": take(PAGE_KSZ, 16).copy().view(np.uint32), "vsz": take(PAGE_VSZ, 16).copy().view(np.uint32),
                 "vl_bits": bits}
+
+
+class CacheSlot:
+    """One sequence of a HybridCache as a B = 1 cache: the descriptor's pointers
+    are offset to batch row b (the page pool, when paged, is shared; the page
+    table row is b's).  Accepted by every entry point of this module."""
+
+    def __init__(self, parent: HybridCache, b: int):
+        if not 0 <= b < parent.B:
+            raise HqError(f"slot {b} outside the batch of {parent.B}")
+        self.parent, self.b = parent, b
+        self.B, self.Hq, self.Hkv, self.D, self.W = 1, parent.Hq, parent.Hkv, parent.D, parent.W
+        self.rho_bp, self.cap, self.vl_cap, self.R = parent.rho_bp, parent.cap, parent.vl_cap, parent.R
+        sl = lambda t: t[b:b + 1]
+        self.kf, self.vf, self.vl_pos = sl(parent.kf), sl(parent.vf), sl(parent.vl_pos)
+        self.kr, self.vr, self.qbuf, self.vl_sel = sl(parent.kr), sl(parent.vr), sl(parent.qbuf), sl(parent.vl_sel)
+        self.state_t = sl(parent.state_t)
+        self.pages = parent.pages if parent.paged else sl(parent.pages)
+        self.page_table = sl(parent.page_table) if parent.paged else None
+        self.score_acc = sl(parent.score_acc) if parent.score_acc is not None else None
+        self.c = HqCacheStruct(1, self.Hq, self.Hkv, self.D, self.W, self.rho_bp, self.cap, self.vl_cap, *[
+            t.data_ptr() for t in (self.pages, self.kf, self.vf, self.vl_pos, self.kr, self.vr, self.qbuf, self.vl_sel,
+                                   self.state_t)], self.page_table.data_ptr() if parent.paged else None,
+            self.score_acc.data_ptr() if self.score_acc is not None else None, parent.n_pages, 0)
+        _check(_lib.hq_cache_validate(ctypes.byref(self.c)), "hq_cache_validate (slot)")
+        self._ws = {}
+
+    workspace = HybridCache.workspace
+
+    def state(self, b: int = None) -> dict:
+        return self.parent.state(self.b)
 
 
 # ----------------------------------------------------------------------------- entry points

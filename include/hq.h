@@ -39,9 +39,15 @@
  *     before anything is launched; on a non-HQ_OK status nothing was launched.
  *   - Conditions that depend on device-resident lengths (a full staging area,
  *     an exhausted capacity) cannot be seen by the host: the kernels skip their
- *     work and OR a HQ_DEVERR_* bit into state[HQ_STATE_ERR]; read it after
- *     synchronising.  No kernel traps or spins without a bound.
- *   - Batches are uniform-length: every (batch, head) has the same length T.
+ *     work and OR a HQ_DEVERR_* bit into state[b][HQ_STATE_ERR] of the sequence
+ *     concerned; read it after synchronising.  No kernel traps or spins
+ *     without a bound.
+ *   - Sequences are independent: each batch row b has its own lengths (a row
+ *     of the state array), so one call serves a batch of sequences of
+ *     different lengths.  The K4V4 store may be paged (page_table), so that the
+ *     pages of a sequence need not be contiguous.  A single sequence is
+ *     addressed by a descriptor whose pointers are offset to its row (B = 1),
+ *     e.g. to install its prefix while the others keep decoding.
  */
 #ifndef HQ_H
 #define HQ_H
@@ -88,13 +94,16 @@ typedef enum hq_status {
   HQ_ERR_CUDA = 5          /* a CUDA runtime call or launch failed */
 } hq_status;
 
-/* device-side error bits, OR-ed into state[HQ_STATE_ERR] */
+/* device-side error bits, OR-ed into state[b][HQ_STATE_ERR] */
 #define HQ_DEVERR_STAGING_FULL 0x1u  /* decode with HQ_STAGE tokens staged: select + merge first */
 #define HQ_DEVERR_CAPACITY 0x2u      /* T would exceed cap */
 #define HQ_DEVERR_VL_CAPACITY 0x4u   /* k = ceil(rho * n) exceeds vl_cap (clamped) */
 #define HQ_DEVERR_TIMEOUT 0x8u       /* a bounded wait gave up (never expected) */
+#define HQ_DEVERR_PAGE 0x10u         /* a page-table entry outside [0, n_pages): pool page 0 was read
+                                        instead (the outputs of that sequence are unspecified) and
+                                        nothing was written through the entry */
 
-/* words of the device-resident state vector (int32[HQ_STATE_WORDS]) */
+/* words of one sequence's row of the device-resident state (int32[B][HQ_STATE_WORDS]) */
 enum {
   HQ_STATE_T = 0,         /* current length: positions 0 .. T-1 are cached */
   HQ_STATE_NPACKED = 1,   /* positions 0 .. n_packed-1 have a K4V4 record */
@@ -110,7 +119,8 @@ enum {
  * device memory laid out as stated ([..] = row-major shape, innermost last).
  * R = HQ_RING_LEN(W) is the FP16 ring length (W + HQ_STAGE rounded up to 16).
  *
- *   pages     uint8  [B, Hkv, cap/64, HQ_PAGE_BYTES]  the K4V4 store, one page per 64
+ *   pages     uint8  [B, Hkv, cap/64, HQ_PAGE_BYTES]  (page_table == NULL) or a page pool
+ *             uint8  [n_pages, HQ_PAGE_BYTES] (page_table != NULL): the K4V4 store, one page per 64
  *             positions (layout HQ_PAGE_*): codes of both K and V, their per-group
  *             (scale, zero) words and the VL bitmap of the page's positions, so
  *             that one contiguous copy brings a whole page on chip, and the VL-store
@@ -121,11 +131,21 @@ enum {
  *   kr, vr    fp16   [B, Hkv, R, D]       recent window + staging; position p at slot p % R
  *   qbuf      fp16   [B, Hq, HQ_QBUF, D]  buffered decode queries; position p at slot p % HQ_QBUF
  *   vl_sel    int32  [B, Hkv, vl_cap]     output of hq_select_vlines, input of hq_pack_merge
- *   state     int32  [HQ_STATE_WORDS]     device-resident lengths (see HQ_STATE_*)
+ *   state     int32  [B, HQ_STATE_WORDS]  device-resident lengths of each sequence (HQ_STATE_*)
+ *   page_table int32 [B, Hkv, cap/64]    optional (NULL: pages is the dense [B, Hkv, cap/64, ..]
+ *             array): entry (b, h, j) is the pool page holding positions 64 j .. 64 j + 63
+ *             of sequence b, kv head h; 4-byte aligned; entries of pages no position
+ *             reaches are not read.  Pages of different (b, h) must be distinct.
+ *   score_acc float [B, Hkv, cap]        optional running column-mass scores (NULL: each
+ *             reselection ranks its own column mass).  When set, the prefix selection
+ *             (init mode) stores its column mass there (zero past the scored prefix) and
+ *             every decode-mode reselection adds its column mass to it and ranks the sums
+ *             (README Overview item 1, "running column-mass score").
  *
  * Limits checked by hq_cache_validate(): D == 128; Hq % Hkv == 0 and
  * Hq / Hkv <= HQ_MAX_GQA; W >= 0; 0 <= rho_bp <= 10000; cap a positive
- * multiple of 128; vl_cap a positive multiple of 16.
+ * multiple of 128; vl_cap a positive multiple of 16; with a page table,
+ * n_pages >= 1.
  * Fields W and rho_bp fix the method's window and VL ratio (basis points:
  * 500 = 5 %).  The fp16 positions in [n_packed, T) live in the ring, VL rows
  * in kf/vf, every other position < n_packed is read from its K4V4 record.
@@ -142,6 +162,10 @@ typedef struct hq_cache {
   uint16_t* qbuf;
   int32_t* vl_sel;
   int32_t* state;
+  int32_t* page_table;
+  float* score_acc;
+  int32_t n_pages;
+  int32_t reserved;   /* 0 */
 } hq_cache;
 
 /* Operation codes for hq_workspace_bytes. */
@@ -168,7 +192,9 @@ HQ_API hq_status hq_cache_validate(const hq_cache* c);
 HQ_API size_t hq_workspace_bytes(const hq_cache* c, int32_t op, int32_t L);
 
 /*
- * Reset the cache to empty: state words to 0 and the VL bitmap of every page cleared.
+ * Reset every sequence of the descriptor to empty: its state row to 0, the
+ * VL bitmap of each of its pages (through the page table, if any) cleared and
+ * its running scores (score_acc, if any) zeroed.
  */
 HQ_API hq_status hq_cache_reset(const hq_cache* c, hq_stream_t stream);
 
@@ -180,7 +206,7 @@ HQ_API hq_status hq_cache_reset(const hq_cache* c, hq_stream_t stream);
  * for j in the non-window prefix [0, n), n = T - W, sm_scale = 1/sqrt(D);
  * then the k = ceil(n * rho_bp / 10000) largest scores (ties -> lower
  * position) are written to c->vl_sel in ascending position order and k to
- * state[HQ_STATE_KSEL].
+ * state[b][HQ_STATE_KSEL]; every sequence b uses its own T, n and k.
  *
  * Init mode (k_dense != NULL): keys are the dense FP16 prefix
  *   k_dense [B, Hkv, L, D], T = L; queries q_ext [B, Hq, nq, D] sit at
@@ -203,13 +229,16 @@ HQ_API hq_status hq_select_vlines(const hq_cache* c, const uint16_t* k_dense, in
  * Init mode (k_dense, v_dense != NULL, both [B, Hkv, L, D] FP16): install a
  *   prefix of L tokens: positions [0, L-W) get their K4V4 records, the last
  *   min(W, L) positions go to the ring, the VL store is filled from c->vl_sel
- *   (state[HQ_STATE_KSEL] entries, FP16 rows taken from the dense prefix);
- *   state becomes T = L, n_packed = max(L-W, 0), n_q = 0.  Requires L <= cap.
+ *   (state[b][HQ_STATE_KSEL] entries, FP16 rows taken from the dense prefix);
+ *   every row b of state becomes T = L, n_packed = max(L-W, 0), n_q = 0.
+ *   Requires L <= cap.  Sequences of different prefix lengths are installed
+ *   one at a time through single-sequence descriptors.
  * Merge mode (both NULL): positions [n_packed, T-W) leave the window and get
  *   their K4V4 records; the VL store is rebuilt from c->vl_sel: a row keeps the
  *   position's current FP16 value when it has one (old VL row or ring),
  *   otherwise it is the dequantised record rounded once to FP16; n_packed
- *   becomes max(n_packed, T-W).  Records are never rewritten.
+ *   becomes max(n_packed, T-W).  Records are never rewritten.  Each sequence
+ *   uses its own lengths.
  */
 HQ_API hq_status hq_pack_merge(const hq_cache* c, const uint16_t* k_dense, const uint16_t* v_dense,
                         int32_t L, void* ws, size_t ws_bytes, hq_stream_t stream);
@@ -221,9 +250,14 @@ HQ_API hq_status hq_pack_merge(const hq_cache* c, const uint16_t* k_dense, const
  *     out[b, h] = softmax(q[b,h] . K^T * sm_scale) V
  * over all T+1 positions, each key/value in its stored representation
  * (dequantisation fused into the scan; split-K over the sequence with a
- * log-sum-exp merge).  out: fp16 [B, Hq, D].  Increments T.
- * If HQ_STAGE tokens are already staged (T - n_packed == W + HQ_STAGE) or
- * T == cap, nothing is written and HQ_DEVERR_STAGING_FULL / _CAPACITY is set.
+ * log-sum-exp merge).  out: fp16 [B, Hq, D].  Increments T.  Every sequence
+ * b attends over its own T_b + 1 positions.
+ * If HQ_STAGE tokens of sequence b are already staged (T - n_packed == W +
+ * HQ_STAGE) or T == cap, nothing of that sequence is written (its out rows
+ * included) and HQ_DEVERR_STAGING_FULL / _CAPACITY is set in its state row;
+ * the other sequences proceed.  B * Hkv <= 2048 (else HQ_ERR_UNSUPPORTED).
+ * After a HQ_DEVERR_TIMEOUT the workspace's counters may not be zero: zero
+ * the workspace again before the next call.
  */
 HQ_API hq_status hq_decode_attn(const hq_cache* c, const uint16_t* q, const uint16_t* k_new,
                          const uint16_t* v_new, uint16_t* out, float sm_scale,

@@ -76,12 +76,13 @@ def check_selection(gpu_scores: np.ndarray, gpu_sel: np.ndarray, ref_scores: np.
 class Pair:
     """A GPU cache and the oracle cache, kept on the same VL sets."""
 
-    def __init__(self, B, Hq, Hkv, L, W, rho_bp, cap, seed=0, n_tail=64):
+    def __init__(self, B, Hq, Hkv, L, W, rho_bp, cap, seed=0, n_tail=64, running=False):
         self.lay = __import__("hybrid_precision_attention_b200.synth", fromlist=["x"]).planted_layer(seed, B, Hq, Hkv, L, n_tail=n_tail)
         self.B, self.Hq, self.Hkv, self.L, self.W, self.rho = B, Hq, Hkv, L, W, rho_bp
+        self.running = running
         H = hq()
-        self.g = H.HybridCache(B, Hq, Hkv, cap, W, rho_bp)
-        self.r = hybrid.HybridCacheRef(B, Hq, Hkv, W, rho_bp, self.g.cap)
+        self.g = H.HybridCache(B, Hq, Hkv, cap, W, rho_bp, running_scores=running)
+        self.r = hybrid.HybridCacheRef(B, Hq, Hkv, W, rho_bp, self.g.cap, accumulate=running)
 
     def init(self, check=True):
         H = hq()
@@ -107,6 +108,8 @@ class Pair:
                     ref = osel.column_mass(self.lay.k[b, h].astype(np.float64), qs, qpos, n, 1 / np.sqrt(128))
                     check_selection(gsc[b, h], vl[b][h], ref, kk, f"init b{b} h{h}")
         self.r.install_prefix(self.lay.k, self.lay.v, vl)
+        if self.running:
+            self.r.start_running_scores(self.lay.k, self.lay.q_tail)
         if check:
             self.check_state()
         return vl
@@ -157,9 +160,10 @@ class Pair:
         assert st["k_sel"] == kk, (st, kk)
         sel = self.g.vl_sel.cpu().numpy()
         vl = [[sel[b, h, :kk].astype(np.int64) for h in range(self.Hkv)] for b in range(self.B)]
-        if check:
+        if check or self.running:   # running scores: the oracle's sums must follow every reselection
             _, ref_scores = self.r.reselect()
             gsc = scores.cpu().numpy()
+        if check:
             for b in range(self.B):
                 for h in range(self.Hkv):
                     check_selection(gsc[b, h], vl[b][h], ref_scores[b][h], kk, f"reselect b{b} h{h}")

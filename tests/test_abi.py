@@ -50,5 +50,13 @@ def test_host_validation_without_gpu():
         bad = HqCacheStruct.from_buffer_copy(good)
         setattr(bad, field, val)
         assert lib.hq_cache_validate(ctypes.byref(bad)) == want, field
+    # the optional page table (4-byte aligned, a non-empty pool) and running scores (16-byte aligned)
+    for fields, want in (({"page_table": base + 4, "n_pages": 3}, 0), ({"page_table": base + 2, "n_pages": 3}, 1),
+                         ({"page_table": base, "n_pages": 0}, 1), ({"score_acc": base + 16}, 0),
+                         ({"score_acc": base + 8}, 1)):
+        opt = HqCacheStruct.from_buffer_copy(good)
+        for k, v in fields.items():
+            setattr(opt, k, v)
+        assert lib.hq_cache_validate(ctypes.byref(opt)) == want, fields
     lib.hq_workspace_bytes.restype = ctypes.c_size_t
     assert lib.hq_workspace_bytes(ctypes.byref(good), 1, 0) > 0

@@ -50,7 +50,7 @@ def test_decode_loop_with_reselection():
         st = p.g.state()
         assert st["err"] & H.DEVERR_STAGING_FULL and st["T"] == L + t
         assert torch.all(sentinel == 7.0)
-        p.g.state_t[H.STATE_ERR] = 0
+        p.g.state_t[:, H.STATE_ERR] = 0
         p.reselect_merge()
         assert p.g.state()["n_packed"] == L + t - W
     for _ in range(3):
@@ -132,3 +132,39 @@ def test_full_size_32k_layer():
     p.reselect_merge()
     out, ref = p.decode(q[64], k[64], v[64])
     check_decode(out, ref, "after merge")
+
+
+def test_running_scores_over_three_periods():
+    """Running (accumulated) column-mass scores: each reselection adds its
+    column mass to the stored sums and ranks the sums; scores and selections
+    against the oracle's running scores over three 64-token periods (the
+    1K layer, B=2), decode checked after every merge."""
+    B, Hq, Hkv, L, W = 2, 32, 8, 1024, 128
+    p = Pair(B, Hq, Hkv, L, W, 500, cap=L + 4 * 64 + 64, seed=13, running=True)
+    p.init()
+    acc0 = p.g.score_acc.cpu().numpy()
+    n0 = L - W
+    for b in range(B):
+        for h in range(Hkv):
+            want = p.r.acc[b, h, :n0]
+            assert np.allclose(acc0[b, h, :n0], want, rtol=5e-4, atol=0), (b, h)
+            assert not acc0[b, h, n0:].any()
+    q, k, v = synth.decode_tokens(13, B, Hq, Hkv, 3 * 64 + 1)
+    t = 0
+    for period in range(3):
+        for i in range(64):   # the first step of a period follows a merge
+            if i % 16 == 0:
+                out, ref = p.decode(q[t], k[t], v[t])
+                check_decode(out, ref, f"step {t}")
+            else:
+                hq().hq_decode_attn(p.g, dev(q[t]), dev(k[t]), dev(v[t]))
+                p.r.append(q[t], k[t], v[t])
+            t += 1
+        p.reselect_merge()
+        acc = p.g.score_acc.cpu().numpy()
+        n = p.r.T - W
+        for b in range(B):
+            for h in range(Hkv):
+                assert np.allclose(acc[b, h, :n], p.r.acc[b, h, :n], rtol=5e-4, atol=0), (period, b, h)
+    out, ref = p.decode(q[t], k[t], v[t])
+    check_decode(out, ref, "after the last merge")
