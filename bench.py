@@ -394,8 +394,8 @@ def run_ours(args, rank, world, local_rank):
 
     # our kernels per step: one decode_kernel per token and copy; per copy a
     # reselection (sel_pass<0>, sel_pass<1>, topk_kernel) and a staging merge
-    # (pack_rows_kernel, vl_gather_kernel, vl_install_kernel)
-    launches_per_step = PERIOD * COPIES + COPIES * (3 + 3)
+    # (pack_rows_kernel, vl_gather_kernel, vl_clear_kernel, vl_install_kernel)
+    launches_per_step = PERIOD * COPIES + COPIES * (3 + 4)
 
     def step(ev=None):
         if ev is not None:

@@ -124,35 +124,6 @@ __device__ __forceinline__ int fp16_before(const UnitGeo& g, int k) {
   return static_cast<int>((static_cast<long long>(k) * g.NF) / g.NT);
 }
 
-// Walks a unit's tiles k, k + stride, k + 2 stride, ... keeping f = fp16_before(k)
-// and the remainder of k NF / NT, so each step needs no division: tile k is an
-// FP16 tile iff the remainder plus NF reaches NT.
-struct TileWalk {
-  int k, f, rem, qd, rd, NF, NT;
-  __device__ __forceinline__ void start(const UnitGeo& g, int k0, int stride) {
-    NF = g.NF;
-    NT = g.NT;
-    k = k0;
-    const long long x = static_cast<long long>(k0) * NF;
-    f = static_cast<int>(x / NT);
-    rem = static_cast<int>(x - static_cast<long long>(f) * NT);
-    const long long y = static_cast<long long>(stride) * NF;
-    qd = static_cast<int>(y / NT);
-    rd = static_cast<int>(y - static_cast<long long>(qd) * NT);
-  }
-  // the packed tile index (>= 0), or -(FP16 tile index) - 1
-  __device__ __forceinline__ int tile() const { return rem + NF >= NT ? -f - 1 : k - f; }
-  __device__ __forceinline__ void step(int stride) {
-    k += stride;
-    f += qd;
-    rem += rd;
-    if (rem >= NT) {
-      rem -= NT;
-      ++f;
-    }
-  }
-};
-
 // 16-bit mask of the valid rows of FP16 tile j (VL tiles, then ring tiles, then the new token)
 __device__ __forceinline__ uint32_t fp16_valid(const UnitGeo& g, int j, int R) {
   if (j < g.NV) {
@@ -173,26 +144,50 @@ __device__ __forceinline__ uint32_t fp16_valid(const UnitGeo& g, int j, int R) {
   return m;
 }
 
-// A CTA's share of one unit: CTA-local tiles [a, b) are the unit's tiles k0 .. k0 + b - a - 1.
+// A CTA's share of one unit: CTA-local tiles [a, b) are the unit's tiles
+// k0 .. k0 + b - a - 1 of the interleaved list, which the CTA runs packed ones
+// first (pages p0 .. p0 + npk - 1), then FP16 ones (f0 ..): a warp that gets
+// one tile more than the others then gets a cheap FP16 tile.
 struct Seg {
-  int u, a, b, k0, first_cta, ncta;
+  int u, a, b, k0, p0, npk, f0, first_cta, ncta;
 };
+
+// CTA-local tile i of segment sg: the packed tile index (>= 0), or -(FP16 tile index) - 1.
+__device__ __forceinline__ int seg_tile(const Seg& sg, int i) {
+  const int j = i - sg.a;
+  return j < sg.npk ? sg.p0 + j : -(sg.f0 + j - sg.npk) - 1;
+}
 
 // The CTA's range and segments (shared memory), built by all NTHREADS threads.
 struct Plan {
-  int nseg, ntile, ceff;
+  int nseg, ntile, u0;
+  long long X, Wt, w0, w1;
+  int ceff;
   Seg seg[MAXSEG];
 };
+
+__device__ __forceinline__ void read_len(const hq_cache& c, int b, bool stale, int& T, int& np, int& nv) {
+  const int32_t* st = state_row(c, b);
+  if (stale) {
+    T = *reinterpret_cast<volatile const int*>(st + HQ_STATE_T);
+    np = min(max(*reinterpret_cast<volatile const int*>(st + HQ_STATE_NPACKED), 0), c.cap);
+    nv = min(max(*reinterpret_cast<volatile const int*>(st + HQ_STATE_NVL), 0), c.vl_cap);
+  } else {
+    T = st[HQ_STATE_T];
+    np = st[HQ_STATE_NPACKED];
+    nv = st[HQ_STATE_NVL];
+  }
+}
 
 // Cut the batch's tile lists into ranges and record this CTA's segments.
 // `stale`: state read with volatile loads before the dependency wait (it may
 // be one step old; the plan then only steers prefetches).  `red` is scratch
-// for NTHREADS / 32 + 2 ints.
-__device__ void make_plan(const hq_cache& c, int R, Plan& p, int* red, bool stale) {
+// for NTHREADS / 32 ints.
+__device__ __noinline__ void make_plan(const hq_cache& c, int R, Plan& p, int* red, bool stale) {
   const int U = c.B * c.Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid < MAXSEG) p.seg[tid].u = -1;
-  // tile counts of this thread's units (refused sequences: none)
+  // tile counts of this thread's units (sequences that take no step: none)
   int nt[SCAN_PER];
   int sum = 0;
 #pragma unroll
@@ -200,19 +195,8 @@ __device__ void make_plan(const hq_cache& c, int R, Plan& p, int* red, bool stal
     const int u = tid * SCAN_PER + i;
     nt[i] = 0;
     if (u < U) {
-      const int32_t* st = state_row(c, u / c.Hkv);
       int T, np, nv;
-      if (stale) {
-        T = *reinterpret_cast<volatile const int*>(st + HQ_STATE_T);
-        np = *reinterpret_cast<volatile const int*>(st + HQ_STATE_NPACKED);
-        nv = *reinterpret_cast<volatile const int*>(st + HQ_STATE_NVL);
-        np = min(max(np, 0), c.cap);
-        nv = min(max(nv, 0), c.vl_cap);
-      } else {
-        T = st[HQ_STATE_T];
-        np = st[HQ_STATE_NPACKED];
-        nv = st[HQ_STATE_NVL];
-      }
+      read_len(c, u / c.Hkv, stale, T, np, nv);
       if (!refused(c, T, np)) nt[i] = unit_geo(np, nv, T, R).NT;
     }
     sum += nt[i];
@@ -227,7 +211,7 @@ __device__ void make_plan(const hq_cache& c, int R, Plan& p, int* red, bool stal
   if (lane == 31) red[warp] = x;
   if (tid == 0) {
     p.nseg = 0;
-    red[NTHREADS / 32] = -1;  // u0
+    p.u0 = -1;
   }
   __syncthreads();
   int before = 0, total = 0;
@@ -237,18 +221,24 @@ __device__ void make_plan(const hq_cache& c, int R, Plan& p, int* red, bool stal
     total += v;
   }
   const int excl = before + x - sum;  // tiles of all units before this thread's first unit
-  // phantom weight X per unit bounds the units a range can touch (at most
-  // N / (ceff X) + U / ceff + 2 <= 32 + 48 + 2 < MAXSEG); ceff CTAs share the work
-  const long long N = total;
-  // (at least U / 48 CTAs, so that with the phantom weight no range touches more than MAXSEG units)
-  const int ceff = static_cast<int>(min(static_cast<long long>(gridDim.x),
-                                        max(max(1ll, (N + MIN_TILES - 1) / MIN_TILES), static_cast<long long>((U + 47) / 48))));
-  const long long X = max(1ll, (N + static_cast<long long>(ceff) * PHANTOM_DIV - 1) / (static_cast<long long>(ceff) * PHANTOM_DIV));
-  const long long Wt = N + static_cast<long long>(U) * X;
-  const long long w0 = (static_cast<long long>(blockIdx.x) * Wt) / ceff;
-  const long long w1 = (static_cast<long long>(blockIdx.x + 1) * Wt) / ceff;
-  // CTA whose range holds weight position w
-  auto cta_of = [&](long long w) { return static_cast<int>(((w + 1) * ceff - 1) / Wt); };
+  if (tid == 0) {
+    // ceff CTAs share the work (at least U / 48 of them); a phantom weight X per
+    // unit bounds the units one range can touch by N / (ceff X) + U / ceff + 2
+    // <= 32 + 48 + 2 < MAXSEG
+    const long long N = total;
+    const long long ceff = min(static_cast<long long>(gridDim.x),
+                               max(max(1ll, (N + MIN_TILES - 1) / MIN_TILES), static_cast<long long>((U + 47) / 48)));
+    const long long X = max(1ll, (N + ceff * PHANTOM_DIV - 1) / (ceff * PHANTOM_DIV));
+    const long long Wt = N + static_cast<long long>(U) * X;
+    p.ceff = static_cast<int>(ceff);
+    p.X = X;
+    p.Wt = Wt;
+    p.w0 = (static_cast<long long>(blockIdx.x) * Wt) / ceff;
+    p.w1 = (static_cast<long long>(blockIdx.x + 1) * Wt) / ceff;
+  }
+  __syncthreads();
+  const long long X = p.X, Wt = p.Wt, w0 = p.w0, w1 = p.w1;
+  const int ceff = p.ceff;
   // the unit holding w0: unit u spans weights [S_u, S_u + X + NT_u), S_u = tiles before + u X
   int tb = excl;
 #pragma unroll
@@ -256,12 +246,12 @@ __device__ void make_plan(const hq_cache& c, int R, Plan& p, int* red, bool stal
     const int u = tid * SCAN_PER + i;
     if (u < U) {
       const long long S = tb + static_cast<long long>(u) * X;
-      if (S <= w0 && w0 < S + X + nt[i]) red[NTHREADS / 32] = u;
+      if (S <= w0 && w0 < S + X + nt[i]) p.u0 = u;
     }
     tb += nt[i];
   }
   __syncthreads();
-  const int u0 = red[NTHREADS / 32];
+  const int u0 = p.u0;
   // every unit of [u0, u0 + MAXSEG) that holds tiles of this CTA's range becomes a segment
   tb = excl;
 #pragma unroll
@@ -272,11 +262,18 @@ __device__ void make_plan(const hq_cache& c, int R, Plan& p, int* red, bool stal
       const long long lo = max(S, w0), hi = min(S + nt[i], w1);
       if (lo < hi) {
         if (u - u0 < MAXSEG) {
+          int T, np, nv;
+          read_len(c, u / c.Hkv, stale, T, np, nv);
+          const UnitGeo g = unit_geo(np, nv, T, R);
           Seg& s = p.seg[u - u0];
+          const int k0 = static_cast<int>(lo - S), k1 = static_cast<int>(hi - S);
           s.u = u;
-          s.k0 = static_cast<int>(lo - S);
-          s.a = static_cast<int>(lo - w0);  // weights of earlier units' phantoms are not tiles: fixed below
-          s.b = static_cast<int>(hi - lo);  // count for now
+          s.k0 = k0;
+          s.b = k1 - k0;  // a count for now; CTA-local positions are set below
+          s.f0 = fp16_before(g, k0);
+          s.p0 = k0 - s.f0;
+          s.npk = (k1 - fp16_before(g, k1)) - s.p0;
+          auto cta_of = [&](long long w) { return static_cast<int>(((w + 1) * ceff - 1) / Wt); };
           s.first_cta = cta_of(S);
           s.ncta = cta_of(S + nt[i] - 1) - s.first_cta + 1;
           atomicMax(&p.nseg, u - u0 + 1);
@@ -292,11 +289,9 @@ __device__ void make_plan(const hq_cache& c, int R, Plan& p, int* red, bool stal
     // CTA-local tile numbering: segments back to back, empty slots skipped
     int at = 0, k = 0;
     for (int i = 0; i < p.nseg; ++i) {
-      Seg& s = p.seg[i];
-      const bool used = s.u == u0 + i && s.b > 0;
-      if (!used) continue;
-      const int n = s.b;
-      Seg t = s;
+      Seg t = p.seg[i];
+      if (t.u != u0 + i || t.b <= 0) continue;
+      const int n = t.b;
       t.a = at;
       t.b = at + n;
       at += n;
@@ -304,7 +299,6 @@ __device__ void make_plan(const hq_cache& c, int R, Plan& p, int* red, bool stal
     }
     p.nseg = blockIdx.x < ceff ? k : 0;
     p.ntile = blockIdx.x < ceff ? at : 0;
-    p.ceff = ceff;
   }
   __syncthreads();
 }
@@ -583,11 +577,11 @@ __device__ __forceinline__ void fp16_src(const hq_cache& c, const UnitGeo& g, in
 __global__ void __launch_bounds__(NTHREADS, 1)
 decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* __restrict__ k_new,
               const uint16_t* __restrict__ v_new, uint16_t* __restrict__ out, float qscale,
-              float* __restrict__ parts, unsigned int* __restrict__ tickets) {
+              float* __restrict__ parts, unsigned int* __restrict__ tickets, int lse_ok) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t full[NSTAGES], empty[NSTAGES];
   __shared__ Plan plan;
-  __shared__ int red[NTHREADS / 32 + 2];
+  __shared__ int red[NTHREADS / 32];
   __shared__ int s_timeout;          // a bounded wait gave up somewhere in this CTA
   __shared__ int s_issued[NSTAGES];  // tiles issued into each stage
   __shared__ int s_held[NC];         // stage holding each consumer warp's state at a segment end (-1: none)
@@ -615,17 +609,16 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
   if (warp == NC) {
     for (int si = 0; si < plan.nseg; ++si) {
       const Seg s = plan.seg[si];
-      const int32_t* st = state_row(c, s.u / c.Hkv);
-      const int np = min(max(*reinterpret_cast<volatile const int*>(st + HQ_STATE_NPACKED), 0), c.cap);
-      const int nv = min(max(*reinterpret_cast<volatile const int*>(st + HQ_STATE_NVL), 0), c.vl_cap);
-      const UnitGeo ug = unit_geo(np, nv, *reinterpret_cast<volatile const int*>(st + HQ_STATE_T), R);
-      const int k1 = s.k0 + (s.b - s.a);
-      const int p0 = s.k0 - fp16_before(ug, s.k0), p1 = min(k1 - fp16_before(ug, k1), c.cap / PK);
+      const int p0 = s.p0, p1 = min(s.p0 + s.npk, c.cap / PK);
       for (int pg = p0 + lane; pg < p1; pg += 32) {  // one page per lane
         const long long idx = page_index(c, s.u, pg);
         if (idx >= 0) prefetch_l2(c.pages + static_cast<size_t>(idx) * HQ_PAGE_BYTES, PK_TX);
       }
-      const int v0 = min(fp16_before(ug, s.k0), ug.NV), v1 = min(fp16_before(ug, k1), min(ug.NV, c.vl_cap / FT));
+      int T, np, nv;
+      read_len(c, s.u / c.Hkv, true, T, np, nv);
+      const int NV = (nv + FT - 1) / FT;
+      const int nf = (s.b - s.a) - s.npk;
+      const int v0 = min(s.f0, NV), v1 = min(s.f0 + nf, min(NV, c.vl_cap / FT));
       if (lane == 0 && v1 > v0) {
         const size_t off = (static_cast<size_t>(s.u) * c.vl_cap + v0 * FT) * D;
         prefetch_l2(c.kf + off, (v1 - v0) * FT * D * 2);
@@ -665,21 +658,12 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
       int k = 0;   // uses of this stage so far
       int si = 0;  // segment cursor
       UnitGeo ug = geo_of_unit(c, plan.seg[0].u, R);
-      TileWalk tw;
-      bool fresh = true;
       for (int i = s; i < ntile; i += NSTAGES, ++k) {
         while (i >= plan.seg[si].b) {
           ++si;
           ug = geo_of_unit(c, plan.seg[si].u, R);
-          fresh = true;
         }
         const Seg sg = plan.seg[si];
-        if (fresh) {
-          tw.start(ug, sg.k0 + (i - sg.a), NSTAGES);
-          fresh = false;
-        } else {
-          tw.step(NSTAGES);
-        }
         int32_t* srow = state_row(c, sg.u / c.Hkv);
         // the k-th refill waits for the consumer's k-th release (phase k - 1)
         if (k > 0 && !mbar_wait(&empty[s], (k - 1) & 1, srow)) {
@@ -687,7 +671,7 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
           break;
         }
         s_issued[s] = k + 1;
-        const int tl = tw.tile();
+        const int tl = seg_tile(sg, i);
         if (tl >= 0) {
           mbar_arrive_expect_tx(&full[s], PK_TX);
           bulk_g2s(st, page_of(c, sg.u, tl * PK), PK_TX, &full[s]);
@@ -721,9 +705,7 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
       // this warp's tiles of the segment: i = sg.a + ((warp - sg.a) mod NC), step NC
       int i = sg.a + ((warp - sg.a) % NC + NC) % NC;
       int held = -1;
-      TileWalk tw;
-      tw.start(ug, sg.k0 + (i - sg.a), NC);
-      for (; i < sg.b; i += NC, tw.step(NC)) {
+      for (; i < sg.b; i += NC) {
         const int s = i % NSTAGES;
         // the timeout decision is made warp-uniform so the warp never splits
         if (!__all_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&s_timeout) == 0 &&
@@ -732,7 +714,7 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
           break;
         }
         const uint8_t* st = smem + s * STAGE_BYTES;
-        const int tl = tw.tile();
+        const int tl = seg_tile(sg, i);
         if (tl >= 0) {
           packed_tile(ws, st, qf, tl, ug.n_packed, qscale, g, t);
         } else {
@@ -879,7 +861,12 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
           }
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) ll += __shfl_xor_sync(0xffffffffu, ll, o);
-          if (lane == 0) sm_inv[qc] = ll > 0.f ? 1.0f / ll : 0.f;
+          if (lane == 0) {
+            sm_inv[qc] = ll > 0.f ? 1.0f / ll : 0.f;
+            if (c.qlse != nullptr)  // the query's log-sum-exp (base 2), kept for the next reselection
+              c.qlse[(static_cast<size_t>(b) * c.Hq + kvh * G + qc) * HQ_QBUF + (T % HQ_QBUF)] =
+                  lse_ok ? mm + __log2f(ll) : __int_as_float(0x7fc00000);
+          }
         }
         consumer_bar();
         if (mine) {
@@ -1004,7 +991,10 @@ hq_status launch_decode(const hq_cache& c, const uint16_t* q, const uint16_t* kn
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const float qs = sm_scale * LOG2E;
-  return cuda_status(cudaLaunchKernelEx(&cfg, decode_kernel, c, q, kn, vn, out, qs, parts, tickets), "decode launch");
+  // the stored log-sum-exps serve the reselection only at its own scale 1/sqrt(D)
+  const int lse_ok = sm_scale == 1.0f / sqrtf(static_cast<float>(D));
+  return cuda_status(cudaLaunchKernelEx(&cfg, decode_kernel, c, q, kn, vn, out, qs, parts, tickets, lse_ok),
+                     "decode launch");
 }
 
 }  // namespace hq

@@ -83,6 +83,7 @@ hq_status hq_cache_validate(const hq_cache* c) {
   if (c->page_table != nullptr && ((reinterpret_cast<uintptr_t>(c->page_table) & 3u) != 0 || c->n_pages < 1))
     return HQ_ERR_INVALID;
   if (c->score_acc != nullptr && (reinterpret_cast<uintptr_t>(c->score_acc) & 15u) != 0) return HQ_ERR_INVALID;
+  if (c->qlse != nullptr && (reinterpret_cast<uintptr_t>(c->qlse) & 15u) != 0) return HQ_ERR_INVALID;
   return HQ_OK;
 }
 

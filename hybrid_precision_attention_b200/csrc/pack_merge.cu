@@ -10,8 +10,10 @@
 // Kernels (all bandwidth-trivial next to decode; one warp per row):
 //   pack_rows      positions [lo, hi) of every (b, kv head) -> K4V4 records
 //   ring_fill      init only: last min(W, L) prefix rows -> FP16 ring
-//   vl_gather      merge only: new VL rows -> workspace (old VL row, ring row,
-//                  or the dequantised record rounded once to fp16); clears old bits
+//   vl_gather      merge only: new VL rows -> workspace (old VL row, found through
+//                  its page's bitmap, ring row, or the dequantised record rounded
+//                  once to fp16)
+//   vl_clear       merge only: bitmap words of the pages holding the old lines -> 0
 //   vl_install     rows -> VL store, positions, bitmap bits, per-page first VL row,
 //                  state update
 #include "common.cuh"
@@ -118,108 +120,119 @@ __global__ void ring_fill_kernel(hq_cache c, const uint16_t* __restrict__ kd, co
   }
 }
 
-__device__ __forceinline__ int find_sorted(const int32_t* __restrict__ a, int n, int key) {
-  int lo = 0, hi = n;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (a[mid] < key) lo = mid + 1; else hi = mid;
-  }
-  return (lo < n && a[lo] == key) ? lo : -1;
+// VL-store row of position p if p is one of the current vertical lines (its
+// page's bitmap bit is set), else -1: the page records the row of its first
+// line, and rows are in position order, so the row is that plus the number of
+// lines of the page below p.
+__device__ __forceinline__ int old_vl_row(const hq_cache& c, size_t bh, int p) {
+  const uint8_t* page = page_of(c, bh, p);
+  const uint2 m = *reinterpret_cast<const uint2*>(page + HQ_PAGE_VLMASK);
+  const int r = p & 63;
+  const uint32_t w = r < 32 ? m.x : m.y;
+  if (!((w >> (r & 31)) & 1u)) return -1;
+  const int below = __popc(w & ((1u << (r & 31)) - 1u)) + (r < 32 ? 0 : __popc(m.x));
+  return *reinterpret_cast<const int32_t*>(page + HQ_PAGE_VLBASE) + below;
 }
 
-// Merge: gather the FP16 rows of the new VL set into the workspace and clear the
-// bitmap bits of the old set.  One warp per (b, h, r, K|V); every sequence
-// uses its own state row.
+// Merge: gather the FP16 rows of the new VL set into the workspace.  One warp
+// per (b, h, row) handles K and V; an old line is found through its page's
+// bitmap (read only here: the bits change in the next two kernels).
 __global__ void vl_gather_kernel(hq_cache c, uint16_t* __restrict__ wsk, uint16_t* __restrict__ wsv) {
   const Dims d = dims_of(c);
   const int lane = threadIdx.x & 31;
   const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
-  const long long total = 2ll * d.B * d.Hkv * d.vl_cap;
+  const long long total = static_cast<long long>(d.B) * d.Hkv * d.vl_cap;
   for (long long w = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); w < total; w += warps) {
-    const int which = static_cast<int>(w & 1);
-    const long long rest = w >> 1;
-    const int r = static_cast<int>(rest % d.vl_cap);
-    const long long bh = rest / d.vl_cap;
+    const int r = static_cast<int>(w % d.vl_cap);
+    const long long bh = w / d.vl_cap;
     int32_t* st = state_row(c, static_cast<int>(bh / d.Hkv));
     const int k = min(st[HQ_STATE_KSEL], d.vl_cap);
     if (r >= k) continue;
     const int n_packed = st[HQ_STATE_NPACKED];
-    const int n_vl = st[HQ_STATE_NVL];
     const int p = c.vl_sel[bh * d.vl_cap + r];
-    uint16_t* dst = (which ? wsv : wsk) + (bh * d.vl_cap + r) * D;
     if (p < 0 || p >= max(n_packed, st[HQ_STATE_T] - d.W)) {  // not a position the merge can hold
       if (lane == 0) set_err(st, HQ_DEVERR_VL_CAPACITY);
       continue;
     }
-    const int old = find_sorted(c.vl_pos + bh * d.vl_cap, n_vl, p);
-    if (old >= 0) {
-      const uint16_t* s = (which ? c.vf : c.kf) + (bh * d.vl_cap + old) * D;
-      reinterpret_cast<uint2*>(dst)[lane] = reinterpret_cast<const uint2*>(s)[lane];
-    } else if (p >= n_packed) {
-      const uint16_t* s = (which ? c.vr : c.kr) + (bh * d.R + (p % d.R)) * D;
-      reinterpret_cast<uint2*>(dst)[lane] = reinterpret_cast<const uint2*>(s)[lane];
-    } else {
-      // promoted packed position: fp16(zero + q * scale); q * scale is exact in
-      // float64 and the sum is rounded once, then once more to fp16 (RN).
-      uint8_t* page = page_of(c, bh, p);
-      const uint8_t* codes = row_codes(page, which, p);
-      const uint32_t szw = row_sz(page, which, p)[lane >> 3];
-      const double sc = static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(szw & 0xFFFFu))));
-      const double ze = static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(szw >> 16))));
-      const uint32_t two = reinterpret_cast<const uint16_t*>(codes)[lane];
-      uint32_t out[2];
+    const int old = p < n_packed ? old_vl_row(c, bh, p) : -1;
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const uint32_t byte = (two >> (8 * i)) & 0xFFu;
-        const double v0 = __dadd_rn(ze, __dmul_rn(static_cast<double>(byte & 15u), sc));
-        const double v1 = __dadd_rn(ze, __dmul_rn(static_cast<double>(byte >> 4), sc));
-        out[i] = static_cast<uint32_t>(__half_as_ushort(__double2half(v0))) |
-                 (static_cast<uint32_t>(__half_as_ushort(__double2half(v1))) << 16);
+    for (int which = 0; which < 2; ++which) {
+      uint16_t* dst = (which ? wsv : wsk) + (bh * d.vl_cap + r) * D;
+      if (old >= 0) {
+        const uint16_t* s = (which ? c.vf : c.kf) + (bh * d.vl_cap + old) * D;
+        reinterpret_cast<uint2*>(dst)[lane] = reinterpret_cast<const uint2*>(s)[lane];
+      } else if (p >= n_packed) {
+        const uint16_t* s = (which ? c.vr : c.kr) + (bh * d.R + (p % d.R)) * D;
+        reinterpret_cast<uint2*>(dst)[lane] = reinterpret_cast<const uint2*>(s)[lane];
+      } else {
+        // promoted packed position: fp16(zero + q * scale); q * scale is exact in
+        // float64 and the sum is rounded once, then once more to fp16 (RN).
+        uint8_t* page = page_of(c, bh, p);
+        const uint8_t* codes = row_codes(page, which, p);
+        const uint32_t szw = row_sz(page, which, p)[lane >> 3];
+        const double sc = static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(szw & 0xFFFFu))));
+        const double ze = static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(szw >> 16))));
+        const uint32_t two = reinterpret_cast<const uint16_t*>(codes)[lane];
+        uint32_t out[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const uint32_t byte = (two >> (8 * i)) & 0xFFu;
+          const double v0 = __dadd_rn(ze, __dmul_rn(static_cast<double>(byte & 15u), sc));
+          const double v1 = __dadd_rn(ze, __dmul_rn(static_cast<double>(byte >> 4), sc));
+          out[i] = static_cast<uint32_t>(__half_as_ushort(__double2half(v0))) |
+                   (static_cast<uint32_t>(__half_as_ushort(__double2half(v1))) << 16);
+        }
+        reinterpret_cast<uint2*>(dst)[lane] = make_uint2(out[0], out[1]);
       }
-      reinterpret_cast<uint2*>(dst)[lane] = make_uint2(out[0], out[1]);
     }
   }
-  // clear the old set's bitmap bits (nothing in this kernel reads the bitmap)
-  const long long tot2 = static_cast<long long>(d.B) * d.Hkv * d.vl_cap;
-  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < tot2;
+}
+
+// Merge: clear the bitmap words of every page that holds a current (old)
+// vertical line (plain stores of zero; the new set's bits are set afterwards).
+__global__ void vl_clear_kernel(hq_cache c) {
+  const Dims d = dims_of(c);
+  const long long total = static_cast<long long>(d.B) * d.Hkv * d.vl_cap;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
     const long long bh = i / d.vl_cap;
     const int r = static_cast<int>(i % d.vl_cap);
     if (r >= state_row(c, static_cast<int>(bh / d.Hkv))[HQ_STATE_NVL]) continue;
-    const int p = c.vl_pos[bh * d.vl_cap + r];
-    uint8_t* page = page_for_write(c, bh, p);
-    if (page) atomicAnd(page_mask(page) + ((p & 63) >> 5), ~(1u << (p & 31)));
+    uint8_t* page = page_for_write(c, bh, c.vl_pos[bh * d.vl_cap + r]);
+    if (page) *reinterpret_cast<uint2*>(page + HQ_PAGE_VLMASK) = make_uint2(0u, 0u);
   }
 }
 
 // Install rows into the VL store.  Init: rows from the dense prefix; merge: rows
-// from the workspace.  Sets bitmap bits, writes vl_pos.  The last block to finish
-// (ticket) updates the state rows.
+// from the workspace.  One warp per (b, h, row): K and V rows, vl_pos, the
+// bitmap bit and (first line of a page) the page's first VL-store row.  The
+// last block to finish (ticket) updates the state rows.
 __global__ void vl_install_kernel(hq_cache c, const uint16_t* __restrict__ srck, const uint16_t* __restrict__ srcv, int L,
                                   int init, unsigned int* __restrict__ ticket) {
   const Dims d = dims_of(c);
-  const long long chunks = 2ll * d.B * d.Hkv * d.vl_cap * (D / 8);
-  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < chunks;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int ch = static_cast<int>(i % (D / 8));
-    long long r = i / (D / 8);
-    const int which = static_cast<int>(r & 1);
-    r >>= 1;
-    const int row = static_cast<int>(r % d.vl_cap);
-    const long long bh = r / d.vl_cap;
+  const int lane = threadIdx.x & 31;
+  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  const long long total = static_cast<long long>(d.B) * d.Hkv * d.vl_cap;
+  for (long long w = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); w < total; w += warps) {
+    const int row = static_cast<int>(w % d.vl_cap);
+    const long long bh = w / d.vl_cap;
     int32_t* st = state_row(c, static_cast<int>(bh / d.Hkv));
     const int k = min(st[HQ_STATE_KSEL], d.vl_cap);
     if (row >= k) continue;
     const int p = c.vl_sel[bh * d.vl_cap + row];
     const int limit = init ? max(L - d.W, 0) : max(st[HQ_STATE_NPACKED], st[HQ_STATE_T] - d.W);
     if (p < 0 || p >= limit) {
-      if (ch == 0 && which == 0) set_err(st, HQ_DEVERR_VL_CAPACITY);
+      if (lane == 0) set_err(st, HQ_DEVERR_VL_CAPACITY);
       continue;
     }
-    const uint16_t* s = init ? ((which ? srcv : srck) + (bh * L + p) * D) : ((which ? srcv : srck) + (bh * d.vl_cap + row) * D);
-    uint16_t* t = (which ? c.vf : c.kf) + (bh * d.vl_cap + row) * D;
-    reinterpret_cast<uint4*>(t)[ch] = reinterpret_cast<const uint4*>(s)[ch];
-    if (ch == 0 && which == 0) {
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      const uint16_t* s = init ? ((which ? srcv : srck) + (bh * L + p) * D)
+                               : ((which ? srcv : srck) + (bh * d.vl_cap + row) * D);
+      uint16_t* t = (which ? c.vf : c.kf) + (bh * d.vl_cap + row) * D;
+      reinterpret_cast<uint2*>(t)[lane] = reinterpret_cast<const uint2*>(s)[lane];
+    }
+    if (lane == 0) {
       c.vl_pos[bh * d.vl_cap + row] = p;
       uint8_t* page = page_for_write(c, bh, p);
       if (page) {
@@ -288,10 +301,11 @@ hq_status launch_pack_merge(const hq_cache& c, const uint16_t* kd, const uint16_
   pack_rows_kernel<<<sms * 4, threads, 0, st>>>(c, kd, vd, L, init);
   if (init) {
     ring_fill_kernel<<<sms, threads, 0, st>>>(c, kd, vd, L);
-    vl_install_kernel<<<sms, threads, 0, st>>>(c, kd, vd, L, 1, ticket);
+    vl_install_kernel<<<sms * 4, threads, 0, st>>>(c, kd, vd, L, 1, ticket);
   } else {
-    vl_gather_kernel<<<sms * 2, threads, 0, st>>>(c, wsk, wsv);
-    vl_install_kernel<<<sms, threads, 0, st>>>(c, wsk, wsv, L, 0, ticket);
+    vl_gather_kernel<<<sms * 4, threads, 0, st>>>(c, wsk, wsv);
+    vl_clear_kernel<<<sms, threads, 0, st>>>(c);
+    vl_install_kernel<<<sms * 4, threads, 0, st>>>(c, wsk, wsv, L, 0, ticket);
   }
   return cuda_status(cudaGetLastError(), "merge launch");
 }

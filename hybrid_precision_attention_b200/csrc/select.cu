@@ -24,6 +24,8 @@
 //                    shared memory, a bit-by-bit search of their low 20 bits ->
 //                    the exact k-th value, then an ordered compaction writes the
 //                    chosen positions ascending, ties to the lowest positions
+// When the decode steps kept their log-sum-exps (c.qlse) and every buffered
+// query came after the last merge, pass 0 is skipped: those are its row sums.
 // With running scores (c.score_acc), pass 1 adds each key's column mass to its
 // stored sum (decode mode) or starts it (init mode) and ranks the sums.
 // Keys are rebuilt as fp16 in their current representation (dense prefix in
@@ -245,6 +247,27 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
   const int M = G * g.nq;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  // Row normalisers from the decode steps: when every buffered query was
+  // decoded after the last merge, its decode step saw exactly the keys this
+  // reselection sees (same VL set, same packed range, the rest FP16), and the
+  // log-sum-exp it stored is the one pass 0 would compute; pass 0 then only
+  // clears its slice of the histogram.
+  bool use_dec = false;
+  if (!a.k_dense && c.qlse != nullptr && g.nq > 0 && g.qpos0 >= g.n_packed + c.W) {
+    bool ok = true;
+    for (int r = threadIdx.x; r < M; r += SEL_THREADS) {
+      const int h = r / g.nq, p = g.qpos0 + r % g.nq;
+      const float z = c.qlse[(static_cast<size_t>(b) * c.Hq + kvh * G + h) * HQ_QBUF + (p % HQ_QBUF)];
+      ok = ok && isfinite(z);
+    }
+    use_dec = __syncthreads_and(ok) != 0;
+  }
+  if (!COL && use_dec) {
+    uint32_t* gh = a.hist + static_cast<size_t>(bh) * HBINS;
+    for (int e = (split * HBINS) / a.S + threadIdx.x; e < ((split + 1) * HBINS) / a.S; e += SEL_THREADS) gh[e] = 0u;
+    return;
+  }
+
   // this CTA's key tiles: pass 0 covers every visible key [0, T), pass 1 the
   // candidates [0, n)
   const int lim = COL ? g.n : g.T;
@@ -307,10 +330,13 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
     for (int e = threadIdx.x; e < HBINS; e += SEL_THREADS) shist[e] = 0u;
   }
   if (COL) {
-    // per-row log-sum-exp over the pass-0 partials of every split
+    // per-row log-sum-exp: stored by the decode steps, or over the pass-0 partials of every split
     for (int r = threadIdx.x; r < Mp; r += SEL_THREADS) {
       float z = INFINITY;
-      if (r < M) {
+      if (r < M && use_dec) {
+        const int h = r / g.nq, p = g.qpos0 + r % g.nq;
+        z = c.qlse[(static_cast<size_t>(b) * c.Hq + kvh * G + h) * HQ_QBUF + (p % HQ_QBUF)];
+      } else if (r < M) {
         const float* lp = a.lse_part + (static_cast<size_t>(bh) * MAX_SPLITS) * Mp * 2 + 2 * r;
         float mm = -INFINITY, ll = 0.f;
 #pragma unroll 8
@@ -550,29 +576,19 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
 }
 
 constexpr int TK_THREADS = 1024;
-constexpr int TK_SMEM_MAX = 49152;  // scores held in shared memory up to this many candidates
+constexpr int TK_SMEM_MAX = 47104;  // scores held in shared memory up to this many candidates (with the static arrays, <= 227 KB)
 constexpr int TK_CAND_MAX = 8192;   // values of the threshold's histogram bin held in shared memory
-
-// block-wide sum of one value per thread (1024 threads); every thread gets it
-__device__ __forceinline__ unsigned int tk_block_sum(unsigned int v, unsigned int* red) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  v = __reduce_add_sync(0xffffffffu, v);
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  const unsigned int tot = __reduce_add_sync(0xffffffffu, red[lane]);
-  __syncthreads();
-  return tot;
-}
 
 // Exact top-k of the column-mass scores of one (b, kv head).  Scores are >= 0,
 // so their fp32 bit patterns order like the values.  (1) The histogram of bits
 // 30..20 that the column-mass pass built gives the bin holding the k-th
 // largest value and how many values lie above it.  (2) The values of that bin
-// are gathered into shared memory.  (3) Its low 20 bits are found bit by bit
-// (keep a bit when at least the needed number of candidates are >= the pattern
-// with it set).  (4) An ordered compaction over contiguous per-thread segments
-// writes the chosen positions ascending, ties at the threshold to the lowest
-// positions.  A bin too large for shared memory is searched in global memory.
+// are gathered into shared memory.  (3) Its low 20 bits are found by two radix
+// passes of 10 bits (a 1024-bin histogram of the candidates, then the sub-bin
+// holding the needed rank).  (4) An ordered compaction, one contiguous range
+// of positions per warp, writes the chosen positions ascending, ties at the
+// threshold to the lowest positions.  A bin too large for shared memory is
+// searched in global memory.
 __global__ void __launch_bounds__(TK_THREADS) topk_kernel(SelArgs a, int smem_scores) {
   const hq_cache& c = a.c;
   const int bh = blockIdx.x;
@@ -592,9 +608,9 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(SelArgs a, int smem_sc
   if (bh % c.Hkv == 0 && threadIdx.x == 0) srow[HQ_STATE_KSEL] = k;
   if (k == 0) return;
   extern __shared__ uint32_t tk_smem[];  // [TK_CAND_MAX] bin values, then [smem_scores] scores
-  __shared__ unsigned int red[32];
   __shared__ unsigned int s_bin, s_above, s_cnt;
   __shared__ unsigned int wsum[TK_THREADS / 32];
+  __shared__ unsigned int tk_hist[TK_THREADS];   // radix sub-bins of the threshold bin
   const uint32_t* gsc = reinterpret_cast<const uint32_t*>(a.scores + static_cast<size_t>(bh) * c.cap);
   uint32_t* cand = tk_smem;
   // the scores are staged in shared memory (all loads in flight at once) when they fit
@@ -656,63 +672,88 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(SelArgs a, int smem_sc
       const unsigned int slot = base + __popc(m & ((1u << lane) - 1u));
       if (hit && slot < nbin) cand[slot] = v;  // nbin <= TK_CAND_MAX: the list never overflows
     }
-    __syncthreads();
   }
+  __syncthreads();
   const int ncand = in_smem ? static_cast<int>(min(s_cnt, nbin)) : n;
-  // (3) low 20 bits of the k-th largest
-  uint32_t thr = bin << 20;
-  for (int bit = 19; bit >= 0; --bit) {
-    const uint32_t cnd = thr | (1u << bit);
-    unsigned int ge = 0u;
+  // (3) the low 20 bits of the k-th largest, by two radix passes of 10 bits over
+  // the bin's values: a 1024-bin histogram of bits 19..10, the sub-bin holding
+  // the needed rank, then a histogram of bits 9..0 inside that sub-bin
+  unsigned int* h10 = tk_hist;
+  uint32_t prefix = bin << 20;   // bits fixed so far
+  uint32_t pmask = 0xFFF00000u;  // which bits are fixed
+  unsigned int above = s_above;  // values above everything that matches the prefix
+#pragma unroll 1
+  for (int pass = 0; pass < 2; ++pass) {
+    const int shift = pass == 0 ? 10 : 0;
+    h10[threadIdx.x] = 0u;
+    __syncthreads();
     for (int e = threadIdx.x; e < ncand; e += TK_THREADS) {
       const uint32_t v = in_smem ? cand[e] : sc[e];
-      ge += ((v >> 20) == bin && v >= cnd) ? 1u : 0u;
-    }
-    if (tk_block_sum(ge, red) >= need) thr = cnd;
-  }
-  // (4) everything above thr, and the lowest-positioned of those equal to it
-  unsigned int gtb = 0u;
-  for (int e = threadIdx.x; e < ncand; e += TK_THREADS) {
-    const uint32_t v = in_smem ? cand[e] : sc[e];
-    gtb += ((v >> 20) == bin && v > thr) ? 1u : 0u;
-  }
-  const unsigned int take_eq = static_cast<unsigned int>(k) - s_above - tk_block_sum(gtb, red);
-  // ordered compaction in rounds of 1024 consecutive positions (coalesced
-  // reads): a position's slot = (#gt before it) + min(#eq before it, take_eq)
-  __shared__ unsigned int rg[TK_THREADS / 32 + 1], re[TK_THREADS / 32 + 1];
-  unsigned int base_gt = 0u, base_eq = 0u;
-  const unsigned int lt_mask = (1u << lane) - 1u;
-  for (int j0 = 0; j0 < n; j0 += TK_THREADS) {
-    const int j = j0 + threadIdx.x;
-    const uint32_t v = j < n ? sc[j] : 0u;
-    const bool gt = j < n && v > thr, eq = j < n && v == thr;
-    const unsigned int bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
-    if (lane == 0) {
-      rg[warp] = __popc(bg);
-      re[warp] = __popc(be);
+      if ((v & pmask) == prefix) atomicAdd(&h10[(v >> shift) & 1023u], 1u);
     }
     __syncthreads();
-    if (warp == 0) {
-      // exclusive prefix over the 32 warps' counts, totals in slot 32
-      unsigned int xg2 = rg[lane], xe2 = re[lane];
-      const unsigned int og = xg2, oe = xe2;
+    // suffix sums over the 1024 sub-bins, highest first: thread i owns sub-bin 1023 - i
+    const unsigned int hv = h10[TK_THREADS - 1 - threadIdx.x];
+    unsigned int x = hv;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const unsigned int yg = __shfl_up_sync(0xffffffffu, xg2, o), ye = __shfl_up_sync(0xffffffffu, xe2, o);
-        if (lane >= o) { xg2 += yg; xe2 += ye; }
-      }
-      rg[lane] = xg2 - og;
-      re[lane] = xe2 - oe;
-      if (lane == 31) { rg[32] = xg2; re[32] = xe2; }
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[warp] = x;
+    __syncthreads();
+    for (int w = 0; w < warp; ++w) x += wsum[w];
+    // x = values in sub-bins >= this one (within the prefix); the needed rank is k - above
+    const unsigned int needp = static_cast<unsigned int>(k) - above;
+    if (x >= needp && x - hv < needp) {
+      s_bin = TK_THREADS - 1 - threadIdx.x;
+      s_above = above + (x - hv);
+      s_cnt = hv;
     }
     __syncthreads();
-    const unsigned int pg = rg[warp], pe = re[warp], tg = rg[32], te = re[32];
-    const unsigned int xg = base_gt + pg + __popc(bg & lt_mask), xe = base_eq + pe + __popc(be & lt_mask);
-    if (gt) out[xg + min(xe, take_eq)] = j;
-    else if (eq && xe < take_eq) out[xg + xe] = j;
-    base_gt += tg;
-    base_eq += te;
+    prefix |= s_bin << shift;
+    pmask |= 1023u << shift;
+    above = s_above;
     __syncthreads();
+  }
+  const uint32_t thr = prefix;
+  // take_eq of the values equal to thr (the lowest positions), all values above it
+  const unsigned int take_eq = static_cast<unsigned int>(k) - above;
+  // (4) ordered compaction: warp w owns positions [w P, (w + 1) P); a first
+  // sweep counts the values above and equal to thr per warp, a block scan gives
+  // each warp its output offsets, a second sweep writes positions in order
+  // (ballots inside the warp, 32 consecutive positions per round)
+  const int P = ((n + TK_THREADS / 32 - 1) / (TK_THREADS / 32) + 31) / 32 * 32;
+  const int j_lo = warp * P, j_hi = min(n, j_lo + P);
+  unsigned int cg = 0u, ce = 0u;
+  for (int j0 = j_lo; j0 < j_hi; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t v = j < j_hi ? sc[j] : 0u;
+    cg += __popc(__ballot_sync(0xffffffffu, j < j_hi && v > thr));
+    ce += __popc(__ballot_sync(0xffffffffu, j < j_hi && v == thr));
+  }
+  __shared__ unsigned int rg[TK_THREADS / 32], re[TK_THREADS / 32];
+  if (lane == 0) {
+    rg[warp] = cg;
+    re[warp] = ce;
+  }
+  __syncthreads();
+  unsigned int xg = 0u, xe = 0u;
+  for (int w = 0; w < warp; ++w) {
+    xg += rg[w];
+    xe += re[w];
+  }
+  const unsigned int lt_mask = (1u << lane) - 1u;
+  for (int j0 = j_lo; j0 < j_hi; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t v = j < j_hi ? sc[j] : 0u;
+    const bool gt = j < j_hi && v > thr, eq = j < j_hi && v == thr;
+    const unsigned int bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
+    const unsigned int mg = xg + __popc(bg & lt_mask), me = xe + __popc(be & lt_mask);
+    if (gt) out[mg + min(me, take_eq)] = j;
+    else if (eq && me < take_eq) out[mg + me] = j;
+    xg += __popc(bg);
+    xe += __popc(be);
   }
 }
 

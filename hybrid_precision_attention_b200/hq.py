@@ -41,7 +41,8 @@ _lib = ctypes.CDLL(LIB_PATH)
 class HqCacheStruct(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("B", "Hq", "Hkv", "D", "W", "rho_bp", "cap", "vl_cap")] + [
         (n, ctypes.c_void_p)
-        for n in ("pages", "kf", "vf", "vl_pos", "kr", "vr", "qbuf", "vl_sel", "state", "page_table", "score_acc")
+        for n in ("pages", "kf", "vf", "vl_pos", "kr", "vr", "qbuf", "vl_sel", "state", "page_table", "score_acc",
+                  "qlse")
     ] + [("n_pages", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
@@ -125,7 +126,7 @@ class HybridCache:
 
     def __init__(self, B: int, Hq: int, Hkv: int, cap: int, W: int = 128, rho_bp: int = 500, vl_cap: int = None,
                  device="cuda", D: int = HQ_HEAD_DIM, paged: bool = False, n_pages: int = None, page_order=None,
-                 running_scores: bool = False):
+                 running_scores: bool = False, decode_lse: bool = True):
         cap = ((cap + 127) // 128) * 128
         if vl_cap is None:
             vl_cap = max(16, ((k_of(max(cap - W, 0), rho_bp) + 15) // 16) * 16)
@@ -154,10 +155,12 @@ class HybridCache:
         self.vl_sel = z((B, Hkv, vl_cap), torch.int32)
         self.state_t = z((B, STATE_WORDS), torch.int32)
         self.score_acc = z((B, Hkv, cap), torch.float32) if running_scores else None
+        self.qlse = torch.full((B, Hq, HQ_QBUF), float("nan"), dtype=torch.float32, device=dev) if decode_lse else None
         self.c = HqCacheStruct(B, Hq, Hkv, D, W, rho_bp, cap, vl_cap, *[t.data_ptr() for t in (
             self.pages, self.kf, self.vf, self.vl_pos, self.kr, self.vr, self.qbuf, self.vl_sel, self.state_t)],
             self.page_table.data_ptr() if paged else None,
-            self.score_acc.data_ptr() if running_scores else None, self.n_pages, 0)
+            self.score_acc.data_ptr() if running_scores else None,
+            self.qlse.data_ptr() if decode_lse else None, self.n_pages, 0)
         _check(_lib.hq_cache_validate(ctypes.byref(self.c)), "hq_cache_validate")
         self._ws = {}
 
@@ -199,7 +202,7 @@ class HybridCache:
 
     def nbytes(self) -> int:
         ts = [self.pages, self.kf, self.vf, self.vl_pos, self.kr, self.vr, self.qbuf, self.vl_sel, self.state_t]
-        for t in (self.page_table, self.score_acc):
+        for t in (self.page_table, self.score_acc, self.qlse):
             if t is not None:
                 ts.append(t)
         return sum(t.numel() * t.element_size() for t in ts)
@@ -244,10 +247,12 @@ class CacheSlot:
         self.pages = parent.pages if parent.paged else sl(parent.pages)
         self.page_table = sl(parent.page_table) if parent.paged else None
         self.score_acc = sl(parent.score_acc) if parent.score_acc is not None else None
+        self.qlse = sl(parent.qlse) if parent.qlse is not None else None
         self.c = HqCacheStruct(1, self.Hq, self.Hkv, self.D, self.W, self.rho_bp, self.cap, self.vl_cap, *[
             t.data_ptr() for t in (self.pages, self.kf, self.vf, self.vl_pos, self.kr, self.vr, self.qbuf, self.vl_sel,
                                    self.state_t)], self.page_table.data_ptr() if parent.paged else None,
-            self.score_acc.data_ptr() if self.score_acc is not None else None, parent.n_pages, 0)
+            self.score_acc.data_ptr() if self.score_acc is not None else None,
+            self.qlse.data_ptr() if self.qlse is not None else None, parent.n_pages, 0)
         _check(_lib.hq_cache_validate(ctypes.byref(self.c)), "hq_cache_validate (slot)")
         self._ws = {}
 

@@ -141,6 +141,12 @@ enum {
  *             (init mode) stores its column mass there (zero past the scored prefix) and
  *             every decode-mode reselection adds its column mass to it and ranks the sums
  *             (README Overview item 1, "running column-mass score").
+ *   qlse      float [B, Hq, HQ_QBUF]     optional (NULL: not kept): each decode step stores the
+ *             log-sum-exp (base 2, over its T + 1 logits q.k / sqrt(D)) of its query next to
+ *             the query itself (slot T % HQ_QBUF).  A decode-mode reselection whose buffered
+ *             queries all came after the last merge (so they saw the keys exactly as the
+ *             reselection does) takes its row normalisers from here instead of a first
+ *             pass over the keys.  Decode steps with sm_scale != 1/sqrt(D) store NaN.
  *
  * Limits checked by hq_cache_validate(): D == 128; Hq % Hkv == 0 and
  * Hq / Hkv <= HQ_MAX_GQA; W >= 0; 0 <= rho_bp <= 10000; cap a positive
@@ -164,6 +170,7 @@ typedef struct hq_cache {
   int32_t* state;
   int32_t* page_table;
   float* score_acc;
+  float* qlse;
   int32_t n_pages;
   int32_t reserved;   /* 0 */
 } hq_cache;

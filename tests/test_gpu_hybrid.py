@@ -84,16 +84,24 @@ def test_decode_from_an_empty_cache():
 
 
 def test_reselect_before_staging_is_full():
-    """A merge with fewer than 64 staged tokens packs only what left the window."""
+    """A merge with fewer than 64 staged tokens packs only what left the window.
+    The second reselection's buffer holds queries from before the first merge
+    (which saw other keys), so the decode steps' stored log-sum-exps are not
+    used for them and the selection's own first pass runs."""
     p = Pair(1, 8, 2, 500, 64, 500, cap=800, seed=9)
     p.init()
-    q, k, v = synth.decode_tokens(9, 1, 8, 2, 20)
+    q, k, v = synth.decode_tokens(9, 1, 8, 2, 25)
     for t in range(10):
         out, ref = p.decode(q[t], k[t], v[t])
         check_decode(out, ref)
-    p.reselect_merge()
+    p.reselect_merge()        # every buffered query is fresh: row sums from the decode steps
     assert p.g.state()["n_packed"] == 510 - 64
     for t in range(10, 20):
+        out, ref = p.decode(q[t], k[t], v[t])
+        check_decode(out, ref)
+    p.reselect_merge()        # 10 queries from before the last merge: the first pass runs
+    assert p.g.state()["n_packed"] == 520 - 64
+    for t in range(20, 25):
         out, ref = p.decode(q[t], k[t], v[t])
         check_decode(out, ref)
 
