@@ -40,7 +40,65 @@ E4M3_MAX = 448.0
 FP8_BLOCK = 128
 
 
-# --------------------------------------------------------------------------- K4V4
+# --------------------------------------------------------------------------- K4V4 and the other widths
+
+BITS = (2, 4, 8)   # per-position code widths of the decode cache (K2 / K4 / K8 and V2 / V4 / V8)
+
+
+def pack_bits(x16: np.ndarray, bits: int):
+    """Pack float16 rows [..., D] with ``bits``-bit codes (2, 4 or 8; README
+    Mode reference: the K8V8, K4V2 and K2V4 modes beside K4V4): the K4V4 rule
+    with ``2**bits - 1`` levels, ``8 // bits`` codes per byte, lowest bits first.
+
+    Returns ``codes`` uint8 [..., D * bits // 8], ``scale`` and ``zero`` float16 [..., D // 32].
+    """
+    assert bits in BITS
+    levels = (1 << bits) - 1
+    x = np.asarray(x16, dtype=np.float16)
+    D = x.shape[-1]
+    assert D % GROUP == 0
+    g = x.reshape(x.shape[:-1] + (D // GROUP, GROUP))
+    mn = g.min(axis=-1)
+    mx = g.max(axis=-1)
+    span = mx.astype(np.float32) - mn.astype(np.float32)          # float32 RN
+    scale = (span / np.float32(levels)).astype(np.float16)          # float32 RN, then RN to fp16
+    zero = mn
+    diff = g.astype(np.float32) - zero.astype(np.float32)[..., None]  # float32 RN
+    s_b = scale.astype(np.float32)[..., None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        ratio = diff / s_b                                          # float32 RN
+    q = np.where(s_b == 0, 0.0, np.rint(ratio))                      # ties to even
+    q = np.clip(q, 0, levels).astype(np.uint32).reshape(x.shape)
+    per = 8 // bits
+    q = q.reshape(x.shape[:-1] + (D // per, per))
+    codes = np.zeros(q.shape[:-1], dtype=np.uint32)
+    for i in range(per):
+        codes |= q[..., i] << (bits * i)
+    return codes.astype(np.uint8), scale, zero
+
+
+def unpack_bits(codes: np.ndarray, bits: int) -> np.ndarray:
+    """uint8 [..., D * bits // 8] -> integer levels [..., D] (lowest bits first)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.uint32)
+    per = 8 // bits
+    mask = (1 << bits) - 1
+    q = np.stack([(c >> (bits * i)) & mask for i in range(per)], axis=-1)
+    return q.reshape(c.shape[:-1] + (c.shape[-1] * per,)).astype(np.uint8)
+
+
+def dequant_bits(codes, scale, zero, bits: int) -> np.ndarray:
+    """Dequantised values ``zero + q * scale`` in float64, shape [..., D]."""
+    q = unpack_bits(codes, bits).astype(np.float64)
+    D = q.shape[-1]
+    qg = q.reshape(q.shape[:-1] + (D // GROUP, GROUP))
+    x = np.asarray(zero).astype(np.float64)[..., None] + qg * np.asarray(scale).astype(np.float64)[..., None]
+    return x.reshape(q.shape)
+
+
+def dequant_bits_fp16(codes, scale, zero, bits: int) -> np.ndarray:
+    """The dequantised values rounded once (RN-even) to float16."""
+    return dequant_bits(codes, scale, zero, bits).astype(np.float16)
+
 
 def pack_k4v4(x16: np.ndarray):
     """Pack float16 rows [..., D] (D a multiple of 32) to K4V4.

@@ -6,7 +6,8 @@ What the pages fix (HyQuant digest, method and prefill/decode paragraphs;
 README Overview items 1 and 3, "Overhead"):
 
 * three key classes: vertical-line (VL) positions and a recent window stay in
-  FP16, every other position is stored K4V4;
+  FP16, every other position is stored K4V4 (or, with ``k_bits`` / ``v_bits``,
+  the README's other code widths: K8V8, K4V2, K2V4);
 * the VL set is chosen on the prefill's tail queries, then re-identified every
   64 tokens from at most 64 buffered FP16 queries — decode does not recompute
   global importance every step;
@@ -47,15 +48,17 @@ QBUF = 64       # buffered queries used by the column-mass estimate
 
 class HybridCacheRef:
     def __init__(self, B: int, Hq: int, Hkv: int, W: int, rho_bp: int, cap: int, D: int = 128,
-                 accumulate: bool = False):
+                 accumulate: bool = False, k_bits: int = 4, v_bits: int = 4):
         assert Hq % Hkv == 0 and D % formats.GROUP == 0
         self.B, self.Hq, self.Hkv, self.D, self.W, self.rho_bp, self.cap = B, Hq, Hkv, D, W, rho_bp, cap
         self.G = Hq // Hkv
         self.sm_scale = 1.0 / np.sqrt(D)
         self.k16 = np.zeros((B, Hkv, cap, D), np.float16)      # FP16 value of each position while it has one
         self.v16 = np.zeros((B, Hkv, cap, D), np.float16)
-        self.kq = np.zeros((B, Hkv, cap, D // 2), np.uint8)
-        self.vq = np.zeros((B, Hkv, cap, D // 2), np.uint8)
+        assert k_bits in formats.BITS and v_bits in formats.BITS
+        self.k_bits, self.v_bits = k_bits, v_bits
+        self.kq = np.zeros((B, Hkv, cap, D * k_bits // 8), np.uint8)
+        self.vq = np.zeros((B, Hkv, cap, D * v_bits // 8), np.uint8)
         self.ks = np.zeros((B, Hkv, cap, D // formats.GROUP), np.float16)
         self.kz = np.zeros_like(self.ks)
         self.vs = np.zeros_like(self.ks)
@@ -73,8 +76,9 @@ class HybridCacheRef:
     def _pack_range(self, lo: int, hi: int):
         if hi <= lo:
             return
-        for arr16, q, s, z in ((self.k16, self.kq, self.ks, self.kz), (self.v16, self.vq, self.vs, self.vz)):
-            c, sc, ze = formats.pack_k4v4(arr16[:, :, lo:hi])
+        for arr16, q, s, z, bits in ((self.k16, self.kq, self.ks, self.kz, self.k_bits),
+                                     (self.v16, self.vq, self.vs, self.vz, self.v_bits)):
+            c, sc, ze = formats.pack_bits(arr16[:, :, lo:hi], bits)
             q[:, :, lo:hi], s[:, :, lo:hi], z[:, :, lo:hi] = c, sc, ze
 
     def rep(self, b: int, h: int, upto: int = None):
@@ -83,8 +87,8 @@ class HybridCacheRef:
         np_ = min(self.n_packed, T)
         K = np.empty((T, self.D))
         V = np.empty((T, self.D))
-        K[:np_] = formats.dequant_k4v4(self.kq[b, h, :np_], self.ks[b, h, :np_], self.kz[b, h, :np_])
-        V[:np_] = formats.dequant_k4v4(self.vq[b, h, :np_], self.vs[b, h, :np_], self.vz[b, h, :np_])
+        K[:np_] = formats.dequant_bits(self.kq[b, h, :np_], self.ks[b, h, :np_], self.kz[b, h, :np_], self.k_bits)
+        V[:np_] = formats.dequant_bits(self.vq[b, h, :np_], self.vs[b, h, :np_], self.vz[b, h, :np_], self.v_bits)
         vl = self.vl[b][h]
         K[vl] = self.kf[b][h].astype(np.float64)
         V[vl] = self.vf[b][h].astype(np.float64)
@@ -216,7 +220,7 @@ class HybridCacheRef:
                     elif p >= old_np:
                         kf[r], vf[r] = self.k16[b, h, p], self.v16[b, h, p]
                     else:
-                        kf[r] = formats.dequant_k4v4_fp16(self.kq[b, h, p], self.ks[b, h, p], self.kz[b, h, p])
-                        vf[r] = formats.dequant_k4v4_fp16(self.vq[b, h, p], self.vs[b, h, p], self.vz[b, h, p])
+                        kf[r] = formats.dequant_bits_fp16(self.kq[b, h, p], self.ks[b, h, p], self.kz[b, h, p], self.k_bits)
+                        vf[r] = formats.dequant_bits_fp16(self.vq[b, h, p], self.vs[b, h, p], self.vz[b, h, p], self.v_bits)
                 self.vl[b][h], self.kf[b][h], self.vf[b][h] = pos, kf, vf
         self.n_packed = new_np

@@ -174,3 +174,35 @@ def test_prefill_ref_maps_query_heads_to_their_kv_head():
     # a subset of heads and rows gives the same rows
     sub = attention.prefill_ref(Q, K, V, vl, W, SM, rows=np.arange(8, 20), heads=[(1, 3), (0, 1)])
     assert np.array_equal(sub[(1, 3)], got[(1, 3)][8:]) and np.array_equal(sub[(0, 1)], got[(0, 1)][8:])
+
+
+def test_code_widths_strict_mode_and_error_order():
+    """The other code widths (README Mode reference: K8V8, K4V2, K2V4): with no
+    window and no lines the cache reduces to dequantise-then-attend at those
+    widths (torch SDPA in float64 on the dequantised rows), and the error
+    against FP16 falls as bits are added."""
+    L, steps = 400, 2
+    lay = synth.planted_layer(9, 1, 4, 1, L)
+    qd, kd, vd = synth.decode_tokens(9, 1, 4, 1, steps)
+    full = None
+    errs = {}
+    for kb, vb in ((8, 8), (4, 4), (4, 2), (2, 4), (16, 16)):
+        if kb == 16:
+            c = hybrid.HybridCacheRef(1, 4, 1, L + 10, 0, cap=L + steps)
+        else:
+            c = hybrid.HybridCacheRef(1, 4, 1, 0, 0, cap=L + steps, k_bits=kb, v_bits=vb)
+        c.init_from_prefix(lay.k, lay.v, lay.q_tail)
+        outs = [c.decode(qd[t], kd[t], vd[t]) for t in range(steps)]
+        if kb == 16:
+            full = outs
+            continue
+        ck, sk, zk = formats.pack_bits(lay.k[0, 0], kb)
+        cv, sv, zv = formats.pack_bits(lay.v[0, 0], vb)
+        Kd, Vd = formats.dequant_bits(ck, sk, zk, kb), formats.dequant_bits(cv, sv, zv, vb)
+        for t, o in enumerate(outs):
+            K = np.concatenate([Kd, kd[:t + 1, 0, 0].astype(np.float64)])
+            V = np.concatenate([Vd, vd[:t + 1, 0, 0].astype(np.float64)])
+            assert np.allclose(o[0], _sdpa(qd[t, 0], K, V), rtol=1e-11, atol=1e-13), (kb, vb, t)
+        errs[(kb, vb)] = outs
+    e = {key: _mse(v, full) for key, v in errs.items()}
+    assert e[(8, 8)] < e[(4, 4)] < e[(4, 2)] and e[(4, 4)] < e[(2, 4)]

@@ -173,3 +173,68 @@ def test_fp8_block_scales_and_quantize():
     rel = np.abs(back - x.astype(np.float64)) / np.maximum(np.abs(x.astype(np.float64)), 1e-3)
     big = np.abs(x.astype(np.float64)) > np.repeat(s, 128, axis=-1)[..., :300, None] * 2.0 ** -6 * 8
     assert np.all(rel[big] <= 2.0 ** -4 + 1e-6)
+
+
+# ------------------------------------------------------------------ the 2-bit and 8-bit widths
+
+GOLD_BITS = os.path.join(os.path.dirname(__file__), "golden", "kv_bits_groups.txt")
+
+
+def _load_bit_groups():
+    rows = []
+    for line in open(GOLD_BITS):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        name, bits, vals, sc, ze, codes = [t.strip() for t in line.split("|")]
+        x = np.array([float(t) for t in vals.split()], dtype=np.float64)
+        assert len(x) == 32 and np.all(x.astype(np.float16).astype(np.float64) == x), name
+        rows.append((name, int(bits), x.astype(np.float16), int(sc, 16), int(ze, 16), bytes.fromhex(codes.replace(" ", ""))))
+    return rows
+
+
+@pytest.mark.parametrize("name,bits,x,scale_bits,zero_bits,codes", _load_bit_groups())
+def test_bits_hand_groups(name, bits, x, scale_bits, zero_bits, codes):
+    c, s, z = formats.pack_bits(x, bits)
+    assert c.tobytes() == codes, name
+    assert int(s.view(np.uint16)[0]) == scale_bits, name
+    assert int(z.view(np.uint16)[0]) == zero_bits, name
+    q = formats.unpack_bits(c, bits)
+    # unpacking reads the codes back lowest bits first
+    per = 8 // bits
+    for j in range(32):
+        assert q[j] == (codes[j // per] >> (bits * (j % per))) & ((1 << bits) - 1)
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_bits_levels_are_nearest(bits):
+    """Brute force over the 2^bits levels: every code is a nearest level of its
+    value (up to the float32 rounding of the ratio), and dequantisation is
+    zero + q * scale exactly."""
+    levels = (1 << bits) - 1
+    rng = np.random.default_rng(bits)
+    for trial in range(200):
+        lo = rng.normal() * 4
+        span = abs(rng.normal()) * 3 + 1e-3
+        x = (lo + span * rng.random(32)).astype(np.float16)
+        c, s, z = formats.pack_bits(x, bits)
+        q = formats.unpack_bits(c, bits).astype(np.int64)
+        sc, ze = float(s[0]), float(z[0])
+        assert ze == float(x.min())
+        assert sc == float(np.float16(np.float32(np.float32(x.max()) - np.float32(x.min())) / np.float32(levels)))
+        for j in range(32):
+            cand = [abs(float(x[j]) - (ze + L * sc)) for L in range(levels + 1)]
+            best = min(cand)
+            assert cand[q[j]] <= best + sc * 1e-6 + 1e-12, (bits, trial, j)
+        deq = formats.dequant_bits(c, s, z, bits)
+        assert np.array_equal(deq, ze + q * sc)
+
+
+def test_bits_four_is_k4v4_and_sizes():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((3, 128)).astype(np.float16)
+    a, b = formats.pack_k4v4(x), formats.pack_bits(x, 4)
+    assert all(np.array_equal(u, v) for u, v in zip(a, b))
+    for bits in (2, 4, 8):
+        c, s, z = formats.pack_bits(x, bits)
+        assert c.shape == (3, 128 * bits // 8) and s.shape == z.shape == (3, 4)
