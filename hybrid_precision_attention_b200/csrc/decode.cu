@@ -43,7 +43,8 @@
 //     the last CTA to finish a unit merges that unit's partials with a
 //     log-sum-exp (atomic ticket, no waiting), appends the unit's new token to
 //     the ring and its queries to the query buffer (every CTA of the unit is
-//     done reading by then); the last CTA of the grid advances the lengths;
+//     done reading by then); the last CTA to take its grid ticket (once it
+//     has read every length it uses) advances the lengths;
 //   * launched with programmatic dependent launch: a CTA prefetches its range's
 //     pages and VL rows into L2 before it waits for the previous grid, and lets
 //     the next grid launch as soon as its own wait is over.
@@ -72,9 +73,10 @@ constexpr int OFF_FV = FT * FSTRIDE;           // V rows of an FP16 tile
 constexpr int STAGE_BYTES = 10368;             // max(10256, 2 * 16 * 256 = 8192), 128-aligned
 constexpr int PART_FLOATS = 16 + 8 * D;        // m[8], l[8], O[8][128]
 constexpr int MAX_UNITS = 2048;                // (b, kv head) units per call
-constexpr int MAXSEG = 96;                     // segments (units) one CTA's range can touch
+constexpr int MAXSEG = 88;                     // segments (units) one CTA's range can touch
 constexpr int PHANTOM_DIV = 32;                // phantom weight per unit = ceil(tiles / (CTAs x 32))
 constexpr int MIN_TILES = 4;                   // at least this many tiles per CTA
+constexpr int MAX_CTAS = 160;                  // one CTA per SM, at most this many (the unit merge keeps one weight per CTA in a stage)
 constexpr int SCAN_PER = (MAX_UNITS + NTHREADS - 1) / NTHREADS;  // units per thread in the scan
 constexpr uint32_t PK_TX = HQ_PAGE_VLMASK + 16;   // codes, scale/zero words and the bitmap: one copy
 static_assert(OFF_VC == HQ_PAGE_VCODES && OFF_KS == HQ_PAGE_KSZ && OFF_VS == HQ_PAGE_VSZ && OFF_MASK == HQ_PAGE_VLMASK,
@@ -144,12 +146,11 @@ __device__ __forceinline__ uint32_t fp16_valid(const UnitGeo& g, int j, int R) {
   return m;
 }
 
-// A CTA's share of one unit: CTA-local tiles [a, b) are the unit's tiles
-// k0 .. k0 + b - a - 1 of the interleaved list, which the CTA runs packed ones
-// first (pages p0 .. p0 + npk - 1), then FP16 ones (f0 ..): a warp that gets
-// one tile more than the others then gets a cheap FP16 tile.
+// A CTA's share of one unit: CTA-local tiles [a, b), which the CTA runs packed
+// ones first (pages p0 .. p0 + npk - 1), then FP16 ones (f0 ..): a warp that
+// gets one tile more than the others then gets a cheap FP16 tile.
 struct Seg {
-  int u, a, b, k0, p0, npk, f0, first_cta, ncta;
+  int u, a, b, p0, npk, f0, first_cta, ncta;
 };
 
 // CTA-local tile i of segment sg: the packed tile index (>= 0), or -(FP16 tile index) - 1.
@@ -176,6 +177,95 @@ __device__ __forceinline__ void read_len(const hq_cache& c, int b, bool stale, i
     T = st[HQ_STATE_T];
     np = st[HQ_STATE_NPACKED];
     nv = st[HQ_STATE_NVL];
+  }
+}
+
+// Few units (4 CTAs or more per unit): every unit gets its own CTAs, in
+// proportion to its tiles (at least one, at most one tile per consumer warp),
+// and each of them an even share of the unit's packed tiles and of its FP16
+// tiles, so a CTA has one segment and no range crosses a unit.  The last
+// ALIGNED_SPARE CTAs get no work: they are the ones the block scheduler starts
+// last (their SMs free up last), so no unit waits for a late CTA.
+constexpr int ALIGNED_SPARE = 12;
+constexpr int ALIGNED_MAX_UNITS = MAX_CTAS / 4;
+
+// The lengths an aligned plan was made from: per sequence (n_packed, n_vl,
+// takes a step), per unit (packed tiles, FP16 tiles).
+struct AlignedSnap {
+  int np[ALIGNED_MAX_UNITS], nv[ALIGNED_MAX_UNITS], go[ALIGNED_MAX_UNITS];
+  int NP[ALIGNED_MAX_UNITS], NF[ALIGNED_MAX_UNITS];
+};
+
+// One thread per unit (U <= ALIGNED_MAX_UNITS) records the lengths.
+__device__ __forceinline__ void aligned_snapshot(const hq_cache& c, int R, AlignedSnap& sn, bool stale) {
+  const int U = c.B * c.Hkv;
+  const int tid = threadIdx.x;
+  if (tid < U) {
+    int T, np, nv;
+    read_len(c, tid / c.Hkv, stale, T, np, nv);
+    const bool go = !refused(c, T, np);
+    const UnitGeo g = unit_geo(np, nv, T, R);
+    sn.NP[tid] = go ? g.NP : 0;
+    sn.NF[tid] = go ? g.NF : 0;
+    if (tid % c.Hkv == 0) {
+      const int b = tid / c.Hkv;
+      sn.np[b] = np;
+      sn.nv[b] = nv;
+      sn.go[b] = go;
+    }
+  }
+}
+
+// True (block-wide) when a sequence's lengths differ from the snapshot in a
+// way that changes the plan (n_packed, n_vl, or whether it takes a step).
+__device__ __forceinline__ bool aligned_changed(const hq_cache& c, const AlignedSnap& sn) {
+  bool ch = false;
+  if (static_cast<int>(threadIdx.x) < c.B) {
+    int T, np, nv;
+    read_len(c, threadIdx.x, false, T, np, nv);
+    ch = np != sn.np[threadIdx.x] || nv != sn.nv[threadIdx.x] || (!refused(c, T, np)) != (sn.go[threadIdx.x] != 0);
+  }
+  return __syncthreads_or(ch) != 0;
+}
+
+// Thread 0: the split table and this CTA's segment.
+__device__ __forceinline__ void aligned_assign(const hq_cache& c, Plan& p, const AlignedSnap& sn) {
+  const int U = c.B * c.Hkv;
+  long long N = 0;
+  for (int u = 0; u < U; ++u) N += sn.NP[u] + sn.NF[u];
+  const int C = static_cast<int>(gridDim.x) - (static_cast<int>(gridDim.x) >= 4 * U + ALIGNED_SPARE ? ALIGNED_SPARE : 0);
+  const long long C2 = C - U;  // CTAs to share out beyond one per unit
+  int at = 0, mine = -1, j = 0, S = 1;
+  for (int u = 0; u < U; ++u) {
+    const int nt = sn.NP[u] + sn.NF[u];
+    const int Su = nt == 0 ? 0
+                           : min(1 + static_cast<int>(N > 0 ? (static_cast<long long>(nt) * C2) / N : 0), (nt + NC - 1) / NC);
+    if (static_cast<int>(blockIdx.x) >= at && static_cast<int>(blockIdx.x) < at + Su) {
+      mine = u;
+      j = blockIdx.x - at;
+      S = Su;
+      p.seg[0].first_cta = at;
+      p.seg[0].ncta = Su;
+    }
+    at += Su;
+  }
+  p.ceff = at;
+  p.nseg = 0;
+  p.ntile = 0;
+  if (mine >= 0) {
+    const int NP = sn.NP[mine], NF = sn.NF[mine];
+    Seg& sg = p.seg[0];
+    sg.u = mine;
+    sg.p0 = (j * NP) / S;
+    sg.npk = ((j + 1) * NP) / S - sg.p0;
+    sg.f0 = (j * NF) / S;
+    const int nf = ((j + 1) * NF) / S - sg.f0;
+    sg.a = 0;
+    sg.b = sg.npk + nf;
+    if (sg.b > 0) {
+      p.nseg = 1;
+      p.ntile = sg.b;
+    }
   }
 }
 
@@ -268,7 +358,6 @@ __device__ __noinline__ void make_plan(const hq_cache& c, int R, Plan& p, int* r
           Seg& s = p.seg[u - u0];
           const int k0 = static_cast<int>(lo - S), k1 = static_cast<int>(hi - S);
           s.u = u;
-          s.k0 = k0;
           s.b = k1 - k0;  // a count for now; CTA-local positions are set below
           s.f0 = fp16_before(g, k0);
           s.p0 = k0 - s.f0;
@@ -526,6 +615,23 @@ __device__ __forceinline__ void fp16_tile(WarpState& ws, const uint8_t* st, cons
 }
 
 
+// The last CTA to take its grid ticket advances every stepping sequence's T
+// (and its count of buffered queries).  Every CTA takes its ticket only after
+// it has read all the lengths it uses, so no CTA sees a T of the next step;
+// the appends of the units need no ordering with this (they were placed from
+// the T each CTA read at its start).
+__device__ __forceinline__ void advance_lengths(const hq_cache& c, int tid, int nthr, unsigned int* tickets) {
+  for (int b = tid; b < c.B; b += nthr) {
+    int32_t* st = state_row(c, b);
+    const int T = st[HQ_STATE_T];
+    if (!refused(c, T, st[HQ_STATE_NPACKED])) {
+      st[HQ_STATE_T] = T + 1;
+      st[HQ_STATE_NQ] = min(st[HQ_STATE_NQ] + 1, HQ_QBUF);
+    }
+  }
+  if (tid == 0) tickets[0] = 0u;
+}
+
 // Load this unit's Q^T fragments (the G query heads of kv head kvh of sequence b,
 // in the permuted dim order: thread t covers dims 32t .. 32t+31); columns >= G are zero.
 __device__ __forceinline__ void load_q(const hq_cache& c, const uint16_t* __restrict__ q, int b, int kvh, int G, int g,
@@ -574,6 +680,196 @@ __device__ __forceinline__ void fp16_src(const hq_cache& c, const UnitGeo& g, in
   }
 }
 
+// The end of a segment, on the consumer warps: merge the warp states held in
+// their stages into the segment's partial, take the unit's ticket (and, with the
+// CTA's last segment, its grid ticket), and in the unit's last CTA merge the
+// unit's partials, write its output and append its new token and queries.
+__device__ __forceinline__ void segment_epilogue(const hq_cache& c, const uint16_t* __restrict__ q,
+                                              const uint16_t* __restrict__ k_new, const uint16_t* __restrict__ v_new,
+                                              uint16_t* __restrict__ out, float* __restrict__ parts,
+                                              unsigned int* __restrict__ tickets, int lse_ok, uint8_t* smem, int* s_held,
+                                              int* s_last_p, int* s_glast_p, const Seg sg, const UnitGeo ug, int si,
+                                              int nseg) {
+  const int G = c.Hq / c.Hkv;
+  const int R = ring_len(c.W);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int NTHR = NC * 32;
+  const int u = sg.u, b = u / c.Hkv, kvh = u % c.Hkv;
+  int& s_last = *s_last_p;
+  int& s_glast = *s_glast_p;
+  consumer_bar();  // (A) warp states visible
+  // ------------------------------------------------------------ CTA merge -> segment partial
+  // each thread owns 4 dims of one query and weighs the warp states itself
+  const int c_slot = blockIdx.x + u;  // partial slot of (this CTA, unit u)
+  float* part = parts + static_cast<size_t>(c_slot) * PART_FLOATS;
+  // scratch for the unit merge: a held stage (every segment has a tile, so some
+  // warp holds one unless a wait timed out; then stage 0, which stays in bounds)
+  int scratch = 0;
+  for (int w = NC - 1; w >= 0; --w)
+    if (s_held[w] >= 0) scratch = s_held[w];
+  for (int it = threadIdx.x; it < 8 * D / 4; it += NTHR) {
+    const int qc = (4 * it) / D;
+    float mm = -INFINITY;
+    for (int w = 0; w < NC; ++w)
+      if (s_held[w] >= 0) mm = fmaxf(mm, reinterpret_cast<const float*>(smem + s_held[w] * STAGE_BYTES)[qc]);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float ll = 0.f;
+    for (int w = 0; w < NC; ++w) {
+      if (s_held[w] < 0) continue;
+      const float* wsm = reinterpret_cast<const float*>(smem + s_held[w] * STAGE_BYTES);
+      const float mw = wsm[qc];
+      const float wt = mw == -INFINITY ? 0.f : ex2(mw - mm);
+      const float4 o = reinterpret_cast<const float4*>(wsm + 16)[it];
+      acc.x = fmaf(wt, o.x, acc.x);
+      acc.y = fmaf(wt, o.y, acc.y);
+      acc.z = fmaf(wt, o.z, acc.z);
+      acc.w = fmaf(wt, o.w, acc.w);
+      ll = fmaf(wt, wsm[8 + qc], ll);
+    }
+    reinterpret_cast<float4*>(part + 16)[it] = acc;
+    if ((4 * it) % D == 0) {
+      part[qc] = mm;
+      part[8 + qc] = ll;
+    }
+  }
+  // the new token's K / V rows and this group's queries, loaded now so that the
+  // append after the ticket is stores only (inputs: no ordering concerns)
+  const int T = ug.T;
+  const int slot = T % R;
+  const int bh = u;
+  constexpr int APPEND_MAX = (2 + HQ_MAX_GQA) * (D / 8);
+  static_assert(APPEND_MAX <= 2 * NC * 32, "at most two 16-byte chunks of the append per consumer thread");
+  uint4 app[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+  uint4* app_dst[2] = {nullptr, nullptr};
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int e = threadIdx.x + k * NTHR;
+    if (e < (2 + G) * (D / 8)) {
+      const int row = e / (D / 8), ch = e % (D / 8);
+      if (row < 2) {
+        app[k] = reinterpret_cast<const uint4*>((row ? v_new : k_new) + static_cast<size_t>(bh) * D)[ch];
+        app_dst[k] = reinterpret_cast<uint4*>((row ? c.vr : c.kr) + (static_cast<size_t>(bh) * R + slot) * D) + ch;
+      } else {
+        const size_t h = static_cast<size_t>(b) * c.Hq + kvh * G + (row - 2);
+        app[k] = reinterpret_cast<const uint4*>(q + h * D)[ch];
+        app_dst[k] = reinterpret_cast<uint4*>(c.qbuf + (h * HQ_QBUF + (T % HQ_QBUF)) * D) + ch;
+      }
+    }
+  }
+  // completion ticket of the unit: the barrier orders every thread's partial
+  // writes before thread 0's gpu-scope release; the last CTA acquires before
+  // the barrier that releases its other threads to read the partials
+  // With its last segment the CTA also takes its grid ticket: it has read
+  // every length it needs, and the last grid ticket advances the lengths.
+  consumer_bar();  // (B) partial written, warp states read
+  if (threadIdx.x == 0) {
+    fence_acq_rel_gpu();
+    const unsigned int th = atomicAdd(&tickets[1 + u], 1u);
+    const bool glast = si == nseg - 1 && atomicAdd(&tickets[0], 1u) == gridDim.x - 1;
+    s_last = th == static_cast<unsigned>(sg.ncta - 1);
+    s_glast = glast;
+    if (s_last || glast) fence_acq_rel_gpu();
+  }
+  consumer_bar();  // (C)
+  if (s_glast) advance_lengths(c, threadIdx.x, NC * 32, tickets);
+  if (s_last) {
+    // log-sum-exp merge of the unit's partials (slots first_cta + u ..), in the
+    // scratch stage.  The threads split into ngrp groups, each summing the O
+    // partials of every ngrp-th CTA for one (query, 4 dims) item; a thread's
+    // first PER O loads are issued before the (m, l) of the partials are
+    // gathered and weighed, so both round trips to L2 overlap.
+    const int S = sg.ncta;
+    const float* pb = parts + static_cast<size_t>(sg.first_cta + u) * PART_FLOATS;
+    float* sm_m = reinterpret_cast<float*>(smem + scratch * STAGE_BYTES);  // [S][8] weights
+    float* sm_inv = sm_m + 8 * S;                                          // [8]
+    float4* red4 = reinterpret_cast<float4*>(sm_inv + 8);                  // [ngrp][items]
+    constexpr int PER = 8;
+    const int items = G * (D / 4);
+    const int room = (STAGE_BYTES - 4 * (8 * S + 8)) / (16 * items);      // groups the scratch stage holds
+    const int ngrp = max(1, min(min(NTHR / items, S), room));
+    const int grp = threadIdx.x / items;
+    const int it0 = threadIdx.x - grp * items;
+    const bool mine = grp < ngrp;
+    const float4* osrc = reinterpret_cast<const float4*>(pb + 16 + (it0 / (D / 4)) * D) + it0 % (D / 4);
+    float4 ov[PER];
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+      const int sp = grp + j * ngrp;
+      ov[j] = (mine && sp < S) ? __ldcg(osrc + sp * (PART_FLOATS / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    // partial weights: warp qc weighs query qc's partials, lane s holding s, s + 32, ...
+    for (int qc = warp; qc < G; qc += NC) {
+      float mm = -INFINITY;
+      for (int sp = lane; sp < S; sp += 32) mm = fmaxf(mm, __ldcg(pb + sp * PART_FLOATS + qc));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, o));
+      float ll = 0.f;
+      for (int sp = lane; sp < S; sp += 32) {
+        const float m0 = __ldcg(pb + sp * PART_FLOATS + qc);
+        const float w0 = m0 == -INFINITY ? 0.f : ex2(m0 - mm);
+        ll = fmaf(w0, __ldcg(pb + sp * PART_FLOATS + 8 + qc), ll);
+        sm_m[sp * 8 + qc] = w0;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ll += __shfl_xor_sync(0xffffffffu, ll, o);
+      if (lane == 0) {
+        sm_inv[qc] = ll > 0.f ? 1.0f / ll : 0.f;
+        if (c.qlse != nullptr)  // the query's log-sum-exp (base 2), kept for the next reselection
+          c.qlse[(static_cast<size_t>(b) * c.Hq + kvh * G + qc) * HQ_QBUF + (T % HQ_QBUF)] =
+              lse_ok ? mm + __log2f(ll) : __int_as_float(0x7fc00000);
+      }
+    }
+    consumer_bar();
+    if (mine) {
+      const int qc = it0 / (D / 4);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < PER; ++j) {
+        const int sp = grp + j * ngrp;
+        const float w = sp < S ? sm_m[sp * 8 + qc] : 0.f;
+        acc.x = fmaf(w, ov[j].x, acc.x);
+        acc.y = fmaf(w, ov[j].y, acc.y);
+        acc.z = fmaf(w, ov[j].z, acc.z);
+        acc.w = fmaf(w, ov[j].w, acc.w);
+      }
+      for (int sp = grp + PER * ngrp; sp < S; sp += ngrp) {  // more than PER partials per group
+        const float4 o = __ldcg(osrc + sp * (PART_FLOATS / 4));
+        const float w = sm_m[sp * 8 + qc];
+        acc.x = fmaf(w, o.x, acc.x);
+        acc.y = fmaf(w, o.y, acc.y);
+        acc.z = fmaf(w, o.z, acc.z);
+        acc.w = fmaf(w, o.w, acc.w);
+      }
+      red4[grp * items + it0] = acc;
+    }
+    consumer_bar();
+    for (int it = threadIdx.x; it < items; it += NTHR) {
+      float4 acc = red4[it];
+      for (int g2 = 1; g2 < ngrp; ++g2) {
+        const float4 o = red4[g2 * items + it];
+        acc.x += o.x;
+        acc.y += o.y;
+        acc.z += o.z;
+        acc.w += o.w;
+      }
+      const int qc = it / (D / 4), d4 = it % (D / 4);
+      const float inv = sm_inv[qc];
+      __half2* dst = reinterpret_cast<__half2*>(out + (static_cast<size_t>(b) * c.Hq + kvh * G + qc) * D) + 2 * d4;
+      dst[0] = __floats2half2_rn(acc.x * inv, acc.y * inv);
+      dst[1] = __floats2half2_rn(acc.z * inv, acc.w * inv);
+    }
+    // every CTA of this unit has consumed its tiles: append the new token to
+    // the ring (slot T % R) and this group's queries to the query buffer
+    if (app_dst[0]) *app_dst[0] = app[0];
+    if (app_dst[1]) *app_dst[1] = app[1];
+    if (threadIdx.x == 0) tickets[1 + u] = 0u;
+  }
+  // (D) scratch and warp states no longer read: give the held stages back (the
+  // generic-proxy writes to them are ordered before the producer's next bulk copy)
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  consumer_bar();
+}
+
 __global__ void __launch_bounds__(NTHREADS, 1)
 decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* __restrict__ k_new,
               const uint16_t* __restrict__ v_new, uint16_t* __restrict__ out, float qscale,
@@ -585,7 +881,7 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
   __shared__ int s_timeout;          // a bounded wait gave up somewhere in this CTA
   __shared__ int s_issued[NSTAGES];  // tiles issued into each stage
   __shared__ int s_held[NC];         // stage holding each consumer warp's state at a segment end (-1: none)
-  __shared__ int s_last;
+  __shared__ int s_last, s_glast;
 
   const int G = c.Hq / c.Hkv;
   const int R = ring_len(c.W);
@@ -605,7 +901,17 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
   // L2 with this range's pages and VL rows: a prefetch is a hint, the ranges
   // are clamped to the buffers, so a stale plan costs bandwidth, never
   // correctness.
-  make_plan(c, R, plan, red, true);
+  // the plan: unit-aligned splits for few units, stream-K ranges for many
+  const bool aligned = c.B * c.Hkv * 4 <= static_cast<int>(gridDim.x);
+  __shared__ AlignedSnap snap;
+  if (aligned) {
+    aligned_snapshot(c, R, snap, true);
+    __syncthreads();
+    if (threadIdx.x == 0) aligned_assign(c, plan, snap);
+    __syncthreads();
+  } else {
+    make_plan(c, R, plan, red, true);
+  }
   if (warp == NC) {
     for (int si = 0; si < plan.nseg; ++si) {
       const Seg s = plan.seg[si];
@@ -633,7 +939,17 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
   griddep_wait();
   griddep_launch_dependents();
   __syncthreads();  // the stale plan is no longer read
-  make_plan(c, R, plan, red, false);
+  if (aligned) {
+    // the plan made before the wait stands unless a length it used changed
+    if (aligned_changed(c, snap)) {
+      aligned_snapshot(c, R, snap, false);
+      __syncthreads();
+      if (threadIdx.x == 0) aligned_assign(c, plan, snap);
+      __syncthreads();
+    }
+  } else {
+    make_plan(c, R, plan, red, false);
+  }
   if (blockIdx.x == 0) {  // sequences that take no step are flagged (once)
     for (int b = threadIdx.x; b < c.B; b += NTHREADS) {
       int32_t* st = state_row(c, b);
@@ -644,7 +960,14 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
   const int ntile = plan.ntile, nseg = plan.nseg;
 
   if (ntile == 0) {
-    // no tiles for this CTA: it only takes its grid ticket below
+    // no tiles for this CTA: it only takes its grid ticket
+    if (threadIdx.x == 0) {
+      fence_acq_rel_gpu();
+      s_glast = atomicAdd(&tickets[0], 1u) == gridDim.x - 1;
+      if (s_glast) fence_acq_rel_gpu();
+    }
+    __syncthreads();
+    if (s_glast) advance_lengths(c, threadIdx.x, NTHREADS, tickets);
   } else if (warp == NC) {
     // ---------------------------------------------------------------- producer
     // lane s owns stage s and issues tiles s, s + NSTAGES, s + 2 NSTAGES, ...
@@ -689,7 +1012,6 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- consumers
-    const int NTHR = NC * 32;
     for (int si = 0; si < nseg; ++si) {
       const Seg sg = plan.seg[si];
       const int u = sg.u, b = u / c.Hkv, kvh = u % c.Hkv;
@@ -751,172 +1073,7 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
         }
       }
       if (lane == 0) s_held[warp] = held;
-      consumer_bar();  // (A) warp states visible
-      // ------------------------------------------------------------ CTA merge -> segment partial
-      // each thread owns 4 dims of one query and weighs the warp states itself
-      const int c_slot = blockIdx.x + u;  // partial slot of (this CTA, unit u)
-      float* part = parts + static_cast<size_t>(c_slot) * PART_FLOATS;
-      // scratch for the unit merge: a held stage (every segment has a tile, so some
-      // warp holds one unless a wait timed out; then stage 0, which stays in bounds)
-      int scratch = 0;
-      for (int w = NC - 1; w >= 0; --w)
-        if (s_held[w] >= 0) scratch = s_held[w];
-      for (int it = threadIdx.x; it < 8 * D / 4; it += NTHR) {
-        const int qc = (4 * it) / D;
-        float mm = -INFINITY;
-        for (int w = 0; w < NC; ++w)
-          if (s_held[w] >= 0) mm = fmaxf(mm, reinterpret_cast<const float*>(smem + s_held[w] * STAGE_BYTES)[qc]);
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        float ll = 0.f;
-        for (int w = 0; w < NC; ++w) {
-          if (s_held[w] < 0) continue;
-          const float* wsm = reinterpret_cast<const float*>(smem + s_held[w] * STAGE_BYTES);
-          const float mw = wsm[qc];
-          const float wt = mw == -INFINITY ? 0.f : ex2(mw - mm);
-          const float4 o = reinterpret_cast<const float4*>(wsm + 16)[it];
-          acc.x = fmaf(wt, o.x, acc.x);
-          acc.y = fmaf(wt, o.y, acc.y);
-          acc.z = fmaf(wt, o.z, acc.z);
-          acc.w = fmaf(wt, o.w, acc.w);
-          ll = fmaf(wt, wsm[8 + qc], ll);
-        }
-        reinterpret_cast<float4*>(part + 16)[it] = acc;
-        if ((4 * it) % D == 0) {
-          part[qc] = mm;
-          part[8 + qc] = ll;
-        }
-      }
-      // the new token's K / V rows and this group's queries, loaded now so that the
-      // append after the ticket is stores only (inputs: no ordering concerns)
-      const int T = ug.T;
-      const int slot = T % R;
-      const int bh = u;
-      constexpr int APPEND_MAX = (2 + HQ_MAX_GQA) * (D / 8);
-      static_assert(APPEND_MAX <= 2 * NC * 32, "at most two 16-byte chunks of the append per consumer thread");
-      uint4 app[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
-      uint4* app_dst[2] = {nullptr, nullptr};
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const int e = threadIdx.x + k * NTHR;
-        if (e < (2 + G) * (D / 8)) {
-          const int row = e / (D / 8), ch = e % (D / 8);
-          if (row < 2) {
-            app[k] = reinterpret_cast<const uint4*>((row ? v_new : k_new) + static_cast<size_t>(bh) * D)[ch];
-            app_dst[k] = reinterpret_cast<uint4*>((row ? c.vr : c.kr) + (static_cast<size_t>(bh) * R + slot) * D) + ch;
-          } else {
-            const size_t h = static_cast<size_t>(b) * c.Hq + kvh * G + (row - 2);
-            app[k] = reinterpret_cast<const uint4*>(q + h * D)[ch];
-            app_dst[k] = reinterpret_cast<uint4*>(c.qbuf + (h * HQ_QBUF + (T % HQ_QBUF)) * D) + ch;
-          }
-        }
-      }
-      // completion ticket of the unit: the barrier orders every thread's partial
-      // writes before thread 0's gpu-scope release; the last CTA acquires before
-      // the barrier that releases its other threads to read the partials
-      consumer_bar();  // (B) partial written, warp states read
-      if (threadIdx.x == 0) {
-        fence_acq_rel_gpu();
-        const unsigned int th = atomicAdd(&tickets[1 + u], 1u);
-        s_last = th == static_cast<unsigned>(sg.ncta - 1);
-        if (s_last) fence_acq_rel_gpu();
-      }
-      consumer_bar();  // (C)
-      if (s_last) {
-        // log-sum-exp merge of the unit's partials (slots first_cta + u ..), in the
-        // scratch stage.  The threads split into ngrp groups, each summing the O
-        // partials of every ngrp-th CTA for one (query, 4 dims) item; a thread's
-        // first PER O loads are issued before the (m, l) of the partials are
-        // gathered and weighed, so both round trips to L2 overlap.
-        const int S = sg.ncta;
-        const float* pb = parts + static_cast<size_t>(sg.first_cta + u) * PART_FLOATS;
-        float* sm_m = reinterpret_cast<float*>(smem + scratch * STAGE_BYTES);  // [S][8] weights
-        float* sm_inv = sm_m + 8 * S;                                          // [8]
-        float4* red4 = reinterpret_cast<float4*>(sm_inv + 8);                  // [ngrp][items]
-        constexpr int PER = 8;
-        const int items = G * (D / 4);
-        const int room = (STAGE_BYTES - 4 * (8 * S + 8)) / (16 * items);      // groups the scratch stage holds
-        const int ngrp = max(1, min(min(NTHR / items, S), room));
-        const int grp = threadIdx.x / items;
-        const int it0 = threadIdx.x - grp * items;
-        const bool mine = grp < ngrp;
-        const float4* osrc = reinterpret_cast<const float4*>(pb + 16 + (it0 / (D / 4)) * D) + it0 % (D / 4);
-        float4 ov[PER];
-#pragma unroll
-        for (int j = 0; j < PER; ++j) {
-          const int sp = grp + j * ngrp;
-          ov[j] = (mine && sp < S) ? __ldcg(osrc + sp * (PART_FLOATS / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        // partial weights: warp qc weighs query qc's partials, lane s holding s, s + 32, ...
-        for (int qc = warp; qc < G; qc += NC) {
-          float mm = -INFINITY;
-          for (int sp = lane; sp < S; sp += 32) mm = fmaxf(mm, __ldcg(pb + sp * PART_FLOATS + qc));
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, o));
-          float ll = 0.f;
-          for (int sp = lane; sp < S; sp += 32) {
-            const float m0 = __ldcg(pb + sp * PART_FLOATS + qc);
-            const float w0 = m0 == -INFINITY ? 0.f : ex2(m0 - mm);
-            ll = fmaf(w0, __ldcg(pb + sp * PART_FLOATS + 8 + qc), ll);
-            sm_m[sp * 8 + qc] = w0;
-          }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) ll += __shfl_xor_sync(0xffffffffu, ll, o);
-          if (lane == 0) {
-            sm_inv[qc] = ll > 0.f ? 1.0f / ll : 0.f;
-            if (c.qlse != nullptr)  // the query's log-sum-exp (base 2), kept for the next reselection
-              c.qlse[(static_cast<size_t>(b) * c.Hq + kvh * G + qc) * HQ_QBUF + (T % HQ_QBUF)] =
-                  lse_ok ? mm + __log2f(ll) : __int_as_float(0x7fc00000);
-          }
-        }
-        consumer_bar();
-        if (mine) {
-          const int qc = it0 / (D / 4);
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-          for (int j = 0; j < PER; ++j) {
-            const int sp = grp + j * ngrp;
-            const float w = sp < S ? sm_m[sp * 8 + qc] : 0.f;
-            acc.x = fmaf(w, ov[j].x, acc.x);
-            acc.y = fmaf(w, ov[j].y, acc.y);
-            acc.z = fmaf(w, ov[j].z, acc.z);
-            acc.w = fmaf(w, ov[j].w, acc.w);
-          }
-          for (int sp = grp + PER * ngrp; sp < S; sp += ngrp) {  // more than PER partials per group
-            const float4 o = __ldcg(osrc + sp * (PART_FLOATS / 4));
-            const float w = sm_m[sp * 8 + qc];
-            acc.x = fmaf(w, o.x, acc.x);
-            acc.y = fmaf(w, o.y, acc.y);
-            acc.z = fmaf(w, o.z, acc.z);
-            acc.w = fmaf(w, o.w, acc.w);
-          }
-          red4[grp * items + it0] = acc;
-        }
-        consumer_bar();
-        for (int it = threadIdx.x; it < items; it += NTHR) {
-          float4 acc = red4[it];
-          for (int g2 = 1; g2 < ngrp; ++g2) {
-            const float4 o = red4[g2 * items + it];
-            acc.x += o.x;
-            acc.y += o.y;
-            acc.z += o.z;
-            acc.w += o.w;
-          }
-          const int qc = it / (D / 4), d4 = it % (D / 4);
-          const float inv = sm_inv[qc];
-          __half2* dst = reinterpret_cast<__half2*>(out + (static_cast<size_t>(b) * c.Hq + kvh * G + qc) * D) + 2 * d4;
-          dst[0] = __floats2half2_rn(acc.x * inv, acc.y * inv);
-          dst[1] = __floats2half2_rn(acc.z * inv, acc.w * inv);
-        }
-        // every CTA of this unit has consumed its tiles: append the new token to
-        // the ring (slot T % R) and this group's queries to the query buffer
-        if (app_dst[0]) *app_dst[0] = app[0];
-        if (app_dst[1]) *app_dst[1] = app[1];
-        if (threadIdx.x == 0) tickets[1 + u] = 0u;
-      }
-      // (D) scratch and warp states no longer read: give the held stages back (the
-      // generic-proxy writes to them are ordered before the producer's next bulk copy)
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      consumer_bar();
+      segment_epilogue(c, q, k_new, v_new, out, parts, tickets, lse_ok, smem, s_held, &s_last, &s_glast, sg, ug, si, nseg);
       if (held >= 0 && lane == 0) mbar_arrive(&empty[held]);
     }
   }
@@ -928,27 +1085,6 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
       for (int st = 0; st < NSTAGES; ++st)
         if (s_issued[st] > 0) mbar_wait(&full[st], (s_issued[st] - 1) & 1, state_row(c, 0));
     __syncthreads();
-  }
-  // The last CTA of the grid advances the lengths.  Every CTA planned from the
-  // state rows, so no T may change before all of them have (a sequence's T
-  // decides whether it takes a step): the grid ticket orders the update after
-  // every CTA's plan and every unit's append.
-  if (threadIdx.x == 0) {
-    fence_acq_rel_gpu();
-    s_last = atomicAdd(&tickets[0], 1u) == gridDim.x - 1;
-    if (s_last) fence_acq_rel_gpu();
-  }
-  __syncthreads();
-  if (s_last) {
-    for (int b = threadIdx.x; b < c.B; b += NTHREADS) {
-      int32_t* st = state_row(c, b);
-      const int T = st[HQ_STATE_T];
-      if (!refused(c, T, st[HQ_STATE_NPACKED])) {
-        st[HQ_STATE_T] = T + 1;
-        st[HQ_STATE_NQ] = min(st[HQ_STATE_NQ] + 1, HQ_QBUF);
-      }
-    }
-    if (threadIdx.x == 0) tickets[0] = 0u;
   }
 }
 
@@ -964,8 +1100,6 @@ size_t decode_workspace(const hq_cache& c, int sms) {
 
 bool decode_supported(const hq_cache& c) { return c.B * c.Hkv <= MAX_UNITS; }
 
-// one CTA per SM, at most MAX_CTAS (the unit merge keeps one weight per CTA in a stage)
-constexpr int MAX_CTAS = 160;
 
 hq_status launch_decode(const hq_cache& c, const uint16_t* q, const uint16_t* kn, const uint16_t* vn, uint16_t* out,
                         float sm_scale, void* ws, int sms, cudaStream_t st) {
