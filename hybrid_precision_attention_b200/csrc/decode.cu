@@ -398,8 +398,6 @@ struct WarpState {
 };
 
 // Online-softmax update for NMT 16-key blocks whose S^T accumulators are in s.
-// Returns the P^T B-fragments (two per block) in pb.
-// Online-softmax update for NMT 16-key blocks whose S^T accumulators are in s.
 // Returns the P^T B-fragments (two per block) in pb.  The running max moves
 // lazily: only when a query's tile max exceeds it by more than LAZY_MAX (log2
 // units), so most tiles skip the rescale of O and l; p then stays below
@@ -414,13 +412,16 @@ __device__ __forceinline__ void softmax_update(WarpState& ws, float (&s)[NMT][4]
     mx0 = fmaxf(mx0, fmaxf(s[i][0], s[i][2]));
     mx1 = fmaxf(mx1, fmaxf(s[i][1], s[i][3]));
   }
+  // the running max only has to move when some logit exceeds it by more than
+  // LAZY_MAX: one vote on the thread-local maxima decides, and the reduction
+  // over the query column's 8 lanes runs only then (rarely after the first tile)
+  if (__any_sync(0xffffffffu, mx0 > ws.m[0] + LAZY_MAX || mx1 > ws.m[1] + LAZY_MAX)) {
 #pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-  }
-  const bool up0 = mx0 > ws.m[0] + LAZY_MAX, up1 = mx1 > ws.m[1] + LAZY_MAX;
-  if (__any_sync(0xffffffffu, up0 || up1)) {
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    const bool up0 = mx0 > ws.m[0] + LAZY_MAX, up1 = mx1 > ws.m[1] + LAZY_MAX;
     // exp2(-inf) = 0 when the old max is -inf (O and l are still zero then)
     const float c0 = up0 ? ex2(ws.m[0] - mx0) : 1.f, c1 = up1 ? ex2(ws.m[1] - mx1) : 1.f;
     ws.m[0] = up0 ? mx0 : ws.m[0];
