@@ -17,7 +17,8 @@ key j of query i is
 * a window key when ``i - W < j <= i``      -> FP16 Q, K, V;
 * else a vertical-line key when j is in the set -> FP16 Q, K, V;
 * else a quantised key                     -> FP8 e4m3 Q, K, V with per-block
-  scales (see ``formats``);
+  scales (see ``formats``), or, with ``qk_format="int8"`` (the README's
+  INT8-QK / FP16-PV kernels), INT8 Q and K with per-block scales and FP16 V;
 
 and a single softmax covers all three classes.  A vertical-line key inside a
 query's window is counted once, as a window key.  The oracle keeps the
@@ -63,25 +64,36 @@ def attend_loops(q, keys, vals, sm_scale):
     return out
 
 
-def prefill_head(q16, k16, v16, is_vl, W: int, sm_scale: float, rows=None, qt=None, kt=None, vt=None):
+def low_precision(x16, fmt: str):
+    """The real values a quantised tile holds for x16 [..., L, D] (float64): e4m3
+    or int8 codes times their per-block scales."""
+    if fmt == "int8":
+        s = formats.int8_block_scales(x16)
+        return formats.fp8_dequant(formats.int8_quantize(x16, s), s)
+    s = formats.fp8_block_scales(x16)
+    return formats.fp8_dequant(formats.fp8_quantize(x16, s), s)
+
+
+def prefill_head(q16, k16, v16, is_vl, W: int, sm_scale: float, rows=None, qt=None, kt=None, vt=None,
+                 qk_format: str = "e4m3"):
     """Hybrid causal prefill for one query head against its kv head.
 
     q16 [L, D], k16/v16 [L, D] float16; is_vl [L] bool (vertical-line keys).
-    ``qt/kt/vt`` are the FP8-represented real values (float64); computed from
-    the FP16 inputs when not given.  Returns float64 [len(rows), D].
+    ``qt/kt/vt`` are the low-precision real values (float64) of the quantised
+    tiles, computed from the FP16 inputs when not given: e4m3 Q, K, V, or with
+    ``qk_format="int8"`` INT8 Q, K and FP16 V.  Returns float64 [len(rows), D].
     """
+    assert qk_format in ("e4m3", "int8")
     L = k16.shape[0]
     if rows is None:
         rows = np.arange(L)
     rows = np.asarray(rows, np.int64)
     if qt is None:
-        qt = formats.fp8_dequant(formats.fp8_quantize(q16, formats.fp8_block_scales(q16)), formats.fp8_block_scales(q16))
+        qt = low_precision(q16, qk_format)
     if kt is None:
-        sk = formats.fp8_block_scales(k16)
-        kt = formats.fp8_dequant(formats.fp8_quantize(k16, sk), sk)
+        kt = low_precision(k16, qk_format)
     if vt is None:
-        sv = formats.fp8_block_scales(v16)
-        vt = formats.fp8_dequant(formats.fp8_quantize(v16, sv), sv)
+        vt = low_precision(v16, "e4m3") if qk_format == "e4m3" else np.asarray(v16, np.float64)
     q64 = q16.astype(np.float64)
     k64 = k16.astype(np.float64)
     v64 = v16.astype(np.float64)
@@ -105,7 +117,7 @@ def prefill_head(q16, k16, v16, is_vl, W: int, sm_scale: float, rows=None, qt=No
     return out
 
 
-def prefill_ref(Q, K, V, vl_pos, W: int, sm_scale: float, rows=None, heads=None):
+def prefill_ref(Q, K, V, vl_pos, W: int, sm_scale: float, rows=None, heads=None, qk_format: str = "e4m3"):
     """Hybrid causal prefill, float64.
 
     Q [B, Hq, L, D], K/V [B, Hkv, L, D] float16; vl_pos[b][h] = vertical-line
@@ -123,15 +135,13 @@ def prefill_ref(Q, K, V, vl_pos, W: int, sm_scale: float, rows=None, heads=None)
     for (b, hq) in heads:
         kvh = hq // G
         if (b, kvh) not in cache:
-            sk = formats.fp8_block_scales(K[b, kvh])
-            sv = formats.fp8_block_scales(V[b, kvh])
-            kt = formats.fp8_dequant(formats.fp8_quantize(K[b, kvh], sk), sk)
-            vt = formats.fp8_dequant(formats.fp8_quantize(V[b, kvh], sv), sv)
+            kt = low_precision(K[b, kvh], qk_format)
+            vt = low_precision(V[b, kvh], "e4m3") if qk_format == "e4m3" else V[b, kvh].astype(np.float64)
             is_vl = np.zeros(L, dtype=bool)
             is_vl[np.asarray(vl_pos[b][kvh], np.int64)] = True
             cache = {(b, kvh): (kt, vt, is_vl)}
         kt, vt, is_vl = cache[(b, kvh)]
-        sq = formats.fp8_block_scales(Q[b, hq])
-        qt = formats.fp8_dequant(formats.fp8_quantize(Q[b, hq], sq), sq)
-        out[(b, hq)] = prefill_head(Q[b, hq], K[b, kvh], V[b, kvh], is_vl, W, sm_scale, rows=rows, qt=qt, kt=kt, vt=vt)
+        qt = low_precision(Q[b, hq], qk_format)
+        out[(b, hq)] = prefill_head(Q[b, hq], K[b, kvh], V[b, kvh], is_vl, W, sm_scale, rows=rows, qt=qt, kt=kt, vt=vt,
+                                    qk_format=qk_format)
     return out

@@ -22,7 +22,9 @@ definition written out:
 
 FP8 e4m3 (prefill's quantised tiles; HyQuant README, Overview item 2: most of
 prefill's attention matrix products use a low-precision format such as INT8
-or FP8).  The
+or FP8).  INT8 (the README's INT8-QK kernels): symmetric per block of 128
+positions, ``scale = fp32(amax) / 127`` (1 when amax is 0), a value stored as
+``clamp(rint_even(fp32(x) / scale), -127, 127)`` with a float32 RN divide.  The
 rounding below is written from the OCP 8-bit floating point specification
 (E4M3: bias 7, 3 mantissa bits, no infinities, largest finite 448, smallest
 subnormal 2^-9), round-to-nearest-even with saturation to +-448.  Per-block
@@ -209,3 +211,29 @@ def fp8_dequant(x8: np.ndarray, scales: np.ndarray, block: int = FP8_BLOCK) -> n
     L = x8.shape[-2]
     s = np.repeat(scales.astype(np.float64), block, axis=-1)[..., :L]
     return x8 * s[..., None]
+
+
+# --------------------------------------------------------------------------- INT8 (symmetric, per block)
+
+INT8_MAX = 127.0
+
+
+def int8_block_scales(x16: np.ndarray, block: int = FP8_BLOCK) -> np.ndarray:
+    """Per-block scales for x16 [..., L, D]: float32 [..., ceil(L / block)], amax / 127 (1 when amax is 0)."""
+    x = np.asarray(x16, dtype=np.float16)
+    L = x.shape[-2]
+    nb = (L + block - 1) // block
+    scales = np.empty(x.shape[:-2] + (nb,), dtype=np.float32)
+    for i in range(nb):
+        amax = np.abs(x[..., i * block:(i + 1) * block, :]).max(axis=(-1, -2)).astype(np.float32)
+        scales[..., i] = np.where(amax == 0, np.float32(1.0), amax / np.float32(INT8_MAX))   # float32 RN
+    return scales
+
+
+def int8_quantize(x16: np.ndarray, scales: np.ndarray, block: int = FP8_BLOCK) -> np.ndarray:
+    """INT8 codes (as float64 integers) of ``fp32(x) / scale`` for x16 [..., L, D]."""
+    x = np.asarray(x16, dtype=np.float16).astype(np.float32)
+    L = x.shape[-2]
+    s = np.repeat(scales, block, axis=-1)[..., :L].astype(np.float32)
+    r = np.rint((x / s[..., None]).astype(np.float32))                 # float32 RN divide, ties to even
+    return np.clip(r, -INT8_MAX, INT8_MAX).astype(np.float64)

@@ -206,3 +206,42 @@ def test_code_widths_strict_mode_and_error_order():
         errs[(kb, vb)] = outs
     e = {key: _mse(v, full) for key, v in errs.items()}
     assert e[(8, 8)] < e[(4, 4)] < e[(4, 2)] and e[(4, 4)] < e[(2, 4)]
+
+
+def test_prefill_int8_qk_format():
+    """INT8-QK / FP16-PV (README: INT8 Q.K with FP16 P.V): per-(i, j) loops on a
+    tiny case; without window or lines it is causal SDPA over the INT8 values
+    of Q and K with V in FP16; with W >= L it is exact FP16 attention."""
+    rng = np.random.default_rng(12)
+    L = 16
+    q, k, v = [(rng.standard_normal((L, 128)) * 2).astype(np.float16) for _ in range(3)]
+    is_vl = np.zeros(L, bool); is_vl[[1, 7]] = True
+    qt = attention.low_precision(q, "int8"); kt = attention.low_precision(k, "int8")
+    for W in (0, 4):
+        got = attention.prefill_head(q, k, v, is_vl, W, SM, qk_format="int8")
+        want = np.zeros((L, 128))
+        for i in range(L):
+            lg, vals = [], []
+            for j in range(i + 1):
+                fp = j > i - W or is_vl[j]
+                lg.append(float((q[i].astype(np.float64) @ k[j].astype(np.float64)) if fp else (qt[i] @ kt[j])) * SM)
+                vals.append(v[j].astype(np.float64))
+            w = np.exp(np.array(lg) - max(lg))
+            want[i] = (w[:, None] * np.array(vals)).sum(0) / w.sum()
+        assert np.allclose(got, want, rtol=1e-11, atol=1e-13), W
+    L = 300
+    q, k, v = [rng.standard_normal((L, 128)).astype(np.float16) for _ in range(3)]
+    none = np.zeros(L, bool)
+    got = attention.prefill_head(q, k, v, none, 0, SM, qk_format="int8")
+    f = lambda x: attention.low_precision(x, "int8")
+    assert np.allclose(got, _sdpa(f(q), f(k), v, causal=True), rtol=1e-11, atol=1e-13)
+    assert np.allclose(attention.prefill_head(q, k, v, none, L, SM, qk_format="int8"), _sdpa(q, k, v, causal=True),
+                       rtol=1e-11, atol=1e-13)
+    # INT8 keeps more of Q.K than e4m3: lower error against exact attention on the planted generator
+    lay = synth.planted_layer(13, 1, 4, 1, 1024)
+    Q = synth.full_queries(13, 1, 4, 1, 1024)
+    ref = _sdpa(Q[0, 0], lay.k[0, 0], lay.v[0, 0], causal=True)
+    none = np.zeros(1024, bool)
+    e8 = _mse(attention.prefill_head(Q[0, 0], lay.k[0, 0], lay.v[0, 0], none, 0, SM, qk_format="e4m3"), ref)
+    ei = _mse(attention.prefill_head(Q[0, 0], lay.k[0, 0], lay.v[0, 0], none, 0, SM, qk_format="int8"), ref)
+    assert ei < e8

@@ -238,3 +238,39 @@ def test_bits_four_is_k4v4_and_sizes():
     for bits in (2, 4, 8):
         c, s, z = formats.pack_bits(x, bits)
         assert c.shape == (3, 128 * bits // 8) and s.shape == z.shape == (3, 4)
+
+
+# ------------------------------------------------------------------ INT8 (prefill's INT8-QK format)
+
+def test_int8_block_hand_examples():
+    """Worked by hand: a block whose amax is 127 has scale exactly 1, so codes
+    are the values rounded half to even; a block with amax 254 has scale 2."""
+    x = np.zeros((128, 128), np.float16)
+    x[0, :8] = [0.5, 1.5, 2.5, -0.5, -1.5, 127, -127, 3.25]
+    s = formats.int8_block_scales(x)
+    assert s.tolist() == [1.0]
+    q = formats.int8_quantize(x, s)
+    assert q[0, :8].tolist() == [0, 2, 2, 0, -2, 127, -127, 3]
+    y = np.zeros((200, 128), np.float16)
+    y[5, 3] = 254
+    y[6, 0:4] = [3, 5, -7, 1]
+    y[150, 0] = -2.0                        # second block: amax 2, scale 2/127
+    s = formats.int8_block_scales(y)
+    assert s[0] == 2.0 and s[1] == np.float32(2.0) / np.float32(127.0)
+    q = formats.int8_quantize(y, s)
+    assert q[6, 0:4].tolist() == [2, 2, -4, 0] and q[5, 3] == 127 and q[150, 0] == -127
+    assert formats.int8_block_scales(np.zeros((10, 128), np.float16)).tolist() == [1.0]
+
+
+def test_int8_codes_are_nearest_and_bounded():
+    rng = np.random.default_rng(9)
+    x = (rng.standard_normal((300, 128)) * rng.uniform(0.1, 50, (300, 1))).astype(np.float16)
+    s = formats.int8_block_scales(x)
+    q = formats.int8_quantize(x, s)
+    assert np.all(np.abs(q) <= 127) and np.all(q == np.round(q))
+    for blk in range(len(s)):
+        rows = slice(128 * blk, 128 * (blk + 1))
+        r = x[rows].astype(np.float64) / float(s[blk])
+        assert np.all(np.abs(q[rows] - r) <= 0.5 + 1e-5)
+        amax = np.abs(x[rows]).max()
+        assert np.abs(q[rows]).max() == 127 or amax == 0
