@@ -112,7 +112,7 @@ def prefill_flops(L, Hq, D=128):
     return 4.0 * D * Hq * L * (L + 1) / 2
 
 
-def run_prefill(dev, reps=5, warmup=2):
+def run_prefill(dev, reps=5, warmup=2, qk_format=0):
     """Time hq_prefill_attn on the 32K layer (B=1, Hq=32, Hkv=8, W=128, 5 % vertical lines chosen
     from the column mass of the last 64 queries); returns the JSON object of the prefill leg."""
     import torch
@@ -130,12 +130,12 @@ def run_prefill(dev, reps=5, warmup=2):
     out = torch.empty_like(q_d)
     ws = torch.empty(hq.hq_prefill_workspace_bytes(1, PF_HQ, PF_HKV, PF_L, vl.shape[2]), dtype=torch.uint8, device=dev)
     for _ in range(warmup):
-        hq.hq_prefill_attn(q_d, k_d, v_d, vl, n_vl, W, out=out, ws=ws)
+        hq.hq_prefill_attn(q_d, k_d, v_d, vl, n_vl, W, out=out, ws=ws, qk_format=qk_format)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(reps):
-        hq.hq_prefill_attn(q_d, k_d, v_d, vl, n_vl, W, out=out, ws=ws)
+        hq.hq_prefill_attn(q_d, k_d, v_d, vl, n_vl, W, out=out, ws=ws, qk_format=qk_format)
     e1.record()
     torch.cuda.synchronize()
     err = int(ws[:4].cpu().numpy().view(np.uint32)[0])
@@ -145,12 +145,15 @@ def run_prefill(dev, reps=5, warmup=2):
     tflops = flops / (ms * 1e-3) / 1e12
     bf16, kind = load_bf16_peak()
     extra = load_extra_peaks()
-    if "fp8_e4m3_tflops" in extra:
-        fp8, fp8_kind = float(extra["fp8_e4m3_tflops"]), "measured e4m3 GEMM (profiles/peaks_b200.json)"
+    key, name = ("int8_tops", "INT8") if qk_format == 1 else ("fp8_e4m3_tflops", "e4m3")
+    if key in extra:
+        fp8, fp8_kind = float(extra[key]), f"measured {name} GEMM (profiles/peaks_b200.json)"
     else:
         fp8, fp8_kind = 2.0 * bf16, f"{kind} bf16 x 2 (nominal fp8/bf16 ratio)"
     mixed = 1.0 / (0.5 / fp8 + 0.5 / bf16)
-    return {"workload": f"causal hybrid prefill, B=1, L=32768, Hq=32, Hkv=8, D=128, W=128, rho=5% ({n_vl} lines per kv head)",
+    fmt = "INT8 Q.K + FP16 P.V" if qk_format == 1 else "e4m3 Q.K (P.V on f16 with e4m3 V values)"
+    return {"workload": f"causal hybrid prefill, B=1, L=32768, Hq=32, Hkv=8, D=128, W=128, rho=5% ({n_vl} lines per kv head), "
+                        f"quantised tiles {fmt}",
             "ms": ms, "tflops": tflops, "calls": reps,
             "roofline": {"kernel": "prefill (pre-pass + prefill_kernel)", "bound": "tensor", "achieved": tflops,
                          "peak": fp8, "unit": "TFLOP/s", "frac": tflops / fp8, "traffic": None,
@@ -494,9 +497,10 @@ def run_ours(args, rank, world, local_rank):
                "d2h_bytes_per_step": PERIOD * COPIES * out.numel() * 2,
                "steps": n_e2e, "api": "hq_decode_attn / hq_select_vlines / hq_pack_merge via the Python binding, eager"}
 
-    prefill = None
+    prefill = prefill_int8 = None
     if not args.no_prefill:
         prefill = run_prefill(dev)
+        prefill_int8 = run_prefill(dev, qk_format=1)
 
     working_set_mb = COPIES * caches[0].nbytes() / 1e6
     legs = {}
@@ -545,7 +549,8 @@ def run_ours(args, rank, world, local_rank):
                        "rho": RHO_BP / 10000, "layer_copies": COPIES, "decode_tokens_per_step": PERIOD,
                        "l2": f"{COPIES} rotating layer copies, {working_set_mb:.0f} MB working set > 126 MB L2",
                        "parallelism": f"replicas x{world}"},
-            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "prefill": prefill, "legs": legs,
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "prefill": prefill, "prefill_int8_qk": prefill_int8,
+            "legs": legs,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": sampler.summary()}
     print(json.dumps(line), flush=True)
@@ -771,6 +776,20 @@ def measure_peaks(dev):
         best = min(best, e0.elapsed_time(e1))
     fp8 = 2.0 * n ** 3 / (best * 1e-3) / 1e12
     del a, bt
+    ai = torch.randint(-127, 128, (n, n), device=dev, dtype=torch.int8)
+    bi = torch.randint(-127, 128, (n, n), device=dev, dtype=torch.int8).t()
+    for _ in range(5):
+        torch._int_mm(ai, bi)
+    besti = 1e9
+    for _ in range(20):
+        e0, e1 = _events(2)
+        e0.record()
+        torch._int_mm(ai, bi)
+        e1.record()
+        torch.cuda.synchronize()
+        besti = min(besti, e0.elapsed_time(e1))
+    i8 = 2.0 * n ** 3 / (besti * 1e-3) / 1e12
+    del ai, bi
     buf = torch.ones(8 << 30, dtype=torch.uint8, device=dev)
     sink = torch.zeros(4, dtype=torch.int32, device=dev)
     rd = {}
@@ -788,10 +807,11 @@ def measure_peaks(dev):
         rd[cps] = buf.numel() / (tb * 1e-3) / 1e9
     best_cps = max(rd, key=rd.get)
     rec = {"fp8_e4m3_tflops": fp8, "fp8_how": f"torch._scaled_mm e4m3 x e4m3 -> bf16, {n}^3 (2 n^3 flops), best of 20, CUDA events",
+           "int8_tops": i8, "int8_how": f"torch._int_mm int8 x int8 -> int32, {n}^3 (2 n^3 ops), best of 20, CUDA events",
            "hbm_read_gbs": rd[best_cps], "hbm_read_how": f"hq_diag_stream_read over 8 GiB (16-byte streaming loads, "
                                                          f"{best_cps} CTAs of 512 threads per SM), best of 10, CUDA events",
            "hbm_read_by_ctas_per_sm": rd, "gpu": torch.cuda.get_device_name(dev),
-           "when": datetime.datetime.utcnow().strftime("%Y-%m-%dT%H:%M:%SZ")}
+           "when": datetime.datetime.now(datetime.timezone.utc).strftime("%Y-%m-%dT%H:%M:%SZ")}
     print(json.dumps(rec), flush=True)
 
 

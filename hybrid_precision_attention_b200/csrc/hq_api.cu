@@ -20,8 +20,8 @@ hq_status launch_select(const hq_cache& c, const uint16_t* kd, int L, const uint
                         void* ws, cudaStream_t st);
 size_t prefill_workspace(int B, int Hq, int Hkv, int L, int vl_stride);
 hq_status launch_prefill(int B, int Hq, int Hkv, int L, const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                         const int32_t* vl_pos, int n_vl, int vl_stride, int W, float sm_scale, uint16_t* out, void* ws,
-                         cudaStream_t st);
+                         const int32_t* vl_pos, int n_vl, int vl_stride, int W, int qk_format, float sm_scale,
+                         uint16_t* out, void* ws, cudaStream_t st);
 }  // namespace hq
 
 namespace {
@@ -165,13 +165,15 @@ size_t hq_prefill_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t L,
 
 hq_status hq_prefill_attn(int32_t B, int32_t Hq, int32_t Hkv, int32_t L, int32_t D, const uint16_t* q,
                           const uint16_t* k, const uint16_t* v, const int32_t* vl_pos, int32_t n_vl, int32_t vl_stride,
-                          int32_t W, float sm_scale, uint16_t* out, void* ws, size_t ws_bytes, hq_stream_t stream) {
+                          int32_t W, int32_t qk_format, float sm_scale, uint16_t* out, void* ws, size_t ws_bytes,
+                          hq_stream_t stream) {
+  if (qk_format != HQ_PREFILL_E4M3 && qk_format != HQ_PREFILL_INT8_QK) return HQ_ERR_INVALID;
   if (D != HQ_HEAD_DIM) return HQ_ERR_UNSUPPORTED;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || L <= 0 || W < 0 || !(sm_scale > 0.0f)) return HQ_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return HQ_ERR_INVALID;
   if (n_vl < 0 || n_vl > vl_stride || (n_vl > 0 && !aligned16(vl_pos))) return HQ_ERR_INVALID;
   if (!aligned16(ws) || ws_bytes < hq::prefill_workspace(B, Hq, Hkv, L, vl_stride)) return HQ_ERR_WORKSPACE;
-  return hq::launch_prefill(B, Hq, Hkv, L, q, k, v, vl_pos, n_vl, vl_stride, W, sm_scale, out, ws,
+  return hq::launch_prefill(B, Hq, Hkv, L, q, k, v, vl_pos, n_vl, vl_stride, W, qk_format, sm_scale, out, ws,
                             reinterpret_cast<cudaStream_t>(stream));
 }
 

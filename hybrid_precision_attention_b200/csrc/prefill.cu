@@ -12,7 +12,9 @@
 //   window key  (i - W < j <= i)            : FP16 Q, K, V
 //   VL key      (j in the vertical-line set) : FP16 Q, K, V
 //   other key                                : FP8 e4m3 Q, K, V, one float32 scale per
-//                                              (b, head, 128 positions): x8 = e4m3(x / s)
+//                                              (b, head, 128 positions): x8 = e4m3(x / s);
+//                                              or (INT8-QK format) INT8 Q, K, scale amax / 127,
+//                                              and FP16 V
 // then one softmax over all of them.  A vertical line inside the window counts
 // once, as a window key.
 //
@@ -76,6 +78,7 @@ constexpr int PF_SMEM = SM_USED + 1024;         // + slack for the 1024-byte ali
 constexpr uint32_t TMEM_COLS = 512;             // S_A 0..127, S_B 128..255, O_A 256..383, O_B 384..511
 constexpr uint32_t TM_S = 0, TM_O = 256;
 constexpr uint32_t IDESC_QK = idesc_make(0, 0, 0, TQ, TKEY);   // K-major A and B
+constexpr uint32_t IDESC_QK_I8 = idesc_i8_make(TQ, TKEY);      // INT8 Q.K, s32 accumulate
 constexpr uint32_t IDESC_PV = idesc_make(0, 0, 1, TQ, 128);    // A = P K-major, B = V MN-major
 
 struct Tmaps {
@@ -91,6 +94,7 @@ struct PfArgs {
   const int32_t* vlpos;  // [B*Hkv][nvlp], INT_MAX padded
   uint16_t* out;         // [B, Hq, L, D]
   uint32_t* err;         // device error word
+  int int_qk;            // quantised tiles: INT8 Q.K (s32 in TMEM) and FP16 V, else e4m3 Q, K, V
 };
 
 __device__ __forceinline__ bool waitb(uint64_t* bar, uint32_t parity, uint32_t* err, int* abort_flag) {
@@ -184,6 +188,11 @@ __device__ __forceinline__ float scale_mask32(float (&x)[32], int c0, int t, con
       bv[4 * c4 + 3] = bb.w;
     }
     const int jlim = i - a.W - (t - nF) * TKEY - c0;  // causal limit: local columns c <= jlim
+    if (a.int_qk) {
+      // s32 accumulators: exact to float by the 1.5 * 2^23 bias (|Q.K| < 128 * 127 * 127 < 2^22)
+#pragma unroll
+      for (int c = 0; c < 32; ++c) x[c] = __uint_as_float(__float_as_uint(x[c]) + 0x4B400000u) - 12582912.0f;
+    }
     float m2[2] = {-INFINITY, -INFINITY};
     if (jlim >= 31) {
 #pragma unroll
@@ -378,9 +387,15 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
         const uint32_t K = sm_base + k_stage(st);
         if (t >= nF) {
           const uint32_t q8 = sm_base + SM_Q8 + g * 16384;
+          if (a.int_qk) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_f8(S, sdesc_sw128(q8 + 32 * kk, 16, 1024), sdesc_sw128(K + 32 * kk, 16, 1024), IDESC_QK, kk > 0);
+            for (int kk = 0; kk < 4; ++kk)
+              umma_i8(S, sdesc_sw128(q8 + 32 * kk, 16, 1024), sdesc_sw128(K + 32 * kk, 16, 1024), IDESC_QK_I8, kk > 0);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_f8(S, sdesc_sw128(q8 + 32 * kk, 16, 1024), sdesc_sw128(K + 32 * kk, 16, 1024), IDESC_QK, kk > 0);
+          }
         } else {
           const uint32_t q16 = sm_base + SM_Q16 + g * 32768;
 #pragma unroll
@@ -662,6 +677,59 @@ __global__ void __launch_bounds__(256) fp8_block_quant(const uint16_t* __restric
   }
 }
 
+// INT8 pre-pass (INT8-QK format): one CTA (256 threads) per (128-position
+// block, head, batch) of x [B, H, L, D]: scale = amax / 127 (1 when amax is 0),
+// codes clamp(rint_even(x / scale), -127, 127) [B*H][Lp][D]; rows past L are zero.
+__global__ void __launch_bounds__(256) int8_block_quant(const uint16_t* __restrict__ x, int H, int L, int Lp, int nblk,
+                                                        int8_t* __restrict__ codes, float* __restrict__ scales) {
+  const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const size_t bh = static_cast<size_t>(b) * H + h;
+  const int r0 = blk * 128;
+  __shared__ float red[8];
+  __shared__ float s_scale;
+  float amax = 0.f;
+  for (int e = threadIdx.x; e < 128 * 32; e += 256) {
+    const int row = r0 + (e >> 5), c4 = e & 31;
+    if (row < L) {
+      const uint2 u = reinterpret_cast<const uint2*>(x + (bh * L + row) * D)[c4];
+      amax = fmaxf(amax, fabsf(__half2float(__ushort_as_half(static_cast<unsigned short>(u.x & 0xFFFFu)))));
+      amax = fmaxf(amax, fabsf(__half2float(__ushort_as_half(static_cast<unsigned short>(u.x >> 16)))));
+      amax = fmaxf(amax, fabsf(__half2float(__ushort_as_half(static_cast<unsigned short>(u.y & 0xFFFFu)))));
+      amax = fmaxf(amax, fabsf(__half2float(__ushort_as_half(static_cast<unsigned short>(u.y >> 16)))));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = 0.f;
+    for (int w = 0; w < 8; ++w) m = fmaxf(m, red[w]);
+    const float s = m == 0.f ? 1.0f : __fdiv_rn(m, 127.0f);
+    s_scale = s;
+    scales[bh * nblk + blk] = s;
+  }
+  __syncthreads();
+  const float s = s_scale;
+  for (int e = threadIdx.x; e < 128 * 32; e += 256) {
+    const int row = r0 + (e >> 5), c4 = e & 31;
+    uint32_t packed = 0u;
+    if (row < L) {
+      const uint2 u = reinterpret_cast<const uint2*>(x + (bh * L + row) * D)[c4];
+      const float v[4] = {__half2float(__ushort_as_half(static_cast<unsigned short>(u.x & 0xFFFFu))),
+                          __half2float(__ushort_as_half(static_cast<unsigned short>(u.x >> 16))),
+                          __half2float(__ushort_as_half(static_cast<unsigned short>(u.y & 0xFFFFu))),
+                          __half2float(__ushort_as_half(static_cast<unsigned short>(u.y >> 16)))};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int qv = min(max(__float2int_rn(__fdiv_rn(v[k], s)), -127), 127);
+        packed |= (static_cast<uint32_t>(qv) & 0xFFu) << (8 * k);
+      }
+    }
+    *reinterpret_cast<uint32_t*>(codes + (bh * Lp + row) * D + 4 * c4) = packed;
+  }
+}
+
 // Score bias of the e4m3 key blocks, [B*Hkv][Lp]: 0 for positions < L, -inf past L
 // (vl_prep then marks the vertical lines -inf too: they are read as fp16 tiles).
 __global__ void kbias_init(float* __restrict__ kbias, int L, int Lp, size_t n) {
@@ -765,8 +833,9 @@ size_t prefill_workspace(int B, int Hq, int Hkv, int L, int vl_stride) {
 }
 
 hq_status launch_prefill(int B, int Hq, int Hkv, int L, const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                         const int32_t* vl_pos, int n_vl, int vl_stride, int W, float sm_scale, uint16_t* out, void* ws,
-                         cudaStream_t st) {
+                         const int32_t* vl_pos, int n_vl, int vl_stride, int W, int qk_format, float sm_scale,
+                         uint16_t* out, void* ws, cudaStream_t st) {
+  const bool int_qk = qk_format == HQ_PREFILL_INT8_QK;
   if (n_vl > L || n_vl > vl_stride) return HQ_ERR_INVALID;
   const PfLayout ly = pf_layout(B, Hq, Hkv, L, n_vl);
   char* w = static_cast<char*>(ws);
@@ -784,22 +853,30 @@ hq_status launch_prefill(int B, int Hq, int Hkv, int L, const uint16_t* q, const
 
   Tmaps tm;
   if (!make_map(&tm.q8, q8, false, ly.Lp, B * Hq, 128) || !make_map(&tm.q16, q, true, L, B * Hq, 64) ||
-      !make_map(&tm.k8, k8, false, ly.Lp, B * Hkv, 128) || !make_map(&tm.v8, v8, true, ly.Lp, B * Hkv, 64) ||
+      !make_map(&tm.k8, k8, false, ly.Lp, B * Hkv, 128) ||
+      // quantised tiles' V: e4m3 values stored as fp16, or (INT8-QK) V itself
+      !(int_qk ? make_map(&tm.v8, v, true, L, B * Hkv, 64) : make_map(&tm.v8, v8, true, ly.Lp, B * Hkv, 64)) ||
       !make_map(&tm.k16, k, true, L, B * Hkv, 64) || !make_map(&tm.v16, v, true, L, B * Hkv, 64) ||
       !make_map(&tm.kvl, kvl, true, ly.nvlp, B * Hkv, 64) || !make_map(&tm.vvl, vvl, true, ly.nvlp, B * Hkv, 64))
     return cuda_fail(cudaSuccess, "prefill tensor maps");
 
   if (cudaMemsetAsync(err, 0, 16, st) != cudaSuccess) return cuda_fail(cudaGetLastError(), "prefill setup");
   kbias_init<<<256, 256, 0, st>>>(kbias, L, ly.Lp, static_cast<size_t>(B) * Hkv * ly.Lp);
-  fp8_block_quant<<<dim3(ly.nblk, Hq, B), 256, 0, st>>>(q, Hq, L, ly.Lp, ly.nblk, q8, nullptr, sq);
-  fp8_block_quant<<<dim3(ly.nblk, Hkv, B), 256, 0, st>>>(k, Hkv, L, ly.Lp, ly.nblk, k8, nullptr, sk);
-  fp8_block_quant<<<dim3(ly.nblk, Hkv, B), 256, 0, st>>>(v, Hkv, L, ly.Lp, ly.nblk, nullptr, v8, sv);
+  if (int_qk) {
+    int8_block_quant<<<dim3(ly.nblk, Hq, B), 256, 0, st>>>(q, Hq, L, ly.Lp, ly.nblk, reinterpret_cast<int8_t*>(q8), sq);
+    int8_block_quant<<<dim3(ly.nblk, Hkv, B), 256, 0, st>>>(k, Hkv, L, ly.Lp, ly.nblk, reinterpret_cast<int8_t*>(k8), sk);
+  } else {
+    fp8_block_quant<<<dim3(ly.nblk, Hq, B), 256, 0, st>>>(q, Hq, L, ly.Lp, ly.nblk, q8, nullptr, sq);
+    fp8_block_quant<<<dim3(ly.nblk, Hkv, B), 256, 0, st>>>(k, Hkv, L, ly.Lp, ly.nblk, k8, nullptr, sk);
+    fp8_block_quant<<<dim3(ly.nblk, Hkv, B), 256, 0, st>>>(v, Hkv, L, ly.Lp, ly.nblk, nullptr, v8, sv);
+  }
   vl_prep<<<dim3(ly.nvlp / TKEY, B * Hkv), 256, 0, st>>>(k, v, vl_pos, n_vl, vl_stride, L, ly.Lp, ly.nvlp, kbias, kvl, vvl,
                                                          vlpos);
   PfArgs a;
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.L = L; a.Lp = ly.Lp; a.nblk = ly.nblk; a.W = W; a.n_vl = n_vl; a.nvlp = ly.nvlp;
   a.qk_scale = sm_scale * LOG2E;
   a.sq = sq; a.sk = sk; a.kbias = kbias; a.vlpos = vlpos; a.out = out; a.err = err;
+  a.int_qk = int_qk ? 1 : 0;
   int dev = 0;
   cudaGetDevice(&dev);
   static DeviceOnce attrs;

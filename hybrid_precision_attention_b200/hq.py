@@ -73,7 +73,8 @@ _lib.hq_decode_attn_noalloc.argtypes = [_CP, _P, _P, _P, _P, ctypes.c_float, _P]
 _lib.hq_prefill_workspace_bytes.restype = _S
 _lib.hq_prefill_workspace_bytes.argtypes = [_I, _I, _I, _I, _I, _I]
 _lib.hq_prefill_attn.restype = _I
-_lib.hq_prefill_attn.argtypes = [_I, _I, _I, _I, _I, _P, _P, _P, _P, _I, _I, _I, ctypes.c_float, _P, _P, _S, _P]
+_lib.hq_prefill_attn.argtypes = [_I, _I, _I, _I, _I, _P, _P, _P, _P, _I, _I, _I, _I, ctypes.c_float, _P, _P, _S, _P]
+PREFILL_E4M3, PREFILL_INT8_QK = 0, 1
 
 _lib.hq_diag_stream_read.restype = _I
 _lib.hq_diag_stream_read.argtypes = [_P, _S, _P, _I, _P]
@@ -342,8 +343,10 @@ def prefill_ws_regions(B, Hq, Hkv, L, D=HQ_HEAD_DIM) -> dict:
     return {"err": 0, "q8": q8, "k8": k8, "v16": v8, "Lp": Lp}
 
 
-def hq_prefill_attn(q, k, v, vl_pos, n_vl: int, W: int, sm_scale: float = None, out=None, ws=None, stream=None):
-    """q [B,Hq,L,D], k/v [B,Hkv,L,D] fp16; vl_pos int32 [B,Hkv,stride] (first n_vl ascending)."""
+def hq_prefill_attn(q, k, v, vl_pos, n_vl: int, W: int, sm_scale: float = None, out=None, ws=None, stream=None,
+                    qk_format: int = PREFILL_E4M3):
+    """q [B,Hq,L,D], k/v [B,Hkv,L,D] fp16; vl_pos int32 [B,Hkv,stride] (first n_vl ascending);
+    qk_format PREFILL_E4M3 (e4m3 Q, K, V) or PREFILL_INT8_QK (INT8 Q, K and FP16 V) for the quantised keys."""
     B, Hq, L, D = q.shape
     Hkv = k.shape[1]
     _need(q, torch.float16, (B, Hq, L, D), "q")
@@ -358,7 +361,7 @@ def hq_prefill_attn(q, k, v, vl_pos, n_vl: int, W: int, sm_scale: float = None, 
     if sm_scale is None:
         sm_scale = D ** -0.5
     _check(_lib.hq_prefill_attn(B, Hq, Hkv, L, D, _ptr(q), _ptr(k), _ptr(v), _ptr(vl_pos), n_vl, vl_pos.shape[2], W,
-                                ctypes.c_float(sm_scale), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
+                                qk_format, ctypes.c_float(sm_scale), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
            "hq_prefill_attn")
     return out
 

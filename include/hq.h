@@ -275,9 +275,15 @@ HQ_API hq_status hq_decode_attn(const hq_cache* c, const uint16_t* q, const uint
  * item 2, modes "vquant_vert" / "hybrid_full"): for query i and key j <= i,
  *   j is a window key if i - W < j <= i, else a VL key if j is in vl_pos[b, kvh],
  *   else a quantised key;
- * window and VL keys use FP16 Q, K, V; quantised keys use FP8 e4m3 Q, K, V with
- * one float32 scale per (b, head, 128 positions) (scale = amax / 448, values
- * stored as e4m3_RN_sat(x / scale)); one softmax covers all three classes.
+ * window and VL keys use FP16 Q, K, V; quantised keys use, by qk_format,
+ *   HQ_PREFILL_E4M3:    FP8 e4m3 Q, K, V with one float32 scale per (b, head,
+ *                       128 positions) (scale = amax / 448, values stored as
+ *                       e4m3_RN_sat(x / scale));
+ *   HQ_PREFILL_INT8_QK: INT8 Q, K with one float32 scale per (b, head, 128
+ *                       positions) (scale = amax / 127, codes
+ *                       clamp(rint_even(x / scale), -127, 127)) and FP16 V
+ *                       (README Overview item 2, the INT8-QK / FP16-PV kernels);
+ * one softmax covers all three classes.
  *   q [B, Hq, L, D], k, v [B, Hkv, L, D], out [B, Hq, L, D]: fp16
  *   vl_pos int32 [B, Hkv, vl_stride], first n_vl entries ascending, < L
  *     (0 <= n_vl <= min(vl_stride, L))
@@ -288,16 +294,18 @@ HQ_API hq_status hq_decode_attn(const hq_cache* c, const uint16_t* q, const uint
  *   bytes [0, 4)  uint32 error word, cleared by the call: non-zero when a
  *                 bounded wait of the kernel gave up (never expected; the
  *                 output is then incomplete); read it after synchronising;
- *   e4m3 codes of Q [B, Hq, Lp, D], e4m3 codes of K [B, Hkv, Lp, D],
- *   fp16 values fp16(fp32(e4m3(V / scale)) * scale) of V [B, Hkv, Lp, D],
- *   then the per-block scales and gathered VL rows (internal).
+ *   e4m3 (or INT8) codes of Q [B, Hq, Lp, D], e4m3 (or INT8) codes of K
+ *   [B, Hkv, Lp, D], fp16 values fp16(fp32(e4m3(V / scale)) * scale) of V
+ *   [B, Hkv, Lp, D] (e4m3 format only), then the per-block scales and gathered
+ *   VL rows (internal).
  * Rows past L of the three coded tensors are zero.
  */
 HQ_API size_t hq_prefill_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t L, int32_t D, int32_t vl_stride);
+enum { HQ_PREFILL_E4M3 = 0, HQ_PREFILL_INT8_QK = 1 };
 HQ_API hq_status hq_prefill_attn(int32_t B, int32_t Hq, int32_t Hkv, int32_t L, int32_t D,
                           const uint16_t* q, const uint16_t* k, const uint16_t* v,
                           const int32_t* vl_pos, int32_t n_vl, int32_t vl_stride, int32_t W,
-                          float sm_scale, uint16_t* out, void* ws, size_t ws_bytes,
+                          int32_t qk_format, float sm_scale, uint16_t* out, void* ws, size_t ws_bytes,
                           hq_stream_t stream);
 
 /*

@@ -24,7 +24,7 @@ def lib():
     for name, args in (("hq_select_vlines", [CP, P, I, P, I, P, P, S, P]),
                        ("hq_pack_merge", [CP, P, P, I, P, S, P]),
                        ("hq_decode_attn", [CP, P, P, P, P, F, P, S, P]),
-                       ("hq_prefill_attn", [I, I, I, I, I, P, P, P, P, I, I, I, F, P, P, S, P]),
+                       ("hq_prefill_attn", [I, I, I, I, I, P, P, P, P, I, I, I, I, F, P, P, S, P]),
                        ("hq_prefill_workspace_bytes", [I, I, I, I, I, I]),
                        ("hq_workspace_bytes", [CP, I, I]),
                        ("hq_status_str", [I]),
@@ -108,8 +108,8 @@ def test_prefill_rejections(lib, mem):
     assert lib.hq_prefill_workspace_bytes(1, 32, 8, 1000, 64, 64) == 0
     assert lib.hq_prefill_workspace_bytes(1, 30, 8, 1000, 128, 64) == 0
     s = 1 / math.sqrt(128)
-    pf = lambda B, Hq, Hkv, L, D, n_vl, stride, W, sc, ws, wsb, vl=a, q=a: lib.hq_prefill_attn(
-        B, Hq, Hkv, L, D, q, a, a, vl, n_vl, stride, W, sc, a, ws, wsb, None)
+    pf = lambda B, Hq, Hkv, L, D, n_vl, stride, W, sc, ws, wsb, vl=a, q=a, fmt=0: lib.hq_prefill_attn(
+        B, Hq, Hkv, L, D, q, a, a, vl, n_vl, stride, W, fmt, sc, a, ws, wsb, None)
     assert pf(1, 32, 8, 1000, 64, 0, 0, 128, s, a, need) == UNSUPPORTED   # head size
     assert pf(1, 30, 8, 1000, 128, 0, 0, 128, s, a, need) == INVALID      # Hq not a multiple of Hkv
     assert pf(1, 32, 8, 0, 128, 0, 0, 128, s, a, need) == INVALID         # empty prompt
@@ -119,6 +119,7 @@ def test_prefill_rejections(lib, mem):
     assert pf(1, 32, 8, 1000, 128, 10, 16, 128, s, a, need, vl=None) == INVALID  # lines without positions
     assert pf(1, 32, 8, 1000, 128, 0, 0, 128, s, a, need, q=a + 4) == INVALID    # misaligned Q
     assert pf(1, 32, 8, 1000, 128, 0, 0, 128, s, a, need - 1) == WORKSPACE
+    assert pf(1, 32, 8, 1000, 128, 0, 0, 128, s, a, need, fmt=2) == INVALID         # unknown Q.K format
 
 
 def test_status_strings(lib):

@@ -47,17 +47,20 @@ def _vl_tensor(vl, B, Hkv):
     return t, n
 
 
-def _run(B, Hq, Hkv, L, W, rho_bp, seed, rows=None, heads=None):
+FORMATS = {"e4m3": 0, "int8": 1}   # hq.PREFILL_E4M3, hq.PREFILL_INT8_QK
+
+
+def _run(B, Hq, Hkv, L, W, rho_bp, seed, rows=None, heads=None, fmt="e4m3"):
     H = hq()
     lay = synth.planted_layer(seed, B, Hq, Hkv, L)
     Q = synth.full_queries(seed, B, Hq, Hkv, L)
     G = Hq // Hkv
     vl = _vl_sets(lay.k, Q, W, rho_bp, G)
     vlt, n_vl = _vl_tensor(vl, B, Hkv)
-    out = H.hq_prefill_attn(dev(Q), dev(lay.k), dev(lay.v), dev(vlt), n_vl, W)
+    out = H.hq_prefill_attn(dev(Q), dev(lay.k), dev(lay.v), dev(vlt), n_vl, W, qk_format=FORMATS[fmt])
     torch.cuda.synchronize()
     got = out.float().cpu().numpy().astype(np.float64)
-    ref = oatt.prefill_ref(Q, lay.k, lay.v, vl, W, SM, rows=rows, heads=heads)
+    ref = oatt.prefill_ref(Q, lay.k, lay.v, vl, W, SM, rows=rows, heads=heads, qk_format=fmt)
     return got, ref
 
 
@@ -70,8 +73,9 @@ def _run(B, Hq, Hkv, L, W, rho_bp, seed, rows=None, heads=None):
     (1, 4, 1, 200, 500, 500),     # window longer than the prompt: plain FP16 causal
     (1, 4, 1, 384, 32, 0),        # no vertical lines
 ])
-def test_prefill_matches_oracle(B, Hq, Hkv, L, W, rho):
-    got, ref = _run(B, Hq, Hkv, L, W, rho, seed=L + W)
+@pytest.mark.parametrize("fmt", ["e4m3", "int8"])
+def test_prefill_matches_oracle(B, Hq, Hkv, L, W, rho, fmt):
+    got, ref = _run(B, Hq, Hkv, L, W, rho, seed=L + W, fmt=fmt)
     assert np.all(np.isfinite(got))
     for (b, h), r in ref.items():
         g = got[b, h]
@@ -124,12 +128,37 @@ def test_prefill_fp8_pre_pass_matches_oracle():
             assert not v16[b, h, L:].view(np.uint16).any(), (b, h)
 
 
+def test_prefill_int8_codes_match_oracle():
+    """INT8-QK format: the pre-pass INT8 codes of Q and K are bit-exact against
+    the oracle's per-block rounding (the workspace's code regions)."""
+    H = hq()
+    B, Hq, Hkv, L = 1, 4, 2, 300
+    lay = synth.planted_layer(4, B, Hq, Hkv, L)
+    Q = synth.full_queries(4, B, Hq, Hkv, L)
+    vlt = np.zeros((B, Hkv, 16), np.int32)
+    ws = torch.zeros(H.hq_prefill_workspace_bytes(B, Hq, Hkv, L, 16), dtype=torch.uint8, device="cuda")
+    H.hq_prefill_attn(dev(Q), dev(lay.k), dev(lay.v), dev(vlt), 0, 64, ws=ws, qk_format=1)
+    torch.cuda.synchronize()
+    r = H.prefill_ws_regions(B, Hq, Hkv, L)
+    Lp = r["Lp"]
+    w = ws.cpu().numpy()
+    assert w[:4].view(np.uint32)[0] == 0
+    q8 = w[r["q8"]:r["q8"] + B * Hq * Lp * 128].view(np.int8).reshape(B, Hq, Lp, 128)
+    k8 = w[r["k8"]:r["k8"] + B * Hkv * Lp * 128].view(np.int8).reshape(B, Hkv, Lp, 128)
+    for name, x, got in (("Q", Q, q8), ("K", lay.k, k8)):
+        for h in range(x.shape[1]):
+            want = formats.int8_quantize(x[0, h], formats.int8_block_scales(x[0, h]))
+            assert np.array_equal(got[0, h, :L].astype(np.float64), want), (name, h)
+            assert not got[0, h, L:].any(), (name, h)
+
+
 @pytest.mark.slow
-def test_prefill_full_size_32k():
+@pytest.mark.parametrize("fmt", ["e4m3", "int8"])
+def test_prefill_full_size_32k(fmt):
     """The 32K prefill layer (B=1, Hq=32, Hkv=8): sampled rows of a few heads against the oracle."""
     L = 32768
     rows = np.unique(np.concatenate([np.arange(0, 64, 7), np.linspace(64, L - 1, 40).astype(np.int64), [L - 1]]))
-    got, ref = _run(1, 32, 8, L, 128, 500, seed=0, rows=rows, heads=[(0, 0), (0, 13), (0, 31)])
+    got, ref = _run(1, 32, 8, L, 128, 500, seed=0, rows=rows, heads=[(0, 0), (0, 13), (0, 31)], fmt=fmt)
     for (b, h), r in ref.items():
         g = got[b, h, rows]
         rel = np.linalg.norm(g - r) / np.linalg.norm(r)
