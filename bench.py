@@ -159,8 +159,8 @@ def run_prefill(dev, reps=5, warmup=2, qk_format=0):
                          "peak": fp8, "unit": "TFLOP/s", "frac": tflops / fp8, "traffic": None,
                          "peak_kind": fp8_kind,
                          "mixed_ceiling": mixed,
-                         "note": "QK of quantised tiles on e4m3 (fp8 rate), P.V on f16 (bf16 rate): half the flops at "
-                                 "each rate, so the ceiling of this mix is the mixed_ceiling figure"}}
+                         "note": f"QK of quantised tiles on {name} ({name} rate), P.V on f16 (bf16 rate): half the "
+                                 "flops at each rate, so the ceiling of this mix is the mixed_ceiling figure"}}
 
 
 def decode_traffic_record(bytes_per_launch):

@@ -45,6 +45,28 @@ struct DeviceOnce {
   }
 };
 
+// Page geometry for the cache's code widths (the HQ_PAGE_SUBPOS layout).
+struct PageGeo {
+  int kb, vb;    // code bits of K and V
+  int pr;        // positions per sub-page
+  int sub;       // bytes per sub-page
+  int mask;      // offset of the bitmap words (the first-VL row follows at + 8)
+  int bytes;     // bytes per page
+};
+__host__ __device__ __forceinline__ int kbits_of(const hq_cache& c) { return c.k_bits ? c.k_bits : 4; }
+__host__ __device__ __forceinline__ int vbits_of(const hq_cache& c) { return c.v_bits ? c.v_bits : 4; }
+__host__ __device__ __forceinline__ PageGeo page_geo(int kb, int vb) {
+  PageGeo g;
+  g.kb = kb;
+  g.vb = vb;
+  g.pr = HQ_PAGE_SUBPOS(kb, vb);
+  g.sub = HQ_PAGE_SUBBYTES(kb, vb);
+  g.mask = HQ_PAGE_MASK_OFF(kb, vb);
+  g.bytes = HQ_PAGE_BYTES_KV(kb, vb);
+  return g;
+}
+__host__ __device__ __forceinline__ PageGeo page_geo(const hq_cache& c) { return page_geo(kbits_of(c), vbits_of(c)); }
+
 // State row of sequence b.
 __host__ __device__ __forceinline__ int32_t* state_row(const hq_cache& c, int b) { return c.state + b * HQ_STATE_WORDS; }
 
@@ -66,7 +88,7 @@ __device__ __forceinline__ uint8_t* page_of(const hq_cache& c, size_t bh, int p)
     atomicOr(reinterpret_cast<unsigned int*>(state_row(c, static_cast<int>(bh / c.Hkv)) + HQ_STATE_ERR), HQ_DEVERR_PAGE);
     return c.pages;
   }
-  return c.pages + static_cast<size_t>(idx) * HQ_PAGE_BYTES;
+  return c.pages + static_cast<size_t>(idx) * page_geo(c).bytes;
 }
 
 // The same for writers: null for an entry outside the pool (flagged; the caller skips the write).
@@ -76,16 +98,25 @@ __device__ __forceinline__ uint8_t* page_for_write(const hq_cache& c, size_t bh,
     atomicOr(reinterpret_cast<unsigned int*>(state_row(c, static_cast<int>(bh / c.Hkv)) + HQ_STATE_ERR), HQ_DEVERR_PAGE);
     return nullptr;
   }
-  return c.pages + static_cast<size_t>(idx) * HQ_PAGE_BYTES;
+  return c.pages + static_cast<size_t>(idx) * page_geo(c).bytes;
 }
-__host__ __device__ __forceinline__ uint8_t* row_codes(uint8_t* page, int which, int p) {
-  return page + (which ? HQ_PAGE_VCODES : HQ_PAGE_KCODES) + (p & 63) * (HQ_HEAD_DIM / 2);
+// codes (16 * bits bytes) of position p (K: which = 0, V: 1) inside its page
+__host__ __device__ __forceinline__ uint8_t* row_codes(const PageGeo& pg, uint8_t* page, int which, int p) {
+  const int r = p & 63, rr = r % pg.pr;
+  uint8_t* sp = page + (r / pg.pr) * pg.sub;
+  return which ? sp + pg.pr * 16 * pg.kb + rr * 16 * pg.vb : sp + rr * 16 * pg.kb;
 }
-__host__ __device__ __forceinline__ uint32_t* row_sz(uint8_t* page, int which, int p) {
-  return reinterpret_cast<uint32_t*>(page + (which ? HQ_PAGE_VSZ : HQ_PAGE_KSZ) + (p & 63) * 16);
+// the 4 (scale | zero << 16) words of position p
+__host__ __device__ __forceinline__ uint32_t* row_sz(const PageGeo& pg, uint8_t* page, int which, int p) {
+  const int r = p & 63, rr = r % pg.pr;
+  uint8_t* sp = page + (r / pg.pr) * pg.sub;
+  return reinterpret_cast<uint32_t*>(sp + pg.pr * 16 * (pg.kb + pg.vb) + (which ? pg.pr * 16 : 0) + rr * 16);
 }
-__host__ __device__ __forceinline__ uint32_t* page_mask(uint8_t* page) {
-  return reinterpret_cast<uint32_t*>(page + HQ_PAGE_VLMASK);
+__host__ __device__ __forceinline__ uint32_t* page_mask(const PageGeo& pg, uint8_t* page) {
+  return reinterpret_cast<uint32_t*>(page + pg.mask);
+}
+__host__ __device__ __forceinline__ int32_t* page_vlbase(const PageGeo& pg, uint8_t* page) {
+  return reinterpret_cast<int32_t*>(page + pg.mask + 8);
 }
 
 // release / acquire fences at GPU scope (cheaper than the sequentially

@@ -65,10 +65,8 @@ namespace {
 constexpr int NC = HQ_DECODE_NC;
 constexpr int NSTAGES = 2 * NC;
 constexpr int NTHREADS = (NC + 1) * 32;
-constexpr int PK = 64;                         // positions per packed tile
 constexpr int FT = 16;                         // rows per FP16 tile
 constexpr int FSTRIDE = 256;                   // bytes per FP16 row in shared memory (one contiguous copy)
-constexpr int OFF_VC = 4096, OFF_KS = 8192, OFF_VS = 9216, OFF_MASK = 10240;
 constexpr int OFF_FV = FT * FSTRIDE;           // V rows of an FP16 tile
 constexpr int STAGE_BYTES = 10368;             // max(10256, 2 * 16 * 256 = 8192), 128-aligned
 constexpr int PART_FLOATS = 16 + 8 * D;        // m[8], l[8], O[8][128]
@@ -78,9 +76,9 @@ constexpr int PHANTOM_DIV = 32;                // phantom weight per unit = ceil
 constexpr int MIN_TILES = 4;                   // at least this many tiles per CTA
 constexpr int MAX_CTAS = 160;                  // one CTA per SM, at most this many (the unit merge keeps one weight per CTA in a stage)
 constexpr int SCAN_PER = (MAX_UNITS + NTHREADS - 1) / NTHREADS;  // units per thread in the scan
-constexpr uint32_t PK_TX = HQ_PAGE_VLMASK + 16;   // codes, scale/zero words and the bitmap: one copy
-static_assert(OFF_VC == HQ_PAGE_VCODES && OFF_KS == HQ_PAGE_KSZ && OFF_VS == HQ_PAGE_VSZ && OFF_MASK == HQ_PAGE_VLMASK,
-              "a packed stage is a verbatim copy of the page prefix");
+static_assert(HQ_PAGE_SUBBYTES(4, 4) + 16 <= STAGE_BYTES && HQ_PAGE_SUBBYTES(8, 8) + 16 <= STAGE_BYTES &&
+                  HQ_PAGE_SUBBYTES(4, 2) + 16 <= STAGE_BYTES && HQ_PAGE_SUBBYTES(2, 4) + 16 <= STAGE_BYTES,
+              "a packed stage holds one sub-page and the page's bitmap words");
 static_assert(PART_FLOATS * 4 <= STAGE_BYTES, "a warp state fits in one stage");
 
 // key slot -> shared-memory row inside a 16-key block.  Packed tiles (64-byte
@@ -104,12 +102,12 @@ struct UnitGeo {
   int NP, NV, NF, NT;   // packed tiles, VL tiles, FP16 tiles (VL + ring + new token), all
 };
 
-__device__ __forceinline__ UnitGeo unit_geo(int n_packed, int n_vl, int T, int R) {
+__device__ __forceinline__ UnitGeo unit_geo(int n_packed, int n_vl, int T, int R, int pr) {
   UnitGeo g;
   g.n_packed = n_packed;
   g.n_vl = n_vl;
   g.T = T;
-  g.NP = (n_packed + PK - 1) / PK;
+  g.NP = (n_packed + pr - 1) / pr;  // packed tiles: sub-pages of pr positions
   g.NV = (n_vl + FT - 1) / FT;
   g.NF = g.NV + R / FT + 1;
   g.NT = g.NP + g.NF;
@@ -204,7 +202,7 @@ __device__ __forceinline__ void aligned_snapshot(const hq_cache& c, int R, Align
     int T, np, nv;
     read_len(c, tid / c.Hkv, stale, T, np, nv);
     const bool go = !refused(c, T, np);
-    const UnitGeo g = unit_geo(np, nv, T, R);
+    const UnitGeo g = unit_geo(np, nv, T, R, page_geo(c).pr);
     sn.NP[tid] = go ? g.NP : 0;
     sn.NF[tid] = go ? g.NF : 0;
     if (tid % c.Hkv == 0) {
@@ -287,7 +285,7 @@ __device__ __noinline__ void make_plan(const hq_cache& c, int R, Plan& p, int* r
     if (u < U) {
       int T, np, nv;
       read_len(c, u / c.Hkv, stale, T, np, nv);
-      if (!refused(c, T, np)) nt[i] = unit_geo(np, nv, T, R).NT;
+      if (!refused(c, T, np)) nt[i] = unit_geo(np, nv, T, R, page_geo(c).pr).NT;
     }
     sum += nt[i];
   }
@@ -354,7 +352,7 @@ __device__ __noinline__ void make_plan(const hq_cache& c, int R, Plan& p, int* r
         if (u - u0 < MAXSEG) {
           int T, np, nv;
           read_len(c, u / c.Hkv, stale, T, np, nv);
-          const UnitGeo g = unit_geo(np, nv, T, R);
+          const UnitGeo g = unit_geo(np, nv, T, R, page_geo(c).pr);
           Seg& s = p.seg[u - u0];
           const int k0 = static_cast<int>(lo - S), k1 = static_cast<int>(hi - S);
           s.u = u;
@@ -449,109 +447,235 @@ __device__ __forceinline__ void softmax_update(WarpState& ws, float (&s)[NMT][4]
   }
 }
 
-// one K4V4 packed tile (64 positions) by one warp: S^T = K^ . Q^T for the four
-// 16-key blocks, one online-softmax step for all 64 keys, O^T += V^T . P^T
+// ------------------------------------------------------------------ packed tiles of any code width
+//
+// A packed tile is one sub-page of PR = HQ_PAGE_SUBPOS(KB, VB) positions (64,
+// or 32 for K8V8) copied verbatim into the stage, followed by the page's two
+// bitmap words at the stage offset SUB = HQ_PAGE_SUBBYTES(KB, VB).  Inside the
+// stage: K codes [PR][16 KB], V codes [PR][16 VB], K (scale | zero << 16) words
+// [PR][4], V words [PR][4].
+
+// 2-bit codes: value j (bits 2j, 2j+1) of the bytes at bits 0..7 and 16..23 of x
+// -> (1024 + 4^j n) in both halves, scaled back by 4^-j and shifted by -1024 4^-j
+// (exact: 1024 + 4^j n < 2048 keeps unit spacing).
+__device__ __forceinline__ uint32_t two_bit(uint32_t x, int j) {
+  const uint32_t m = and_or(x, 0x00030003u << (2 * j), MAGIC);
+  if (j == 0) return hsub2_u(m, H2_1024);
+  const uint32_t sc = j == 1 ? 0x34003400u : (j == 2 ? 0x2C002C00u : 0x24002400u);   // 1/4, 1/16, 1/64
+  const uint32_t off = j == 1 ? 0xDC00DC00u : (j == 2 ? 0xD400D400u : 0xCC00CC00u);  // -256, -64, -16
+  return hfma2_u(m, sc, off);
+}
+// 8-bit codes: bytes b0 (bits 0..7) and b1 (bits 16..23) of p -> (b0, b1) as fp16
+__device__ __forceinline__ uint32_t eight_bit(uint32_t p) { return hsub2_u(and_or(p, 0x00FF00FFu, MAGIC), H2_1024); }
+
+// Q^T fragments of the thread's 32 dims in the order the K codes of width KB
+// dequantise to (k-step kk: b0 = Q at the dims of a0, b1 = Q at the dims of a2).
+template <int KB>
+__device__ __forceinline__ void q_frags(const uint4 (&u)[4], uint32_t (&qf)[8][2]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (KB == 4) {  // word i, byte h: (d 8i+2h, 8i+2h+4) and (8i+2h+1, 8i+2h+5)
+      qf[2 * i][0] = prmt(u[i].x, u[i].z, 0x5410);
+      qf[2 * i][1] = prmt(u[i].x, u[i].z, 0x7632);
+      qf[2 * i + 1][0] = prmt(u[i].y, u[i].w, 0x5410);
+      qf[2 * i + 1][1] = prmt(u[i].y, u[i].w, 0x7632);
+    } else if (KB == 8) {  // word kk: (d 4kk, 4kk+1) and (4kk+2, 4kk+3)
+      qf[2 * i][0] = u[i].x;
+      qf[2 * i][1] = u[i].y;
+      qf[2 * i + 1][0] = u[i].z;
+      qf[2 * i + 1][1] = u[i].w;
+    }
+  }
+  if (KB == 2) {  // k-step kk = 4 w + j: (d 16w+j, 16w+8+j) and (16w+4+j, 16w+12+j)
+    const uint32_t h[16] = {u[0].x, u[0].y, u[0].z, u[0].w, u[1].x, u[1].y, u[1].z, u[1].w,
+                            u[2].x, u[2].y, u[2].z, u[2].w, u[3].x, u[3].y, u[3].z, u[3].w};
+#pragma unroll
+    for (int w = 0; w < 2; ++w)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int b = 8 * w;  // half2 words of dims 16w ..
+        const uint32_t sel = (j & 1) ? 0x7632 : 0x5410;
+        qf[4 * w + j][0] = prmt(h[b + (j >> 1)], h[b + 4 + (j >> 1)], sel);
+        qf[4 * w + j][1] = prmt(h[b + 2 + (j >> 1)], h[b + 6 + (j >> 1)], sel);
+      }
+  }
+}
+
+// The A-fragment halves of k-step kk for one key row whose group-t codes are
+// in w[] (4 KB bytes): lo = the dims of a0 (or a1), hi = those of a2 (or a3),
+// dequantised with the group's (scale, zero) pair s2, z2.
+template <int KB>
+__device__ __forceinline__ void k_step(const uint32_t (&w)[KB], int kk, uint32_t s2, uint32_t z2, uint32_t& lo,
+                                       uint32_t& hi) {
+  if (KB == 4) {
+    const uint32_t x = w[kk >> 1] >> (8 * (kk & 1));
+    lo = hfma2_u(nib_lo(x), s2, z2);
+    hi = hfma2_u(nib_hi(x), s2, z2);
+  } else if (KB == 8) {
+    lo = hfma2_u(eight_bit(prmt(w[kk], 0u, 0x4140)), s2, z2);
+    hi = hfma2_u(eight_bit(prmt(w[kk], 0u, 0x4342)), s2, z2);
+  } else {
+    const uint32_t x = w[kk >> 2];
+    lo = hfma2_u(two_bit(x, kk & 3), s2, z2);
+    hi = hfma2_u(two_bit(x >> 8, kk & 3), s2, z2);
+  }
+}
+
+// one packed tile by one warp: S^T = K^ . Q^T for its 16-key blocks, one
+// online-softmax step for all of them, O^T += V^T . P^T
+template <int KB, int VB>
 __device__ __forceinline__ void packed_tile(WarpState& ws, const uint8_t* st, const uint32_t (&qf)[8][2], int tile, int n_packed,
                                             float qscale, int g, int t) {
+  constexpr int PR = HQ_PAGE_SUBPOS(KB, VB), NMT = PR / 16;
+  constexpr int OFFV = PR * 16 * KB, OFFKS = PR * 16 * (KB + VB), OFFVS = OFFKS + PR * 16, OFFM = HQ_PAGE_SUBBYTES(KB, VB);
   const uint8_t* kc = st;
-  const uint8_t* vc = st + OFF_VC;
-  const uint32_t* ks = reinterpret_cast<const uint32_t*>(st + OFF_KS);
-  const uint32_t* vs = reinterpret_cast<const uint32_t*>(st + OFF_VS);
-  const uint32_t* mk = reinterpret_cast<const uint32_t*>(st + OFF_MASK);
-  const int base = tile * PK;
-  const bool full = base + PK <= n_packed;
+  const uint8_t* vc = st + OFFV;
+  const uint32_t* ks = reinterpret_cast<const uint32_t*>(st + OFFKS);
+  const uint32_t* vs = reinterpret_cast<const uint32_t*>(st + OFFVS);
+  const uint32_t* mk = reinterpret_cast<const uint32_t*>(st + OFFM);
+  const int base = tile * PR;
+  const int prow0 = base & 63;  // first page row of the tile
+  const bool full = base + PR <= n_packed;
   const int pa = pi_pk(g), pbk = pi_pk(g + 8);
-  // additive score bias of this thread's 8 key rows: -inf beyond n_packed or on
+  // additive score bias of this thread's key rows: -inf beyond n_packed or on
   // a vertical line (its FP16 row is read instead), else 0
-  const uint32_t m0 = mk[0], m1 = mk[1];
-  float bias[4][2];
+  float bias[NMT][2];
 #pragma unroll
-  for (int mt = 0; mt < 4; ++mt) {
-    const uint32_t w = (mt >> 1) ? m1 : m0;
+  for (int mt = 0; mt < NMT; ++mt) {
     const int ra = 16 * mt + pa, rb = 16 * mt + pbk;
-    const bool va = (full || base + ra < n_packed) && !((w >> (ra & 31)) & 1u);
-    const bool vb = (full || base + rb < n_packed) && !((w >> (rb & 31)) & 1u);
+    const int qa = prow0 + ra, qb = prow0 + rb;
+    const bool va = (full || base + ra < n_packed) && !((mk[qa >> 5] >> (qa & 31)) & 1u);
+    const bool vb = (full || base + rb < n_packed) && !((mk[qb >> 5] >> (qb & 31)) & 1u);
     bias[mt][0] = va ? 0.f : -INFINITY;
     bias[mt][1] = vb ? 0.f : -INFINITY;
   }
 
-  float s[4][4];
+  float s[NMT][4];
 #pragma unroll
-  for (int mt = 0; mt < 4; ++mt) {
+  for (int mt = 0; mt < NMT; ++mt) {
     const int ra = 16 * mt + pa, rb = 16 * mt + pbk;
-    const uint4 ka = *reinterpret_cast<const uint4*>(kc + ra * 64 + 16 * t);
-    const uint4 kb = *reinterpret_cast<const uint4*>(kc + rb * 64 + 16 * t);
+    uint32_t wa[KB], wb[KB];  // group t of rows a and b: 4 KB bytes = KB words each
+#pragma unroll
+    for (int i = 0; i < KB / 4; ++i) {
+      const uint4 x = *reinterpret_cast<const uint4*>(kc + ra * 16 * KB + 4 * KB * t + 16 * i);
+      const uint4 y = *reinterpret_cast<const uint4*>(kc + rb * 16 * KB + 4 * KB * t + 16 * i);
+      wa[4 * i] = x.x; wa[4 * i + 1] = x.y; wa[4 * i + 2] = x.z; wa[4 * i + 3] = x.w;
+      wb[4 * i] = y.x; wb[4 * i + 1] = y.y; wb[4 * i + 2] = y.z; wb[4 * i + 3] = y.w;
+    }
+    if (KB == 2) {
+      const uint2 x = *reinterpret_cast<const uint2*>(kc + ra * 32 + 8 * t);
+      const uint2 y = *reinterpret_cast<const uint2*>(kc + rb * 32 + 8 * t);
+      wa[0] = x.x; wa[1] = x.y;
+      wb[0] = y.x; wb[1] = y.y;
+    }
     const uint32_t za = ks[ra * 4 + t], zb = ks[rb * 4 + t];
     const uint32_t sa2 = prmt(za, za, 0x1010), za2 = prmt(za, za, 0x3232);
     const uint32_t sb2 = prmt(zb, zb, 0x1010), zb2 = prmt(zb, zb, 0x3232);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w};
-    const uint32_t wb[4] = {kb.x, kb.y, kb.z, kb.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t xa = wa[i] >> (8 * h), xb = wb[i] >> (8 * h);
-        const uint32_t a0 = hfma2_u(nib_lo(xa), sa2, za2);
-        const uint32_t a2 = hfma2_u(nib_hi(xa), sa2, za2);
-        const uint32_t a1 = hfma2_u(nib_lo(xb), sb2, zb2);
-        const uint32_t a3 = hfma2_u(nib_hi(xb), sb2, zb2);
-        mma16816(acc, a0, a1, a2, a3, qf[2 * i + h][0], qf[2 * i + h][1]);
-      }
+    for (int kk = 0; kk < 8; ++kk) {
+      uint32_t a0, a1, a2, a3;
+      k_step<KB>(wa, kk, sa2, za2, a0, a2);
+      k_step<KB>(wb, kk, sb2, zb2, a1, a3);
+      mma16816(acc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
     }
     s[mt][0] = fmaf(acc[0], qscale, bias[mt][0]);
     s[mt][1] = fmaf(acc[1], qscale, bias[mt][0]);
     s[mt][2] = fmaf(acc[2], qscale, bias[mt][1]);
     s[mt][3] = fmaf(acc[3], qscale, bias[mt][1]);
   }
-  uint32_t pb[4][2];
-  softmax_update<4>(ws, s, pb);
+  uint32_t pb[NMT][2];
+  softmax_update<NMT>(ws, s, pb);
 
 #pragma unroll
-  for (int mt = 0; mt < 4; ++mt) {
+  for (int mt = 0; mt < NMT; ++mt) {
     const int r0 = 16 * mt + pi_pk(2 * t), r1 = 16 * mt + pi_pk(2 * t + 1);
     const int r2 = 16 * mt + pi_pk(2 * t + 8), r3 = 16 * mt + pi_pk(2 * t + 9);
-    // two 32-bit loads per row, issued in a per-thread order that keeps the
-    // warp's accesses on distinct banks
-    const int e = t >> 1;
-    const uint32_t* v0 = reinterpret_cast<const uint32_t*>(vc + r0 * 64) + 2 * g;
-    const uint32_t* v1 = reinterpret_cast<const uint32_t*>(vc + r1 * 64) + 2 * g;
-    const uint32_t* v2 = reinterpret_cast<const uint32_t*>(vc + r2 * 64) + 2 * g;
-    const uint32_t* v3 = reinterpret_cast<const uint32_t*>(vc + r3 * 64) + 2 * g;
-    const uint32_t x0a = v0[e], x0b = v0[e ^ 1], x1a = v1[e], x1b = v1[e ^ 1];
-    const uint32_t x2a = v2[e], x2b = v2[e ^ 1], x3a = v3[e], x3b = v3[e ^ 1];
-    // un-rotate: w?0 = word 2g, w?1 = word 2g+1
-    const uint32_t w00 = e ? x0b : x0a, w01 = e ? x0a : x0b;
-    const uint32_t w10 = e ? x1b : x1a, w11 = e ? x1a : x1b;
-    const uint32_t w20 = e ? x2b : x2a, w21 = e ? x2a : x2b;
-    const uint32_t w30 = e ? x3b : x3a, w31 = e ? x3a : x3b;
     const int grp = g >> 1;
     const uint32_t z0 = vs[r0 * 4 + grp], z1 = vs[r1 * 4 + grp], z2 = vs[r2 * 4 + grp], z3 = vs[r3 * 4 + grp];
     const uint32_t s01 = prmt(z0, z1, 0x5410), o01 = prmt(z0, z1, 0x7632);
     const uint32_t s23 = prmt(z2, z3, 0x5410), o23 = prmt(z2, z3, 0x7632);
-    // pair nibbles of the two keys: x?[k] holds dims 16g + 4k .. 16g + 4k + 3 of both keys
-    uint32_t xab[4], xcd[4];
-    xab[0] = prmt(w00, w10, 0x5410);
-    xab[1] = prmt(w00, w10, 0x7632);
-    xab[2] = prmt(w01, w11, 0x5410);
-    xab[3] = prmt(w01, w11, 0x7632);
-    xcd[0] = prmt(w20, w30, 0x5410);
-    xcd[1] = prmt(w20, w30, 0x7632);
-    xcd[2] = prmt(w21, w31, 0x5410);
-    xcd[3] = prmt(w21, w31, 0x7632);
     uint32_t keep_ab = 0xFFFFFFFFu, keep_cd = 0xFFFFFFFFu;
     if (!full) {  // rows past n_packed may hold stale records: zero them out of P.V
       keep_ab = (base + r0 < n_packed ? 0x0000FFFFu : 0u) | (base + r1 < n_packed ? 0xFFFF0000u : 0u);
       keep_cd = (base + r2 < n_packed ? 0x0000FFFFu : 0u) | (base + r3 < n_packed ? 0xFFFF0000u : 0u);
     }
+    // a0 / a1: keys (r0, r1) at dims 16g + 2m and 16g + 2m + 1; a2 / a3: keys (r2, r3)
+    uint32_t A[8][4];
+    if (VB == 4) {
+      // two 32-bit loads per row, issued in a per-thread order that keeps the
+      // warp's accesses on distinct banks
+      const int e = t >> 1;
+      const uint32_t* v0 = reinterpret_cast<const uint32_t*>(vc + r0 * 64) + 2 * g;
+      const uint32_t* v1 = reinterpret_cast<const uint32_t*>(vc + r1 * 64) + 2 * g;
+      const uint32_t* v2 = reinterpret_cast<const uint32_t*>(vc + r2 * 64) + 2 * g;
+      const uint32_t* v3 = reinterpret_cast<const uint32_t*>(vc + r3 * 64) + 2 * g;
+      const uint32_t x0a = v0[e], x0b = v0[e ^ 1], x1a = v1[e], x1b = v1[e ^ 1];
+      const uint32_t x2a = v2[e], x2b = v2[e ^ 1], x3a = v3[e], x3b = v3[e ^ 1];
+      // un-rotate: w?0 = word 2g, w?1 = word 2g+1
+      const uint32_t w00 = e ? x0b : x0a, w01 = e ? x0a : x0b;
+      const uint32_t w10 = e ? x1b : x1a, w11 = e ? x1a : x1b;
+      const uint32_t w20 = e ? x2b : x2a, w21 = e ? x2a : x2b;
+      const uint32_t w30 = e ? x3b : x3a, w31 = e ? x3a : x3b;
+      // pair nibbles of the two keys: x?[k] holds dims 16g + 4k .. 16g + 4k + 3 of both keys
+      uint32_t xab[4], xcd[4];
+      xab[0] = prmt(w00, w10, 0x5410);
+      xab[1] = prmt(w00, w10, 0x7632);
+      xab[2] = prmt(w01, w11, 0x5410);
+      xab[3] = prmt(w01, w11, 0x7632);
+      xcd[0] = prmt(w20, w30, 0x5410);
+      xcd[1] = prmt(w20, w30, 0x7632);
+      xcd[2] = prmt(w21, w31, 0x5410);
+      xcd[3] = prmt(w21, w31, 0x7632);
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const uint32_t yab = xab[m >> 1] >> (8 * (m & 1));
+        const uint32_t ycd = xcd[m >> 1] >> (8 * (m & 1));
+        A[m][0] = hfma2_u(nib_lo(yab), s01, o01);
+        A[m][1] = hfma2_u(nib_hi(yab), s01, o01);
+        A[m][2] = hfma2_u(nib_lo(ycd), s23, o23);
+        A[m][3] = hfma2_u(nib_hi(ycd), s23, o23);
+      }
+    } else if (VB == 8) {
+      // 16 bytes per row (dims 16g .. 16g + 15): byte d of key r0 beside byte d of key r1
+      const uint4 u0 = *reinterpret_cast<const uint4*>(vc + r0 * 128 + 16 * g);
+      const uint4 u1 = *reinterpret_cast<const uint4*>(vc + r1 * 128 + 16 * g);
+      const uint4 u2 = *reinterpret_cast<const uint4*>(vc + r2 * 128 + 16 * g);
+      const uint4 u3 = *reinterpret_cast<const uint4*>(vc + r3 * 128 + 16 * g);
+      const uint32_t q0[4] = {u0.x, u0.y, u0.z, u0.w}, q1[4] = {u1.x, u1.y, u1.z, u1.w};
+      const uint32_t q2[4] = {u2.x, u2.y, u2.z, u2.w}, q3[4] = {u3.x, u3.y, u3.z, u3.w};
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const int b = 2 * (m & 1);  // byte of dim 2m in word m / 2
+        const uint32_t sl = b | (b << 4) | ((4 + b) << 8) | ((4 + b) << 12);
+        const uint32_t sh = (b + 1) | ((b + 1) << 4) | ((5 + b) << 8) | ((5 + b) << 12);
+        A[m][0] = hfma2_u(eight_bit(prmt(q0[m >> 1], q1[m >> 1], sl)), s01, o01);
+        A[m][1] = hfma2_u(eight_bit(prmt(q0[m >> 1], q1[m >> 1], sh)), s01, o01);
+        A[m][2] = hfma2_u(eight_bit(prmt(q2[m >> 1], q3[m >> 1], sl)), s23, o23);
+        A[m][3] = hfma2_u(eight_bit(prmt(q2[m >> 1], q3[m >> 1], sh)), s23, o23);
+      }
+    } else {
+      // 4 bytes per row (dims 16g .. 16g + 15, byte k = dims 4k .. 4k + 3)
+      const uint32_t w0 = reinterpret_cast<const uint32_t*>(vc + r0 * 32)[g];
+      const uint32_t w1 = reinterpret_cast<const uint32_t*>(vc + r1 * 32)[g];
+      const uint32_t w2 = reinterpret_cast<const uint32_t*>(vc + r2 * 32)[g];
+      const uint32_t w3 = reinterpret_cast<const uint32_t*>(vc + r3 * 32)[g];
+      const uint32_t xab[2] = {prmt(w0, w1, 0x5410), prmt(w0, w1, 0x7632)};  // dims 0..7, 8..15 of both keys
+      const uint32_t xcd[2] = {prmt(w2, w3, 0x5410), prmt(w2, w3, 0x7632)};
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const uint32_t yab = xab[m >> 2] >> (8 * ((m >> 1) & 1));
+        const uint32_t ycd = xcd[m >> 2] >> (8 * ((m >> 1) & 1));
+        const int j = 2 * (m & 1);
+        A[m][0] = hfma2_u(two_bit(yab, j), s01, o01);
+        A[m][1] = hfma2_u(two_bit(yab, j + 1), s01, o01);
+        A[m][2] = hfma2_u(two_bit(ycd, j), s23, o23);
+        A[m][3] = hfma2_u(two_bit(ycd, j + 1), s23, o23);
+      }
+    }
 #pragma unroll
     for (int m = 0; m < 8; ++m) {
-      const uint32_t yab = xab[m >> 1] >> (8 * (m & 1));
-      const uint32_t ycd = xcd[m >> 1] >> (8 * (m & 1));
-      uint32_t a0 = hfma2_u(nib_lo(yab), s01, o01);
-      uint32_t a1 = hfma2_u(nib_hi(yab), s01, o01);
-      uint32_t a2 = hfma2_u(nib_lo(ycd), s23, o23);
-      uint32_t a3 = hfma2_u(nib_hi(ycd), s23, o23);
+      uint32_t a0 = A[m][0], a1 = A[m][1], a2 = A[m][2], a3 = A[m][3];
       if (!full) {
         a0 &= keep_ab; a1 &= keep_ab;
         a2 &= keep_cd; a3 &= keep_cd;
@@ -562,21 +686,48 @@ __device__ __forceinline__ void packed_tile(WarpState& ws, const uint8_t* st, co
 }
 
 // one FP16 tile (16 rows at FSTRIDE) by one warp; bit r of `valid` marks row r as real
+template <int KB>
 __device__ __forceinline__ void fp16_tile(WarpState& ws, const uint8_t* st, const uint32_t (&qf)[8][2], uint32_t valid,
                                           float qscale, int g, int t) {
   const uint8_t* kb = st;
   const uint8_t* vb = st + OFF_FV;
   const int ra = pi_fp(g), rb = pi_fp(g + 8);
+  const uint8_t* ka = kb + ra * FSTRIDE + 64 * t;  // the thread's 32 dims of key rows a and b
+  const uint8_t* kbr = kb + rb * FSTRIDE + 64 * t;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  // the K A-fragments follow the dim order of the Q fragments (q_frags<KB>)
+  if (KB == 2) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint4 ua = *reinterpret_cast<const uint4*>(kb + ra * FSTRIDE + 64 * t + 16 * i);
-    const uint4 ub = *reinterpret_cast<const uint4*>(kb + rb * FSTRIDE + 64 * t + 16 * i);
-    // k-step 2i: (d0,d4) and (d1,d5); k-step 2i+1: (d2,d6) and (d3,d7)
-    mma16816(acc, prmt(ua.x, ua.z, 0x5410), prmt(ub.x, ub.z, 0x5410), prmt(ua.x, ua.z, 0x7632), prmt(ub.x, ub.z, 0x7632),
-             qf[2 * i][0], qf[2 * i][1]);
-    mma16816(acc, prmt(ua.y, ua.w, 0x5410), prmt(ub.y, ub.w, 0x5410), prmt(ua.y, ua.w, 0x7632), prmt(ub.y, ub.w, 0x7632),
-             qf[2 * i + 1][0], qf[2 * i + 1][1]);
+    for (int w = 0; w < 2; ++w) {
+      const uint4 a0 = *reinterpret_cast<const uint4*>(ka + 32 * w), a1 = *reinterpret_cast<const uint4*>(ka + 32 * w + 16);
+      const uint4 b0 = *reinterpret_cast<const uint4*>(kbr + 32 * w), b1 = *reinterpret_cast<const uint4*>(kbr + 32 * w + 16);
+      const uint32_t ha[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const uint32_t hb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {  // k-step 4w + j: (d 16w+j, 16w+8+j) and (16w+4+j, 16w+12+j)
+        const uint32_t sel = (j & 1) ? 0x7632 : 0x5410;
+        const int h = j >> 1;
+        mma16816(acc, prmt(ha[h], ha[4 + h], sel), prmt(hb[h], hb[4 + h], sel), prmt(ha[2 + h], ha[6 + h], sel),
+                 prmt(hb[2 + h], hb[6 + h], sel), qf[4 * w + j][0], qf[4 * w + j][1]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 ua = *reinterpret_cast<const uint4*>(ka + 16 * i);
+      const uint4 ub = *reinterpret_cast<const uint4*>(kbr + 16 * i);
+      if (KB == 4) {
+        // k-step 2i: (d0,d4) and (d1,d5); k-step 2i+1: (d2,d6) and (d3,d7)
+        mma16816(acc, prmt(ua.x, ua.z, 0x5410), prmt(ub.x, ub.z, 0x5410), prmt(ua.x, ua.z, 0x7632),
+                 prmt(ub.x, ub.z, 0x7632), qf[2 * i][0], qf[2 * i][1]);
+        mma16816(acc, prmt(ua.y, ua.w, 0x5410), prmt(ub.y, ub.w, 0x5410), prmt(ua.y, ua.w, 0x7632),
+                 prmt(ub.y, ub.w, 0x7632), qf[2 * i + 1][0], qf[2 * i + 1][1]);
+      } else {
+        // k-step 2i: (d0,d1) and (d2,d3); k-step 2i+1: (d4,d5) and (d6,d7)
+        mma16816(acc, ua.x, ub.x, ua.y, ub.y, qf[2 * i][0], qf[2 * i][1]);
+        mma16816(acc, ua.z, ub.z, ua.w, ub.w, qf[2 * i + 1][0], qf[2 * i + 1][1]);
+      }
+    }
   }
   float s[1][4];
   const bool va = (valid >> ra) & 1u, vbv = (valid >> rb) & 1u;
@@ -634,19 +785,15 @@ __device__ __forceinline__ void advance_lengths(const hq_cache& c, int tid, int 
 }
 
 // Load this unit's Q^T fragments (the G query heads of kv head kvh of sequence b,
-// in the permuted dim order: thread t covers dims 32t .. 32t+31); columns >= G are zero.
+// in the dim order the K codes dequantise to: thread t covers dims 32t .. 32t+31);
+// columns >= G are zero.
+template <int KB>
 __device__ __forceinline__ void load_q(const hq_cache& c, const uint16_t* __restrict__ q, int b, int kvh, int G, int g,
                                        int t, uint32_t (&qf)[8][2]) {
   if (g < G) {
     const uint4* qp = reinterpret_cast<const uint4*>(q + (static_cast<size_t>(b) * c.Hq + kvh * G + g) * D + 32 * t);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 u = qp[i];
-      qf[2 * i][0] = prmt(u.x, u.z, 0x5410);
-      qf[2 * i][1] = prmt(u.x, u.z, 0x7632);
-      qf[2 * i + 1][0] = prmt(u.y, u.w, 0x5410);
-      qf[2 * i + 1][1] = prmt(u.y, u.w, 0x7632);
-    }
+    const uint4 u[4] = {qp[0], qp[1], qp[2], qp[3]};
+    q_frags<KB>(u, qf);
   } else {
 #pragma unroll
     for (int j = 0; j < 8; ++j) qf[j][0] = qf[j][1] = 0u;
@@ -657,7 +804,7 @@ __device__ __forceinline__ void consumer_bar() { asm volatile("bar.sync 1, %0;" 
 
 __device__ __forceinline__ UnitGeo geo_of_unit(const hq_cache& c, int u, int R) {
   const int32_t* st = state_row(c, u / c.Hkv);
-  return unit_geo(st[HQ_STATE_NPACKED], st[HQ_STATE_NVL], st[HQ_STATE_T], R);
+  return unit_geo(st[HQ_STATE_NPACKED], st[HQ_STATE_NVL], st[HQ_STATE_T], R, page_geo(c).pr);
 }
 
 // Source of FP16 tile j of unit bh (K rows, V rows, bytes per half)
@@ -871,6 +1018,7 @@ __device__ __forceinline__ void segment_epilogue(const hq_cache& c, const uint16
   consumer_bar();
 }
 
+template <int KB, int VB>
 __global__ void __launch_bounds__(NTHREADS, 1)
 decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* __restrict__ k_new,
               const uint16_t* __restrict__ v_new, uint16_t* __restrict__ out, float qscale,
@@ -916,10 +1064,12 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
   if (warp == NC) {
     for (int si = 0; si < plan.nseg; ++si) {
       const Seg s = plan.seg[si];
-      const int p0 = s.p0, p1 = min(s.p0 + s.npk, c.cap / PK);
+      constexpr int PR = HQ_PAGE_SUBPOS(KB, VB);
+      constexpr int PB = HQ_PAGE_BYTES_KV(KB, VB);
+      const int p0 = (s.p0 * PR) / 64, p1 = min(((s.p0 + s.npk) * PR + 63) / 64, c.cap / 64);
       for (int pg = p0 + lane; pg < p1; pg += 32) {  // one page per lane
         const long long idx = page_index(c, s.u, pg);
-        if (idx >= 0) prefetch_l2(c.pages + static_cast<size_t>(idx) * HQ_PAGE_BYTES, PK_TX);
+        if (idx >= 0) prefetch_l2(c.pages + static_cast<size_t>(idx) * PB, HQ_PAGE_MASK_OFF(KB, VB) + 16);
       }
       int T, np, nv;
       read_len(c, s.u / c.Hkv, true, T, np, nv);
@@ -997,8 +1147,17 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
         s_issued[s] = k + 1;
         const int tl = seg_tile(sg, i);
         if (tl >= 0) {
-          mbar_arrive_expect_tx(&full[s], PK_TX);
-          bulk_g2s(st, page_of(c, sg.u, tl * PK), PK_TX, &full[s]);
+          // packed tile tl = sub-page tl % (64 / PR) of page tl / (64 / PR); the
+          // page's bitmap words follow the sub-page in the stage
+          constexpr int PR = HQ_PAGE_SUBPOS(KB, VB), SUB = HQ_PAGE_SUBBYTES(KB, VB), MOFF = HQ_PAGE_MASK_OFF(KB, VB);
+          const uint8_t* page = page_of(c, sg.u, tl * PR);
+          mbar_arrive_expect_tx(&full[s], SUB + 16);
+          if (PR == 64) {
+            bulk_g2s(st, page, SUB + 16, &full[s]);
+          } else {
+            bulk_g2s(st, page + (tl % (64 / PR)) * SUB, SUB, &full[s]);
+            bulk_g2s(st + SUB, page + MOFF, 16, &full[s]);
+          }
         } else {
           const uint16_t *ks, *vs;
           uint32_t bytes;
@@ -1019,7 +1178,7 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
       int32_t* srow = state_row(c, b);
       const UnitGeo ug = geo_of_unit(c, u, R);
       uint32_t qf[8][2];
-      load_q(c, q, b, kvh, G, g, t, qf);
+      load_q<KB>(c, q, b, kvh, G, g, t, qf);
       WarpState ws;
       ws.m[0] = ws.m[1] = -INFINITY;
       ws.l[0] = ws.l[1] = 0.f;
@@ -1039,9 +1198,9 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
         const uint8_t* st = smem + s * STAGE_BYTES;
         const int tl = seg_tile(sg, i);
         if (tl >= 0) {
-          packed_tile(ws, st, qf, tl, ug.n_packed, qscale, g, t);
+          packed_tile<KB, VB>(ws, st, qf, tl, ug.n_packed, qscale, g, t);
         } else {
-          fp16_tile(ws, st, qf, fp16_valid(ug, -tl - 1, R), qscale, g, t);
+          fp16_tile<KB>(ws, st, qf, fp16_valid(ug, -tl - 1, R), qscale, g, t);
         }
         __syncwarp();
         if (i + NC < sg.b) {
@@ -1099,7 +1258,11 @@ size_t decode_workspace(const hq_cache& c, int sms) {
   return decode_counter_bytes(c) + (static_cast<size_t>(sms) + static_cast<size_t>(c.B) * c.Hkv) * PART_FLOATS * sizeof(float);
 }
 
-bool decode_supported(const hq_cache& c) { return c.B * c.Hkv <= MAX_UNITS; }
+bool decode_supported(const hq_cache& c) {
+  const int kb = kbits_of(c), vb = vbits_of(c);
+  const bool fmt = (kb == 4 && vb == 4) || (kb == 8 && vb == 8) || (kb == 4 && vb == 2) || (kb == 2 && vb == 4);
+  return fmt && c.B * c.Hkv <= MAX_UNITS;
+}
 
 
 hq_status launch_decode(const hq_cache& c, const uint16_t* q, const uint16_t* kn, const uint16_t* vn, uint16_t* out,
@@ -1110,7 +1273,14 @@ hq_status launch_decode(const hq_cache& c, const uint16_t* q, const uint16_t* kn
   cudaGetDevice(&dev);
   static DeviceOnce attrs;
   const cudaError_t ea = attrs.run(dev, [] {
-    return cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, NSTAGES * STAGE_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<4, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, NSTAGES * STAGE_BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(decode_kernel<8, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, NSTAGES * STAGE_BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(decode_kernel<4, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, NSTAGES * STAGE_BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(decode_kernel<2, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, NSTAGES * STAGE_BYTES);
+    return e;
   });
   if (ea != cudaSuccess) return cuda_fail(ea, "decode attributes");
   unsigned int* tickets = reinterpret_cast<unsigned int*>(ws);
@@ -1128,8 +1298,13 @@ hq_status launch_decode(const hq_cache& c, const uint16_t* q, const uint16_t* kn
   const float qs = sm_scale * LOG2E;
   // the stored log-sum-exps serve the reselection only at its own scale 1/sqrt(D)
   const int lse_ok = sm_scale == 1.0f / sqrtf(static_cast<float>(D));
-  return cuda_status(cudaLaunchKernelEx(&cfg, decode_kernel, c, q, kn, vn, out, qs, parts, tickets, lse_ok),
-                     "decode launch");
+  const int kb = kbits_of(c), vb = vbits_of(c);
+  cudaError_t e;
+  if (kb == 8) e = cudaLaunchKernelEx(&cfg, decode_kernel<8, 8>, c, q, kn, vn, out, qs, parts, tickets, lse_ok);
+  else if (vb == 2) e = cudaLaunchKernelEx(&cfg, decode_kernel<4, 2>, c, q, kn, vn, out, qs, parts, tickets, lse_ok);
+  else if (kb == 2) e = cudaLaunchKernelEx(&cfg, decode_kernel<2, 4>, c, q, kn, vn, out, qs, parts, tickets, lse_ok);
+  else e = cudaLaunchKernelEx(&cfg, decode_kernel<4, 4>, c, q, kn, vn, out, qs, parts, tickets, lse_ok);
+  return cuda_status(e, "decode launch");
 }
 
 }  // namespace hq

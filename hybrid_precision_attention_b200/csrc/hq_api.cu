@@ -84,6 +84,12 @@ hq_status hq_cache_validate(const hq_cache* c) {
     return HQ_ERR_INVALID;
   if (c->score_acc != nullptr && (reinterpret_cast<uintptr_t>(c->score_acc) & 15u) != 0) return HQ_ERR_INVALID;
   if (c->qlse != nullptr && (reinterpret_cast<uintptr_t>(c->qlse) & 15u) != 0) return HQ_ERR_INVALID;
+  {
+    const int kb = c->k_bits ? c->k_bits : 4, vb = c->v_bits ? c->v_bits : 4;
+    if ((kb != 2 && kb != 4 && kb != 8) || (vb != 2 && vb != 4 && vb != 8)) return HQ_ERR_INVALID;
+    if (!((kb == 4 && vb == 4) || (kb == 8 && vb == 8) || (kb == 4 && vb == 2) || (kb == 2 && vb == 4)))
+      return HQ_ERR_UNSUPPORTED;
+  }
   return HQ_OK;
 }
 

@@ -27,10 +27,11 @@ struct Dims {
 
 __device__ __forceinline__ Dims dims_of(const hq_cache& c) { return Dims{c.B, c.Hkv, c.cap, c.vl_cap, ring_len(c.W), c.W}; }
 
-// Pack one 128-value fp16 row into 64 code bytes + 4 (scale, zero) words.
-// Warp-cooperative: lane l owns values 4l .. 4l+3 (group l / 8).
+// Pack one 128-value fp16 row into 16 * bits code bytes + 4 (scale, zero)
+// words, with 2^bits - 1 levels.  Warp-cooperative: lane l owns values 4l ..
+// 4l+3 (group l / 8), i.e. 4 * bits consecutive bits of the codes.
 __device__ __forceinline__ void pack_row_warp(const uint16_t* __restrict__ src, uint8_t* __restrict__ codes,
-                                              uint32_t* __restrict__ sz, int lane) {
+                                              uint32_t* __restrict__ sz, int lane, int bits) {
   const uint2 raw = *reinterpret_cast<const uint2*>(src + 4 * lane);
   float x[4];
   x[0] = __half2float(__ushort_as_half(static_cast<unsigned short>(raw.x & 0xFFFFu)));
@@ -44,19 +45,21 @@ __device__ __forceinline__ void pack_row_warp(const uint16_t* __restrict__ src, 
     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   }
-  // scale = fp16_RN(fp32(mx - mn) / 15), zero = mn (an fp16 value, exact in fp32)
+  const float levels = static_cast<float>((1 << bits) - 1);
+  // scale = fp16_RN(fp32(mx - mn) / levels), zero = mn (an fp16 value, exact in fp32)
   const float span = __fsub_rn(mx, mn);
-  const __half scale_h = __float2half_rn(__fdiv_rn(span, 15.0f));
+  const __half scale_h = __float2half_rn(__fdiv_rn(span, levels));
   const float scale = __half2float(scale_h);
-  uint32_t q[4];
+  uint32_t q = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     float r = scale == 0.0f ? 0.0f : rintf(__fdiv_rn(__fsub_rn(x[i], mn), scale));
-    r = fminf(fmaxf(r, 0.0f), 15.0f);
-    q[i] = static_cast<uint32_t>(r);
+    r = fminf(fmaxf(r, 0.0f), levels);
+    q |= static_cast<uint32_t>(r) << (bits * i);
   }
-  const uint32_t two = (q[0] | (q[1] << 4)) | ((q[2] | (q[3] << 4)) << 8);
-  reinterpret_cast<uint16_t*>(codes)[lane] = static_cast<uint16_t>(two);
+  if (bits == 4) reinterpret_cast<uint16_t*>(codes)[lane] = static_cast<uint16_t>(q);
+  else if (bits == 8) reinterpret_cast<uint32_t*>(codes)[lane] = q;
+  else codes[lane] = static_cast<uint8_t>(q);
   if ((lane & 7) == 0) {
     const uint32_t zbits = __half_as_ushort(__float2half_rn(mn));  // exact: mn is an fp16 value
     sz[lane >> 3] = static_cast<uint32_t>(__half_as_ushort(scale_h)) | (zbits << 16);
@@ -95,7 +98,8 @@ __global__ void pack_rows_kernel(hq_cache c, const uint16_t* __restrict__ kd, co
     }
     uint8_t* page = page_for_write(c, bh, p);
     if (page == nullptr) continue;
-    pack_row_warp(src, row_codes(page, which, p), row_sz(page, which, p), lane);
+    const PageGeo pg = page_geo(c);
+    pack_row_warp(src, row_codes(pg, page, which, p), row_sz(pg, page, which, p), lane, which ? pg.vb : pg.kb);
   }
 }
 
@@ -125,13 +129,14 @@ __global__ void ring_fill_kernel(hq_cache c, const uint16_t* __restrict__ kd, co
 // line, and rows are in position order, so the row is that plus the number of
 // lines of the page below p.
 __device__ __forceinline__ int old_vl_row(const hq_cache& c, size_t bh, int p) {
-  const uint8_t* page = page_of(c, bh, p);
-  const uint2 m = *reinterpret_cast<const uint2*>(page + HQ_PAGE_VLMASK);
+  const PageGeo pg = page_geo(c);
+  uint8_t* page = page_of(c, bh, p);
+  const uint2 m = *reinterpret_cast<const uint2*>(page_mask(pg, page));
   const int r = p & 63;
   const uint32_t w = r < 32 ? m.x : m.y;
   if (!((w >> (r & 31)) & 1u)) return -1;
   const int below = __popc(w & ((1u << (r & 31)) - 1u)) + (r < 32 ? 0 : __popc(m.x));
-  return *reinterpret_cast<const int32_t*>(page + HQ_PAGE_VLBASE) + below;
+  return *page_vlbase(pg, page) + below;
 }
 
 // Merge: gather the FP16 rows of the new VL set into the workspace.  One warp
@@ -167,18 +172,22 @@ __global__ void vl_gather_kernel(hq_cache c, uint16_t* __restrict__ wsk, uint16_
       } else {
         // promoted packed position: fp16(zero + q * scale); q * scale is exact in
         // float64 and the sum is rounded once, then once more to fp16 (RN).
+        // Lane l dequantises values 4l .. 4l+3 (4 * bits code bits).
+        const PageGeo pg = page_geo(c);
         uint8_t* page = page_of(c, bh, p);
-        const uint8_t* codes = row_codes(page, which, p);
-        const uint32_t szw = row_sz(page, which, p)[lane >> 3];
+        const int bits = which ? pg.vb : pg.kb;
+        const uint8_t* codes = row_codes(pg, page, which, p);
+        const uint32_t szw = row_sz(pg, page, which, p)[lane >> 3];
         const double sc = static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(szw & 0xFFFFu))));
         const double ze = static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(szw >> 16))));
-        const uint32_t two = reinterpret_cast<const uint16_t*>(codes)[lane];
+        const uint32_t qw = bits == 4 ? reinterpret_cast<const uint16_t*>(codes)[lane]
+                                      : (bits == 8 ? reinterpret_cast<const uint32_t*>(codes)[lane] : codes[lane]);
+        const uint32_t mask = (1u << bits) - 1u;
         uint32_t out[2];
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
-          const uint32_t byte = (two >> (8 * i)) & 0xFFu;
-          const double v0 = __dadd_rn(ze, __dmul_rn(static_cast<double>(byte & 15u), sc));
-          const double v1 = __dadd_rn(ze, __dmul_rn(static_cast<double>(byte >> 4), sc));
+          const double v0 = __dadd_rn(ze, __dmul_rn(static_cast<double>((qw >> (bits * 2 * i)) & mask), sc));
+          const double v1 = __dadd_rn(ze, __dmul_rn(static_cast<double>((qw >> (bits * (2 * i + 1))) & mask), sc));
           out[i] = static_cast<uint32_t>(__half_as_ushort(__double2half(v0))) |
                    (static_cast<uint32_t>(__half_as_ushort(__double2half(v1))) << 16);
         }
@@ -199,7 +208,7 @@ __global__ void vl_clear_kernel(hq_cache c) {
     const int r = static_cast<int>(i % d.vl_cap);
     if (r >= state_row(c, static_cast<int>(bh / d.Hkv))[HQ_STATE_NVL]) continue;
     uint8_t* page = page_for_write(c, bh, c.vl_pos[bh * d.vl_cap + r]);
-    if (page) *reinterpret_cast<uint2*>(page + HQ_PAGE_VLMASK) = make_uint2(0u, 0u);
+    if (page) *reinterpret_cast<uint2*>(page_mask(page_geo(c), page)) = make_uint2(0u, 0u);
   }
 }
 
@@ -236,11 +245,11 @@ __global__ void vl_install_kernel(hq_cache c, const uint16_t* __restrict__ srck,
       c.vl_pos[bh * d.vl_cap + row] = p;
       uint8_t* page = page_for_write(c, bh, p);
       if (page) {
-        atomicOr(page_mask(page) + ((p & 63) >> 5), 1u << (p & 31));
+        const PageGeo pg = page_geo(c);
+        atomicOr(page_mask(pg, page) + ((p & 63) >> 5), 1u << (p & 31));
         // the first vertical line of a page records its VL-store row (rows are in
         // ascending position order), so readers find a line's row by a popcount
-        if (row == 0 || (c.vl_sel[bh * d.vl_cap + row - 1] >> 6) != (p >> 6))
-          *reinterpret_cast<int32_t*>(page + HQ_PAGE_VLBASE) = row;
+        if (row == 0 || (c.vl_sel[bh * d.vl_cap + row - 1] >> 6) != (p >> 6)) *page_vlbase(pg, page) = row;
       }
     }
   }
@@ -277,7 +286,8 @@ __global__ void clear_bitmaps_kernel(hq_cache c) {
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
     const long long idx = page_index(c, static_cast<size_t>(i / npg), static_cast<int>(i % npg));
     if (idx < 0) continue;
-    *reinterpret_cast<uint2*>(c.pages + static_cast<size_t>(idx) * HQ_PAGE_BYTES + HQ_PAGE_VLMASK) = make_uint2(0u, 0u);
+    const PageGeo pg = page_geo(c);
+    *reinterpret_cast<uint2*>(c.pages + static_cast<size_t>(idx) * pg.bytes + pg.mask) = make_uint2(0u, 0u);
   }
 }
 

@@ -117,7 +117,7 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int ch, int half_bytes) {
 // vertical line's FP16 row is found from the bitmap once the loads are back.
 struct KeyRow {
   const uint4* src;  // FP16 source row, or null
-  uint4 code[4];
+  uint4 code[8];     // 16 * bits code bytes (bits = 4: code[0..3], 8: code[0..7], 2: code[0..1])
   uint4 sz;
   uint2 mask;       // the page's bitmap words
   int vlbase;        // VL-store row of the page's first vertical line
@@ -139,13 +139,15 @@ __device__ __forceinline__ KeyRow fetch_key_row(const SelArgs& a, const SelGeo& 
   } else if (j >= g.n_packed) {
     k.src = reinterpret_cast<const uint4*>(c.kr + (static_cast<size_t>(bh) * ring_len(c.W) + (j % ring_len(c.W))) * D);
   } else {
+    const PageGeo pg = page_geo(c);
     uint8_t* page = page_of(c, bh, j);
-    const uint4* codes = reinterpret_cast<const uint4*>(row_codes(page, 0, j));
+    const uint4* codes = reinterpret_cast<const uint4*>(row_codes(pg, page, 0, j));
 #pragma unroll
-    for (int i = 0; i < 4; ++i) k.code[i] = codes[i];
-    k.sz = *reinterpret_cast<const uint4*>(row_sz(page, 0, j));
-    k.mask = *reinterpret_cast<const uint2*>(page_mask(page));
-    k.vlbase = *reinterpret_cast<const int32_t*>(page + HQ_PAGE_VLBASE);
+    for (int i = 0; i < 8; ++i)
+      if (i < pg.kb) k.code[i] = codes[i];
+    k.sz = *reinterpret_cast<const uint4*>(row_sz(pg, page, 0, j));
+    k.mask = *reinterpret_cast<const uint2*>(page_mask(pg, page));
+    k.vlbase = *page_vlbase(pg, page);
     k.packed = true;
   }
   if (k.src) prefetch_l2(k.src, D * 2);
@@ -175,6 +177,37 @@ __device__ __forceinline__ void store_key_row(const SelArgs& a, int bh, const Ke
   if (src) {
 #pragma unroll
     for (int ch = 0; ch < 16; ++ch) cp_async16(stage + sw128_off(r, ch, KT * 128), src + ch);
+    return;
+  }
+  if (k.packed && kbits_of(a.c) != 4) {
+    // 8- or 2-bit codes: each 8-dim chunk from its codes, fp16(zero + q * scale) by one fma
+    const int kb = kbits_of(a.c);
+    const uint32_t szw[4] = {k.sz.x, k.sz.y, k.sz.z, k.sz.w};
+#pragma unroll
+    for (int ch = 0; ch < 16; ++ch) {
+      const uint32_t s2 = prmt(szw[ch >> 2], szw[ch >> 2], 0x1010), z2 = prmt(szw[ch >> 2], szw[ch >> 2], 0x3232);
+      uint32_t h[4];
+      if (kb == 8) {  // 8 bytes: words 2 ch, 2 ch + 1 of the 128 code bytes
+        const uint4 cw = k.code[ch >> 1];
+        const uint32_t w0 = (ch & 1) ? cw.z : cw.x, w1 = (ch & 1) ? cw.w : cw.y;
+        h[0] = prmt(w0, 0x64646464u, 0x4140);
+        h[1] = prmt(w0, 0x64646464u, 0x4342);
+        h[2] = prmt(w1, 0x64646464u, 0x4140);
+        h[3] = prmt(w1, 0x64646464u, 0x4342);
+      } else {        // 2 bytes (4 values each): bytes 2 ch, 2 ch + 1 of the 32 code bytes
+        const uint4 cw = k.code[ch >> 3];
+        const uint32_t wsel = ((ch >> 1) & 3) == 0 ? cw.x : (((ch >> 1) & 3) == 1 ? cw.y : (((ch >> 1) & 3) == 2 ? cw.z : cw.w));
+        const uint32_t x = (wsel >> (16 * (ch & 1))) & 0xFFFFu;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {  // values 2e, 2e+1 of the 8
+          const uint32_t v0 = (x >> (4 * e)) & 3u, v1 = (x >> (4 * e + 2)) & 3u;
+          h[e] = v0 | (v1 << 16) | 0x64006400u;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) h[e] = hfma2_u(hsub2_u(h[e], H2_1024), s2, z2);
+      *reinterpret_cast<uint4*>(stage + sw128_off(r, ch, KT * 128)) = make_uint4(h[0], h[1], h[2], h[3]);
+    }
     return;
   }
   if (k.packed) {
@@ -221,10 +254,13 @@ __device__ __forceinline__ void prefetch_keys(const SelArgs& a, const SelGeo& g,
     for (int q = pg; q < min(pg + 8, p1); ++q) {
       const long long idx = page_index(c, bh, q);   // a hint: entries outside the pool are skipped
       if (idx < 0) continue;
-      const uint8_t* page = c.pages + static_cast<size_t>(idx) * HQ_PAGE_BYTES;
-      prefetch_l2(page + HQ_PAGE_KCODES, 4096);
-      prefetch_l2(page + HQ_PAGE_KSZ, 1024);
-      prefetch_l2(page + HQ_PAGE_VLMASK, 16);
+      const PageGeo pgm = page_geo(c);
+      uint8_t* page = c.pages + static_cast<size_t>(idx) * pgm.bytes;
+      for (int sp = 0; sp < 64; sp += pgm.pr) {  // K codes and K (scale, zero) words of each sub-page
+        prefetch_l2(row_codes(pgm, page, 0, sp), pgm.pr * 16 * pgm.kb);
+        prefetch_l2(row_sz(pgm, page, 0, sp), pgm.pr * 16);
+      }
+      prefetch_l2(page_mask(pgm, page), 16);
     }
 }
 

@@ -43,7 +43,17 @@ class HqCacheStruct(ctypes.Structure):
         (n, ctypes.c_void_p)
         for n in ("pages", "kf", "vf", "vl_pos", "kr", "vr", "qbuf", "vl_sel", "state", "page_table", "score_acc",
                   "qlse")
-    ] + [("n_pages", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+    ] + [("n_pages", ctypes.c_int32), ("k_bits", ctypes.c_int32), ("v_bits", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+def page_layout(k_bits: int = 4, v_bits: int = 4) -> dict:
+    """Page geometry of a code width pair (include/hq.h, HQ_PAGE_SUBPOS and friends)."""
+    pr = 32 if k_bits + v_bits > 8 else 64
+    sub = pr * (16 * k_bits + 16 * v_bits + 32)
+    mask = (64 // pr) * sub
+    return {"pr": pr, "sub": sub, "mask": mask, "bytes": (mask + 16 + 63) // 64 * 64,
+            "kcodes": 0, "vcodes": pr * 16 * k_bits, "ksz": pr * 16 * (k_bits + v_bits),
+            "vsz": pr * 16 * (k_bits + v_bits) + pr * 16}
 
 
 _P = ctypes.c_void_p
@@ -127,25 +137,28 @@ class HybridCache:
 
     def __init__(self, B: int, Hq: int, Hkv: int, cap: int, W: int = 128, rho_bp: int = 500, vl_cap: int = None,
                  device="cuda", D: int = HQ_HEAD_DIM, paged: bool = False, n_pages: int = None, page_order=None,
-                 running_scores: bool = False, decode_lse: bool = True):
+                 running_scores: bool = False, decode_lse: bool = True, k_bits: int = 4, v_bits: int = 4):
         cap = ((cap + 127) // 128) * 128
         if vl_cap is None:
             vl_cap = max(16, ((k_of(max(cap - W, 0), rho_bp) + 15) // 16) * 16)
         self.B, self.Hq, self.Hkv, self.D, self.W, self.rho_bp, self.cap, self.vl_cap = B, Hq, Hkv, D, W, rho_bp, cap, vl_cap
         self.R = ((W + HQ_STAGE + 15) // 16) * 16   # HQ_RING_LEN(W)
         self.npg = cap // PAGE_POSITIONS
+        self.k_bits, self.v_bits = k_bits, v_bits
+        self.layout = page_layout(k_bits, v_bits)
+        PB = self.layout["bytes"]
         dev = torch.device(device)
         z = lambda shape, dt: torch.zeros(shape, dtype=dt, device=dev)
         self.paged = paged
         if paged:
             self.n_pages = n_pages if n_pages is not None else B * Hkv * self.npg
-            self.pages = z((self.n_pages, PAGE_BYTES), torch.uint8)
+            self.pages = z((self.n_pages, PB), torch.uint8)
             order = torch.arange(B * Hkv * self.npg, dtype=torch.int32) if page_order is None else \
                 torch.as_tensor(page_order, dtype=torch.int32)
             self.page_table = order.reshape(B, Hkv, self.npg).to(dev).contiguous()
         else:
             self.n_pages = 0
-            self.pages = z((B, Hkv, self.npg, PAGE_BYTES), torch.uint8)
+            self.pages = z((B, Hkv, self.npg, PB), torch.uint8)
             self.page_table = None
         self.kf = z((B, Hkv, vl_cap, D), torch.float16)
         self.vf = z((B, Hkv, vl_cap, D), torch.float16)
@@ -161,7 +174,7 @@ class HybridCache:
             self.pages, self.kf, self.vf, self.vl_pos, self.kr, self.vr, self.qbuf, self.vl_sel, self.state_t)],
             self.page_table.data_ptr() if paged else None,
             self.score_acc.data_ptr() if running_scores else None,
-            self.qlse.data_ptr() if decode_lse else None, self.n_pages, 0)
+            self.qlse.data_ptr() if decode_lse else None, self.n_pages, k_bits, v_bits, 0)
         _check(_lib.hq_cache_validate(ctypes.byref(self.c)), "hq_cache_validate")
         self._ws = {}
 
@@ -217,16 +230,21 @@ class HybridCache:
         return pg[np.clip(tab, 0, self.n_pages - 1)]
 
     def packed(self) -> dict:
-        """The K4V4 store by position (host copies): codes kq/vq uint8 [B,Hkv,cap,D/2],
+        """The packed store by position (host copies): codes kq/vq uint8 [B,Hkv,cap,16*bits],
         scale/zero words ksz/vsz uint32 [B,Hkv,cap,D/32], VL bitmap vl_bits bool [B,Hkv,cap]."""
         pg = self.page_bytes()
         B, H, npg, _ = pg.shape
-        D = self.D
-        take = lambda off, width: pg[..., off:off + 64 * width].reshape(B, H, npg * 64, width)
-        m = pg[..., PAGE_VLMASK:PAGE_VLMASK + 8].copy()
+        ly = self.layout
+        pr, nsub = ly["pr"], 64 // ly["pr"]
+
+        def take(off, width):
+            parts = [pg[..., s * ly["sub"] + off:s * ly["sub"] + off + pr * width].reshape(B, H, npg, pr, width)
+                     for s in range(nsub)]
+            return np.concatenate(parts, axis=3).reshape(B, H, npg * 64, width)
+        m = pg[..., ly["mask"]:ly["mask"] + 8].copy()
         bits = np.unpackbits(m, axis=-1, bitorder="little").reshape(B, H, npg * 64).astype(bool)
-        return {"kq": take(PAGE_KCODES, D // 2), "vq": take(PAGE_VCODES, D // 2),
-                "ksz": take(PAGE_KSZ, 16).copy().view(np.uint32), "vsz": take(PAGE_VSZ, 16).copy().view(np.uint32),
+        return {"kq": take(ly["kcodes"], 16 * self.k_bits), "vq": take(ly["vcodes"], 16 * self.v_bits),
+                "ksz": take(ly["ksz"], 16).copy().view(np.uint32), "vsz": take(ly["vsz"], 16).copy().view(np.uint32),
                 "vl_bits": bits}
 
 
@@ -253,7 +271,8 @@ class CacheSlot:
             t.data_ptr() for t in (self.pages, self.kf, self.vf, self.vl_pos, self.kr, self.vr, self.qbuf, self.vl_sel,
                                    self.state_t)], self.page_table.data_ptr() if parent.paged else None,
             self.score_acc.data_ptr() if self.score_acc is not None else None,
-            self.qlse.data_ptr() if self.qlse is not None else None, parent.n_pages, 0)
+            self.qlse.data_ptr() if self.qlse is not None else None, parent.n_pages, parent.k_bits, parent.v_bits, 0)
+        self.k_bits, self.v_bits, self.layout = parent.k_bits, parent.v_bits, parent.layout
         _check(_lib.hq_cache_validate(ctypes.byref(self.c)), "hq_cache_validate (slot)")
         self._ws = {}
 

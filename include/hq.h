@@ -74,6 +74,17 @@ extern "C" {
 #define HQ_PAGE_VSZ 9216        /* [64][D/32] uint32 V (scale | zero << 16) */
 #define HQ_PAGE_VLMASK 10240    /* 2 uint32: bit r of word r/32 <=> position 64 j + r is a vertical line */
 #define HQ_PAGE_VLBASE 10248    /* int32: VL-store row of the page's first vertical line (valid when the bitmap is non-zero) */
+/* Other code widths (k_bits, v_bits in {2, 4, 8}; README Mode reference: K8V8,
+ * K4V2, K2V4 beside K4V4).  Same scale/zero rule with 2^bits - 1 levels and
+ * 8 / bits codes per byte, lowest bits first.  A page of 64 positions is cut
+ * into sub-pages of HQ_PAGE_SUBPOS(kb, vb) positions (64, or 32 when kb + vb >
+ * 8), each laid out [K codes][V codes][K (scale|zero) words][V words] with
+ * 16 * bits bytes of codes per position; the bitmap and the first-VL row follow
+ * the sub-pages.  For kb = vb = 4 this is exactly the HQ_PAGE_* layout above. */
+#define HQ_PAGE_SUBPOS(kb, vb) (((kb) + (vb)) > 8 ? 32 : 64)
+#define HQ_PAGE_SUBBYTES(kb, vb) (HQ_PAGE_SUBPOS(kb, vb) * (16 * (kb) + 16 * (vb) + 32))
+#define HQ_PAGE_MASK_OFF(kb, vb) ((64 / HQ_PAGE_SUBPOS(kb, vb)) * HQ_PAGE_SUBBYTES(kb, vb))
+#define HQ_PAGE_BYTES_KV(kb, vb) (((HQ_PAGE_MASK_OFF(kb, vb) + 16) + 63) / 64 * 64)
 /* FP16 ring length for a window W: W + HQ_STAGE rounded up to a multiple of 16 */
 #define HQ_RING_LEN(W) ((((W) + HQ_STAGE) + 15) / 16 * 16)
 
@@ -119,8 +130,8 @@ enum {
  * device memory laid out as stated ([..] = row-major shape, innermost last).
  * R = HQ_RING_LEN(W) is the FP16 ring length (W + HQ_STAGE rounded up to 16).
  *
- *   pages     uint8  [B, Hkv, cap/64, HQ_PAGE_BYTES]  (page_table == NULL) or a page pool
- *             uint8  [n_pages, HQ_PAGE_BYTES] (page_table != NULL): the K4V4 store, one page per 64
+ *   pages     uint8  [B, Hkv, cap/64, PB]  (page_table == NULL) or a page pool uint8 [n_pages, PB]
+ *             (page_table != NULL), PB = HQ_PAGE_BYTES_KV(k_bits, v_bits): the K4V4 store, one page per 64
  *             positions (layout HQ_PAGE_*): codes of both K and V, their per-group
  *             (scale, zero) words and the VL bitmap of the page's positions, so
  *             that one contiguous copy brings a whole page on chip, and the VL-store
@@ -151,7 +162,8 @@ enum {
  * Limits checked by hq_cache_validate(): D == 128; Hq % Hkv == 0 and
  * Hq / Hkv <= HQ_MAX_GQA; W >= 0; 0 <= rho_bp <= 10000; cap a positive
  * multiple of 128; vl_cap a positive multiple of 16; with a page table,
- * n_pages >= 1.
+ * n_pages >= 1; (k_bits, v_bits) one of (4, 4), (8, 8), (4, 2), (2, 4).
+ * Pages are HQ_PAGE_BYTES_KV(k_bits, v_bits) bytes.
  * Fields W and rho_bp fix the method's window and VL ratio (basis points:
  * 500 = 5 %).  The fp16 positions in [n_packed, T) live in the ring, VL rows
  * in kf/vf, every other position < n_packed is read from its K4V4 record.
@@ -172,6 +184,8 @@ typedef struct hq_cache {
   float* score_acc;
   float* qlse;
   int32_t n_pages;
+  int32_t k_bits;     /* code bits of packed keys: 4 (0 means 4), 8 or 2 */
+  int32_t v_bits;     /* code bits of packed values: 4 (0 means 4), 8 or 2 */
   int32_t reserved;   /* 0 */
 } hq_cache;
 

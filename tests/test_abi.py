@@ -53,7 +53,9 @@ def test_host_validation_without_gpu():
     # the optional page table (4-byte aligned, a non-empty pool) and running scores (16-byte aligned)
     for fields, want in (({"page_table": base + 4, "n_pages": 3}, 0), ({"page_table": base + 2, "n_pages": 3}, 1),
                          ({"page_table": base, "n_pages": 0}, 1), ({"score_acc": base + 16}, 0),
-                         ({"score_acc": base + 8}, 1)):
+                         ({"score_acc": base + 8}, 1), ({"k_bits": 8, "v_bits": 8}, 0), ({"k_bits": 4, "v_bits": 2}, 0),
+                         ({"k_bits": 2, "v_bits": 4}, 0), ({"k_bits": 8, "v_bits": 4}, 2), ({"k_bits": 3}, 1),
+                         ({"v_bits": 16}, 1)):
         opt = HqCacheStruct.from_buffer_copy(good)
         for k, v in fields.items():
             setattr(opt, k, v)
