@@ -878,6 +878,41 @@ def profile_decode():
     print("profile-decode ok", st)
 
 
+PROFILE_DECODE_CAPTURED = 2   # the decode launch the ncu capture of --profile-decode selects (-s 2 -c 1)
+
+
+def write_traffic_record(csv_path):
+    """Write profiles/decode_kernel_32k.traffic.json from the raw page of the
+    ncu capture of --profile-decode (`ncu -i <report> --page raw --csv`): the
+    captured launch's DRAM read + write bytes beside its T and its algorithmic
+    bytes, stamped with the kernel sources it was taken on."""
+    import csv
+    rows = list(csv.reader(open(csv_path)))
+    head, units = rows[0], rows[1]
+    data = [r for r in rows[2:] if len(r) == len(head) and "decode_kernel" in " ".join(r)]
+    assert len(data) == 1, f"expected one decode_kernel launch in {csv_path}, found {len(data)}"
+    scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "KB": 1e3, "MB": 1e6, "GB": 1e9}
+
+    def metric(name):
+        i = head.index(name)
+        return float(data[0][i].replace(",", "")) * scale[units[i]]
+    rd, wr = metric("dram__bytes_read.sum"), metric("dram__bytes_write.sum")
+    T = L + PROFILE_DECODE_CAPTURED
+    n_packed = L - W
+    rec = {"kernel": "decode_kernel", "workload": f"one decode launch of the 32K layer (B={B}, Hq={HQ}, Hkv={HKV}), "
+                                                  f"launch {PROFILE_DECODE_CAPTURED} of --profile-decode, L2 flushed before it",
+           "T": T, "n_packed": n_packed, "n_vl": k_of(n_packed, RHO_BP),
+           "algorithmic_bytes": decode_bytes(n_packed, k_of(n_packed, RHO_BP), T),
+           "dram_read_bytes": rd, "dram_write_bytes": wr, "dram_bytes": rd + wr,
+           "command": "ncu --set full --clock-control none -k regex:decode_kernel -s 2 -c 1 -o prof_decode "
+                      "python bench.py --profile-decode",
+           "sources_sha256": kernel_sources_sha("decode.cu")}
+    rec["traffic_over_algorithmic"] = rec["dram_bytes"] / rec["algorithmic_bytes"]
+    out = os.path.join(ROOT, "profiles", "decode_kernel_32k.traffic.json")
+    json.dump(rec, open(out, "w"), indent=1)
+    print(json.dumps(rec))
+
+
 def profile_select():
     """Small case for ncu captures: a decode-mode reselection of one 32K layer (prefix install, 64 decode
     steps filling the query buffer, L2 flushed, then hq_select_vlines: two passes and the top-k)."""
@@ -935,7 +970,12 @@ def main():
     ap.add_argument("--profile-decode", action="store_true", help="small case for ncu: 4 decode steps of one 32K layer")
     ap.add_argument("--profile-prefill", action="store_true", help="small case for ncu: 3 prefill calls at L=8192")
     ap.add_argument("--profile-select", action="store_true", help="small case for ncu: one decode-mode reselection at 32K")
+    ap.add_argument("--traffic-record", metavar="CSV", help="write the decode DRAM-traffic record from the raw-page csv "
+                                                           "of the --profile-decode ncu capture")
     args = ap.parse_args()
+    if args.traffic_record:
+        write_traffic_record(args.traffic_record)
+        return
     if args.profile_decode:
         profile_decode()
         return

@@ -131,12 +131,12 @@ enum {
  * R = HQ_RING_LEN(W) is the FP16 ring length (W + HQ_STAGE rounded up to 16).
  *
  *   pages     uint8  [B, Hkv, cap/64, PB]  (page_table == NULL) or a page pool uint8 [n_pages, PB]
- *             (page_table != NULL), PB = HQ_PAGE_BYTES_KV(k_bits, v_bits): the K4V4 store, one page per 64
- *             positions (layout HQ_PAGE_*): codes of both K and V, their per-group
- *             (scale, zero) words and the VL bitmap of the page's positions, so
- *             that one contiguous copy brings a whole page on chip, and the VL-store
- *             row of the page's first vertical line; bytes 10252 .. HQ_PAGE_BYTES-1
- *             are padding
+ *             (page_table != NULL), PB = HQ_PAGE_BYTES_KV(k_bits, v_bits): the packed store, one page per
+ *             64 positions (layout HQ_PAGE_* for K4V4, sub-pages for the other widths): codes
+ *             of both K and V, their per-group (scale, zero) words and the VL bitmap of the
+ *             page's positions, so that one contiguous copy brings a whole (sub-)page on chip,
+ *             then the VL-store row of the page's first vertical line (at
+ *             HQ_PAGE_MASK_OFF(k_bits, v_bits) + 8); the bytes after it up to PB are padding
  *   kf, vf    fp16   [B, Hkv, vl_cap, D]  VL store rows, in vl_pos order
  *   vl_pos    int32  [B, Hkv, vl_cap]     VL positions, ascending (first n_vl valid)
  *   kr, vr    fp16   [B, Hkv, R, D]       recent window + staging; position p at slot p % R
