@@ -122,6 +122,13 @@ __host__ __device__ __forceinline__ int32_t* page_vlbase(const PageGeo& pg, uint
 // release / acquire fences at GPU scope (cheaper than the sequentially
 // consistent fence behind __threadfence)
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+// atomic add with acquire-release semantics at gpu scope (a completion ticket:
+// releases what this CTA did before it, acquires what earlier ticket holders did)
+__device__ __forceinline__ unsigned int atom_add_acq_rel_gpu(unsigned int* p, unsigned int v) {
+  unsigned int r;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(r) : "l"(p), "r"(v) : "memory");
+  return r;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

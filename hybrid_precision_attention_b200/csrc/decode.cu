@@ -909,14 +909,12 @@ __device__ __forceinline__ void segment_epilogue(const hq_cache& c, const uint16
   // the barrier that releases its other threads to read the partials
   // With its last segment the CTA also takes its grid ticket: it has read
   // every length it needs, and the last grid ticket advances the lengths.
+  // The two tickets are taken by two threads at once (one round trip to L2).
   consumer_bar();  // (B) partial written, warp states read
   if (threadIdx.x == 0) {
-    fence_acq_rel_gpu();
-    const unsigned int th = atomicAdd(&tickets[1 + u], 1u);
-    const bool glast = si == nseg - 1 && atomicAdd(&tickets[0], 1u) == gridDim.x - 1;
-    s_last = th == static_cast<unsigned>(sg.ncta - 1);
-    s_glast = glast;
-    if (s_last || glast) fence_acq_rel_gpu();
+    s_last = atom_add_acq_rel_gpu(&tickets[1 + u], 1u) == static_cast<unsigned>(sg.ncta - 1);
+  } else if (threadIdx.x == 32) {
+    s_glast = si == nseg - 1 && atom_add_acq_rel_gpu(&tickets[0], 1u) == gridDim.x - 1;
   }
   consumer_bar();  // (C)
   if (s_glast) advance_lengths(c, threadIdx.x, NC * 32, tickets);
@@ -931,7 +929,7 @@ __device__ __forceinline__ void segment_epilogue(const hq_cache& c, const uint16
     float* sm_m = reinterpret_cast<float*>(smem + scratch * STAGE_BYTES);  // [S][8] weights
     float* sm_inv = sm_m + 8 * S;                                          // [8]
     float4* red4 = reinterpret_cast<float4*>(sm_inv + 8);                  // [ngrp][items]
-    constexpr int PER = 8;
+    constexpr int PER = 12;
     const int items = G * (D / 4);
     const int room = (STAGE_BYTES - 4 * (8 * S + 8)) / (16 * items);      // groups the scratch stage holds
     const int ngrp = max(1, min(min(NTHR / items, S), room));
@@ -946,17 +944,30 @@ __device__ __forceinline__ void segment_epilogue(const hq_cache& c, const uint16
       ov[j] = (mine && sp < S) ? __ldcg(osrc + sp * (PART_FLOATS / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     // partial weights: warp qc weighs query qc's partials, lane s holding s, s + 32, ...
+    // (each lane loads its partials' m and l once, in one round trip)
+    constexpr int SPL = (MAX_CTAS + 31) / 32;  // partials per lane
     for (int qc = warp; qc < G; qc += NC) {
-      float mm = -INFINITY;
-      for (int sp = lane; sp < S; sp += 32) mm = fmaxf(mm, __ldcg(pb + sp * PART_FLOATS + qc));
+      float mv[SPL], lv[SPL];
+#pragma unroll
+      for (int j = 0; j < SPL; ++j) {
+        const int sp = lane + 32 * j;
+        mv[j] = sp < S ? __ldcg(pb + sp * PART_FLOATS + qc) : -INFINITY;
+        lv[j] = sp < S ? __ldcg(pb + sp * PART_FLOATS + 8 + qc) : 0.f;
+      }
+      float mm = mv[0];
+#pragma unroll
+      for (int j = 1; j < SPL; ++j) mm = fmaxf(mm, mv[j]);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, o));
       float ll = 0.f;
-      for (int sp = lane; sp < S; sp += 32) {
-        const float m0 = __ldcg(pb + sp * PART_FLOATS + qc);
-        const float w0 = m0 == -INFINITY ? 0.f : ex2(m0 - mm);
-        ll = fmaf(w0, __ldcg(pb + sp * PART_FLOATS + 8 + qc), ll);
-        sm_m[sp * 8 + qc] = w0;
+#pragma unroll
+      for (int j = 0; j < SPL; ++j) {
+        const int sp = lane + 32 * j;
+        if (sp < S) {
+          const float w0 = mv[j] == -INFINITY ? 0.f : ex2(mv[j] - mm);
+          ll = fmaf(w0, lv[j], ll);
+          sm_m[sp * 8 + qc] = w0;
+        }
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) ll += __shfl_xor_sync(0xffffffffu, ll, o);
@@ -1112,11 +1123,7 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
 
   if (ntile == 0) {
     // no tiles for this CTA: it only takes its grid ticket
-    if (threadIdx.x == 0) {
-      fence_acq_rel_gpu();
-      s_glast = atomicAdd(&tickets[0], 1u) == gridDim.x - 1;
-      if (s_glast) fence_acq_rel_gpu();
-    }
+    if (threadIdx.x == 0) s_glast = atom_add_acq_rel_gpu(&tickets[0], 1u) == gridDim.x - 1;
     __syncthreads();
     if (s_glast) advance_lengths(c, threadIdx.x, NTHREADS, tickets);
   } else if (warp == NC) {
