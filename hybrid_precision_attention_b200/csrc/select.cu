@@ -19,11 +19,14 @@
 //                    exp2(s - lse) -> score_j, and a histogram of the scores'
 //                    bits 30..20 (scores are >= 0, so the bit order is the value
 //                    order).  Each key's score is finished inside one CTA.
-//   topk             one CTA per (b, kv head): the bin holding the k-th largest
-//                    score from the histogram, the bin's scores gathered into
-//                    shared memory, a bit-by-bit search of their low 20 bits ->
-//                    the exact k-th value, then an ordered compaction writes the
-//                    chosen positions ascending, ties to the lowest positions
+//   topk             a cluster of 8 CTAs per (b, kv head), each over an eighth
+//                    of the positions (one CTA when a range would not fit its
+//                    shared memory): the bin holding the k-th largest score from
+//                    the histogram, the bin's scores gathered, two 10-bit radix
+//                    passes over their low 20 bits (histograms summed across the
+//                    cluster) -> the exact k-th value, then an ordered compaction
+//                    writes the chosen positions ascending, ties to the lowest
+//                    positions
 // When the decode steps kept their log-sum-exps (c.qlse) and every buffered
 // query came after the last merge, pass 0 is skipped: those are its row sums.
 // With running scores (c.score_acc), pass 1 adds each key's column mass to its
@@ -36,6 +39,8 @@
 // warp 12 TMEM allocation and the MMA issue.  Every mbarrier wait is bounded
 // (about 1 s); a timeout sets HQ_DEVERR_TIMEOUT and the CTA drains its MMAs
 // before releasing TMEM.
+#include <cooperative_groups.h>
+
 #include "tc.cuh"
 
 namespace hq {
@@ -794,6 +799,203 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(SelArgs a, int smem_sc
 }
 
 
+// The same top-k spread over a cluster of TKC_CS CTAs per (b, kv head): CTA r
+// owns positions [r P, (r + 1) P).  Each CTA takes the threshold bin from the
+// global histogram, gathers its range's values of that bin, and builds a local
+// histogram of each radix pass; the cluster sums the local histograms through
+// distributed shared memory, so every CTA finds the same sub-bin.  The ordered
+// compaction offsets each CTA by the counts of the lower-ranked CTAs (read the
+// same way).  Same result as topk_kernel, bit for bit.
+constexpr int TKC_CS = 8;                 // CTAs per (b, kv head): one portable cluster
+constexpr int TKC_THREADS = 512;
+constexpr int TKC_PMAX = 24576;           // positions per CTA held in shared memory (scores and bin values)
+
+__device__ __forceinline__ unsigned int tkc_block_scan(unsigned int x, unsigned int* wsum, int lane, int warp) {
+  // inclusive scan over the block's threads in thread order
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wsum[warp] = x;
+  __syncthreads();
+  for (int w = 0; w < warp; ++w) x += wsum[w];
+  return x;
+}
+
+__global__ void __cluster_dims__(TKC_CS, 1, 1) __launch_bounds__(TKC_THREADS) topk_cluster_kernel(SelArgs a) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  const hq_cache& c = a.c;
+  const int rank = static_cast<int>(cl.block_rank());
+  const int bh = blockIdx.x / TKC_CS;
+  const int b = bh / c.Hkv;
+  int32_t* const srow = state_row(c, b);
+  const SelGeo g = sel_geo(a, b);
+  const int n = g.n;
+  int k = 0;
+  if (n > 0 && c.rho_bp > 0) {
+    const long long kk = (static_cast<long long>(n) * c.rho_bp + 9999) / 10000;
+    k = static_cast<int>(min(static_cast<long long>(n), kk));
+  }
+  if (k > c.vl_cap) {
+    if (rank == 0 && bh % c.Hkv == 0 && threadIdx.x == 0) set_err(srow, HQ_DEVERR_VL_CAPACITY);
+    k = c.vl_cap;
+  }
+  if (rank == 0 && bh % c.Hkv == 0 && threadIdx.x == 0) srow[HQ_STATE_KSEL] = k;
+  if (k == 0) return;  // the same for every CTA of the cluster: no shared-memory exchange follows
+  extern __shared__ uint32_t tkc_smem[];  // [P] scores of the range, then [P] values of the threshold bin
+  __shared__ unsigned int h10[1024];       // local histogram of the current radix pass
+  __shared__ unsigned int wsum[TKC_THREADS / 32], rg[TKC_THREADS / 32], re[TKC_THREADS / 32];
+  __shared__ unsigned int s_bin, s_above, s_cnt, s_tot[2];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int P = ((n + TKC_CS - 1) / TKC_CS + 31) / 32 * 32;
+  const int lo = min(n, rank * P), hi = min(n, lo + P), m = hi - lo;
+  uint32_t* sc = tkc_smem;
+  uint32_t* cand = tkc_smem + P;
+  const uint32_t* gsc = reinterpret_cast<const uint32_t*>(a.scores + static_cast<size_t>(bh) * c.cap);
+#pragma unroll 4
+  for (int j = threadIdx.x; j < m; j += TKC_THREADS) sc[j] = __ldcg(gsc + lo + j);
+  const uint32_t* hh = a.hist + static_cast<size_t>(bh) * HBINS;
+  int32_t* out = c.vl_sel + static_cast<size_t>(bh) * c.vl_cap;
+
+  // (1) the threshold bin: thread i owns bins 2047 - 4i .. 2044 - 4i (descending)
+  {
+    const int d_hi = HBINS - 1 - 4 * static_cast<int>(threadIdx.x);
+    unsigned int h[4], x = 0u;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      h[j] = __ldcg(hh + d_hi - j);
+      x += h[j];
+    }
+    if (threadIdx.x == 0) {
+      s_bin = 0u;  // only if the histogram disagreed with the scores (never expected)
+      s_above = 0u;
+      s_cnt = 0u;
+    }
+    const unsigned int X = tkc_block_scan(x, wsum, lane, warp);
+    unsigned int above = X - x;  // values in bins > d_hi
+    const unsigned int kk = static_cast<unsigned int>(k);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (above < kk && above + h[j] >= kk) {
+        s_bin = static_cast<unsigned int>(d_hi - j);
+        s_above = above;
+      }
+      above += h[j];
+    }
+    __syncthreads();
+  }
+  const uint32_t bin = s_bin;
+  // (2) this range's values of the threshold bin
+  for (int j0 = 0; j0 < m; j0 += TKC_THREADS) {
+    const int j = j0 + threadIdx.x;
+    const uint32_t v = j < m ? sc[j] : 0u;
+    const bool hit = j < m && (v >> 20) == bin;
+    const unsigned int msk = __ballot_sync(0xffffffffu, hit);
+    unsigned int base = 0u;
+    if (lane == 0 && msk) base = atomicAdd(&s_cnt, static_cast<unsigned>(__popc(msk)));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    if (hit) cand[base + __popc(msk & ((1u << lane) - 1u))] = v;  // at most m <= P values
+  }
+  __syncthreads();
+  const int ncand = static_cast<int>(s_cnt);
+  // (3) the low 20 bits of the k-th largest: two radix passes of 10 bits, the
+  // cluster's histograms summed from every CTA's shared memory
+  uint32_t prefix = bin << 20, pmask = 0xFFF00000u;
+  unsigned int above = s_above;
+#pragma unroll 1
+  for (int pass = 0; pass < 2; ++pass) {
+    const int shift = pass == 0 ? 10 : 0;
+    h10[threadIdx.x] = 0u;
+    h10[threadIdx.x + TKC_THREADS] = 0u;
+    __syncthreads();
+    for (int e = threadIdx.x; e < ncand; e += TKC_THREADS) {
+      const uint32_t v = cand[e];
+      if ((v & pmask) == prefix) atomicAdd(&h10[(v >> shift) & 1023u], 1u);
+    }
+    cl.sync();  // every CTA's histogram complete
+    // thread i owns sub-bins 1023 - 2i and 1022 - 2i (descending)
+    const int d1 = 1023 - 2 * static_cast<int>(threadIdx.x), d0 = d1 - 1;
+    unsigned int g1 = 0u, g0 = 0u;
+#pragma unroll
+    for (int r = 0; r < TKC_CS; ++r) {
+      const unsigned int* rh = cl.map_shared_rank(h10, r);
+      g1 += rh[d1];
+      g0 += rh[d0];
+    }
+    cl.sync();  // every CTA done reading the histograms before they are cleared or reused
+    const unsigned int X = tkc_block_scan(g1 + g0, wsum, lane, warp);
+    const unsigned int up = X - g1 - g0;  // values (within the prefix) in sub-bins above d1
+    const unsigned int needp = static_cast<unsigned int>(k) - above;
+    if (up < needp && up + g1 >= needp) {
+      s_bin = static_cast<unsigned int>(d1);
+      s_above = above + up;
+    } else if (up + g1 < needp && up + g1 + g0 >= needp) {
+      s_bin = static_cast<unsigned int>(d0);
+      s_above = above + up + g1;
+    }
+    __syncthreads();
+    prefix |= s_bin << shift;
+    pmask |= 1023u << shift;
+    above = s_above;
+    __syncthreads();
+  }
+  const uint32_t thr = prefix;
+  const unsigned int take_eq = static_cast<unsigned int>(k) - above;
+  // (4) ordered compaction: warp w owns the range's positions [w Pw, (w + 1) Pw);
+  // counts per warp, per CTA, then the lower-ranked CTAs' totals give the offsets
+  const int Pw = ((m + TKC_THREADS / 32 - 1) / (TKC_THREADS / 32) + 31) / 32 * 32;
+  const int j_lo = min(m, warp * Pw), j_hi = min(m, j_lo + Pw);
+  unsigned int cg_ = 0u, ce = 0u;
+  for (int j0 = j_lo; j0 < j_hi; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t v = j < j_hi ? sc[j] : 0u;
+    cg_ += __popc(__ballot_sync(0xffffffffu, j < j_hi && v > thr));
+    ce += __popc(__ballot_sync(0xffffffffu, j < j_hi && v == thr));
+  }
+  if (lane == 0) {
+    rg[warp] = cg_;
+    re[warp] = ce;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned int tg = 0u, te = 0u;
+    for (int w = 0; w < TKC_THREADS / 32; ++w) {
+      tg += rg[w];
+      te += re[w];
+    }
+    s_tot[0] = tg;
+    s_tot[1] = te;
+  }
+  cl.sync();  // every CTA's totals visible
+  unsigned int xg = 0u, xe = 0u;
+  for (int r = 0; r < rank; ++r) {
+    const unsigned int* rt = cl.map_shared_rank(s_tot, r);
+    xg += rt[0];
+    xe += rt[1];
+  }
+  for (int w = 0; w < warp; ++w) {
+    xg += rg[w];
+    xe += re[w];
+  }
+  const unsigned int lt_mask = (1u << lane) - 1u;
+  for (int j0 = j_lo; j0 < j_hi; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t v = j < j_hi ? sc[j] : 0u;
+    const bool gt = j < j_hi && v > thr, eq = j < j_hi && v == thr;
+    const unsigned int bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
+    const unsigned int mg = xg + __popc(bg & lt_mask), me = xe + __popc(be & lt_mask);
+    // (the bounds hold whenever the histogram agrees with the scores, as it does by construction)
+    const unsigned int kk = static_cast<unsigned int>(k);
+    if (gt && mg + min(me, take_eq) < kk) out[mg + min(me, take_eq)] = lo + j;
+    else if (eq && me < take_eq && mg + me < kk) out[mg + me] = lo + j;
+    xg += __popc(bg);
+    xe += __popc(be);
+  }
+  cl.sync();  // no CTA leaves while another may still read its shared memory
+}
+
 int sel_mp(const hq_cache& c) { return (((c.Hq / c.Hkv) * HQ_QBUF + 127) / 128) * 128; }
 
 size_t sel_smem_bytes(int Mp) {
@@ -843,6 +1045,8 @@ hq_status launch_select(const hq_cache& c, const uint16_t* kd, int L, const uint
     if (e == cudaSuccess) e = cudaFuncSetAttribute(sel_pass<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (TK_CAND_MAX + TK_SMEM_MAX) * 4);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * TKC_PMAX * 4);
     return e;
   });
   if (ea != cudaSuccess) return cuda_fail(ea, "select setup");
@@ -852,9 +1056,17 @@ hq_status launch_select(const hq_cache& c, const uint16_t* kd, int L, const uint
   dim3 grid(S, c.Hkv, c.B);
   sel_pass<false><<<grid, SEL_THREADS, smem, st>>>(a);
   sel_pass<true><<<grid, SEL_THREADS, smem, st>>>(a);
-  // shared memory: the bin's values and, when they fit, the scores themselves
-  const int smem_scores = min(max(keys_cap - c.W, 0), TK_SMEM_MAX);
-  topk_kernel<<<c.B * c.Hkv, TK_THREADS, static_cast<size_t>(TK_CAND_MAX + smem_scores) * 4, st>>>(a, smem_scores);
+  // top-k: a cluster of TKC_CS CTAs per (b, kv head) when a CTA's range of
+  // the candidates fits its shared memory, else one CTA per (b, kv head)
+  const int n_max = max(keys_cap - c.W, 0);
+  const int P_max = ((n_max + TKC_CS - 1) / TKC_CS + 31) / 32 * 32;
+  if (P_max <= TKC_PMAX) {
+    topk_cluster_kernel<<<c.B * c.Hkv * TKC_CS, TKC_THREADS, static_cast<size_t>(2 * max(P_max, 32)) * 4, st>>>(a);
+  } else {
+    // shared memory: the bin's values and, when they fit, the scores themselves
+    const int smem_scores = min(n_max, TK_SMEM_MAX);
+    topk_kernel<<<c.B * c.Hkv, TK_THREADS, static_cast<size_t>(TK_CAND_MAX + smem_scores) * 4, st>>>(a, smem_scores);
+  }
   return cuda_status(cudaGetLastError(), "select launch");
 }
 
