@@ -13,6 +13,7 @@ import pytest
 
 from hybrid_precision_attention_b200 import synth
 from tests._gpu import Pair, check_decode, dev, hq
+from tests.test_gpu_varlen import Ragged
 
 pytestmark = pytest.mark.gpu
 
@@ -61,3 +62,55 @@ def test_widths_full_size_32k(kb, vb):
     p.reselect_merge()
     out, ref = p.decode(q[64], k[64], v[64])
     check_decode(out, ref, f"K{kb}V{vb} after merge")
+
+
+@pytest.mark.parametrize("kb,vb", [(8, 8), (2, 4), (4, 2)])
+def test_widths_ragged_paged_batch(kb, vb):
+    """Three sequences of 200, 700 and 1000 tokens (GQA 4, W = 64) in a shuffled
+    page pool at each width (K8V8 pages hold two 32-position sub-pages): one
+    install per sequence, a batched period, reselection and merge, three more
+    steps, every sequence against its own oracle."""
+    rg = Ragged([200, 700, 1000], 8, 2, 64, 500, cap=1300, seed=40 + kb + vb, k_bits=kb, v_bits=vb)
+    for b in range(rg.B):
+        rg.install(b)
+        rg.check_store(b)
+    q, k, v = synth.decode_tokens(41, rg.B, 8, 2, 67)
+    for t in range(64):
+        rg.decode(q[t], k[t], v[t], check=(t % 13 == 0 or t == 63))
+    rg.reselect_merge()
+    for t in range(64, 67):
+        rg.decode(q[t], k[t], v[t])
+
+
+@pytest.mark.parametrize("kb,vb", [(8, 8), (2, 4)])
+def test_widths_running_scores(kb, vb):
+    """Running column-mass scores at the other widths: two periods, the summed
+    scores and the sets they choose against the oracle's running sums."""
+    p = Pair(1, 8, 2, 900, 64, 500, cap=1200, seed=50 + kb, running=True, k_bits=kb, v_bits=vb)
+    p.init()
+    q, k, v = synth.decode_tokens(51, 1, 8, 2, 130)
+    for period in range(2):
+        for t in range(64 * period, 64 * period + 64):
+            if t % 21 == 0:
+                out, ref = p.decode(q[t], k[t], v[t])
+                check_decode(out, ref, f"K{kb}V{vb} running, step {t}")
+            else:
+                hq().hq_decode_attn(p.g, dev(q[t]), dev(k[t]), dev(v[t]))
+                p.r.append(q[t], k[t], v[t])
+        p.reselect_merge()
+    out, ref = p.decode(q[128], k[128], v[128])
+    check_decode(out, ref, f"K{kb}V{vb} running, after two merges")
+
+
+def test_widths_allocation_free_decode():
+    """hq_decode_attn_noalloc on a K8V8 cache: the same step as the oracle's."""
+    p = Pair(1, 32, 8, 2000, 128, 500, cap=2200, seed=60, k_bits=8, v_bits=8)
+    p.init()
+    q, k, v = synth.decode_tokens(61, 1, 32, 8, 3)
+    H = hq()
+    for t in range(3):
+        out = H.hq_decode_attn_noalloc(p.g, dev(q[t]), dev(k[t]), dev(v[t]))
+        ref = p.r.decode(q[t], k[t], v[t])
+        st = p.g.state()
+        assert st["err"] == 0 and st["T"] == p.r.T, st
+        check_decode(out, ref, f"K8V8 allocation-free step {t}")

@@ -22,7 +22,7 @@ pytestmark = pytest.mark.gpu
 
 
 class Ragged:
-    def __init__(self, lengths, Hq, Hkv, W, rho, cap, seed, paged=True, spare_pages=5):
+    def __init__(self, lengths, Hq, Hkv, W, rho, cap, seed, paged=True, spare_pages=5, k_bits=4, v_bits=4):
         H = hq()
         self.lengths, self.Hq, self.Hkv, self.W, self.rho = list(lengths), Hq, Hkv, W, rho
         self.B = len(lengths)
@@ -31,8 +31,9 @@ class Ragged:
         n_pages = self.B * Hkv * npg + spare_pages
         order = np.random.default_rng(seed).permutation(n_pages)[:self.B * Hkv * npg] if paged else None
         self.g = H.HybridCache(self.B, Hq, Hkv, cap, W, rho, paged=paged, n_pages=n_pages if paged else None,
-                               page_order=order)
-        self.refs = [hybrid.HybridCacheRef(1, Hq, Hkv, W, rho, self.g.cap) for _ in lengths]
+                               page_order=order, k_bits=k_bits, v_bits=v_bits)
+        self.refs = [hybrid.HybridCacheRef(1, Hq, Hkv, W, rho, self.g.cap, k_bits=k_bits, v_bits=v_bits)
+                     for _ in lengths]
         self.lays = [synth.planted_layer(seed + 10 * b, 1, Hq, Hkv, L) for b, L in enumerate(lengths)]
 
     def install(self, b, check=True):
