@@ -72,6 +72,8 @@ def _run(B, Hq, Hkv, L, W, rho_bp, seed, rows=None, heads=None, fmt="e4m3"):
     (1, 8, 1, 400, 0, 500),       # no window: FP8 and VL only
     (1, 4, 1, 200, 500, 500),     # window longer than the prompt: plain FP16 causal
     (1, 4, 1, 384, 32, 0),        # no vertical lines
+    (1, 4, 1, 1, 128, 500),       # a one-token prompt
+    (1, 4, 2, 17, 4, 10000),      # rho = 100 %: every key outside the window is a vertical line
 ])
 @pytest.mark.parametrize("fmt", ["e4m3", "int8"])
 def test_prefill_matches_oracle(B, Hq, Hkv, L, W, rho, fmt):

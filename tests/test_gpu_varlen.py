@@ -203,3 +203,21 @@ def test_ragged_paged_batch_1k_3k_32k():
     r.reselect_merge()
     for t in range(65, 67):
         r.decode(q[t], k[t], v[t])
+
+
+def test_ragged_batch_on_the_stream_k_grid():
+    """Twelve sequences of 300 .. 2500 tokens with 4 kv heads (48 units: more
+    than a quarter of the grid, so the decode cuts the batch's tile list into
+    equal stream-K ranges whose segments cross sequences): one install per
+    sequence, a batched period, reselection and merge, two more steps, every
+    sequence against its own oracle."""
+    lengths = [300, 2500, 700, 1200, 450, 2000, 900, 1600, 333, 1800, 1100, 640]
+    rg = Ragged(lengths, 16, 4, 64, 500, cap=2700, seed=70)
+    for b in range(rg.B):
+        rg.install(b, check=(b % 4 == 0))
+    q, k, v = _tokens(71, rg.B, 16, 4, 66)
+    for t in range(64):
+        rg.decode(q[t], k[t], v[t], check=(t % 16 == 0 or t == 63))
+    rg.reselect_merge()
+    for t in range(64, 66):
+        rg.decode(q[t], k[t], v[t])
