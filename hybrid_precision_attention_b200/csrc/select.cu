@@ -345,10 +345,11 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
     tmem_alloc(&tmem_base_sh, TMEM_COLS);
     tmem_relinquish();
   }
-  // queries: row r = h * nq + i (head kvh*G + h, position qpos0 + i); rows >= M are zero
+  // queries: row r = h * nq + i (head kvh*G + h, position qpos0 + i); rows >= M are zero.
+  // Asynchronous 16-byte copies, all in flight at once (waited for below).
   for (int e = threadIdx.x; e < Mp * (D / 8); e += SEL_THREADS) {
     const int r = e / (D / 8), ch = e % (D / 8);
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    uint8_t* dst = qs + sw128_off(r, ch, Mp * 128);
     if (r < M) {
       const int h = r / g.nq, i = r % g.nq;
       const uint4* src;
@@ -358,9 +359,10 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
         const int p = g.qpos0 + i;
         src = reinterpret_cast<const uint4*>(c.qbuf + ((static_cast<size_t>(b) * c.Hq + kvh * G + h) * HQ_QBUF + (p % HQ_QBUF)) * D) + ch;
       }
-      v = *src;
+      cp_async16(dst, src);
+    } else {
+      *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
     }
-    *reinterpret_cast<uint4*>(qs + sw128_off(r, ch, Mp * 128)) = v;
   }
   for (int r = threadIdx.x; r < Mp; r += SEL_THREADS) qpos[r] = r < M ? g.qpos0 + r % max(g.nq, 1) : -1;
   if (!COL) {
@@ -394,6 +396,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
       lse[r] = z;
     }
   }
+  cp_async_wait_all();  // this thread's query copies
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
