@@ -5,6 +5,7 @@ import pytest
 import torch
 
 from hybrid_precision_attention_b200 import synth
+from oracle import hybrid
 from tests._gpu import Pair, check_decode, dev, hq
 
 pytestmark = pytest.mark.gpu
@@ -176,3 +177,38 @@ def test_running_scores_over_three_periods():
                 assert np.allclose(acc[b, h, :n], p.r.acc[b, h, :n], rtol=5e-4, atol=0), (period, b, h)
     out, ref = p.decode(q[t], k[t], v[t])
     check_decode(out, ref, "after the last merge")
+
+
+def test_reset_then_reinstall_with_running_scores():
+    """hq_cache_reset empties a used cache: every state row zero, every VL
+    bitmap cleared, the running scores zero; a different prefix installed
+    afterwards through the same buffers then matches a fresh oracle cache
+    (selection, records, decode, reselection and merge)."""
+    p = Pair(2, 8, 2, 700, 64, 500, cap=1000, seed=81, running=True)
+    p.init()
+    q, k, v = synth.decode_tokens(81, 2, 8, 2, 64)
+    for t in range(64):
+        hq().hq_decode_attn(p.g, dev(q[t]), dev(k[t]), dev(v[t]))
+        p.r.append(q[t], k[t], v[t])
+    p.reselect_merge()
+    hq().hq_cache_reset(p.g)
+    torch.cuda.synchronize()
+    assert not p.g.state_t.any()
+    assert not p.g.packed()["vl_bits"].any()
+    assert not p.g.score_acc.any()
+    # a shorter, different prefix through the same cache
+    p.lay = synth.planted_layer(82, 2, 8, 2, 400)
+    p.L = 400
+    p.r = hybrid.HybridCacheRef(2, 8, 2, 64, 500, p.g.cap, accumulate=True)
+    p.init()
+    q, k, v = synth.decode_tokens(83, 2, 8, 2, 66)
+    for t in range(64):
+        if t % 16 == 0:
+            out, ref = p.decode(q[t], k[t], v[t])
+            check_decode(out, ref, f"after reset, step {t}")
+        else:
+            hq().hq_decode_attn(p.g, dev(q[t]), dev(k[t]), dev(v[t]))
+            p.r.append(q[t], k[t], v[t])
+    p.reselect_merge()
+    out, ref = p.decode(q[64], k[64], v[64])
+    check_decode(out, ref, "after reset and a merge")

@@ -221,3 +221,31 @@ def test_ragged_batch_on_the_stream_k_grid():
     rg.reselect_merge()
     for t in range(64, 66):
         rg.decode(q[t], k[t], v[t])
+
+
+def test_one_sequence_reset_and_reused_in_a_running_batch():
+    """A finished request's slot reused: sequence 1 of a ragged paged batch is
+    reset through its single-sequence descriptor (its state row, its pages'
+    bitmaps) and given a new prompt, while sequences 0 and 2 keep their
+    caches; the batch then decodes on, every sequence against its own oracle."""
+    rg = Ragged([600, 900, 300], 8, 2, 64, 500, cap=1200, seed=90)
+    for b in range(rg.B):
+        rg.install(b, check=False)
+    q, k, v = _tokens(91, rg.B, 8, 2, 40)
+    for t in range(20):
+        rg.decode(q[t], k[t], v[t], check=(t == 19))
+    H = hq()
+    H.hq_cache_reset(rg.g.slot(1))
+    torch.cuda.synchronize()
+    st = rg.g.states()
+    assert st[1]["T"] == 0 and st[1]["n_vl"] == 0 and not rg.g.packed()["vl_bits"][1].any(), st[1]
+    assert st[0]["T"] == 620 and st[2]["T"] == 320, st
+    rg.lengths[1] = 450
+    rg.lays[1] = synth.planted_layer(92, 1, 8, 2, 450)
+    rg.refs[1] = hybrid.HybridCacheRef(1, 8, 2, 64, 500, rg.g.cap)
+    rg.install(1)
+    rg.check_store(1)
+    for t in range(20, 40):
+        rg.decode(q[t], k[t], v[t], check=(t % 6 == 0 or t == 39))
+    for b in range(rg.B):
+        rg.check_store(b)
