@@ -180,10 +180,15 @@ def decode_traffic_record(bytes_per_launch):
 
 
 def kernel_sources_sha(*names):
-    """sha256 over the named kernel sources plus the shared device header."""
+    """sha256 over the code of the named kernel sources plus the shared device
+    header: comments removed and whitespace collapsed, so a comment-only edit
+    keeps a record taken on the same code."""
     h = hashlib.sha256()
     for n in list(names) + ["common.cuh"]:
-        h.update(open(os.path.join(ROOT, "hybrid_precision_attention_b200", "csrc", n), "rb").read())
+        src = open(os.path.join(ROOT, "hybrid_precision_attention_b200", "csrc", n)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        h.update(re.sub(r"\s+", " ", src).strip().encode())
     return h.hexdigest()
 
 

@@ -8,27 +8,32 @@
 //
 // Design (bandwidth-bound: ~160 B of K4V4 per token and kv head):
 //   * work: every (b, kv head) is a unit whose tile list holds its packed
-//     tiles (one page of 64 positions: 4 KB K codes, 4 KB V codes, 1 KB + 1 KB
-//     scale/zero, the VL bitmap), its FP16 tiles (16 rows of the VL store, 16
-//     slots of the FP16 ring, which is a multiple of 16 long, so a tile is one
-//     contiguous copy) and a last tile with the new token read straight from
-//     its input pointer; the FP16 tiles are interleaved evenly among the
-//     packed ones;
-//   * grid: persistent, one CTA per SM (stream-K).  The units' tile lists are
-//     concatenated and cut into equal contiguous ranges, one per CTA, so every
-//     SM streams the same number of tiles whatever the batch size or the
-//     sequences' lengths (each sequence has its own state row); a range may
-//     cover parts of several units, one segment per unit.  Every unit also
-//     carries a small phantom weight in the cut, which bounds how many
-//     segments a range can hold;
+//     tiles (one sub-page of 64 positions, or 32 when K and V take more than 8
+//     bits together: K codes, V codes, their scale/zero words, then the page's
+//     VL bitmap), its FP16 tiles (16 rows of the VL store, 16 slots of the
+//     FP16 ring, which is a multiple of 16 long, so a tile is one contiguous
+//     copy) and a last tile with the new token read straight from its input
+//     pointer; a CTA runs its packed tiles first, then its FP16 ones;
+//   * grid: persistent, one CTA per SM, each sequence with its own state row.
+//     Few units (4 CTAs or more each): every unit gets its own CTAs in
+//     proportion to its tiles, each an even share of the unit's packed and
+//     FP16 tiles (the last 12 CTAs, which the scheduler starts last, stay
+//     idle).  Many units (stream-K): the units' tile lists are concatenated
+//     and cut into equal contiguous ranges, one per CTA, so every SM streams
+//     the same number of tiles whatever the batch size or the sequences'
+//     lengths; a range may cover parts of several units, one segment per
+//     unit, and a small phantom weight per unit bounds the segments of a
+//     range.  The plan is made before the dependency wait and kept when the
+//     lengths it used did not change;
 //   * a producer warp streams tiles into a 2 NC-stage shared-memory ring with
 //     large 1-D bulk async copies (cp.async.bulk, mbarrier completion, no
 //     multicast): 1 copy per packed tile, 2 per FP16 tile;
 //   * NC consumer warps take tiles round-robin, each owning 2 of the 2 NC
 //     stages (tile i -> stage i % 2NC -> warp i % NC), so every stage has a
 //     single consumer and a waiter is never a full barrier phase behind.
-//     Nibbles become fp16 in registers (exponent-bias trick + one fma with the
-//     group's scale/zero), and both products run on tensor cores with
+//     Codes become fp16 in registers (exponent-bias tricks for 2-, 4- and
+//     8-bit codes + one fma with the group's scale/zero; the kernel is
+//     instantiated per code width), and both products run on tensor cores with
 //     mma.m16n8k16 (f32 accumulate):
 //       S^T[keys x 8 queries] = K^ (16 keys x 16 dims) . Q^T
 //       O^T[dims x 8 queries] += V^T (16 dims x 16 keys) . P^T
@@ -41,10 +46,12 @@
 //     back from the producer until the merge is done), the consumers merge the
 //     warp states into the segment's partial (m, l, O) in the workspace, and
 //     the last CTA to finish a unit merges that unit's partials with a
-//     log-sum-exp (atomic ticket, no waiting), appends the unit's new token to
+//     log-sum-exp (an acquire-release ticket, no waiting), writes each query's
+//     log-sum-exp for the next reselection, appends the unit's new token to
 //     the ring and its queries to the query buffer (every CTA of the unit is
-//     done reading by then); the last CTA to take its grid ticket (once it
-//     has read every length it uses) advances the lengths;
+//     done reading by then); the last CTA to take its grid ticket (taken with
+//     the unit ticket, once it has read every length it uses) advances the
+//     lengths;
 //   * launched with programmatic dependent launch: a CTA prefetches its range's
 //     pages and VL rows into L2 before it waits for the previous grid, and lets
 //     the next grid launch as soon as its own wait is over.

@@ -3,12 +3,13 @@
 // HyQuant digest (agihunt.info), prefill/decode paragraph: new decode tokens
 // are staged first and merged into the hybrid layout later; the VL set chosen
 // by the selector keeps FP16 rows, everything that leaves the recent window
-// is stored 4-bit.  The K4V4 arithmetic follows the format definition in
-// hq.h exactly (float32 RN subtract/divide, rint to even, fp16 RN), so the
-// packed bytes are bit-identical to the definition.
+// is stored 4-bit (or, with the cache's k_bits / v_bits, 2- or 8-bit; README
+// Mode reference).  The arithmetic follows the format definition in hq.h
+// exactly (float32 RN subtract/divide, rint to even, fp16 RN), so the packed
+// bytes are bit-identical to the definition.
 //
 // Kernels (all bandwidth-trivial next to decode; one warp per row):
-//   pack_rows      positions [lo, hi) of every (b, kv head) -> K4V4 records
+//   pack_rows      positions [lo, hi) of every (b, kv head) -> packed records
 //   ring_fill      init only: last min(W, L) prefix rows -> FP16 ring
 //   vl_gather      merge only: new VL rows -> workspace (old VL row, found through
 //                  its page's bitmap, ring row, or the dequantised record rounded
