@@ -212,3 +212,18 @@ def test_reset_then_reinstall_with_running_scores():
     p.reselect_merge()
     out, ref = p.decode(q[64], k[64], v[64])
     check_decode(out, ref, "after reset and a merge")
+
+
+def test_reselection_after_decode_steps_at_another_scale():
+    """Decode steps run at a scale other than 1/sqrt(D) store no usable
+    log-sum-exp (NaN), so the reselection computes its own row normalisers
+    (its first pass) and still matches the oracle's column mass."""
+    p = Pair(1, 8, 2, 700, 64, 500, cap=900, seed=95)
+    p.init()
+    q, k, v = synth.decode_tokens(95, 1, 8, 2, 64)
+    for t in range(64):
+        hq().hq_decode_attn(p.g, dev(q[t]), dev(k[t]), dev(v[t]), sm_scale=0.05)
+        p.r.append(q[t], k[t], v[t])
+    torch.cuda.synchronize()
+    assert torch.isnan(p.g.qlse).all()
+    p.reselect_merge()
