@@ -1,0 +1,46 @@
+"""Seeded random combinations of the cache's options, each through install,
+decode, a full 64-token period, reselection and merge, every sequence against
+its own oracle cache (bit-exact records and VL store, decode within its
+tolerances, selections against the oracle's column mass).
+
+The draws cover batch sizes 1-3 with ragged lengths (1 .. 900 tokens),
+GQA 1-8, windows that are not multiples of the 16-row tile (0 .. 128), line
+ratios from 0 to 100 %, the four code widths, and dense or shuffled paged
+stores."""
+import numpy as np
+import pytest
+
+from tests.test_gpu_varlen import Ragged, _tokens
+
+pytestmark = pytest.mark.gpu
+
+WIDTHS = [(4, 4), (8, 8), (4, 2), (2, 4)]
+
+
+def _draw(case):
+    rng = np.random.default_rng(1000 + case)
+    B = int(rng.integers(1, 4))
+    Hkv = int(rng.choice([1, 2]))
+    G = int(rng.choice([1, 2, 4, 8]))
+    W = int(rng.choice([0, 5, 16, 33, 64, 100, 128]))
+    rho = int(rng.choice([0, 100, 500, 2500, 10000]))
+    kb, vb = WIDTHS[int(rng.integers(0, 4))]
+    paged = bool(rng.integers(0, 2))
+    lengths = [int(x) for x in rng.integers(1, 901, size=B)]
+    return B, Hkv, G, W, rho, kb, vb, paged, lengths
+
+
+@pytest.mark.parametrize("case", range(48))
+def test_random_option_combinations(case):
+    B, Hkv, G, W, rho, kb, vb, paged, lengths = _draw(case)
+    Hq = G * Hkv
+    rg = Ragged(lengths, Hq, Hkv, W, rho, cap=max(lengths) + 200, seed=2000 + case, paged=paged, k_bits=kb, v_bits=vb)
+    for b in range(B):
+        rg.install(b, check=True)
+        rg.check_store(b)
+    q, k, v = _tokens(3000 + case, B, Hq, Hkv, 67)
+    for t in range(64):
+        rg.decode(q[t], k[t], v[t], check=(t % 9 == 0 or t == 63))
+    rg.reselect_merge()
+    for t in range(64, 67):
+        rg.decode(q[t], k[t], v[t])
