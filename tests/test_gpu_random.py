@@ -44,3 +44,25 @@ def test_random_option_combinations(case):
     rg.reselect_merge()
     for t in range(64, 67):
         rg.decode(q[t], k[t], v[t])
+
+
+@pytest.mark.parametrize("case", range(24))
+def test_random_prefill_shapes(case):
+    """Seeded random prefill shapes (L 1 .. 700, GQA 1-8, batch 1-2, window
+    0 .. 300, line ratio 0 .. 100 %), both Q.K formats, whole output against
+    the oracle within the prefill bound."""
+    from tests.test_gpu_prefill import PF_RELL2, _run
+    rng = np.random.default_rng(4000 + case)
+    B = int(rng.integers(1, 3))
+    Hkv = int(rng.choice([1, 2]))
+    G = int(rng.choice([1, 2, 4, 8]))
+    L = int(rng.integers(1, 701))
+    W = int(rng.choice([0, 7, 64, 128, 300]))
+    rho = int(rng.choice([0, 250, 500, 10000]))
+    fmt = "int8" if case % 2 else "e4m3"
+    got, ref = _run(B, G * Hkv, Hkv, L, W, rho, seed=5000 + case, fmt=fmt)
+    assert np.all(np.isfinite(got))
+    for (b, h), r in ref.items():
+        g = got[b, h]
+        rel = np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-30)
+        assert rel <= PF_RELL2, (case, b, h, rel, (B, G * Hkv, Hkv, L, W, rho, fmt))
