@@ -66,3 +66,29 @@ def test_random_prefill_shapes(case):
         g = got[b, h]
         rel = np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-30)
         assert rel <= PF_RELL2, (case, b, h, rel, (B, G * Hkv, Hkv, L, W, rho, fmt))
+
+
+@pytest.mark.parametrize("case", range(8))
+def test_random_large_ragged_batches(case):
+    """Seeded random batches of 10 .. 40 sequences with 4 or 8 kv heads (more
+    than 37 units: the stream-K decode grid), ragged lengths 1 .. 2000, a
+    random code width, dense or paged: installs, a period with checked steps,
+    reselection and merge, against per-sequence oracles."""
+    rng = np.random.default_rng(6000 + case)
+    B = int(rng.integers(10, 41))
+    Hkv = int(rng.choice([4, 8]))
+    G = int(rng.choice([1, 4]))
+    W = int(rng.choice([16, 64, 128]))
+    kb, vb = WIDTHS[int(rng.integers(0, 4))]
+    paged = bool(rng.integers(0, 2))
+    lengths = [int(x) for x in rng.integers(1, 2001, size=B)]
+    rg = Ragged(lengths, G * Hkv, Hkv, W, 500, cap=max(lengths) + 200, seed=7000 + case, paged=paged,
+                k_bits=kb, v_bits=vb)
+    for b in range(B):
+        rg.install(b, check=(b % 8 == 0))
+    q, k, v = _tokens(8000 + case, B, G * Hkv, Hkv, 66)
+    for t in range(64):
+        rg.decode(q[t], k[t], v[t], check=(t % 21 == 0 or t == 63))
+    rg.reselect_merge()
+    for t in range(64, 66):
+        rg.decode(q[t], k[t], v[t])
