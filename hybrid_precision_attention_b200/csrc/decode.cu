@@ -52,9 +52,11 @@
 //     done reading by then); the last CTA to take its grid ticket (taken with
 //     the unit ticket, once it has read every length it uses) advances the
 //     lengths;
-//   * launched with programmatic dependent launch: a CTA prefetches its range's
-//     pages and VL rows into L2 before it waits for the previous grid, and lets
-//     the next grid launch as soon as its own wait is over.
+//   * launched with programmatic dependent launch: a CTA makes its aligned
+//     plan before it waits for the previous grid, and lets the next grid
+//     launch as soon as its own wait is over.  (An L2 prefetch of the CTA's
+//     pages before the wait was measured and removed: it cost 1.1 us at B=1
+//     and 18 % at B=16, where the ranges exceed L2.)
 #include "common.cuh"
 
 namespace hq {
@@ -275,9 +277,8 @@ __device__ __forceinline__ void aligned_assign(const hq_cache& c, Plan& p, const
 }
 
 // Cut the batch's tile lists into ranges and record this CTA's segments.
-// `stale`: state read with volatile loads before the dependency wait (it may
-// be one step old; the plan then only steers prefetches).  `red` is scratch
-// for NTHREADS / 32 ints.
+// `stale`: state read with volatile loads (it may be one step old).  `red`
+// is scratch for NTHREADS / 32 ints.
 __device__ __noinline__ void make_plan(const hq_cache& c, int R, Plan& p, int* red, bool stale) {
   const int U = c.B * c.Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -1064,11 +1065,9 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
     s_timeout = 0;
     fence_mbar_init();
   }
-  // Before the dependency wait, plan on the (possibly stale) lengths and warm
-  // L2 with this range's pages and VL rows: a prefetch is a hint, the ranges
-  // are clamped to the buffers, so a stale plan costs bandwidth, never
-  // correctness.
-  // the plan: unit-aligned splits for few units, stream-K ranges for many
+  // the plan: unit-aligned splits for few units (made before the dependency
+  // wait on the lengths as they stand, kept after it when they did not
+  // change), stream-K ranges for many (made after the wait)
   const bool aligned = c.B * c.Hkv * 4 <= static_cast<int>(gridDim.x);
   __shared__ AlignedSnap snap;
   if (aligned) {
@@ -1076,30 +1075,6 @@ decode_kernel(const hq_cache c, const uint16_t* __restrict__ q, const uint16_t* 
     __syncthreads();
     if (threadIdx.x == 0) aligned_assign(c, plan, snap);
     __syncthreads();
-  } else {
-    make_plan(c, R, plan, red, true);
-  }
-  if (warp == NC) {
-    for (int si = 0; si < plan.nseg; ++si) {
-      const Seg s = plan.seg[si];
-      constexpr int PR = HQ_PAGE_SUBPOS(KB, VB);
-      constexpr int PB = HQ_PAGE_BYTES_KV(KB, VB);
-      const int p0 = (s.p0 * PR) / 64, p1 = min(((s.p0 + s.npk) * PR + 63) / 64, c.cap / 64);
-      for (int pg = p0 + lane; pg < p1; pg += 32) {  // one page per lane
-        const long long idx = page_index(c, s.u, pg);
-        if (idx >= 0) prefetch_l2(c.pages + static_cast<size_t>(idx) * PB, HQ_PAGE_MASK_OFF(KB, VB) + 16);
-      }
-      int T, np, nv;
-      read_len(c, s.u / c.Hkv, true, T, np, nv);
-      const int NV = (nv + FT - 1) / FT;
-      const int nf = (s.b - s.a) - s.npk;
-      const int v0 = min(s.f0, NV), v1 = min(s.f0 + nf, min(NV, c.vl_cap / FT));
-      if (lane == 0 && v1 > v0) {
-        const size_t off = (static_cast<size_t>(s.u) * c.vl_cap + v0 * FT) * D;
-        prefetch_l2(c.kf + off, (v1 - v0) * FT * D * 2);
-        prefetch_l2(c.vf + off, (v1 - v0) * FT * D * 2);
-      }
-    }
   }
   // programmatic dependent launch: everything this kernel reads (the state, the
   // cache, the previous step's appended token) was written by earlier kernels,
