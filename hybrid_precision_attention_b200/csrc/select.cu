@@ -243,32 +243,6 @@ __device__ __forceinline__ void store_key_row(const SelArgs& a, int bh, const Ke
   for (int ch = 0; ch < 16; ++ch) *reinterpret_cast<uint4*>(stage + sw128_off(r, ch, KT * 128)) = make_uint4(0u, 0u, 0u, 0u);
 }
 
-// L2 prefetch of the key bytes of tiles [k_lo, k_hi) (a hint, clamped to the buffers)
-__device__ __forceinline__ void prefetch_keys(const SelArgs& a, const SelGeo& g, int bh, int k_lo, int k_hi) {
-  const hq_cache& c = a.c;
-  const int j0 = k_lo * KT, j1 = min(k_hi * KT, g.T);
-  if (j1 <= j0) return;
-  if (a.k_dense) {
-    const uint8_t* p = reinterpret_cast<const uint8_t*>(a.k_dense + (static_cast<size_t>(bh) * a.L + j0) * D);
-    for (int off = 0; off < (j1 - j0) * D * 2; off += 65536) prefetch_l2(p + off, min(65536, (j1 - j0) * D * 2 - off));
-    return;
-  }
-  const int p0 = j0 / HQ_PAGE_POSITIONS, p1 = min((j1 + HQ_PAGE_POSITIONS - 1) / HQ_PAGE_POSITIONS,
-                                                  (g.n_packed + HQ_PAGE_POSITIONS - 1) / HQ_PAGE_POSITIONS);
-  for (int pg = p0; pg < p1; pg += 8)  // K codes, K (scale, zero) words and the bitmap of 8 pages at a time
-    for (int q = pg; q < min(pg + 8, p1); ++q) {
-      const long long idx = page_index(c, bh, q);   // a hint: entries outside the pool are skipped
-      if (idx < 0) continue;
-      const PageGeo pgm = page_geo(c);
-      uint8_t* page = c.pages + static_cast<size_t>(idx) * pgm.bytes;
-      for (int sp = 0; sp < 64; sp += pgm.pr) {  // K codes and K (scale, zero) words of each sub-page
-        prefetch_l2(row_codes(pgm, page, 0, sp), pgm.pr * 16 * pgm.kb);
-        prefetch_l2(row_sz(pgm, page, 0, sp), pgm.pr * 16);
-      }
-      prefetch_l2(page_mask(pgm, page), 16);
-    }
-}
-
 template <bool COL>
 __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -340,7 +314,6 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) sel_pass(SelArgs a) {
     abort_flag = 0;
     fence_mbar_init();
   }
-  if (threadIdx.x == EPI_WARPS * 32 && M > 0) prefetch_keys(a, g, bh, k_lo, k_hi);
   if (warp == MMA_WARP) {
     tmem_alloc(&tmem_base_sh, TMEM_COLS);
     tmem_relinquish();
