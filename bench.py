@@ -401,9 +401,9 @@ def run_ours(args, rank, world, local_rank):
     # capture does not run the work; the caches are still at T = L + 64, just merged
 
     # our kernels per step: one decode_kernel per token and copy; per copy a
-    # reselection (sel_pass<0>, sel_pass<1>, topk_kernel) and a staging merge
-    # (pack_rows_kernel, vl_gather_kernel, vl_clear_kernel, vl_install_kernel)
-    launches_per_step = PERIOD * COPIES + COPIES * (3 + 4)
+    # reselection (sel_pass<0>, sel_pass<1>, the top-k) and a staging merge
+    # (merge_gather_kernel, vl_install_kernel)
+    launches_per_step = PERIOD * COPIES + COPIES * (3 + 2)
 
     def step(ev=None):
         if ev is not None:

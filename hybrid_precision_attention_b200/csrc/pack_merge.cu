@@ -9,14 +9,17 @@
 // bytes are bit-identical to the definition.
 //
 // Kernels (all bandwidth-trivial next to decode; one warp per row):
-//   pack_rows      positions [lo, hi) of every (b, kv head) -> packed records
+//   pack_rows      init only: prefix positions [0, L - W) of every (b, kv head)
+//                  -> packed records
 //   ring_fill      init only: last min(W, L) prefix rows -> FP16 ring
-//   vl_gather      merge only: new VL rows -> workspace (old VL row, found through
-//                  its page's bitmap, ring row, or the dequantised record rounded
-//                  once to fp16)
-//   vl_clear       merge only: bitmap words of the pages holding the old lines -> 0
-//   vl_install     rows -> VL store, positions, bitmap bits, per-page first VL row,
-//                  state update
+//   merge_gather   merge only, one launch for three kinds of item: the rows
+//                  leaving the window -> packed records; new VL rows ->
+//                  workspace (old VL row, found through its page's bitmap, ring
+//                  row, or the dequantised record rounded once to fp16); the
+//                  bitmap words of the pages that keep no line -> 0
+//   vl_install     rows -> VL store, positions, each page's bitmap word and
+//                  first VL row (written whole by the page's first line), state
+//                  update
 #include "common.cuh"
 
 namespace hq {
@@ -67,41 +70,46 @@ __device__ __forceinline__ void pack_row_warp(const uint16_t* __restrict__ src, 
   }
 }
 
-// Rows [lo, hi) of every (b, kv head), K and V.  Init: src = dense [B,Hkv,L,D],
-// lo = 0, hi = max(L - W, 0) for every sequence.  Merge: src = ring, and per
-// sequence lo = n_packed, hi = T - W (from its state row; at most R rows, the
-// ring's length, since the ring holds every position in [n_packed, T)).
-__global__ void pack_rows_kernel(hq_cache c, const uint16_t* __restrict__ kd, const uint16_t* __restrict__ vd, int L,
-                                 int init) {
+// Pack item w of 2 B Hkv nmax (K or V) x (b, h) x rows.  Init: src = dense
+// [B,Hkv,L,D], rows [0, max(L - W, 0)) of every sequence.  Merge: src = ring,
+// and per sequence rows [n_packed, T - W) (from its state row; at most R rows,
+// the ring's length, since the ring holds every position in [n_packed, T)).
+__device__ __forceinline__ void pack_item(const hq_cache& c, const Dims& d, const uint16_t* __restrict__ kd,
+                                          const uint16_t* __restrict__ vd, int L, int init, int nmax, long long w,
+                                          int lane) {
+  const int which = static_cast<int>(w & 1);
+  const long long rest = w >> 1;
+  const int r = static_cast<int>(rest % nmax);
+  const long long bh = rest / nmax;
+  int p;
+  const uint16_t* src;
+  if (init) {
+    p = r;
+    src = (which ? vd : kd) + (bh * L + p) * D;
+  } else {
+    const int32_t* st = state_row(c, static_cast<int>(bh / d.Hkv));
+    const int lo = st[HQ_STATE_NPACKED];
+    const int hi = max(lo, st[HQ_STATE_T] - d.W);
+    p = lo + r;
+    if (p >= hi) return;
+    src = (which ? c.vr : c.kr) + (bh * d.R + (p % d.R)) * D;
+  }
+  uint8_t* page = page_for_write(c, bh, p);
+  if (page == nullptr) return;
+  const PageGeo pg = page_geo(c);
+  pack_row_warp(src, row_codes(pg, page, which, p), row_sz(pg, page, which, p), lane, which ? pg.vb : pg.kb);
+}
+
+// Init: the prefix rows [0, L - W) of every (b, kv head), K and V.
+__global__ void pack_rows_kernel(hq_cache c, const uint16_t* __restrict__ kd, const uint16_t* __restrict__ vd, int L) {
   const Dims d = dims_of(c);
-  const int nmax = init ? max(L - d.W, 0) : d.R;
+  const int nmax = max(L - d.W, 0);
   if (nmax <= 0) return;
   const int lane = threadIdx.x & 31;
   const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
-  const long long total = 2ll * d.B * d.Hkv * nmax;  // (K or V) x (b, h) x rows
-  for (long long w = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); w < total; w += warps) {
-    const int which = static_cast<int>(w & 1);
-    const long long rest = w >> 1;
-    const int r = static_cast<int>(rest % nmax);
-    const long long bh = rest / nmax;
-    int p;
-    const uint16_t* src;
-    if (init) {
-      p = r;
-      src = (which ? vd : kd) + (bh * L + p) * D;
-    } else {
-      const int32_t* st = state_row(c, static_cast<int>(bh / d.Hkv));
-      const int lo = st[HQ_STATE_NPACKED];
-      const int hi = max(lo, st[HQ_STATE_T] - d.W);
-      p = lo + r;
-      if (p >= hi) continue;
-      src = (which ? c.vr : c.kr) + (bh * d.R + (p % d.R)) * D;
-    }
-    uint8_t* page = page_for_write(c, bh, p);
-    if (page == nullptr) continue;
-    const PageGeo pg = page_geo(c);
-    pack_row_warp(src, row_codes(pg, page, which, p), row_sz(pg, page, which, p), lane, which ? pg.vb : pg.kb);
-  }
+  const long long total = 2ll * d.B * d.Hkv * nmax;
+  for (long long w = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); w < total; w += warps)
+    pack_item(c, d, kd, vd, L, 1, nmax, w, lane);
 }
 
 // Init: prefix rows [max(L-W,0), L) -> ring slots p % R.
@@ -140,17 +148,64 @@ __device__ __forceinline__ int old_vl_row(const hq_cache& c, size_t bh, int p) {
   return *page_vlbase(pg, page) + below;
 }
 
-// Merge: gather the FP16 rows of the new VL set into the workspace.  One warp
-// per (b, h, row) handles K and V; an old line is found through its page's
-// bitmap (read only here: the bits change in the next two kernels).
-__global__ void vl_gather_kernel(hq_cache c, uint16_t* __restrict__ wsk, uint16_t* __restrict__ wsv) {
+// Does the new VL set hold a line of page pg (positions 64 pg .. 64 pg + 63)
+// that the merge installs (below limit)?  The set is in ascending position
+// order: a binary search for its first position at or above 64 pg.
+__device__ __forceinline__ bool new_line_in_page(const int32_t* __restrict__ sel, int k, int pg, int limit) {
+  int lo = 0, hi = k;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (sel[mid] < pg * HQ_PAGE_POSITIONS) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo < k && sel[lo] < min((pg + 1) * HQ_PAGE_POSITIONS, limit);
+}
+
+// Merge, first launch.  One index space of warp items, in three kinds:
+//   [0, n_pack)                  pack one row leaving the window (K or V);
+//   [n_pack, + B Hkv vl_cap)     gather one row of the new VL set into the
+//                                workspace, K and V; an old line is found
+//                                through its page's bitmap;
+//   [.., + B Hkv ceil(vl_cap/32)) 32 rows of the old VL set: the bitmap words of
+//                                the pages where the new set keeps no line -> 0
+//                                (the install writes the others whole).
+// No item reads what another writes: packing writes the records of positions
+// at or above n_packed, which no gather reads; a gather reads the bitmap of a
+// page that holds a new line, and only pages without one are zeroed.
+__global__ void merge_gather_kernel(hq_cache c, uint16_t* __restrict__ wsk, uint16_t* __restrict__ wsv) {
   const Dims d = dims_of(c);
   const int lane = threadIdx.x & 31;
+  const long long nbh = static_cast<long long>(d.B) * d.Hkv;
+  const long long n_pack = 2ll * nbh * d.R;
+  const long long n_gather = nbh * d.vl_cap;
+  const int cw = (d.vl_cap + 31) / 32;
+  const long long total = n_pack + n_gather + nbh * cw;
   const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
-  const long long total = static_cast<long long>(d.B) * d.Hkv * d.vl_cap;
   for (long long w = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); w < total; w += warps) {
-    const int r = static_cast<int>(w % d.vl_cap);
-    const long long bh = w / d.vl_cap;
+    if (w < n_pack) {
+      pack_item(c, d, nullptr, nullptr, 0, 0, d.R, w, lane);
+      continue;
+    }
+    if (w >= n_pack + n_gather) {
+      const long long i = w - n_pack - n_gather;
+      const long long bh = i / cw;
+      const int r = static_cast<int>(i % cw) * 32 + lane;
+      const int32_t* st = state_row(c, static_cast<int>(bh / d.Hkv));
+      if (r >= st[HQ_STATE_NVL]) continue;
+      const int32_t* pos = c.vl_pos + bh * d.vl_cap;
+      const int p = pos[r];
+      // the old set is in ascending position order too: one lane per page
+      if (p < 0 || (r > 0 && (pos[r - 1] >> 6) == (p >> 6))) continue;
+      const int k = min(st[HQ_STATE_KSEL], d.vl_cap);
+      const int limit = max(st[HQ_STATE_NPACKED], st[HQ_STATE_T] - d.W);
+      if (new_line_in_page(c.vl_sel + bh * d.vl_cap, k, p >> 6, limit)) continue;
+      uint8_t* page = page_for_write(c, bh, p);
+      if (page) *reinterpret_cast<uint2*>(page_mask(page_geo(c), page)) = make_uint2(0u, 0u);
+      continue;
+    }
+    const long long g = w - n_pack;
+    const int r = static_cast<int>(g % d.vl_cap);
+    const long long bh = g / d.vl_cap;
     int32_t* st = state_row(c, static_cast<int>(bh / d.Hkv));
     const int k = min(st[HQ_STATE_KSEL], d.vl_cap);
     if (r >= k) continue;
@@ -198,25 +253,11 @@ __global__ void vl_gather_kernel(hq_cache c, uint16_t* __restrict__ wsk, uint16_
   }
 }
 
-// Merge: clear the bitmap words of every page that holds a current (old)
-// vertical line (plain stores of zero; the new set's bits are set afterwards).
-__global__ void vl_clear_kernel(hq_cache c) {
-  const Dims d = dims_of(c);
-  const long long total = static_cast<long long>(d.B) * d.Hkv * d.vl_cap;
-  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long bh = i / d.vl_cap;
-    const int r = static_cast<int>(i % d.vl_cap);
-    if (r >= state_row(c, static_cast<int>(bh / d.Hkv))[HQ_STATE_NVL]) continue;
-    uint8_t* page = page_for_write(c, bh, c.vl_pos[bh * d.vl_cap + r]);
-    if (page) *reinterpret_cast<uint2*>(page_mask(page_geo(c), page)) = make_uint2(0u, 0u);
-  }
-}
-
 // Install rows into the VL store.  Init: rows from the dense prefix; merge: rows
-// from the workspace.  One warp per (b, h, row): K and V rows, vl_pos, the
-// bitmap bit and (first line of a page) the page's first VL-store row.  The
-// last block to finish (ticket) updates the state rows.
+// from the workspace.  One warp per (b, h, row): K and V rows and vl_pos; the
+// first line of a page writes the page's bitmap word whole (every line of the
+// set in that page: they follow it in position order) and its first VL-store
+// row.  The last block to finish (ticket) updates the state rows.
 __global__ void vl_install_kernel(hq_cache c, const uint16_t* __restrict__ srck, const uint16_t* __restrict__ srcv, int L,
                                   int init, unsigned int* __restrict__ ticket) {
   const Dims d = dims_of(c);
@@ -244,13 +285,24 @@ __global__ void vl_install_kernel(hq_cache c, const uint16_t* __restrict__ srck,
     }
     if (lane == 0) {
       c.vl_pos[bh * d.vl_cap + row] = p;
-      uint8_t* page = page_for_write(c, bh, p);
-      if (page) {
-        const PageGeo pg = page_geo(c);
-        atomicOr(page_mask(pg, page) + ((p & 63) >> 5), 1u << (p & 31));
-        // the first vertical line of a page records its VL-store row (rows are in
-        // ascending position order), so readers find a line's row by a popcount
-        if (row == 0 || (c.vl_sel[bh * d.vl_cap + row - 1] >> 6) != (p >> 6)) *page_vlbase(pg, page) = row;
+      const int32_t* sel = c.vl_sel + bh * d.vl_cap;
+      if (row == 0 || (sel[row - 1] >> 6) != (p >> 6)) {
+        // the first vertical line of its page: the page's bitmap word, and its
+        // VL-store row (rows are in ascending position order), so readers find
+        // a line's row by a popcount
+        uint8_t* page = page_for_write(c, bh, p);
+        if (page) {
+          uint32_t m0 = 0u, m1 = 0u;
+          for (int j = row; j < k; ++j) {
+            const int pj = sel[j];
+            if ((pj >> 6) != (p >> 6) || pj >= limit) break;
+            if (pj & 32) m1 |= 1u << (pj & 31);
+            else m0 |= 1u << (pj & 31);
+          }
+          const PageGeo pg = page_geo(c);
+          *reinterpret_cast<uint2*>(page_mask(pg, page)) = make_uint2(m0, m1);
+          *page_vlbase(pg, page) = row;
+        }
       }
     }
   }
@@ -308,15 +360,21 @@ hq_status launch_pack_merge(const hq_cache& c, const uint16_t* kd, const uint16_
   unsigned int* ticket = reinterpret_cast<unsigned int*>(ws);
   uint16_t* wsk = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + 256);
   uint16_t* wsv = wsk + static_cast<size_t>(c.B) * c.Hkv * c.vl_cap * D;
-  if (init) clear_bitmaps_kernel<<<sms, threads, 0, st>>>(c);
-  pack_rows_kernel<<<sms * 4, threads, 0, st>>>(c, kd, vd, L, init);
+  // warp items -> blocks of 8 warps, at most 8 blocks per SM (one wave)
+  const auto blocks = [&](long long items) {
+    return static_cast<int>(max(1ll, min((items + 7) / 8, 8ll * sms)));
+  };
+  const long long nbh = static_cast<long long>(c.B) * c.Hkv;
+  const long long install_items = nbh * c.vl_cap;
   if (init) {
+    clear_bitmaps_kernel<<<sms, threads, 0, st>>>(c);
+    pack_rows_kernel<<<sms * 4, threads, 0, st>>>(c, kd, vd, L);
     ring_fill_kernel<<<sms, threads, 0, st>>>(c, kd, vd, L);
-    vl_install_kernel<<<sms * 4, threads, 0, st>>>(c, kd, vd, L, 1, ticket);
+    vl_install_kernel<<<blocks(install_items), threads, 0, st>>>(c, kd, vd, L, 1, ticket);
   } else {
-    vl_gather_kernel<<<sms * 4, threads, 0, st>>>(c, wsk, wsv);
-    vl_clear_kernel<<<sms, threads, 0, st>>>(c);
-    vl_install_kernel<<<sms * 4, threads, 0, st>>>(c, wsk, wsv, L, 0, ticket);
+    const long long gather_items = 2 * nbh * ring_len(c.W) + nbh * c.vl_cap + nbh * ((c.vl_cap + 31) / 32);
+    merge_gather_kernel<<<blocks(gather_items), threads, 0, st>>>(c, wsk, wsv);
+    vl_install_kernel<<<blocks(install_items), threads, 0, st>>>(c, wsk, wsv, L, 0, ticket);
   }
   return cuda_status(cudaGetLastError(), "merge launch");
 }
