@@ -148,6 +148,44 @@ __device__ __forceinline__ int old_vl_row(const hq_cache& c, size_t bh, int p) {
   return *page_vlbase(pg, page) + below;
 }
 
+// Values 16 s .. 16 s + 15 of a packed row (codes: the row's 16 * BITS code
+// bytes, value j at bit BITS * j; szw: the (scale, zero) word of their group)
+// as fp16(zero + q * scale): q * scale is exact in float64 and the sum is
+// rounded once, then once more to fp16 (RN).
+template <int BITS>
+__device__ __forceinline__ void dequant16(const uint8_t* __restrict__ codes, uint32_t szw, int s, uint4& o0, uint4& o1) {
+  constexpr int NW = BITS / 2;  // 32-bit code words holding 16 values
+  uint32_t cw[NW];
+  if constexpr (BITS == 8) {
+    const uint4 t = *reinterpret_cast<const uint4*>(codes + 16 * s);
+    cw[0] = t.x;
+    cw[1] = t.y;
+    cw[2] = t.z;
+    cw[3] = t.w;
+  } else if constexpr (BITS == 4) {
+    const uint2 t = *reinterpret_cast<const uint2*>(codes + 8 * s);
+    cw[0] = t.x;
+    cw[1] = t.y;
+  } else {
+    cw[0] = *reinterpret_cast<const uint32_t*>(codes + 4 * s);
+  }
+  const double sc = static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(szw & 0xFFFFu))));
+  const double ze = static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(szw >> 16))));
+  constexpr uint32_t mask = (1u << BITS) - 1u;
+  uint32_t h[8];
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) {
+    const uint32_t q0 = (cw[(BITS * i) >> 5] >> ((BITS * i) & 31)) & mask;
+    const uint32_t q1 = (cw[(BITS * (i + 1)) >> 5] >> ((BITS * (i + 1)) & 31)) & mask;
+    const double v0 = __dadd_rn(ze, __dmul_rn(static_cast<double>(q0), sc));
+    const double v1 = __dadd_rn(ze, __dmul_rn(static_cast<double>(q1), sc));
+    h[i / 2] = static_cast<uint32_t>(__half_as_ushort(__double2half(v0))) |
+               (static_cast<uint32_t>(__half_as_ushort(__double2half(v1))) << 16);
+  }
+  o0 = make_uint4(h[0], h[1], h[2], h[3]);
+  o1 = make_uint4(h[4], h[5], h[6], h[7]);
+}
+
 // Does the new VL set hold a line of page pg (positions 64 pg .. 64 pg + 63)
 // that the merge installs (below limit)?  The set is in ascending position
 // order: a binary search for its first position at or above 64 pg.
@@ -162,13 +200,13 @@ __device__ __forceinline__ bool new_line_in_page(const int32_t* __restrict__ sel
 }
 
 // Merge, first launch.  One index space of warp items, in three kinds:
-//   [0, n_pack)                  pack one row leaving the window (K or V);
-//   [n_pack, + B Hkv vl_cap)     gather one row of the new VL set into the
-//                                workspace, K and V; an old line is found
-//                                through its page's bitmap;
-//   [.., + B Hkv ceil(vl_cap/32)) 32 rows of the old VL set: the bitmap words of
-//                                the pages where the new set keeps no line -> 0
-//                                (the install writes the others whole).
+//   [0, n_pack)                   pack one row leaving the window (K or V);
+//   [n_pack, + B Hkv ceil(vl_cap/4)) gather 4 rows of the new VL set into the
+//                                 workspace, 8 lanes per row, K and V; an old
+//                                 line is found through its page's bitmap;
+//   [.., + B Hkv ceil(vl_cap/32)) 32 rows of the old VL set: the bitmap words
+//                                 of the pages where the new set keeps no line
+//                                 -> 0 (the install writes the others whole).
 // No item reads what another writes: packing writes the records of positions
 // at or above n_packed, which no gather reads; a gather reads the bitmap of a
 // page that holds a new line, and only pages without one are zeroed.
@@ -177,7 +215,8 @@ __global__ void merge_gather_kernel(hq_cache c, uint16_t* __restrict__ wsk, uint
   const int lane = threadIdx.x & 31;
   const long long nbh = static_cast<long long>(d.B) * d.Hkv;
   const long long n_pack = 2ll * nbh * d.R;
-  const long long n_gather = nbh * d.vl_cap;
+  const int rq = (d.vl_cap + 3) / 4;
+  const long long n_gather = nbh * rq;
   const int cw = (d.vl_cap + 31) / 32;
   const long long total = n_pack + n_gather + nbh * cw;
   const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
@@ -204,106 +243,117 @@ __global__ void merge_gather_kernel(hq_cache c, uint16_t* __restrict__ wsk, uint
       continue;
     }
     const long long g = w - n_pack;
-    const int r = static_cast<int>(g % d.vl_cap);
-    const long long bh = g / d.vl_cap;
+    const int sub = lane & 7;  // 16 of the row's 128 values: 2 x 16 bytes of fp16
+    const int r = static_cast<int>(g % rq) * 4 + (lane >> 3);
+    const long long bh = g / rq;
     int32_t* st = state_row(c, static_cast<int>(bh / d.Hkv));
     const int k = min(st[HQ_STATE_KSEL], d.vl_cap);
     if (r >= k) continue;
     const int n_packed = st[HQ_STATE_NPACKED];
     const int p = c.vl_sel[bh * d.vl_cap + r];
     if (p < 0 || p >= max(n_packed, st[HQ_STATE_T] - d.W)) {  // not a position the merge can hold
-      if (lane == 0) set_err(st, HQ_DEVERR_VL_CAPACITY);
+      if (sub == 0) set_err(st, HQ_DEVERR_VL_CAPACITY);
       continue;
     }
     const int old = p < n_packed ? old_vl_row(c, bh, p) : -1;
 #pragma unroll
     for (int which = 0; which < 2; ++which) {
-      uint16_t* dst = (which ? wsv : wsk) + (bh * d.vl_cap + r) * D;
-      if (old >= 0) {
-        const uint16_t* s = (which ? c.vf : c.kf) + (bh * d.vl_cap + old) * D;
-        reinterpret_cast<uint2*>(dst)[lane] = reinterpret_cast<const uint2*>(s)[lane];
-      } else if (p >= n_packed) {
-        const uint16_t* s = (which ? c.vr : c.kr) + (bh * d.R + (p % d.R)) * D;
-        reinterpret_cast<uint2*>(dst)[lane] = reinterpret_cast<const uint2*>(s)[lane];
+      uint4* dst = reinterpret_cast<uint4*>((which ? wsv : wsk) + (bh * d.vl_cap + r) * D) + 2 * sub;
+      if (old >= 0 || p >= n_packed) {
+        const uint16_t* src = old >= 0 ? (which ? c.vf : c.kf) + (bh * d.vl_cap + old) * D
+                                       : (which ? c.vr : c.kr) + (bh * d.R + (p % d.R)) * D;
+        const uint4* s4 = reinterpret_cast<const uint4*>(src) + 2 * sub;
+        const uint4 x0 = s4[0], x1 = s4[1];
+        dst[0] = x0;
+        dst[1] = x1;
       } else {
-        // promoted packed position: fp16(zero + q * scale); q * scale is exact in
-        // float64 and the sum is rounded once, then once more to fp16 (RN).
-        // Lane l dequantises values 4l .. 4l+3 (4 * bits code bits).
+        // promoted packed position: the record dequantised once
         const PageGeo pg = page_geo(c);
         uint8_t* page = page_of(c, bh, p);
         const int bits = which ? pg.vb : pg.kb;
         const uint8_t* codes = row_codes(pg, page, which, p);
-        const uint32_t szw = row_sz(pg, page, which, p)[lane >> 3];
-        const double sc = static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(szw & 0xFFFFu))));
-        const double ze = static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(szw >> 16))));
-        const uint32_t qw = bits == 4 ? reinterpret_cast<const uint16_t*>(codes)[lane]
-                                      : (bits == 8 ? reinterpret_cast<const uint32_t*>(codes)[lane] : codes[lane]);
-        const uint32_t mask = (1u << bits) - 1u;
-        uint32_t out[2];
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const double v0 = __dadd_rn(ze, __dmul_rn(static_cast<double>((qw >> (bits * 2 * i)) & mask), sc));
-          const double v1 = __dadd_rn(ze, __dmul_rn(static_cast<double>((qw >> (bits * (2 * i + 1))) & mask), sc));
-          out[i] = static_cast<uint32_t>(__half_as_ushort(__double2half(v0))) |
-                   (static_cast<uint32_t>(__half_as_ushort(__double2half(v1))) << 16);
-        }
-        reinterpret_cast<uint2*>(dst)[lane] = make_uint2(out[0], out[1]);
+        const uint32_t szw = row_sz(pg, page, which, p)[sub >> 1];
+        uint4 o0, o1;
+        if (bits == 4) dequant16<4>(codes, szw, sub, o0, o1);
+        else if (bits == 8) dequant16<8>(codes, szw, sub, o0, o1);
+        else dequant16<2>(codes, szw, sub, o0, o1);
+        dst[0] = o0;
+        dst[1] = o1;
       }
     }
   }
 }
 
 // Install rows into the VL store.  Init: rows from the dense prefix; merge: rows
-// from the workspace.  One warp per (b, h, row): K and V rows and vl_pos; the
-// first line of a page writes the page's bitmap word whole (every line of the
-// set in that page: they follow it in position order) and its first VL-store
-// row.  The last block to finish (ticket) updates the state rows.
+// from the workspace.  One warp per 4 rows of a (b, h), 8 lanes per row: K and
+// V rows and vl_pos; the first line of a page writes the page's bitmap word
+// whole (every line of the set in that page: they follow it in position order)
+// and its first VL-store row.  The last block to finish (ticket) updates the
+// state rows.
 __global__ void vl_install_kernel(hq_cache c, const uint16_t* __restrict__ srck, const uint16_t* __restrict__ srcv, int L,
                                   int init, unsigned int* __restrict__ ticket) {
   const Dims d = dims_of(c);
   const int lane = threadIdx.x & 31;
+  const int sub = lane & 7;                            // 16 of the row's 128 values
+  const unsigned int gmask = 0xFFu << (lane & ~7);     // the row's 8 lanes
+  const int rq = (d.vl_cap + 3) / 4;
   const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
-  const long long total = static_cast<long long>(d.B) * d.Hkv * d.vl_cap;
+  const long long total = static_cast<long long>(d.B) * d.Hkv * rq;
   for (long long w = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); w < total; w += warps) {
-    const int row = static_cast<int>(w % d.vl_cap);
-    const long long bh = w / d.vl_cap;
+    const int row = static_cast<int>(w % rq) * 4 + (lane >> 3);
+    const long long bh = w / rq;
     int32_t* st = state_row(c, static_cast<int>(bh / d.Hkv));
     const int k = min(st[HQ_STATE_KSEL], d.vl_cap);
-    if (row >= k) continue;
-    const int p = c.vl_sel[bh * d.vl_cap + row];
+    if (row >= k) continue;  // the same for the row's 8 lanes, as is every branch below
+    const int32_t* sel = c.vl_sel + bh * d.vl_cap;
+    const int p = sel[row];
     const int limit = init ? max(L - d.W, 0) : max(st[HQ_STATE_NPACKED], st[HQ_STATE_T] - d.W);
     if (p < 0 || p >= limit) {
-      if (lane == 0) set_err(st, HQ_DEVERR_VL_CAPACITY);
+      if (sub == 0) set_err(st, HQ_DEVERR_VL_CAPACITY);
       continue;
     }
 #pragma unroll
     for (int which = 0; which < 2; ++which) {
-      const uint16_t* s = init ? ((which ? srcv : srck) + (bh * L + p) * D)
-                               : ((which ? srcv : srck) + (bh * d.vl_cap + row) * D);
-      uint16_t* t = (which ? c.vf : c.kf) + (bh * d.vl_cap + row) * D;
-      reinterpret_cast<uint2*>(t)[lane] = reinterpret_cast<const uint2*>(s)[lane];
+      const uint16_t* src = init ? ((which ? srcv : srck) + (bh * L + p) * D)
+                                 : ((which ? srcv : srck) + (bh * d.vl_cap + row) * D);
+      const uint4* s4 = reinterpret_cast<const uint4*>(src) + 2 * sub;
+      uint4* t4 = reinterpret_cast<uint4*>((which ? c.vf : c.kf) + (bh * d.vl_cap + row) * D) + 2 * sub;
+      const uint4 x0 = s4[0], x1 = s4[1];
+      t4[0] = x0;
+      t4[1] = x1;
     }
-    if (lane == 0) {
-      c.vl_pos[bh * d.vl_cap + row] = p;
-      const int32_t* sel = c.vl_sel + bh * d.vl_cap;
-      if (row == 0 || (sel[row - 1] >> 6) != (p >> 6)) {
-        // the first vertical line of its page: the page's bitmap word, and its
-        // VL-store row (rows are in ascending position order), so readers find
-        // a line's row by a popcount
-        uint8_t* page = page_for_write(c, bh, p);
-        if (page) {
-          uint32_t m0 = 0u, m1 = 0u;
-          for (int j = row; j < k; ++j) {
-            const int pj = sel[j];
-            if ((pj >> 6) != (p >> 6) || pj >= limit) break;
-            if (pj & 32) m1 |= 1u << (pj & 31);
-            else m0 |= 1u << (pj & 31);
-          }
-          const PageGeo pg = page_geo(c);
-          *reinterpret_cast<uint2*>(page_mask(pg, page)) = make_uint2(m0, m1);
-          *page_vlbase(pg, page) = row;
-        }
+    if (sub == 0) c.vl_pos[bh * d.vl_cap + row] = p;
+    if (row > 0 && (sel[row - 1] >> 6) == (p >> 6)) continue;
+    // the first vertical line of its page: the page's bitmap word, and its
+    // VL-store row (rows are in ascending position order), so readers find a
+    // line's row by a popcount.  The page's lines are the rows from here on
+    // while they stay in the page: 8 of them per round, one per lane.
+    const long long idx = page_index(c, bh, p >> 6);
+    if (idx < 0) {
+      if (sub == 0) set_err(st, HQ_DEVERR_PAGE);
+      continue;
+    }
+    uint32_t m0 = 0u, m1 = 0u;
+    for (int j0 = row; j0 < k; j0 += 8) {
+      const int j = j0 + sub;
+      const int pj = j < k ? sel[j] : -1;
+      const bool in = j < k && (pj >> 6) == (p >> 6) && pj < limit;
+      if (in) {
+        if (pj & 32) m1 |= 1u << (pj & 31);
+        else m0 |= 1u << (pj & 31);
       }
+      if (((__ballot_sync(gmask, in) >> (lane & ~7)) & 0xFFu) != 0xFFu) break;
+    }
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+      m0 |= __shfl_xor_sync(gmask, m0, o);
+      m1 |= __shfl_xor_sync(gmask, m1, o);
+    }
+    if (sub == 0) {
+      const PageGeo pg = page_geo(c);
+      uint8_t* page = c.pages + static_cast<size_t>(idx) * pg.bytes;
+      *reinterpret_cast<uint2*>(page_mask(pg, page)) = make_uint2(m0, m1);
+      *page_vlbase(pg, page) = row;
     }
   }
   // state update by the last block (every block has read the state rows above)
@@ -365,14 +415,14 @@ hq_status launch_pack_merge(const hq_cache& c, const uint16_t* kd, const uint16_
     return static_cast<int>(max(1ll, min((items + 7) / 8, 8ll * sms)));
   };
   const long long nbh = static_cast<long long>(c.B) * c.Hkv;
-  const long long install_items = nbh * c.vl_cap;
+  const long long install_items = nbh * ((c.vl_cap + 3) / 4);
   if (init) {
     clear_bitmaps_kernel<<<sms, threads, 0, st>>>(c);
     pack_rows_kernel<<<sms * 4, threads, 0, st>>>(c, kd, vd, L);
     ring_fill_kernel<<<sms, threads, 0, st>>>(c, kd, vd, L);
     vl_install_kernel<<<blocks(install_items), threads, 0, st>>>(c, kd, vd, L, 1, ticket);
   } else {
-    const long long gather_items = 2 * nbh * ring_len(c.W) + nbh * c.vl_cap + nbh * ((c.vl_cap + 31) / 32);
+    const long long gather_items = 2 * nbh * ring_len(c.W) + nbh * ((c.vl_cap + 3) / 4) + nbh * ((c.vl_cap + 31) / 32);
     merge_gather_kernel<<<blocks(gather_items), threads, 0, st>>>(c, wsk, wsv);
     vl_install_kernel<<<blocks(install_items), threads, 0, st>>>(c, wsk, wsv, L, 0, ticket);
   }
