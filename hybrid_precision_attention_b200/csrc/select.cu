@@ -821,7 +821,7 @@ __global__ void __cluster_dims__(TKC_CS, 1, 1) __launch_bounds__(TKC_THREADS) to
   if (rank == 0 && bh % c.Hkv == 0 && threadIdx.x == 0) srow[HQ_STATE_KSEL] = k;
   if (k == 0) return;  // the same for every CTA of the cluster: no shared-memory exchange follows
   extern __shared__ uint32_t tkc_smem[];  // [P] scores of the range, then [P] values of the threshold bin
-  __shared__ unsigned int h10[1024];       // local histogram of the current radix pass
+  __shared__ unsigned int h10[2][1024];    // local histograms of the two radix passes
   __shared__ unsigned int wsum[TKC_THREADS / 32], rg[TKC_THREADS / 32], re[TKC_THREADS / 32];
   __shared__ unsigned int s_bin, s_above, s_cnt, s_tot[2];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -834,6 +834,7 @@ __global__ void __cluster_dims__(TKC_CS, 1, 1) __launch_bounds__(TKC_THREADS) to
   for (int j = threadIdx.x; j < m; j += TKC_THREADS) sc[j] = __ldcg(gsc + lo + j);
   const uint32_t* hh = a.hist + static_cast<size_t>(bh) * HBINS;
   int32_t* out = c.vl_sel + static_cast<size_t>(bh) * c.vl_cap;
+  for (int e = threadIdx.x; e < 2 * 1024; e += TKC_THREADS) (&h10[0][0])[e] = 0u;  // before the barriers below
 
   // (1) the threshold bin: thread i owns bins 2047 - 4i .. 2044 - 4i (descending)
   {
@@ -877,18 +878,16 @@ __global__ void __cluster_dims__(TKC_CS, 1, 1) __launch_bounds__(TKC_THREADS) to
   __syncthreads();
   const int ncand = static_cast<int>(s_cnt);
   // (3) the low 20 bits of the k-th largest: two radix passes of 10 bits, the
-  // cluster's histograms summed from every CTA's shared memory
+  // cluster's histograms summed from every CTA's shared memory (one histogram
+  // per pass, so no CTA has to wait for the others' reads before the next)
   uint32_t prefix = bin << 20, pmask = 0xFFF00000u;
   unsigned int above = s_above;
 #pragma unroll 1
   for (int pass = 0; pass < 2; ++pass) {
     const int shift = pass == 0 ? 10 : 0;
-    h10[threadIdx.x] = 0u;
-    h10[threadIdx.x + TKC_THREADS] = 0u;
-    __syncthreads();
     for (int e = threadIdx.x; e < ncand; e += TKC_THREADS) {
       const uint32_t v = cand[e];
-      if ((v & pmask) == prefix) atomicAdd(&h10[(v >> shift) & 1023u], 1u);
+      if ((v & pmask) == prefix) atomicAdd(&h10[pass][(v >> shift) & 1023u], 1u);
     }
     cl.sync();  // every CTA's histogram complete
     // thread i owns sub-bins 1023 - 2i and 1022 - 2i (descending)
@@ -896,11 +895,10 @@ __global__ void __cluster_dims__(TKC_CS, 1, 1) __launch_bounds__(TKC_THREADS) to
     unsigned int g1 = 0u, g0 = 0u;
 #pragma unroll
     for (int r = 0; r < TKC_CS; ++r) {
-      const unsigned int* rh = cl.map_shared_rank(h10, r);
+      const unsigned int* rh = cl.map_shared_rank(&h10[pass][0], r);
       g1 += rh[d1];
       g0 += rh[d0];
     }
-    cl.sync();  // every CTA done reading the histograms before they are cleared or reused
     const unsigned int X = tkc_block_scan(g1 + g0, wsum, lane, warp);
     const unsigned int up = X - g1 - g0;  // values (within the prefix) in sub-bins above d1
     const unsigned int needp = static_cast<unsigned int>(k) - above;
@@ -951,6 +949,8 @@ __global__ void __cluster_dims__(TKC_CS, 1, 1) __launch_bounds__(TKC_THREADS) to
     xg += rt[0];
     xe += rt[1];
   }
+  // done reading the other CTAs' shared memory: arrive now, wait before leaving
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
   for (int w = 0; w < warp; ++w) {
     xg += rg[w];
     xe += re[w];
@@ -969,7 +969,7 @@ __global__ void __cluster_dims__(TKC_CS, 1, 1) __launch_bounds__(TKC_THREADS) to
     xg += __popc(bg);
     xe += __popc(be);
   }
-  cl.sync();  // no CTA leaves while another may still read its shared memory
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");  // no CTA leaves while another may still read its shared memory
 }
 
 int sel_mp(const hq_cache& c) { return (((c.Hq / c.Hkv) * HQ_QBUF + 127) / 128) * 128; }
